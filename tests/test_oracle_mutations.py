@@ -1,0 +1,132 @@
+"""Plants plausible mistakes in the oracle (CPU only, via monkeypatch) and checks
+that at least one pin in test_oracle_pins.py fails for each of them."""
+import numpy as np
+import pytest
+
+from oracle import vdn_oracle as O
+import test_oracle_pins as pins
+
+_orig = {name: getattr(O, name) for name in
+         ("window_bounds", "frame_statistics", "rule_step", "gather_state", "seed_state",
+          "prepare_features", "readout", "short_conv_frame")}
+
+
+def _window_hi_plus_one(t, F, chunk, radius):
+    c = t // chunk
+    return max(0, chunk * (c - radius)), min(F - 1, chunk * (c + radius + 1))
+
+
+def _stats_B_transposed(kf, vf, beta):
+    A, Bm = _orig["frame_statistics"](kf, vf, beta)
+    return A, np.swapaxes(Bm, -1, -2)
+
+
+def _stats_no_beta(kf, vf, beta):
+    return _orig["frame_statistics"](kf, vf, np.ones_like(beta))
+
+
+def _rule_D_on_left(S_in, A_f, B_f, alpha_f, rule, c=1.0):
+    return _orig["rule_step"](np.diag(alpha_f) @ S_in @ np.diag(1 / alpha_f), A_f, B_f, alpha_f, rule, c)
+
+
+def _rule_sana_sign(S_in, A_f, B_f, alpha_f, rule, c=1.0):
+    if rule == "sana_scaled":
+        return (S_in @ np.diag(alpha_f)) @ (np.eye(A_f.shape[0]) + c * c * A_f) + c * B_f
+    return _orig["rule_step"](S_in, A_f, B_f, alpha_f, rule, c)
+
+
+def _rule_solve_transposed(S_in, A_f, B_f, alpha_f, rule, c=1.0):
+    if rule in ("vdn_solve", "vdn_scaled"):
+        cc = 1.0 if rule == "vdn_solve" else c
+        X = S_in @ np.diag(alpha_f) + cc * B_f
+        return np.linalg.solve(np.eye(A_f.shape[0]) + cc * cc * A_f + 0.01 * np.triu(A_f, 1), X)
+    return _orig["rule_step"](S_in, A_f, B_f, alpha_f, rule, c)
+
+
+def _rule_c_dropped(S_in, A_f, B_f, alpha_f, rule, c=1.0):
+    if rule == "vdn_scaled":
+        return _orig["rule_step"](S_in, A_f, B_f, alpha_f, "vdn_solve")
+    return _orig["rule_step"](S_in, A_f, B_f, alpha_f, rule, c)
+
+
+def _gather_whole_window(P, Q, seed, alpha_h, t, chunk, radius, bridge="to_query"):
+    return _orig["gather_state"](P, Q, seed, alpha_h, t, chunk, radius, "window")
+
+
+def _gather_no_bridge(P, Q, seed, alpha_h, t, chunk, radius, bridge="to_query"):
+    F = P.shape[0]
+    lo, hi = O.window_bounds(t, F, chunk, radius)
+    pre = seed if lo == 0 else P[lo - 1]
+    suf = seed if hi == F - 1 else Q[hi + 1]
+    return pre + suf
+
+
+def _seed_full(text_state_h, d):
+    return 2.0 * _orig["seed_state"](text_state_h, d)
+
+
+def _features_no_silu_k(qh, kh, vh, F, S, wk=None, wv=None, silu_v=True, causal=False):
+    d = qh.shape[-1]
+    qf, _, vf = _orig["prepare_features"](qh, kh, vh, F, S, wk, wv, silu_v, causal)
+    k = kh.reshape(F, S, d)
+    kc = np.stack([O.short_conv_frame(k[f], wk, causal) for f in range(F)])
+    return qf, O.l2_normalize(kc), vf
+
+
+def _conv_flipped(x, w, causal=False):
+    return _orig["short_conv_frame"](x, None if w is None else w[:, ::-1], causal)
+
+
+def _readout_no_gate(W_t, qf_tokens, gate_tokens, rms_w, prenorm=False):
+    return _orig["readout"](W_t, qf_tokens, np.ones_like(gate_tokens), rms_w, prenorm)
+
+
+def _readout_W_transposed(W_t, qf_tokens, gate_tokens, rms_w, prenorm=False):
+    return _orig["readout"](W_t.T, qf_tokens, gate_tokens, rms_w, prenorm)
+
+
+MUTANTS = {
+    "window_hi_plus_one": ("window_bounds", _window_hi_plus_one),
+    "stats_B_transposed": ("frame_statistics", _stats_B_transposed),
+    "stats_no_beta": ("frame_statistics", _stats_no_beta),
+    "rule_D_on_left": ("rule_step", _rule_D_on_left),
+    "rule_sana_sign": ("rule_step", _rule_sana_sign),
+    "rule_solve_wrong_matrix": ("rule_step", _rule_solve_transposed),
+    "rule_c_dropped": ("rule_step", _rule_c_dropped),
+    "gather_whole_window": ("gather_state", _gather_whole_window),
+    "gather_no_bridge": ("gather_state", _gather_no_bridge),
+    "seed_full_text": ("seed_state", _seed_full),
+    "features_no_silu_k": ("prepare_features", _features_no_silu_k),
+    "conv_flipped": ("short_conv_frame", _conv_flipped),
+    "readout_no_gate": ("readout", _readout_no_gate),
+    "readout_W_transposed": ("readout", _readout_W_transposed),
+}
+
+PINS = [
+    lambda: pins.test_window_partitions_frames(3, 1),
+    lambda: pins.test_window_page_geometry(),
+    lambda: pins.test_short_conv_is_numpy_convolve_same(3),
+    lambda: pins.test_frame_statistics_is_sum_of_outer_products(),
+    lambda: pins.test_solve_is_ridge_regression_least_squares(0.5),
+    lambda: pins.test_sana_vs_vdn_scaled_small_c(),
+    lambda: pins.test_one_token_per_frame_is_gated_delta_rule("vdn_solve"),
+    lambda: pins.test_one_token_per_frame_is_gated_delta_rule("sana_scaled"),
+    lambda: pins.test_text_state_only_decays_to_half_prompt("vdn_solve"),
+    lambda: pins.test_additive_unit_alpha_is_bruteforce_far_field_attention(2, 1),
+    lambda: pins.test_bridge_decays_across_exactly_the_frames_between(),
+    lambda: pins.test_rmsnorm_gate_readout(),
+    lambda: pins.test_prepare_features_from_library_routines(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    fn, mutant = MUTANTS[name]
+    monkeypatch.setattr(O, fn, mutant)
+    caught = 0
+    for pin in PINS:
+        try:
+            pin()
+        except (AssertionError, np.linalg.LinAlgError, ValueError):
+            caught += 1
+    assert caught > 0, f"no pin fails with mutant {name}"
