@@ -1,0 +1,180 @@
+/*
+ * vdn.h -- C ABI of libvdn: the forward pass of the VDN-H3 bidirectional
+ * linear-attention branch on one NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "VDN-Minimax-H3 bidirectional linear branch in five
+ * steps" (icman.com.cn/news/81972), sections "Step 1" .. "Step 5" and "text
+ * state".  The page printed its formulas with every '+' and '=' lost; the
+ * restored forms used throughout are
+ *     A_f = sum_s beta_s k'_s k'_s^T          B_f = sum_s beta_s v'_s k'_s^T
+ *     vdn_solve    S_out = (S_in D_f + B_f)(I + A_f)^-1
+ *     vdn_scaled   S_out = (S_in D_f + c B_f)(I + c^2 A_f)^-1
+ *     sana_scaled  S_out = (S_in D_f)(I - c^2 A_f) + c B_f
+ * with D_f = diag(alpha_f) (per key channel) and the state S a d_v x d_k map
+ * read out as o = S q'.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates device memory and keeps no global state, so calls on
+ *     different streams with different workspaces may run concurrently.
+ *   - Every tensor is dense and contiguous in the layout given beside it, with
+ *     a 16-byte aligned base address (VDN_ERR_ALIGNMENT otherwise).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are reported before any launch; a
+ *     failed launch returns VDN_ERR_CUDA.  Errors during device execution
+ *     surface at the caller's next synchronisation.
+ *   - Element types: q, k, v, gate and out share `shape->dtype` (fp32 or
+ *     bf16); beta, alpha, rms_w, the conv taps and the text state are fp32.
+ *     State and accumulation are fp32 in every configuration.
+ */
+#ifndef VDN_H
+#define VDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VDN_OK = 0,
+    VDN_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, bad enum, out/in overlap */
+    VDN_ERR_UNSUPPORTED = 2,   /* d not in {16,128}, conv_width not in {1,3}, bf16 with d != 128 */
+    VDN_ERR_ALIGNMENT = 3,     /* a tensor base not 16-byte aligned (workspace: 256-byte) */
+    VDN_ERR_WORKSPACE = 4,     /* workspace smaller than vdn_branch_workspace_size() */
+    VDN_ERR_CUDA = 5,          /* a CUDA runtime / driver call or a launch failed */
+    VDN_ERR_TIMEOUT = 6        /* a bounded device-side wait expired (device status word) */
+} vdn_status;
+
+/* Update rule of the per-frame recurrence (page section "Step 3", rules table). */
+typedef enum {
+    VDN_RULE_SANA_SCALED = 0,  /* (S D)(I - c^2 A) + c B : first-order truncation          */
+    VDN_RULE_VDN_SOLVE = 1,    /* (S D + B)(I + A)^-1    : exact solve, the released rule  */
+    VDN_RULE_VDN_SCALED = 2,   /* (S D + c B)(I + c^2 A)^-1 : scaled exact solve           */
+    VDN_RULE_ADDITIVE = 3      /* S D + B (A taken as 0) : test rule, not on the page      */
+} vdn_rule;
+
+typedef enum { VDN_DTYPE_F32 = 0, VDN_DTYPE_BF16 = 1 } vdn_dtype;
+
+/* Implementation selector of the debug entry point.  AUTO picks the tensor-core
+ * path for bf16 with d == 128 and the SIMT path otherwise. */
+typedef enum { VDN_IMPL_AUTO = 0, VDN_IMPL_SIMT = 1, VDN_IMPL_TC = 2 } vdn_impl;
+
+/* Problem sizes.  N = F * S tokens per batch element, token n = f * S + s
+ * belongs to latent frame f.  d is the head dimension (d_k = d_v = d). */
+typedef struct {
+    int B;           /* batch                                  >= 1 */
+    int H;           /* heads                                  >= 1 */
+    int F;           /* latent frames                          >= 1 */
+    int S;           /* tokens per latent frame                >= 1 */
+    int d;           /* head dimension: 16 or 128                    */
+    int conv_width;  /* taps of the k/v short conv: 1 or 3           */
+    int dtype;       /* vdn_dtype of q, k, v, gate, out              */
+} vdn_shape;
+
+/* Bytes of device workspace that vdn_branch_forward needs for `shape` and
+ * `rule` (0 if the arguments are invalid).  The caller allocates it (256-byte
+ * aligned) and may reuse it across calls that do not overlap in time. */
+size_t vdn_branch_workspace_size(const vdn_shape* shape, int rule);
+
+/* Same, for an explicit implementation (VDN_IMPL_*), as the debug entry point needs. */
+size_t vdn_branch_workspace_size_impl(const vdn_shape* shape, int rule, int impl);
+
+/*
+ * vdn_branch_forward -- the whole branch, page sections "Step 1" to "Step 5".
+ *
+ *   q, k, v    [B, F*S, H, d] dtype   pre-RoPE ("NoPE") features, token-major
+ *   beta       [B, F*S, H]    fp32    per-token, per-head write strength (post-sigmoid)
+ *   alpha      [B, F, H, d]   fp32    per-frame, per-channel forget gate in (0, 1]
+ *   gate       [B, F*S, H, d] dtype   output gate values (post-sigmoid)
+ *   rms_w      [d]            fp32    RMSNorm weight (shared by the heads)
+ *   conv_k_w   [H, d, conv_width] fp32  depthwise taps of the k short conv, or NULL (identity)
+ *   conv_v_w   [H, d, conv_width] fp32  same for v, or NULL
+ *   text_state [H, d, d]      fp32    per-head text state T (v x k, row-major), or
+ *                                     NULL: both scans then start from zero.  Each
+ *                                     scan starts from 0.5 * T (TEXT_STATE_SCALE).
+ *   rule, c    vdn_rule and its scale c (ignored by VDN_SOLVE and ADDITIVE)
+ *   chunk      softmax-window chunk in frames (>= 1); the page's value is 5
+ *   radius     chunks added on each side of the query's chunk (>= 0); page: 1
+ *   workspace  device scratch of at least vdn_branch_workspace_size() bytes
+ *   out        [B, F*S, H, d] dtype   branch output (RMSNorm-ed and gated); must not
+ *                                     overlap any input
+ *
+ * Step 1: k, v -> depthwise conv along each frame's token order (centred, zero
+ * padding at the frame edges), SiLU on q, k, v, then L2 normalisation of q, k.
+ * Step 2: per (batch, head, frame) the statistics A_f and B_f.
+ * Step 3-4: the forward prefix scan P_f and backward suffix scan Q_f of the rule.
+ * Step 4: query frame t with window [lo, hi] (vdn_window_bounds) reads
+ *         W_t = P_{lo-1} diag(prod_{f=lo..t} alpha_f) + Q_{hi+1} diag(prod_{f=t..hi} alpha_f),
+ *         where P_{-1} = Q_F = 0.5 * T (the decayed prompt at a clip edge).
+ * Step 5: out = RMSNorm(W_t q') * gate, RMSNorm over d with eps 1e-6.
+ */
+vdn_status vdn_branch_forward(const vdn_shape* shape,
+                              const void* q, const void* k, const void* v,
+                              const float* beta, const float* alpha,
+                              const void* gate, const float* rms_w,
+                              const float* conv_k_w, const float* conv_v_w,
+                              const float* text_state,
+                              int rule, float c, int chunk, int radius,
+                              void* workspace, size_t workspace_bytes,
+                              void* out, void* stream);
+
+/* Intermediates for per-stage checks.  Every non-NULL pointer receives an fp32
+ * device array [B, H, F, d, d] (row-major d x d per frame):
+ *   A, B : frame statistics of "Step 2";
+ *   N    : per-frame operator of "Step 3": (I + c^2 A)^-1 (vdn rules),
+ *          I - c^2 A (sana_scaled) or I (additive);
+ *   P, Q : prefix state after absorbing frames 0..f and suffix state after
+ *          absorbing frames f..F-1 ("Step 4");
+ *   W    : gathered, bridged state of query frame f ("Step 4"). */
+typedef struct {
+    int impl;        /* vdn_impl */
+    float* A;
+    float* B;
+    float* N;
+    float* P;
+    float* Q;
+    float* W;
+} vdn_debug_out;
+
+/* vdn_branch_forward plus the intermediates requested in `dbg` (which may be
+ * NULL).  Uses the workspace size of vdn_branch_workspace_size_impl(dbg->impl).
+ * Not meant for timed runs: exporting intermediates adds device work. */
+vdn_status vdn_branch_forward_debug(const vdn_shape* shape,
+                                    const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha,
+                                    const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w,
+                                    const float* text_state,
+                                    int rule, float c, int chunk, int radius,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* out, void* stream,
+                                    const vdn_debug_out* dbg);
+
+/* "Step 1" alone (page: NoPE features): q' = L2(SiLU(q)), k' = L2(SiLU(conv_k(k))),
+ * v' = SiLU(conv_v(v)), all [B, F*S, H, d] in shape->dtype.  Outputs must not
+ * overlap the inputs.  Needs no workspace. */
+vdn_status vdn_feature_prep(const vdn_shape* shape,
+                            const void* q, const void* k, const void* v,
+                            const float* conv_k_w, const float* conv_v_w,
+                            void* q_out, void* k_out, void* v_out, void* stream);
+
+/* Chunk-aligned softmax window of query frame t (page: "what is the far
+ * field", chunk 5 / radius 1): c = t / chunk, lo = max(0, chunk (c - radius)),
+ * hi = min(F - 1, chunk (c + radius + 1) - 1).  Host function, no CUDA calls. */
+vdn_status vdn_window_bounds(int t, int F, int chunk, int radius, int* lo, int* hi);
+
+/* Reads the device status word that bounded waits inside the kernels set (it
+ * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
+ * Synchronises `stream`. */
+vdn_status vdn_workspace_status(const void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* vdn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDN_H */

@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI: the library loads, exports every function that
+include/vdn.h declares, and rejects bad arguments before any CUDA call (so these
+run without a GPU: the pointers below are never dereferenced)."""
+import ctypes
+
+import pytest
+
+from oracle import vdn_oracle as O
+from video_diffusion_linear_b200 import _lib
+from video_diffusion_linear_b200._lib import (VDN_ERR_ALIGNMENT, VDN_ERR_INVALID_ARG, VDN_ERR_UNSUPPORTED,
+                                              VDN_ERR_WORKSPACE, VDN_OK, VdnShape)
+
+
+def test_exports_every_header_symbol(lib):
+    names = _lib.header_symbols()
+    assert "vdn_branch_forward" in names and len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.vdn_status_string(s).decode() != "unknown status"
+    assert lib.vdn_status_string(99).decode() == "unknown status"
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 5, 7])
+@pytest.mark.parametrize("radius", [0, 1, 3])
+def test_window_bounds_matches_oracle(lib, chunk, radius):
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    for F in (1, 9, 31, 85):
+        for t in range(F):
+            assert lib.vdn_window_bounds(t, F, chunk, radius, ctypes.byref(lo), ctypes.byref(hi)) == VDN_OK
+            assert (lo.value, hi.value) == O.window_bounds(t, F, chunk, radius)
+    assert lib.vdn_window_bounds(5, 5, 5, 1, ctypes.byref(lo), ctypes.byref(hi)) == VDN_ERR_INVALID_ARG
+    assert lib.vdn_window_bounds(0, 5, 0, 1, ctypes.byref(lo), ctypes.byref(hi)) == VDN_ERR_INVALID_ARG
+
+
+def _shape(**kw):
+    base = dict(B=1, H=2, F=12, S=100, d=128, conv_width=3, dtype=1)
+    base.update(kw)
+    return VdnShape(**base)
+
+
+BASE = 1 << 40      # fake, 4 KiB-aligned device addresses, far apart
+GAP = 1 << 34
+
+
+def _args(shape, ws_bytes=None, **over):
+    ptr = {name: BASE + i * GAP for i, name in enumerate(
+        ["q", "k", "v", "beta", "alpha", "gate", "rms_w", "conv_k_w", "conv_v_w", "text", "ws", "out"])}
+    ptr.update(over)
+    if ws_bytes is None:
+        ws_bytes = _lib.load().vdn_branch_workspace_size(ctypes.byref(shape), 1)
+    P = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n])
+    return (ctypes.byref(shape), P("q"), P("k"), P("v"), P("beta"), P("alpha"), P("gate"), P("rms_w"),
+            P("conv_k_w"), P("conv_v_w"), P("text"), 1, 1.0, 5, 1, P("ws"), ws_bytes, P("out"), None)
+
+
+def test_workspace_size(lib):
+    s = _shape()
+    n = lib.vdn_branch_workspace_size(ctypes.byref(s), 1)
+    assert n > 0 and n % 256 == 0
+    assert lib.vdn_branch_workspace_size(ctypes.byref(_shape(d=64)), 1) == 0
+    assert lib.vdn_branch_workspace_size(ctypes.byref(s), 9) == 0
+    assert lib.vdn_branch_workspace_size_impl(ctypes.byref(_shape(dtype=1, d=16)), 1, 0) == 0
+    assert lib.vdn_branch_workspace_size_impl(ctypes.byref(_shape(dtype=0, d=16)), 1, 2) == 0
+    assert lib.vdn_branch_workspace_size_impl(ctypes.byref(_shape(dtype=0, d=16)), 1, 1) > 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(shape=dict(d=64)), VDN_ERR_UNSUPPORTED),
+    (dict(shape=dict(d=16, dtype=1)), VDN_ERR_UNSUPPORTED),
+    (dict(shape=dict(conv_width=5)), VDN_ERR_UNSUPPORTED),
+    (dict(shape=dict(S=0)), VDN_ERR_INVALID_ARG),
+    (dict(shape=dict(B=-1)), VDN_ERR_INVALID_ARG),
+    (dict(shape=dict(dtype=7)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(q=None)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(out=None)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(ws=None)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(q=BASE + 8)), VDN_ERR_ALIGNMENT),
+    (dict(ptr=dict(beta=BASE + 3 * GAP + 4)), VDN_ERR_ALIGNMENT),
+    (dict(ptr=dict(ws=BASE + 10 * GAP + 64)), VDN_ERR_ALIGNMENT),
+    (dict(ptr=dict(out=BASE + 64)), VDN_ERR_INVALID_ARG),               # out overlaps q
+    (dict(ptr=dict(out=BASE + 10 * GAP + 256)), VDN_ERR_INVALID_ARG),   # out overlaps the workspace
+    (dict(ws_bytes=1024), VDN_ERR_WORKSPACE),
+])
+def test_validation_rejects_before_launch(lib, case, expect):
+    s = _shape(**case.get("shape", {}))
+    args = _args(s, case.get("ws_bytes", 1 << 40), **case.get("ptr", {}))
+    assert lib.vdn_branch_forward(*args) == expect
+
+
+def test_bad_rule_and_window_args(lib):
+    s = _shape()
+    args = list(_args(s, 1 << 40))
+    for idx, val in ((11, 4), (11, -1), (13, 0), (14, -1), (12, float("nan"))):
+        a = list(args)
+        a[idx] = val
+        assert lib.vdn_branch_forward(*a) == VDN_ERR_INVALID_ARG, (idx, val)
+
+
+def test_feature_prep_validation(lib):
+    s = _shape()
+    p = lambda i: ctypes.c_void_p(BASE + i * GAP)
+    assert lib.vdn_feature_prep(ctypes.byref(s), p(0), p(1), p(2), None, None, p(0), p(4), p(5), None) == \
+        VDN_ERR_INVALID_ARG
+    assert lib.vdn_feature_prep(ctypes.byref(s), p(0), p(1), p(2), None, None, p(3), p(3), p(5), None) == \
+        VDN_ERR_INVALID_ARG
+    assert lib.vdn_feature_prep(ctypes.byref(s), None, p(1), p(2), None, None, p(3), p(4), p(5), None) == \
+        VDN_ERR_INVALID_ARG
+    assert lib.vdn_feature_prep(ctypes.byref(_shape(d=32)), p(0), p(1), p(2), None, None, p(3), p(4), p(5),
+                                None) == VDN_ERR_UNSUPPORTED

@@ -1,0 +1,174 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle, on the
+same seeded inputs, at sizes the oracle finishes in seconds (several tiles and a
+ragged tail), plus per-stage intermediates and edge cases."""
+import numpy as np
+import pytest
+import torch
+
+from harness import TOL_BF16, TOL_F32, gpu_forward, oracle_forward, rel_err, to_np
+from oracle import vdn_oracle as O
+from video_diffusion_linear_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+def test_tiny_workload_is_exactly_zero():
+    """Every window of the 10-frame tiny workload covers the whole clip and there
+    is no text state: the output is identically zero on both sides."""
+    w = W["tiny"]
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp)
+    assert torch.count_nonzero(out).item() == 0
+    assert np.all(oracle_forward(w, inp) == 0.0)
+
+
+@pytest.mark.parametrize("name", ["tiny_f20", "tiny_f20_text"])
+def test_tiny_f20_fp32(name):
+    w = W[name]
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp)
+    ref = oracle_forward(w, inp)
+    assert rel_err(to_np(out), ref) <= TOL_F32
+
+
+RULE_CASES = [("vdn_solve", 1.0), ("vdn_scaled", 0.5), ("vdn_scaled", 1.0), ("sana_scaled", 0.5),
+              ("sana_scaled", 1.0), ("additive", 1.0)]
+
+
+@pytest.mark.parametrize("rule,c", RULE_CASES)
+@pytest.mark.parametrize("text", [False, True])
+def test_rules_fp32_d16(rule, c, text):
+    w = synth.Workload("r16", B=2, H=2, d=16, F=14, S=9, dtype="f32", alpha_mu=2.0, text=text, seed=21,
+                       chunk=3, radius=1)
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp, rule=rule, c=c)
+    ref = oracle_forward(w, inp, rule=rule, c=c)
+    assert rel_err(to_np(out), ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("impl", ["simt"])
+def test_fp32_d128(impl):
+    w = synth.Workload("f32d128", B=1, H=2, d=128, F=12, S=70, dtype="f32", alpha_mu=2.0, text=True, seed=22)
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp, impl=impl, debug=True, want=())
+    ref = oracle_forward(w, inp)
+    assert rel_err(to_np(out), ref) <= TOL_F32
+
+
+BF16_SMALL = synth.Workload("bf16s", B=2, H=3, d=128, F=12, S=200, dtype="bf16", alpha_mu=2.0, text=True, seed=23)
+
+
+@pytest.mark.parametrize("impl", ["auto", "simt"])
+def test_bf16_small(impl):
+    w = BF16_SMALL
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp, impl=impl, debug=impl != "auto", want=())
+    ref = oracle_forward(w, inp)
+    assert rel_err(to_np(out), ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("rule,c", [("vdn_solve", 1.0), ("vdn_scaled", 0.5), ("sana_scaled", 1.0),
+                                    ("additive", 1.0)])
+def test_bf16_rules_small(rule, c):
+    w = BF16_SMALL.replace(B=1, H=2, F=16, S=130, seed=24)
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp, rule=rule, c=c)
+    ref = oracle_forward(w, inp, rule=rule, c=c)
+    assert rel_err(to_np(out), ref) <= TOL_BF16
+
+
+STAGE_TOL = {"f32": dict(A=1e-5, B=1e-5, N=1e-5, P=1e-4, Q=1e-4, W=1e-4),
+             "bf16": dict(A=5e-3, B=5e-3, N=5e-3, P=1e-2, Q=1e-2, W=1e-2)}
+
+
+@pytest.mark.parametrize("w,impl", [
+    (synth.Workload("st16", B=1, H=2, d=16, F=13, S=11, dtype="f32", alpha_mu=2.0, text=True, seed=25), "simt"),
+    (synth.Workload("st128", B=1, H=2, d=128, F=11, S=150, dtype="bf16", alpha_mu=2.0, text=True, seed=26), "auto"),
+    (synth.Workload("st128", B=1, H=2, d=128, F=11, S=150, dtype="bf16", alpha_mu=2.0, text=True, seed=26), "simt"),
+])
+@pytest.mark.parametrize("rule", ["vdn_solve", "sana_scaled"])
+def test_stage_intermediates(w, impl, rule):
+    inp = synth.make_inputs(w)
+    out, mats = gpu_forward(w, inp, rule=rule, c=0.7, impl=impl, debug=True)
+    tol = STAGE_TOL[w.dtype]
+    for b in range(w.B):
+        for h in range(w.H):
+            st = O.head_state(inp, b, h, w.F, w.S, rule, 0.7, w.chunk, w.radius)
+            d = w.d
+            cc = 1.0 if rule == "vdn_solve" else 0.7
+            if rule in ("vdn_solve", "vdn_scaled"):
+                Nref = np.stack([np.linalg.inv(np.eye(d) + cc * cc * a) for a in st["A"]])
+            else:
+                Nref = np.stack([np.eye(d) - cc * cc * a for a in st["A"]])
+            ref = dict(A=st["A"], B=st["B"], N=Nref, P=st["P"], Q=st["Q"], W=st["W"])
+            for name, r in ref.items():
+                got = to_np(mats[name][b, h])
+                assert rel_err(got, r) <= tol[name], (name, b, h, rel_err(got, r))
+
+
+@pytest.mark.parametrize("dtype,d,tol", [("f32", 16, 1e-5), ("f32", 128, 1e-5), ("bf16", 128, 8e-3)])
+@pytest.mark.parametrize("K", [1, 3])
+def test_feature_prep(dtype, d, tol, K):
+    w = synth.Workload("fp", B=2, H=3, d=d, F=4, S=37, dtype=dtype, alpha_mu=2.0, text=False, seed=27,
+                       conv_width=K)
+    inp = synth.make_inputs(w)
+    dev = api.to_device(inp)
+    qo, ko, vo = api.feature_prep(dev["q"], dev["k"], dev["v"], dev["conv_k_w"], dev["conv_v_w"], F=w.F)
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        for h in range(w.H):
+            wk = None if inp["conv_k_w"] is None else inp["conv_k_w"][h].double().numpy()
+            wv = None if inp["conv_v_w"] is None else inp["conv_v_w"][h].double().numpy()
+            ref = O.prepare_features(inp["q"][b, :, h].double().numpy(), inp["k"][b, :, h].double().numpy(),
+                                     inp["v"][b, :, h].double().numpy(), w.F, w.S, wk, wv)
+            for got, r in zip((qo, ko, vo), ref):
+                g = to_np(got[b, :, h]).reshape(w.F, w.S, d)
+                assert np.abs(g - r).max() <= tol * max(1.0, np.abs(r).max())
+
+
+EDGE = [
+    dict(F=1, S=40, text=True),                  # one frame: only the seeds, decayed
+    dict(F=1, S=40, text=False),                 # one frame, no text: exactly zero
+    dict(F=7, S=1, text=True),                   # one token per frame
+    dict(F=9, S=65, chunk=1, radius=0),          # window = own frame only
+    dict(F=6, S=64, chunk=10, radius=1),         # chunk longer than the clip
+    dict(F=23, S=129, chunk=2, radius=2),
+    dict(F=11, S=63, conv_width=1),              # no conv taps
+    dict(F=13, S=3, B=3, H=1, text=True),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[str(i) for i in range(len(EDGE))])
+@pytest.mark.parametrize("dtype,d", [("f32", 16), ("bf16", 128)])
+def test_edge_cases(case, dtype, d):
+    kw = dict(B=1, H=2, text=True, chunk=5, radius=1, conv_width=3)
+    kw.update(case)
+    w = synth.Workload("edge", kw["B"], kw["H"], d, kw["F"], kw["S"], dtype, 2.0, kw["text"], 28,
+                       conv_width=kw["conv_width"], chunk=kw["chunk"], radius=kw["radius"])
+    inp = synth.make_inputs(w)
+    out, _ = gpu_forward(w, inp)
+    ref = oracle_forward(w, inp)
+    if np.abs(ref).max() == 0:
+        assert torch.count_nonzero(out).item() == 0
+    else:
+        assert rel_err(to_np(out), ref) <= (TOL_F32 if dtype == "f32" else TOL_BF16)
+
+
+def test_run_to_run_bitwise():
+    w = BF16_SMALL
+    inp = synth.make_inputs(w)
+    a, _ = gpu_forward(w, inp)
+    b, _ = gpu_forward(w, inp)
+    assert torch.equal(a, b)
+
+
+def test_device_status_word_clear_after_run():
+    w = BF16_SMALL
+    inp = synth.make_inputs(w)
+    dev = api.to_device(inp)
+    shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
+    ws = api.alloc_workspace(shape)
+    api.branch_forward(*api.forward_inputs(dev), F=w.F, workspace=ws)
+    assert api.workspace_status(ws) == 0

@@ -1,0 +1,131 @@
+"""Thin Python binding of libvdn (include/vdn.h).
+
+Argument marshalling only: torch supplies device memory and the stream, every
+step of the branch runs in the library's CUDA kernels.  Tensors must be CUDA
+tensors in the layouts documented in vdn.h.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import VDN_DTYPE, VDN_IMPL, VDN_RULE, VdnDebugOut, VdnShape, check
+
+_TORCH_DTYPE = {torch.float32: "f32", torch.bfloat16: "bf16"}
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libvdn must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_shape(B, H, F, S, d, conv_width=3, dtype="bf16") -> VdnShape:
+    if isinstance(dtype, torch.dtype):
+        dtype = _TORCH_DTYPE[dtype]
+    return VdnShape(B, H, F, S, d, conv_width, VDN_DTYPE[dtype])
+
+
+def shape_from(q: torch.Tensor, F: int, conv_k_w=None) -> VdnShape:
+    B, N, H, d = q.shape
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    K = 1 if conv_k_w is None else conv_k_w.shape[-1]
+    return make_shape(B, H, F, N // F, d, K, q.dtype)
+
+
+def workspace_size(shape: VdnShape, rule="vdn_solve", impl="auto") -> int:
+    n = _lib.load().vdn_branch_workspace_size_impl(ctypes.byref(shape), VDN_RULE[rule], VDN_IMPL[impl])
+    if n == 0:
+        raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_branch_workspace_size")
+    return n
+
+
+def alloc_workspace(shape: VdnShape, rule="vdn_solve", impl="auto", device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(shape, rule, impl), dtype=torch.uint8, device=device)
+
+
+def _forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                  radius, workspace, out, stream):
+    return (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
+            _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
+            _ptr(workspace), workspace.numel(), _ptr(out), _stream_ptr(stream))
+
+
+def branch_forward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *,
+                   F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, out=None, workspace=None, stream=None):
+    """vdn_branch_forward: the whole branch.  Returns `out` ([B, F*S, H, d], q's dtype)."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(shape, rule, "auto", q.device)
+    st = _lib.load().vdn_branch_forward(*_forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w,
+                                                       conv_v_w, text_state, rule, c, chunk, radius, workspace,
+                                                       out, stream))
+    check(st, "vdn_branch_forward")
+    return out
+
+
+DEBUG_FIELDS = ("A", "B", "N", "P", "Q", "W")
+
+
+def branch_forward_debug(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *,
+                         F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, impl="auto", want=DEBUG_FIELDS,
+                         out=None, workspace=None, stream=None):
+    """vdn_branch_forward_debug: returns (out, {name: fp32 [B, H, F, d, d]}) for the requested intermediates."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(shape, rule, impl, q.device)
+    B, N, H, d = q.shape
+    mats = {name: torch.full((B, H, F, d, d), float("nan"), dtype=torch.float32, device=q.device) for name in want}
+    dbg = VdnDebugOut(VDN_IMPL[impl], *[mats[n].data_ptr() if n in mats else None for n in DEBUG_FIELDS])
+    st = _lib.load().vdn_branch_forward_debug(*_forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w,
+                                                             conv_v_w, text_state, rule, c, chunk, radius,
+                                                             workspace, out, stream), ctypes.byref(dbg))
+    check(st, "vdn_branch_forward_debug")
+    return out, mats
+
+
+def feature_prep(q, k, v, conv_k_w=None, conv_v_w=None, *, F: int, stream=None):
+    """vdn_feature_prep: Step 1 alone.  Returns (q', k', v') in q's dtype."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    qo, ko, vo = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = _lib.load().vdn_feature_prep(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_k_w),
+                                      _ptr(conv_v_w), _ptr(qo), _ptr(ko), _ptr(vo), _stream_ptr(stream))
+    check(st, "vdn_feature_prep")
+    return qo, ko, vo
+
+
+def window_bounds(t: int, F: int, chunk: int = 5, radius: int = 1):
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    check(_lib.load().vdn_window_bounds(t, F, chunk, radius, ctypes.byref(lo), ctypes.byref(hi)),
+          "vdn_window_bounds")
+    return lo.value, hi.value
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    return _lib.load().vdn_workspace_status(_ptr(workspace), workspace.numel(), _stream_ptr(stream))
+
+
+def to_device(inp: dict, device="cuda") -> dict:
+    """Copies the host tensors of synth.make_inputs to the device (None stays None)."""
+    return {k: (None if t is None else t.to(device)) for k, t in inp.items()}
+
+
+def forward_inputs(dev: dict):
+    """Positional tensor arguments of branch_forward from a synth-style dict."""
+    return (dev["q"], dev["k"], dev["v"], dev["beta"], dev["alpha"], dev["gate"], dev["rms_w"],
+            dev.get("conv_k_w"), dev.get("conv_v_w"), dev.get("text_state"))

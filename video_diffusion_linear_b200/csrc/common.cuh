@@ -1,0 +1,90 @@
+// Device helpers shared by the libvdn kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "vdn.h"
+
+namespace vdn {
+
+constexpr float kL2Eps = 1e-12f;     // q', k' = x / sqrt(sum x^2 + 1e-12)
+constexpr float kRmsEps = 1e-6f;     // RMSNorm over d
+constexpr float kTextStateScale = 0.5f;
+
+// ---------------------------------------------------------------- element access
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// bf16x2 packed in a 32-bit word -> two floats (exact)
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// two floats -> bf16x2 (round to nearest even), lo in the low half
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// SiLU with the accurate exponential (SIMT paths, fp32 parity).
+__device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
+
+// SiLU through the identity sigmoid(x) = (1 + tanh(x/2)) / 2 and the hardware
+// tanh approximation (one MUFU op); used where operands are rounded to bf16.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float silu_fast(float x) {
+  float hx = 0.5f * x;
+  return fmaf(hx, tanh_approx(hx), hx);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- window geometry
+// Chunk-aligned softmax window of query frame t (page: "what is the far field").
+__host__ __device__ __forceinline__ void window_bounds(int t, int F, int chunk, int radius, int& lo, int& hi) {
+  int c = t / chunk;
+  long long l = (long long)chunk * (c - radius);
+  long long h = (long long)chunk * (c + radius + 1) - 1;
+  lo = l < 0 ? 0 : (int)l;
+  hi = h > F - 1 ? F - 1 : (int)h;
+}
+
+// Coefficients of the generic step  S_f = (S_{f-1} D_f + cpre B_f) N_f + cpost B_f,
+// which covers the three rules of the page plus the additive test rule.
+struct RuleCoef {
+  float cpre, cpost, c2;   // c2: scale of A inside N_f
+  bool solve;              // N_f = (I + c2 A)^-1 (else I - c2 A, or I for additive)
+  bool identity;
+};
+__host__ __device__ __forceinline__ RuleCoef rule_coef(int rule, float c) {
+  RuleCoef r;
+  switch (rule) {
+    case VDN_RULE_VDN_SOLVE: r = {1.f, 0.f, 1.f, true, false}; break;
+    case VDN_RULE_VDN_SCALED: r = {c, 0.f, c * c, true, false}; break;
+    case VDN_RULE_SANA_SCALED: r = {0.f, c, c * c, false, false}; break;
+    default: r = {1.f, 0.f, 0.f, false, true}; break;   // additive
+  }
+  return r;
+}
+
+// ---------------------------------------------------------------- device status word
+// Written only by bounded waits that gave up; read by vdn_workspace_status().
+constexpr uint32_t kStatusTimeout = 0x7100u;
+
+}  // namespace vdn

@@ -1,0 +1,72 @@
+// Internal interface between the C-ABI host code and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "vdn.h"
+
+namespace vdn {
+
+struct Args {
+  vdn_shape sh;
+  const void* q; const void* k; const void* v;
+  const float* beta; const float* alpha;
+  const void* gate; const float* rms_w;
+  const float* conv_k_w; const float* conv_v_w;
+  const float* text_state;
+  int rule; float c; int chunk; int radius;
+  void* out;
+  cudaStream_t stream;
+  const vdn_debug_out* dbg;   // may be NULL
+  long long N() const { return (long long)sh.F * sh.S; }
+  long long NF() const { return (long long)sh.B * sh.H * sh.F; }   // (batch, head, frame) triples
+};
+
+// CTAs of the persistent frame-statistics kernel of the tensor-core path.  A
+// fixed count (the SM count of a B200) keeps the workspace a pure function of
+// the shape; correctness does not depend on it.
+constexpr int kStatsGrid = 148;
+constexpr int kStatsTokens = 64;     // tokens per statistics block
+
+// Byte offsets of the workspace regions (each 256-byte aligned).
+struct WsPlan {
+  size_t status = 0;
+  // SIMT path
+  size_t qf = 0, kf = 0, vf = 0;        // fp32 [B, N, H, d]
+  size_t A = 0, Bm = 0, Nm = 0;         // fp32 [B, H, F, d, d]
+  size_t P = 0, Q = 0, W = 0;           // fp32 [B, H, F, d, d]
+  // tensor-core path
+  size_t part = 0;                      // fp32 [slots][d][2d]: rows of [A | B^T] partial sums
+  size_t nimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of N_f
+  size_t wimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of W_t
+  size_t total = 0;
+};
+
+bool use_tc(const vdn_shape& sh, int impl);
+WsPlan plan_workspace(const vdn_shape& sh, int rule, bool tc);
+
+// ---- launchers; each returns cudaSuccess or the launch error
+// SIMT path (any supported d, fp32 or bf16 I/O)
+cudaError_t launch_features_simt(const Args& a, float* qf, float* kf, float* vf);
+cudaError_t launch_stats_simt(const Args& a, const float* kf, const float* vf, float* A, float* Bm);
+cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nimg, const float* partials,
+                         float* Bsum, float* Aout);
+cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q);
+cudaError_t launch_gather(const Args& a, const float* P, const float* Q, float* W, uint16_t* wimg);
+cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W);
+cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst);
+
+// standalone step 1 (dtype in, dtype out)
+cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,
+                                const float* wk, const float* wv, void* qo, void* ko, void* vo,
+                                cudaStream_t st);
+
+// tensor-core path (bf16, d = 128)
+cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
+cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q,
+                           bool all_frames, uint32_t* status);
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, uint32_t* status);
+
+}  // namespace vdn

@@ -1,0 +1,350 @@
+// SIMT (CUDA-core) kernels of the branch: the fp32 path for every supported d,
+// and the reference-grade GPU path used for per-stage checks.
+//
+// Steps follow the page "VDN-Minimax-H3 bidirectional linear branch in five
+// steps": Step 1 (NoPE features), Step 2 (frame statistics), Step 3/4 (delta
+// rule, bidirectional scan) and Step 5 (read-out, RMSNorm, output gate).
+#include "common.cuh"
+#include "internal.h"
+
+namespace vdn {
+
+// ---------------------------------------------------------------- Step 1
+// One warp per (batch, token, head); lane handles channels lane + 32 r.
+// k, v: depthwise conv over the frame's tokens (centred, zero padding at the
+// frame edge), SiLU; q: SiLU; q and k L2-normalised.
+template <typename TI, typename TO, int D>
+__global__ void __launch_bounds__(256) k_features_simt(const TI* __restrict__ q, const TI* __restrict__ k,
+                                                       const TI* __restrict__ v, const float* __restrict__ wk,
+                                                       const float* __restrict__ wv, int K, TO* __restrict__ qo,
+                                                       TO* __restrict__ ko, TO* __restrict__ vo, int B, int F,
+                                                       int S, int H) {
+  constexpr int PER = (D + 31) / 32;
+  long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  long long N = (long long)F * S;
+  long long total = (long long)B * N * H;
+  if (warp >= total) return;
+  int h = (int)(warp % H);
+  long long bn = warp / H;
+  long long n = bn % N;
+  long long b = bn / N;
+  int s = (int)(n % S);
+  int pad = (K - 1) / 2;
+  float qv[PER], kv[PER], vv[PER];
+  float sq = 0.f, sk = 0.f;
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    int c = lane + 32 * r;
+    qv[r] = kv[r] = vv[r] = 0.f;
+    if (c < D) {
+      long long base = ((b * N + n) * H + h) * D + c;
+      float x = to_f32(q[base]);
+      qv[r] = silu_precise(x);
+      float ak = 0.f, av = 0.f;
+      if (wk == nullptr) ak = to_f32(k[base]);
+      if (wv == nullptr) av = to_f32(v[base]);
+      for (int j = 0; j < K; ++j) {
+        int ss = s + j - pad;
+        if (ss < 0 || ss >= S) continue;
+        long long nb = ((b * N + (n - s + ss)) * H + h) * D + c;
+        if (wk) ak = fmaf(wk[((long long)h * D + c) * K + j], to_f32(k[nb]), ak);
+        if (wv) av = fmaf(wv[((long long)h * D + c) * K + j], to_f32(v[nb]), av);
+      }
+      kv[r] = silu_precise(ak);
+      vv[r] = silu_precise(av);
+      sq += qv[r] * qv[r];
+      sk += kv[r] * kv[r];
+    }
+  }
+  sq = warp_sum(sq);
+  sk = warp_sum(sk);
+  float iq = rsqrtf(sq + kL2Eps), ik = rsqrtf(sk + kL2Eps);
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    int c = lane + 32 * r;
+    if (c < D) {
+      long long base = ((b * N + n) * H + h) * D + c;
+      qo[base] = from_f32<TO>(qv[r] * iq);
+      ko[base] = from_f32<TO>(kv[r] * ik);
+      vo[base] = from_f32<TO>(vv[r]);
+    }
+  }
+}
+
+template <typename TI, typename TO>
+static cudaError_t features_dispatch(const vdn_shape& sh, const void* q, const void* k, const void* v,
+                                     const float* wk, const float* wv, void* qo, void* ko, void* vo,
+                                     cudaStream_t st) {
+  long long warps = (long long)sh.B * sh.F * sh.S * sh.H;
+  long long blocks = (warps * 32 + 255) / 256;
+  int K = (wk || wv) ? sh.conv_width : 1;
+  auto go = [&](auto kern) {
+    kern<<<(unsigned)blocks, 256, 0, st>>>((const TI*)q, (const TI*)k, (const TI*)v, wk, wv, K, (TO*)qo, (TO*)ko,
+                                           (TO*)vo, sh.B, sh.F, sh.S, sh.H);
+  };
+  if (sh.d == 16) go(k_features_simt<TI, TO, 16>);
+  else go(k_features_simt<TI, TO, 128>);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_features_simt(const Args& a, float* qf, float* kf, float* vf) {
+  if (a.sh.dtype == VDN_DTYPE_BF16)
+    return features_dispatch<__nv_bfloat16, float>(a.sh, a.q, a.k, a.v, a.conv_k_w, a.conv_v_w, qf, kf, vf,
+                                                   a.stream);
+  return features_dispatch<float, float>(a.sh, a.q, a.k, a.v, a.conv_k_w, a.conv_v_w, qf, kf, vf, a.stream);
+}
+
+// ---------------------------------------------------------------- Step 2
+// A_f = sum_s beta_s k'_s k'_s^T, B_f = sum_s beta_s v'_s k'_s^T.
+// Block: one TLxTL tile of A or B of one (batch, head, frame); 16x16 threads,
+// each accumulating an MTxMT micro-tile over the frame's tokens.
+template <int D>
+__global__ void __launch_bounds__(256) k_stats_simt(const float* __restrict__ kf, const float* __restrict__ vf,
+                                                    const float* __restrict__ beta, float* __restrict__ A,
+                                                    float* __restrict__ Bm, int H, int F, int S) {
+  constexpr int TL = D < 64 ? D : 64;
+  constexpr int NT = D / TL;
+  constexpr int MT = TL / 16;
+  constexpr int CH = 32;
+  __shared__ float xs[CH][TL + 1];
+  __shared__ float ys[CH][TL + 1];
+  long long fi = blockIdx.x;
+  int tile = blockIdx.y;
+  int mat = tile / (NT * NT), ti = (tile / NT) % NT, tj = tile % NT;
+  int f = (int)(fi % F);
+  long long bh = fi / F;
+  int h = (int)(bh % H);
+  long long b = bh / H;
+  long long N = (long long)F * S;
+  const float* X = mat == 0 ? kf : vf;
+  int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[MT][MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int n = 0; n < MT; ++n) acc[m][n] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += CH) {
+    for (int e = tid; e < CH * TL; e += 256) {
+      int r = e / TL, cc = e % TL, s = s0 + r;
+      float xv = 0.f, yv = 0.f;
+      if (s < S) {
+        long long n = (long long)f * S + s;
+        long long base = ((b * N + n) * H + h) * D;
+        xv = X[base + ti * TL + cc];
+        yv = beta[(b * N + n) * H + h] * kf[base + tj * TL + cc];
+      }
+      xs[r][cc] = xv;
+      ys[r][cc] = yv;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < CH; ++r) {
+      float xr[MT], yr[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        xr[m] = xs[r][ty * MT + m];
+        yr[m] = ys[r][tx * MT + m];
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int n = 0; n < MT; ++n) acc[m][n] = fmaf(xr[m], yr[n], acc[m][n]);
+    }
+    __syncthreads();
+  }
+  float* out = (mat == 0 ? A : Bm) + fi * D * D;
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int n = 0; n < MT; ++n) out[(ti * TL + ty * MT + m) * D + tj * TL + tx * MT + n] = acc[m][n];
+}
+
+cudaError_t launch_stats_simt(const Args& a, const float* kf, const float* vf, float* A, float* Bm) {
+  dim3 grid((unsigned)a.NF(), a.sh.d == 16 ? 2 : 8);
+  if (a.sh.d == 16) k_stats_simt<16><<<grid, 256, 0, a.stream>>>(kf, vf, a.beta, A, Bm, a.sh.H, a.sh.F, a.sh.S);
+  else k_stats_simt<128><<<grid, 256, 0, a.stream>>>(kf, vf, a.beta, A, Bm, a.sh.H, a.sh.F, a.sh.S);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- Step 3/4
+// Bidirectional scan, one block per (batch, head, direction):
+//   S_f = (S_{f-1} D_f + cpre B_f) N_f + cpost B_f,
+// forward over f = 0..F-1 (prefix P_f) and backward over f = F-1..0 (suffix
+// Q_f), both seeded with 0.5 * text_state.  Thread (ty, tx) owns state
+// elements (ty + 16 ia, tx + 16 ib).
+template <int D>
+__global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm, const float* __restrict__ Nm,
+                                                   const float* __restrict__ alpha, const float* __restrict__ text,
+                                                   RuleCoef rc, float* __restrict__ P, float* __restrict__ Q,
+                                                   int H, int F) {
+  constexpr int R = D / 16;
+  constexpr int LD = D + 1;
+  extern __shared__ float sm[];
+  float* X = sm;
+  float* Ns = sm + D * LD;
+  int dir = blockIdx.x & 1;
+  long long bh = blockIdx.x >> 1;
+  int h = (int)(bh % H);
+  long long b = bh / H;
+  int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float s[R][R];
+#pragma unroll
+  for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+    for (int ib = 0; ib < R; ++ib) {
+      int i = ty + 16 * ia, k = tx + 16 * ib;
+      s[ia][ib] = text ? kTextStateScale * text[((long long)h * D + i) * D + k] : 0.f;
+    }
+  for (int step = 0; step < F; ++step) {
+    int f = dir == 0 ? step : F - 1 - step;
+    long long fi = bh * F + f;
+    const float* Bf = Bm + fi * D * D;
+    const float* Nf = Nm + fi * D * D;
+    const float* al = alpha + ((b * F + f) * H + h) * D;
+    for (int e = tid; e < D * D; e += 256) Ns[(e / D) * LD + (e % D)] = Nf[e];
+#pragma unroll
+    for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+      for (int ib = 0; ib < R; ++ib) {
+        int i = ty + 16 * ia, k = tx + 16 * ib;
+        X[i * LD + k] = fmaf(s[ia][ib], al[k], rc.cpre * Bf[i * D + k]);
+      }
+    __syncthreads();
+    float acc[R][R];
+#pragma unroll
+    for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+      for (int ib = 0; ib < R; ++ib) acc[ia][ib] = 0.f;
+    for (int j = 0; j < D; ++j) {
+      float xr[R], nr[R];
+#pragma unroll
+      for (int ia = 0; ia < R; ++ia) xr[ia] = X[(ty + 16 * ia) * LD + j];
+#pragma unroll
+      for (int ib = 0; ib < R; ++ib) nr[ib] = Ns[j * LD + tx + 16 * ib];
+#pragma unroll
+      for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+        for (int ib = 0; ib < R; ++ib) acc[ia][ib] = fmaf(xr[ia], nr[ib], acc[ia][ib]);
+    }
+    float* dst = (dir == 0 ? P : Q) + fi * D * D;
+#pragma unroll
+    for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+      for (int ib = 0; ib < R; ++ib) {
+        int i = ty + 16 * ia, k = tx + 16 * ib;
+        s[ia][ib] = fmaf(rc.cpost, Bf[i * D + k], acc[ia][ib]);
+        dst[i * D + k] = s[ia][ib];
+      }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q) {
+  RuleCoef rc = rule_coef(a.rule, a.c);
+  unsigned grid = (unsigned)(2LL * a.sh.B * a.sh.H);
+  if (a.sh.d == 16) {
+    size_t smem = 2 * 16 * 17 * sizeof(float);
+    k_scan_simt<16><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F);
+  } else {
+    size_t smem = 2 * 128 * 129 * sizeof(float);
+    cudaFuncSetAttribute(k_scan_simt<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_scan_simt<128><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- Step 5
+// One block per (batch, head, frame, 64-token tile); W_t in shared memory,
+// one warp per token: o = W_t q', RMSNorm over d, times rms_w and the gate.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_readout_simt(const float* __restrict__ qf, const T* __restrict__ gate,
+                                                      const float* __restrict__ rms_w, const float* __restrict__ W,
+                                                      T* __restrict__ out, int H, int F, int S) {
+  constexpr int LD = D + 1;
+  constexpr int PER = (D + 31) / 32;
+  constexpr int TT = 64;
+  extern __shared__ float sm[];
+  float* Ws = sm;
+  float* qs = sm + D * LD;   // [8][D]
+  long long fi = blockIdx.x;
+  int f = (int)(fi % F);
+  long long bh = fi / F;
+  int h = (int)(bh % H);
+  long long b = bh / H;
+  long long N = (long long)F * S;
+  const float* Wt = W + fi * D * D;
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Ws[(e / D) * LD + (e % D)] = Wt[e];
+  __syncthreads();
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* qrow = qs + warp * D;
+  int s_end = min(S, (int)(blockIdx.y + 1) * TT);
+  for (int s = blockIdx.y * TT + warp; s < s_end; s += 8) {
+    long long n = (long long)f * S + s;
+    long long base = ((b * N + n) * H + h) * D;
+    for (int c = lane; c < D; c += 32) qrow[c] = qf[base + c];
+    __syncwarp();
+    float o[PER];
+    float ss = 0.f;
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      int i = lane + 32 * r;
+      float acc = 0.f;
+      if (i < D) {
+        for (int j = 0; j < D; ++j) acc = fmaf(Ws[i * LD + j], qrow[j], acc);
+      }
+      o[r] = acc;
+      ss += acc * acc;
+    }
+    ss = warp_sum(ss);
+    float inv = rsqrtf(ss / D + kRmsEps);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      int i = lane + 32 * r;
+      if (i < D) out[base + i] = from_f32<T>(o[r] * inv * rms_w[i] * to_f32(gate[base + i]));
+    }
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W) {
+  dim3 grid((unsigned)a.NF(), (unsigned)((a.sh.S + 63) / 64));
+  int d = a.sh.d;
+  size_t smem = ((size_t)d * (d + 1) + 8 * d) * sizeof(float);
+  auto go = [&](auto kern, auto tag) {
+    using T = decltype(tag);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, 256, smem, a.stream>>>(qf, (const T*)a.gate, a.rms_w, W, (T*)a.out, a.sh.H, a.sh.F, a.sh.S);
+  };
+  if (a.sh.dtype == VDN_DTYPE_BF16) {
+    if (d == 16) go(k_readout_simt<__nv_bfloat16, 16>, __nv_bfloat16());
+    else go(k_readout_simt<__nv_bfloat16, 128>, __nv_bfloat16());
+  } else {
+    if (d == 16) go(k_readout_simt<float, 16>, float());
+    else go(k_readout_simt<float, 128>, float());
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- standalone Step 1
+cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,
+                                const float* wk, const float* wv, void* qo, void* ko, void* vo,
+                                cudaStream_t st) {
+  if (sh.dtype == VDN_DTYPE_BF16)
+    return features_dispatch<__nv_bfloat16, __nv_bfloat16>(sh, q, k, v, wk, wv, qo, ko, vo, st);
+  return features_dispatch<float, float>(sh, q, k, v, wk, wv, qo, ko, vo, st);
+}
+
+// ---------------------------------------------------------------- debug copies
+__global__ void k_copy(const float* __restrict__ s, float* __restrict__ d, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    d[i] = s[i];
+}
+
+cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst) {
+  long long n = a.NF() * a.sh.d * a.sh.d;
+  k_copy<<<1184, 256, 0, a.stream>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

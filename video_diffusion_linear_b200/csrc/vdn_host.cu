@@ -1,0 +1,303 @@
+// C ABI of libvdn: argument validation, the workspace plan and the launch
+// sequence of the branch on the caller's stream.  See include/vdn.h.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "image.cuh"
+#include "internal.h"
+
+using namespace vdn;
+
+namespace vdn {
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+#ifndef VDN_HAVE_TC
+#define VDN_HAVE_TC 0
+#endif
+
+bool use_tc(const vdn_shape& sh, int impl) {
+  bool ok = sh.dtype == VDN_DTYPE_BF16 && sh.d == 128;
+  if (impl == VDN_IMPL_SIMT) return false;
+  if (impl == VDN_IMPL_AUTO && !VDN_HAVE_TC) return false;
+  return ok;
+}
+
+WsPlan plan_workspace(const vdn_shape& sh, int /*rule*/, bool tc) {
+  WsPlan p;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t d = (size_t)sh.d;
+  const size_t NF = (size_t)sh.B * sh.H * sh.F;
+  const size_t frame_mats = NF * d * d * sizeof(float);
+  p.status = take(256);
+  if (!tc) {
+    const size_t feat = (size_t)sh.B * sh.F * sh.S * sh.H * d * sizeof(float);
+    p.qf = take(feat);
+    p.kf = take(feat);
+    p.vf = take(feat);
+    p.A = take(frame_mats);
+    p.Bm = take(frame_mats);
+    p.Nm = take(frame_mats);
+    p.P = take(frame_mats);
+    p.Q = take(frame_mats);
+    p.W = take(frame_mats);
+  } else {
+    const size_t slots = NF + kStatsGrid;
+    p.part = take(slots * d * 2 * d * sizeof(float));
+    p.Bm = take(frame_mats);
+    p.nimg = take(NF * (size_t)kImgBytes);
+    p.P = take(frame_mats);
+    p.Q = take(frame_mats);
+    p.wimg = take(NF * (size_t)kImgBytes);
+  }
+  p.total = off;
+  return p;
+}
+
+}  // namespace vdn
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+vdn_status check_shape(const vdn_shape* sh) {
+  if (!sh) return VDN_ERR_INVALID_ARG;
+  if (sh->B < 1 || sh->H < 1 || sh->F < 1 || sh->S < 1 || sh->d < 1 || sh->conv_width < 1)
+    return VDN_ERR_INVALID_ARG;
+  if (sh->dtype != VDN_DTYPE_F32 && sh->dtype != VDN_DTYPE_BF16) return VDN_ERR_INVALID_ARG;
+  if (sh->d != 16 && sh->d != 128) return VDN_ERR_UNSUPPORTED;
+  if (sh->conv_width != 1 && sh->conv_width != 3) return VDN_ERR_UNSUPPORTED;
+  if (sh->dtype == VDN_DTYPE_BF16 && sh->d != 128) return VDN_ERR_UNSUPPORTED;
+  // index ranges used by the kernels: tokens of one batch element and frame
+  // triples must fit in int32, and the whole tensor in 2^62 bytes.
+  long long N = (long long)sh->F * sh->S;
+  long long NF = (long long)sh->B * sh->H * sh->F;
+  if (N > 0x7fffffffLL || NF > 0x7fffffffLL || 2LL * sh->B * sh->H > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  double bytes = (double)sh->B * N * sh->H * sh->d * 4.0;
+  if (bytes > 4.0e18) return VDN_ERR_UNSUPPORTED;
+  return VDN_OK;
+}
+
+size_t elem_size(int dtype) { return dtype == VDN_DTYPE_BF16 ? 2 : 4; }
+
+vdn_status validate(const vdn_shape* sh, const void* q, const void* k, const void* v, const float* beta,
+                    const float* alpha, const void* gate, const float* rms_w, const float* conv_k_w,
+                    const float* conv_v_w, const float* text_state, int rule, float c, int chunk, int radius,
+                    void* workspace, size_t workspace_bytes, void* out, int impl) {
+  vdn_status s = check_shape(sh);
+  if (s != VDN_OK) return s;
+  if (rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE) return VDN_ERR_INVALID_ARG;
+  if (impl < VDN_IMPL_AUTO || impl > VDN_IMPL_TC) return VDN_ERR_INVALID_ARG;
+  if (impl == VDN_IMPL_TC && !(sh->dtype == VDN_DTYPE_BF16 && sh->d == 128)) return VDN_ERR_UNSUPPORTED;
+  if (chunk < 1 || radius < 0 || !std::isfinite(c)) return VDN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !beta || !alpha || !gate || !rms_w || !out || !workspace) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, out};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  if (!aligned(workspace, 256)) return VDN_ERR_ALIGNMENT;
+  WsPlan plan = plan_workspace(*sh, rule, use_tc(*sh, impl));
+  if (workspace_bytes < plan.total) return VDN_ERR_WORKSPACE;
+  // out must not overlap any input nor the workspace
+  const size_t es = elem_size(sh->dtype);
+  const size_t tok = (size_t)sh->B * sh->F * sh->S * sh->H;
+  const size_t big = tok * sh->d * es;
+  const size_t d = (size_t)sh->d;
+  Range ro{(uintptr_t)out, (uintptr_t)out + big};
+  Range rin[] = {
+      {(uintptr_t)q, (uintptr_t)q + big},
+      {(uintptr_t)k, (uintptr_t)k + big},
+      {(uintptr_t)v, (uintptr_t)v + big},
+      {(uintptr_t)gate, (uintptr_t)gate + big},
+      {(uintptr_t)beta, (uintptr_t)beta + tok * 4},
+      {(uintptr_t)alpha, (uintptr_t)alpha + (size_t)sh->B * sh->F * sh->H * d * 4},
+      {(uintptr_t)rms_w, (uintptr_t)rms_w + d * 4},
+      {(uintptr_t)conv_k_w, conv_k_w ? (uintptr_t)conv_k_w + (size_t)sh->H * d * sh->conv_width * 4 : 0},
+      {(uintptr_t)conv_v_w, conv_v_w ? (uintptr_t)conv_v_w + (size_t)sh->H * d * sh->conv_width * 4 : 0},
+      {(uintptr_t)text_state, text_state ? (uintptr_t)text_state + (size_t)sh->H * d * d * 4 : 0},
+      {(uintptr_t)workspace, (uintptr_t)workspace + plan.total},
+  };
+  for (const Range& r : rin)
+    if (r.hi > r.lo && overlap(ro, r)) return VDN_ERR_INVALID_ARG;
+  return VDN_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+#define VDN_LAUNCH(expr)                   \
+  do {                                     \
+    cudaError_t e_ = (expr);               \
+    if (e_ != cudaSuccess) return VDN_ERR_CUDA; \
+  } while (0)
+
+vdn_status run_forward(const Args& a, void* ws, int impl) {
+  const bool tc = use_tc(a.sh, impl);
+  WsPlan p = plan_workspace(a.sh, a.rule, tc);
+  const vdn_debug_out* dbg = a.dbg;
+  uint32_t* status = at<uint32_t>(ws, p.status);
+  VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), a.stream));
+  if (!tc) {
+    float *qf = at<float>(ws, p.qf), *kf = at<float>(ws, p.kf), *vf = at<float>(ws, p.vf);
+    float *A = at<float>(ws, p.A), *Bm = at<float>(ws, p.Bm), *Nm = at<float>(ws, p.Nm);
+    float *P = at<float>(ws, p.P), *Q = at<float>(ws, p.Q), *W = at<float>(ws, p.W);
+    VDN_LAUNCH(launch_features_simt(a, qf, kf, vf));
+    VDN_LAUNCH(launch_stats_simt(a, kf, vf, A, Bm));
+    VDN_LAUNCH(launch_solve(a, A, Nm, nullptr, nullptr, nullptr, nullptr));
+    VDN_LAUNCH(launch_scan_simt(a, Bm, Nm, P, Q));
+    VDN_LAUNCH(launch_gather(a, P, Q, W, nullptr));
+    VDN_LAUNCH(launch_readout_simt(a, qf, W));
+    if (dbg) {
+      if (dbg->A) VDN_LAUNCH(launch_copy_frames(a, A, dbg->A));
+      if (dbg->B) VDN_LAUNCH(launch_copy_frames(a, Bm, dbg->B));
+      if (dbg->N) VDN_LAUNCH(launch_copy_frames(a, Nm, dbg->N));
+      if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P));
+      if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q));
+      if (dbg->W) VDN_LAUNCH(launch_copy_frames(a, W, dbg->W));
+    }
+    return VDN_OK;
+  }
+  float* part = at<float>(ws, p.part);
+  float* Bsum = at<float>(ws, p.Bm);
+  uint16_t* nimg = at<uint16_t>(ws, p.nimg);
+  float *P = at<float>(ws, p.P), *Q = at<float>(ws, p.Q);
+  uint16_t* wimg = at<uint16_t>(ws, p.wimg);
+  bool all_frames = dbg && (dbg->P || dbg->Q);
+  VDN_LAUNCH(launch_stats_tc(a, part, status));
+  VDN_LAUNCH(launch_solve(a, nullptr, dbg ? dbg->N : nullptr, nimg, part, Bsum, dbg ? dbg->A : nullptr));
+  VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, P, Q, all_frames, status));
+  VDN_LAUNCH(launch_gather(a, P, Q, dbg ? dbg->W : nullptr, wimg));
+  VDN_LAUNCH(launch_readout_tc(a, wimg, status));
+  if (dbg) {
+    if (dbg->B) VDN_LAUNCH(launch_copy_frames(a, Bsum, dbg->B));
+    if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P));
+    if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q));
+  }
+  return VDN_OK;
+}
+
+vdn_status forward_common(const vdn_shape* shape, const void* q, const void* k, const void* v, const float* beta,
+                          const float* alpha, const void* gate, const float* rms_w, const float* conv_k_w,
+                          const float* conv_v_w, const float* text_state, int rule, float c, int chunk, int radius,
+                          void* workspace, size_t workspace_bytes, void* out, void* stream,
+                          const vdn_debug_out* dbg) {
+  int impl = dbg ? dbg->impl : VDN_IMPL_AUTO;
+  vdn_status s = validate(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                          radius, workspace, workspace_bytes, out, impl);
+  if (s != VDN_OK) return s;
+  if (dbg) {
+    const float* dp[] = {dbg->A, dbg->B, dbg->N, dbg->P, dbg->Q, dbg->W};
+    for (const float* p : dp)
+      if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  }
+  Args a;
+  a.sh = *shape;
+  a.q = q; a.k = k; a.v = v;
+  a.beta = beta; a.alpha = alpha; a.gate = gate; a.rms_w = rms_w;
+  a.conv_k_w = conv_k_w; a.conv_v_w = conv_v_w; a.text_state = text_state;
+  a.rule = rule; a.c = (rule == VDN_RULE_VDN_SOLVE || rule == VDN_RULE_ADDITIVE) ? 1.0f : c;
+  a.chunk = chunk; a.radius = radius;
+  a.out = out;
+  a.stream = (cudaStream_t)stream;
+  a.dbg = dbg;
+  return run_forward(a, workspace, impl);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vdn_branch_workspace_size_impl(const vdn_shape* shape, int rule, int impl) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  if (rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE) return 0;
+  if (impl < VDN_IMPL_AUTO || impl > VDN_IMPL_TC) return 0;
+  if (impl == VDN_IMPL_TC && !(shape->dtype == VDN_DTYPE_BF16 && shape->d == 128)) return 0;
+  return plan_workspace(*shape, rule, use_tc(*shape, impl)).total;
+}
+
+size_t vdn_branch_workspace_size(const vdn_shape* shape, int rule) {
+  return vdn_branch_workspace_size_impl(shape, rule, VDN_IMPL_AUTO);
+}
+
+vdn_status vdn_branch_forward(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                              const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                              const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,
+                              float c, int chunk, int radius, void* workspace, size_t workspace_bytes, void* out,
+                              void* stream) {
+  return forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                        radius, workspace, workspace_bytes, out, stream, nullptr);
+}
+
+vdn_status vdn_branch_forward_debug(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w, const float* text_state,
+                                    int rule, float c, int chunk, int radius, void* workspace,
+                                    size_t workspace_bytes, void* out, void* stream, const vdn_debug_out* dbg) {
+  return forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                        radius, workspace, workspace_bytes, out, stream, dbg);
+}
+
+vdn_status vdn_feature_prep(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                            const float* conv_k_w, const float* conv_v_w, void* q_out, void* k_out, void* v_out,
+                            void* stream) {
+  vdn_status s = check_shape(shape);
+  if (s != VDN_OK) return s;
+  if (!q || !k || !v || !q_out || !k_out || !v_out) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, conv_k_w, conv_v_w, q_out, k_out, v_out};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  const size_t big = (size_t)shape->B * shape->F * shape->S * shape->H * shape->d * elem_size(shape->dtype);
+  const void* ins[] = {q, k, v};
+  void* outs[] = {q_out, k_out, v_out};
+  for (void* o : outs)
+    for (const void* i : ins)
+      if (overlap({(uintptr_t)o, (uintptr_t)o + big}, {(uintptr_t)i, (uintptr_t)i + big})) return VDN_ERR_INVALID_ARG;
+  if (overlap({(uintptr_t)q_out, (uintptr_t)q_out + big}, {(uintptr_t)k_out, (uintptr_t)k_out + big}) ||
+      overlap({(uintptr_t)q_out, (uintptr_t)q_out + big}, {(uintptr_t)v_out, (uintptr_t)v_out + big}) ||
+      overlap({(uintptr_t)k_out, (uintptr_t)k_out + big}, {(uintptr_t)v_out, (uintptr_t)v_out + big}))
+    return VDN_ERR_INVALID_ARG;
+  cudaError_t e = launch_feature_prep(*shape, q, k, v, conv_k_w, conv_v_w, q_out, k_out, v_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+vdn_status vdn_window_bounds(int t, int F, int chunk, int radius, int* lo, int* hi) {
+  if (!lo || !hi || F < 1 || t < 0 || t >= F || chunk < 1 || radius < 0) return VDN_ERR_INVALID_ARG;
+  vdn::window_bounds(t, F, chunk, radius, *lo, *hi);
+  return VDN_OK;
+}
+
+vdn_status vdn_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < 256) return VDN_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VDN_ERR_CUDA;
+  return word == 0 ? VDN_OK : VDN_ERR_TIMEOUT;
+}
+
+const char* vdn_status_string(int status) {
+  switch (status) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument";
+    case VDN_ERR_UNSUPPORTED: return "unsupported size or type";
+    case VDN_ERR_ALIGNMENT: return "misaligned pointer";
+    case VDN_ERR_WORKSPACE: return "workspace too small";
+    case VDN_ERR_CUDA: return "CUDA error";
+    case VDN_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"
