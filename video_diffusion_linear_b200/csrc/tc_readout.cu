@@ -1,0 +1,286 @@
+// Read-out, RMSNorm and output gate on the tensor cores (page section "Step 5").
+//
+// Persistent kernel: CTA i owns a contiguous range of 128-token tiles in the
+// order (batch, head, frame, tile), so W_t changes only at frame boundaries.
+// Per tile, O[128 tokens x 128] = Q'[128 x 128] W_t^T runs as tcgen05 MMAs with
+// the accumulator in TMEM (two buffers), Q' = L2(SiLU(q)) produced in place in
+// shared memory, and W_t given as a bf16 hi/lo image (two MMAs, fp32 accumulate).
+// The epilogue reads one token row per thread from TMEM (32x32b layout), so the
+// RMSNorm needs no cross-thread reduction; it multiplies rms_w and the gate and
+// writes bf16 through shared memory and a TMA store.
+//
+// Warp roles (320 threads): 0 TMA producer, 1 MMA issuer (and TMEM owner),
+// 2-5 q transform (one token row each), 6-9 epilogue (one TMEM lane each).
+#include "common.cuh"
+#include "image.cuh"
+#include "internal.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace vdn {
+
+namespace {
+
+struct __align__(1024) ReadSmem {
+  uint8_t wimg[65536];     // W_t hi | lo (K-major SW128 B operand)
+  uint8_t qt[2][32768];    // raw q tile -> Q' (K-major SW128 A operand), two stages
+  uint8_t gt[2][32768];    // gate tile -> output tile, two stages
+  float rms_w[128];
+  uint64_t bar_w_full, bar_w_empty;
+  uint64_t bar_q_full[2], bar_q_ready[2], bar_q_empty[2];
+  uint64_t bar_g_full[2], bar_g_empty[2];
+  uint64_t bar_acc_full[2], bar_acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, false, false);
+constexpr int kThreads = 320;
+
+// swizzled byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] bf16 tile
+__device__ __forceinline__ uint32_t row_chunk(int r, int c) {
+  return (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constant__ CUtensorMap tmQ,
+                                                           const __grid_constant__ CUtensorMap tmG,
+                                                           const __grid_constant__ CUtensorMap tmO,
+                                                           const uint16_t* __restrict__ wimg_g,
+                                                           const float* __restrict__ rms_w, int H, int F,
+                                                           int ntile, long long T, uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  ReadSmem& sm = *reinterpret_cast<ReadSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort;
+  const long long G = gridDim.x;
+  const long long x0 = (long long)blockIdx.x * T / G, x1 = ((long long)blockIdx.x + 1) * T / G;
+
+  if (tid == 0) {
+    tc::mbar_init(&sm.bar_w_full, 1);
+    tc::mbar_init(&sm.bar_w_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&sm.bar_q_full[s], 1);
+      tc::mbar_init(&sm.bar_q_ready[s], 128);
+      tc::mbar_init(&sm.bar_q_empty[s], 1);
+      tc::mbar_init(&sm.bar_g_full[s], 1);
+      tc::mbar_init(&sm.bar_g_empty[s], 1);
+      tc::mbar_init(&sm.bar_acc_full[s], 1);
+      tc::mbar_init(&sm.bar_acc_empty[s], 128);
+    }
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, 256);
+    tc::tmem_relinquish();
+  }
+  if (tid >= 192) sm.rms_w[tid - 192] = rms_w[tid - 192];
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  auto coords = [&](long long x, int& h, int& s0, int& fb) {
+    long long fi = x / ntile;
+    int j = (int)(x % ntile);
+    int t = (int)(fi % F);
+    long long bh = fi / F;
+    h = (int)(bh % H);
+    fb = (int)((bh / H) * F + t);
+    s0 = j * 128;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      long long cur = -1;
+      uint32_t wph = 0;
+      int it = 0;
+      for (long long x = x0; x < x1; ++x, ++it) {
+        long long fi = x / ntile;
+        if (fi != cur) {
+          if (cur >= 0) {
+            if (!tc::mbar_wait(&sm.bar_w_empty, wph, abort_flag, status)) break;
+            wph ^= 1;
+          }
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(wimg_g + fi * (kImgBytes / 2));
+          tc::mbar_arrive_expect_tx(&sm.bar_w_full, kImgBytes);
+          for (int q = 0; q < 4; ++q) tc::bulk_load(sm.wimg + q * 16384, src + q * 16384, 16384, &sm.bar_w_full);
+          cur = fi;
+        }
+        int h, s0, fb;
+        coords(x, h, s0, fb);
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&sm.bar_q_empty[st], ph ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.bar_q_full[st], 32768);
+        tc::tma_load_4d(&tmQ, &sm.bar_q_full[st], sm.qt[st], 0, h, s0, fb);
+        tc::tma_load_4d(&tmQ, &sm.bar_q_full[st], sm.qt[st] + 16384, 64, h, s0, fb);
+        if (!tc::mbar_wait(&sm.bar_g_empty[st], ph ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.bar_g_full[st], 32768);
+        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st], 0, h, s0, fb);
+        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st] + 16384, 64, h, s0, fb);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      long long cur = -1;
+      uint32_t wph = 0;
+      int it = 0;
+      const uint32_t w_hi = tc::smem_u32(sm.wimg), w_lo = w_hi + 32768;
+      for (long long x = x0; x < x1; ++x, ++it) {
+        long long fi = x / ntile;
+        if (fi != cur) {
+          if (!tc::mbar_wait(&sm.bar_w_full, wph, abort_flag, status)) break;
+          wph ^= 1;
+          cur = fi;
+        }
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&sm.bar_q_ready[st], ph, abort_flag, status)) break;
+        if (!tc::mbar_wait(&sm.bar_acc_empty[st], ph ^ 1, abort_flag, status)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + st * 128;
+        const uint32_t a = tc::smem_u32(sm.qt[st]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          uint64_t ad = tc::smem_desc(a + koff, 16, 1024);
+          tc::umma_bf16(d, ad, tc::smem_desc(w_hi + koff, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+          tc::umma_bf16(d, ad, tc::smem_desc(w_lo + koff, 16, 1024), kIdesc, 1u);
+        }
+        tc::umma_commit(&sm.bar_q_empty[st]);
+        tc::umma_commit(&sm.bar_acc_full[st]);
+        if (x + 1 == x1 || (x + 1) / ntile != fi) tc::umma_commit(&sm.bar_w_empty);
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ q' = L2(SiLU(q)), in place
+    const int r = tid - 64;
+    int it = 0;
+    for (long long x = x0; x < x1; ++x, ++it) {
+      const int st = it & 1;
+      const uint32_t ph = (it >> 1) & 1;
+      if (!tc::mbar_wait(&sm.bar_q_full[st], ph, abort_flag, status)) break;
+      uint8_t* base = sm.qt[st];
+      float v[128];
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
+        uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float a0 = silu_fast(bf16lo(ws[e])), a1 = silu_fast(bf16hi(ws[e]));
+          v[8 * c + 2 * e] = a0;
+          v[8 * c + 2 * e + 1] = a1;
+          ss = fmaf(a0, a0, ss);
+          ss = fmaf(a1, a1, ss);
+        }
+      }
+      const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * c + 0] * inv, v[8 * c + 1] * inv);
+        w.y = pack_bf16x2(v[8 * c + 2] * inv, v[8 * c + 3] * inv);
+        w.z = pack_bf16x2(v[8 * c + 4] * inv, v[8 * c + 5] * inv);
+        w.w = pack_bf16x2(v[8 * c + 6] * inv, v[8 * c + 7] * inv);
+        *reinterpret_cast<uint4*>(base + row_chunk(r, c)) = w;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&sm.bar_q_ready[st]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;
+    const bool leader = tid == 192;
+    int it = 0;
+    for (long long x = x0; x < x1; ++x, ++it) {
+      const int st = it & 1;
+      const uint32_t ph = (it >> 1) & 1;
+      if (leader && it > 0) {
+        tc::bulk_wait_read_all();                       // the previous tile's store has read its buffer
+        tc::mbar_arrive(&sm.bar_g_empty[(it - 1) & 1]);
+      }
+      if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
+      tc::tc_fence_after();
+      float o[128];
+      const uint32_t taddr = tmem + st * 128 + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t rr[32];
+        tc::tmem_ld32(taddr + 32 * j, rr);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[32 * j + e] = __uint_as_float(rr[e]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&sm.bar_acc_empty[st]);
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < 128; ++k) ss = fmaf(o[k], o[k], ss);
+      const float inv = rsqrtf(ss * (1.0f / 128.0f) + kRmsEps);
+      if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
+      uint8_t* base = sm.gt[st];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4 g = *reinterpret_cast<const uint4*>(base + row_chunk(m, c));
+        uint32_t gs[4] = {g.x, g.y, g.z, g.w};
+        uint32_t outw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int k = 8 * c + 2 * e;
+          float y0 = o[k] * inv * sm.rms_w[k] * bf16lo(gs[e]);
+          float y1 = o[k + 1] * inv * sm.rms_w[k + 1] * bf16hi(gs[e]);
+          outw[e] = pack_bf16x2(y0, y1);
+        }
+        *reinterpret_cast<uint4*>(base + row_chunk(m, c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+      }
+      tc::fence_proxy_async_smem();
+      tc::named_bar(1, 128);
+      if (leader) {
+        int h, s0, fb;
+        coords(x, h, s0, fb);
+        tc::tma_store_4d(&tmO, base, 0, h, s0, fb);
+        tc::tma_store_4d(&tmO, base + 16384, 64, h, s0, fb);
+        tc::bulk_commit();
+      }
+    }
+    if (leader) tc::bulk_wait_all();
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, uint32_t* status) {
+  const vdn_shape& sh = a.sh;
+  CUtensorMap tq, tg, to;
+  long long BF = (long long)sh.B * sh.F;
+  if (!tmap_tokens_bf16(&tq, a.q, sh.d, sh.H, sh.S, BF, 128) ||
+      !tmap_tokens_bf16(&tg, a.gate, sh.d, sh.H, sh.S, BF, 128) ||
+      !tmap_tokens_bf16(&to, a.out, sh.d, sh.H, sh.S, BF, 128))
+    return cudaErrorInvalidValue;
+  int ntile = (sh.S + 127) / 128;
+  long long T = a.NF() * ntile;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long G = T < sms ? T : sms;
+  size_t smem = sizeof(ReadSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_readout_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tq, tg, to, wimg, a.rms_w, sh.H, sh.F, ntile, T, status);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

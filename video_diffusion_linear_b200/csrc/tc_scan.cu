@@ -1,0 +1,214 @@
+// Bidirectional scan of the delta rule on the tensor cores (page sections
+// "Step 3" and "Step 4": the forward prefix scan and backward suffix scan over
+// frames, each seeded with 0.5 x the text state).
+//
+// One CTA per (batch, head, direction) walks the frames serially:
+//     X_f = S_{f-1} D_f + cpre B_f            (fp32, one state row per thread)
+//     S_f = X_f N_f + cpost B_f               (tcgen05, 128x128x128)
+// The product runs in bf16 with hi/lo splitting of both operands
+// (X = Xh + Xl, N = Nh + Nl; D = Xh Nh + Xh Nl + Xl Nh), which keeps about 16
+// significant bits in every term and accumulates in fp32 in TMEM, so the state
+// stays an fp32 quantity at tensor-core speed.  N_f arrives as a pre-swizzled
+// operand image (written by the per-frame solve) through one bulk copy, B_f
+// through TMA with a 128-byte swizzle so that each thread reads its own row
+// without bank conflicts.  Only the states the window gather needs are stored:
+// P at chunk ends, Q at chunk starts (or every frame for the debug export).
+#include "common.cuh"
+#include "image.cuh"
+#include "internal.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace vdn {
+
+namespace {
+
+struct __align__(1024) ScanSmem {
+  uint8_t aop[2][32768];     // X hi, X lo: K-major SW128 A operands
+  uint8_t nimg[65536];       // N_f hi | lo image
+  float bf[4][128 * 32];     // B_f, four swizzled [128 rows][32 cols] boxes
+  float alpha[128];
+  uint64_t bar_n, bar_b, bar_mma;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, false, false);
+
+// byte offset of B_f[row][col] inside the swizzled box array
+__device__ __forceinline__ uint32_t bf_offset(int row, int col) {
+  int box = col >> 5, c16 = (col & 31) >> 2;
+  return box * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4) + (col & 3) * 4;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmB,
+                                                   const uint16_t* __restrict__ nimg_g,
+                                                   const float* __restrict__ alpha,
+                                                   const float* __restrict__ text, RuleCoef rc,
+                                                   float* __restrict__ P, float* __restrict__ Q, int H, int F,
+                                                   int chunk, int all_frames, uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int m = threadIdx.x;
+  const int warp = m >> 5;
+  const int dir = blockIdx.x & 1;
+  const long long bh = blockIdx.x >> 1;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  volatile int* abort_flag = &sm.abort;
+
+  if (m == 0) {
+    tc::mbar_init(&sm.bar_n, 1);
+    tc::mbar_init(&sm.bar_b, 1);
+    tc::mbar_init(&sm.bar_mma, 1);
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&sm.tmem_base, 128);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+
+  float s[128];
+  {
+    const float* T = text ? text + ((long long)h * 128 + m) * 128 : nullptr;
+#pragma unroll
+    for (int k = 0; k < 128; ++k) s[k] = T ? kTextStateScale * T[k] : 0.f;
+  }
+
+  auto frame_of = [&](int step) { return dir == 0 ? step : F - 1 - step; };
+  auto load_n = [&](int step) {
+    long long fi = bh * F + frame_of(step);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2));
+    tc::mbar_arrive_expect_tx(&sm.bar_n, kImgBytes);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tc::bulk_load(sm.nimg + j * 16384, src + j * 16384, 16384, &sm.bar_n);
+  };
+  auto load_b = [&](int step) {
+    long long fi = bh * F + frame_of(step);
+    tc::mbar_arrive_expect_tx(&sm.bar_b, 65536);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tc::tma_load_2d(&tmB, &sm.bar_b, sm.bf[j], 32 * j, (int)(fi * 128));
+  };
+  if (m == 0) {
+    load_n(0);
+    load_b(0);
+  }
+
+  const bool early_b = rc.cpost == 0.f;   // B_f is only read before the product
+  uint32_t ph = 0;
+  const uint32_t a_hi = tc::smem_u32(sm.aop[0]), a_lo = tc::smem_u32(sm.aop[1]);
+  const uint32_t n_hi = tc::smem_u32(sm.nimg), n_lo = n_hi + 32768;
+  const uint8_t* bfb = reinterpret_cast<const uint8_t*>(sm.bf);
+
+  for (int step = 0; step < F; ++step) {
+    const int f = frame_of(step);
+    const long long fi = bh * F + f;
+    sm.alpha[m] = alpha[((b * F + f) * H + h) * 128 + m];
+    __syncthreads();
+    if (!tc::mbar_wait(&sm.bar_b, ph, abort_flag, status)) break;
+
+    // X = S D + cpre B  ->  bf16 hi / lo A operands (row m)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float4 b0 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, 8 * c));
+      float4 b1 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, 8 * c + 4));
+      float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float x0 = fmaf(s[8 * c + e], sm.alpha[8 * c + e], rc.cpre * bv[e]);
+        float x1 = fmaf(s[8 * c + e + 1], sm.alpha[8 * c + e + 1], rc.cpre * bv[e + 1]);
+        float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+        float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+        hw[e / 2] = pack_bf16x2(h0, h1);
+        lw[e / 2] = pack_bf16x2(x0 - h0, x1 - h1);
+      }
+      uint32_t off = img_offset(0, m, 8 * c);
+      *reinterpret_cast<uint4*>(sm.aop[0] + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm.aop[1] + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+
+    if (m == 0) {
+      if (early_b && step + 1 < F) load_b(step + 1);
+      if (tc::mbar_wait(&sm.bar_n, ph, abort_flag, status)) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          uint64_t ah = tc::smem_desc(a_hi + koff, 16, 1024), al = tc::smem_desc(a_lo + koff, 16, 1024);
+          uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024), bld = tc::smem_desc(n_lo + koff, 16, 1024);
+          tc::umma_bf16(tmem, ah, bhd, kIdesc, kk > 0 ? 1u : 0u);
+          tc::umma_bf16(tmem, ah, bld, kIdesc, 1u);
+          tc::umma_bf16(tmem, al, bhd, kIdesc, 1u);
+        }
+        tc::umma_commit(&sm.bar_mma);
+      }
+    }
+    if (!tc::mbar_wait(&sm.bar_mma, ph, abort_flag, status)) break;
+    tc::tc_fence_after();
+    if (m == 0 && step + 1 < F) load_n(step + 1);   // the product that read N_f is complete
+
+    // S_f = D + cpost B_f
+    const bool store = all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0));
+    float* dst = (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t r[32];
+      tc::tmem_ld32(t_row + 32 * j, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        // with early_b the buffer already receives B_{f+1}: do not read it
+        float4 bv = early_b ? make_float4(0.f, 0.f, 0.f, 0.f)
+                            : *reinterpret_cast<const float4*>(bfb + bf_offset(m, 32 * j + e));
+        s[32 * j + e + 0] = fmaf(rc.cpost, bv.x, __uint_as_float(r[e + 0]));
+        s[32 * j + e + 1] = fmaf(rc.cpost, bv.y, __uint_as_float(r[e + 1]));
+        s[32 * j + e + 2] = fmaf(rc.cpost, bv.z, __uint_as_float(r[e + 2]));
+        s[32 * j + e + 3] = fmaf(rc.cpost, bv.w, __uint_as_float(r[e + 3]));
+        if (store)
+          *reinterpret_cast<float4*>(dst + 32 * j + e) =
+              make_float4(s[32 * j + e], s[32 * j + e + 1], s[32 * j + e + 2], s[32 * j + e + 3]);
+      }
+    }
+    tc::tc_fence_before();
+    __syncthreads();   // accumulator and B_f reads done, alpha slot free
+    if (m == 0 && !early_b && step + 1 < F) load_b(step + 1);
+    ph ^= 1;
+  }
+
+  // teardown: make sure no copy or product of ours is still in flight
+  __syncthreads();
+  if (sm.abort && m == 0) {
+    tc::mbar_wait(&sm.bar_n, ph, abort_flag, nullptr);
+    tc::mbar_wait(&sm.bar_b, ph, abort_flag, nullptr);
+  }
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
+cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q,
+                           bool all_frames, uint32_t* status) {
+  CUtensorMap tmB;
+  if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
+  size_t smem = sizeof(ScanSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  RuleCoef rc = rule_coef(a.rule, a.c);
+  k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), 128, smem, a.stream>>>(
+      tmB, nimg, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, status);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

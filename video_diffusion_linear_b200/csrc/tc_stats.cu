@@ -1,0 +1,312 @@
+// Frame statistics on the tensor cores (page sections "Step 1" and "Step 2").
+//
+// For every (batch, head, frame):  A_f = sum_s beta_s k'_s k'_s^T,
+//                                  B_f = sum_s beta_s v'_s k'_s^T,
+// a dense contraction over the frame's S tokens.  With X = sqrt(beta) k' and
+// Y = sqrt(beta) v' (tokens x channels) one MMA of M = 128, N = 256 per 16
+// tokens gives  X^T [X | Y] = [A | B^T]  in a TMEM accumulator, so beta is
+// applied once, while the operands are produced, and no operand is written
+// twice.  The k/v feature prep of Step 1 (short conv within the frame, SiLU,
+// L2 normalisation of k) is fused into that operand production: raw bf16 rows
+// arrive by TMA (64 tokens plus one halo row on each side, zero outside the
+// frame), the transform warps compute X and Y in fp32 and store them as bf16 in
+// the MN-major 128-byte-swizzled layout the tensor cores read.
+//
+// Work split: the (frame, 64-token block) pairs, frames ordered (batch, frame,
+// head), are cut into gridDim.x contiguous ranges (stream-K).  A CTA flushes its
+// accumulator whenever its range leaves a frame, into partial slot
+// (blockIdx.x + frame); the per-frame solve adds the slots of each frame in a
+// fixed order, so the result is deterministic.
+//
+// Warp roles (448 threads): 0 TMA producer, 1 MMA issuer (TMEM owner),
+// 2-9 transform (4 tokens x 8 channels per thread), 10-13 flush (one TMEM lane each).
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace vdn {
+
+namespace {
+
+constexpr int kRS = 3;                 // raw TMA stages
+constexpr int kRawRows = kStatsTokens + 2;
+constexpr int kRawHalf = 9216;         // 66 rows x 128 B, padded to 9 KB (1024-aligned)
+constexpr int kRawBytes = 4 * kRawRows * 128;   // k and v, two channel halves each
+constexpr int kThreads = 448;
+
+struct __align__(1024) StatsSmem {
+  uint8_t raw[kRS][2][2][kRawHalf];    // [stage][k|v][channel half]
+  uint8_t op[2][32768];                // [stage]: X (16 KB) | Y (16 KB), MN-major SW128
+  uint64_t raw_full[kRS], raw_empty[kRS];
+  uint64_t op_full[2], op_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 256, true, true);
+
+// byte offset of the 16-byte chunk holding channels 8c..8c+7 of token t in an
+// MN-major SW128 operand of 128 channels x 64 tokens (atoms of 64 ch x 8 tokens)
+__device__ __forceinline__ uint32_t op_chunk(int c, int t) {
+  return (c >> 3) * 8192 + (t >> 3) * 1024 + (t & 7) * 128 + ((((c & 7) ^ (t & 7))) << 4);
+}
+
+__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
+  f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
+  f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant__ CUtensorMap tmK,
+                                                         const __grid_constant__ CUtensorMap tmV,
+                                                         const float* __restrict__ beta,
+                                                         const float* __restrict__ wk_g, const float* __restrict__ wv_g,
+                                                         int K, int H, int F, int S, int nb, long long T,
+                                                         float* __restrict__ part, uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  StatsSmem& sm = *reinterpret_cast<StatsSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort;
+  const long long G = gridDim.x;
+  const long long x0 = (long long)blockIdx.x * T / G, x1 = ((long long)blockIdx.x + 1) * T / G;
+
+  if (tid == 0) {
+    for (int s = 0; s < kRS; ++s) {
+      tc::mbar_init(&sm.raw_full[s], 1);
+      tc::mbar_init(&sm.raw_empty[s], 256);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&sm.op_full[s], 256);
+      tc::mbar_init(&sm.op_empty[s], 1);
+      tc::mbar_init(&sm.acc_full[s], 1);
+      tc::mbar_init(&sm.acc_empty[s], 128);
+    }
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  // block x -> frame pf (order b, f, h) and block j in the frame
+  auto decode = [&](long long x, int& h, int& fb, int& s0) {
+    long long pf = x / nb;
+    s0 = (int)(x % nb) * kStatsTokens;
+    h = (int)(pf % H);
+    fb = (int)(pf / H);   // b * F + f
+  };
+  auto seg_last = [&](long long x) { return x + 1 == x1 || (x + 1) % nb == 0; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      for (long long x = x0; x < x1; ++x, ++it) {
+        int h, fb, s0;
+        decode(x, h, fb, s0);
+        const int rs = it % kRS;
+        const uint32_t ph = (it / kRS) & 1;
+        if (!tc::mbar_wait(&sm.raw_empty[rs], ph ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.raw_full[rs], kRawBytes);
+        for (int hf = 0; hf < 2; ++hf) {
+          tc::tma_load_4d(&tmK, &sm.raw_full[rs], sm.raw[rs][0][hf], 64 * hf, h, s0 - 1, fb);
+          tc::tma_load_4d(&tmV, &sm.raw_full[rs], sm.raw[rs][1][hf], 64 * hf, h, s0 - 1, fb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, seg = 0;
+      bool first = true;
+      for (long long x = x0; x < x1; ++x, ++it) {
+        const int os = it & 1;
+        const uint32_t oph = (it >> 1) & 1;
+        const int ab = seg & 1;
+        if (first) {
+          if (!tc::mbar_wait(&sm.acc_empty[ab], ((seg >> 1) & 1) ^ 1, abort_flag, status)) break;
+        }
+        if (!tc::mbar_wait(&sm.op_full[os], oph, abort_flag, status)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + ab * 256;
+        const uint32_t base = tc::smem_u32(sm.op[os]);
+#pragma unroll
+        for (int kk = 0; kk < kStatsTokens / 16; ++kk) {
+          uint64_t desc = tc::smem_desc(base + kk * 2048, 8192, 1024);
+          tc::umma_bf16(d, desc, desc, kIdesc, (first && kk == 0) ? 0u : 1u);
+        }
+        tc::umma_commit(&sm.op_empty[os]);
+        first = false;
+        if (seg_last(x)) {
+          tc::umma_commit(&sm.acc_full[ab]);
+          ++seg;
+          first = true;
+        }
+      }
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ transform
+    const int tt = tid - 64;
+    const int w8 = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
+    const int half = c >> 3, cc = c & 7;
+    const int tok0 = 8 * w8 + 4 * tg;       // first of this thread's 4 tokens in the block
+    const long long N = (long long)F * S;
+    int it = 0;
+    for (long long x = x0; x < x1; ++x, ++it) {
+      int h, fb, s0;
+      decode(x, h, fb, s0);
+      const int rs = it % kRS;
+      const uint32_t rph = (it / kRS) & 1;
+      const int os = it & 1;
+      const uint32_t oph = (it >> 1) & 1;
+      // conv taps of this thread's 8 channels (identity when no weights)
+      float wk[3][8], wv[3][8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const long long wi = ((long long)h * 128 + 8 * c + e) * K;
+        wk[0][e] = (wk_g && K == 3) ? wk_g[wi] : 0.f;
+        wk[1][e] = wk_g ? wk_g[wi + (K == 3 ? 1 : 0)] : 1.f;
+        wk[2][e] = (wk_g && K == 3) ? wk_g[wi + 2] : 0.f;
+        wv[0][e] = (wv_g && K == 3) ? wv_g[wi] : 0.f;
+        wv[1][e] = wv_g ? wv_g[wi + (K == 3 ? 1 : 0)] : 1.f;
+        wv[2][e] = (wv_g && K == 3) ? wv_g[wi + 2] : 0.f;
+      }
+      float sb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s = s0 + tok0 + i;
+        const long long n = (long long)(fb / F) * N + (long long)(fb % F) * S + s;
+        sb[i] = s < S ? sqrtf(beta[n * H + h]) : 0.f;
+      }
+      if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
+
+      // ---- k: conv, SiLU, L2 norm, * sqrt(beta)
+      float kx[4][8];
+      float ssq[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        float r[6][8];
+        const uint8_t* src = sm.raw[rs][0][half];
+#pragma unroll
+        for (int rr = 0; rr < 6; ++rr) {
+          const int row = tok0 + rr;
+          unpack8(*reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4)), r[rr]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float a = fmaf(wk[0][e], r[i][e], fmaf(wk[1][e], r[i + 1][e], wk[2][e] * r[i + 2][e]));
+            a = silu_fast(a);
+            kx[i][e] = a;
+            ssq[i] = fmaf(a, a, ssq[i]);
+          }
+      }
+      // ---- v: conv, SiLU, * sqrt(beta)
+      float vx[4][8];
+      {
+        float r[6][8];
+        const uint8_t* src = sm.raw[rs][1][half];
+#pragma unroll
+        for (int rr = 0; rr < 6; ++rr) {
+          const int row = tok0 + rr;
+          unpack8(*reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4)), r[rr]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            vx[i][e] = sb[i] * silu_fast(fmaf(wv[0][e], r[i][e], fmaf(wv[1][e], r[i + 1][e], wv[2][e] * r[i + 2][e])));
+      }
+      tc::mbar_arrive(&sm.raw_empty[rs]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], o);
+        ssq[i] = sb[i] * rsqrtf(ssq[i] + kL2Eps);
+      }
+      if (!tc::mbar_wait(&sm.op_empty[os], oph ^ 1, abort_flag, status)) break;
+      uint8_t* dst = sm.op[os];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = tok0 + i;
+        uint4 wx, wy;
+        wx.x = pack_bf16x2(kx[i][0] * ssq[i], kx[i][1] * ssq[i]);
+        wx.y = pack_bf16x2(kx[i][2] * ssq[i], kx[i][3] * ssq[i]);
+        wx.z = pack_bf16x2(kx[i][4] * ssq[i], kx[i][5] * ssq[i]);
+        wx.w = pack_bf16x2(kx[i][6] * ssq[i], kx[i][7] * ssq[i]);
+        wy.x = pack_bf16x2(vx[i][0], vx[i][1]);
+        wy.y = pack_bf16x2(vx[i][2], vx[i][3]);
+        wy.z = pack_bf16x2(vx[i][4], vx[i][5]);
+        wy.w = pack_bf16x2(vx[i][6], vx[i][7]);
+        *reinterpret_cast<uint4*>(dst + op_chunk(c, t)) = wx;
+        *reinterpret_cast<uint4*>(dst + 16384 + op_chunk(c, t)) = wy;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&sm.op_full[os]);
+    }
+  } else {
+    // ------------------------------------------------------------ flush [A | B^T] partials
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;
+    int seg = 0;
+    for (long long x = x0; x < x1; ++x) {
+      if (!seg_last(x)) continue;
+      const int ab = seg & 1;
+      if (!tc::mbar_wait(&sm.acc_full[ab], (seg >> 1) & 1, abort_flag, status)) break;
+      tc::tc_fence_after();
+      const long long pf = x / nb;
+      float* dst = part + ((long long)blockIdx.x + pf) * (128 * 256) + (long long)m * 256;
+      const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int j = 0; j < 8; ++j) {
+        uint32_t r[32];
+        tc::tmem_ld32(taddr + 32 * j, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<uint4*>(dst + 32 * j + e) = make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&sm.acc_empty[ab]);
+      ++seg;
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status) {
+  const vdn_shape& sh = a.sh;
+  CUtensorMap tk, tv;
+  long long BF = (long long)sh.B * sh.F;
+  if (!tmap_tokens_bf16(&tk, a.k, sh.d, sh.H, sh.S, BF, kRawRows) ||
+      !tmap_tokens_bf16(&tv, a.v, sh.d, sh.H, sh.S, BF, kRawRows))
+    return cudaErrorInvalidValue;
+  int nb = (sh.S + kStatsTokens - 1) / kStatsTokens;
+  long long T = a.NF() * nb;
+  long long G = T < kStatsGrid ? T : kStatsGrid;
+  size_t smem = sizeof(StatsSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int K = (a.conv_k_w || a.conv_v_w) ? sh.conv_width : 1;
+  k_stats_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tk, tv, a.beta, a.conv_k_w, a.conv_v_w, K, sh.H, sh.F, sh.S,
+                                                       nb, T, partials, status);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

@@ -14,7 +14,7 @@ namespace vdn {
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 #ifndef VDN_HAVE_TC
-#define VDN_HAVE_TC 0
+#define VDN_HAVE_TC 1
 #endif
 
 bool use_tc(const vdn_shape& sh, int impl) {
