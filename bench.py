@@ -1,0 +1,429 @@
+"""Benchmark of the VDN-H3 linear-branch forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 768p] [--impl reference]
+
+One step is one vdn_branch_forward call over the whole workload (all heads,
+all frames) with the inputs resident in HBM.  Prints ONE JSON line (rank 0):
+latent tokens/s over all ranks, the roofline of the dominant kernel (live CUDA
+event timing per kernel, algorithmic bytes / duration against the measured HBM
+copy bandwidth), the whole-path roofline fraction, an end-to-end figure through
+the same C ABI with host buffers, clocks sampled during the timed region, and
+the float64 oracle timed on the host cores on a bounded sample.
+
+Multi-GPU (torchrun, one rank per GPU): the branch needs no communication, each
+rank runs its own clip (seed + 1000 * rank) of the same workload: weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from video_diffusion_linear_b200 import synth  # noqa: E402
+
+METRIC = "latent tokens/sec through VDN linear branch fwd (1 B200); % of roofline"
+DEFAULT_WORKLOAD = "768p"
+KERNELS_TC = ["frame_stats", "frame_solve", "scan", "gather", "readout"]
+KERNEL_SOURCES = {"frame_stats": "tc_stats.cu", "frame_solve": "solve_gather.cu", "scan": "tc_scan.cu",
+                  "gather": "solve_gather.cu", "readout": "tc_readout.cu"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ----------------------------------------------------------------------------- workload arithmetic
+def describe(w: synth.Workload) -> str:
+    txt = "with text state" if w.text else "no text state"
+    return (f"{w.name}: B={w.B} H={w.H} d={w.d} F={w.F} S={w.S} ({w.tokens} latent tokens), {w.dtype}, "
+            f"{w.rule} c={w.c}, chunk {w.chunk}, radius {w.radius}, {txt}")
+
+
+def algorithmic_bytes(w: synth.Workload) -> dict:
+    """Bytes each kernel must move at least once ('roofline')."""
+    d = w.d
+    TH = w.B * w.F * w.S * w.H                 # token-heads
+    NF = w.B * w.H * w.F                       # (batch, head, frame) triples
+    mat = d * d * 4                            # one fp32 d x d matrix
+    img = d * d * 2 * 2                        # bf16 hi/lo operand image
+    stored = 2 * w.B * w.H * (-(-w.F // w.chunk))   # chunk-boundary states written by the scan
+    return {
+        "frame_stats": TH * (2 * d * 2 + 4) + NF * 2 * mat,
+        "frame_solve": NF * (2 * mat + mat + img),
+        "scan": 2 * NF * (img + mat) + stored * mat,
+        "gather": NF * (2 * mat + img),
+        "readout": TH * 3 * d * 2 + NF * img,
+    }
+
+
+def path_roofline(w: synth.Workload, peaks: dict) -> dict:
+    """Whole-branch roofline: algorithmic bytes (q, k, v, gate, beta in, out once;
+    per frame alpha, the per-frame maps written and read once, chunk-boundary
+    states) and FLOPs (A, B: 4 d^2 and read-out 2 d^2 per token-head, about
+    7 d^3 per frame for the solve and the two scans)."""
+    d = w.d
+    TH = w.B * w.F * w.S * w.H
+    NF = w.B * w.H * w.F
+    states = 2 * w.B * w.H * (-(-w.F // w.chunk)) * d * d * 4 * 2
+    nbytes = TH * (4 * d * 2 + 4 + d * 2) + NF * (d * 4 + 4 * d * d * 4) + states
+    flops = TH * 6 * d * d + NF * 7 * d ** 3
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    return {"bytes": nbytes, "flops": flops, "t_roof_us": max(t_hbm, t_tc) * 1e6,
+            "bound": "hbm" if t_hbm >= t_tc else "tensor"}
+
+
+def load_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"])}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "video_diffusion_linear_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/dram_traffic.txt: 'kernel workload source_sha1 bytes'), or None when
+    absent or when the kernel's source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and parts[0] == kernel and not line.startswith("#"):
+                if parts[2] == source_hash(KERNEL_SOURCES[kernel]):
+                    return {"workload": parts[1], "bytes": float(parts[3])}
+    return None
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+def dist_env() -> tuple[int, int, int]:
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Each rank runs its own clip of the workload (weak scaling, no exchange)."""
+    return w.replace(seed=w.seed + 1000 * rank)
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every `period` s."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period: float = 0.01):
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = getattr(torch.cuda.get_device_properties(device_index), "uuid", None)
+            h = None
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report it instead of clocks
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                bits = fn(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if self._h is None:
+            return {"error": getattr(self, "error", "nvml unavailable")}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample(inp: dict, w: synth.Workload, heads) -> tuple[float, int]:
+    """Runs the float64 oracle over all frames and tokens of the given heads of
+    batch 0; returns (seconds, token-heads processed)."""
+    from oracle import vdn_oracle as O
+    rms_w = O._f64(inp["rms_w"])
+    t0 = time.perf_counter()
+    for h in heads:
+        st = O.head_state(inp, 0, h, w.F, w.S, w.rule, w.c, w.chunk, w.radius)
+        g = O._f64(inp["gate"][0, :, h, :]).reshape(w.F, w.S, w.d)
+        for t in range(w.F):
+            O.readout(st["W"][t], st["qf"][t], g[t], rms_w)
+    return time.perf_counter() - t0, len(heads) * w.F * w.S
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(blas[0]["num_threads"])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, w: synth.Workload) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    inp = synth.make_inputs(w)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, th = oracle_sample(inp, w, [i % w.H])
+        if i >= args.warmup:
+            times.append(dt)
+    step = sum(times) / len(times)
+    tokens_equiv = th / w.H                    # one head of H: tokens x (1/H)
+    value = tokens_equiv / step
+    cores = blas_threads()
+    sample = f"one head of {w.H} per step (all {w.F} frames x {w.S} tokens), batch 0; tokens counted x 1/H"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(w)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, w: synth.Workload) -> None:
+    from video_diffusion_linear_b200 import _lib, api
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    _lib.load()
+    wr = rank_workload(w, rank)
+    host = synth.make_inputs(wr)
+    dev = api.to_device(host, device)
+    args_t = api.forward_inputs(dev)
+    shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
+    ws = api.alloc_workspace(shape, w.rule, "auto", device)
+    out = torch.empty_like(dev["q"])
+    nl = api.launch_count(shape)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events=None):
+        if events is None:
+            api.branch_forward(*args_t, F=w.F, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius, out=out,
+                               workspace=ws, stream=stream)
+        else:
+            api.branch_forward_timed(*args_t, F=w.F, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius,
+                                     out=out, workspace=ws, stream=stream, events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if api.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+
+    # per-kernel events for every timed step (recorded once so their handles exist)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(args.steps)]
+    for evs in kev:
+        for e in evs:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(kev[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end)
+    ms_max = reduce_max(ms, device)
+    tokens = w.tokens * world * args.steps
+    value = tokens / (ms_max / 1e3)
+
+    names = KERNELS_TC if nl == 5 else [f"kernel{i}" for i in range(nl)]
+    per = {n: statistics.fmean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
+           for j, n in enumerate(names)}
+    peaks, peak_src = load_peaks()
+    alg = algorithmic_bytes(w)
+    dom = max(per, key=per.get)
+    dom_ms = per[dom]
+    achieved = alg.get(dom, 0) / (dom_ms / 1e3) / 1e9 if dom in alg else None
+    traffic = recorded_traffic(dom)
+    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": (achieved / peaks["hbm_gbs"]) if achieved else None, "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": alg.get(dom),
+            "traffic": traffic["bytes"] if traffic else None,
+            "traffic_workload": traffic["workload"] if traffic else None}
+    pr = path_roofline(w, peaks)
+    step_us = ms_max / args.steps * 1e3
+    kernels = {n: {"us": per[n] * 1e3, "share": per[n] / sum(per.values()),
+                   "gbs": (alg[n] / (per[n] / 1e3) / 1e9) if n in alg else None} for n in per}
+
+    # end to end through the same C ABI: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        keys = ["q", "k", "v", "beta", "alpha", "gate"]
+        pinned = {k: host[k].pin_memory() for k in keys}
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
+        d2h = out_host.numel() * out_host.element_size()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        for _ in range(2):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu and world == 1:
+        heads = list(range(min(w.H, args.cpu_heads)))
+        dt, th = oracle_sample(host, w, heads)
+        cpu = {"value": (th / w.H) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"heads 0..{len(heads) - 1} of {w.H}, batch 0, all {w.F} frames x {w.S} tokens "
+                         f"({dt:.1f} s); tokens counted x heads/H"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w), "global_batch": w.B * world, "tokens_per_step": w.tokens * world,
+                   "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step)" % (4 * w.tokens * w.H * w.d * 2 / 1e9),
+                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+        "roofline": roof,
+        "path_roofline": {"t_roof_us": pr["t_roof_us"], "t_step_us": step_us, "frac": pr["t_roof_us"] / step_us,
+                          "bound": pr["bound"], "algorithmic_bytes": pr["bytes"], "flops": pr["flops"],
+                          "peaks": peaks, "peak_source": peak_src},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": nl * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--rule", default=None)
+    ap.add_argument("--c", type=float, default=None)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=2)
+    ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = synth.WORKLOADS[args.workload]
+    if args.rule:
+        w = w.replace(rule=args.rule)
+    if args.c is not None:
+        w = w.replace(c=args.c)
+    if args.heads:
+        w = w.replace(H=args.heads)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -152,6 +152,28 @@ vdn_status vdn_branch_forward_debug(const vdn_shape* shape,
                                     void* out, void* stream,
                                     const vdn_debug_out* dbg);
 
+/* Number of kernels one vdn_branch_forward call launches for `shape` with the
+ * given implementation (VDN_IMPL_*): 5 on the tensor-core path (frame
+ * statistics, per-frame solve, scan, gather + bridge, read-out), 6 on the SIMT
+ * path (feature prep, statistics, solve, scan, gather, read-out); 0 if invalid. */
+int vdn_branch_launch_count(const vdn_shape* shape, int impl);
+
+/* vdn_branch_forward that also records caller-created CUDA events (cudaEvent_t
+ * handles, timing enabled) on `stream`: events[0] before the first kernel and
+ * events[i] right after kernel i, i = 1..vdn_branch_launch_count().  It adds
+ * no device work; n_events must be at least launch_count + 1.  For per-kernel
+ * timing by the caller (cudaEventElapsedTime between consecutive events). */
+vdn_status vdn_branch_forward_timed(const vdn_shape* shape,
+                                    const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha,
+                                    const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w,
+                                    const float* text_state,
+                                    int rule, float c, int chunk, int radius,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* out, void* stream,
+                                    void* const* events, int n_events);
+
 /* "Step 1" alone (page: NoPE features): q' = L2(SiLU(q)), k' = L2(SiLU(conv_k(k))),
  * v' = SiLU(conv_v(v)), all [B, F*S, H, d] in shape->dtype.  Outputs must not
  * overlap the inputs.  Needs no workspace. */

@@ -44,6 +44,8 @@ _SIGNATURES = {
     "vdn_branch_workspace_size_impl": (ctypes.c_size_t, [ctypes.POINTER(VdnShape), ctypes.c_int, ctypes.c_int]),
     "vdn_branch_forward": (ctypes.c_int, _FORWARD_ARGS),
     "vdn_branch_forward_debug": (ctypes.c_int, _FORWARD_ARGS + [ctypes.POINTER(VdnDebugOut)]),
+    "vdn_branch_launch_count": (ctypes.c_int, [ctypes.POINTER(VdnShape), ctypes.c_int]),
+    "vdn_branch_forward_timed": (ctypes.c_int, _FORWARD_ARGS + [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "vdn_feature_prep": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vdn_window_bounds": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),

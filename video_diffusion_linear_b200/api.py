@@ -77,6 +77,29 @@ def branch_forward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=No
     return out
 
 
+def launch_count(shape: VdnShape, impl="auto") -> int:
+    return _lib.load().vdn_branch_launch_count(ctypes.byref(shape), VDN_IMPL[impl])
+
+
+def branch_forward_timed(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *,
+                         F: int, events, rule="vdn_solve", c=1.0, chunk=5, radius=1, out=None, workspace=None,
+                         stream=None):
+    """vdn_branch_forward_timed: like branch_forward, recording `events` (torch.cuda.Event
+    objects with timing enabled, already recorded once so their handles exist) before the
+    first kernel and after each kernel."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(shape, rule, "auto", q.device)
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    st = _lib.load().vdn_branch_forward_timed(*_forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w,
+                                                             conv_v_w, text_state, rule, c, chunk, radius,
+                                                             workspace, out, stream), arr, len(events))
+    check(st, "vdn_branch_forward_timed")
+    return out
+
+
 DEBUG_FIELDS = ("A", "B", "N", "P", "Q", "W")
 
 

@@ -83,6 +83,16 @@ __host__ __device__ __forceinline__ RuleCoef rule_coef(int rule, float c) {
   return r;
 }
 
+// Block exponent of the scan states.  A rule whose per-frame operator has
+// eigenvalues beyond 1 in magnitude (sana_scaled with c^2 |A| > 2) makes the
+// state grow without bound; the scans keep X with true state 2^e X and rescale
+// X by 2^-64 (exactly) whenever an entry passes 2^64, so the state never leaves
+// the fp32 range.  The read-out's RMSNorm is scale-free up to eps, which is
+// scaled by 2^(-2e) accordingly.
+constexpr float kRenormAbove = 18446744073709551616.0f;     // 2^64
+constexpr float kRenormScale = 5.42101086242752217e-20f;    // 2^-64
+constexpr int kRenormExp = 64;
+
 // ---------------------------------------------------------------- device status word
 // Written only by bounded waits that gave up; read by vdn_workspace_status().
 constexpr uint32_t kStatusTimeout = 0x7100u;

@@ -37,6 +37,8 @@ struct WsPlan {
   size_t qf = 0, kf = 0, vf = 0;        // fp32 [B, N, H, d]
   size_t A = 0, Bm = 0, Nm = 0;         // fp32 [B, H, F, d, d]
   size_t P = 0, Q = 0, W = 0;           // fp32 [B, H, F, d, d]
+  // block exponents: a stored state X means 2^e X (int32 [B, H, F] each)
+  size_t pexp = 0, qexp = 0, wexp = 0;
   // tensor-core path
   size_t part = 0;                      // fp32 [slots][d][2d]: rows of [A | B^T] partial sums
   size_t nimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of N_f
@@ -53,10 +55,13 @@ cudaError_t launch_features_simt(const Args& a, float* qf, float* kf, float* vf)
 cudaError_t launch_stats_simt(const Args& a, const float* kf, const float* vf, float* A, float* Bm);
 cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nimg, const float* partials,
                          float* Bsum, float* Aout);
-cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q);
-cudaError_t launch_gather(const Args& a, const float* P, const float* Q, float* W, uint16_t* wimg);
-cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W);
-cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst);
+cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q, int* pexp,
+                             int* qexp);
+cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
+                          uint16_t* wimg, int* wexp);
+cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, const int* wexp);
+// dst = src * 2^expo[frame] (expo may be NULL)
+cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo = nullptr);
 
 // standalone step 1 (dtype in, dtype out)
 cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,
@@ -65,8 +70,8 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 
 // tensor-core path (bf16, d = 128)
 cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
-cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q,
-                           bool all_frames, uint32_t* status);
-cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, uint32_t* status);
+cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
+                           int* qexp, bool all_frames, uint32_t* status);
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, uint32_t* status);
 
 }  // namespace vdn

@@ -177,7 +177,7 @@ template <int D>
 __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm, const float* __restrict__ Nm,
                                                    const float* __restrict__ alpha, const float* __restrict__ text,
                                                    RuleCoef rc, float* __restrict__ P, float* __restrict__ Q,
-                                                   int H, int F) {
+                                                   int* __restrict__ pexp, int* __restrict__ qexp, int H, int F) {
   constexpr int R = D / 16;
   constexpr int LD = D + 1;
   extern __shared__ float sm[];
@@ -196,9 +196,11 @@ __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm,
       int i = ty + 16 * ia, k = tx + 16 * ib;
       s[ia][ib] = text ? kTextStateScale * text[((long long)h * D + i) * D + k] : 0.f;
     }
+  int e = 0;   // block exponent: the true state is 2^e s
   for (int step = 0; step < F; ++step) {
     int f = dir == 0 ? step : F - 1 - step;
     long long fi = bh * F + f;
+    const float cpre = ldexpf(rc.cpre, -e), cpost = ldexpf(rc.cpost, -e);
     const float* Bf = Bm + fi * D * D;
     const float* Nf = Nm + fi * D * D;
     const float* al = alpha + ((b * F + f) * H + h) * D;
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm,
 #pragma unroll
       for (int ib = 0; ib < R; ++ib) {
         int i = ty + 16 * ia, k = tx + 16 * ib;
-        X[i * LD + k] = fmaf(s[ia][ib], al[k], rc.cpre * Bf[i * D + k]);
+        X[i * LD + k] = fmaf(s[ia][ib], al[k], cpre * Bf[i * D + k]);
       }
     __syncthreads();
     float acc[R][R];
@@ -228,28 +230,40 @@ __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm,
         for (int ib = 0; ib < R; ++ib) acc[ia][ib] = fmaf(xr[ia], nr[ib], acc[ia][ib]);
     }
     float* dst = (dir == 0 ? P : Q) + fi * D * D;
+    float amax = 0.f;
 #pragma unroll
     for (int ia = 0; ia < R; ++ia)
 #pragma unroll
       for (int ib = 0; ib < R; ++ib) {
         int i = ty + 16 * ia, k = tx + 16 * ib;
-        s[ia][ib] = fmaf(rc.cpost, Bf[i * D + k], acc[ia][ib]);
+        s[ia][ib] = fmaf(cpost, Bf[i * D + k], acc[ia][ib]);
         dst[i * D + k] = s[ia][ib];
+        amax = fmaxf(amax, fabsf(s[ia][ib]));
       }
-    __syncthreads();
+    if (tid == 0) (dir == 0 ? pexp : qexp)[fi] = e;
+    if (__syncthreads_or(amax > kRenormAbove)) {
+#pragma unroll
+      for (int ia = 0; ia < R; ++ia)
+#pragma unroll
+        for (int ib = 0; ib < R; ++ib) s[ia][ib] *= kRenormScale;
+      e += kRenormExp;
+    }
   }
 }
 
-cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q) {
+cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q, int* pexp,
+                             int* qexp) {
   RuleCoef rc = rule_coef(a.rule, a.c);
   unsigned grid = (unsigned)(2LL * a.sh.B * a.sh.H);
   if (a.sh.d == 16) {
     size_t smem = 2 * 16 * 17 * sizeof(float);
-    k_scan_simt<16><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F);
+    k_scan_simt<16><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H,
+                                                    a.sh.F);
   } else {
     size_t smem = 2 * 128 * 129 * sizeof(float);
     cudaFuncSetAttribute(k_scan_simt<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_scan_simt<128><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F);
+    k_scan_simt<128><<<grid, 256, smem, a.stream>>>(Bm, Nm, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H,
+                                                     a.sh.F);
   }
   return cudaGetLastError();
 }
@@ -260,7 +274,8 @@ cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, fl
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_readout_simt(const float* __restrict__ qf, const T* __restrict__ gate,
                                                       const float* __restrict__ rms_w, const float* __restrict__ W,
-                                                      T* __restrict__ out, int H, int F, int S) {
+                                                      const int* __restrict__ wexp, T* __restrict__ out, int H, int F,
+                                                      int S) {
   constexpr int LD = D + 1;
   constexpr int PER = (D + 31) / 32;
   constexpr int TT = 64;
@@ -274,6 +289,7 @@ __global__ void __launch_bounds__(256) k_readout_simt(const float* __restrict__ 
   long long b = bh / H;
   long long N = (long long)F * S;
   const float* Wt = W + fi * D * D;
+  const float eps = ldexpf(kRmsEps, -2 * wexp[fi]);   // W_t is stored as 2^-e W_t
   for (int e = threadIdx.x; e < D * D; e += blockDim.x) Ws[(e / D) * LD + (e % D)] = Wt[e];
   __syncthreads();
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -297,7 +313,7 @@ __global__ void __launch_bounds__(256) k_readout_simt(const float* __restrict__ 
       ss += acc * acc;
     }
     ss = warp_sum(ss);
-    float inv = rsqrtf(ss / D + kRmsEps);
+    float inv = rsqrtf(ss / D + eps);
 #pragma unroll
     for (int r = 0; r < PER; ++r) {
       int i = lane + 32 * r;
@@ -307,14 +323,14 @@ __global__ void __launch_bounds__(256) k_readout_simt(const float* __restrict__ 
   }
 }
 
-cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W) {
+cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, const int* wexp) {
   dim3 grid((unsigned)a.NF(), (unsigned)((a.sh.S + 63) / 64));
   int d = a.sh.d;
   size_t smem = ((size_t)d * (d + 1) + 8 * d) * sizeof(float);
   auto go = [&](auto kern, auto tag) {
     using T = decltype(tag);
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, 256, smem, a.stream>>>(qf, (const T*)a.gate, a.rms_w, W, (T*)a.out, a.sh.H, a.sh.F, a.sh.S);
+    kern<<<grid, 256, smem, a.stream>>>(qf, (const T*)a.gate, a.rms_w, W, wexp, (T*)a.out, a.sh.H, a.sh.F, a.sh.S);
   };
   if (a.sh.dtype == VDN_DTYPE_BF16) {
     if (d == 16) go(k_readout_simt<__nv_bfloat16, 16>, __nv_bfloat16());
@@ -336,14 +352,16 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 }
 
 // ---------------------------------------------------------------- debug copies
-__global__ void k_copy(const float* __restrict__ s, float* __restrict__ d, long long n) {
+__global__ void k_copy(const float* __restrict__ s, float* __restrict__ d, const int* __restrict__ expo,
+                       long long per_frame, long long n) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-    d[i] = s[i];
+    d[i] = expo ? ldexpf(s[i], expo[i / per_frame]) : s[i];
 }
 
-cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst) {
-  long long n = a.NF() * a.sh.d * a.sh.d;
-  k_copy<<<1184, 256, 0, a.stream>>>(src, dst, n);
+cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo) {
+  long long per = (long long)a.sh.d * a.sh.d;
+  long long n = a.NF() * per;
+  k_copy<<<1184, 256, 0, a.stream>>>(src, dst, expo, per, n);
   return cudaGetLastError();
 }
 

@@ -171,11 +171,18 @@ cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nim
 // Query frame t with window [lo, hi]:
 //   W_t = P_{lo-1} diag(prod_{g=lo..t} alpha_g) + Q_{hi+1} diag(prod_{g=t..hi} alpha_g),
 // where P_{-1} = Q_F = 0.5 * text_state (zero without one).
+// States carry block exponents (true state = 2^e X); the two sides are brought
+// to the larger exponent, the sum is scaled by the power of two that puts its
+// largest entry in [0.5, 1), and W_t is stored as 2^-e_w W_t with e_w in wexp.
+// Power-of-two scaling is exact, so for states that never needed rescaling the
+// stored W_t differs from the plain sum only in its exponent; the read-out never
+// sees entries that could overflow its sum of squares.
 template <int D>
 __global__ void __launch_bounds__(256) k_gather(const float* __restrict__ P, const float* __restrict__ Q,
+                                                const int* __restrict__ pexp, const int* __restrict__ qexp,
                                                 const float* __restrict__ alpha, const float* __restrict__ text,
                                                 int H, int F, int chunk, int radius, float* __restrict__ W,
-                                                uint16_t* __restrict__ wimg) {
+                                                uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
   constexpr int LD = D + 1;
   extern __shared__ float sm[];
   float* dpre = sm;
@@ -199,11 +206,36 @@ __global__ void __launch_bounds__(256) k_gather(const float* __restrict__ P, con
   const float* pre = lo > 0 ? P + (bh * F + (lo - 1)) * D * D : nullptr;
   const float* suf = hi < F - 1 ? Q + (bh * F + (hi + 1)) * D * D : nullptr;
   const float* seed = text ? text + (long long)h * D * D : nullptr;
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-    int i = e / D, k = e % D;
+  const int ep = pre ? pexp[bh * F + (lo - 1)] : 0;
+  const int eq = suf ? qexp[bh * F + (hi + 1)] : 0;
+  const int ew = ep > eq ? ep : eq;
+  const float sp = ldexpf(1.f, ep - ew), sq = ldexpf(1.f, eq - ew);
+  constexpr int PER = D * D / 256;     // blockDim.x == 256
+  float wv[PER];
+  float amax = 0.f;
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    const int e = threadIdx.x + 256 * r, k = e % D;
     float pv = pre ? pre[e] : (seed ? kTextStateScale * seed[e] : 0.f);
     float sv = suf ? suf[e] : (seed ? kTextStateScale * seed[e] : 0.f);
-    float w = fmaf(pv, dpre[k], sv * dsuf[k]);
+    wv[r] = fmaf(pv * sp, dpre[k], sv * sq * dsuf[k]);
+    amax = fmaxf(amax, fabsf(wv[r]));
+  }
+  float* red = stage + (D == 128 && wimg ? D * LD : 0);   // 8 floats after the staging tile
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w8 = 1; w8 < 8; ++w8) amax = fmaxf(amax, red[w8]);
+  int ek = 0;
+  if (amax > 0.f) frexpf(amax, &ek);
+  if (threadIdx.x == 0) wexp[fi] = ew + ek;
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    const int e = threadIdx.x + 256 * r, i = e / D, k = e % D;
+    const float w = ldexpf(wv[r], -ek);
     if (W) W[fi * D * D + e] = w;
     if (D == 128 && wimg) stage[i * LD + k] = w;
   }
@@ -216,16 +248,17 @@ __global__ void __launch_bounds__(256) k_gather(const float* __restrict__ P, con
   }
 }
 
-cudaError_t launch_gather(const Args& a, const float* P, const float* Q, float* W, uint16_t* wimg) {
+cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
+                          uint16_t* wimg, int* wexp) {
   int d = a.sh.d;
-  size_t smem = (2 * (size_t)d + (wimg ? (size_t)d * (d + 1) : 0)) * sizeof(float);
+  size_t smem = (2 * (size_t)d + (wimg ? (size_t)d * (d + 1) : 0) + 8) * sizeof(float);
   if (d == 16) {
-    k_gather<16><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
-                                                            a.radius, W, nullptr);
+    k_gather<16><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
+                                                            a.chunk, a.radius, W, nullptr, wexp);
   } else {
     cudaFuncSetAttribute(k_gather<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_gather<128><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, a.alpha, a.text_state, a.sh.H, a.sh.F,
-                                                             a.chunk, a.radius, W, wimg);
+    k_gather<128><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H,
+                                                             a.sh.F, a.chunk, a.radius, W, wimg, wexp);
   }
   return cudaGetLastError();
 }

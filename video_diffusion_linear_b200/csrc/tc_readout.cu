@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
                                                            const __grid_constant__ CUtensorMap tmG,
                                                            const __grid_constant__ CUtensorMap tmO,
                                                            const uint16_t* __restrict__ wimg_g,
+                                                           const int* __restrict__ wexp,
                                                            const float* __restrict__ rms_w, int H, int F,
                                                            int ntile, long long T, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -207,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         tc::bulk_wait_read_all();                       // the previous tile's store has read its buffer
         tc::mbar_arrive(&sm.bar_g_empty[(it - 1) & 1]);
       }
+      const int ew = wexp[x / ntile];   // issued before the wait, used after it
       if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
       tc::tc_fence_after();
       float o[128];
@@ -224,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       float ss = 0.f;
 #pragma unroll
       for (int k = 0; k < 128; ++k) ss = fmaf(o[k], o[k], ss);
-      const float inv = rsqrtf(ss * (1.0f / 128.0f) + kRmsEps);
+      // W_t is stored as 2^-e W_t: the RMSNorm eps scales by 2^-2e
+      const float inv = rsqrtf(ss * (1.0f / 128.0f) + ldexpf(kRmsEps, -2 * ew));
       if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
       uint8_t* base = sm.gt[st];
 #pragma unroll
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
   }
 }
 
-cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, uint32_t* status) {
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, uint32_t* status) {
   const vdn_shape& sh = a.sh;
   CUtensorMap tq, tg, to;
   long long BF = (long long)sh.B * sh.F;
@@ -279,7 +282,8 @@ cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, uint32_t* sta
   size_t smem = sizeof(ReadSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_readout_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tq, tg, to, wimg, a.rms_w, sh.H, sh.F, ntile, T, status);
+  k_readout_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tq, tg, to, wimg, wexp, a.rms_w, sh.H, sh.F, ntile, T,
+                                                             status);
   return cudaGetLastError();
 }
 

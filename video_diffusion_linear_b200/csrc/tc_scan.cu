@@ -47,7 +47,8 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
                                                    const uint16_t* __restrict__ nimg_g,
                                                    const float* __restrict__ alpha,
                                                    const float* __restrict__ text, RuleCoef rc,
-                                                   float* __restrict__ P, float* __restrict__ Q, int H, int F,
+                                                   float* __restrict__ P, float* __restrict__ Q,
+                                                   int* __restrict__ pexp, int* __restrict__ qexp, int H, int F,
                                                    int chunk, int all_frames, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -108,9 +109,11 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
   const uint32_t n_hi = tc::smem_u32(sm.nimg), n_lo = n_hi + 32768;
   const uint8_t* bfb = reinterpret_cast<const uint8_t*>(sm.bf);
 
+  int ex = 0;   // block exponent: the true state is 2^ex s
   for (int step = 0; step < F; ++step) {
     const int f = frame_of(step);
     const long long fi = bh * F + f;
+    const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
     sm.alpha[m] = alpha[((b * F + f) * H + h) * 128 + m];
     __syncthreads();
     if (!tc::mbar_wait(&sm.bar_b, ph, abort_flag, status)) break;
@@ -124,8 +127,8 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
       uint32_t hw[4], lw[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        float x0 = fmaf(s[8 * c + e], sm.alpha[8 * c + e], rc.cpre * bv[e]);
-        float x1 = fmaf(s[8 * c + e + 1], sm.alpha[8 * c + e + 1], rc.cpre * bv[e + 1]);
+        float x0 = fmaf(s[8 * c + e], sm.alpha[8 * c + e], cpre * bv[e]);
+        float x1 = fmaf(s[8 * c + e + 1], sm.alpha[8 * c + e + 1], cpre * bv[e + 1]);
         float h0 = __bfloat162float(__float2bfloat16_rn(x0));
         float h1 = __bfloat162float(__float2bfloat16_rn(x1));
         hw[e / 2] = pack_bf16x2(h0, h1);
@@ -173,17 +176,26 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
         // with early_b the buffer already receives B_{f+1}: do not read it
         float4 bv = early_b ? make_float4(0.f, 0.f, 0.f, 0.f)
                             : *reinterpret_cast<const float4*>(bfb + bf_offset(m, 32 * j + e));
-        s[32 * j + e + 0] = fmaf(rc.cpost, bv.x, __uint_as_float(r[e + 0]));
-        s[32 * j + e + 1] = fmaf(rc.cpost, bv.y, __uint_as_float(r[e + 1]));
-        s[32 * j + e + 2] = fmaf(rc.cpost, bv.z, __uint_as_float(r[e + 2]));
-        s[32 * j + e + 3] = fmaf(rc.cpost, bv.w, __uint_as_float(r[e + 3]));
+        s[32 * j + e + 0] = fmaf(cpost, bv.x, __uint_as_float(r[e + 0]));
+        s[32 * j + e + 1] = fmaf(cpost, bv.y, __uint_as_float(r[e + 1]));
+        s[32 * j + e + 2] = fmaf(cpost, bv.z, __uint_as_float(r[e + 2]));
+        s[32 * j + e + 3] = fmaf(cpost, bv.w, __uint_as_float(r[e + 3]));
         if (store)
           *reinterpret_cast<float4*>(dst + 32 * j + e) =
               make_float4(s[32 * j + e], s[32 * j + e + 1], s[32 * j + e + 2], s[32 * j + e + 3]);
       }
     }
+    if (store && m == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 128; ++k) amax = fmaxf(amax, fabsf(s[k]));
     tc::tc_fence_before();
-    __syncthreads();   // accumulator and B_f reads done, alpha slot free
+    // accumulator and B_f reads done, alpha slot free; rescale if any entry passed 2^64
+    if (__syncthreads_or(amax > kRenormAbove)) {
+#pragma unroll
+      for (int k = 0; k < 128; ++k) s[k] *= kRenormScale;
+      ex += kRenormExp;
+    }
     if (m == 0 && !early_b && step + 1 < F) load_b(step + 1);
     ph ^= 1;
   }
@@ -198,8 +210,8 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
 
-cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q,
-                           bool all_frames, uint32_t* status) {
+cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
+                           int* qexp, bool all_frames, uint32_t* status) {
   CUtensorMap tmB;
   if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
   size_t smem = sizeof(ScanSmem) + 1024;
@@ -207,7 +219,7 @@ cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nim
   if (e != cudaSuccess) return e;
   RuleCoef rc = rule_coef(a.rule, a.c);
   k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), 128, smem, a.stream>>>(
-      tmB, nimg, a.alpha, a.text_state, rc, P, Q, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, status);
+      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, status);
   return cudaGetLastError();
 }
 

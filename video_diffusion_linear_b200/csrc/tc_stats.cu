@@ -38,6 +38,8 @@ constexpr int kThreads = 448;
 struct __align__(1024) StatsSmem {
   uint8_t raw[kRS][2][2][kRawHalf];    // [stage][k|v][channel half]
   uint8_t op[2][32768];                // [stage]: X (16 KB) | Y (16 KB), MN-major SW128
+  float taps[kRS][2][3][128];          // [stage][k|v][tap][channel] conv taps of the stage's head
+  float sqb[kRS][kStatsTokens];        // [stage][token] sqrt(beta), 0 past the frame end
   uint64_t raw_full[kRS], raw_empty[kRS];
   uint64_t op_full[2], op_empty[2];
   uint64_t acc_full[2], acc_empty[2];
@@ -108,21 +110,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   auto seg_last = [&](long long x) { return x + 1 == x1 || (x + 1) % nb == 0; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int it = 0;
-      for (long long x = x0; x < x1; ++x, ++it) {
-        int h, fb, s0;
-        decode(x, h, fb, s0);
-        const int rs = it % kRS;
-        const uint32_t ph = (it / kRS) & 1;
-        if (!tc::mbar_wait(&sm.raw_empty[rs], ph ^ 1, abort_flag, status)) break;
-        tc::mbar_arrive_expect_tx(&sm.raw_full[rs], kRawBytes);
+    // ------------------------------------------------------------ producer (whole warp)
+    // lane 0 issues the TMA copies; all lanes stage sqrt(beta) of the block's
+    // tokens and, when the stage's head changes, the conv taps of that head.
+    const long long N = (long long)F * S;
+    int slot_head[kRS];
+#pragma unroll
+    for (int r = 0; r < kRS; ++r) slot_head[r] = -1;
+    int it = 0;
+    for (long long x = x0; x < x1; ++x, ++it) {
+      int h, fb, s0;
+      decode(x, h, fb, s0);
+      const int rs = it % kRS;
+      const uint32_t ph = (it / kRS) & 1;
+      if (!tc::mbar_wait(&sm.raw_empty[rs], ph ^ 1, abort_flag, status)) break;
+      if (lane == 0) {
         for (int hf = 0; hf < 2; ++hf) {
           tc::tma_load_4d(&tmK, &sm.raw_full[rs], sm.raw[rs][0][hf], 64 * hf, h, s0 - 1, fb);
           tc::tma_load_4d(&tmV, &sm.raw_full[rs], sm.raw[rs][1][hf], 64 * hf, h, s0 - 1, fb);
         }
       }
+      const long long nbase = (long long)(fb / F) * N + (long long)(fb % F) * S;
+#pragma unroll
+      for (int u = 0; u < kStatsTokens / 32; ++u) {
+        const int t = lane + 32 * u, s = s0 + t;
+        sm.sqb[rs][t] = s < S ? sqrtf(beta[(nbase + s) * H + h]) : 0.f;
+      }
+      int cached = slot_head[0];
+#pragma unroll
+      for (int r = 0; r < kRS; ++r)
+        if (r == rs) cached = slot_head[r];
+      if (cached != h) {
+        for (int e = lane; e < 2 * 3 * 128; e += 32) {
+          const int ten = e / 384, tap = (e / 128) % 3, ch = e % 128;
+          const float* wg = ten == 0 ? wk_g : wv_g;
+          float val;
+          if (!wg) val = tap == 1 ? 1.f : 0.f;                       // identity
+          else if (K == 3) val = wg[((long long)h * 128 + ch) * 3 + tap];
+          else val = tap == 1 ? wg[(long long)h * 128 + ch] : 0.f;   // one tap: centre
+          sm.taps[rs][ten][tap][ch] = val;
+        }
+#pragma unroll
+        for (int r = 0; r < kRS; ++r)
+          if (r == rs) slot_head[r] = h;
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_expect_tx(&sm.raw_full[rs], kRawBytes);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -160,73 +193,61 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     const int w8 = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
     const int half = c >> 3, cc = c & 7;
     const int tok0 = 8 * w8 + 4 * tg;       // first of this thread's 4 tokens in the block
-    const long long N = (long long)F * S;
+    const float2 half2 = make_float2(0.5f, 0.5f);
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
-      int h, fb, s0;
-      decode(x, h, fb, s0);
       const int rs = it % kRS;
       const uint32_t rph = (it / kRS) & 1;
       const int os = it & 1;
       const uint32_t oph = (it >> 1) & 1;
-      // conv taps of this thread's 8 channels (identity when no weights)
-      float wk[3][8], wv[3][8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const long long wi = ((long long)h * 128 + 8 * c + e) * K;
-        wk[0][e] = (wk_g && K == 3) ? wk_g[wi] : 0.f;
-        wk[1][e] = wk_g ? wk_g[wi + (K == 3 ? 1 : 0)] : 1.f;
-        wk[2][e] = (wk_g && K == 3) ? wk_g[wi + 2] : 0.f;
-        wv[0][e] = (wv_g && K == 3) ? wv_g[wi] : 0.f;
-        wv[1][e] = wv_g ? wv_g[wi + (K == 3 ? 1 : 0)] : 1.f;
-        wv[2][e] = (wv_g && K == 3) ? wv_g[wi + 2] : 0.f;
-      }
+      if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
       float sb[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int s = s0 + tok0 + i;
-        const long long n = (long long)(fb / F) * N + (long long)(fb % F) * S + s;
-        sb[i] = s < S ? sqrtf(beta[n * H + h]) : 0.f;
-      }
-      if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
+      for (int i = 0; i < 4; ++i) sb[i] = sm.sqb[rs][tok0 + i];
 
-      // ---- k: conv, SiLU, L2 norm, * sqrt(beta)
-      float kx[4][8];
-      float ssq[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        float r[6][8];
-        const uint8_t* src = sm.raw[rs][0][half];
+      // conv (3 taps, packed pairs of channels), SiLU; k also sums its squares
+      auto conv_silu = [&](int ten, float2 (&outp)[4][4], float (&ss)[4]) {
+        float2 w[3][4];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const float4 a = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c]);
+          const float4 b = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c + 4]);
+          w[j][0] = make_float2(a.x, a.y); w[j][1] = make_float2(a.z, a.w);
+          w[j][2] = make_float2(b.x, b.y); w[j][3] = make_float2(b.z, b.w);
+        }
+        float2 r[6][4];
+        const uint8_t* src = sm.raw[rs][ten][half];
 #pragma unroll
         for (int rr = 0; rr < 6; ++rr) {
           const int row = tok0 + rr;
-          unpack8(*reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4)), r[rr]);
+          const uint4 q = *reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4));
+          r[rr][0] = make_float2(bf16lo(q.x), bf16hi(q.x));
+          r[rr][1] = make_float2(bf16lo(q.y), bf16hi(q.y));
+          r[rr][2] = make_float2(bf16lo(q.z), bf16hi(q.z));
+          r[rr][3] = make_float2(bf16lo(q.w), bf16hi(q.w));
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i) {
+          float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float a = fmaf(wk[0][e], r[i][e], fmaf(wk[1][e], r[i + 1][e], wk[2][e] * r[i + 2][e]));
-            a = silu_fast(a);
-            kx[i][e] = a;
-            ssq[i] = fmaf(a, a, ssq[i]);
+          for (int p = 0; p < 4; ++p) {
+            float2 a = __fmul2_rn(w[2][p], r[i + 2][p]);
+            a = __ffma2_rn(w[1][p], r[i + 1][p], a);
+            a = __ffma2_rn(w[0][p], r[i][p], a);
+            const float2 hx = __fmul2_rn(a, half2);
+            const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
+            const float2 y = __ffma2_rn(hx, th, hx);         // x sigmoid(x) = h + h tanh(h), h = x/2
+            outp[i][p] = y;
+            acc = __ffma2_rn(y, y, acc);
           }
-      }
-      // ---- v: conv, SiLU, * sqrt(beta)
-      float vx[4][8];
-      {
-        float r[6][8];
-        const uint8_t* src = sm.raw[rs][1][half];
-#pragma unroll
-        for (int rr = 0; rr < 6; ++rr) {
-          const int row = tok0 + rr;
-          unpack8(*reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4)), r[rr]);
+          ss[i] = acc.x + acc.y;
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            vx[i][e] = sb[i] * silu_fast(fmaf(wv[0][e], r[i][e], fmaf(wv[1][e], r[i + 1][e], wv[2][e] * r[i + 2][e])));
-      }
+      };
+
+      float2 kx[4][4], vx[4][4];
+      float ssq[4], unused[4];
+      conv_silu(0, kx, ssq);
+      conv_silu(1, vx, unused);
       tc::mbar_arrive(&sm.raw_empty[rs]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -239,17 +260,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = tok0 + i;
-        uint4 wx, wy;
-        wx.x = pack_bf16x2(kx[i][0] * ssq[i], kx[i][1] * ssq[i]);
-        wx.y = pack_bf16x2(kx[i][2] * ssq[i], kx[i][3] * ssq[i]);
-        wx.z = pack_bf16x2(kx[i][4] * ssq[i], kx[i][5] * ssq[i]);
-        wx.w = pack_bf16x2(kx[i][6] * ssq[i], kx[i][7] * ssq[i]);
-        wy.x = pack_bf16x2(vx[i][0], vx[i][1]);
-        wy.y = pack_bf16x2(vx[i][2], vx[i][3]);
-        wy.z = pack_bf16x2(vx[i][4], vx[i][5]);
-        wy.w = pack_bf16x2(vx[i][6], vx[i][7]);
-        *reinterpret_cast<uint4*>(dst + op_chunk(c, t)) = wx;
-        *reinterpret_cast<uint4*>(dst + 16384 + op_chunk(c, t)) = wy;
+        const float2 sk = make_float2(ssq[i], ssq[i]), sv = make_float2(sb[i], sb[i]);
+        uint32_t wxv[4], wyv[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 a = __fmul2_rn(kx[i][p], sk);
+          const float2 b = __fmul2_rn(vx[i][p], sv);
+          wxv[p] = pack_bf16x2(a.x, a.y);
+          wyv[p] = pack_bf16x2(b.x, b.y);
+        }
+        *reinterpret_cast<uint4*>(dst + op_chunk(c, t)) = make_uint4(wxv[0], wxv[1], wxv[2], wxv[3]);
+        *reinterpret_cast<uint4*>(dst + 16384 + op_chunk(c, t)) = make_uint4(wyv[0], wyv[1], wyv[2], wyv[3]);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&sm.op_full[os]);

@@ -36,6 +36,9 @@ WsPlan plan_workspace(const vdn_shape& sh, int /*rule*/, bool tc) {
   const size_t NF = (size_t)sh.B * sh.H * sh.F;
   const size_t frame_mats = NF * d * d * sizeof(float);
   p.status = take(256);
+  p.pexp = take(NF * sizeof(int));
+  p.qexp = take(NF * sizeof(int));
+  p.wexp = take(NF * sizeof(int));
   if (!tc) {
     const size_t feat = (size_t)sh.B * sh.F * sh.S * sh.H * d * sizeof(float);
     p.qf = take(feat);
@@ -143,29 +146,42 @@ T* at(void* ws, size_t off) {
     if (e_ != cudaSuccess) return VDN_ERR_CUDA; \
   } while (0)
 
-vdn_status run_forward(const Args& a, void* ws, int impl) {
+vdn_status run_forward(const Args& a, void* ws, int impl, void* const* events = nullptr) {
   const bool tc = use_tc(a.sh, impl);
+  int ev = 0;
+  auto mark = [&]() -> cudaError_t {
+    if (!events) return cudaSuccess;
+    return cudaEventRecord((cudaEvent_t)events[ev++], a.stream);
+  };
   WsPlan p = plan_workspace(a.sh, a.rule, tc);
   const vdn_debug_out* dbg = a.dbg;
   uint32_t* status = at<uint32_t>(ws, p.status);
   VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), a.stream));
+  VDN_LAUNCH(mark());
   if (!tc) {
     float *qf = at<float>(ws, p.qf), *kf = at<float>(ws, p.kf), *vf = at<float>(ws, p.vf);
     float *A = at<float>(ws, p.A), *Bm = at<float>(ws, p.Bm), *Nm = at<float>(ws, p.Nm);
     float *P = at<float>(ws, p.P), *Q = at<float>(ws, p.Q), *W = at<float>(ws, p.W);
+    int *pexp = at<int>(ws, p.pexp), *qexp = at<int>(ws, p.qexp), *wexp = at<int>(ws, p.wexp);
     VDN_LAUNCH(launch_features_simt(a, qf, kf, vf));
+    VDN_LAUNCH(mark());
     VDN_LAUNCH(launch_stats_simt(a, kf, vf, A, Bm));
+    VDN_LAUNCH(mark());
     VDN_LAUNCH(launch_solve(a, A, Nm, nullptr, nullptr, nullptr, nullptr));
-    VDN_LAUNCH(launch_scan_simt(a, Bm, Nm, P, Q));
-    VDN_LAUNCH(launch_gather(a, P, Q, W, nullptr));
-    VDN_LAUNCH(launch_readout_simt(a, qf, W));
+    VDN_LAUNCH(mark());
+    VDN_LAUNCH(launch_scan_simt(a, Bm, Nm, P, Q, pexp, qexp));
+    VDN_LAUNCH(mark());
+    VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, W, nullptr, wexp));
+    VDN_LAUNCH(mark());
+    VDN_LAUNCH(launch_readout_simt(a, qf, W, wexp));
+    VDN_LAUNCH(mark());
     if (dbg) {
       if (dbg->A) VDN_LAUNCH(launch_copy_frames(a, A, dbg->A));
       if (dbg->B) VDN_LAUNCH(launch_copy_frames(a, Bm, dbg->B));
       if (dbg->N) VDN_LAUNCH(launch_copy_frames(a, Nm, dbg->N));
-      if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P));
-      if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q));
-      if (dbg->W) VDN_LAUNCH(launch_copy_frames(a, W, dbg->W));
+      if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P, pexp));
+      if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q, qexp));
+      if (dbg->W) VDN_LAUNCH(launch_copy_frames(a, W, dbg->W, wexp));
     }
     return VDN_OK;
   }
@@ -174,16 +190,24 @@ vdn_status run_forward(const Args& a, void* ws, int impl) {
   uint16_t* nimg = at<uint16_t>(ws, p.nimg);
   float *P = at<float>(ws, p.P), *Q = at<float>(ws, p.Q);
   uint16_t* wimg = at<uint16_t>(ws, p.wimg);
+  int *pexp = at<int>(ws, p.pexp), *qexp = at<int>(ws, p.qexp), *wexp = at<int>(ws, p.wexp);
   bool all_frames = dbg && (dbg->P || dbg->Q);
+  // the debug export of W: the gather writes 2^-wexp W_t into dbg->W, rescaled in place below
   VDN_LAUNCH(launch_stats_tc(a, part, status));
+  VDN_LAUNCH(mark());
   VDN_LAUNCH(launch_solve(a, nullptr, dbg ? dbg->N : nullptr, nimg, part, Bsum, dbg ? dbg->A : nullptr));
-  VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, P, Q, all_frames, status));
-  VDN_LAUNCH(launch_gather(a, P, Q, dbg ? dbg->W : nullptr, wimg));
-  VDN_LAUNCH(launch_readout_tc(a, wimg, status));
+  VDN_LAUNCH(mark());
+  VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, P, Q, pexp, qexp, all_frames, status));
+  VDN_LAUNCH(mark());
+  VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, dbg ? dbg->W : nullptr, wimg, wexp));
+  VDN_LAUNCH(mark());
+  VDN_LAUNCH(launch_readout_tc(a, wimg, wexp, status));
+  VDN_LAUNCH(mark());
   if (dbg) {
     if (dbg->B) VDN_LAUNCH(launch_copy_frames(a, Bsum, dbg->B));
-    if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P));
-    if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q));
+    if (dbg->P) VDN_LAUNCH(launch_copy_frames(a, P, dbg->P, pexp));
+    if (dbg->Q) VDN_LAUNCH(launch_copy_frames(a, Q, dbg->Q, qexp));
+    if (dbg->W) VDN_LAUNCH(launch_copy_frames(a, dbg->W, dbg->W, wexp));
   }
   return VDN_OK;
 }
@@ -192,7 +216,7 @@ vdn_status forward_common(const vdn_shape* shape, const void* q, const void* k, 
                           const float* alpha, const void* gate, const float* rms_w, const float* conv_k_w,
                           const float* conv_v_w, const float* text_state, int rule, float c, int chunk, int radius,
                           void* workspace, size_t workspace_bytes, void* out, void* stream,
-                          const vdn_debug_out* dbg) {
+                          const vdn_debug_out* dbg, void* const* events = nullptr, int n_events = 0) {
   int impl = dbg ? dbg->impl : VDN_IMPL_AUTO;
   vdn_status s = validate(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
                           radius, workspace, workspace_bytes, out, impl);
@@ -212,7 +236,13 @@ vdn_status forward_common(const vdn_shape* shape, const void* q, const void* k, 
   a.out = out;
   a.stream = (cudaStream_t)stream;
   a.dbg = dbg;
-  return run_forward(a, workspace, impl);
+  if (events) {
+    const int need = (use_tc(a.sh, impl) ? 5 : 6) + 1;
+    if (n_events < need) return VDN_ERR_INVALID_ARG;
+    for (int i = 0; i < need; ++i)
+      if (!events[i]) return VDN_ERR_INVALID_ARG;
+  }
+  return run_forward(a, workspace, impl, events);
 }
 
 }  // namespace
@@ -247,6 +277,23 @@ vdn_status vdn_branch_forward_debug(const vdn_shape* shape, const void* q, const
                                     size_t workspace_bytes, void* out, void* stream, const vdn_debug_out* dbg) {
   return forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
                         radius, workspace, workspace_bytes, out, stream, dbg);
+}
+
+int vdn_branch_launch_count(const vdn_shape* shape, int impl) {
+  if (check_shape(shape) != VDN_OK || impl < VDN_IMPL_AUTO || impl > VDN_IMPL_TC) return 0;
+  if (impl == VDN_IMPL_TC && !(shape->dtype == VDN_DTYPE_BF16 && shape->d == 128)) return 0;
+  return use_tc(*shape, impl) ? 5 : 6;
+}
+
+vdn_status vdn_branch_forward_timed(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w, const float* text_state,
+                                    int rule, float c, int chunk, int radius, void* workspace,
+                                    size_t workspace_bytes, void* out, void* stream, void* const* events,
+                                    int n_events) {
+  if (!events) return VDN_ERR_INVALID_ARG;
+  return forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                        radius, workspace, workspace_bytes, out, stream, nullptr, events, n_events);
 }
 
 vdn_status vdn_feature_prep(const vdn_shape* shape, const void* q, const void* k, const void* v,
