@@ -65,7 +65,22 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
       for (int ia = 0; ia < R; ++ia)
 #pragma unroll
         for (int ib = 0; ib < R; ++ib) a[ia][ib] += p[(ty + 16 * ia) * (2 * D) + tx + 16 * ib];
-      for (int e = tid; e < D * D; e += 256) stage[(e / D) * LD + (e % D)] += p[(e / D) * (2 * D) + D + (e % D)];
+      // B^T half of the slot: float4 loads, all issued before use
+      constexpr int NV4 = D * D / 4, NV = (NV4 + 255) / 256;
+      float4 bv[NV];
+#pragma unroll
+      for (int r = 0; r < NV; ++r) {
+        const int e4 = tid + 256 * r, row = e4 / (D / 4), c4 = e4 % (D / 4);
+        if (e4 < NV4) bv[r] = *reinterpret_cast<const float4*>(p + row * (2 * D) + D + 4 * c4);
+      }
+#pragma unroll
+      for (int r = 0; r < NV; ++r) {
+        const int e4 = tid + 256 * r, row = e4 / (D / 4), c4 = e4 % (D / 4);
+        if (e4 < NV4) {
+          float* st = stage + row * LD + 4 * c4;
+          st[0] += bv[r].x; st[1] += bv[r].y; st[2] += bv[r].z; st[3] += bv[r].w;
+        }
+      }
     }
     __syncthreads();
     float* Bf = Bsum + fi * D * D;   // B[i][j] = (B^T)[j][i]
@@ -248,18 +263,119 @@ __global__ void __launch_bounds__(256) k_gather(const float* __restrict__ P, con
   }
 }
 
+// d = 128: 512 threads, four per row of W_t (32 columns each).  The state rows
+// are loaded first (float4), the decay vectors meanwhile by one thread per
+// channel, then each thread writes its part of the bf16 hi/lo operand image
+// directly (four 16-byte chunks per part, 128-byte swizzle).
+__global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, const float* __restrict__ Q,
+                                                   const int* __restrict__ pexp, const int* __restrict__ qexp,
+                                                   const float* __restrict__ alpha, const float* __restrict__ text,
+                                                   int H, int F, int chunk, int radius, float* __restrict__ W,
+                                                   uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
+  constexpr int D = 128;
+  __shared__ float dpre[D], dsuf[D], red[16];
+  const int tid = threadIdx.x, n = tid >> 2, k0 = (tid & 3) * 32;
+  const long long fi = blockIdx.x;
+  const int t = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  int lo, hi;
+  window_bounds(t, F, chunk, radius, lo, hi);
+  const float* pre = lo > 0 ? P + (bh * F + (lo - 1)) * D * D : nullptr;
+  const float* suf = hi < F - 1 ? Q + (bh * F + (hi + 1)) * D * D : nullptr;
+  const float* seed = text ? text + (long long)h * D * D : nullptr;
+  float4 pv[8], sv[8];
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int off = n * D + k0 + 4 * j;
+    pv[j] = pre ? *reinterpret_cast<const float4*>(pre + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
+    sv[j] = suf ? *reinterpret_cast<const float4*>(suf + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
+  }
+  if (tid < D) {
+    float dp = 1.f, ds = 1.f;
+    const float* al = alpha + (b * F * H + h) * D + tid;   // alpha[b][g][h][c] = al[g * H * D]
+    for (int g0 = lo; g0 <= hi; g0 += 8) {
+      float av[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) av[u] = (g0 + u <= hi) ? al[(long long)(g0 + u) * H * D] : 1.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int g = g0 + u;
+        if (g <= t) dp *= av[u];
+        if (g >= t) ds *= av[u];
+      }
+    }
+    dpre[tid] = dp;
+    dsuf[tid] = ds;
+  }
+  const int ep = pre ? pexp[bh * F + (lo - 1)] : 0;
+  const int eq = suf ? qexp[bh * F + (hi + 1)] : 0;
+  const int ew = ep > eq ? ep : eq;
+  const float sp = (pre ? 1.f : (seed ? kTextStateScale : 0.f)) * ldexpf(1.f, ep - ew);
+  const float sq = (suf ? 1.f : (seed ? kTextStateScale : 0.f)) * ldexpf(1.f, eq - ew);
+  __syncthreads();
+  float w[32];
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int k = k0 + 4 * j;
+    w[4 * j + 0] = fmaf(pv[j].x * sp, dpre[k + 0], sv[j].x * sq * dsuf[k + 0]);
+    w[4 * j + 1] = fmaf(pv[j].y * sp, dpre[k + 1], sv[j].y * sq * dsuf[k + 1]);
+    w[4 * j + 2] = fmaf(pv[j].z * sp, dpre[k + 2], sv[j].z * sq * dsuf[k + 2]);
+    w[4 * j + 3] = fmaf(pv[j].w * sp, dpre[k + 3], sv[j].w * sq * dsuf[k + 3]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(w[4 * j + u]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int u = 1; u < 16; ++u) amax = fmaxf(amax, red[u]);
+  int ek = 0;
+  if (amax > 0.f) frexpf(amax, &ek);
+  if (tid == 0) wexp[fi] = ew + ek;
+#pragma unroll
+  for (int u = 0; u < 32; ++u) w[u] = ldexpf(w[u], -ek);
+  if (W) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(W + fi * D * D + n * D + k0 + 4 * j) =
+          make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+  if (wimg) {
+    uint8_t* img = reinterpret_cast<uint8_t*>(wimg + fi * (kImgBytes / 2));
+#pragma unroll
+    for (int cch = 0; cch < 4; ++cch) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        __nv_bfloat16 h0, l0, h1, l1;
+        split_bf16(w[8 * cch + e], h0, l0);
+        split_bf16(w[8 * cch + e + 1], h1, l1);
+        hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+      }
+      const uint32_t off = img_offset(0, n, k0 + 8 * cch);
+      *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  }
+}
+
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
                           uint16_t* wimg, int* wexp) {
-  int d = a.sh.d;
-  size_t smem = (2 * (size_t)d + (wimg ? (size_t)d * (d + 1) : 0) + 8) * sizeof(float);
-  if (d == 16) {
-    k_gather<16><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
-                                                            a.chunk, a.radius, W, nullptr, wexp);
-  } else {
-    cudaFuncSetAttribute(k_gather<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_gather<128><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H,
-                                                             a.sh.F, a.chunk, a.radius, W, wimg, wexp);
+  if (a.sh.d == 128) {
+    k_gather128<<<(unsigned)a.NF(), 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
+                                                        a.chunk, a.radius, W, wimg, wexp);
+    return cudaGetLastError();
   }
+  size_t smem = (2 * 16 + 8) * sizeof(float);
+  k_gather<16><<<(unsigned)a.NF(), 256, smem, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
+                                                          a.chunk, a.radius, W, nullptr, wexp);
   return cudaGetLastError();
 }
 

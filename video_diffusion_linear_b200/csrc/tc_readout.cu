@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ q' = L2(SiLU(q)), in place
+    // two passes over the row (sum of squares, then scale and store): SiLU is
+    // evaluated twice, which keeps the loop rolled and the row out of registers
     const int r = tid - 64;
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
@@ -167,36 +169,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       const uint32_t ph = (it >> 1) & 1;
       if (!tc::mbar_wait(&sm.bar_q_full[st], ph, abort_flag, status)) break;
       uint8_t* base = sm.qt[st];
-      float v[128];
       float ss = 0.f;
-#pragma unroll
+#pragma unroll 2
       for (int c = 0; c < 16; ++c) {
-        uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
-        uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float a0 = silu_fast(bf16lo(ws[e])), a1 = silu_fast(bf16hi(ws[e]));
-          v[8 * c + 2 * e] = a0;
-          v[8 * c + 2 * e + 1] = a1;
-          ss = fmaf(a0, a0, ss);
-          ss = fmaf(a1, a1, ss);
+          const float a0 = silu_fast(bf16lo(ws[e])), a1 = silu_fast(bf16hi(ws[e]));
+          ss = fmaf(a0, a0, fmaf(a1, a1, ss));
         }
       }
       const float inv = rsqrtf(ss + kL2Eps);
-#pragma unroll
+#pragma unroll 2
       for (int c = 0; c < 16; ++c) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * c + 0] * inv, v[8 * c + 1] * inv);
-        w.y = pack_bf16x2(v[8 * c + 2] * inv, v[8 * c + 3] * inv);
-        w.z = pack_bf16x2(v[8 * c + 4] * inv, v[8 * c + 5] * inv);
-        w.w = pack_bf16x2(v[8 * c + 6] * inv, v[8 * c + 7] * inv);
-        *reinterpret_cast<uint4*>(base + row_chunk(r, c)) = w;
+        uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o4[e] = pack_bf16x2(silu_fast(bf16lo(ws[e])) * inv, silu_fast(bf16hi(ws[e])) * inv);
+        *reinterpret_cast<uint4*>(base + row_chunk(r, c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&sm.bar_q_ready[st]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // pass 1 reads the accumulator row from TMEM for the sum of squares, pass 2
+    // reads it again to scale, gate and store (TMEM reads are cheap, registers not)
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const bool leader = tid == 192;
@@ -211,39 +212,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       const int ew = wexp[x / ntile];   // issued before the wait, used after it
       if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
       tc::tc_fence_after();
-      float o[128];
       const uint32_t taddr = tmem + st * 128 + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll
+      float ss = 0.f;
+#pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         uint32_t rr[32];
         tc::tmem_ld32(taddr + 32 * j, rr);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[32 * j + e] = __uint_as_float(rr[e]);
+        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(rr[e]), __uint_as_float(rr[e]), ss);
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&sm.bar_acc_empty[st]);
-      float ss = 0.f;
-#pragma unroll
-      for (int k = 0; k < 128; ++k) ss = fmaf(o[k], o[k], ss);
       // W_t is stored as 2^-e W_t: the RMSNorm eps scales by 2^-2e
       const float inv = rsqrtf(ss * (1.0f / 128.0f) + ldexpf(kRmsEps, -2 * ew));
       if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
       uint8_t* base = sm.gt[st];
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        uint32_t rr[32];
+        tc::tmem_ld32(taddr + 32 * j, rr);
+        tc::tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 g = *reinterpret_cast<const uint4*>(base + row_chunk(m, c));
-        uint32_t gs[4] = {g.x, g.y, g.z, g.w};
-        uint32_t outw[4];
+        for (int cq = 0; cq < 4; ++cq) {
+          const int c = 4 * j + cq;
+          const uint4 g = *reinterpret_cast<const uint4*>(base + row_chunk(m, c));
+          const uint32_t gs[4] = {g.x, g.y, g.z, g.w};
+          uint32_t outw[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int k = 8 * c + 2 * e;
-          float y0 = o[k] * inv * sm.rms_w[k] * bf16lo(gs[e]);
-          float y1 = o[k + 1] * inv * sm.rms_w[k + 1] * bf16hi(gs[e]);
-          outw[e] = pack_bf16x2(y0, y1);
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * c + 2 * e;
+            const float y0 = __uint_as_float(rr[8 * cq + 2 * e]) * inv * sm.rms_w[k] * bf16lo(gs[e]);
+            const float y1 = __uint_as_float(rr[8 * cq + 2 * e + 1]) * inv * sm.rms_w[k + 1] * bf16hi(gs[e]);
+            outw[e] = pack_bf16x2(y0, y1);
+          }
+          *reinterpret_cast<uint4*>(base + row_chunk(m, c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
-        *reinterpret_cast<uint4*>(base + row_chunk(m, c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
       }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&sm.bar_acc_empty[st]);
       tc::fence_proxy_async_smem();
       tc::named_bar(1, 128);
       if (leader) {

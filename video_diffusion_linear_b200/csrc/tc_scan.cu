@@ -110,11 +110,13 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
   const uint8_t* bfb = reinterpret_cast<const uint8_t*>(sm.bf);
 
   int ex = 0;   // block exponent: the true state is 2^ex s
+  float a_next = alpha[((b * F + frame_of(0)) * H + h) * 128 + m];
   for (int step = 0; step < F; ++step) {
     const int f = frame_of(step);
     const long long fi = bh * F + f;
     const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
-    sm.alpha[m] = alpha[((b * F + f) * H + h) * 128 + m];
+    sm.alpha[m] = a_next;
+    if (step + 1 < F) a_next = alpha[((b * F + frame_of(step + 1)) * H + h) * 128 + m];   // used next step
     __syncthreads();
     if (!tc::mbar_wait(&sm.bar_b, ph, abort_flag, status)) break;
 

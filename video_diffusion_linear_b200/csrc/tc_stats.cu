@@ -55,13 +55,6 @@ __device__ __forceinline__ uint32_t op_chunk(int c, int t) {
   return (c >> 3) * 8192 + (t >> 3) * 1024 + (t & 7) * 128 + ((((c & 7) ^ (t & 7))) << 4);
 }
 
-__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
-  f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
-  f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant__ CUtensorMap tmK,
@@ -117,6 +110,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     int slot_head[kRS];
 #pragma unroll
     for (int r = 0; r < kRS; ++r) slot_head[r] = -1;
+    // beta of the next block is loaded one iteration ahead, so its latency
+    // overlaps the wait for a free stage instead of delaying the next TMA issue
+    constexpr int BU = kStatsTokens / 32;
+    float bnext[BU];
+    auto load_beta = [&](long long x) {
+      int h, fb, s0;
+      decode(x, h, fb, s0);
+      const long long nbase = (long long)(fb / F) * N + (long long)(fb % F) * S;
+#pragma unroll
+      for (int u = 0; u < BU; ++u) {
+        const int s = s0 + lane + 32 * u;
+        bnext[u] = s < S ? beta[(nbase + s) * H + h] : 0.f;
+      }
+    };
+    if (x0 < x1) load_beta(x0);
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
       int h, fb, s0;
@@ -130,12 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           tc::tma_load_4d(&tmV, &sm.raw_full[rs], sm.raw[rs][1][hf], 64 * hf, h, s0 - 1, fb);
         }
       }
-      const long long nbase = (long long)(fb / F) * N + (long long)(fb % F) * S;
 #pragma unroll
-      for (int u = 0; u < kStatsTokens / 32; ++u) {
-        const int t = lane + 32 * u, s = s0 + t;
-        sm.sqb[rs][t] = s < S ? sqrtf(beta[(nbase + s) * H + h]) : 0.f;
-      }
+      for (int u = 0; u < BU; ++u) sm.sqb[rs][lane + 32 * u] = sqrtf(bnext[u]);
+      if (x + 1 < x1) load_beta(x + 1);
       int cached = slot_head[0];
 #pragma unroll
       for (int r = 0; r < kRS; ++r)
