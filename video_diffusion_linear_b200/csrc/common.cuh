@@ -49,6 +49,23 @@ __device__ __forceinline__ float silu_fast(float x) {
   return fmaf(hx, tanh_approx(hx), hx);
 }
 
+// tanh of a pair of floats.  Default: two hardware tanh.approx.f32 ops.
+// With VDN_TANH_F16X2 defined, one packed tanh.approx.f16x2 op (f16 keeps an
+// 11-bit mantissa, below the bf16 rounding of the tensor-core operands).
+__device__ __forceinline__ float2 tanh2(float2 h) {
+#ifdef VDN_TANH_F16X2
+  uint32_t hp, tp;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hp) : "f"(h.y), "f"(h.x));
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(tp) : "r"(hp));
+  float t0, t1;
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(t0), "=f"(t1) : "r"(tp));
+  return make_float2(t0, t1);
+#else
+  return make_float2(tanh_approx(h.x), tanh_approx(h.y));
+#endif
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

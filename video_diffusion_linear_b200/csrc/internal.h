@@ -28,7 +28,7 @@ struct Args {
 // fixed count (the SM count of a B200) keeps the workspace a pure function of
 // the shape; correctness does not depend on it.
 constexpr int kStatsGrid = 148;
-constexpr int kStatsTokens = 64;     // tokens per statistics block
+constexpr int kStatsTokens = 96;     // tokens per statistics block
 
 // Byte offsets of the workspace regions (each 256-byte aligned).
 struct WsPlan {

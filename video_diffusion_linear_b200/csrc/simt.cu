@@ -196,11 +196,11 @@ __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm,
       int i = ty + 16 * ia, k = tx + 16 * ib;
       s[ia][ib] = text ? kTextStateScale * text[((long long)h * D + i) * D + k] : 0.f;
     }
-  int e = 0;   // block exponent: the true state is 2^e s
+  int ex = 0;   // block exponent: the true state is 2^ex s
   for (int step = 0; step < F; ++step) {
     int f = dir == 0 ? step : F - 1 - step;
     long long fi = bh * F + f;
-    const float cpre = ldexpf(rc.cpre, -e), cpost = ldexpf(rc.cpost, -e);
+    const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
     const float* Bf = Bm + fi * D * D;
     const float* Nf = Nm + fi * D * D;
     const float* al = alpha + ((b * F + f) * H + h) * D;
@@ -240,13 +240,13 @@ __global__ void __launch_bounds__(256) k_scan_simt(const float* __restrict__ Bm,
         dst[i * D + k] = s[ia][ib];
         amax = fmaxf(amax, fabsf(s[ia][ib]));
       }
-    if (tid == 0) (dir == 0 ? pexp : qexp)[fi] = e;
+    if (tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
     if (__syncthreads_or(amax > kRenormAbove)) {
 #pragma unroll
       for (int ia = 0; ia < R; ++ia)
 #pragma unroll
         for (int ib = 0; ib < R; ++ib) s[ia][ib] *= kRenormScale;
-      e += kRenormExp;
+      ex += kRenormExp;
     }
   }
 }

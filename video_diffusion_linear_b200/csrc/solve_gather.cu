@@ -163,8 +163,183 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
   }
 }
 
+// d = 128 solve.  Thread (ty, tx) owns the 8x8 block rows 8 ty.., columns 8 tx..
+// (contiguous, so pivot row and column segments are two 16-byte loads), the
+// elimination update runs on packed fp32 pairs, and the pivot reciprocal is
+// the hardware approximation refined by one Newton step (relative error near
+// 2^-23, the same as a correctly rounded division up to one unit).
+__global__ void __launch_bounds__(256, 2) k_solve128(const float* __restrict__ part, long long Tblocks, int nb, int G,
+                                                     RuleCoef rc, float* __restrict__ Nm, uint16_t* __restrict__ nimg,
+                                                     float* __restrict__ Bsum, float* __restrict__ Aout, int H, int F) {
+  constexpr int D = 128, LD = D + 4;   // +4 keeps rows 16-byte aligned
+  extern __shared__ float sm[];
+  float* stage = sm;                   // [D][LD]
+  float* colv = sm + D * LD;           // [2][D]
+  float* rowv = colv + 2 * D;          // [2][D]
+  const long long fi = blockIdx.x;
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int r0 = 8 * ty, c0 = 8 * tx;
+  float2 a[8][4];                      // a[i][p] = (A[r0+i][c0+2p], A[r0+i][c0+2p+1])
+
+  // sum the [A | B^T] partial rows of this frame's statistics slots
+  {
+    const long long pf = ((long long)b * F + f) * H + h;
+    const long long x0 = pf * nb, x1 = x0 + nb - 1;
+    const int i0 = sk_owner(x0, Tblocks, G), i1 = sk_owner(x1, Tblocks, G);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) a[i][p] = make_float2(0.f, 0.f);
+    for (int e = tid; e < D * D / 4; e += 256) *reinterpret_cast<float4*>(stage + (e / 32) * LD + 4 * (e % 32)) = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ci = i0; ci <= i1; ++ci) {
+      const float* pp = part + (long long)(ci + pf) * (D * 2 * D);
+      float4 av[8][2];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        av[i][0] = *reinterpret_cast<const float4*>(pp + (r0 + i) * (2 * D) + c0);
+        av[i][1] = *reinterpret_cast<const float4*>(pp + (r0 + i) * (2 * D) + c0 + 4);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        a[i][0] = __fadd2_rn(a[i][0], make_float2(av[i][0].x, av[i][0].y));
+        a[i][1] = __fadd2_rn(a[i][1], make_float2(av[i][0].z, av[i][0].w));
+        a[i][2] = __fadd2_rn(a[i][2], make_float2(av[i][1].x, av[i][1].y));
+        a[i][3] = __fadd2_rn(a[i][3], make_float2(av[i][1].z, av[i][1].w));
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float4 bv[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int e4 = tid + 256 * (8 * half + r), row = e4 / 32, c4 = e4 % 32;
+          bv[r] = *reinterpret_cast<const float4*>(pp + row * (2 * D) + D + 4 * c4);
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int e4 = tid + 256 * (8 * half + r), row = e4 / 32, c4 = e4 % 32;
+          float4* st = reinterpret_cast<float4*>(stage + row * LD + 4 * c4);
+          float4 v = *st;
+          v.x += bv[r].x; v.y += bv[r].y; v.z += bv[r].z; v.w += bv[r].w;
+          *st = v;
+        }
+      }
+    }
+    __syncthreads();
+    float* Bf = Bsum + fi * D * D;     // B[i][j] = (B^T)[j][i]
+    for (int e = tid; e < D * D; e += 256) Bf[e] = stage[(e % D) * LD + (e / D)];
+    if (Aout) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          *reinterpret_cast<float2*>(Aout + fi * D * D + (r0 + i) * D + c0 + 2 * p) = a[i][p];
+    }
+    __syncthreads();
+  }
+
+  // N = I + c^2 A (solve rules), I - c^2 A (sana) or I (additive)
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float d0 = (r0 + i == c0 + 2 * p) ? 1.f : 0.f, d1 = (r0 + i == c0 + 2 * p + 1) ? 1.f : 0.f;
+      const float s = rc.solve ? rc.c2 : -rc.c2;
+      a[i][p] = rc.identity ? make_float2(d0, d1) : make_float2(fmaf(s, a[i][p].x, d0), fmaf(s, a[i][p].y, d1));
+    }
+
+  if (rc.solve) {
+    // in-place Gauss-Jordan; pivot j = 8 jt + jj
+    for (int jt = 0; jt < 16; ++jt) {
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = 8 * jt + jj;
+        float* cv = colv + (j & 1) * D;
+        float* rv = rowv + (j & 1) * D;
+        if (tx == jt) {   // column j segment: rows r0..r0+7
+          float col[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) col[i] = (jj & 1) ? a[i][jj >> 1].y : a[i][jj >> 1].x;
+          *reinterpret_cast<float4*>(cv + r0) = make_float4(col[0], col[1], col[2], col[3]);
+          *reinterpret_cast<float4*>(cv + r0 + 4) = make_float4(col[4], col[5], col[6], col[7]);
+        }
+        if (ty == jt) {   // row j segment: columns c0..c0+7
+          *reinterpret_cast<float4*>(rv + c0) = make_float4(a[jj][0].x, a[jj][0].y, a[jj][1].x, a[jj][1].y);
+          *reinterpret_cast<float4*>(rv + c0 + 4) = make_float4(a[jj][2].x, a[jj][2].y, a[jj][3].x, a[jj][3].y);
+        }
+        __syncthreads();
+        const float pv = cv[j];
+        float r;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(pv));
+        r = r * fmaf(-pv, r, 2.0f);                       // one Newton step
+        const float4 ca = *reinterpret_cast<const float4*>(cv + r0);
+        const float4 cb = *reinterpret_cast<const float4*>(cv + r0 + 4);
+        const float4 ra = *reinterpret_cast<const float4*>(rv + c0);
+        const float4 rb = *reinterpret_cast<const float4*>(rv + c0 + 4);
+        const float cr[8] = {ca.x * r, ca.y * r, ca.z * r, ca.w * r, cb.x * r, cb.y * r, cb.z * r, cb.w * r};
+        const float2 rk[4] = {make_float2(ra.x, ra.y), make_float2(ra.z, ra.w), make_float2(rb.x, rb.y),
+                              make_float2(rb.z, rb.w)};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 m = make_float2(-cr[i], -cr[i]);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) a[i][p] = __ffma2_rn(m, rk[p], a[i][p]);
+        }
+        if (ty == jt) {   // row j: A[j][k] / p
+#pragma unroll
+          for (int p = 0; p < 4; ++p) a[jj][p] = make_float2(rk[p].x * r, rk[p].y * r);
+        }
+        if (tx == jt) {   // column j: -A[i][j] / p
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (jj & 1) a[i][jj >> 1].y = -cr[i];
+            else a[i][jj >> 1].x = -cr[i];
+          }
+        }
+        if (ty == jt && tx == jt) {
+          if (jj & 1) a[jj][jj >> 1].y = r;
+          else a[jj][jj >> 1].x = r;
+        }
+      }
+    }
+  }
+
+  if (Nm) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) *reinterpret_cast<float2*>(Nm + fi * D * D + (r0 + i) * D + c0 + 2 * p) = a[i][p];
+  }
+  if (nimg) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      *reinterpret_cast<float4*>(stage + (r0 + i) * LD + c0) = make_float4(a[i][0].x, a[i][0].y, a[i][1].x, a[i][1].y);
+      *reinterpret_cast<float4*>(stage + (r0 + i) * LD + c0 + 4) =
+          make_float4(a[i][2].x, a[i][2].y, a[i][3].x, a[i][3].y);
+    }
+    __syncthreads();
+    // B operand of the scan: row n holds N_f[n][k]; N_f is symmetric, so this is
+    // its column n as the product S N_f needs (up to fp32 rounding of the inverse)
+    write_image128_rows(stage, LD, nimg + fi * (kImgBytes / 2));
+  }
+}
+
 cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nimg, const float* partials,
                          float* Bsum, float* Aout) {
+  if (a.sh.d == 128 && partials) {
+    RuleCoef rc = rule_coef(a.rule, a.c);
+    int nb = (a.sh.S + kStatsTokens - 1) / kStatsTokens;
+    long long T = a.NF() * nb;
+    int G = (int)(T < kStatsGrid ? T : kStatsGrid);
+    size_t smem = ((size_t)128 * 132 + 4 * 128) * sizeof(float);
+    cudaFuncSetAttribute(k_solve128, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_solve128<<<(unsigned)a.NF(), 256, smem, a.stream>>>(partials, T, nb, G, rc, Nm, nimg, Bsum, Aout, a.sh.H,
+                                                          a.sh.F);
+    return cudaGetLastError();
+  }
   RuleCoef rc = rule_coef(a.rule, a.c);
   int d = a.sh.d;
   size_t smem = ((size_t)d * (d + 1) + 4 * d) * sizeof(float);

@@ -19,7 +19,9 @@
 // fixed order, so the result is deterministic.
 //
 // Warp roles (448 threads): 0 TMA producer, 1 MMA issuer (TMEM owner),
-// 2-9 transform (4 tokens x 8 channels per thread), 10-13 flush (one TMEM lane each).
+// 2-13 transform (4 tokens x 8 channels per thread, 96-token blocks); transform
+// warps 2-5 (one per TMEM lane quarter) also flush the accumulator when a
+// frame segment ends.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -31,17 +33,23 @@ namespace {
 
 constexpr int kRS = 3;                 // raw TMA stages
 constexpr int kRawRows = kStatsTokens + 2;
-constexpr int kRawHalf = 9216;         // 66 rows x 128 B, padded to 9 KB (1024-aligned)
+constexpr int kRawHalf = 13312;        // 98 rows x 128 B, padded to 13 KB (1024-aligned)
 constexpr int kRawBytes = 4 * kRawRows * 128;   // k and v, two channel halves each
-constexpr int kThreads = 448;
+constexpr int kTransformWarps = 12;    // 8 tokens each
+constexpr int kTransformThreads = 32 * kTransformWarps;
+constexpr int kThreads = 64 + kTransformThreads;
+constexpr int kKAtoms = kStatsTokens / 8;       // 8-token swizzle atoms along K
+constexpr int kOpHalf = kKAtoms * 2048;         // X (or Y): 128 channels x kStatsTokens bf16
+constexpr int kMnAtomStride = kKAtoms * 1024;   // descriptor leading offset: next 64 channels
 
 struct __align__(1024) StatsSmem {
   uint8_t raw[kRS][2][2][kRawHalf];    // [stage][k|v][channel half]
-  uint8_t op[2][32768];                // [stage]: X (16 KB) | Y (16 KB), MN-major SW128
+  uint8_t op[2 * kOpHalf];             // X | Y, MN-major SW128; one stage: the transform
+                                       // computes block i+1 while the MMA reads block i
   float taps[kRS][2][3][128];          // [stage][k|v][tap][channel] conv taps of the stage's head
   float sqb[kRS][kStatsTokens];        // [stage][token] sqrt(beta), 0 past the frame end
   uint64_t raw_full[kRS], raw_empty[kRS];
-  uint64_t op_full[2], op_empty[2];
+  uint64_t op_full, op_empty;
   uint64_t acc_full[2], acc_empty[2];
   uint32_t tmem_base;
   int abort;
@@ -50,9 +58,10 @@ struct __align__(1024) StatsSmem {
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 256, true, true);
 
 // byte offset of the 16-byte chunk holding channels 8c..8c+7 of token t in an
-// MN-major SW128 operand of 128 channels x 64 tokens (atoms of 64 ch x 8 tokens)
+// MN-major SW128 operand of 128 channels x kStatsTokens tokens (atoms of
+// 64 channels x 8 tokens, 1 KB each; K atoms contiguous, channel halves apart)
 __device__ __forceinline__ uint32_t op_chunk(int c, int t) {
-  return (c >> 3) * 8192 + (t >> 3) * 1024 + (t & 7) * 128 + ((((c & 7) ^ (t & 7))) << 4);
+  return (c >> 3) * kMnAtomStride + (t >> 3) * 1024 + (t & 7) * 128 + ((((c & 7) ^ (t & 7))) << 4);
 }
 
 }  // namespace
@@ -73,11 +82,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < kRS; ++s) {
       tc::mbar_init(&sm.raw_full[s], 1);
-      tc::mbar_init(&sm.raw_empty[s], 256);
+      tc::mbar_init(&sm.raw_empty[s], kTransformThreads);
     }
+    tc::mbar_init(&sm.op_full, kTransformThreads);
+    tc::mbar_init(&sm.op_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&sm.op_full[s], 256);
-      tc::mbar_init(&sm.op_empty[s], 1);
       tc::mbar_init(&sm.acc_full[s], 1);
       tc::mbar_init(&sm.acc_empty[s], 128);
     }
@@ -168,22 +177,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       int it = 0, seg = 0;
       bool first = true;
       for (long long x = x0; x < x1; ++x, ++it) {
-        const int os = it & 1;
-        const uint32_t oph = (it >> 1) & 1;
+        const uint32_t oph = it & 1;
         const int ab = seg & 1;
         if (first) {
           if (!tc::mbar_wait(&sm.acc_empty[ab], ((seg >> 1) & 1) ^ 1, abort_flag, status)) break;
         }
-        if (!tc::mbar_wait(&sm.op_full[os], oph, abort_flag, status)) break;
+        if (!tc::mbar_wait(&sm.op_full, oph, abort_flag, status)) break;
         tc::tc_fence_after();
         const uint32_t d = tmem + ab * 256;
-        const uint32_t base = tc::smem_u32(sm.op[os]);
+        const uint32_t base = tc::smem_u32(sm.op);
 #pragma unroll
         for (int kk = 0; kk < kStatsTokens / 16; ++kk) {
-          uint64_t desc = tc::smem_desc(base + kk * 2048, 8192, 1024);
+          uint64_t desc = tc::smem_desc(base + kk * 2048, kMnAtomStride, 1024);
           tc::umma_bf16(d, desc, desc, kIdesc, (first && kk == 0) ? 0u : 1u);
         }
-        tc::umma_commit(&sm.op_empty[os]);
+        tc::umma_commit(&sm.op_empty);
         first = false;
         if (seg_last(x)) {
           tc::umma_commit(&sm.acc_full[ab]);
@@ -192,25 +200,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
         }
       }
     }
-  } else if (warp < 10) {
-    // ------------------------------------------------------------ transform
+  } else {
+    // ------------------------------------------------------------ transform (+ flush)
     const int tt = tid - 64;
-    const int w8 = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
+    const int w12 = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
     const int half = c >> 3, cc = c & 7;
-    const int tok0 = 8 * w8 + 4 * tg;       // first of this thread's 4 tokens in the block
-    const float2 half2 = make_float2(0.5f, 0.5f);
+    const int tok0 = 8 * w12 + 4 * tg;      // first of this thread's 4 tokens in the block
+    const bool flusher = w12 < 4;           // warps 2-5: TMEM lane quarters 2, 3, 0, 1
+    const int quarter = warp & 3;
+    int seg = 0;
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
       const int rs = it % kRS;
       const uint32_t rph = (it / kRS) & 1;
-      const int os = it & 1;
-      const uint32_t oph = (it >> 1) & 1;
+      const uint32_t oph = it & 1;
       if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
       float sb[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) sb[i] = sm.sqb[rs][tok0 + i];
 
-      // conv (3 taps, packed pairs of channels), SiLU; k also sums its squares
+      // conv (3 taps, packed pairs of channels), SiLU; k also sums its squares.
+      // Written stage by stage (all convolutions, then all tanh, then the
+      // combination) so the 16 independent chains issue back to back.
       auto conv_silu = [&](int ten, float2 (&outp)[4][4], float (&ss)[4]) {
         float2 w[3][4];
 #pragma unroll
@@ -231,17 +242,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           r[rr][2] = make_float2(bf16lo(q.z), bf16hi(q.z));
           r[rr][3] = make_float2(bf16lo(q.w), bf16hi(q.w));
         }
+        float2 hx[4][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float2 acc = make_float2(0.f, 0.f);
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
             float2 a = __fmul2_rn(w[2][p], r[i + 2][p]);
             a = __ffma2_rn(w[1][p], r[i + 1][p], a);
             a = __ffma2_rn(w[0][p], r[i][p], a);
-            const float2 hx = __fmul2_rn(a, half2);
-            const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
-            const float2 y = __ffma2_rn(hx, th, hx);         // x sigmoid(x) = h + h tanh(h), h = x/2
+            hx[i][p] = __fmul2_rn(a, make_float2(0.5f, 0.5f));
+          }
+        float2 th[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int p = 0; p < 4; ++p) th[i][p] = tanh2(hx[i][p]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 y = __ffma2_rn(hx[i][p], th[i][p], hx[i][p]);   // x sigmoid(x) = h + h tanh(h)
             outp[i][p] = y;
             acc = __ffma2_rn(y, y, acc);
           }
@@ -252,16 +273,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       float2 kx[4][4], vx[4][4];
       float ssq[4], unused[4];
       conv_silu(0, kx, ssq);
+      // the k row sums travel through the 16 lanes of the token group while v is computed
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], 1);
       conv_silu(1, vx, unused);
       tc::mbar_arrive(&sm.raw_empty[rs]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
 #pragma unroll
-        for (int o = 1; o < 16; o <<= 1) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], o);
+        for (int o = 2; o < 16; o <<= 1) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], o);
         ssq[i] = sb[i] * rsqrtf(ssq[i] + kL2Eps);
       }
-      if (!tc::mbar_wait(&sm.op_empty[os], oph ^ 1, abort_flag, status)) break;
-      uint8_t* dst = sm.op[os];
+      if (!tc::mbar_wait(&sm.op_empty, oph ^ 1, abort_flag, status)) break;
+      uint8_t* dst = sm.op;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = tok0 + i;
@@ -275,36 +299,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           wyv[p] = pack_bf16x2(b.x, b.y);
         }
         *reinterpret_cast<uint4*>(dst + op_chunk(c, t)) = make_uint4(wxv[0], wxv[1], wxv[2], wxv[3]);
-        *reinterpret_cast<uint4*>(dst + 16384 + op_chunk(c, t)) = make_uint4(wyv[0], wyv[1], wyv[2], wyv[3]);
+        *reinterpret_cast<uint4*>(dst + kOpHalf + op_chunk(c, t)) = make_uint4(wyv[0], wyv[1], wyv[2], wyv[3]);
       }
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&sm.op_full[os]);
-    }
-  } else {
-    // ------------------------------------------------------------ flush [A | B^T] partials
-    const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;
-    int seg = 0;
-    for (long long x = x0; x < x1; ++x) {
-      if (!seg_last(x)) continue;
-      const int ab = seg & 1;
-      if (!tc::mbar_wait(&sm.acc_full[ab], (seg >> 1) & 1, abort_flag, status)) break;
-      tc::tc_fence_after();
-      const long long pf = x / nb;
-      float* dst = part + ((long long)blockIdx.x + pf) * (128 * 256) + (long long)m * 256;
-      const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quarter * 32) << 16);
+      tc::mbar_arrive(&sm.op_full);
+      if (flusher && seg_last(x)) {
+        // the segment of this frame is complete once its last block's MMA is:
+        // copy the [A | B^T] accumulator rows to partial slot (blockIdx.x + frame)
+        const int ab = seg & 1;
+        if (!tc::mbar_wait(&sm.acc_full[ab], (seg >> 1) & 1, abort_flag, status)) break;
+        tc::tc_fence_after();
+        const long long pf = x / nb;
+        const int m = quarter * 32 + lane;
+        float* dstp = part + ((long long)blockIdx.x + pf) * (128 * 256) + (long long)m * 256;
+        const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        uint32_t r[32];
-        tc::tmem_ld32(taddr + 32 * j, r);
-        tc::tmem_ld_wait();
+        for (int j = 0; j < 8; ++j) {
+          uint32_t r[32];
+          tc::tmem_ld32(taddr + 32 * j, r);
+          tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<uint4*>(dst + 32 * j + e) = make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<uint4*>(dstp + 32 * j + e) = make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.acc_empty[ab]);
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&sm.acc_empty[ab]);
-      ++seg;
+      if (seg_last(x)) ++seg;
     }
   }
 
