@@ -1,0 +1,81 @@
+"""Host logic of bench.py: roofline arithmetic, the traffic table, and the
+multi-rank helpers on two gloo ranks (CPU, 127.0.0.1)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from video_diffusion_linear_b200 import synth
+
+
+def test_path_roofline_768p():
+    w = synth.WORKLOADS["768p"]
+    pr = bench.path_roofline(w, {"hbm_gbs": 6546.9, "bf16_tflops": 1590.1})
+    assert pr["bound"] == "hbm"
+    assert abs(pr["bytes"] / 1e9 - 4.09) < 0.01          # q, k, v, gate, beta in, out, per-frame maps
+    assert abs(pr["t_roof_us"] - 625) < 2
+    assert abs(pr["flops"] / 1e9 - 305.8) < 0.5
+
+
+def test_algorithmic_bytes_cover_the_path():
+    w = synth.WORKLOADS["768p"]
+    alg = bench.algorithmic_bytes(w)
+    TH = w.B * w.F * w.S * w.H
+    assert alg["frame_stats"] >= TH * 516 and alg["readout"] >= TH * 768
+    assert set(alg) == set(bench.KERNELS_TC)
+
+
+def test_recorded_traffic_tracks_source():
+    for k in bench.KERNELS_TC:
+        rec = bench.recorded_traffic(k)
+        if rec is not None:                      # present only while the kernel source is unchanged
+            assert rec["bytes"] > 0 and rec["workload"] == "768p"
+
+
+def test_rank_workloads_are_distinct_clips():
+    w = synth.WORKLOADS["768p"]
+    seeds = {bench.rank_workload(w, r).seed for r in range(8)}
+    assert len(seeds) == 8
+    assert all(bench.rank_workload(w, r).tokens == w.tokens for r in range(8))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier()
+        m = bench.reduce_max(float(10 + rank))
+        q.put((rank, m, bench.dist_env()[:2]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [11.0, 11.0]
+    assert [tuple(r[2]) for r in res] == [(0, 2), (1, 2)]
+
+
+def test_reduce_max_without_process_group():
+    assert bench.reduce_max(3.5) == 3.5
