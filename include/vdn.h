@@ -174,6 +174,30 @@ vdn_status vdn_branch_forward_timed(const vdn_shape* shape,
                                     void* out, void* stream,
                                     void* const* events, int n_events);
 
+/* vdn_branch_forward without a caller workspace (the page has no counterpart:
+ * this is a deployment variant).  For callers that cannot allocate device
+ * memory where they run the branch -- code running while a stream is captured
+ * into a CUDA graph, where cudaMalloc is refused, or runtimes whose device
+ * memory belongs to a framework allocator or a fixed arena -- the scratch lives
+ * in one library-owned device array of 64 MiB, which every GPU that loads the
+ * library holds until the process exits.  Problems whose workspace
+ * (vdn_branch_workspace_size) exceeds 64 MiB are refused with VDN_ERR_WORKSPACE
+ * before any CUDA call.  Inputs, output and errors are those of
+ * vdn_branch_forward.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, which may load the library's device code), so
+ * make that first call before any stream capture.  All calls share the array
+ * and it keeps the last call's contents: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller.  Calls no
+ * cudaMalloc, cudaFree or allocating library routine. */
+vdn_status vdn_branch_forward_static(const vdn_shape* shape,
+                                     const void* q, const void* k, const void* v,
+                                     const float* beta, const float* alpha,
+                                     const void* gate, const float* rms_w,
+                                     const float* conv_k_w, const float* conv_v_w,
+                                     const float* text_state,
+                                     int rule, float c, int chunk, int radius,
+                                     void* out, void* stream);
+
 /* "Step 1" alone (page: NoPE features): q' = L2(SiLU(q)), k' = L2(SiLU(conv_k(k))),
  * v' = SiLU(conv_v(v)), all [B, F*S, H, d] in shape->dtype.  Outputs must not
  * overlap the inputs.  Needs no workspace. */
