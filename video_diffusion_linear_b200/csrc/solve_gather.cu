@@ -541,8 +541,128 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
   }
 }
 
+// d = 128, one CTA per (batch, head, window chunk): every query frame of a chunk
+// has the same window [lo, hi], hence the same two boundary states; they are
+// read once and each frame's W_t differs only in its two decay vectors.
+constexpr int kGatherMaxChunk = 16;
+
+__global__ void __launch_bounds__(512) k_gather128_chunk(const float* __restrict__ P, const float* __restrict__ Q,
+                                                         const int* __restrict__ pexp, const int* __restrict__ qexp,
+                                                         const float* __restrict__ alpha,
+                                                         const float* __restrict__ text, int H, int F, int chunk,
+                                                         int radius, float* __restrict__ W,
+                                                         uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
+  constexpr int D = 128;
+  __shared__ float dpre[kGatherMaxChunk][D], dsuf[kGatherMaxChunk][D], red[2][16];
+  const int tid = threadIdx.x, n = tid >> 2, k0 = (tid & 3) * 32;
+  const long long bh = blockIdx.x;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const int t0 = blockIdx.y * chunk, t1 = min(F, t0 + chunk);   // query frames of this chunk
+  int lo, hi;
+  window_bounds(t0, F, chunk, radius, lo, hi);
+  const float* pre = lo > 0 ? P + (bh * F + (lo - 1)) * D * D : nullptr;
+  const float* suf = hi < F - 1 ? Q + (bh * F + (hi + 1)) * D * D : nullptr;
+  const float* seed = text ? text + (long long)h * D * D : nullptr;
+  float4 pv[8], sv[8];
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int off = n * D + k0 + 4 * j;
+    pv[j] = pre ? *reinterpret_cast<const float4*>(pre + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
+    sv[j] = suf ? *reinterpret_cast<const float4*>(suf + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
+  }
+  if (tid < D) {
+    // dpre[t] = prod_{g=lo..t} alpha_g,  dsuf[t] = prod_{g=t..hi} alpha_g
+    const float* al = alpha + (b * F * H + h) * D + tid;
+    float dp = 1.f;
+    for (int g = lo; g < t0; ++g) dp *= al[(long long)g * H * D];
+    for (int t = t0; t < t1; ++t) {
+      dp *= al[(long long)t * H * D];
+      dpre[t - t0][tid] = dp;
+    }
+    float ds = 1.f;
+    for (int g = hi; g >= t1; --g) ds *= al[(long long)g * H * D];
+    for (int t = t1 - 1; t >= t0; --t) {
+      ds *= al[(long long)t * H * D];
+      dsuf[t - t0][tid] = ds;
+    }
+  }
+  const int ep = pre ? pexp[bh * F + (lo - 1)] : 0;
+  const int eq = suf ? qexp[bh * F + (hi + 1)] : 0;
+  const int ew = ep > eq ? ep : eq;
+  const float sp = (pre ? 1.f : (seed ? kTextStateScale : 0.f)) * ldexpf(1.f, ep - ew);
+  const float sq = (suf ? 1.f : (seed ? kTextStateScale : 0.f)) * ldexpf(1.f, eq - ew);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    pv[j].x *= sp; pv[j].y *= sp; pv[j].z *= sp; pv[j].w *= sp;
+    sv[j].x *= sq; sv[j].y *= sq; sv[j].z *= sq; sv[j].w *= sq;
+  }
+  __syncthreads();
+  for (int t = t0; t < t1; ++t) {
+    const float* dp = dpre[t - t0];
+    const float* ds = dsuf[t - t0];
+    float w[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = k0 + 4 * j;
+      w[4 * j + 0] = fmaf(pv[j].x, dp[k + 0], sv[j].x * ds[k + 0]);
+      w[4 * j + 1] = fmaf(pv[j].y, dp[k + 1], sv[j].y * ds[k + 1]);
+      w[4 * j + 2] = fmaf(pv[j].z, dp[k + 2], sv[j].z * ds[k + 2]);
+      w[4 * j + 3] = fmaf(pv[j].w, dp[k + 3], sv[j].w * ds[k + 3]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(w[4 * j + u]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float* rd = red[t & 1];   // double buffer: one barrier per frame
+    if ((tid & 31) == 0) rd[tid >> 5] = amax;
+    __syncthreads();
+    amax = rd[0];
+#pragma unroll
+    for (int u = 1; u < 16; ++u) amax = fmaxf(amax, rd[u]);
+    int ek = 0;
+    if (amax > 0.f) frexpf(amax, &ek);
+    const long long fi = bh * F + t;
+    if (tid == 0) wexp[fi] = ew + ek;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) w[u] = ldexpf(w[u], -ek);
+    if (W) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(W + fi * D * D + n * D + k0 + 4 * j) =
+            make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    }
+    if (wimg) {
+      uint8_t* img = reinterpret_cast<uint8_t*>(wimg + fi * (kImgBytes / 2));
+#pragma unroll
+      for (int cch = 0; cch < 4; ++cch) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          __nv_bfloat16 h0, l0, h1, l1;
+          split_bf16(w[8 * cch + e], h0, l0);
+          split_bf16(w[8 * cch + e + 1], h1, l1);
+          hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const uint32_t off = img_offset(0, n, k0 + 8 * cch);
+        *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
+  }
+}
+
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
                           uint16_t* wimg, int* wexp) {
+  if (a.sh.d == 128 && a.chunk <= kGatherMaxChunk) {
+    dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((a.sh.F + a.chunk - 1) / a.chunk));
+    k_gather128_chunk<<<grid, 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
+                                                   a.radius, W, wimg, wexp);
+    return cudaGetLastError();
+  }
   if (a.sh.d == 128) {
     k_gather128<<<(unsigned)a.NF(), 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
                                                         a.chunk, a.radius, W, wimg, wexp);

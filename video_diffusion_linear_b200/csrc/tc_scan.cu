@@ -3,7 +3,7 @@
 // frames, each seeded with 0.5 x the text state).
 //
 // One CTA per (batch, head, direction) walks the frames serially:
-//     X_f = S_{f-1} D_f + cpre B_f            (fp32, one state row per thread)
+//     X_f = S_{f-1} D_f + cpre B_f            (fp32, two threads per state row)
 //     S_f = X_f N_f + cpost B_f               (tcgen05, 128x128x128)
 // The product runs in bf16 with hi/lo splitting of both operands
 // (X = Xh + Xl, N = Nh + Nl; D = Xh Nh + Xh Nl + Xl Nh), which keeps about 16
@@ -43,24 +43,40 @@ __device__ __forceinline__ uint32_t bf_offset(int row, int col) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmB,
-                                                   const uint16_t* __restrict__ nimg_g,
-                                                   const float* __restrict__ alpha,
-                                                   const float* __restrict__ text, RuleCoef rc,
-                                                   float* __restrict__ P, float* __restrict__ Q,
-                                                   int* __restrict__ pexp, int* __restrict__ qexp, int H, int F,
-                                                   int chunk, int all_frames, uint32_t* __restrict__ status) {
+// Two threads per state row: thread t owns row m = 32 (warp % 4) + lane (the
+// TMEM lane quarter its warp may read) and columns 64 ch .. 64 ch + 63, ch = t / 128.
+constexpr int kScanThreads = 256;
+
+// bf16 hi/lo split of a pair: hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split_pair(float2 x, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(x.x, x.y);
+  const float2 hf = make_float2(bf16lo(hi), bf16hi(hi));
+  const float2 r = __fadd2_rn(x, make_float2(-hf.x, -hf.y));
+  lo = pack_bf16x2(r.x, r.y);
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmB,
+                                                            const uint16_t* __restrict__ nimg_g,
+                                                            const float* __restrict__ alpha,
+                                                            const float* __restrict__ text, RuleCoef rc,
+                                                            float* __restrict__ P, float* __restrict__ Q,
+                                                            int* __restrict__ pexp, int* __restrict__ qexp, int H,
+                                                            int F, int chunk, int all_frames,
+                                                            uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int m = threadIdx.x;
-  const int warp = m >> 5;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int m = 32 * (warp & 3) + lane;     // state row (v channel) = TMEM lane
+  const int ch = tid >> 7;                   // column half
+  const int k0 = 64 * ch;
   const int dir = blockIdx.x & 1;
   const long long bh = blockIdx.x >> 1;
   const int h = (int)(bh % H);
   const long long b = bh / H;
   volatile int* abort_flag = &sm.abort;
 
-  if (m == 0) {
+  if (tid == 0) {
     tc::mbar_init(&sm.bar_n, 1);
     tc::mbar_init(&sm.bar_b, 1);
     tc::mbar_init(&sm.bar_mma, 1);
@@ -75,13 +91,14 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t t_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + k0;
 
-  float s[128];
+  float2 s[32];   // s[p] = state[m][k0 + 2p .. k0 + 2p + 1]
   {
-    const float* T = text ? text + ((long long)h * 128 + m) * 128 : nullptr;
+    const float* T = text ? text + ((long long)h * 128 + m) * 128 + k0 : nullptr;
 #pragma unroll
-    for (int k = 0; k < 128; ++k) s[k] = T ? kTextStateScale * T[k] : 0.f;
+    for (int p = 0; p < 32; ++p)
+      s[p] = T ? make_float2(kTextStateScale * T[2 * p], kTextStateScale * T[2 * p + 1]) : make_float2(0.f, 0.f);
   }
 
   auto frame_of = [&](int step) { return dir == 0 ? step : F - 1 - step; };
@@ -98,9 +115,14 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
 #pragma unroll
     for (int j = 0; j < 4; ++j) tc::tma_load_2d(&tmB, &sm.bar_b, sm.bf[j], 32 * j, (int)(fi * 128));
   };
-  if (m == 0) {
+  auto prefetch = [&](int step) {   // next frame's operands into L2 (hint only)
+    long long fi = bh * F + frame_of(step);
+    tc::prefetch_l2(reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2)), kImgBytes);
+  };
+  if (tid == 0) {
     load_n(0);
     load_b(0);
+    if (F > 1) prefetch(1);
   }
 
   const bool early_b = rc.cpost == 0.f;   // B_f is only read before the product
@@ -110,33 +132,37 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
   const uint8_t* bfb = reinterpret_cast<const uint8_t*>(sm.bf);
 
   int ex = 0;   // block exponent: the true state is 2^ex s
-  float a_next = alpha[((b * F + frame_of(0)) * H + h) * 128 + m];
+  float a_next = tid < 128 ? alpha[((b * F + frame_of(0)) * H + h) * 128 + tid] : 0.f;
   for (int step = 0; step < F; ++step) {
     const int f = frame_of(step);
     const long long fi = bh * F + f;
     const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
-    sm.alpha[m] = a_next;
-    if (step + 1 < F) a_next = alpha[((b * F + frame_of(step + 1)) * H + h) * 128 + m];   // used next step
+    if (tid < 128) {
+      sm.alpha[tid] = a_next;
+      if (step + 1 < F) a_next = alpha[((b * F + frame_of(step + 1)) * H + h) * 128 + tid];   // used next step
+    }
+    if (tid == 0 && step + 2 < F) prefetch(step + 2);
     __syncthreads();
     if (!tc::mbar_wait(&sm.bar_b, ph, abort_flag, status)) break;
 
-    // X = S D + cpre B  ->  bf16 hi / lo A operands (row m)
+    // X = S D + cpre B  ->  bf16 hi / lo A operands (row m, columns k0 .. k0 + 63)
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      float4 b0 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, 8 * c));
-      float4 b1 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, 8 * c + 4));
-      float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    for (int c = 0; c < 8; ++c) {
+      const int k = k0 + 8 * c;
+      const float4 al0 = *reinterpret_cast<const float4*>(&sm.alpha[k]);
+      const float4 al1 = *reinterpret_cast<const float4*>(&sm.alpha[k + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, k));
+      const float4 b1 = *reinterpret_cast<const float4*>(bfb + bf_offset(m, k + 4));
+      const float2 cp = make_float2(cpre, cpre);
+      float2 x[4];
+      x[0] = __ffma2_rn(s[4 * c + 0], make_float2(al0.x, al0.y), __fmul2_rn(cp, make_float2(b0.x, b0.y)));
+      x[1] = __ffma2_rn(s[4 * c + 1], make_float2(al0.z, al0.w), __fmul2_rn(cp, make_float2(b0.z, b0.w)));
+      x[2] = __ffma2_rn(s[4 * c + 2], make_float2(al1.x, al1.y), __fmul2_rn(cp, make_float2(b1.x, b1.y)));
+      x[3] = __ffma2_rn(s[4 * c + 3], make_float2(al1.z, al1.w), __fmul2_rn(cp, make_float2(b1.z, b1.w)));
       uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        float x0 = fmaf(s[8 * c + e], sm.alpha[8 * c + e], cpre * bv[e]);
-        float x1 = fmaf(s[8 * c + e + 1], sm.alpha[8 * c + e + 1], cpre * bv[e + 1]);
-        float h0 = __bfloat162float(__float2bfloat16_rn(x0));
-        float h1 = __bfloat162float(__float2bfloat16_rn(x1));
-        hw[e / 2] = pack_bf16x2(h0, h1);
-        lw[e / 2] = pack_bf16x2(x0 - h0, x1 - h1);
-      }
-      uint32_t off = img_offset(0, m, 8 * c);
+      for (int q = 0; q < 4; ++q) split_pair(x[q], hw[q], lw[q]);
+      const uint32_t off = img_offset(0, m, k);
       *reinterpret_cast<uint4*>(sm.aop[0] + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(sm.aop[1] + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
@@ -145,7 +171,7 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
     __syncthreads();
     tc::tc_fence_after();
 
-    if (m == 0) {
+    if (tid == 0) {
       if (early_b && step + 1 < F) load_b(step + 1);
       if (tc::mbar_wait(&sm.bar_n, ph, abort_flag, status)) {
         tc::tc_fence_after();
@@ -163,48 +189,47 @@ __global__ void __launch_bounds__(128, 1) k_scan_tc(const __grid_constant__ CUte
     }
     if (!tc::mbar_wait(&sm.bar_mma, ph, abort_flag, status)) break;
     tc::tc_fence_after();
-    if (m == 0 && step + 1 < F) load_n(step + 1);   // the product that read N_f is complete
+    if (tid == 0 && step + 1 < F) load_n(step + 1);   // the product that read N_f is complete
 
     // S_f = D + cpost B_f
     const bool store = all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0));
-    float* dst = (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128;
+    float* dst = (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0;
+    float amax = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 2; ++j) {
       uint32_t r[32];
       tc::tmem_ld32(t_row + 32 * j, r);
       tc::tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
+        const int p = 16 * j + e / 2;
         // with early_b the buffer already receives B_{f+1}: do not read it
-        float4 bv = early_b ? make_float4(0.f, 0.f, 0.f, 0.f)
-                            : *reinterpret_cast<const float4*>(bfb + bf_offset(m, 32 * j + e));
-        s[32 * j + e + 0] = fmaf(cpost, bv.x, __uint_as_float(r[e + 0]));
-        s[32 * j + e + 1] = fmaf(cpost, bv.y, __uint_as_float(r[e + 1]));
-        s[32 * j + e + 2] = fmaf(cpost, bv.z, __uint_as_float(r[e + 2]));
-        s[32 * j + e + 3] = fmaf(cpost, bv.w, __uint_as_float(r[e + 3]));
+        const float4 bv = early_b ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                  : *reinterpret_cast<const float4*>(bfb + bf_offset(m, k0 + 32 * j + e));
+        const float2 cq = make_float2(cpost, cpost);
+        s[p] = __ffma2_rn(cq, make_float2(bv.x, bv.y), make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])));
+        s[p + 1] = __ffma2_rn(cq, make_float2(bv.z, bv.w),
+                              make_float2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(s[p].x), fabsf(s[p].y)), fmaxf(fabsf(s[p + 1].x), fabsf(s[p + 1].y))));
         if (store)
-          *reinterpret_cast<float4*>(dst + 32 * j + e) =
-              make_float4(s[32 * j + e], s[32 * j + e + 1], s[32 * j + e + 2], s[32 * j + e + 3]);
+          *reinterpret_cast<float4*>(dst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
       }
     }
-    if (store && m == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 128; ++k) amax = fmaxf(amax, fabsf(s[k]));
+    if (store && tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
     tc::tc_fence_before();
     // accumulator and B_f reads done, alpha slot free; rescale if any entry passed 2^64
     if (__syncthreads_or(amax > kRenormAbove)) {
 #pragma unroll
-      for (int k = 0; k < 128; ++k) s[k] *= kRenormScale;
+      for (int p = 0; p < 32; ++p) s[p] = __fmul2_rn(s[p], make_float2(kRenormScale, kRenormScale));
       ex += kRenormExp;
     }
-    if (m == 0 && !early_b && step + 1 < F) load_b(step + 1);
+    if (tid == 0 && !early_b && step + 1 < F) load_b(step + 1);
     ph ^= 1;
   }
 
   // teardown: make sure no copy or product of ours is still in flight
   __syncthreads();
-  if (sm.abort && m == 0) {
+  if (sm.abort && tid == 0) {
     tc::mbar_wait(&sm.bar_n, ph, abort_flag, nullptr);
     tc::mbar_wait(&sm.bar_b, ph, abort_flag, nullptr);
   }
@@ -220,7 +245,7 @@ cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nim
   cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   RuleCoef rc = rule_coef(a.rule, a.c);
-  k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), 128, smem, a.stream>>>(
+  k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
       tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, status);
   return cudaGetLastError();
 }
