@@ -9,8 +9,9 @@
 // RMSNorm needs no cross-thread reduction; it multiplies rms_w and the gate and
 // writes bf16 through shared memory and a TMA store.
 //
-// Warp roles (320 threads): 0 TMA producer, 1 MMA issuer (and TMEM owner),
-// 2-5 q transform (one token row each), 6-9 epilogue (one TMEM lane each).
+// Warp roles (576 threads): 0 TMA producer, 1 MMA issuer (and TMEM owner),
+// 2-9 q transform and 10-17 epilogue, two threads per token row (64 channels
+// each; the row sums of squares meet in shared memory).
 #include "common.cuh"
 #include "image.cuh"
 #include "internal.h"
@@ -26,6 +27,8 @@ struct __align__(1024) ReadSmem {
   uint8_t qt[2][32768];    // raw q tile -> Q' (K-major SW128 A operand), two stages
   uint8_t gt[2][32768];    // gate tile -> output tile, two stages
   float rms_w[128];
+  float ssq_t[2][2][128];  // [stage][channel half][row] partial sums of the q transform
+  float ssq_e[2][2][128];  // same for the epilogue
   uint64_t bar_w_full, bar_w_empty;
   uint64_t bar_q_full[2], bar_q_ready[2], bar_q_empty[2];
   uint64_t bar_g_full[2], bar_g_empty[2];
@@ -35,7 +38,7 @@ struct __align__(1024) ReadSmem {
 };
 
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, false, false);
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 
 // swizzled byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] bf16 tile
 __device__ __forceinline__ uint32_t row_chunk(int r, int c) {
@@ -63,12 +66,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     tc::mbar_init(&sm.bar_w_empty, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&sm.bar_q_full[s], 1);
-      tc::mbar_init(&sm.bar_q_ready[s], 128);
+      tc::mbar_init(&sm.bar_q_ready[s], 256);
       tc::mbar_init(&sm.bar_q_empty[s], 1);
       tc::mbar_init(&sm.bar_g_full[s], 1);
       tc::mbar_init(&sm.bar_g_empty[s], 1);
       tc::mbar_init(&sm.bar_acc_full[s], 1);
-      tc::mbar_init(&sm.bar_acc_empty[s], 128);
+      tc::mbar_init(&sm.bar_acc_empty[s], 256);
     }
     sm.abort = 0;
     tc::fence_barrier_init();
@@ -77,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     tc::tmem_alloc(&sm.tmem_base, 256);
     tc::tmem_relinquish();
   }
-  if (tid >= 192) sm.rms_w[tid - 192] = rms_w[tid - 192];
+  if (tid >= 320 && tid < 448) sm.rms_w[tid - 320] = rms_w[tid - 320];
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -158,49 +161,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         if (x + 1 == x1 || (x + 1) / ntile != fi) tc::umma_commit(&sm.bar_w_empty);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ q' = L2(SiLU(q)), in place
-    // two passes over the row (sum of squares, then scale and store): SiLU is
-    // evaluated twice, which keeps the loop rolled and the row out of registers
-    const int r = tid - 64;
+    const int tt = tid - 64;
+    const int r = tt & 127, hf = tt >> 7;   // row, channel half (chunks 8 hf .. 8 hf + 7)
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
       const int st = it & 1;
       const uint32_t ph = (it >> 1) & 1;
       if (!tc::mbar_wait(&sm.bar_q_full[st], ph, abort_flag, status)) break;
       uint8_t* base = sm.qt[st];
-      float ss = 0.f;
-#pragma unroll 2
-      for (int c = 0; c < 16; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
+      float2 v[32];
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int cq = 0; cq < 8; ++cq) {
+        const uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, 8 * hf + cq));
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a0 = silu_fast(bf16lo(ws[e])), a1 = silu_fast(bf16hi(ws[e]));
-          ss = fmaf(a0, a0, fmaf(a1, a1, ss));
+          const float2 a = make_float2(silu_fast(bf16lo(ws[e])), silu_fast(bf16hi(ws[e])));
+          v[4 * cq + e] = a;
+          acc = __ffma2_rn(a, a, acc);
         }
       }
-      const float inv = rsqrtf(ss + kL2Eps);
-#pragma unroll 2
-      for (int c = 0; c < 16; ++c) {
-        uint4 w = *reinterpret_cast<const uint4*>(base + row_chunk(r, c));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      sm.ssq_t[st][hf][r] = acc.x + acc.y;
+      tc::named_bar(2, 256);
+      const float inv = rsqrtf(sm.ssq_t[st][0][r] + sm.ssq_t[st][1][r] + kL2Eps);
+      const float2 iv = make_float2(inv, inv);
+#pragma unroll
+      for (int cq = 0; cq < 8; ++cq) {
         uint32_t o4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          o4[e] = pack_bf16x2(silu_fast(bf16lo(ws[e])) * inv, silu_fast(bf16hi(ws[e])) * inv);
-        *reinterpret_cast<uint4*>(base + row_chunk(r, c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 y = __fmul2_rn(v[4 * cq + e], iv);
+          o4[e] = pack_bf16x2(y.x, y.y);
+        }
+        *reinterpret_cast<uint4*>(base + row_chunk(r, 8 * hf + cq)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&sm.bar_q_ready[st]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // pass 1 reads the accumulator row from TMEM for the sum of squares, pass 2
-    // reads it again to scale, gate and store (TMEM reads are cheap, registers not)
+    // thread (row m = TMEM lane, channel half hf) keeps its 64 accumulator values
+    // in registers; the two halves' sums of squares meet in shared memory
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
-    const bool leader = tid == 192;
+    const int hf = (warp - 10) >> 2;
+    const bool leader = tid == 320;
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
       const int st = it & 1;
@@ -212,45 +220,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       const int ew = wexp[x / ntile];   // issued before the wait, used after it
       if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
       tc::tc_fence_after();
-      const uint32_t taddr = tmem + st * 128 + ((uint32_t)(quarter * 32) << 16);
-      float ss = 0.f;
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        uint32_t rr[32];
-        tc::tmem_ld32(taddr + 32 * j, rr);
+      const uint32_t taddr = tmem + st * 128 + 64 * hf + ((uint32_t)(quarter * 32) << 16);
+      uint32_t o[64];
+      {
+        uint32_t (&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+        uint32_t (&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+        tc::tmem_ld32(taddr, o0);
+        tc::tmem_ld32(taddr + 32, o1);
         tc::tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(rr[e]), __uint_as_float(rr[e]), ss);
-      }
-      // W_t is stored as 2^-e W_t: the RMSNorm eps scales by 2^-2e
-      const float inv = rsqrtf(ss * (1.0f / 128.0f) + ldexpf(kRmsEps, -2 * ew));
-      if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
-      uint8_t* base = sm.gt[st];
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        uint32_t rr[32];
-        tc::tmem_ld32(taddr + 32 * j, rr);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int cq = 0; cq < 4; ++cq) {
-          const int c = 4 * j + cq;
-          const uint4 g = *reinterpret_cast<const uint4*>(base + row_chunk(m, c));
-          const uint32_t gs[4] = {g.x, g.y, g.z, g.w};
-          uint32_t outw[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 8 * c + 2 * e;
-            const float y0 = __uint_as_float(rr[8 * cq + 2 * e]) * inv * sm.rms_w[k] * bf16lo(gs[e]);
-            const float y1 = __uint_as_float(rr[8 * cq + 2 * e + 1]) * inv * sm.rms_w[k + 1] * bf16hi(gs[e]);
-            outw[e] = pack_bf16x2(y0, y1);
-          }
-          *reinterpret_cast<uint4*>(base + row_chunk(m, c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        }
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&sm.bar_acc_empty[st]);
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        const float2 a = make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1]));
+        acc = __ffma2_rn(a, a, acc);
+      }
+      sm.ssq_e[st][hf][m] = acc.x + acc.y;
+      tc::named_bar(1, 256);
+      // W_t is stored as 2^-e W_t: the RMSNorm eps scales by 2^-2e
+      const float ss = sm.ssq_e[st][0][m] + sm.ssq_e[st][1][m];
+      const float inv = rsqrtf(ss * (1.0f / 128.0f) + ldexpf(kRmsEps, -2 * ew));
+      if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
+      uint8_t* base = sm.gt[st];
+#pragma unroll
+      for (int cq = 0; cq < 8; ++cq) {
+        const int c = 8 * hf + cq;
+        const uint4 g = *reinterpret_cast<const uint4*>(base + row_chunk(m, c));
+        const uint32_t gs[4] = {g.x, g.y, g.z, g.w};
+        const float4 w0 = *reinterpret_cast<const float4*>(&sm.rms_w[8 * c]);
+        const float4 w1 = *reinterpret_cast<const float4*>(&sm.rms_w[8 * c + 4]);
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t outw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 8 * cq + 2 * e;
+          const float2 y = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                                 make_float2(inv * wv[2 * e], inv * wv[2 * e + 1])),
+                                      make_float2(bf16lo(gs[e]), bf16hi(gs[e])));
+          outw[e] = pack_bf16x2(y.x, y.y);
+        }
+        *reinterpret_cast<uint4*>(base + row_chunk(m, c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+      }
       tc::fence_proxy_async_smem();
-      tc::named_bar(1, 128);
+      tc::named_bar(1, 256);
       if (leader) {
         int h, s0, fb;
         coords(x, h, s0, fb);
