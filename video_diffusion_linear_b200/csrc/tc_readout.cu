@@ -9,9 +9,11 @@
 // RMSNorm needs no cross-thread reduction; it multiplies rms_w and the gate and
 // writes bf16 through shared memory and a TMA store.
 //
-// Warp roles (576 threads): 0 TMA producer, 1 MMA issuer (and TMEM owner),
-// 2-9 q transform and 10-17 epilogue, two threads per token row (64 channels
-// each; the row sums of squares meet in shared memory).
+// Warp roles (608 threads): 0 TMA producer of W and q, 1 MMA issuer (and TMEM
+// owner), 2-9 q transform and 10-17 epilogue, two threads per token row (64
+// channels each; the row sums of squares meet in shared memory), 18 TMA
+// producer of the gate tiles (its buffers free up later, after the output
+// store, so it runs apart from the q loads).
 #include "common.cuh"
 #include "image.cuh"
 #include "internal.h"
@@ -38,7 +40,7 @@ struct __align__(1024) ReadSmem {
 };
 
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, false, false);
-constexpr int kThreads = 576;
+constexpr int kThreads = 608;
 
 // swizzled byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] bf16 tile
 __device__ __forceinline__ uint32_t row_chunk(int r, int c) {
@@ -122,10 +124,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         tc::mbar_arrive_expect_tx(&sm.bar_q_full[st], 32768);
         tc::tma_load_4d(&tmQ, &sm.bar_q_full[st], sm.qt[st], 0, h, s0, fb);
         tc::tma_load_4d(&tmQ, &sm.bar_q_full[st], sm.qt[st] + 16384, 64, h, s0, fb);
-        if (!tc::mbar_wait(&sm.bar_g_empty[st], ph ^ 1, abort_flag, status)) break;
-        tc::mbar_arrive_expect_tx(&sm.bar_g_full[st], 32768);
-        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st], 0, h, s0, fb);
-        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st] + 16384, 64, h, s0, fb);
       }
     }
   } else if (warp == 1) {
@@ -159,6 +157,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         tc::umma_commit(&sm.bar_q_empty[st]);
         tc::umma_commit(&sm.bar_acc_full[st]);
         if (x + 1 == x1 || (x + 1) / ntile != fi) tc::umma_commit(&sm.bar_w_empty);
+      }
+    }
+  } else if (warp == 18) {
+    // ------------------------------------------------------------ gate producer
+    if (lane == 0) {
+      int it = 0;
+      for (long long x = x0; x < x1; ++x, ++it) {
+        int h, s0, fb;
+        coords(x, h, s0, fb);
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&sm.bar_g_empty[st], ph ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.bar_g_full[st], 32768);
+        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st], 0, h, s0, fb);
+        tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st] + 16384, 64, h, s0, fb);
       }
     }
   } else if (warp < 10) {
