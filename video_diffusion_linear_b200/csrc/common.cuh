@@ -103,12 +103,15 @@ __host__ __device__ __forceinline__ RuleCoef rule_coef(int rule, float c) {
 // Block exponent of the scan states.  A rule whose per-frame operator has
 // eigenvalues beyond 1 in magnitude (sana_scaled with c^2 |A| > 2) makes the
 // state grow without bound; the scans keep X with true state 2^e X and rescale
-// X by 2^-64 (exactly) whenever an entry passes 2^64, so the state never leaves
-// the fp32 range.  The read-out's RMSNorm is scale-free up to eps, which is
-// scaled by 2^(-2e) accordingly.
-constexpr float kRenormAbove = 18446744073709551616.0f;     // 2^64
-constexpr float kRenormScale = 5.42101086242752217e-20f;    // 2^-64
-constexpr int kRenormExp = 64;
+// X by 2^-32 (exactly) whenever an entry passes 2^32.  One step multiplies a
+// row norm by at most |D| |N| <= 1 + c^2 sum_s beta_s |k'_s|^2 <= 1 + c^2 S
+// (about 2^12 for S = 4096), and a row norm is at most sqrt(128) times the
+// largest entry, so stored states stay below 2^48 and the read-out's sum of
+// squares of o = W_t q' (|q'| = 1, below 2^111) cannot overflow.  Its RMSNorm is scale-free up to eps,
+// which is scaled by 2^(-2e) accordingly.
+constexpr float kRenormAbove = 4294967296.0f;               // 2^32
+constexpr float kRenormScale = 2.3283064365386963e-10f;    // 2^-32
+constexpr int kRenormExp = 32;
 
 // ---------------------------------------------------------------- device status word
 // Written only by bounded waits that gave up; read by vdn_workspace_status().

@@ -541,20 +541,23 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
   }
 }
 
-// d = 128, one CTA per (batch, head, window chunk): every query frame of a chunk
-// has the same window [lo, hi], hence the same two boundary states; they are
-// read once and each frame's W_t differs only in its two decay vectors.
+// d = 128: one CTA per (batch, head, window chunk, block of 32 rows).  Every
+// query frame of a chunk has the same window [lo, hi], hence the same two
+// boundary states; their rows are read once and each frame's W_t differs only
+// in its two decay vectors.  The sides are aligned to the larger block exponent
+// (stored states are below 2^48, see the scans' block exponent), W_t is stored as 2^-e W_t.
 constexpr int kGatherMaxChunk = 16;
+constexpr int kGatherRows = 32;
 
-__global__ void __launch_bounds__(512) k_gather128_chunk(const float* __restrict__ P, const float* __restrict__ Q,
+__global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict__ P, const float* __restrict__ Q,
                                                          const int* __restrict__ pexp, const int* __restrict__ qexp,
                                                          const float* __restrict__ alpha,
                                                          const float* __restrict__ text, int H, int F, int chunk,
                                                          int radius, float* __restrict__ W,
                                                          uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
   constexpr int D = 128;
-  __shared__ float dpre[kGatherMaxChunk][D], dsuf[kGatherMaxChunk][D], red[2][16];
-  const int tid = threadIdx.x, n = tid >> 2, k0 = (tid & 3) * 32;
+  __shared__ float dpre[kGatherMaxChunk][D], dsuf[kGatherMaxChunk][D];
+  const int tid = threadIdx.x, n = blockIdx.z * kGatherRows + (tid >> 2), k0 = (tid & 3) * 32;
   const long long bh = blockIdx.x;
   const int h = (int)(bh % H);
   const long long b = bh / H;
@@ -572,8 +575,8 @@ __global__ void __launch_bounds__(512) k_gather128_chunk(const float* __restrict
     pv[j] = pre ? *reinterpret_cast<const float4*>(pre + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
     sv[j] = suf ? *reinterpret_cast<const float4*>(suf + off) : (seed ? *reinterpret_cast<const float4*>(seed + off) : z);
   }
-  if (tid < D) {
-    // dpre[t] = prod_{g=lo..t} alpha_g,  dsuf[t] = prod_{g=t..hi} alpha_g
+  {
+    // dpre[t] = prod_{g=lo..t} alpha_g,  dsuf[t] = prod_{g=t..hi} alpha_g  (one channel per thread)
     const float* al = alpha + (b * F * H + h) * D + tid;
     float dp = 1.f;
     for (int g = lo; g < t0; ++g) dp *= al[(long long)g * H * D];
@@ -602,32 +605,19 @@ __global__ void __launch_bounds__(512) k_gather128_chunk(const float* __restrict
   for (int t = t0; t < t1; ++t) {
     const float* dp = dpre[t - t0];
     const float* ds = dsuf[t - t0];
+    const long long fi = bh * F + t;
+    if (tid == 0 && blockIdx.z == 0) wexp[fi] = ew;
     float w[32];
-    float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int k = k0 + 4 * j;
-      w[4 * j + 0] = fmaf(pv[j].x, dp[k + 0], sv[j].x * ds[k + 0]);
-      w[4 * j + 1] = fmaf(pv[j].y, dp[k + 1], sv[j].y * ds[k + 1]);
-      w[4 * j + 2] = fmaf(pv[j].z, dp[k + 2], sv[j].z * ds[k + 2]);
-      w[4 * j + 3] = fmaf(pv[j].w, dp[k + 3], sv[j].w * ds[k + 3]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(w[4 * j + u]));
+      const float4 a = *reinterpret_cast<const float4*>(dp + k);
+      const float4 c = *reinterpret_cast<const float4*>(ds + k);
+      w[4 * j + 0] = fmaf(pv[j].x, a.x, sv[j].x * c.x);
+      w[4 * j + 1] = fmaf(pv[j].y, a.y, sv[j].y * c.y);
+      w[4 * j + 2] = fmaf(pv[j].z, a.z, sv[j].z * c.z);
+      w[4 * j + 3] = fmaf(pv[j].w, a.w, sv[j].w * c.w);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    float* rd = red[t & 1];   // double buffer: one barrier per frame
-    if ((tid & 31) == 0) rd[tid >> 5] = amax;
-    __syncthreads();
-    amax = rd[0];
-#pragma unroll
-    for (int u = 1; u < 16; ++u) amax = fmaxf(amax, rd[u]);
-    int ek = 0;
-    if (amax > 0.f) frexpf(amax, &ek);
-    const long long fi = bh * F + t;
-    if (tid == 0) wexp[fi] = ew + ek;
-#pragma unroll
-    for (int u = 0; u < 32; ++u) w[u] = ldexpf(w[u], -ek);
     if (W) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -658,8 +648,8 @@ __global__ void __launch_bounds__(512) k_gather128_chunk(const float* __restrict
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
                           uint16_t* wimg, int* wexp) {
   if (a.sh.d == 128 && a.chunk <= kGatherMaxChunk) {
-    dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((a.sh.F + a.chunk - 1) / a.chunk));
-    k_gather128_chunk<<<grid, 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
+    dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((a.sh.F + a.chunk - 1) / a.chunk), 128 / kGatherRows);
+    k_gather128_chunk<<<grid, 128, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
                                                    a.radius, W, wimg, wexp);
     return cudaGetLastError();
   }
