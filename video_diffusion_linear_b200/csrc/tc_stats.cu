@@ -8,20 +8,22 @@
 // applied once, while the operands are produced, and no operand is written
 // twice.  The k/v feature prep of Step 1 (short conv within the frame, SiLU,
 // L2 normalisation of k) is fused into that operand production: raw bf16 rows
-// arrive by TMA (64 tokens plus one halo row on each side, zero outside the
+// arrive by TMA (96 tokens plus one halo row on each side, zero outside the
 // frame), the transform warps compute X and Y in fp32 and store them as bf16 in
-// the MN-major 128-byte-swizzled layout the tensor cores read.
+// the MN-major 128-byte-swizzled layout the tensor cores read.  Y needs no
+// reduction across threads, so it is computed first and stored as soon as the
+// tensor cores release the operand buffer; X follows once the norms of k are
+// known.
 //
-// Work split: the (frame, 64-token block) pairs, frames ordered (batch, frame,
+// Work split: the (frame, 96-token block) pairs, frames ordered (batch, frame,
 // head), are cut into gridDim.x contiguous ranges (stream-K).  A CTA flushes its
 // accumulator whenever its range leaves a frame, into partial slot
 // (blockIdx.x + frame); the per-frame solve adds the slots of each frame in a
 // fixed order, so the result is deterministic.
 //
 // Warp roles (448 threads): 0 TMA producer, 1 MMA issuer (TMEM owner),
-// 2-13 transform (4 tokens x 8 channels per thread, 96-token blocks); transform
-// warps 2-5 (one per TMEM lane quarter) also flush the accumulator when a
-// frame segment ends.
+// 2-13 transform (4 tokens x 8 channels per thread); transform warps 2-5 (one
+// per TMEM lane quarter) also flush the accumulator when a frame segment ends.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -31,25 +33,29 @@ namespace vdn {
 
 namespace {
 
-constexpr int kRS = 3;                 // raw TMA stages
-constexpr int kRawRows = kStatsTokens + 2;
-constexpr int kRawHalf = 13312;        // 98 rows x 128 B, padded to 13 KB (1024-aligned)
-constexpr int kRawBytes = 4 * kRawRows * 128;   // k and v, two channel halves each
-constexpr int kTransformWarps = 12;    // 8 tokens each
+constexpr int kTPT = 4;                               // tokens per transform thread
+constexpr int kTransformWarps = 12;
+constexpr int kBT = 2 * kTPT * kTransformWarps;       // tokens per block
+static_assert(kBT == kStatsTokens, "block size");
+static_assert(kBT % 32 == 0, "block size");
+constexpr int kRS = 3;                                // raw TMA stages
+constexpr int kOS = 1;                                // operand stages
+constexpr int kRawRows = kBT + 2;
+constexpr int kRawHalf = (kRawRows * 128 + 1023) / 1024 * 1024;
+constexpr int kRawBytes = 4 * kRawRows * 128;         // k and v, two channel halves each
 constexpr int kTransformThreads = 32 * kTransformWarps;
 constexpr int kThreads = 64 + kTransformThreads;
-constexpr int kKAtoms = kStatsTokens / 8;       // 8-token swizzle atoms along K
-constexpr int kOpHalf = kKAtoms * 2048;         // X (or Y): 128 channels x kStatsTokens bf16
-constexpr int kMnAtomStride = kKAtoms * 1024;   // descriptor leading offset: next 64 channels
+constexpr int kKAtoms = kBT / 8;                      // 8-token swizzle atoms along K
+constexpr int kOpHalf = kKAtoms * 2048;               // X (or Y): 128 channels x kBT bf16
+constexpr int kMnAtomStride = kKAtoms * 1024;         // descriptor leading offset: next 64 channels
 
 struct __align__(1024) StatsSmem {
   uint8_t raw[kRS][2][2][kRawHalf];    // [stage][k|v][channel half]
-  uint8_t op[2 * kOpHalf];             // X | Y, MN-major SW128; one stage: the transform
-                                       // computes block i+1 while the MMA reads block i
-  float taps[kRS][2][3][128];          // [stage][k|v][tap][channel] conv taps of the stage's head
-  float sqb[kRS][kStatsTokens];        // [stage][token] sqrt(beta), 0 past the frame end
+  uint8_t op[kOS][2 * kOpHalf];        // X | Y, MN-major SW128
+  float taps[kRS][2][3][128];          // [stage][k|v][tap][channel] conv taps / 2 of the stage's head
+  float sqb[kRS][kBT];                 // [stage][token] sqrt(beta), 0 past the frame end
   uint64_t raw_full[kRS], raw_empty[kRS];
-  uint64_t op_full, op_empty;
+  uint64_t op_full[kOS], op_empty[kOS];
   uint64_t acc_full[2], acc_empty[2];
   uint32_t tmem_base;
   int abort;
@@ -58,8 +64,8 @@ struct __align__(1024) StatsSmem {
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 256, true, true);
 
 // byte offset of the 16-byte chunk holding channels 8c..8c+7 of token t in an
-// MN-major SW128 operand of 128 channels x kStatsTokens tokens (atoms of
-// 64 channels x 8 tokens, 1 KB each; K atoms contiguous, channel halves apart)
+// MN-major SW128 operand of 128 channels x kBT tokens (atoms of 64 channels x
+// 8 tokens, 1 KB each; K atoms contiguous, channel halves kMnAtomStride apart)
 __device__ __forceinline__ uint32_t op_chunk(int c, int t) {
   return (c >> 3) * kMnAtomStride + (t >> 3) * 1024 + (t & 7) * 128 + ((((c & 7) ^ (t & 7))) << 4);
 }
@@ -82,10 +88,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < kRS; ++s) {
       tc::mbar_init(&sm.raw_full[s], 1);
-      tc::mbar_init(&sm.raw_empty[s], kTransformThreads);
+      tc::mbar_init(&sm.raw_empty[s], kTransformWarps);
     }
-    tc::mbar_init(&sm.op_full, kTransformThreads);
-    tc::mbar_init(&sm.op_empty, 1);
+    for (int s = 0; s < kOS; ++s) {
+      tc::mbar_init(&sm.op_full[s], kTransformWarps);
+      tc::mbar_init(&sm.op_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&sm.acc_full[s], 1);
       tc::mbar_init(&sm.acc_empty[s], 128);
@@ -102,10 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  // block x -> frame pf (order b, f, h) and block j in the frame
   auto decode = [&](long long x, int& h, int& fb, int& s0) {
     long long pf = x / nb;
-    s0 = (int)(x % nb) * kStatsTokens;
+    s0 = (int)(x % nb) * kBT;
     h = (int)(pf % H);
     fb = (int)(pf / H);   // b * F + f
   };
@@ -115,13 +122,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     // ------------------------------------------------------------ producer (whole warp)
     // lane 0 issues the TMA copies; all lanes stage sqrt(beta) of the block's
     // tokens and, when the stage's head changes, the conv taps of that head.
+    // beta of the next block is loaded one iteration ahead, so its latency
+    // overlaps the wait for a free stage.
     const long long N = (long long)F * S;
     int slot_head[kRS];
 #pragma unroll
     for (int r = 0; r < kRS; ++r) slot_head[r] = -1;
-    // beta of the next block is loaded one iteration ahead, so its latency
-    // overlaps the wait for a free stage instead of delaying the next TMA issue
-    constexpr int BU = kStatsTokens / 32;
+    constexpr int BU = kBT / 32;
     float bnext[BU];
     auto load_beta = [&](long long x) {
       int h, fb, s0;
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           if (!wg) val = tap == 1 ? 1.f : 0.f;                       // identity
           else if (K == 3) val = wg[((long long)h * 128 + ch) * 3 + tap];
           else val = tap == 1 ? wg[(long long)h * 128 + ch] : 0.f;   // one tap: centre
-          sm.taps[rs][ten][tap][ch] = val;
+          sm.taps[rs][ten][tap][ch] = 0.5f * val;
         }
 #pragma unroll
         for (int r = 0; r < kRS; ++r)
@@ -177,21 +184,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       int it = 0, seg = 0;
       bool first = true;
       for (long long x = x0; x < x1; ++x, ++it) {
-        const uint32_t oph = it & 1;
+        const int os = it % kOS;
+        const uint32_t oph = (it / kOS) & 1;
         const int ab = seg & 1;
         if (first) {
           if (!tc::mbar_wait(&sm.acc_empty[ab], ((seg >> 1) & 1) ^ 1, abort_flag, status)) break;
         }
-        if (!tc::mbar_wait(&sm.op_full, oph, abort_flag, status)) break;
+        if (!tc::mbar_wait(&sm.op_full[os], oph, abort_flag, status)) break;
         tc::tc_fence_after();
         const uint32_t d = tmem + ab * 256;
-        const uint32_t base = tc::smem_u32(sm.op);
+        const uint32_t base = tc::smem_u32(sm.op[os]);
 #pragma unroll
-        for (int kk = 0; kk < kStatsTokens / 16; ++kk) {
+        for (int kk = 0; kk < kBT / 16; ++kk) {
           uint64_t desc = tc::smem_desc(base + kk * 2048, kMnAtomStride, 1024);
           tc::umma_bf16(d, desc, desc, kIdesc, (first && kk == 0) ? 0u : 1u);
         }
-        tc::umma_commit(&sm.op_empty);
+        tc::umma_commit(&sm.op_empty[os]);
         first = false;
         if (seg_last(x)) {
           tc::umma_commit(&sm.acc_full[ab]);
@@ -203,38 +211,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   } else {
     // ------------------------------------------------------------ transform (+ flush)
     const int tt = tid - 64;
-    const int w12 = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
+    const int w = tt >> 5, tg = (tt >> 4) & 1, c = tt & 15;
     const int half = c >> 3, cc = c & 7;
-    const int tok0 = 8 * w12 + 4 * tg;      // first of this thread's 4 tokens in the block
-    const bool flusher = w12 < 4;           // warps 2-5: TMEM lane quarters 2, 3, 0, 1
+    const int tok0 = 2 * kTPT * w + kTPT * tg;   // first of this thread's kTPT tokens in the block
+    const bool flusher = w < 4;                  // warps 2-5: TMEM lane quarters 2, 3, 0, 1
     const int quarter = warp & 3;
     int seg = 0;
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
       const int rs = it % kRS;
       const uint32_t rph = (it / kRS) & 1;
-      const uint32_t oph = it & 1;
+      const int os = it % kOS;
+      const uint32_t oph = (it / kOS) & 1;
       if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
-      float sb[4];
+      float sb[kTPT];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sb[i] = sm.sqb[rs][tok0 + i];
+      for (int i = 0; i < kTPT; ++i) sb[i] = sm.sqb[rs][tok0 + i];
 
-      // conv (3 taps, packed pairs of channels), SiLU; k also sums its squares.
-      // Written stage by stage (all convolutions, then all tanh, then the
-      // combination) so the 16 independent chains issue back to back.
-      auto conv_silu = [&](int ten, float2 (&outp)[4][4], float (&ss)[4]) {
-        float2 w[3][4];
+      // y = SiLU(conv(x)) = h + h tanh(h), h = conv(x) / 2 (the taps carry the 1/2);
+      // ss = sum of y^2 over this thread's channels
+      auto conv_silu = [&](int ten, float2 (&y)[kTPT][4], float (&ss)[kTPT]) {
+        float2 w3[3][4];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
           const float4 a = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c]);
           const float4 b = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c + 4]);
-          w[j][0] = make_float2(a.x, a.y); w[j][1] = make_float2(a.z, a.w);
-          w[j][2] = make_float2(b.x, b.y); w[j][3] = make_float2(b.z, b.w);
+          w3[j][0] = make_float2(a.x, a.y); w3[j][1] = make_float2(a.z, a.w);
+          w3[j][2] = make_float2(b.x, b.y); w3[j][3] = make_float2(b.z, b.w);
         }
-        float2 r[6][4];
+        float2 r[kTPT + 2][4];
         const uint8_t* src = sm.raw[rs][ten][half];
 #pragma unroll
-        for (int rr = 0; rr < 6; ++rr) {
+        for (int rr = 0; rr < kTPT + 2; ++rr) {
           const int row = tok0 + rr;
           const uint4 q = *reinterpret_cast<const uint4*>(src + row * 128 + ((cc ^ (row & 7)) << 4));
           r[rr][0] = make_float2(bf16lo(q.x), bf16hi(q.x));
@@ -242,67 +250,67 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           r[rr][2] = make_float2(bf16lo(q.z), bf16hi(q.z));
           r[rr][3] = make_float2(bf16lo(q.w), bf16hi(q.w));
         }
-        float2 hx[4][4];
+        float2 hx[kTPT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < kTPT; ++i)
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            float2 a = __fmul2_rn(w[2][p], r[i + 2][p]);
-            a = __ffma2_rn(w[1][p], r[i + 1][p], a);
-            a = __ffma2_rn(w[0][p], r[i][p], a);
-            hx[i][p] = __fmul2_rn(a, make_float2(0.5f, 0.5f));
+            float2 a = __fmul2_rn(w3[2][p], r[i + 2][p]);
+            a = __ffma2_rn(w3[1][p], r[i + 1][p], a);
+            hx[i][p] = __ffma2_rn(w3[0][p], r[i][p], a);
           }
-        float2 th[4][4];
+        float2 th[kTPT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < kTPT; ++i)
 #pragma unroll
           for (int p = 0; p < 4; ++p) th[i][p] = tanh2(hx[i][p]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kTPT; ++i) {
           float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            const float2 y = __ffma2_rn(hx[i][p], th[i][p], hx[i][p]);   // x sigmoid(x) = h + h tanh(h)
-            outp[i][p] = y;
-            acc = __ffma2_rn(y, y, acc);
+            y[i][p] = __ffma2_rn(hx[i][p], th[i][p], hx[i][p]);
+            acc = __ffma2_rn(y[i][p], y[i][p], acc);
           }
           ss[i] = acc.x + acc.y;
         }
       };
+      auto store = [&](const float2 (&y)[kTPT][4], const float (&scale)[kTPT], uint8_t* dst) {
+#pragma unroll
+        for (int i = 0; i < kTPT; ++i) {
+          const float2 s2 = make_float2(scale[i], scale[i]);
+          uint32_t wv[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 a = __fmul2_rn(y[i][p], s2);
+            wv[p] = pack_bf16x2(a.x, a.y);
+          }
+          *reinterpret_cast<uint4*>(dst + op_chunk(c, tok0 + i)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      };
 
-      float2 kx[4][4], vx[4][4];
-      float ssq[4], unused[4];
-      conv_silu(0, kx, ssq);
-      // the k row sums travel through the 16 lanes of the token group while v is computed
+      {
+        float2 vy[kTPT][4];
+        float unused[kTPT];
+        conv_silu(1, vy, unused);
+        if (!tc::mbar_wait(&sm.op_empty[os], oph ^ 1, abort_flag, status)) break;
+        store(vy, sb, sm.op[os] + kOpHalf);      // Y = sqrt(beta) v'
+      }
+      float2 ky[kTPT][4];
+      float ssq[kTPT];
+      conv_silu(0, ky, ssq);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.raw_empty[rs]);      // one arrival per warp
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], 1);
-      conv_silu(1, vx, unused);
-      tc::mbar_arrive(&sm.raw_empty[rs]);
+      for (int i = 0; i < kTPT; ++i) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int o = 2; o < 16; o <<= 1) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], o);
+        for (int o = 1; o < 16; o <<= 1) ssq[i] += __shfl_xor_sync(0xffffffffu, ssq[i], o);
         ssq[i] = sb[i] * rsqrtf(ssq[i] + kL2Eps);
       }
-      if (!tc::mbar_wait(&sm.op_empty, oph ^ 1, abort_flag, status)) break;
-      uint8_t* dst = sm.op;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = tok0 + i;
-        const float2 sk = make_float2(ssq[i], ssq[i]), sv = make_float2(sb[i], sb[i]);
-        uint32_t wxv[4], wyv[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 a = __fmul2_rn(kx[i][p], sk);
-          const float2 b = __fmul2_rn(vx[i][p], sv);
-          wxv[p] = pack_bf16x2(a.x, a.y);
-          wyv[p] = pack_bf16x2(b.x, b.y);
-        }
-        *reinterpret_cast<uint4*>(dst + op_chunk(c, t)) = make_uint4(wxv[0], wxv[1], wxv[2], wxv[3]);
-        *reinterpret_cast<uint4*>(dst + kOpHalf + op_chunk(c, t)) = make_uint4(wyv[0], wyv[1], wyv[2], wyv[3]);
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&sm.op_full);
+      store(ky, ssq, sm.op[os]);                  // X = sqrt(beta) k'
+      tc::fence_proxy_async_smem();   // each thread's stores, then one arrival per warp
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.op_full[os]);
       if (flusher && seg_last(x)) {
         // the segment of this frame is complete once its last block's MMA is:
         // copy the [A | B^T] accumulator rows to partial slot (blockIdx.x + frame)
