@@ -163,85 +163,143 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
   }
 }
 
-// d = 128 solve.  Thread (ty, tx) owns the 8x8 block rows 8 ty.., columns 8 tx..
-// (contiguous, so pivot row and column segments are two 16-byte loads), the
-// elimination update runs on packed fp32 pairs, and the pivot reciprocal is
-// the hardware approximation refined by one Newton step (relative error near
-// 2^-23, the same as a correctly rounded division up to one unit).
-__global__ void __launch_bounds__(256, 2) k_solve128(const float* __restrict__ part, long long Tblocks, int nb, int G,
-                                                     RuleCoef rc, float* __restrict__ Nm, uint16_t* __restrict__ nimg,
-                                                     float* __restrict__ Bsum, float* __restrict__ Aout, int H, int F) {
-  constexpr int D = 128, LD = D + 4;   // +4 keeps rows 16-byte aligned
-  extern __shared__ float sm[];
-  float* stage = sm;                   // [D][LD]
-  float* colv = sm + D * LD;           // [2][D]
-  float* rowv = colv + 2 * D;          // [2][D]
+// d = 128 solve by the symmetric sweep operator.  N_f^-1 = I + c^2 A_f is
+// symmetric positive definite; sweeping pivot k (d = a_kk):
+//   a_ij <- a_ij - a_ik a_kj / d   (i, j != k),   a_ik, a_kj <- a_ik / d, a_kj / d,   a_kk <- -1 / d
+// keeps the matrix symmetric, and sweeping every pivot in turn leaves -M^-1
+// (Gauss-Jordan elimination without pivoting, with every pivot a Schur
+// complement of an SPD matrix, so positive).  Symmetry halves the work: the
+// 136 threads that own the upper-triangle 8x8 blocks (I <= J) of a 16 x 16 block
+// grid do all of it, one pivot per barrier, with pivot row k broadcast through
+// shared memory (its entries left of the diagonal block come from column k of
+// the blocks above it).  Updates run on packed fp32 pairs; the pivot reciprocal
+// is the hardware approximation refined by one Newton step (relative error near
+// 2^-23, the same as a correctly rounded division up to one unit).  Three frames
+// share an SM.  The scan's operand image and the debug copies are written from
+// the blocks directly, each off-diagonal block once as itself and once
+// transposed.
+constexpr int kSolveThreads = 160;     // 136 block owners + 24 that only help with the sums
+constexpr int kSolveBlocks = 136;      // 16 * 17 / 2
+
+__device__ __forceinline__ void store_chunk_image(uint8_t* img, int n, int c, const float (&v)[8]) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(v[e], h0, l0);
+    split_bf16(v[e + 1], h1, l1);
+    hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+    lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+  }
+  const uint32_t off = img_offset(0, n, 8 * c);
+  *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+__global__ void __launch_bounds__(kSolveThreads, 3) k_solve128(const float* __restrict__ part, long long Tblocks,
+                                                              int nb, int G, RuleCoef rc, float* __restrict__ Nm,
+                                                              uint16_t* __restrict__ nimg, float* __restrict__ Bsum,
+                                                              float* __restrict__ Aout, int H, int F) {
+  constexpr int D = 128;
+  __shared__ __align__(16) float rowv[2][D];      // pivot row, double-buffered
   const long long fi = blockIdx.x;
   const int f = (int)(fi % F);
   const long long bh = fi / F;
   const int h = (int)(bh % H);
   const long long b = bh / H;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int r0 = 8 * ty, c0 = 8 * tx;
+  const int tid = threadIdx.x;
+  const bool owner = tid < kSolveBlocks;
+  // block (I, J), I <= J, row-major over the upper triangle
+  int I = 0, J = 0;
+  {
+    int t = owner ? tid : 0;
+    while (t >= 16 - I) { t -= 16 - I; ++I; }
+    J = I + t;
+  }
+  const int r0 = 8 * I, c0 = 8 * J;
   float2 a[8][4];                      // a[i][p] = (A[r0+i][c0+2p], A[r0+i][c0+2p+1])
 
-  // sum the [A | B^T] partial rows of this frame's statistics slots
+  const long long pf = ((long long)b * F + f) * H + h;
+  const long long x0 = pf * nb, x1 = x0 + nb - 1;
+  const int i0 = sk_owner(x0, Tblocks, G), i1 = sk_owner(x1, Tblocks, G);
+
+  // ---- B = (B^T)^T: 4 x 8 pieces of B^T, summed and written transposed
   {
-    const long long pf = ((long long)b * F + f) * H + h;
-    const long long x0 = pf * nb, x1 = x0 + nb - 1;
-    const int i0 = sk_owner(x0, Tblocks, G), i1 = sk_owner(x1, Tblocks, G);
+    float* Bf = Bsum + fi * D * D;
+    for (int q = tid; q < 512; q += kSolveThreads) {
+      const int ib = q >> 5, jb = (q >> 1) & 15, hf = q & 1;   // B rows 8 ib.., B columns 8 jb + 4 hf ..
+      float acc[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int p = 0; p < 4; ++p) a[i][p] = make_float2(0.f, 0.f);
-    for (int e = tid; e < D * D / 4; e += 256) *reinterpret_cast<float4*>(stage + (e / 32) * LD + 4 * (e % 32)) = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int ci = i0; ci <= i1; ++ci) {
-      const float* pp = part + (long long)(ci + pf) * (D * 2 * D);
-      float4 av[8][2];
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+      for (int ci = i0; ci <= i1; ++ci) {
+        const float* pp = part + (long long)(ci + pf) * (D * 2 * D) + (8 * jb + 4 * hf) * (2 * D) + D + 8 * ib;
+        float4 v[4][2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        av[i][0] = *reinterpret_cast<const float4*>(pp + (r0 + i) * (2 * D) + c0);
-        av[i][1] = *reinterpret_cast<const float4*>(pp + (r0 + i) * (2 * D) + c0 + 4);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        a[i][0] = __fadd2_rn(a[i][0], make_float2(av[i][0].x, av[i][0].y));
-        a[i][1] = __fadd2_rn(a[i][1], make_float2(av[i][0].z, av[i][0].w));
-        a[i][2] = __fadd2_rn(a[i][2], make_float2(av[i][1].x, av[i][1].y));
-        a[i][3] = __fadd2_rn(a[i][3], make_float2(av[i][1].z, av[i][1].w));
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float4 bv[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int e4 = tid + 256 * (8 * half + r), row = e4 / 32, c4 = e4 % 32;
-          bv[r] = *reinterpret_cast<const float4*>(pp + row * (2 * D) + D + 4 * c4);
+        for (int r = 0; r < 4; ++r) {
+          v[r][0] = *reinterpret_cast<const float4*>(pp + r * (2 * D));
+          v[r][1] = *reinterpret_cast<const float4*>(pp + r * (2 * D) + 4);
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int e4 = tid + 256 * (8 * half + r), row = e4 / 32, c4 = e4 % 32;
-          float4* st = reinterpret_cast<float4*>(stage + row * LD + 4 * c4);
-          float4 v = *st;
-          v.x += bv[r].x; v.y += bv[r].y; v.z += bv[r].z; v.w += bv[r].w;
-          *st = v;
+        for (int r = 0; r < 4; ++r) {
+          acc[r][0] += v[r][0].x; acc[r][1] += v[r][0].y; acc[r][2] += v[r][0].z; acc[r][3] += v[r][0].w;
+          acc[r][4] += v[r][1].x; acc[r][5] += v[r][1].y; acc[r][6] += v[r][1].z; acc[r][7] += v[r][1].w;
         }
       }
-    }
-    __syncthreads();
-    float* Bf = Bsum + fi * D * D;     // B[i][j] = (B^T)[j][i]
-    for (int e = tid; e < D * D; e += 256) Bf[e] = stage[(e % D) * LD + (e / D)];
-    if (Aout) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          *reinterpret_cast<float2*>(Aout + fi * D * D + (r0 + i) * D + c0 + 2 * p) = a[i][p];
+      for (int c = 0; c < 8; ++c)   // B[8 ib + c][8 jb + 4 hf + r] = B^T[8 jb + 4 hf + r][8 ib + c]
+        *reinterpret_cast<float4*>(Bf + (8 * ib + c) * D + 8 * jb + 4 * hf) =
+            make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
     }
-    __syncthreads();
   }
 
-  // N = I + c^2 A (solve rules), I - c^2 A (sana) or I (additive)
+  // ---- A: sum this block of the [A | B^T] partial slots of the frame
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int p = 0; p < 4; ++p) a[i][p] = make_float2(0.f, 0.f);
+  if (owner) {
+    for (int ci = i0; ci <= i1; ++ci) {
+      const float* pp = part + (long long)(ci + pf) * (D * 2 * D) + r0 * (2 * D) + c0;
+#pragma unroll
+      for (int ih = 0; ih < 8; ih += 4) {   // four rows (8 float4) in flight
+        float4 v[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[i][0] = *reinterpret_cast<const float4*>(pp + (ih + i) * (2 * D));
+          v[i][1] = *reinterpret_cast<const float4*>(pp + (ih + i) * (2 * D) + 4);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[ih + i][0] = __fadd2_rn(a[ih + i][0], make_float2(v[i][0].x, v[i][0].y));
+          a[ih + i][1] = __fadd2_rn(a[ih + i][1], make_float2(v[i][0].z, v[i][0].w));
+          a[ih + i][2] = __fadd2_rn(a[ih + i][2], make_float2(v[i][1].x, v[i][1].y));
+          a[ih + i][3] = __fadd2_rn(a[ih + i][3], make_float2(v[i][1].z, v[i][1].w));
+        }
+      }
+    }
+    if (Aout) {
+      float* Af = Aout + fi * D * D;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        *reinterpret_cast<float4*>(Af + (r0 + i) * D + c0) = make_float4(a[i][0].x, a[i][0].y, a[i][1].x, a[i][1].y);
+        *reinterpret_cast<float4*>(Af + (r0 + i) * D + c0 + 4) = make_float4(a[i][2].x, a[i][2].y, a[i][3].x, a[i][3].y);
+      }
+      if (I != J) {   // the mirror block
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          float cvv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cvv[i] = (m & 1) ? a[i][m >> 1].y : a[i][m >> 1].x;
+          *reinterpret_cast<float4*>(Af + (c0 + m) * D + r0) = make_float4(cvv[0], cvv[1], cvv[2], cvv[3]);
+          *reinterpret_cast<float4*>(Af + (c0 + m) * D + r0 + 4) = make_float4(cvv[4], cvv[5], cvv[6], cvv[7]);
+        }
+      }
+    }
+  }
+
+  // ---- N^-1 = I + c^2 A (solve rules); N = I - c^2 A (sana) or I (additive)
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -251,79 +309,90 @@ __global__ void __launch_bounds__(256, 2) k_solve128(const float* __restrict__ p
       a[i][p] = rc.identity ? make_float2(d0, d1) : make_float2(fmaf(s, a[i][p].x, d0), fmaf(s, a[i][p].y, d1));
     }
 
+  float sign = 1.f;
   if (rc.solve) {
-    // in-place Gauss-Jordan; pivot j = 8 jt + jj
-    for (int jt = 0; jt < 16; ++jt) {
+    sign = -1.f;                       // the sweep leaves -N
+    for (int K = 0; K < 16; ++K) {
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int j = 8 * jt + jj;
-        float* cv = colv + (j & 1) * D;
-        float* rv = rowv + (j & 1) * D;
-        if (tx == jt) {   // column j segment: rows r0..r0+7
-          float col[8];
+      for (int kk = 0; kk < 8; ++kk) {
+        const int k = 8 * K + kk;
+        float* rv = rowv[kk & 1];
+        if (owner && I == K) {         // row kk of the blocks right of (and at) the diagonal
+          *reinterpret_cast<float4*>(rv + c0) = make_float4(a[kk][0].x, a[kk][0].y, a[kk][1].x, a[kk][1].y);
+          *reinterpret_cast<float4*>(rv + c0 + 4) = make_float4(a[kk][2].x, a[kk][2].y, a[kk][3].x, a[kk][3].y);
+        } else if (owner && J == K) {  // column kk of the blocks above the diagonal (a_ik = a_ki)
+          float cvv[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) col[i] = (jj & 1) ? a[i][jj >> 1].y : a[i][jj >> 1].x;
-          *reinterpret_cast<float4*>(cv + r0) = make_float4(col[0], col[1], col[2], col[3]);
-          *reinterpret_cast<float4*>(cv + r0 + 4) = make_float4(col[4], col[5], col[6], col[7]);
-        }
-        if (ty == jt) {   // row j segment: columns c0..c0+7
-          *reinterpret_cast<float4*>(rv + c0) = make_float4(a[jj][0].x, a[jj][0].y, a[jj][1].x, a[jj][1].y);
-          *reinterpret_cast<float4*>(rv + c0 + 4) = make_float4(a[jj][2].x, a[jj][2].y, a[jj][3].x, a[jj][3].y);
+          for (int i = 0; i < 8; ++i) cvv[i] = (kk & 1) ? a[i][kk >> 1].y : a[i][kk >> 1].x;
+          *reinterpret_cast<float4*>(rv + r0) = make_float4(cvv[0], cvv[1], cvv[2], cvv[3]);
+          *reinterpret_cast<float4*>(rv + r0 + 4) = make_float4(cvv[4], cvv[5], cvv[6], cvv[7]);
         }
         __syncthreads();
-        const float pv = cv[j];
-        float r;
-        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(pv));
-        r = r * fmaf(-pv, r, 2.0f);                       // one Newton step
-        const float4 ca = *reinterpret_cast<const float4*>(cv + r0);
-        const float4 cb = *reinterpret_cast<const float4*>(cv + r0 + 4);
-        const float4 ra = *reinterpret_cast<const float4*>(rv + c0);
-        const float4 rb = *reinterpret_cast<const float4*>(rv + c0 + 4);
-        const float cr[8] = {ca.x * r, ca.y * r, ca.z * r, ca.w * r, cb.x * r, cb.y * r, cb.z * r, cb.w * r};
-        const float2 rk[4] = {make_float2(ra.x, ra.y), make_float2(ra.z, ra.w), make_float2(rb.x, rb.y),
-                              make_float2(rb.z, rb.w)};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 m = make_float2(-cr[i], -cr[i]);
-#pragma unroll
-          for (int p = 0; p < 4; ++p) a[i][p] = __ffma2_rn(m, rk[p], a[i][p]);
-        }
-        if (ty == jt) {   // row j: A[j][k] / p
-#pragma unroll
-          for (int p = 0; p < 4; ++p) a[jj][p] = make_float2(rk[p].x * r, rk[p].y * r);
-        }
-        if (tx == jt) {   // column j: -A[i][j] / p
+        if (owner) {
+          const float pv = rv[k];
+          float r;
+          asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(pv));
+          r = r * fmaf(-pv, r, 2.0f);                   // one Newton step
+          const float4 ra = *reinterpret_cast<const float4*>(rv + r0);
+          const float4 rb = *reinterpret_cast<const float4*>(rv + r0 + 4);
+          const float4 ca = *reinterpret_cast<const float4*>(rv + c0);
+          const float4 cb = *reinterpret_cast<const float4*>(rv + c0 + 4);
+          const float cr[8] = {ra.x * r, ra.y * r, ra.z * r, ra.w * r, rb.x * r, rb.y * r, rb.z * r, rb.w * r};
+          const float2 rk[4] = {make_float2(ca.x, ca.y), make_float2(ca.z, ca.w), make_float2(cb.x, cb.y),
+                                make_float2(cb.z, cb.w)};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            if (jj & 1) a[i][jj >> 1].y = -cr[i];
-            else a[i][jj >> 1].x = -cr[i];
+            const float2 m = make_float2(-cr[i], -cr[i]);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) a[i][p] = __ffma2_rn(m, rk[p], a[i][p]);
           }
-        }
-        if (ty == jt && tx == jt) {
-          if (jj & 1) a[jj][jj >> 1].y = r;
-          else a[jj][jj >> 1].x = r;
+          if (I == K) {                // row k: a_kj / d
+#pragma unroll
+            for (int p = 0; p < 4; ++p) a[kk][p] = make_float2(rk[p].x * r, rk[p].y * r);
+          }
+          if (J == K) {                // column k: a_ik / d
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              if (kk & 1) a[i][kk >> 1].y = cr[i];
+              else a[i][kk >> 1].x = cr[i];
+            }
+          }
+          if (I == K && J == K) {
+            if (kk & 1) a[kk][kk >> 1].y = -r;
+            else a[kk][kk >> 1].x = -r;
+          }
         }
       }
     }
   }
 
-  if (Nm) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int p = 0; p < 4; ++p) *reinterpret_cast<float2*>(Nm + fi * D * D + (r0 + i) * D + c0 + 2 * p) = a[i][p];
-  }
-  if (nimg) {
+  if (owner) {
+    uint8_t* img = nimg ? reinterpret_cast<uint8_t*>(nimg + fi * (kImgBytes / 2)) : nullptr;
+    float* Nf = Nm ? Nm + fi * D * D : nullptr;
+    // B operand image of the scan: row n holds N_f[n][k] (N_f symmetric)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      *reinterpret_cast<float4*>(stage + (r0 + i) * LD + c0) = make_float4(a[i][0].x, a[i][0].y, a[i][1].x, a[i][1].y);
-      *reinterpret_cast<float4*>(stage + (r0 + i) * LD + c0 + 4) =
-          make_float4(a[i][2].x, a[i][2].y, a[i][3].x, a[i][3].y);
+      const float v[8] = {sign * a[i][0].x, sign * a[i][0].y, sign * a[i][1].x, sign * a[i][1].y,
+                          sign * a[i][2].x, sign * a[i][2].y, sign * a[i][3].x, sign * a[i][3].y};
+      if (img) store_chunk_image(img, r0 + i, J, v);
+      if (Nf) {
+        *reinterpret_cast<float4*>(Nf + (r0 + i) * D + c0) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4*>(Nf + (r0 + i) * D + c0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
+      }
     }
-    __syncthreads();
-    // B operand of the scan: row n holds N_f[n][k]; N_f is symmetric, so this is
-    // its column n as the product S N_f needs (up to fp32 rounding of the inverse)
-    write_image128_rows(stage, LD, nimg + fi * (kImgBytes / 2));
+    if (I != J) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = sign * ((m & 1) ? a[i][m >> 1].y : a[i][m >> 1].x);
+        if (img) store_chunk_image(img, c0 + m, I, v);
+        if (Nf) {
+          *reinterpret_cast<float4*>(Nf + (c0 + m) * D + r0) = make_float4(v[0], v[1], v[2], v[3]);
+          *reinterpret_cast<float4*>(Nf + (c0 + m) * D + r0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
+        }
+      }
+    }
   }
 }
 
@@ -334,9 +403,7 @@ cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nim
     int nb = (a.sh.S + kStatsTokens - 1) / kStatsTokens;
     long long T = a.NF() * nb;
     int G = (int)(T < kStatsGrid ? T : kStatsGrid);
-    size_t smem = ((size_t)128 * 132 + 4 * 128) * sizeof(float);
-    cudaFuncSetAttribute(k_solve128, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_solve128<<<(unsigned)a.NF(), 256, smem, a.stream>>>(partials, T, nb, G, rc, Nm, nimg, Bsum, Aout, a.sh.H,
+    k_solve128<<<(unsigned)a.NF(), kSolveThreads, 0, a.stream>>>(partials, T, nb, G, rc, Nm, nimg, Bsum, Aout, a.sh.H,
                                                           a.sh.F);
     return cudaGetLastError();
   }
