@@ -34,6 +34,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 2^e for e in [-126, 127], built from the exponent field (exact)
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+// two floats -> f16x2 (round to nearest even), lo in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // SiLU with the accurate exponential (SIMT paths, fp32 parity).
 __device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
 

@@ -21,6 +21,22 @@ __host__ __device__ __forceinline__ uint32_t img_offset(int part, int n, int k) 
   return part * 32768u + (k >> 6) * 16384u + n * 128u + ((((k & 63) >> 3) ^ (n & 7)) << 4) + (k & 7) * 2u;
 }
 
+// Read-out operand image of W_t: one fp16 part in the same layout (32 KB), each
+// block of 32 rows b scaled by 2^-e_b so its largest entry lies in [0.5, 1)
+// (e_b stored beside the image; power-of-two scaling is exact).  fp16 keeps 11
+// significant bits against 8 for bf16, which the read-out's RMSNorm needs when
+// a dominant component of W_t cancels in W_t q'.
+constexpr int kWImgBytes = 128 * 128 * 2;
+constexpr int kWRowBlocks = 4;
+constexpr int kWBlockRows = 128 / kWRowBlocks;
+
+__device__ __forceinline__ void store_chunk_f16(uint8_t* img, int n, int k, const float* v) {
+  uint32_t hw[4];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hw[e / 2]) : "f"(v[e + 1]), "f"(v[e]));
+  *reinterpret_cast<uint4*>(img + img_offset(0, n, k)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+}
+
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));

@@ -42,7 +42,8 @@ struct WsPlan {
   // tensor-core path
   size_t part = 0;                      // fp32 [slots][d][2d]: rows of [A | B^T] partial sums
   size_t nimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of N_f
-  size_t wimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of W_t
+  size_t wimg = 0;                      // fp16 [B,H,F][d][d] read-out operand images of W_t
+  size_t wbexp = 0;                     // int32 [B,H,F][4] row-block exponents of those images
   size_t total = 0;
 };
 
@@ -58,7 +59,7 @@ cudaError_t launch_solve(const Args& a, const float* A, float* Nm, uint16_t* nim
 cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, float* P, float* Q, int* pexp,
                              int* qexp);
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
-                          uint16_t* wimg, int* wexp);
+                          uint16_t* wimg, int* wexp, int* wbexp);
 cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, const int* wexp);
 // dst = src * 2^expo[frame] (expo may be NULL)
 cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo = nullptr);
@@ -72,6 +73,7 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
                            int* qexp, bool all_frames, uint32_t* status);
-cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, uint32_t* status);
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, const int* wbexp,
+                              uint32_t* status);
 
 }  // namespace vdn

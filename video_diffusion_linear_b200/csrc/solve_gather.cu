@@ -513,7 +513,8 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
                                                    const int* __restrict__ pexp, const int* __restrict__ qexp,
                                                    const float* __restrict__ alpha, const float* __restrict__ text,
                                                    int H, int F, int chunk, int radius, float* __restrict__ W,
-                                                   uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
+                                                   uint16_t* __restrict__ wimg, int* __restrict__ wexp,
+                                                   int* __restrict__ wbexp) {
   constexpr int D = 128;
   __shared__ float dpre[D], dsuf[D], red[16];
   const int tid = threadIdx.x, n = tid >> 2, k0 = (tid & 3) * 32;
@@ -588,23 +589,11 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
       *reinterpret_cast<float4*>(W + fi * D * D + n * D + k0 + 4 * j) =
           make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
   }
-  if (wimg) {
-    uint8_t* img = reinterpret_cast<uint8_t*>(wimg + fi * (kImgBytes / 2));
+  if (wimg) {   // fp16 image; W is already normalised as a whole, so every row block has exponent 0
+    uint8_t* img = reinterpret_cast<uint8_t*>(wimg) + fi * kWImgBytes;
 #pragma unroll
-    for (int cch = 0; cch < 4; ++cch) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split_bf16(w[8 * cch + e], h0, l0);
-        split_bf16(w[8 * cch + e + 1], h1, l1);
-        hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-      }
-      const uint32_t off = img_offset(0, n, k0 + 8 * cch);
-      *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
+    for (int cch = 0; cch < 4; ++cch) store_chunk_f16(img, n, k0 + 8 * cch, &w[8 * cch]);
+    if (tid < kWRowBlocks) wbexp[fi * kWRowBlocks + tid] = 0;
   }
 }
 
@@ -615,15 +604,18 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
 // (stored states are below 2^48, see the scans' block exponent), W_t is stored as 2^-e W_t.
 constexpr int kGatherMaxChunk = 16;
 constexpr int kGatherRows = 32;
+static_assert(kWBlockRows == kGatherRows, "one gather CTA per row block of the W image");
 
 __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict__ P, const float* __restrict__ Q,
                                                          const int* __restrict__ pexp, const int* __restrict__ qexp,
                                                          const float* __restrict__ alpha,
                                                          const float* __restrict__ text, int H, int F, int chunk,
                                                          int radius, float* __restrict__ W,
-                                                         uint16_t* __restrict__ wimg, int* __restrict__ wexp) {
+                                                         uint16_t* __restrict__ wimg, int* __restrict__ wexp,
+                                                         int* __restrict__ wbexp) {
   constexpr int D = 128;
   __shared__ float dpre[kGatherMaxChunk][D], dsuf[kGatherMaxChunk][D];
+  __shared__ float red[2][4];
   const int tid = threadIdx.x, n = blockIdx.z * kGatherRows + (tid >> 2), k0 = (tid & 3) * 32;
   const long long bh = blockIdx.x;
   const int h = (int)(bh % H);
@@ -692,37 +684,45 @@ __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict
             make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
     }
     if (wimg) {
-      uint8_t* img = reinterpret_cast<uint8_t*>(wimg + fi * (kImgBytes / 2));
+      // this CTA's 32 rows form one row block of the fp16 image: scale it by the
+      // power of two that puts its largest entry in [0.5, 1)
+      float amax = 0.f;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) amax = fmaxf(amax, fabsf(w[u]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      float* rb = red[(t - t0) & 1];   // double-buffered: one barrier per frame
+      if ((tid & 31) == 0) rb[tid >> 5] = amax;
+      __syncthreads();
+      amax = fmaxf(fmaxf(rb[0], rb[1]), fmaxf(rb[2], rb[3]));
+      int eb = 0;
+      if (amax > 0.f) frexpf(amax, &eb);
+      eb = min(max(eb, -125), 126);    // 2^-eb stays a normal float
+      if (tid == 0) wbexp[fi * kWRowBlocks + blockIdx.z] = eb;
+      const float sc = pow2f(-eb);
+      uint8_t* img = reinterpret_cast<uint8_t*>(wimg) + fi * kWImgBytes;
 #pragma unroll
       for (int cch = 0; cch < 4; ++cch) {
-        uint32_t hw[4], lw[4];
+        float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          __nv_bfloat16 h0, l0, h1, l1;
-          split_bf16(w[8 * cch + e], h0, l0);
-          split_bf16(w[8 * cch + e + 1], h1, l1);
-          hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-          lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-        }
-        const uint32_t off = img_offset(0, n, k0 + 8 * cch);
-        *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        for (int e = 0; e < 8; ++e) v[e] = w[8 * cch + e] * sc;
+        store_chunk_f16(img, n, k0 + 8 * cch, v);
       }
     }
   }
 }
 
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
-                          uint16_t* wimg, int* wexp) {
+                          uint16_t* wimg, int* wexp, int* wbexp) {
   if (a.sh.d == 128 && a.chunk <= kGatherMaxChunk) {
     dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((a.sh.F + a.chunk - 1) / a.chunk), 128 / kGatherRows);
     k_gather128_chunk<<<grid, 128, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
-                                                   a.radius, W, wimg, wexp);
+                                                   a.radius, W, wimg, wexp, wbexp);
     return cudaGetLastError();
   }
   if (a.sh.d == 128) {
     k_gather128<<<(unsigned)a.NF(), 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
-                                                        a.chunk, a.radius, W, wimg, wexp);
+                                                        a.chunk, a.radius, W, wimg, wexp, wbexp);
     return cudaGetLastError();
   }
   size_t smem = (2 * 16 + 8) * sizeof(float);

@@ -4,7 +4,12 @@
 // order (batch, head, frame, tile), so W_t changes only at frame boundaries.
 // Per tile, O[128 tokens x 128] = Q'[128 x 128] W_t^T runs as tcgen05 MMAs with
 // the accumulator in TMEM (two buffers), Q' = L2(SiLU(q)) produced in place in
-// shared memory, and W_t given as a bf16 hi/lo image (two MMAs, fp32 accumulate).
+// shared memory.  The product runs on fp16 operands, one MMA per K step: Q'
+// (unit rows) and W_t, whose image the gather writes in fp16 with a power-of-two
+// exponent per block of 32 rows (its largest entry in [0.5, 1)); the epilogue
+// folds 2^e of each row block into the RMSNorm.  The gate / output tiles have
+// three stages, so the store of a tile has a whole tile's time to read its
+// buffer before that buffer is handed back to the gate loads.
 // The epilogue reads one token row per thread from TMEM (32x32b layout), so the
 // RMSNorm needs no cross-thread reduction; it multiplies rms_w and the gate and
 // writes bf16 through shared memory and a TMA store.
@@ -24,22 +29,25 @@ namespace vdn {
 
 namespace {
 
+constexpr int kQS = 2;      // q stages
+constexpr int kGS = 3;      // gate stages
+
 struct __align__(1024) ReadSmem {
-  uint8_t wimg[65536];     // W_t hi | lo (K-major SW128 B operand)
-  uint8_t qt[2][32768];    // raw q tile -> Q' (K-major SW128 A operand), two stages
-  uint8_t gt[2][32768];    // gate tile -> output tile, two stages
+  uint8_t wimg[32768];     // W_t, fp16 (K-major SW128 B operand)
+  uint8_t qt[kQS][32768];  // raw q tile -> Q' (K-major SW128 A operand)
+  uint8_t gt[kGS][32768];  // gate tile -> output tile
   float rms_w[128];
-  float ssq_t[2][2][128];  // [stage][channel half][row] partial sums of the q transform
+  float ssq_t[kQS][2][128];  // [stage][channel half][row] partial sums of the q transform
   float ssq_e[2][2][128];  // same for the epilogue
   uint64_t bar_w_full, bar_w_empty;
-  uint64_t bar_q_full[2], bar_q_ready[2], bar_q_empty[2];
-  uint64_t bar_g_full[2], bar_g_empty[2];
+  uint64_t bar_q_full[kQS], bar_q_ready[kQS], bar_q_empty[kQS];
+  uint64_t bar_g_full[kGS], bar_g_empty[kGS];
   uint64_t bar_acc_full[2], bar_acc_empty[2];
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdesc = tc::idesc_f16_f32(128, 128, false, false);
 constexpr int kThreads = 608;
 
 // swizzled byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] bf16 tile
@@ -54,6 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
                                                            const __grid_constant__ CUtensorMap tmO,
                                                            const uint16_t* __restrict__ wimg_g,
                                                            const int* __restrict__ wexp,
+                                                           const int* __restrict__ wbexp,
                                                            const float* __restrict__ rms_w, int H, int F,
                                                            int ntile, long long T, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -66,12 +75,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
   if (tid == 0) {
     tc::mbar_init(&sm.bar_w_full, 1);
     tc::mbar_init(&sm.bar_w_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQS; ++s) {
       tc::mbar_init(&sm.bar_q_full[s], 1);
       tc::mbar_init(&sm.bar_q_ready[s], 256);
       tc::mbar_init(&sm.bar_q_empty[s], 1);
+    }
+    for (int s = 0; s < kGS; ++s) {
       tc::mbar_init(&sm.bar_g_full[s], 1);
       tc::mbar_init(&sm.bar_g_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&sm.bar_acc_full[s], 1);
       tc::mbar_init(&sm.bar_acc_empty[s], 256);
     }
@@ -111,15 +124,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
             if (!tc::mbar_wait(&sm.bar_w_empty, wph, abort_flag, status)) break;
             wph ^= 1;
           }
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(wimg_g + fi * (kImgBytes / 2));
-          tc::mbar_arrive_expect_tx(&sm.bar_w_full, kImgBytes);
-          for (int q = 0; q < 4; ++q) tc::bulk_load(sm.wimg + q * 16384, src + q * 16384, 16384, &sm.bar_w_full);
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(wimg_g) + fi * kWImgBytes;
+          tc::mbar_arrive_expect_tx(&sm.bar_w_full, kWImgBytes);
+          for (int q = 0; q < 2; ++q) tc::bulk_load(sm.wimg + q * 16384, src + q * 16384, 16384, &sm.bar_w_full);
           cur = fi;
         }
         int h, s0, fb;
         coords(x, h, s0, fb);
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
+        const int st = it % kQS;
+        const uint32_t ph = (it / kQS) & 1;
         if (!tc::mbar_wait(&sm.bar_q_empty[st], ph ^ 1, abort_flag, status)) break;
         tc::mbar_arrive_expect_tx(&sm.bar_q_full[st], 32768);
         tc::tma_load_4d(&tmQ, &sm.bar_q_full[st], sm.qt[st], 0, h, s0, fb);
@@ -132,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       long long cur = -1;
       uint32_t wph = 0;
       int it = 0;
-      const uint32_t w_hi = tc::smem_u32(sm.wimg), w_lo = w_hi + 32768;
+      const uint32_t w = tc::smem_u32(sm.wimg);
       for (long long x = x0; x < x1; ++x, ++it) {
         long long fi = x / ntile;
         if (fi != cur) {
@@ -140,22 +153,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
           wph ^= 1;
           cur = fi;
         }
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!tc::mbar_wait(&sm.bar_q_ready[st], ph, abort_flag, status)) break;
-        if (!tc::mbar_wait(&sm.bar_acc_empty[st], ph ^ 1, abort_flag, status)) break;
+        const int qs = it % kQS, ab = it & 1;
+        const uint32_t qph = (it / kQS) & 1, aph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&sm.bar_q_ready[qs], qph, abort_flag, status)) break;
+        if (!tc::mbar_wait(&sm.bar_acc_empty[ab], aph ^ 1, abort_flag, status)) break;
         tc::tc_fence_after();
-        const uint32_t d = tmem + st * 128;
-        const uint32_t a = tc::smem_u32(sm.qt[st]);
+        const uint32_t d = tmem + ab * 128;
+        const uint32_t a = tc::smem_u32(sm.qt[qs]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          uint64_t ad = tc::smem_desc(a + koff, 16, 1024);
-          tc::umma_bf16(d, ad, tc::smem_desc(w_hi + koff, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
-          tc::umma_bf16(d, ad, tc::smem_desc(w_lo + koff, 16, 1024), kIdesc, 1u);
+          tc::umma_bf16(d, tc::smem_desc(a + koff, 16, 1024), tc::smem_desc(w + koff, 16, 1024), kIdesc,
+                        kk > 0 ? 1u : 0u);
         }
-        tc::umma_commit(&sm.bar_q_empty[st]);
-        tc::umma_commit(&sm.bar_acc_full[st]);
+        tc::umma_commit(&sm.bar_q_empty[qs]);
+        tc::umma_commit(&sm.bar_acc_full[ab]);
         if (x + 1 == x1 || (x + 1) / ntile != fi) tc::umma_commit(&sm.bar_w_empty);
       }
     }
@@ -166,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       for (long long x = x0; x < x1; ++x, ++it) {
         int h, s0, fb;
         coords(x, h, s0, fb);
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
+        const int st = it % kGS;
+        const uint32_t ph = (it / kGS) & 1;
         if (!tc::mbar_wait(&sm.bar_g_empty[st], ph ^ 1, abort_flag, status)) break;
         tc::mbar_arrive_expect_tx(&sm.bar_g_full[st], 32768);
         tc::tma_load_4d(&tmG, &sm.bar_g_full[st], sm.gt[st], 0, h, s0, fb);
@@ -180,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     const int r = tt & 127, hf = tt >> 7;   // row, channel half (chunks 8 hf .. 8 hf + 7)
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
-      const int st = it & 1;
-      const uint32_t ph = (it >> 1) & 1;
+      const int st = it % kQS;
+      const uint32_t ph = (it / kQS) & 1;
       if (!tc::mbar_wait(&sm.bar_q_full[st], ph, abort_flag, status)) break;
       uint8_t* base = sm.qt[st];
       float2 v[32];
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 y = __fmul2_rn(v[4 * cq + e], iv);
-          o4[e] = pack_bf16x2(y.x, y.y);
+          o4[e] = pack_f16x2(y.x, y.y);
         }
         *reinterpret_cast<uint4*>(base + row_chunk(r, 8 * hf + cq)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
@@ -226,11 +238,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     for (long long x = x0; x < x1; ++x, ++it) {
       const int st = it & 1;
       const uint32_t ph = (it >> 1) & 1;
-      if (leader && it > 0) {
-        tc::bulk_wait_read_all();                       // the previous tile's store has read its buffer
-        tc::mbar_arrive(&sm.bar_g_empty[(it - 1) & 1]);
+      if (leader && it > 1) {
+        tc::bulk_wait_read<1>();                        // the store of tile it - 2 has read its buffer
+        tc::mbar_arrive(&sm.bar_g_empty[(it - 2) % kGS]);
       }
-      const int ew = wexp[x / ntile];   // issued before the wait, used after it
+      // exponents of W_t (issued before the wait, used after it): the whole
+      // matrix (RMSNorm eps) and the two row blocks of this channel half
+      const long long fi = x / ntile;
+      const int ew = wexp[fi];
+      const int eb0 = wbexp[fi * kWRowBlocks + 2 * hf], eb1 = wbexp[fi * kWRowBlocks + 2 * hf + 1];
       if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
       tc::tc_fence_after();
       const uint32_t taddr = tmem + st * 128 + 64 * hf + ((uint32_t)(quarter * 32) << 16);
@@ -244,19 +260,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&sm.bar_acc_empty[st]);
-      float2 acc = make_float2(0.f, 0.f);
+      // the true channel j of this half is 2^eb o_j, eb = eb0 for the first 32
+      // channels, eb1 for the last 32 (row blocks of the fp16 image): the scales
+      // enter the two partial sums of squares and the per-channel multiplier
+      const float sc0 = pow2f(eb0), sc1 = pow2f(eb1);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
+      for (int e = 0; e < 32; e += 2) {
         const float2 a = make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1]));
-        acc = __ffma2_rn(a, a, acc);
+        acc0 = __ffma2_rn(a, a, acc0);
+        const float2 c = make_float2(__uint_as_float(o[e + 32]), __uint_as_float(o[e + 33]));
+        acc1 = __ffma2_rn(c, c, acc1);
       }
-      sm.ssq_e[st][hf][m] = acc.x + acc.y;
+      sm.ssq_e[st][hf][m] = (acc0.x + acc0.y) * (sc0 * sc0) + (acc1.x + acc1.y) * (sc1 * sc1);
       tc::named_bar(1, 256);
       // W_t is stored as 2^-e W_t: the RMSNorm eps scales by 2^-2e
       const float ss = sm.ssq_e[st][0][m] + sm.ssq_e[st][1][m];
       const float inv = rsqrtf(ss * (1.0f / 128.0f) + ldexpf(kRmsEps, -2 * ew));
-      if (!tc::mbar_wait(&sm.bar_g_full[st], ph, abort_flag, status)) break;
-      uint8_t* base = sm.gt[st];
+      const float inv0 = inv * sc0, inv1 = inv * sc1;
+      const int gs = it % kGS;
+      if (!tc::mbar_wait(&sm.bar_g_full[gs], (it / kGS) & 1, abort_flag, status)) break;
+      uint8_t* base = sm.gt[gs];
 #pragma unroll
       for (int cq = 0; cq < 8; ++cq) {
         const int c = 8 * hf + cq;
@@ -265,12 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         const float4 w0 = *reinterpret_cast<const float4*>(&sm.rms_w[8 * c]);
         const float4 w1 = *reinterpret_cast<const float4*>(&sm.rms_w[8 * c + 4]);
         const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const float iv = cq < 4 ? inv0 : inv1;   // chunks 0-3: first row block of the half
         uint32_t outw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = 8 * cq + 2 * e;
           const float2 y = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                                 make_float2(inv * wv[2 * e], inv * wv[2 * e + 1])),
+                                                 make_float2(iv * wv[2 * e], iv * wv[2 * e + 1])),
                                       make_float2(bf16lo(gs[e]), bf16hi(gs[e])));
           outw[e] = pack_bf16x2(y.x, y.y);
         }
@@ -297,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
   }
 }
 
-cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, uint32_t* status) {
+cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, const int* wbexp,
+                              uint32_t* status) {
   const vdn_shape& sh = a.sh;
   CUtensorMap tq, tg, to;
   long long BF = (long long)sh.B * sh.F;
@@ -314,7 +340,7 @@ cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* we
   size_t smem = sizeof(ReadSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_readout_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tq, tg, to, wimg, wexp, a.rms_w, sh.H, sh.F, ntile, T,
+  k_readout_tc<<<(unsigned)G, kThreads, smem, a.stream>>>(tq, tg, to, wimg, wexp, wbexp, a.rms_w, sh.H, sh.F, ntile, T,
                                                              status);
   return cudaGetLastError();
 }

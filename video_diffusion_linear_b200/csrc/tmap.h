@@ -22,14 +22,16 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
 }
 
 // Token tensor [B*F frames][S tokens][H heads][d] of 16-bit elements, viewed
-// as 4-D (d, H, S, B*F); box {64 channels, 1 head, box_rows tokens, 1 frame},
-// 128-byte swizzle.  Rows past S (or before 0) read as zero and are not written.
-inline bool tmap_tokens_bf16(CUtensorMap* m, const void* base, int d, int H, int S, long long BF, int box_rows) {
+// as 4-D (d, H, S, B*F); box {64 channels, box_heads heads, box_rows tokens,
+// 1 frame}, 128-byte swizzle (box rows ordered token-major, head-minor).  Rows
+// past S (or before 0) and heads past H read as zero and are not written.
+inline bool tmap_tokens_bf16(CUtensorMap* m, const void* base, int d, int H, int S, long long BF, int box_rows,
+                             int box_heads = 1) {
   auto enc = tmap_encoder();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)BF};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)S * H * d * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

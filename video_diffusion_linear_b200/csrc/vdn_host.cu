@@ -57,7 +57,8 @@ WsPlan plan_workspace(const vdn_shape& sh, int /*rule*/, bool tc) {
     p.nimg = take(NF * (size_t)kImgBytes);
     p.P = take(frame_mats);
     p.Q = take(frame_mats);
-    p.wimg = take(NF * (size_t)kImgBytes);
+    p.wimg = take(NF * (size_t)kWImgBytes);
+    p.wbexp = take(NF * kWRowBlocks * sizeof(int));
   }
   p.total = off;
   return p;
@@ -171,7 +172,7 @@ vdn_status run_forward(const Args& a, void* ws, int impl, void* const* events = 
     VDN_LAUNCH(mark());
     VDN_LAUNCH(launch_scan_simt(a, Bm, Nm, P, Q, pexp, qexp));
     VDN_LAUNCH(mark());
-    VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, W, nullptr, wexp));
+    VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, W, nullptr, wexp, nullptr));
     VDN_LAUNCH(mark());
     VDN_LAUNCH(launch_readout_simt(a, qf, W, wexp));
     VDN_LAUNCH(mark());
@@ -190,6 +191,7 @@ vdn_status run_forward(const Args& a, void* ws, int impl, void* const* events = 
   uint16_t* nimg = at<uint16_t>(ws, p.nimg);
   float *P = at<float>(ws, p.P), *Q = at<float>(ws, p.Q);
   uint16_t* wimg = at<uint16_t>(ws, p.wimg);
+  int* wbexp = at<int>(ws, p.wbexp);
   int *pexp = at<int>(ws, p.pexp), *qexp = at<int>(ws, p.qexp), *wexp = at<int>(ws, p.wexp);
   bool all_frames = dbg && (dbg->P || dbg->Q);
   // the debug export of W: the gather writes 2^-wexp W_t into dbg->W, rescaled in place below
@@ -199,9 +201,9 @@ vdn_status run_forward(const Args& a, void* ws, int impl, void* const* events = 
   VDN_LAUNCH(mark());
   VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, P, Q, pexp, qexp, all_frames, status));
   VDN_LAUNCH(mark());
-  VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, dbg ? dbg->W : nullptr, wimg, wexp));
+  VDN_LAUNCH(launch_gather(a, P, Q, pexp, qexp, dbg ? dbg->W : nullptr, wimg, wexp, wbexp));
   VDN_LAUNCH(mark());
-  VDN_LAUNCH(launch_readout_tc(a, wimg, wexp, status));
+  VDN_LAUNCH(launch_readout_tc(a, wimg, wexp, wbexp, status));
   VDN_LAUNCH(mark());
   if (dbg) {
     if (dbg->B) VDN_LAUNCH(launch_copy_frames(a, Bsum, dbg->B));
