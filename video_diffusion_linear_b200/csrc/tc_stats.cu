@@ -38,8 +38,9 @@ constexpr int kTransformWarps = 12;
 constexpr int kBT = 2 * kTPT * kTransformWarps;       // tokens per block
 static_assert(kBT == kStatsTokens, "block size");
 static_assert(kBT % 32 == 0, "block size");
-constexpr int kRS = 3;                                // raw TMA stages
-constexpr int kOS = 1;                                // operand stages
+constexpr int kRS = 2;                                // raw TMA stages
+constexpr int kOS = 2;                                // operand stages: the transform fills one while
+                                                      // the tensor cores read the other
 constexpr int kRawRows = kBT + 2;
 constexpr int kRawHalf = (kRawRows * 128 + 1023) / 1024 * 1024;
 constexpr int kRawBytes = 4 * kRawRows * 128;         // k and v, two channel halves each
@@ -62,6 +63,7 @@ struct __align__(1024) StatsSmem {
 };
 
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 256, true, true);
+
 
 // byte offset of the 16-byte chunk holding channels 8c..8c+7 of token t in an
 // MN-major SW128 operand of 128 channels x kBT tokens (atoms of 64 channels x
