@@ -54,14 +54,15 @@ def algorithmic_bytes(w: synth.Workload) -> dict:
     TH = w.B * w.F * w.S * w.H                 # token-heads
     NF = w.B * w.H * w.F                       # (batch, head, frame) triples
     mat = d * d * 4                            # one fp32 d x d matrix
-    img = d * d * 2 * 2                        # bf16 hi/lo operand image
+    img = d * d * 2 * 2                        # bf16 hi/lo operand image of N_f
+    wimg = d * d * 2                           # fp16 read-out operand image of W_t
     stored = 2 * w.B * w.H * (-(-w.F // w.chunk))   # chunk-boundary states written by the scan
     return {
         "frame_stats": TH * (2 * d * 2 + 4) + NF * 2 * mat,
         "frame_solve": NF * (2 * mat + mat + img),
         "scan": 2 * NF * (img + mat) + stored * mat,
-        "gather": NF * (2 * mat + img),
-        "readout": TH * 3 * d * 2 + NF * img,
+        "gather": NF * (2 * mat + wimg),
+        "readout": TH * 3 * d * 2 + NF * wimg,
     }
 
 

@@ -291,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
         }
       };
 
+      if (!tc::mbar_wait(&sm.op_empty[os], oph ^ 1, abort_flag, status)) break;
       {
         float2 vy[kTPT][4];
         float unused[kTPT];
         conv_silu(1, vy, unused);
-        if (!tc::mbar_wait(&sm.op_empty[os], oph ^ 1, abort_flag, status)) break;
         store(vy, sb, sm.op[os] + kOpHalf);      // Y = sqrt(beta) v'
       }
       float2 ky[kTPT][4];
