@@ -28,7 +28,7 @@ struct __align__(1024) ScanSmem {
   uint8_t nimg[65536];       // N_f hi | lo image
   float bf[4][128 * 32];     // B_f, four swizzled [128 rows][32 cols] boxes
   float alpha[128];
-  uint64_t bar_n, bar_b, bar_mma;
+  uint64_t bar_n, bar_b, bar_mma, bar_nhi;
   uint32_t tmem_base;
   int abort;
 };
@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     tc::mbar_init(&sm.bar_n, 1);
     tc::mbar_init(&sm.bar_b, 1);
     tc::mbar_init(&sm.bar_mma, 1);
+    tc::mbar_init(&sm.bar_nhi, 1);
     sm.abort = 0;
     tc::fence_barrier_init();
   }
@@ -102,12 +103,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   }
 
   auto frame_of = [&](int step) { return dir == 0 ? step : F - 1 - step; };
-  auto load_n = [&](int step) {
+  // N_f image: the hi part (first 32 KB) and the lo part arrive on the same
+  // barrier but are requested separately, each as soon as its buffer is free
+  auto load_n_part = [&](int step, int part) {
     long long fi = bh * F + frame_of(step);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2));
-    tc::mbar_arrive_expect_tx(&sm.bar_n, kImgBytes);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2)) + part * 32768;
+    if (part == 0) tc::mbar_arrive_expect_tx(&sm.bar_n, kImgBytes);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tc::bulk_load(sm.nimg + j * 16384, src + j * 16384, 16384, &sm.bar_n);
+    for (int j = 0; j < 2; ++j)
+      tc::bulk_load(sm.nimg + part * 32768 + j * 16384, src + j * 16384, 16384, &sm.bar_n);
   };
   auto load_b = [&](int step) {
     long long fi = bh * F + frame_of(step);
@@ -120,7 +124,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     tc::prefetch_l2(reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2)), kImgBytes);
   };
   if (tid == 0) {
-    load_n(0);
+    load_n_part(0, 0);
+    load_n_part(0, 1);
     load_b(0);
     if (F > 1) prefetch(1);
   }
@@ -175,21 +180,29 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
       if (early_b && step + 1 < F) load_b(step + 1);
       if (tc::mbar_wait(&sm.bar_n, ph, abort_flag, status)) {
         tc::tc_fence_after();
+        // the terms with N_hi first (Xh Nh, Xl Nh), then Xh Nl: N_hi is free a
+        // third of the product earlier, and the next frame's N_hi can load
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
           uint64_t ah = tc::smem_desc(a_hi + koff, 16, 1024), al = tc::smem_desc(a_lo + koff, 16, 1024);
-          uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024), bld = tc::smem_desc(n_lo + koff, 16, 1024);
+          uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024);
           tc::umma_bf16(tmem, ah, bhd, kIdesc, kk > 0 ? 1u : 0u);
-          tc::umma_bf16(tmem, ah, bld, kIdesc, 1u);
           tc::umma_bf16(tmem, al, bhd, kIdesc, 1u);
         }
+        tc::umma_commit(&sm.bar_nhi);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::umma_bf16(tmem, tc::smem_desc(a_hi + koff, 16, 1024), tc::smem_desc(n_lo + koff, 16, 1024), kIdesc, 1u);
+        }
         tc::umma_commit(&sm.bar_mma);
+        if (step + 1 < F && tc::mbar_wait(&sm.bar_nhi, ph, abort_flag, status)) load_n_part(step + 1, 0);
       }
     }
     if (!tc::mbar_wait(&sm.bar_mma, ph, abort_flag, status)) break;
     tc::tc_fence_after();
-    if (tid == 0 && step + 1 < F) load_n(step + 1);   // the product that read N_f is complete
+    if (tid == 0 && step + 1 < F) load_n_part(step + 1, 1);   // the product that read N_lo is complete
 
     // S_f = D + cpost B_f
     const bool store = all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0));
