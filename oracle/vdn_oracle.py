@@ -27,8 +27,17 @@ Readings taken where the page is silent (each one is a keyword argument here):
   * read-out o = W_t q', RMSNorm over d with eps 1e-6 and weight rms_w[d], then
     the (post-sigmoid) output gate.
 
-Parity status: every function here is pinned by tests/test_oracle_pins.py against
-closed forms, textbook reductions, library routines or brute force.
+The page also places the branch in its layer: the windowed softmax branch sees
+the frames of the chunk-aligned window through the RoPE-rotated q/k, the linear
+branch everything outside it, and the two outputs are added (section on why
+video models stall on attention and what the far field is).  Readings: scaled
+dot-product softmax with scale 1/sqrt(d), bidirectional over all keys of frames
+lo..hi, no mask inside the window; the rotation is applied by the caller (its
+parameters are not on the page), so the softmax branch takes q_rope, k_rope.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py and
+tests/test_oracle_softmax_pins.py against closed forms, textbook reductions,
+library routines or brute force.
 """
 from __future__ import annotations
 
@@ -254,3 +263,69 @@ def sampled_outputs(inp: dict, F: int, S: int, rule: str, c: float, chunk: int, 
         t, s = divmod(int(n), S)
         res[i] = readout(st["W"][t], st["qf"][t, s][None, :], g[n][None, :], rms_w, prenorm)[0]
     return res
+
+
+# --------------------------------------------------------------------------- windowed softmax branch
+def window_softmax_frame(qr_t, kr_win, v_win, scale):
+    """softmax(q k^T * scale) v for the query rows qr_t [n, d] against the keys
+    kr_win [m, d] and values v_win [m, d] of their window (one frame's queries
+    share the window).  Max-subtracted, so large scores do not overflow."""
+    sc = (qr_t @ kr_win.T) * scale
+    sc -= sc.max(axis=1, keepdims=True)
+    w = np.exp(sc)
+    w /= w.sum(axis=1, keepdims=True)
+    return w @ v_win
+
+
+def window_softmax_head(qr_h, kr_h, v_h, F: int, S: int, chunk: int, radius: int, scale=None, frames=None):
+    """Windowed softmax branch of one (batch, head): query frame t attends to
+    every token of frames lo..hi = window_bounds(t).  Inputs [F*S, d]; returns
+    [F*S, d] (rows of frames not in `frames` stay NaN)."""
+    d = qr_h.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    out = np.full(qr_h.shape, np.nan)
+    for t in (range(F) if frames is None else frames):
+        lo, hi = window_bounds(t, F, chunk, radius)
+        keys = slice(lo * S, (hi + 1) * S)
+        out[t * S:(t + 1) * S] = window_softmax_frame(qr_h[t * S:(t + 1) * S], kr_h[keys], v_h[keys], scale)
+    return out
+
+
+def window_softmax_forward(inp: dict, F: int, S: int, chunk: int = 5, radius: int = 1, heads=None, batches=None,
+                           scale=None):
+    """The windowed softmax branch for the selected (batch, head) pairs:
+    [B, F*S, H, d] float64 (unselected entries NaN).  Uses inp["q_rope"],
+    inp["k_rope"] and inp["v"]."""
+    qr = inp["q_rope"]
+    B, N, H, d = qr.shape
+    out = np.full((B, N, H, d), np.nan)
+    for b in (range(B) if batches is None else batches):
+        for h in (range(H) if heads is None else heads):
+            out[b, :, h, :] = window_softmax_head(_f64(inp["q_rope"][b, :, h, :]), _f64(inp["k_rope"][b, :, h, :]),
+                                                  _f64(inp["v"][b, :, h, :]), F, S, chunk, radius, scale)
+    return out
+
+
+def sampled_window_softmax(inp: dict, F: int, S: int, chunk: int, radius: int, b: int, h: int, tokens, scale=None):
+    """Softmax-branch outputs of selected tokens (indices into F*S) of one (batch, head)."""
+    qr = _f64(inp["q_rope"][b, :, h, :])
+    kr = _f64(inp["k_rope"][b, :, h, :])
+    v = _f64(inp["v"][b, :, h, :])
+    d = qr.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    tokens = np.asarray(tokens)
+    res = np.empty((len(tokens), d))
+    for i, n in enumerate(tokens):
+        t = int(n) // S
+        lo, hi = window_bounds(t, F, chunk, radius)
+        keys = slice(lo * S, (hi + 1) * S)
+        res[i] = window_softmax_frame(qr[int(n)][None, :], kr[keys], v[keys], scale)[0]
+    return res
+
+
+def hybrid_forward(inp: dict, F: int, S: int, rule: str = "vdn_solve", c: float = 1.0, chunk: int = 5,
+                   radius: int = 1, heads=None, batches=None, scale=None):
+    """The hybrid attention layer's two branches summed: windowed softmax over
+    the near field plus the bidirectional linear branch over the far field."""
+    return (window_softmax_forward(inp, F, S, chunk, radius, heads, batches, scale)
+            + branch_forward(inp, F, S, rule, c, chunk, radius, heads, batches))

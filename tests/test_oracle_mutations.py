@@ -130,3 +130,63 @@ def test_planted_mistake_is_caught(name, monkeypatch):
         except (AssertionError, np.linalg.LinAlgError, ValueError):
             caught += 1
     assert caught > 0, f"no pin fails with mutant {name}"
+
+
+# ----------------------------------------------------------------------------- windowed softmax branch
+import test_oracle_softmax_pins as spins  # noqa: E402
+
+_orig_soft = {name: getattr(O, name) for name in ("window_softmax_frame", "window_bounds")}
+
+
+def _soft_scale_over_d(qr_t, kr_win, v_win, scale):
+    return _orig_soft["window_softmax_frame"](qr_t, kr_win, v_win, scale * scale)   # 1/d instead of 1/sqrt(d)
+
+
+def _soft_no_max_shift(qr_t, kr_win, v_win, scale):
+    with np.errstate(over="ignore", invalid="ignore"):
+        w = np.exp((qr_t @ kr_win.T) * scale)
+        return (w / w.sum(axis=1, keepdims=True)) @ v_win
+
+
+def _soft_columns_normalised(qr_t, kr_win, v_win, scale):
+    sc = (qr_t @ kr_win.T) * scale
+    w = np.exp(sc - sc.max())
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return (w / w.sum(axis=0, keepdims=True)) @ v_win / max(1, w.shape[0])
+
+
+def _soft_keys_as_values(qr_t, kr_win, v_win, scale):
+    return _orig_soft["window_softmax_frame"](qr_t, kr_win, kr_win, scale)
+
+
+def _soft_window_short(t, F, chunk, radius):
+    lo, hi = _orig_soft["window_bounds"](t, F, chunk, radius)
+    return lo, max(lo, hi - 1)
+
+
+SOFT_MUTANTS = {
+    "softmax_scale_over_d": ("window_softmax_frame", _soft_scale_over_d),
+    "softmax_no_max_shift": ("window_softmax_frame", _soft_no_max_shift),
+    "softmax_columns_normalised": ("window_softmax_frame", _soft_columns_normalised),
+    "softmax_keys_as_values": ("window_softmax_frame", _soft_keys_as_values),
+    "softmax_window_one_frame_short": ("window_bounds", _soft_window_short),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SOFT_MUTANTS))
+def test_planted_softmax_mistake_is_caught(name, monkeypatch):
+    fn, mutant = SOFT_MUTANTS[name]
+    monkeypatch.setattr(O, fn, mutant)
+    tests = [getattr(spins, n) for n in dir(spins) if n.startswith("test_")]
+    caught = 0
+    for t in tests:
+        args = []
+        if getattr(t, "pytestmark", None):
+            params = [m for m in t.pytestmark if m.name == "parametrize"]
+            if params:
+                args = list(params[0].args[1][0]) if isinstance(params[0].args[1][0], tuple) else [params[0].args[1][0]]
+        try:
+            t(*args)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught += 1
+    assert caught > 0, f"no pin fails with mutant {name}"

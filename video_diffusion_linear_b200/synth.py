@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 # draw order / stream ids
-_Q, _K, _V, _BETA, _ALPHA, _GATE, _RMSW, _CONVK, _CONVV, _TEXT = range(10)
+_Q, _K, _V, _BETA, _ALPHA, _GATE, _RMSW, _CONVK, _CONVV, _TEXT, _QR, _KR = range(12)
 _CHUNK = 1 << 22
 
 RULE_IDS = {"sana_scaled": 0, "vdn_solve": 1, "vdn_scaled": 2, "additive": 3}
@@ -97,7 +97,8 @@ def _draw(seed: int, tid: int, shape, kind: str, mu: float, sd: float, dtype: to
     return torch.cat(parts).reshape(shape)
 
 
-def make_inputs(w: Workload, *, threads: int | None = None, with_text: bool | None = None) -> dict:
+def make_inputs(w: Workload, *, threads: int | None = None, with_text: bool | None = None,
+                with_rope_side: bool = False) -> dict:
     """Host (CPU) tensors in the library's argument layout.
 
     q, k, v, gate: [B, F*S, H, d] in the run dtype (token-major, heads interleaved)
@@ -106,6 +107,9 @@ def make_inputs(w: Workload, *, threads: int | None = None, with_text: bool | No
     rms_w:         [d] float32, 1 + 0.1 N(0,1)
     conv_k_w/v_w:  [H, d, K] float32, N(0, 1/K)   (None when K == 1: identity tap)
     text_state:    [H, d, d] float32, 0.5 * R with R ~ N(0, 0.1^2)   (None without text)
+    q_rope, k_rope: [B, F*S, H, d] in the run dtype, N(0, 2^2) and N(0, 1) (only with
+                   with_rope_side: the softmax branch's rotated q / k, drawn as independent
+                   tensors; scores q.k / sqrt(d) then have standard deviation 2)
     """
     threads = threads or min(32, os.cpu_count() or 1)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -134,4 +138,7 @@ def make_inputs(w: Workload, *, threads: int | None = None, with_text: bool | No
                                              torch.float64, pool)).to(f32)
         else:
             out["text_state"] = None
+        if with_rope_side:
+            out["q_rope"] = _draw(w.seed, _QR, (B, N, H, d), "normal", 0.0, 2.0, dt, pool)
+            out["k_rope"] = _draw(w.seed, _KR, (B, N, H, d), "normal", 0.0, 1.0, dt, pool)
     return out
