@@ -211,6 +211,39 @@ vdn_status vdn_feature_prep(const vdn_shape* shape,
  * hi = min(F - 1, chunk (c + radius + 1) - 1).  Host function, no CUDA calls. */
 vdn_status vdn_window_bounds(int t, int F, int chunk, int radius, int* lo, int* hi);
 
+/* Windowed softmax branch of the hybrid attention layer (page: the window
+ * softmax sees the frames near the query, the linear branch the far field, and
+ * the layer adds the two branches).  Every query token of frame t attends to
+ * all tokens of frames lo..hi = vdn_window_bounds(t):
+ *   o = softmax(q_rope k_rope^T * scale) v     (per batch and head, over d)
+ * q_rope, k_rope: the RoPE-rotated q and k of the softmax branch (the rotation
+ * is the caller's), v the shared values, all [B, F*S, H, d] in shape->dtype;
+ * scale <= 0 selects 1/sqrt(d).  accumulate = 0 writes o to out, 1 adds it to
+ * out (which then holds, e.g., the linear branch's output).  out must not
+ * overlap the inputs.  workspace: at least vdn_window_softmax_workspace_size()
+ * bytes (the device status word of the bounded waits), 256-byte aligned;
+ * shape->conv_width is not used.  Asynchronous on `stream`. */
+size_t vdn_window_softmax_workspace_size(const vdn_shape* shape);
+vdn_status vdn_window_softmax_forward(const vdn_shape* shape,
+                                      const void* q_rope, const void* k_rope, const void* v,
+                                      int chunk, int radius, float scale, int accumulate,
+                                      void* workspace, size_t workspace_bytes,
+                                      void* out, void* stream);
+
+/* The hybrid attention layer: out = windowed softmax branch (q_rope, k_rope,
+ * v) + bidirectional linear branch (q, k, v, ... as vdn_branch_forward, whose
+ * workspace this takes).  scale as above. */
+vdn_status vdn_hybrid_forward(const vdn_shape* shape,
+                              const void* q_rope, const void* k_rope,
+                              const void* q, const void* k, const void* v,
+                              const float* beta, const float* alpha,
+                              const void* gate, const float* rms_w,
+                              const float* conv_k_w, const float* conv_v_w,
+                              const float* text_state,
+                              int rule, float c, int chunk, int radius, float scale,
+                              void* workspace, size_t workspace_bytes,
+                              void* out, void* stream);
+
 /* Reads the device status word that bounded waits inside the kernels set (it
  * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
  * Synchronises `stream`. */

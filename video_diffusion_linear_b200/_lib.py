@@ -47,6 +47,12 @@ _SIGNATURES = {
     "vdn_branch_launch_count": (ctypes.c_int, [ctypes.POINTER(VdnShape), ctypes.c_int]),
     "vdn_branch_forward_timed": (ctypes.c_int, _FORWARD_ARGS + [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "vdn_feature_prep": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vdn_window_softmax_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(VdnShape)]),
+    "vdn_window_softmax_forward": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_float, ctypes.c_int, _P, ctypes.c_size_t, _P, _P]),
+    "vdn_hybrid_forward": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                          _P, ctypes.c_size_t, _P, _P]),
     "vdn_window_bounds": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "vdn_workspace_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),

@@ -77,6 +77,39 @@ def branch_forward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=No
     return out
 
 
+def window_softmax_forward(q_rope, k_rope, v, *, F: int, chunk=5, radius=1, scale=0.0, accumulate=False,
+                           out=None, workspace=None, stream=None):
+    """vdn_window_softmax_forward: the windowed softmax branch (out = or += its
+    output).  Returns `out` ([B, F*S, H, d], q_rope's dtype)."""
+    shape = shape_from(q_rope, F)
+    if out is None:
+        out = torch.zeros_like(q_rope) if accumulate else torch.empty_like(q_rope)
+    if workspace is None:
+        workspace = torch.empty(_lib.load().vdn_window_softmax_workspace_size(ctypes.byref(shape)),
+                                dtype=torch.uint8, device=q_rope.device)
+    st = _lib.load().vdn_window_softmax_forward(ctypes.byref(shape), _ptr(q_rope), _ptr(k_rope), _ptr(v), int(chunk),
+                                                int(radius), float(scale), int(bool(accumulate)), _ptr(workspace),
+                                                workspace.numel(), _ptr(out), _stream_ptr(stream))
+    check(st, "vdn_window_softmax_forward")
+    return out
+
+
+def hybrid_forward(q_rope, k_rope, q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None,
+                   text_state=None, *, F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, scale=0.0, out=None,
+                   workspace=None, stream=None):
+    """vdn_hybrid_forward: windowed softmax branch + linear branch.  Returns `out`."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(shape, rule, "auto", q.device)
+    fa = _forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                       radius, workspace, out, stream)
+    st = _lib.load().vdn_hybrid_forward(fa[0], _ptr(q_rope), _ptr(k_rope), *fa[1:15], float(scale), *fa[15:])
+    check(st, "vdn_hybrid_forward")
+    return out
+
+
 def launch_count(shape: VdnShape, impl="auto") -> int:
     return _lib.load().vdn_branch_launch_count(ctypes.byref(shape), VDN_IMPL[impl])
 

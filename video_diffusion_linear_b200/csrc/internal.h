@@ -73,6 +73,11 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
                            int* qexp, bool all_frames, uint32_t* status);
+cudaError_t launch_window_softmax_simt(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
+                                       int radius, float scale, int accumulate, void* out, cudaStream_t stream);
+cudaError_t launch_window_softmax_tc(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
+                                     int radius, float scale, int accumulate, void* out, uint32_t* status,
+                                     cudaStream_t stream);
 cudaError_t launch_readout_tc(const Args& a, const uint16_t* wimg, const int* wexp, const int* wbexp,
                               uint32_t* status);
 

@@ -1,0 +1,426 @@
+// Windowed softmax branch of the hybrid attention layer (page sections on why
+// video models stall on attention and what the far field is): every query token
+// of frame t attends, through the RoPE-rotated q / k, to all tokens of frames
+// lo..hi of its chunk-aligned window, o = softmax(q k^T * scale) v; the linear
+// branch covers the frames outside the window and the layer adds the two.
+//
+// SIMT path (any dtype, d = 16 or 128): a block takes up to 128 query tokens of
+// one window chunk (all share the window), stages 32 keys at a time in shared
+// memory, and every query keeps a running maximum, normaliser and output
+// (online softmax, fp32, exp2 with log2(e) folded into the scale).  A query is
+// spread over d / 16 threads of 16 channels each; its dot products meet by
+// shuffles within those threads.
+//
+// Tensor-core path (bf16, d = 128): one CTA per tile of 128 query tokens of a
+// window chunk, two passes over the window's key tiles of 128.  Pass 1: the
+// tensor cores write S = Q K^T to TMEM (two buffers), the softmax warps read it
+// and keep each row's running maximum and normaliser.  Pass 2: S is computed
+// again; the softmax warps turn it into P = exp(S - m) / l, stored in bf16 as
+// the K-major A operand of O += P V, which accumulates in TMEM.  With the row
+// statistics final before pass 2, O never needs rescaling.  Warp roles (320
+// threads): 0 TMA producer (Q once, then K tiles, and V tiles in pass 2), 1
+// MMA issuer (TMEM owner), 2-9 softmax and epilogue, two threads per query row
+// (64 key columns each; their statistics merge once, after pass 1).
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace vdn {
+
+namespace {
+
+constexpr int kSoftThreads = 128;
+constexpr int kSoftKeys = 32;
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kSoftThreads) k_wsoft_simt(const T* __restrict__ qr, const T* __restrict__ kr,
+                                                            const T* __restrict__ v, int H, int F, int S, int chunk,
+                                                            int radius, int tiles_per_chunk, float scale,
+                                                            int accumulate, T* __restrict__ out) {
+  constexpr int CPT = 16, TPQ = D / CPT, QPB = kSoftThreads / TPQ;
+  __shared__ float ks[kSoftKeys][D], vs[kSoftKeys][D];
+  const int tid = threadIdx.x, qi = tid / TPQ, part = tid % TPQ;
+  const long long bh = blockIdx.x;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const int c = blockIdx.y / tiles_per_chunk, tile = blockIdx.y % tiles_per_chunk;
+  const int f0 = c * chunk;
+  if (f0 >= F) return;
+  const long long N = (long long)F * S;
+  const long long cq0 = (long long)f0 * S, cq1 = (long long)min(F, f0 + chunk) * S;   // queries of the chunk
+  const long long n = cq0 + (long long)tile * QPB + qi;
+  if (cq0 + (long long)tile * QPB >= cq1) return;       // tile past the (shorter) last chunk: whole block leaves
+  const bool valid = n < cq1;
+  int lo, hi;
+  window_bounds(f0, F, chunk, radius, lo, hi);
+  const long long k0 = (long long)lo * S, k1 = (long long)(hi + 1) * S;
+  const float sc = scale * kLog2e;
+
+  float q[CPT], o[CPT];
+  const long long row = ((b * N + (valid ? n : cq0)) * H + h) * D + part * CPT;
+#pragma unroll
+  for (int e = 0; e < CPT; ++e) {
+    q[e] = to_f32(qr[row + e]) * sc;
+    o[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (long long kb = k0; kb < k1; kb += kSoftKeys) {
+    const int nk = (int)min((long long)kSoftKeys, k1 - kb);
+    __syncthreads();
+    for (int e = tid; e < kSoftKeys * D; e += kSoftThreads) {
+      const int j = e / D, ch = e % D;
+      float kv = 0.f, vv = 0.f;
+      if (j < nk) {
+        const long long off = ((b * N + kb + j) * H + h) * D + ch;
+        kv = to_f32(kr[off]);
+        vv = to_f32(v[off]);
+      }
+      ks[j][ch] = kv;
+      vs[j][ch] = vv;
+    }
+    __syncthreads();
+    for (int j = 0; j < nk; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) s = fmaf(q[e], ks[j][part * CPT + e], s);
+#pragma unroll
+      for (int w = 1; w < TPQ; w <<= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
+      const float mn = fmaxf(m, s);
+      const float corr = exp2f(m - mn), p = exp2f(s - mn);
+      l = fmaf(l, corr, p);
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) o[e] = fmaf(o[e], corr, p * vs[j][part * CPT + e]);
+      m = mn;
+    }
+  }
+  if (!valid) return;
+  const float inv = 1.f / l;
+  const long long orow = ((b * N + n) * H + h) * D + part * CPT;
+#pragma unroll
+  for (int e = 0; e < CPT; ++e) {
+    float y = o[e] * inv;
+    if (accumulate) y += to_f32(out[orow + e]);
+    out[orow + e] = from_f32<T>(y);
+  }
+}
+
+cudaError_t launch_window_softmax_simt(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
+                                       int radius, float scale, int accumulate, void* out, cudaStream_t stream) {
+  const int nchunks = (sh.F + chunk - 1) / chunk;
+  const int qpb = kSoftThreads / (sh.d / 16);
+  const int tiles = (int)(((long long)chunk * sh.S + qpb - 1) / qpb);
+  if ((long long)nchunks * tiles > 65535) return cudaErrorInvalidConfiguration;
+  dim3 grid((unsigned)((long long)sh.B * sh.H), (unsigned)(nchunks * tiles));
+#define VDN_WSOFT(D_, T_)                                                                                       \
+  k_wsoft_simt<D_, T_><<<grid, kSoftThreads, 0, stream>>>(                                                   \
+      static_cast<const T_*>(qr), static_cast<const T_*>(kr), static_cast<const T_*>(v), sh.H, sh.F, sh.S, chunk, \
+      radius, tiles, scale, accumulate, static_cast<T_*>(out))
+  if (sh.dtype == VDN_DTYPE_BF16) {
+    VDN_WSOFT(128, __nv_bfloat16);
+  } else if (sh.d == 16) {
+    VDN_WSOFT(16, float);
+  } else {
+    VDN_WSOFT(128, float);
+  }
+#undef VDN_WSOFT
+  return cudaGetLastError();
+}
+
+namespace {
+
+constexpr int kTcThreads = 320;
+constexpr int kKS = 2, kVS = 2;            // K and V tile stages
+constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 128, false, false);   // Q, K tiles: K-major
+constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(128, 128, false, true);    // P K-major, V MN-major
+
+struct __align__(1024) WsoftSmem {
+  uint8_t q[32768];          // Q tile: [channel half][128 rows x 128 B], SW128 (K-major A operand)
+  uint8_t k[kKS][32768];     // K tiles: same layout (K-major B operand)
+  uint8_t v[kVS][32768];     // V tiles: same layout (MN-major B operand of P V)
+  uint8_t p[32768];          // P: [key half][128 rows x 128 B], SW128 (K-major A operand)
+  float stat_m[2][128], stat_l[2][128];
+  uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
+  uint64_t s_full[2], s_empty[2], p_full, p_empty, o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// byte offset of the 16-byte chunk c (0..15) of row r in a 128 x 128 bf16 SW128 tile
+__device__ __forceinline__ uint32_t tile_chunk(int r, int c) {
+  return (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constant__ CUtensorMap tmQ,
+                                                           const __grid_constant__ CUtensorMap tmK,
+                                                           const __grid_constant__ CUtensorMap tmV, int H, int F,
+                                                           int S, int chunk, int radius, int tiles_per_chunk,
+                                                           float scale, int accumulate,
+                                                           __nv_bfloat16* __restrict__ out,
+                                                           uint32_t* __restrict__ status) {
+  const long long bh = blockIdx.x;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const int c = blockIdx.y / tiles_per_chunk, tile = blockIdx.y % tiles_per_chunk;
+  const int f0 = c * chunk;
+  if (f0 >= F) return;
+  const long long N = (long long)F * S;
+  const long long cq1 = (long long)min(F, f0 + chunk) * S;
+  const long long q0 = (long long)f0 * S + 128LL * tile;      // first query token of the tile
+  if (q0 >= cq1) return;                                     // past the (shorter) last chunk
+  int lo, hi;
+  window_bounds(f0, F, chunk, radius, lo, hi);
+  const long long k0 = (long long)lo * S, k1 = (long long)(hi + 1) * S;
+  const int nkt = (int)((k1 - k0 + 127) / 128);
+
+  extern __shared__ uint8_t smem_raw[];
+  WsoftSmem& sm = *reinterpret_cast<WsoftSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort;
+  if (tid == 0) {
+    tc::mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kKS; ++s) {
+      tc::mbar_init(&sm.k_full[s], 1);
+      tc::mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      tc::mbar_init(&sm.v_full[s], 1);
+      tc::mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&sm.s_full[s], 1);
+      tc::mbar_init(&sm.s_empty[s], 8);
+    }
+    tc::mbar_init(&sm.p_full, 8);
+    tc::mbar_init(&sm.p_empty, 1);
+    tc::mbar_init(&sm.o_full, 1);
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;       // S buffers at columns 0 and 128, O at 256
+  const int rowq = (int)(b * N + q0), rowk = (int)(b * N + k0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&sm.q_full, 32768);
+      tc::tma_load_3d(&tmQ, &sm.q_full, sm.q, 0, h, rowq);
+      tc::tma_load_3d(&tmQ, &sm.q_full, sm.q + 16384, 64, h, rowq);
+      int ik = 0, iv = 0;
+      for (int pass = 0; pass < 2; ++pass) {
+        bool ok = true;
+        for (int j = 0; j < nkt && ok; ++j) {
+          const int ks = ik % kKS;
+          if (!tc::mbar_wait(&sm.k_empty[ks], ((ik / kKS) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&sm.k_full[ks], 32768);
+          tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks], 0, h, rowk + 128 * j);
+          tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks] + 16384, 64, h, rowk + 128 * j);
+          ++ik;
+          if (pass == 1) {
+            const int vs = iv % kVS;
+            if (!tc::mbar_wait(&sm.v_empty[vs], ((iv / kVS) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+            tc::mbar_arrive_expect_tx(&sm.v_full[vs], 32768);
+            tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs], 0, h, rowk + 128 * j);
+            tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs] + 16384, 64, h, rowk + 128 * j);
+            ++iv;
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t aq = tc::smem_u32(sm.q), ap = tc::smem_u32(sm.p);
+      int ik = 0, iv = 0, is = 0;
+      bool ok = tc::mbar_wait(&sm.q_full, 0, abort_flag, status);
+      auto qk = [&]() -> bool {   // S = Q K^T for the next K tile into the next S buffer
+        const int ks = ik % kKS, sb = is % 2;
+        if (!tc::mbar_wait(&sm.k_full[ks], (ik / kKS) & 1, abort_flag, status)) return false;
+        if (!tc::mbar_wait(&sm.s_empty[sb], ((is / 2) & 1) ^ 1, abort_flag, status)) return false;
+        tc::tc_fence_after();
+        const uint32_t bk = tc::smem_u32(sm.k[ks]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::umma_bf16(tmem + sb * 128, tc::smem_desc(aq + off, 16, 1024), tc::smem_desc(bk + off, 16, 1024),
+                        kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(&sm.s_full[sb]);
+        tc::umma_commit(&sm.k_empty[ks]);
+        ++ik;
+        ++is;
+        return true;
+      };
+      auto pv = [&](int j) -> bool {   // O += P_j V_j
+        const int vs = iv % kVS;
+        if (!tc::mbar_wait(&sm.p_full, j & 1, abort_flag, status)) return false;
+        if (!tc::mbar_wait(&sm.v_full[vs], (iv / kVS) & 1, abort_flag, status)) return false;
+        tc::tc_fence_after();
+        const uint32_t bv = tc::smem_u32(sm.v[vs]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          tc::umma_bf16(tmem + 256, tc::smem_desc(ap + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        tc::smem_desc(bv + kk * 2048, 16384, 1024), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::umma_commit(&sm.p_empty);
+        tc::umma_commit(&sm.v_empty[vs]);
+        ++iv;
+        return true;
+      };
+      for (int j = 0; j < nkt && ok; ++j) ok = qk();                 // pass 1
+      for (int j = 0; j < nkt && ok; ++j) {                          // pass 2, P V one tile behind
+        ok = qk();
+        if (ok && j > 0) ok = pv(j - 1);
+      }
+      if (ok && nkt > 0) ok = pv(nkt - 1);
+      if (ok) tc::umma_commit(&sm.o_full);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3, hf = (warp - 2) >> 2;
+    const int m = 32 * quarter + lane;                 // query row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    int is = 0;
+    float mrun = -INFINITY, lrun = 0.f;
+    bool ok = true;
+    auto load_s = [&](uint32_t (&r)[64]) -> bool {     // this thread's 64 columns of the next S buffer
+      const int sb = is % 2;
+      if (!tc::mbar_wait(&sm.s_full[sb], (is / 2) & 1, abort_flag, status)) return false;
+      tc::tc_fence_after();
+      uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+      uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+      tc::tmem_ld32(tmem + sb * 128 + 64 * hf + lane_off, r0);
+      tc::tmem_ld32(tmem + sb * 128 + 64 * hf + 32 + lane_off, r1);
+      tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.s_empty[sb]);
+      ++is;
+      return true;
+    };
+    // pass 1: running maximum and normaliser of this thread's columns (scaled by log2 e)
+    for (int j = 0; j < nkt && ok; ++j) {
+      uint32_t r[64];
+      if (!(ok = load_s(r))) break;
+      const int nvalid = (int)min(64LL, max(0LL, k1 - (k0 + 128LL * j + 64 * hf)));
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]) * scale);
+      const float mn = fmaxf(mrun, tmax);
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (e < nvalid) sum += exp2f(__uint_as_float(r[e]) * scale - mn);
+      lrun = (mrun == -INFINITY ? 0.f : lrun * exp2f(mrun - mn)) + sum;   // no keys yet: nothing to rescale
+      mrun = mn;
+    }
+    // merge the two halves of each row
+    sm.stat_m[hf][m] = mrun;
+    sm.stat_l[hf][m] = lrun;
+    tc::named_bar(1, 256);
+    const float m0 = sm.stat_m[0][m], m1 = sm.stat_m[1][m];
+    const float mf = fmaxf(m0, m1);
+    // a half that saw no key (m = -inf, l = 0) adds nothing
+    const float lf = (m0 == -INFINITY ? 0.f : sm.stat_l[0][m] * exp2f(m0 - mf)) +
+                     (m1 == -INFINITY ? 0.f : sm.stat_l[1][m] * exp2f(m1 - mf));
+    const float inv_l = 1.f / lf;
+    // pass 2: P = exp(S - m) / l into the A operand of P V
+    for (int j = 0; j < nkt && ok; ++j) {
+      uint32_t r[64];
+      if (!(ok = load_s(r))) break;
+      const int nvalid = (int)min(64LL, max(0LL, k1 - (k0 + 128LL * j + 64 * hf)));
+      uint32_t pw[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        const float p0 = e < nvalid ? exp2f(__uint_as_float(r[e]) * scale - mf) * inv_l : 0.f;
+        const float p1 = e + 1 < nvalid ? exp2f(__uint_as_float(r[e + 1]) * scale - mf) * inv_l : 0.f;
+        pw[e / 2] = pack_bf16x2(p0, p1);
+      }
+      if (!(ok = tc::mbar_wait(&sm.p_empty, (j & 1) ^ 1, abort_flag, status))) break;
+#pragma unroll
+      for (int cq = 0; cq < 8; ++cq)
+        *reinterpret_cast<uint4*>(sm.p + tile_chunk(m, 8 * hf + cq)) =
+            make_uint4(pw[4 * cq], pw[4 * cq + 1], pw[4 * cq + 2], pw[4 * cq + 3]);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.p_full);
+    }
+    // epilogue: this thread's 64 output channels of its row
+    if (ok && tc::mbar_wait(&sm.o_full, 0, abort_flag, status)) {
+      tc::tc_fence_after();
+      uint32_t o[64];
+      {
+        uint32_t (&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+        uint32_t (&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+        tc::tmem_ld32(tmem + 256 + 64 * hf + lane_off, o0);
+        tc::tmem_ld32(tmem + 256 + 64 * hf + 32 + lane_off, o1);
+        tc::tmem_ld_wait();
+      }
+      if (q0 + m < cq1) {
+        uint4* dst = reinterpret_cast<uint4*>(out + ((b * N + q0 + m) * H + h) * 128 + 64 * hf);
+#pragma unroll
+        for (int cq = 0; cq < 8; ++cq) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(o[8 * cq + e]);
+          if (accumulate) {
+            const uint4 prev = dst[cq];
+            const uint32_t pv4[4] = {prev.x, prev.y, prev.z, prev.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              y[2 * e] += bf16lo(pv4[e]);
+              y[2 * e + 1] += bf16hi(pv4[e]);
+            }
+          }
+          dst[cq] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                               pack_bf16x2(y[6], y[7]));
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_window_softmax_tc(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
+                                     int radius, float scale, int accumulate, void* out, uint32_t* status,
+                                     cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  const long long rows = (long long)sh.B * sh.F * sh.S;
+  if (rows > 0x7fffffffLL - 256) return cudaErrorInvalidValue;
+  if (!tmap_token_rows_bf16(&tq, qr, sh.d, sh.H, rows, 128) || !tmap_token_rows_bf16(&tk, kr, sh.d, sh.H, rows, 128) ||
+      !tmap_token_rows_bf16(&tv, v, sh.d, sh.H, rows, 128))
+    return cudaErrorInvalidValue;
+  const int nchunks = (sh.F + chunk - 1) / chunk;
+  const int tiles = (int)(((long long)chunk * sh.S + 127) / 128);
+  if ((long long)nchunks * tiles > 65535) return cudaErrorInvalidConfiguration;
+  const size_t smem = sizeof(WsoftSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_wsoft_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((long long)sh.B * sh.H), (unsigned)(nchunks * tiles));
+  k_wsoft_tc<<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, sh.H, sh.F, sh.S, chunk, radius, tiles,
+                                                 scale * kLog2e, accumulate, static_cast<__nv_bfloat16*>(out),
+                                                 status);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

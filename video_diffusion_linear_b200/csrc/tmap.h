@@ -39,6 +39,22 @@ inline bool tmap_tokens_bf16(CUtensorMap* m, const void* base, int d, int H, int
   return r == CUDA_SUCCESS;
 }
 
+// Token tensor [rows][H heads][d] of 16-bit elements (rows = batch x tokens,
+// frames back to back), viewed as 3-D (d, H, rows); box {64 channels, 1 head,
+// box_rows rows}, 128-byte swizzle.  Rows past the end read as zero.
+inline bool tmap_token_rows_bf16(CUtensorMap* m, const void* base, int d, int H, long long rows, int box_rows) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // fp32 matrices [rows][128] viewed 2-D; box {32 columns, 128 rows}, 128-byte swizzle.
 inline bool tmap_rows_f32(CUtensorMap* m, const void* base, long long rows) {
   auto enc = tmap_encoder();

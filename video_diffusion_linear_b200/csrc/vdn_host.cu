@@ -247,6 +247,40 @@ vdn_status forward_common(const vdn_shape* shape, const void* q, const void* k, 
   return run_forward(a, workspace, impl, events);
 }
 
+vdn_status check_softmax_args(const vdn_shape* sh, const void* qr, const void* kr, const void* v, int chunk,
+                              int radius, float scale, int accumulate, const void* workspace,
+                              size_t workspace_bytes, size_t need, const void* out) {
+  vdn_status s = check_shape(sh);
+  if (s != VDN_OK) return s;
+  if (chunk < 1 || radius < 0 || !std::isfinite(scale) || (accumulate != 0 && accumulate != 1))
+    return VDN_ERR_INVALID_ARG;
+  if (!qr || !kr || !v || !out || !workspace) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {qr, kr, v, out};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  if (!aligned(workspace, 256)) return VDN_ERR_ALIGNMENT;
+  if (workspace_bytes < need) return VDN_ERR_WORKSPACE;
+  const size_t big = (size_t)sh->B * sh->F * sh->S * sh->H * sh->d * elem_size(sh->dtype);
+  const Range ro{(uintptr_t)out, (uintptr_t)out + big};
+  const Range rin[] = {{(uintptr_t)qr, (uintptr_t)qr + big},
+                       {(uintptr_t)kr, (uintptr_t)kr + big},
+                       {(uintptr_t)v, (uintptr_t)v + big},
+                       {(uintptr_t)workspace, (uintptr_t)workspace + need}};
+  for (const Range& r : rin)
+    if (overlap(ro, r)) return VDN_ERR_INVALID_ARG;
+  return VDN_OK;
+}
+
+vdn_status run_window_softmax(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
+                              int radius, float scale, int accumulate, uint32_t* status, void* out,
+                              cudaStream_t stream) {
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)sh.d);
+  cudaError_t e = (sh.dtype == VDN_DTYPE_BF16 && sh.d == 128 && VDN_HAVE_TC)
+                      ? launch_window_softmax_tc(sh, qr, kr, v, chunk, radius, sc, accumulate, out, status, stream)
+                      : launch_window_softmax_simt(sh, qr, kr, v, chunk, radius, sc, accumulate, out, stream);
+  return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -319,6 +353,38 @@ vdn_status vdn_feature_prep(const vdn_shape* shape, const void* q, const void* k
     return VDN_ERR_INVALID_ARG;
   cudaError_t e = launch_feature_prep(*shape, q, k, v, conv_k_w, conv_v_w, q_out, k_out, v_out, (cudaStream_t)stream);
   return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+size_t vdn_window_softmax_workspace_size(const vdn_shape* shape) {
+  return check_shape(shape) == VDN_OK ? 256 : 0;
+}
+
+vdn_status vdn_window_softmax_forward(const vdn_shape* shape, const void* q_rope, const void* k_rope, const void* v,
+                                      int chunk, int radius, float scale, int accumulate, void* workspace,
+                                      size_t workspace_bytes, void* out, void* stream) {
+  vdn_status s = check_softmax_args(shape, q_rope, k_rope, v, chunk, radius, scale, accumulate, workspace,
+                                    workspace_bytes, 256, out);
+  if (s != VDN_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return VDN_ERR_CUDA;
+  return run_window_softmax(*shape, q_rope, k_rope, v, chunk, radius, scale, accumulate,
+                            static_cast<uint32_t*>(workspace), out, st);
+}
+
+vdn_status vdn_hybrid_forward(const vdn_shape* shape, const void* q_rope, const void* k_rope, const void* q,
+                              const void* k, const void* v, const float* beta, const float* alpha, const void* gate,
+                              const float* rms_w, const float* conv_k_w, const float* conv_v_w,
+                              const float* text_state, int rule, float c, int chunk, int radius, float scale,
+                              void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  vdn_status s = check_softmax_args(shape, q_rope, k_rope, v, chunk, radius, scale, 1, workspace, workspace_bytes,
+                                    256, out);
+  if (s != VDN_OK) return s;
+  // the linear branch validates the rest and writes out; the softmax branch adds to it
+  s = forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                     radius, workspace, workspace_bytes, out, stream, nullptr);
+  if (s != VDN_OK) return s;
+  return run_window_softmax(*shape, q_rope, k_rope, v, chunk, radius, scale, 1, static_cast<uint32_t*>(workspace),
+                            out, (cudaStream_t)stream);
 }
 
 vdn_status vdn_window_bounds(int t, int F, int chunk, int radius, int* lo, int* hi) {
