@@ -34,6 +34,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 2^x by the hardware approximation (one MUFU op; relative error about 2^-22,
+// 2^-inf = 0), for the softmax weights that are rounded to bf16 afterwards
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 2^e for e in [-126, 127], built from the exponent field (exact)
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
 

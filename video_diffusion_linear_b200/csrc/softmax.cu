@@ -324,8 +324,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       float sum = 0.f;
 #pragma unroll
       for (int e = 0; e < 64; ++e)
-        if (e < nvalid) sum += exp2f(__uint_as_float(r[e]) * scale - mn);
-      lrun = (mrun == -INFINITY ? 0.f : lrun * exp2f(mrun - mn)) + sum;   // no keys yet: nothing to rescale
+        if (e < nvalid) sum += ex2_approx(__uint_as_float(r[e]) * scale - mn);
+      lrun = (mrun == -INFINITY ? 0.f : lrun * ex2_approx(mrun - mn)) + sum;   // no keys yet: nothing to rescale
       mrun = mn;
     }
     // merge the two halves of each row
@@ -346,8 +346,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       uint32_t pw[32];
 #pragma unroll
       for (int e = 0; e < 64; e += 2) {
-        const float p0 = e < nvalid ? exp2f(__uint_as_float(r[e]) * scale - mf) * inv_l : 0.f;
-        const float p1 = e + 1 < nvalid ? exp2f(__uint_as_float(r[e + 1]) * scale - mf) * inv_l : 0.f;
+        const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mf) * inv_l : 0.f;
+        const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mf) * inv_l : 0.f;
         pw[e / 2] = pack_bf16x2(p0, p1);
       }
       if (!(ok = tc::mbar_wait(&sm.p_empty, (j & 1) ^ 1, abort_flag, status))) break;
