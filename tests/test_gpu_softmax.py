@@ -92,3 +92,20 @@ def test_480p_sampled_tokens():
         g = got[b, torch.as_tensor(toks, device=got.device), h, :].float().cpu().numpy().astype(np.float64)
         assert rel_err(g, ref) <= TOL_BF16, (b, h, rel_err(g, ref))
     assert torch.isfinite(got.float()).all()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_scores_rising_along_the_window(dtype):
+    # key norms grow along the sequence, so a row's running maximum keeps rising from key
+    # tile to key tile: the tensor-core path must bring O and the normaliser to each new
+    # reference maximum (and stays exact when it does not move)
+    w = synth.Workload("sm_rising", B=1, H=2, d=128, F=10, S=96, dtype=dtype, alpha_mu=2.0, text=False, seed=47,
+                       chunk=5, radius=1)
+    inp = synth.make_inputs(w, with_rope_side=True)
+    N = w.F * w.S
+    ramp = torch.linspace(0.2, 6.0, N, dtype=torch.float64).view(1, N, 1, 1)
+    inp["k_rope"] = (inp["k_rope"].double() * ramp).to(inp["k_rope"].dtype)
+    got = _run(w, inp)
+    ref = O.window_softmax_forward(inp, w.F, w.S, w.chunk, w.radius)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    assert rel_err(to_np(got), ref) <= tol, rel_err(to_np(got), ref)

@@ -134,6 +134,7 @@ namespace {
 
 constexpr int kTcThreads = 320;
 constexpr int kKS = 2, kVS = 2;            // K and V tile stages
+constexpr float kRescaleAbove = 8.f;      // log2 units: the running maximum moves only when a score exceeds it by 2^8
 constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 128, false, false);   // Q, K tiles: K-major
 constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(128, 128, false, true);    // P K-major, V MN-major
 
@@ -142,7 +143,8 @@ struct __align__(1024) WsoftSmem {
   uint8_t k[kKS][32768];     // K tiles: same layout (K-major B operand)
   uint8_t v[kVS][32768];     // V tiles: same layout (MN-major B operand of P V)
   uint8_t p[32768];          // P: [key half][128 rows x 128 B], SW128 (K-major A operand)
-  float stat_m[2][128], stat_l[2][128];
+  float xmax[2][2][128];      // [tile parity][column half][row]: tile maxima exchanged between the two halves
+  float stat_l[2][128];
   uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
   uint64_t s_full[2], s_empty[2], p_full, p_empty, o_full;
   uint32_t tmem_base;
@@ -218,26 +220,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       tc::mbar_arrive_expect_tx(&sm.q_full, 32768);
       tc::tma_load_3d(&tmQ, &sm.q_full, sm.q, 0, h, rowq);
       tc::tma_load_3d(&tmQ, &sm.q_full, sm.q + 16384, 64, h, rowq);
-      int ik = 0, iv = 0;
-      for (int pass = 0; pass < 2; ++pass) {
-        bool ok = true;
-        for (int j = 0; j < nkt && ok; ++j) {
-          const int ks = ik % kKS;
-          if (!tc::mbar_wait(&sm.k_empty[ks], ((ik / kKS) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-          tc::mbar_arrive_expect_tx(&sm.k_full[ks], 32768);
-          tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks], 0, h, rowk + 128 * j);
-          tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks] + 16384, 64, h, rowk + 128 * j);
-          ++ik;
-          if (pass == 1) {
-            const int vs = iv % kVS;
-            if (!tc::mbar_wait(&sm.v_empty[vs], ((iv / kVS) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-            tc::mbar_arrive_expect_tx(&sm.v_full[vs], 32768);
-            tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs], 0, h, rowk + 128 * j);
-            tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs] + 16384, 64, h, rowk + 128 * j);
-            ++iv;
-          }
-        }
-        if (!ok) break;
+      for (int j = 0; j < nkt; ++j) {
+        const int ks = j % kKS, vs = j % kVS;
+        if (!tc::mbar_wait(&sm.k_empty[ks], ((j / kKS) & 1) ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.k_full[ks], 32768);
+        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks], 0, h, rowk + 128 * j);
+        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks] + 16384, 64, h, rowk + 128 * j);
+        if (!tc::mbar_wait(&sm.v_empty[vs], ((j / kVS) & 1) ^ 1, abort_flag, status)) break;
+        tc::mbar_arrive_expect_tx(&sm.v_full[vs], 32768);
+        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs], 0, h, rowk + 128 * j);
+        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs] + 16384, 64, h, rowk + 128 * j);
       }
     }
   } else if (warp == 1) {
@@ -280,12 +272,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         ++iv;
         return true;
       };
-      for (int j = 0; j < nkt && ok; ++j) ok = qk();                 // pass 1
-      for (int j = 0; j < nkt && ok; ++j) {                          // pass 2, P V one tile behind
-        ok = qk();
-        if (ok && j > 0) ok = pv(j - 1);
+      // S for tile j+1 is computed while the softmax warps turn S_j into P_j
+      if (ok && nkt > 0) ok = qk();
+      for (int j = 0; j < nkt && ok; ++j) {
+        if (j + 1 < nkt) ok = qk();
+        if (ok) ok = pv(j);
       }
-      if (ok && nkt > 0) ok = pv(nkt - 1);
       if (ok) tc::umma_commit(&sm.o_full);
     }
   } else {
@@ -294,7 +286,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
     const int m = 32 * quarter + lane;                 // query row = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     int is = 0;
-    float mrun = -INFINITY, lrun = 0.f;
+    // mref: the reference maximum (log2 units) that every exponent of this row is taken against; it
+    // moves only when a tile's maximum exceeds it by more than 2^8, and then O and l are rescaled
+    float mref = -INFINITY, lrun = 0.f;
     bool ok = true;
     auto load_s = [&](uint32_t (&r)[64]) -> bool {     // this thread's 64 columns of the next S buffer
       const int sb = is % 2;
@@ -311,7 +305,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       ++is;
       return true;
     };
-    // pass 1: running maximum and normaliser of this thread's columns (scaled by log2 e)
     for (int j = 0; j < nkt && ok; ++j) {
       uint32_t r[64];
       if (!(ok = load_s(r))) break;
@@ -319,38 +312,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       float tmax = -INFINITY;
 #pragma unroll
       for (int e = 0; e < 64; ++e)
-        if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]) * scale);
-      const float mn = fmaxf(mrun, tmax);
+        if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
+      // the row's maximum over both column halves (the warp with the same TMEM lanes holds the other)
+      sm.xmax[j & 1][hf][m] = tmax;
+      tc::named_bar(2 + quarter, 64);
+      const float mt = fmaxf(tmax, sm.xmax[j & 1][hf ^ 1][m]) * scale;
+      float corr = 1.f;
+      const bool move = mt > mref + kRescaleAbove;
+      if (move) {
+        corr = mref == -INFINITY ? 0.f : ex2_approx(mref - mt);
+        lrun *= corr;
+        mref = mt;
+      }
+      uint32_t pw[32];
       float sum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (e < nvalid) sum += ex2_approx(__uint_as_float(r[e]) * scale - mn);
-      lrun = (mrun == -INFINITY ? 0.f : lrun * ex2_approx(mrun - mn)) + sum;   // no keys yet: nothing to rescale
-      mrun = mn;
-    }
-    // merge the two halves of each row
-    sm.stat_m[hf][m] = mrun;
-    sm.stat_l[hf][m] = lrun;
-    tc::named_bar(1, 256);
-    const float m0 = sm.stat_m[0][m], m1 = sm.stat_m[1][m];
-    const float mf = fmaxf(m0, m1);
-    // a half that saw no key (m = -inf, l = 0) adds nothing
-    const float lf = (m0 == -INFINITY ? 0.f : sm.stat_l[0][m] * exp2f(m0 - mf)) +
-                     (m1 == -INFINITY ? 0.f : sm.stat_l[1][m] * exp2f(m1 - mf));
-    const float inv_l = 1.f / lf;
-    // pass 2: P = exp(S - m) / l into the A operand of P V
-    for (int j = 0; j < nkt && ok; ++j) {
-      uint32_t r[64];
-      if (!(ok = load_s(r))) break;
-      const int nvalid = (int)min(64LL, max(0LL, k1 - (k0 + 128LL * j + 64 * hf)));
-      uint32_t pw[32];
-#pragma unroll
       for (int e = 0; e < 64; e += 2) {
-        const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mf) * inv_l : 0.f;
-        const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mf) * inv_l : 0.f;
+        const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mref) : 0.f;
+        const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mref) : 0.f;
+        sum += p0 + p1;
         pw[e / 2] = pack_bf16x2(p0, p1);
       }
+      lrun += sum;
+      // P_{j-1} V_{j-1} has completed once the P buffer is free
       if (!(ok = tc::mbar_wait(&sm.p_empty, (j & 1) ^ 1, abort_flag, status))) break;
+      // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any of its
+      // rows moved (corr = 1 for the others)
+      if (__any_sync(0xffffffffu, move) && j > 0) {
+        // the reference maximum moved: bring this thread's half of the O row to the new reference
+        tc::tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          uint32_t o[32];
+          const uint32_t taddr = tmem + 256 + 64 * hf + 32 * part + lane_off;
+          tc::tmem_ld32(taddr, o);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+          tc::tmem_st32(taddr, o);
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+      }
 #pragma unroll
       for (int cq = 0; cq < 8; ++cq)
         *reinterpret_cast<uint4*>(sm.p + tile_chunk(m, 8 * hf + cq)) =
@@ -359,6 +362,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.p_full);
     }
+    // the row's normaliser: both halves used the same reference maximum
+    sm.stat_l[hf][m] = lrun;
+    tc::named_bar(2 + quarter, 64);
+    const float inv_l = 1.f / (lrun + sm.stat_l[hf ^ 1][m]);
     // epilogue: this thread's 64 output channels of its row
     if (ok && tc::mbar_wait(&sm.o_full, 0, abort_flag, status)) {
       tc::tc_fence_after();
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         for (int cq = 0; cq < 8; ++cq) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(o[8 * cq + e]);
+          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(o[8 * cq + e]) * inv_l;
           if (accumulate) {
             const uint4 prev = dst[cq];
             const uint32_t pv4[4] = {prev.x, prev.y, prev.z, prev.w};
