@@ -143,10 +143,9 @@ struct __align__(1024) WsoftSmem {
   uint8_t k[kKS][32768];     // K tiles: same layout (K-major B operand)
   uint8_t v[kVS][32768];     // V tiles: same layout (MN-major B operand of P V)
   uint8_t p[32768];          // P: [key half][128 rows x 128 B], SW128 (K-major A operand)
-  float xmax[2][2][128];      // [tile parity][column half][row]: tile maxima exchanged between the two halves
-  float stat_l[2][128];
+  float stat_m[2][128], stat_l[2][128];   // [key half][row]: reference maxima and normalisers
   uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
-  uint64_t s_full[2], s_empty[2], p_full, p_empty, o_full;
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full;
   uint32_t tmem_base;
   int abort;
 };
@@ -198,8 +197,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       tc::mbar_init(&sm.s_full[s], 1);
       tc::mbar_init(&sm.s_empty[s], 8);
     }
-    tc::mbar_init(&sm.p_full, 8);
-    tc::mbar_init(&sm.p_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&sm.p_full[s], 4);
+      tc::mbar_init(&sm.p_empty[s], 1);
+    }
     tc::mbar_init(&sm.o_full, 1);
     sm.abort = 0;
     tc::fence_barrier_init();
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;       // S buffers at columns 0 and 128, O at 256
+  const uint32_t tmem = sm.tmem_base;       // S buffers at columns 0 and 128, O_0 at 256, O_1 at 384
   const int rowq = (int)(b * N + q0), rowk = (int)(b * N + k0);
 
   if (warp == 0) {
@@ -256,18 +257,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         ++is;
         return true;
       };
-      auto pv = [&](int j) -> bool {   // O += P_j V_j
+      auto pv = [&](int j) -> bool {   // O_hf += P_j[:, keys of half hf] V_j[keys of half hf, :]
         const int vs = iv % kVS;
-        if (!tc::mbar_wait(&sm.p_full, j & 1, abort_flag, status)) return false;
         if (!tc::mbar_wait(&sm.v_full[vs], (iv / kVS) & 1, abort_flag, status)) return false;
-        tc::tc_fence_after();
         const uint32_t bv = tc::smem_u32(sm.v[vs]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          tc::umma_bf16(tmem + 256, tc::smem_desc(ap + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        tc::smem_desc(bv + kk * 2048, 16384, 1024), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!tc::mbar_wait(&sm.p_full[hf], j & 1, abort_flag, status)) return false;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            tc::umma_bf16(tmem + 256 + 128 * hf, tc::smem_desc(ap + hf * 16384 + kk * 32, 16, 1024),
+                          tc::smem_desc(bv + (4 * hf + kk) * 2048, 16384, 1024), kIdescPV,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::umma_commit(&sm.p_empty[hf]);
         }
-        tc::umma_commit(&sm.p_empty);
         tc::umma_commit(&sm.v_empty[vs]);
         ++iv;
         return true;
@@ -286,8 +291,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
     const int m = 32 * quarter + lane;                 // query row = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     int is = 0;
-    // mref: the reference maximum (log2 units) that every exponent of this row is taken against; it
-    // moves only when a tile's maximum exceeds it by more than 2^8, and then O and l are rescaled
+    // Each key half (columns 64 hf .. 64 hf + 63 of every S tile) keeps its own accumulator O_hf, so
+    // the two warps on a row never wait for each other inside the loop.  mref: the reference maximum
+    // (log2 units) that every exponent of this row's half is taken against; it moves only when a
+    // tile's maximum exceeds it by more than 2^8, and then O_hf and l are rescaled
     float mref = -INFINITY, lrun = 0.f;
     bool ok = true;
     auto load_s = [&](uint32_t (&r)[64]) -> bool {     // this thread's 64 columns of the next S buffer
@@ -309,14 +316,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       uint32_t r[64];
       if (!(ok = load_s(r))) break;
       const int nvalid = (int)min(64LL, max(0LL, k1 - (k0 + 128LL * j + 64 * hf)));
-      float tmax = -INFINITY;
+      float tmax;
+      if (nvalid == 64) {                     // every tile but the window's last: a tree of maxima
+        float t8[8];
 #pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
-      // the row's maximum over both column halves (the warp with the same TMEM lanes holds the other)
-      sm.xmax[j & 1][hf][m] = tmax;
-      tc::named_bar(2 + quarter, 64);
-      const float mt = fmaxf(tmax, sm.xmax[j & 1][hf ^ 1][m]) * scale;
+        for (int a = 0; a < 8; ++a) t8[a] = __uint_as_float(r[a]);
+#pragma unroll
+        for (int e = 8; e < 64; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(r[e]));
+        tmax = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+      } else {
+        tmax = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
+      }
+      const float mt = tmax * scale;
       float corr = 1.f;
       const bool move = mt > mref + kRescaleAbove;
       if (move) {
@@ -325,26 +339,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         mref = mt;
       }
       uint32_t pw[32];
-      float sum = 0.f;
+      float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
       for (int e = 0; e < 64; e += 2) {
         const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mref) : 0.f;
         const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mref) : 0.f;
-        sum += p0 + p1;
+        sum0 += p0;
+        sum1 += p1;
         pw[e / 2] = pack_bf16x2(p0, p1);
       }
-      lrun += sum;
-      // P_{j-1} V_{j-1} has completed once the P buffer is free
-      if (!(ok = tc::mbar_wait(&sm.p_empty, (j & 1) ^ 1, abort_flag, status))) break;
+      lrun += sum0 + sum1;
+      // this half's P_{j-1} V_{j-1} has completed once its P buffer is free
+      if (!(ok = tc::mbar_wait(&sm.p_empty[hf], (j & 1) ^ 1, abort_flag, status))) break;
       // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any of its
       // rows moved (corr = 1 for the others)
       if (__any_sync(0xffffffffu, move) && j > 0) {
-        // the reference maximum moved: bring this thread's half of the O row to the new reference
+        // the reference maximum moved: bring this half's O row to the new reference
         tc::tc_fence_after();
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < 4; ++part) {
           uint32_t o[32];
-          const uint32_t taddr = tmem + 256 + 64 * hf + 32 * part + lane_off;
+          const uint32_t taddr = tmem + 256 + 128 * hf + 32 * part + lane_off;
           tc::tmem_ld32(taddr, o);
           tc::tmem_ld_wait();
 #pragma unroll
@@ -360,22 +375,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
             make_uint4(pw[4 * cq], pw[4 * cq + 1], pw[4 * cq + 2], pw[4 * cq + 3]);
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.p_full);
+      if (lane == 0) tc::mbar_arrive(&sm.p_full[hf]);
     }
-    // the row's normaliser: both halves used the same reference maximum
+    // combine the two key halves of the row: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l
+    sm.stat_m[hf][m] = mref;
     sm.stat_l[hf][m] = lrun;
     tc::named_bar(2 + quarter, 64);
-    const float inv_l = 1.f / (lrun + sm.stat_l[hf ^ 1][m]);
+    const float m0 = sm.stat_m[0][m], m1 = sm.stat_m[1][m];
+    const float mx = fmaxf(m0, m1);
+    const float w0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mx), w1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mx);
+    const float inv_l = 1.f / (sm.stat_l[0][m] * w0 + sm.stat_l[1][m] * w1);
+    const float c0 = w0 * inv_l, c1 = w1 * inv_l;
     // epilogue: this thread's 64 output channels of its row
     if (ok && tc::mbar_wait(&sm.o_full, 0, abort_flag, status)) {
       tc::tc_fence_after();
-      uint32_t o[64];
-      {
-        uint32_t (&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-        uint32_t (&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
-        tc::tmem_ld32(tmem + 256 + 64 * hf + lane_off, o0);
-        tc::tmem_ld32(tmem + 256 + 64 * hf + 32 + lane_off, o1);
+      float o[64];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        uint32_t a0[32], a1[32];
+        tc::tmem_ld32(tmem + 256 + 64 * hf + 32 * part + lane_off, a0);
+        tc::tmem_ld32(tmem + 384 + 64 * hf + 32 * part + lane_off, a1);
         tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[32 * part + e] = __uint_as_float(a0[e]) * c0 + __uint_as_float(a1[e]) * c1;
       }
       if (q0 + m < cq1) {
         uint4* dst = reinterpret_cast<uint4*>(out + ((b * N + q0 + m) * H + h) * 128 + 64 * hf);
@@ -383,7 +405,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         for (int cq = 0; cq < 8; ++cq) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(o[8 * cq + e]) * inv_l;
+          for (int e = 0; e < 8; ++e) y[e] = o[8 * cq + e];
           if (accumulate) {
             const uint4 prev = dst[cq];
             const uint32_t pv4[4] = {prev.x, prev.y, prev.z, prev.w};
