@@ -134,21 +134,29 @@ namespace {
 
 constexpr int kTcThreads = 320;
 constexpr int kKS = 2, kVS = 2;            // K and V tile stages
-constexpr float kRescaleAbove = 8.f;      // log2 units: the running maximum moves only when a score exceeds it by 2^8
+constexpr float kRescaleAbove = 8.f;      // log2 units: a reference maximum moves only when a score exceeds it by 2^8
 constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 128, false, false);   // Q, K tiles: K-major
 constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(128, 128, false, true);    // P K-major, V MN-major
 
+// Key tiles alternate between two groups of four softmax warps (group g takes the tiles j with
+// j % 2 == g).  Each group has its own S buffer, P buffer and O accumulator, so the two warps that
+// share an SM sub-partition (same TMEM lanes, one per group) work one Q K^T apart: one computes
+// exponentials while the other loads, reduces and stores.
 struct __align__(1024) WsoftSmem {
   uint8_t q[32768];          // Q tile: [channel half][128 rows x 128 B], SW128 (K-major A operand)
   uint8_t k[kKS][32768];     // K tiles: same layout (K-major B operand)
   uint8_t v[kVS][32768];     // V tiles: same layout (MN-major B operand of P V)
-  uint8_t p[32768];          // P: [key half][128 rows x 128 B], SW128 (K-major A operand)
-  float stat_m[2][128], stat_l[2][128];   // [key half][row]: reference maxima and normalisers
+  uint8_t p[2][32768];       // P per group: [key half][128 rows x 128 B], SW128 (K-major A operand)
   uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full;
   uint32_t tmem_base;
   int abort;
 };
+// after the last MMA the K stages hold the groups' reference maxima and normalisers
+struct WsoftStats {
+  float m[2][128], l[2][128];   // [group][row]
+};
+static_assert(sizeof(WsoftStats) <= kKS * 32768, "statistics fit in the K stages");
 
 // byte offset of the 16-byte chunk c (0..15) of row r in a 128 x 128 bf16 SW128 tile
 __device__ __forceinline__ uint32_t tile_chunk(int r, int c) {
@@ -193,13 +201,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
       tc::mbar_init(&sm.v_full[s], 1);
       tc::mbar_init(&sm.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&sm.s_full[s], 1);
-      tc::mbar_init(&sm.s_empty[s], 8);
-    }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&sm.p_full[s], 4);
-      tc::mbar_init(&sm.p_empty[s], 1);
+    for (int g = 0; g < 2; ++g) {
+      tc::mbar_init(&sm.s_full[g], 1);
+      tc::mbar_init(&sm.s_empty[g], 4);
+      tc::mbar_init(&sm.p_full[g], 4);
+      tc::mbar_init(&sm.p_empty[g], 1);
     }
     tc::mbar_init(&sm.o_full, 1);
     sm.abort = 0;
@@ -212,122 +218,116 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;       // S buffers at columns 0 and 128, O_0 at 256, O_1 at 384
+  const uint32_t tmem = sm.tmem_base;       // S of group g at columns 128 g, O of group g at 256 + 128 g
   const int rowq = (int)(b * N + q0), rowk = (int)(b * N + k0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // K runs two tiles ahead of V: Q K^T for tile j+2 is issued before P V for tile j
     if (lane == 0) {
+      auto load_k = [&](int t) -> bool {
+        const int ks = t % kKS;
+        if (!tc::mbar_wait(&sm.k_empty[ks], ((t / kKS) & 1) ^ 1, abort_flag, status)) return false;
+        tc::mbar_arrive_expect_tx(&sm.k_full[ks], 32768);
+        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks], 0, h, rowk + 128 * t);
+        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks] + 16384, 64, h, rowk + 128 * t);
+        return true;
+      };
+      auto load_v = [&](int t) -> bool {
+        const int vs = t % kVS;
+        if (!tc::mbar_wait(&sm.v_empty[vs], ((t / kVS) & 1) ^ 1, abort_flag, status)) return false;
+        tc::mbar_arrive_expect_tx(&sm.v_full[vs], 32768);
+        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs], 0, h, rowk + 128 * t);
+        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs] + 16384, 64, h, rowk + 128 * t);
+        return true;
+      };
       tc::mbar_arrive_expect_tx(&sm.q_full, 32768);
       tc::tma_load_3d(&tmQ, &sm.q_full, sm.q, 0, h, rowq);
       tc::tma_load_3d(&tmQ, &sm.q_full, sm.q + 16384, 64, h, rowq);
-      for (int j = 0; j < nkt; ++j) {
-        const int ks = j % kKS, vs = j % kVS;
-        if (!tc::mbar_wait(&sm.k_empty[ks], ((j / kKS) & 1) ^ 1, abort_flag, status)) break;
-        tc::mbar_arrive_expect_tx(&sm.k_full[ks], 32768);
-        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks], 0, h, rowk + 128 * j);
-        tc::tma_load_3d(&tmK, &sm.k_full[ks], sm.k[ks] + 16384, 64, h, rowk + 128 * j);
-        if (!tc::mbar_wait(&sm.v_empty[vs], ((j / kVS) & 1) ^ 1, abort_flag, status)) break;
-        tc::mbar_arrive_expect_tx(&sm.v_full[vs], 32768);
-        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs], 0, h, rowk + 128 * j);
-        tc::tma_load_3d(&tmV, &sm.v_full[vs], sm.v[vs] + 16384, 64, h, rowk + 128 * j);
+      bool ok = load_k(0) && (nkt < 2 || load_k(1)) && load_v(0);
+      for (int j = 0; j < nkt && ok; ++j) {
+        if (j + 2 < nkt) ok = load_k(j + 2);
+        if (ok && j + 1 < nkt) ok = load_v(j + 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t aq = tc::smem_u32(sm.q), ap = tc::smem_u32(sm.p);
-      int ik = 0, iv = 0, is = 0;
+      const uint32_t aq = tc::smem_u32(sm.q);
       bool ok = tc::mbar_wait(&sm.q_full, 0, abort_flag, status);
-      auto qk = [&]() -> bool {   // S = Q K^T for the next K tile into the next S buffer
-        const int ks = ik % kKS, sb = is % 2;
-        if (!tc::mbar_wait(&sm.k_full[ks], (ik / kKS) & 1, abort_flag, status)) return false;
-        if (!tc::mbar_wait(&sm.s_empty[sb], ((is / 2) & 1) ^ 1, abort_flag, status)) return false;
+      auto qk = [&](int t) -> bool {   // S_t = Q K_t^T into the S buffer of group t % 2
+        const int ks = t % kKS, g = t % 2;
+        if (!tc::mbar_wait(&sm.k_full[ks], (t / kKS) & 1, abort_flag, status)) return false;
+        if (!tc::mbar_wait(&sm.s_empty[g], ((t / 2) & 1) ^ 1, abort_flag, status)) return false;
         tc::tc_fence_after();
         const uint32_t bk = tc::smem_u32(sm.k[ks]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::umma_bf16(tmem + sb * 128, tc::smem_desc(aq + off, 16, 1024), tc::smem_desc(bk + off, 16, 1024),
+          tc::umma_bf16(tmem + g * 128, tc::smem_desc(aq + off, 16, 1024), tc::smem_desc(bk + off, 16, 1024),
                         kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc::umma_commit(&sm.s_full[sb]);
+        tc::umma_commit(&sm.s_full[g]);
         tc::umma_commit(&sm.k_empty[ks]);
-        ++ik;
-        ++is;
         return true;
       };
-      auto pv = [&](int j) -> bool {   // O_hf += P_j[:, keys of half hf] V_j[keys of half hf, :]
-        const int vs = iv % kVS;
-        if (!tc::mbar_wait(&sm.v_full[vs], (iv / kVS) & 1, abort_flag, status)) return false;
-        const uint32_t bv = tc::smem_u32(sm.v[vs]);
+      auto pv = [&](int j) -> bool {   // O_g += P_j V_j, g = j % 2
+        const int vs = j % kVS, g = j % 2;
+        if (!tc::mbar_wait(&sm.v_full[vs], (j / kVS) & 1, abort_flag, status)) return false;
+        if (!tc::mbar_wait(&sm.p_full[g], (j / 2) & 1, abort_flag, status)) return false;
+        tc::tc_fence_after();
+        const uint32_t ap = tc::smem_u32(sm.p[g]), bv = tc::smem_u32(sm.v[vs]);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          if (!tc::mbar_wait(&sm.p_full[hf], j & 1, abort_flag, status)) return false;
-          tc::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            tc::umma_bf16(tmem + 256 + 128 * hf, tc::smem_desc(ap + hf * 16384 + kk * 32, 16, 1024),
-                          tc::smem_desc(bv + (4 * hf + kk) * 2048, 16384, 1024), kIdescPV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc::umma_commit(&sm.p_empty[hf]);
+        for (int kk = 0; kk < 8; ++kk) {
+          tc::umma_bf16(tmem + 256 + 128 * g, tc::smem_desc(ap + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        tc::smem_desc(bv + kk * 2048, 16384, 1024), kIdescPV, (j >= 2 || kk > 0) ? 1u : 0u);
         }
+        tc::umma_commit(&sm.p_empty[g]);
         tc::umma_commit(&sm.v_empty[vs]);
-        ++iv;
         return true;
       };
-      // S for tile j+1 is computed while the softmax warps turn S_j into P_j
-      if (ok && nkt > 0) ok = qk();
+      ok = ok && qk(0) && (nkt < 2 || qk(1));
       for (int j = 0; j < nkt && ok; ++j) {
-        if (j + 1 < nkt) ok = qk();
+        if (j + 2 < nkt) ok = qk(j + 2);
         if (ok) ok = pv(j);
       }
       if (ok) tc::umma_commit(&sm.o_full);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int quarter = warp & 3, hf = (warp - 2) >> 2;
+    const int quarter = warp & 3, g = (warp - 2) >> 2;
     const int m = 32 * quarter + lane;                 // query row = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    int is = 0;
-    // Each key half (columns 64 hf .. 64 hf + 63 of every S tile) keeps its own accumulator O_hf, so
-    // the two warps on a row never wait for each other inside the loop.  mref: the reference maximum
-    // (log2 units) that every exponent of this row's half is taken against; it moves only when a
-    // tile's maximum exceeds it by more than 2^8, and then O_hf and l are rescaled
+    // mref: the reference maximum (log2 units) that every exponent of this row in this group is taken
+    // against; it moves only when a tile's maximum exceeds it by more than 2^8, and then O_g and l are
+    // rescaled
     float mref = -INFINITY, lrun = 0.f;
     bool ok = true;
-    auto load_s = [&](uint32_t (&r)[64]) -> bool {     // this thread's 64 columns of the next S buffer
-      const int sb = is % 2;
-      if (!tc::mbar_wait(&sm.s_full[sb], (is / 2) & 1, abort_flag, status)) return false;
+    for (int j = g, n = 0; j < nkt && ok; j += 2, ++n) {
+      // this group's n-th tile: its S buffer, then the tile maximum
+      if (!(ok = tc::mbar_wait(&sm.s_full[g], n & 1, abort_flag, status))) break;
       tc::tc_fence_after();
-      uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
-      uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
-      tc::tmem_ld32(tmem + sb * 128 + 64 * hf + lane_off, r0);
-      tc::tmem_ld32(tmem + sb * 128 + 64 * hf + 32 + lane_off, r1);
+      uint32_t r[128];
+#pragma unroll
+      for (int part = 0; part < 4; ++part)
+        tc::tmem_ld32(tmem + g * 128 + 32 * part + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * part]));
       tc::tmem_ld_wait();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.s_empty[sb]);
-      ++is;
-      return true;
-    };
-    for (int j = 0; j < nkt && ok; ++j) {
-      uint32_t r[64];
-      if (!(ok = load_s(r))) break;
-      const int nvalid = (int)min(64LL, max(0LL, k1 - (k0 + 128LL * j + 64 * hf)));
+      if (lane == 0) tc::mbar_arrive(&sm.s_empty[g]);
+      const int nvalid = (int)min(128LL, k1 - (k0 + 128LL * j));
       float tmax;
-      if (nvalid == 64) {                     // every tile but the window's last: a tree of maxima
+      if (nvalid == 128) {                    // every tile but the window's last: a tree of maxima
         float t8[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) t8[a] = __uint_as_float(r[a]);
 #pragma unroll
-        for (int e = 8; e < 64; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(r[e]));
+        for (int e = 8; e < 128; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(r[e]));
         tmax = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
       } else {
         tmax = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
+        for (int e = 0; e < 128; ++e)
           if (e < nvalid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
       }
       const float mt = tmax * scale;
@@ -338,10 +338,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         lrun *= corr;
         mref = mt;
       }
-      uint32_t pw[32];
+      uint32_t pw[64];
       float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
+      for (int e = 0; e < 128; e += 2) {
         const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mref) : 0.f;
         const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mref) : 0.f;
         sum0 += p0;
@@ -349,17 +349,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         pw[e / 2] = pack_bf16x2(p0, p1);
       }
       lrun += sum0 + sum1;
-      // this half's P_{j-1} V_{j-1} has completed once its P buffer is free
-      if (!(ok = tc::mbar_wait(&sm.p_empty[hf], (j & 1) ^ 1, abort_flag, status))) break;
+      // this group's previous P V has completed once its P buffer is free
+      if (!(ok = tc::mbar_wait(&sm.p_empty[g], (n & 1) ^ 1, abort_flag, status))) break;
       // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any of its
       // rows moved (corr = 1 for the others)
-      if (__any_sync(0xffffffffu, move) && j > 0) {
-        // the reference maximum moved: bring this half's O row to the new reference
+      if (__any_sync(0xffffffffu, move) && n > 0) {
         tc::tc_fence_after();
 #pragma unroll
         for (int part = 0; part < 4; ++part) {
           uint32_t o[32];
-          const uint32_t taddr = tmem + 256 + 128 * hf + 32 * part + lane_off;
+          const uint32_t taddr = tmem + 256 + 128 * g + 32 * part + lane_off;
           tc::tmem_ld32(taddr, o);
           tc::tmem_ld_wait();
 #pragma unroll
@@ -370,37 +369,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         tc::tc_fence_before();
       }
 #pragma unroll
-      for (int cq = 0; cq < 8; ++cq)
-        *reinterpret_cast<uint4*>(sm.p + tile_chunk(m, 8 * hf + cq)) =
+      for (int cq = 0; cq < 16; ++cq)
+        *reinterpret_cast<uint4*>(sm.p[g] + tile_chunk(m, cq)) =
             make_uint4(pw[4 * cq], pw[4 * cq + 1], pw[4 * cq + 2], pw[4 * cq + 3]);
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.p_full[hf]);
+      if (lane == 0) tc::mbar_arrive(&sm.p_full[g]);
     }
-    // combine the two key halves of the row: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l
-    sm.stat_m[hf][m] = mref;
-    sm.stat_l[hf][m] = lrun;
+    // epilogue, once every MMA has completed (the K stages are then free for the statistics):
+    // O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)); a group that saw
+    // no tile (m = -inf) adds nothing and its accumulator is never read
+    if (ok) ok = tc::mbar_wait(&sm.o_full, 0, abort_flag, status);
+    WsoftStats& st = *reinterpret_cast<WsoftStats*>(sm.k[0]);
+    if (ok) {
+      st.m[g][m] = mref;
+      st.l[g][m] = lrun;
+    }
     tc::named_bar(2 + quarter, 64);
-    const float m0 = sm.stat_m[0][m], m1 = sm.stat_m[1][m];
-    const float mx = fmaxf(m0, m1);
-    const float w0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mx), w1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mx);
-    const float inv_l = 1.f / (sm.stat_l[0][m] * w0 + sm.stat_l[1][m] * w1);
-    const float c0 = w0 * inv_l, c1 = w1 * inv_l;
-    // epilogue: this thread's 64 output channels of its row
-    if (ok && tc::mbar_wait(&sm.o_full, 0, abort_flag, status)) {
+    if (ok) {
       tc::tc_fence_after();
-      float o[64];
+      const float m0 = st.m[0][m], m1 = st.m[1][m];
+      const float mx = fmaxf(m0, m1);
+      const float w0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mx), w1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mx);
+      const float inv_l = 1.f / (st.l[0][m] * w0 + st.l[1][m] * w1);
+      const float c0 = w0 * inv_l, c1 = w1 * inv_l;
+      const bool use1 = nkt > 1;
+      float o[64];       // this thread's 64 output channels (64 g .. 64 g + 63) of its row
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         uint32_t a0[32], a1[32];
-        tc::tmem_ld32(tmem + 256 + 64 * hf + 32 * part + lane_off, a0);
-        tc::tmem_ld32(tmem + 384 + 64 * hf + 32 * part + lane_off, a1);
+        tc::tmem_ld32(tmem + 256 + 64 * g + 32 * part + lane_off, a0);
+        tc::tmem_ld32(tmem + 384 + 64 * g + 32 * part + lane_off, a1);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[32 * part + e] = __uint_as_float(a0[e]) * c0 + __uint_as_float(a1[e]) * c1;
+        for (int e = 0; e < 32; ++e)
+          o[32 * part + e] = __uint_as_float(a0[e]) * c0 + (use1 ? __uint_as_float(a1[e]) * c1 : 0.f);
       }
       if (q0 + m < cq1) {
-        uint4* dst = reinterpret_cast<uint4*>(out + ((b * N + q0 + m) * H + h) * 128 + 64 * hf);
+        uint4* dst = reinterpret_cast<uint4*>(out + ((b * N + q0 + m) * H + h) * 128 + 64 * g);
 #pragma unroll
         for (int cq = 0; cq < 8; ++cq) {
           float y[8];
