@@ -1,6 +1,7 @@
 """Benchmark of the VDN-H3 linear-branch forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 768p] [--impl reference]
+    python bench.py --path softmax|hybrid --steps 10 --warmup 3     # the windowed softmax branch / whole layer
 
 One step is one vdn_branch_forward call over the whole workload (all heads,
 all frames) with the inputs resident in HBM.  Prints ONE JSON line (rank 0):
@@ -12,6 +13,12 @@ the float64 oracle timed on the host cores on a bounded sample.
 
 Multi-GPU (torchrun, one rank per GPU): the branch needs no communication, each
 rank runs its own clip (seed + 1000 * rank) of the same workload: weak scaling.
+
+--path softmax times vdn_window_softmax_forward (the near-field branch over the
+RoPE-side q/k) and --path hybrid times vdn_hybrid_forward (softmax branch plus
+linear branch, the whole attention layer) on the same workload; their roofline is
+the tensor-core one of the softmax kernel (algorithmic Q K^T and P V FLOPs over
+the window's key tokens against the measured sustained bf16 GEMM rate).
 """
 from __future__ import annotations
 
@@ -34,11 +41,13 @@ import torch  # noqa: E402
 from video_diffusion_linear_b200 import synth  # noqa: E402
 
 METRIC = "latent tokens/sec through VDN linear branch fwd (1 B200); % of roofline"
+METRIC_PATH = {"softmax": "latent tokens/sec through the windowed softmax branch fwd (1 B200)",
+               "hybrid": "latent tokens/sec through the VDN-H3 hybrid attention layer fwd (softmax + linear branch, 1 B200)"}
 DEFAULT_WORKLOAD = "768p"
 KERNELS_TC = ["frame_stats", "frame_solve", "scan", "gather", "readout"]
 KERNEL_SOURCES = {"frame_stats": "tc_stats.cu", "frame_solve": "solve_gather.cu", "scan": "tc_scan.cu",
-                  "gather": "solve_gather.cu", "readout": "tc_readout.cu"}
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+                  "gather": "solve_gather.cu", "readout": "tc_readout.cu", "window_softmax": "softmax.cu"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 # ----------------------------------------------------------------------------- workload arithmetic
@@ -83,12 +92,25 @@ def path_roofline(w: synth.Workload, peaks: dict) -> dict:
             "bound": "hbm" if t_hbm >= t_tc else "tensor"}
 
 
+def softmax_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of the windowed softmax branch: Q K^T and P V, 2 d each per
+    (query, key) pair inside the query's window (exponentials not counted)."""
+    pairs = 0
+    for t in range(w.F):
+        c = t // w.chunk
+        lo = max(0, w.chunk * (c - w.radius))
+        hi = min(w.F - 1, w.chunk * (c + w.radius + 1) - 1)
+        pairs += w.S * (hi - lo + 1) * w.S
+    return 4.0 * w.d * pairs * w.B * w.H
+
+
 def load_peaks() -> tuple[dict, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
-        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"])}, "measured"
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"]))}, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
@@ -234,10 +256,23 @@ def blas_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def softmax_oracle_sample(inp: dict, w: synth.Workload, n_tokens: int) -> tuple[float, int]:
+    """Runs the float64 oracle's windowed softmax for n_tokens query tokens of
+    (batch 0, head 0), spread over every frame; returns (seconds, token-heads)."""
+    from oracle import vdn_oracle as O
+    N = w.F * w.S
+    toks = sorted(set(int(x) for x in torch.linspace(0, N - 1, n_tokens).round().tolist()))
+    t0 = time.perf_counter()
+    O.sampled_window_softmax(inp, w.F, w.S, w.chunk, w.radius, 0, 0, toks)
+    return time.perf_counter() - t0, len(toks)
+
+
 def run_reference(args, w: synth.Workload) -> None:
     rank, world, _ = dist_env()
     if rank != 0:
         return
+    if args.path != "linear":
+        return run_reference_softmax(args, w)
     inp = synth.make_inputs(w)
     times = []
     for i in range(args.warmup + args.steps):
@@ -259,7 +294,168 @@ def run_reference(args, w: synth.Workload) -> None:
     }), flush=True)
 
 
+def run_reference_softmax(args, w: synth.Workload) -> None:
+    inp = synth.make_inputs(w, with_rope_side=True)
+    times, th = [], 0
+    for i in range(args.warmup + args.steps):
+        dt_s, th_s = softmax_oracle_sample(inp, w, args.cpu_tokens)
+        dt, th = dt_s, th_s
+        if args.path == "hybrid":
+            dt_l, th_l = oracle_sample(inp, w, [i % w.H])
+            dt = dt_s + dt_l * th_s / th_l     # linear-branch cost of the same token-heads
+        if i >= args.warmup:
+            times.append(dt)
+    step = sum(times) / len(times)
+    value = (th / w.H) / step
+    cores = blas_threads()
+    sample = (f"{th} query tokens of head 0 (of {w.H}), batch 0, spread over all {w.F} frames, per step"
+              + (" (+ the linear branch's per-token-head cost from one full head)" if args.path == "hybrid" else "")
+              + "; tokens counted x 1/H")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC_PATH[args.path], "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(w)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 # ----------------------------------------------------------------------------- GPU arm
+def run_gpu_softmax(args, w: synth.Workload) -> None:
+    """The windowed softmax branch (--path softmax) or the whole hybrid layer
+    (--path hybrid) on one or more GPUs (independent clips per rank)."""
+    from video_diffusion_linear_b200 import _lib, api
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    _lib.load()
+    wr = rank_workload(w, rank)
+    host = synth.make_inputs(wr, with_rope_side=True)
+    dev = api.to_device(host, device)
+    out = torch.empty_like(dev["q"])
+    stream = torch.cuda.current_stream(device)
+    hybrid = args.path == "hybrid"
+    if hybrid:
+        args_t = api.forward_inputs(dev)
+        shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
+        ws = api.alloc_workspace(shape, w.rule, "auto", device)
+        launches = api.launch_count(shape) + 1
+    else:
+        ws = torch.empty(256, dtype=torch.uint8, device=device)
+        launches = 1
+
+    def step():
+        if hybrid:
+            api.hybrid_forward(dev["q_rope"], dev["k_rope"], *args_t, F=w.F, rule=w.rule, c=w.c, chunk=w.chunk,
+                               radius=w.radius, out=out, workspace=ws, stream=stream)
+        else:
+            api.window_softmax_forward(dev["q_rope"], dev["k_rope"], dev["v"], F=w.F, chunk=w.chunk,
+                                       radius=w.radius, out=out, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if api.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+    # the softmax kernel alone, for the roofline of the dominant kernel (same stream, CUDA events)
+    kev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if hybrid:
+            kev[0].record(stream)
+            for i in range(args.steps):
+                api.window_softmax_forward(dev["q_rope"], dev["k_rope"], dev["v"], F=w.F, chunk=w.chunk,
+                                           radius=w.radius, out=out, stream=stream)
+                kev[i + 1].record(stream)
+            torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    if api.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during the timed steps")
+    ms = start.elapsed_time(end)
+    ms_max = reduce_max(ms, device)
+    value = w.tokens * world * args.steps / (ms_max / 1e3)
+    soft_ms = (statistics.fmean(kev[i].elapsed_time(kev[i + 1]) for i in range(args.steps)) if hybrid
+               else ms / args.steps)
+    peaks, peak_src = load_peaks()
+    flops = softmax_flops(w)
+    achieved = flops / (soft_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roof = {"kernel": "window_softmax", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "peak_source": peak_src + " (sustained bf16 GEMM: the kernel runs ~0.1 s)",
+            "algorithmic_flops_per_launch": flops, "traffic": recorded_traffic("window_softmax"),
+            "us_per_launch": soft_ms * 1e3}
+    if roof["traffic"] is not None:
+        roof["traffic_workload"] = roof["traffic"]["workload"]
+        roof["traffic"] = roof["traffic"]["bytes"]
+
+    e2e = None
+    if not args.no_e2e:
+        keys = ["q_rope", "k_rope", "v"] + (["q", "k", "beta", "alpha", "gate"] if hybrid else [])
+        pinned = {k: host[k].pin_memory() for k in keys}
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
+        d2h = out_host.numel() * out_host.element_size()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu and world == 1:
+        dt, th = softmax_oracle_sample(host, w, args.cpu_tokens)
+        sample = f"{th} query tokens of head 0 (of {w.H}), batch 0, over all {w.F} frames ({dt:.1f} s)"
+        if hybrid:
+            dl, tl = oracle_sample(host, w, [0])
+            dt += dl * th / tl
+            sample += f" + the linear branch's per-token-head cost from head 0 ({dl:.1f} s)"
+        cpu = {"value": (th / w.H) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": sample + "; tokens counted x 1/H"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC_PATH[args.path], "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w) + f", softmax window = chunk {w.chunk} +- {w.radius} chunks, "
+                   "scale 1/sqrt(d)", "global_batch": w.B * world, "tokens_per_step": w.tokens * world,
+                   "l2": "inputs larger than L2 (q_rope, k_rope, v: %.2f GB)" % (3 * w.tokens * w.H * w.d * 2 / 1e9),
+                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }), flush=True)
+
+
 def run_gpu(args, w: synth.Workload) -> None:
     from video_diffusion_linear_b200 import _lib, api
     rank, world, local = dist_env()
@@ -410,6 +606,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=2)
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
+    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid"],
+                    help="linear branch (default), windowed softmax branch, or the whole hybrid layer")
+    ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -422,6 +621,8 @@ def main(argv=None):
         w = w.replace(H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.path != "linear":
+        run_gpu_softmax(args, w)
     else:
         run_gpu(args, w)
 

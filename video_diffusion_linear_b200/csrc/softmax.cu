@@ -339,16 +339,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
         mref = mt;
       }
       uint32_t pw[64];
-      float sum0 = 0.f, sum1 = 0.f;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      if (nvalid == 128) {
 #pragma unroll
-      for (int e = 0; e < 128; e += 2) {
-        const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mref) : 0.f;
-        const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mref) : 0.f;
-        sum0 += p0;
-        sum1 += p1;
-        pw[e / 2] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 128; e += 2) {
+          const float p0 = ex2_approx(__uint_as_float(r[e]) * scale - mref);
+          const float p1 = ex2_approx(__uint_as_float(r[e + 1]) * scale - mref);
+          sum[(e >> 1) & 3] += p0 + p1;
+          pw[e / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 128; e += 2) {
+          const float p0 = e < nvalid ? ex2_approx(__uint_as_float(r[e]) * scale - mref) : 0.f;
+          const float p1 = e + 1 < nvalid ? ex2_approx(__uint_as_float(r[e + 1]) * scale - mref) : 0.f;
+          sum[(e >> 1) & 3] += p0 + p1;
+          pw[e / 2] = pack_bf16x2(p0, p1);
+        }
       }
-      lrun += sum0 + sum1;
+      lrun += (sum[0] + sum[1]) + (sum[2] + sum[3]);
       // this group's previous P V has completed once its P buffer is free
       if (!(ok = tc::mbar_wait(&sm.p_empty[g], (n & 1) ^ 1, abort_flag, status))) break;
       // tcgen05.ld/st are warp-collective: the warp rescales its O rows together when any of its
