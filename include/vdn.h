@@ -244,6 +244,49 @@ vdn_status vdn_hybrid_forward(const vdn_shape* shape,
                               void* workspace, size_t workspace_bytes,
                               void* out, void* stream);
 
+/* Bytes of device workspace that vdn_branch_backward needs (0 if invalid). */
+size_t vdn_branch_backward_workspace_size(const vdn_shape* shape, int rule);
+
+/*
+ * vdn_branch_backward -- gradients of the branch (vdn_branch_forward, same
+ * arguments) for an upstream gradient `dout` = dL/d out, [B, F*S, H, d] dtype.
+ * The page trains the branch (stages A1/A2 of "VDN-Minimax-H3 bidirectional
+ * linear branch in five steps") without printing a backward; this is the exact
+ * gradient of the five steps and of the text-state seeds, in reverse order:
+ * read-out and RMSNorm, gather and bridge, both scans (adjoint recurrences
+ * through N_f), frame statistics, L2 norm, SiLU and the short conv.
+ *
+ * Outputs (written, not accumulated; caller-owned device memory):
+ *   dq, dk, dv, dgate   [B, F*S, H, d] dtype
+ *   dbeta               [B, F*S, H]    fp32
+ *   dalpha              [B, F, H, d]   fp32
+ *   drms_w              [d]            fp32  (summed over batch and heads)
+ *   dconv_k_w, dconv_v_w [H, d, conv_width] fp32 (summed over the batch); NULL
+ *                       exactly when the matching taps are NULL
+ *   dtext_state         [H, d, d]      fp32 (summed over the batch); NULL exactly
+ *                       when text_state is NULL
+ * The forward runs first, inside the call (its per-frame statistics, operators and
+ * states are kept in the workspace); then fp32 kernels for d = 16 and 128.  No
+ * output may overlap another output, an input or the workspace.  Rules whose
+ * states leave the fp32 range (divergent sana_scaled settings) give non-finite
+ * gradients.  Errors: as vdn_branch_forward, plus VDN_ERR_INVALID_ARG for a
+ * missing or overlapping gradient buffer.  The device status word (first word
+ * of the workspace) is that of the forward pass.
+ */
+vdn_status vdn_branch_backward(const vdn_shape* shape,
+                               const void* q, const void* k, const void* v,
+                               const float* beta, const float* alpha,
+                               const void* gate, const float* rms_w,
+                               const float* conv_k_w, const float* conv_v_w,
+                               const float* text_state,
+                               int rule, float c, int chunk, int radius,
+                               const void* dout,
+                               void* workspace, size_t workspace_bytes,
+                               void* dq, void* dk, void* dv,
+                               float* dbeta, float* dalpha, void* dgate, float* drms_w,
+                               float* dconv_k_w, float* dconv_v_w, float* dtext_state,
+                               void* stream);
+
 /* Reads the device status word that bounded waits inside the kernels set (it
  * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
  * Synchronises `stream`. */

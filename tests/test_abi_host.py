@@ -111,3 +111,42 @@ def test_feature_prep_validation(lib):
         VDN_ERR_INVALID_ARG
     assert lib.vdn_feature_prep(ctypes.byref(_shape(d=32)), p(0), p(1), p(2), None, None, p(3), p(4), p(5),
                                 None) == VDN_ERR_UNSUPPORTED
+
+
+def _bwd_args(shape, ws_bytes=1 << 40, **over):
+    names = ["q", "k", "v", "beta", "alpha", "gate", "rms_w", "conv_k_w", "conv_v_w", "text", "dout", "ws",
+             "dq", "dk", "dv", "dbeta", "dalpha", "dgate", "drms_w", "dconv_k_w", "dconv_v_w", "dtext"]
+    ptr = {name: BASE + i * GAP for i, name in enumerate(names)}
+    ptr.update(over)
+    P = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n])
+    return (ctypes.byref(shape), P("q"), P("k"), P("v"), P("beta"), P("alpha"), P("gate"), P("rms_w"),
+            P("conv_k_w"), P("conv_v_w"), P("text"), 1, 1.0, 5, 1, P("dout"), P("ws"), ws_bytes, P("dq"), P("dk"),
+            P("dv"), P("dbeta"), P("dalpha"), P("dgate"), P("drms_w"), P("dconv_k_w"), P("dconv_v_w"), P("dtext"),
+            None)
+
+
+def test_backward_workspace_size(lib):
+    s = _shape()
+    n = lib.vdn_branch_backward_workspace_size(ctypes.byref(s), 1)
+    assert n > lib.vdn_branch_workspace_size(ctypes.byref(s), 1) and n % 256 == 0
+    assert lib.vdn_branch_backward_workspace_size(ctypes.byref(_shape(d=64)), 1) == 0
+    assert lib.vdn_branch_backward_workspace_size(ctypes.byref(s), 9) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(ptr=dict(dout=None)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(dalpha=None)), VDN_ERR_INVALID_ARG),
+    (dict(ptr=dict(dconv_k_w=None)), VDN_ERR_INVALID_ARG),              # taps given, no tap gradient
+    (dict(ptr=dict(text=None)), VDN_ERR_INVALID_ARG),                   # text gradient without a text state
+    (dict(ptr=dict(dq=BASE + 64)), VDN_ERR_INVALID_ARG),                # dq overlaps q
+    (dict(ptr=dict(dk=BASE + 12 * GAP + 512)), VDN_ERR_INVALID_ARG),    # dk overlaps dq
+    (dict(ptr=dict(dbeta=BASE + 10 * GAP)), VDN_ERR_INVALID_ARG),       # dbeta overlaps dout
+    (dict(ptr=dict(dgate=BASE + 11 * GAP + 4096)), VDN_ERR_INVALID_ARG),  # dgate overlaps the workspace
+    (dict(ptr=dict(dalpha=BASE + 16 * GAP + 8)), VDN_ERR_ALIGNMENT),
+    (dict(ws_bytes=1 << 20), VDN_ERR_WORKSPACE),
+    (dict(shape=dict(d=64)), VDN_ERR_UNSUPPORTED),
+])
+def test_backward_validation_rejects_before_launch(lib, case, expect):
+    s = _shape(**case.get("shape", {}))
+    args = _bwd_args(s, case.get("ws_bytes", 1 << 40), **case.get("ptr", {}))
+    assert lib.vdn_branch_backward(*args) == expect

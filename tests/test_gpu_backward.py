@@ -1,0 +1,92 @@
+"""Parity of vdn_branch_backward (the branch's gradients) with the float64
+backward oracle, through the C ABI: every gradient (q, k, v, beta, alpha, gate,
+rms_w, both conv taps, text state) for each rule, fp32 at d = 16 and d = 128
+(SIMT forward) and bf16 at d = 128 (tensor-core forward), ragged token tiles,
+windows clipped at both clip ends, and the optional inputs left out.  Bound per
+gradient: max |gpu - ref| / max |ref| <= 1e-4 (fp32 inputs) or 2e-2 (bf16)."""
+import numpy as np
+import pytest
+import torch
+
+from harness import TOL_BF16, rel_err, to_np
+from oracle import vdn_backward as BW
+from video_diffusion_linear_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ["dq", "dk", "dv", "dbeta", "dalpha", "dgate", "drms_w", "dconv_k_w", "dconv_v_w", "dtext_state"]
+TOL_F32_BWD = 1e-4
+
+
+def _run(w):
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w)
+    dev = api.to_device(inp)
+    shape = api.shape_from(dev["q"], w.F, dev.get("conv_k_w"))
+    ws = torch.empty(api.backward_workspace_size(shape, w.rule), dtype=torch.uint8, device="cuda")
+    got = api.branch_backward(*api.forward_inputs(dev), dout=dout.cuda(), F=w.F, rule=w.rule, c=w.c,
+                              chunk=w.chunk, radius=w.radius, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.workspace_status(ws) == 0
+    ref = BW.branch_backward(inp, dout, w.F, w.S, w.rule, w.c, w.chunk, w.radius)
+    return got, ref
+
+
+def _compare(w, got, ref, tol):
+    errs = {}
+    for n in NAMES:
+        if ref[n] is None:
+            assert got[n] is None
+            continue
+        g = to_np(got[n])
+        assert np.isfinite(g).all(), n
+        errs[n] = rel_err(g, ref[n])
+    bad = {n: e for n, e in errs.items() if e > tol}
+    assert not bad, (w.name, bad, errs)
+
+
+CASES = [
+    synth.Workload("bw_d16_solve", B=1, H=2, d=16, F=10, S=16, dtype="f32", alpha_mu=2.0, text=True, seed=50),
+    synth.Workload("bw_d16_sana", B=2, H=1, d=16, F=9, S=12, dtype="f32", alpha_mu=2.0, text=True, seed=51,
+                   rule="sana_scaled", c=0.5, chunk=2, radius=1),
+    synth.Workload("bw_d16_scaled", B=1, H=2, d=16, F=8, S=20, dtype="f32", alpha_mu=2.0, text=True, seed=52,
+                   rule="vdn_scaled", c=0.7, chunk=3, radius=0),
+    synth.Workload("bw_d16_additive", B=1, H=1, d=16, F=7, S=9, dtype="f32", alpha_mu=2.0, text=True, seed=53,
+                   rule="additive", chunk=2, radius=1),
+    synth.Workload("bw_d16_bare", B=1, H=2, d=16, F=10, S=16, dtype="f32", alpha_mu=2.0, text=False, seed=54,
+                   conv_width=1),
+    synth.Workload("bw_d128_f32", B=1, H=2, d=128, F=7, S=40, dtype="f32", alpha_mu=2.0, text=True, seed=55,
+                   chunk=3, radius=1),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
+def test_fp32_gradients_match_oracle(w):
+    got, ref = _run(w)
+    _compare(w, got, ref, TOL_F32_BWD)
+
+
+BF16 = [
+    synth.Workload("bw_bf16_solve", B=1, H=2, d=128, F=12, S=48, dtype="bf16", alpha_mu=2.0, text=True, seed=56),
+    synth.Workload("bw_bf16_ragged", B=2, H=1, d=128, F=8, S=70, dtype="bf16", alpha_mu=2.0, text=False, seed=57,
+                   chunk=2, radius=1, conv_width=1),
+]
+
+
+@pytest.mark.parametrize("w", BF16, ids=[c.name for c in BF16])
+def test_bf16_gradients_match_oracle(w):
+    got, ref = _run(w)
+    _compare(w, got, ref, TOL_BF16)
+
+
+def test_backward_is_deterministic():
+    w = CASES[5]
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w).cuda()
+    dev = api.to_device(inp)
+    a = api.branch_backward(*api.forward_inputs(dev), dout=dout, F=w.F, chunk=w.chunk, radius=w.radius)
+    b = api.branch_backward(*api.forward_inputs(dev), dout=dout, F=w.F, chunk=w.chunk, radius=w.radius)
+    torch.cuda.synchronize()
+    for n in NAMES:
+        if a[n] is not None:
+            assert torch.equal(a[n], b[n]), n

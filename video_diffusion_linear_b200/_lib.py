@@ -55,6 +55,10 @@ _SIGNATURES = {
                                           _P, ctypes.c_size_t, _P, _P]),
     "vdn_window_bounds": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "vdn_branch_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(VdnShape), ctypes.c_int]),
+    "vdn_branch_backward": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P, _P,
+                                           ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vdn_workspace_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "vdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }

@@ -181,6 +181,41 @@ def to_device(inp: dict, device="cuda") -> dict:
     return {k: (None if t is None else t.to(device)) for k, t in inp.items()}
 
 
+def backward_workspace_size(shape: VdnShape, rule="vdn_solve") -> int:
+    n = _lib.load().vdn_branch_backward_workspace_size(ctypes.byref(shape), VDN_RULE[rule])
+    if n == 0:
+        raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_branch_backward_workspace_size")
+    return n
+
+
+def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *, dout,
+                    F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, grads=None, workspace=None, stream=None):
+    """vdn_branch_backward: gradients of <dout, branch_forward(...)> with respect to every
+    input.  Returns a dict dq, dk, dv, dgate (q's dtype), dbeta, dalpha, drms_w, and
+    dconv_k_w, dconv_v_w, dtext_state (fp32; None where the input is None)."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    dev = q.device
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+                 "dgate": torch.empty_like(gate), "dbeta": torch.empty(beta.shape, **f32),
+                 "dalpha": torch.empty(alpha.shape, **f32), "drms_w": torch.empty(rms_w.shape, **f32),
+                 "dconv_k_w": None if conv_k_w is None else torch.empty(conv_k_w.shape, **f32),
+                 "dconv_v_w": None if conv_v_w is None else torch.empty(conv_v_w.shape, **f32),
+                 "dtext_state": None if text_state is None else torch.empty(text_state.shape, **f32)}
+    if workspace is None:
+        workspace = torch.empty(backward_workspace_size(shape, rule), dtype=torch.uint8, device=dev)
+    g = grads
+    st = _lib.load().vdn_branch_backward(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
+        _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
+        _ptr(dout), _ptr(workspace), workspace.numel(), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+        _ptr(g["dbeta"]), _ptr(g["dalpha"]), _ptr(g["dgate"]), _ptr(g["drms_w"]), _ptr(g["dconv_k_w"]),
+        _ptr(g["dconv_v_w"]), _ptr(g["dtext_state"]), _stream_ptr(stream))
+    check(st, "vdn_branch_backward")
+    return grads
+
+
 def forward_inputs(dev: dict):
     """Positional tensor arguments of branch_forward from a synth-style dict."""
     return (dev["q"], dev["k"], dev["v"], dev["beta"], dev["alpha"], dev["gate"], dev["rms_w"],

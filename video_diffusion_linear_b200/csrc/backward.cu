@@ -1,0 +1,758 @@
+// Backward pass of the VDN-H3 linear branch: the gradients of the five steps of
+// "VDN-Minimax-H3 bidirectional linear branch in five steps" and of the
+// text-state seeds, taken in reverse order (the page trains the branch, stages
+// A1/A2, but prints no backward; this is the exact gradient of the forward).
+//
+// The forward runs first with its per-frame export (A_f, B_f, N_f, P_f, Q_f, W_t
+// in fp32); then, all in fp32 SIMT for d = 16 and 128:
+//   k_bwd_readout  (batch, head, frame): recompute q', o = W_t q', RMSNorm; write
+//                  dgate and dq; dW_t = sum_s do_s q'_s^T; RMS-weight partials
+//   k_bwd_gather   (batch, head): dW_t onto the boundary states P_{lo-1} and
+//                  Q_{hi+1} (or the seed at a clip edge), d alpha of the bridge
+//   k_bwd_scan     (batch, head, direction): the adjoint of each scan, frame by
+//                  frame in reverse order of absorption
+//   k_bwd_stats    (batch, head, frame): dk', dv', d beta from dA_f, dB_f; L2-norm
+//                  and SiLU reversed into the gradients of the conv outputs
+//   k_bwd_conv     the short conv reversed (dk, dv, tap partials)
+//   k_bwd_finish   reductions over CTAs, heads and batch; d alpha summed
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vdn {
+namespace {
+
+constexpr int kBT = 256;   // threads of every backward block
+constexpr int kTok = 32;   // tokens per tile of the per-token kernels
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
+// d silu(x) = sigma(x) (1 + x (1 - sigma(x))) dx
+__device__ __forceinline__ float silu_grad(float x, float g) {
+  const float s = sigmoidf_(x);
+  return g * s * (1.f + x * (1.f - s));
+}
+
+// ---------------------------------------------------------------- per-token helpers (one warp per token)
+// Lane `lane` holds channels c = lane + 32 r, r < PER (d = 16: lanes 16..31 hold nothing).
+template <int D>
+struct Lanes {
+  static constexpr int PER = D >= 32 ? D / 32 : 1;
+  __device__ static bool has(int lane, int r) { return lane + 32 * r < D; }
+};
+
+// x_hat = x / n, n = sqrt(sum x^2 + eps): dx = (g - x_hat (x_hat . g)) / n
+template <int D>
+__device__ __forceinline__ void l2n_grad(const float (&x)[Lanes<D>::PER], const float (&g)[Lanes<D>::PER],
+                                         float (&dx)[Lanes<D>::PER], int lane) {
+  constexpr int PER = Lanes<D>::PER;
+  float ss = 0.f;
+#pragma unroll
+  for (int r = 0; r < PER; ++r) ss += Lanes<D>::has(lane, r) ? x[r] * x[r] : 0.f;
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss + kL2Eps);
+  float xg = 0.f;
+#pragma unroll
+  for (int r = 0; r < PER; ++r) xg += Lanes<D>::has(lane, r) ? x[r] * inv * g[r] : 0.f;
+  xg = warp_sum(xg);
+#pragma unroll
+  for (int r = 0; r < PER; ++r) dx[r] = (g[r] - x[r] * inv * xg) * inv;
+}
+
+// ---------------------------------------------------------------- tile products in shared memory
+// out[t][i] = sum_j in[t][j] M(i, j) over a tile of kTok tokens, with M(i, j) read
+// from a row-padded (stride D + 1) shared matrix as m[i (D+1) + j] or, transposed,
+// m[j (D+1) + i].  Thread tid owns token t = tid / 8 and channels i = tid % 8 + 8 u.
+template <int D, bool kTrans>
+__device__ __forceinline__ void tile_matvec(float* out, const float* in, const float* m) {
+  constexpr int U = D / 8;
+  const int t = threadIdx.x >> 3, i0 = threadIdx.x & 7;
+  float acc[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) acc[u] = 0.f;
+  const float* x = in + t * (D + 1);
+  for (int j = 0; j < D; ++j) {
+    const float xj = x[j];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + 8 * u;
+      acc[u] = fmaf(xj, kTrans ? m[j * (D + 1) + i] : m[i * (D + 1) + j], acc[u]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) out[t * (D + 1) + i0 + 8 * u] = acc[u];
+}
+
+// C = alpha op(A) op(B) for D x D row-major matrices in global memory, by the whole
+// block (kBT threads; thread (ty, tx) owns rows ty + 16 r and columns tx + 16 s).
+// `slab` is 2 * 16 * (D + 1) floats of shared memory.  Ends with a block barrier.
+template <int D>
+__device__ void cta_mm(float* __restrict__ C, const float* __restrict__ A, bool tA, const float* __restrict__ Bm,
+                       bool tB, float alpha, float* slab) {
+  constexpr int R = D / 16;
+  float* As = slab;                 // As[kk][i] = op(A)[i][k0 + kk]
+  float* Bs = slab + 16 * (D + 1);  // Bs[kk][j] = op(B)[k0 + kk][j]
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[R][R];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int s = 0; s < R; ++s) acc[r][s] = 0.f;
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    for (int e = tid; e < 16 * D; e += kBT) {
+      const int kk = e / D, i = e % D, k = k0 + kk;
+      As[kk * (D + 1) + i] = tA ? A[k * D + i] : A[i * D + k];
+      Bs[kk * (D + 1) + i] = tB ? Bm[i * D + k] : Bm[k * D + i];
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[R], b[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) a[r] = As[kk * (D + 1) + ty + 16 * r];
+#pragma unroll
+      for (int s = 0; s < R; ++s) b[s] = Bs[kk * (D + 1) + tx + 16 * s];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int s = 0; s < R; ++s) acc[r][s] = fmaf(a[r], b[s], acc[r][s]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int s = 0; s < R; ++s) C[(ty + 16 * r) * D + tx + 16 * s] = alpha * acc[r][s];
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- step 5 reversed
+template <int D>
+struct ReadoutSmem {
+  float W[D * (D + 1)];     // W_t, rows padded
+  float qf[kTok * (D + 1)];
+  float dov[kTok * (D + 1)];
+  float o[kTok * (D + 1)];  // o, then dq'
+  float rms[kBT / 32][D];   // per-warp RMS-weight partials
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT) k_bwd_readout(const T* __restrict__ q, const T* __restrict__ gate,
+                                                     const T* __restrict__ dout, const float* __restrict__ rms_w,
+                                                     const float* __restrict__ Wall, float* __restrict__ dWall,
+                                                     float* __restrict__ rms_part, T* __restrict__ dq,
+                                                     T* __restrict__ dgate, int H, int F, int S) {
+  constexpr int PER = Lanes<D>::PER;
+  extern __shared__ float smem_f[];
+  ReadoutSmem<D>& sm = *reinterpret_cast<ReadoutSmem<D>*>(smem_f);
+  const long long fi = blockIdx.x;             // (b, h, f)
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long N = (long long)F * S;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* Wt = Wall + fi * D * D;
+  for (int e = tid; e < D * D; e += kBT) sm.W[(e / D) * (D + 1) + e % D] = Wt[e];
+  float rw[PER], racc[PER];
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    rw[r] = Lanes<D>::has(lane, r) ? rms_w[lane + 32 * r] : 0.f;
+    racc[r] = 0.f;
+  }
+  constexpr int R = D / 16;
+  float dW[R][R];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int s = 0; s < R; ++s) dW[r][s] = 0.f;
+  __syncthreads();
+
+  for (int s0 = 0; s0 < S; s0 += kTok) {
+    // q' of the tile's tokens (zero rows past the frame)
+    for (int t = warp; t < kTok; t += kBT / 32) {
+      const int s = s0 + t;
+      float qs[PER];
+      float ss = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        qs[r] = 0.f;
+        if (s < S && Lanes<D>::has(lane, r))
+          qs[r] = silu_precise(to_f32(q[((b * N + (long long)f * S + s) * H + h) * D + lane + 32 * r]));
+        ss += qs[r] * qs[r];
+      }
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (Lanes<D>::has(lane, r)) sm.qf[t * (D + 1) + lane + 32 * r] = s < S ? qs[r] * inv : 0.f;
+    }
+    __syncthreads();
+    tile_matvec<D, false>(sm.o, sm.qf, sm.W);          // o = W_t q'
+    __syncthreads();
+    // RMSNorm and gate reversed: dgate, d rms_w, do
+    for (int t = warp; t < kTok; t += kBT / 32) {
+      const int s = s0 + t;
+      if (s >= S) {
+#pragma unroll
+        for (int r = 0; r < PER; ++r)
+          if (Lanes<D>::has(lane, r)) sm.dov[t * (D + 1) + lane + 32 * r] = 0.f;
+        continue;
+      }
+      const long long row = ((b * N + (long long)f * S + s) * H + h) * D;
+      float o[PER], dy[PER];
+      float ss = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        o[r] = Lanes<D>::has(lane, r) ? sm.o[t * (D + 1) + lane + 32 * r] : 0.f;
+        ss += o[r] * o[r];
+      }
+      ss = warp_sum(ss);
+      const float rr = rsqrtf(ss / D + kRmsEps);
+      float so = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        if (!Lanes<D>::has(lane, r)) {
+          dy[r] = 0.f;
+          continue;
+        }
+        const int c = lane + 32 * r;
+        const float go = to_f32(dout[row + c]), g = to_f32(gate[row + c]);
+        const float oh = o[r] * rr;
+        dgate[row + c] = from_f32<T>(go * oh * rw[r]);
+        dy[r] = go * g;
+        racc[r] = fmaf(dy[r], oh, racc[r]);
+        so += dy[r] * rw[r] * o[r];
+      }
+      so = warp_sum(so);
+      const float k3 = rr * rr * rr * so / D;
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (Lanes<D>::has(lane, r)) sm.dov[t * (D + 1) + lane + 32 * r] = rr * dy[r] * rw[r] - k3 * o[r];
+    }
+    __syncthreads();
+    tile_matvec<D, true>(sm.o, sm.dov, sm.W);          // dq' = W_t^T do
+    // dW_t += do q'^T over the tile
+    {
+      const int ty = tid >> 4, tx = tid & 15;
+      for (int t = 0; t < kTok; ++t) {
+        float a[R], c[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[r] = sm.dov[t * (D + 1) + ty + 16 * r];
+#pragma unroll
+        for (int s = 0; s < R; ++s) c[s] = sm.qf[t * (D + 1) + tx + 16 * s];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int s = 0; s < R; ++s) dW[r][s] = fmaf(a[r], c[s], dW[r][s]);
+      }
+    }
+    __syncthreads();
+    // q' = l2n(silu(q)) reversed
+    for (int t = warp; t < kTok; t += kBT / 32) {
+      const int s = s0 + t;
+      if (s >= S) continue;
+      const long long row = ((b * N + (long long)f * S + s) * H + h) * D;
+      float x[PER], qs[PER], g[PER], dqs[PER];
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        x[r] = Lanes<D>::has(lane, r) ? to_f32(q[row + lane + 32 * r]) : 0.f;
+        qs[r] = Lanes<D>::has(lane, r) ? silu_precise(x[r]) : 0.f;
+        g[r] = Lanes<D>::has(lane, r) ? sm.o[t * (D + 1) + lane + 32 * r] : 0.f;
+      }
+      l2n_grad<D>(qs, g, dqs, lane);
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (Lanes<D>::has(lane, r)) dq[row + lane + 32 * r] = from_f32<T>(silu_grad(x[r], dqs[r]));
+    }
+    __syncthreads();
+  }
+  {
+    const int ty = tid >> 4, tx = tid & 15;
+    float* dWt = dWall + fi * D * D;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int s = 0; s < R; ++s) dWt[(ty + 16 * r) * D + tx + 16 * s] = dW[r][s];
+  }
+#pragma unroll
+  for (int r = 0; r < PER; ++r)
+    if (Lanes<D>::has(lane, r)) sm.rms[warp][lane + 32 * r] = racc[r];
+  __syncthreads();
+  for (int c = tid; c < D; c += kBT) {
+    float sacc = 0.f;
+    for (int w = 0; w < kBT / 32; ++w) sacc += sm.rms[w][c];
+    rms_part[fi * D + c] = sacc;
+  }
+}
+
+// ---------------------------------------------------------------- step 4 (gather + bridge) reversed
+// dPin[b, h][0] receives the gradient of the seed as P_{-1}, dPin[b, h][f + 1] that of P_f;
+// dQin[b, h][f] that of Q_f, dQin[b, h][F] that of the seed as Q_F.  dalpha_g [B, H, F, D].
+template <int D>
+__global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P, const float* __restrict__ Q,
+                                                    const float* __restrict__ alpha,
+                                                    const float* __restrict__ text_state,
+                                                    const float* __restrict__ dWall, float* __restrict__ dPin,
+                                                    float* __restrict__ dQin, float* __restrict__ dalpha_g, int H,
+                                                    int F, int chunk, int radius) {
+  const long long bh = blockIdx.x;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const int j = threadIdx.x;
+  if (j >= D) return;                          // thread j owns column j
+  const long long DD = (long long)D * D;
+  float* dP = dPin + bh * (F + 1) * DD;
+  float* dQ = dQin + bh * (F + 1) * DD;
+  float* dal = dalpha_g + bh * F * D;
+  auto alpha_at = [&](int f) { return alpha[((b * F + f) * H + h) * D + j]; };
+  auto seed_at = [&](int i) { return text_state ? 0.5f * text_state[((long long)h * D + i) * D + j] : 0.f; };
+  for (int t = 0; t < F; ++t) {
+    int lo, hi;
+    window_bounds(t, F, chunk, radius, lo, hi);
+    float a = 1.f, bb = 1.f;
+    for (int f = lo; f <= t; ++f) a *= alpha_at(f);
+    for (int f = t; f <= hi; ++f) bb *= alpha_at(f);
+    const float* dW = dWall + (bh * F + t) * DD;
+    const float* pre = lo == 0 ? nullptr : P + (bh * F + lo - 1) * DD;
+    const float* suf = hi == F - 1 ? nullptr : Q + (bh * F + hi + 1) * DD;
+    float* dpre = dP + (long long)lo * DD;          // slot lo: P_{lo-1} (slot 0: the seed)
+    float* dsuf = dQ + (long long)(hi + 1) * DD;    // slot hi + 1: Q_{hi+1} (slot F: the seed)
+    float da = 0.f, db = 0.f;
+    for (int i = 0; i < D; ++i) {
+      const float g = dW[i * D + j];
+      dpre[i * D + j] += g * a;
+      dsuf[i * D + j] += g * bb;
+      da = fmaf(pre ? pre[i * D + j] : seed_at(i), g, da);
+      db = fmaf(suf ? suf[i * D + j] : seed_at(i), g, db);
+    }
+    // d prod / d alpha_f = product of the other factors
+    for (int f = lo; f <= t; ++f) {
+      float pr = 1.f;
+      for (int g2 = lo; g2 <= t; ++g2)
+        if (g2 != f) pr *= alpha_at(g2);
+      dal[f * D + j] += da * pr;
+    }
+    for (int f = t; f <= hi; ++f) {
+      float pr = 1.f;
+      for (int g2 = t; g2 <= hi; ++g2)
+        if (g2 != f) pr *= alpha_at(g2);
+      dal[f * D + j] += db * pr;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- steps 3-4 (scans) reversed
+// Block (b, h, dir): dir 0 reverses the prefix scan P_f = step(P_{f-1}, f) from f = F-1 down,
+// dir 1 the suffix scan Q_f = step(Q_{f+1}, f) from f = 0 up.  For the generic step
+// S_out = (S_in D + cpre B) N + cpost B:
+//   dX = lam N^T (N symmetric), dS_in = dX D, dalpha_j = sum_i S_in[i][j] dX[i][j],
+//   dB = cpre dX + cpost lam, dA = -c2 S_out^T dX (N = (I + c2 A)^-1) or -c2 X^T lam (N = I - c2 A).
+// scratch: 4 D x D per block (lam, dX, X, seed).
+template <int D>
+__global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Bm, const float* __restrict__ Nm,
+                                                  const float* __restrict__ P, const float* __restrict__ Q,
+                                                  const float* __restrict__ alpha,
+                                                  const float* __restrict__ text_state, RuleCoef rc,
+                                                  const float* __restrict__ dPin, const float* __restrict__ dQin,
+                                                  float* __restrict__ dA2, float* __restrict__ dB2,
+                                                  float* __restrict__ dalpha2, float* __restrict__ dseed2,
+                                                  float* __restrict__ scratch, int H, int F) {
+  __shared__ float slab[2 * 16 * (D + 1)];
+  const long long bh = blockIdx.x;
+  const int dir = blockIdx.y;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long DD = (long long)D * D;
+  const long long BH = gridDim.x;
+  const int tid = threadIdx.x;
+  float* lam = scratch + (bh * 2 + dir) * 4 * DD;
+  float* dX = lam + DD;
+  float* X = dX + DD;
+  float* seed = X + DD;
+  const float* S = dir == 0 ? P : Q;
+  const float* din = (dir == 0 ? dPin : dQin) + bh * (F + 1) * DD;
+  for (long long e = tid; e < DD; e += kBT) {
+    seed[e] = text_state ? 0.5f * text_state[(long long)h * DD + e] : 0.f;
+    lam[e] = 0.f;
+  }
+  __syncthreads();
+  for (int it = 0; it < F; ++it) {
+    const int f = dir == 0 ? F - 1 - it : it;
+    const long long fo = (bh * F + f) * DD;
+    const float* S_out = S + fo;
+    const float* S_in = dir == 0 ? (f == 0 ? seed : S + fo - DD) : (f == F - 1 ? seed : S + fo + DD);
+    const float* gin = din + (long long)(dir == 0 ? f + 1 : f) * DD;
+    for (long long e = tid; e < DD; e += kBT) lam[e] += gin[e];
+    __syncthreads();
+    cta_mm<D>(dX, lam, false, Nm + fo, true, 1.f, slab);
+    float* dA = dA2 + ((long long)dir * BH * F + bh * F + f) * DD;
+    float* dB = dB2 + ((long long)dir * BH * F + bh * F + f) * DD;
+    if (rc.solve) {
+      cta_mm<D>(dA, S_out, true, dX, false, -rc.c2, slab);
+    } else if (rc.c2 != 0.f) {
+      for (long long e = tid; e < DD; e += kBT) {
+        const int jj = (int)(e % D);
+        X[e] = S_in[e] * alpha[((b * F + f) * H + h) * D + jj] + rc.cpre * Bm[fo + e];
+      }
+      __syncthreads();
+      cta_mm<D>(dA, X, true, lam, false, -rc.c2, slab);
+    } else {
+      for (long long e = tid; e < DD; e += kBT) dA[e] = 0.f;
+    }
+    for (long long e = tid; e < DD; e += kBT) dB[e] = rc.cpre * dX[e] + rc.cpost * lam[e];
+    if (tid < D) {
+      float acc = 0.f;
+      for (int i = 0; i < D; ++i) acc = fmaf(S_in[i * D + tid], dX[i * D + tid], acc);
+      dalpha2[((long long)dir * BH * F + bh * F + f) * D + tid] = acc;
+    }
+    __syncthreads();
+    for (long long e = tid; e < DD; e += kBT) {
+      const int jj = (int)(e % D);
+      lam[e] = dX[e] * alpha[((b * F + f) * H + h) * D + jj];
+    }
+    __syncthreads();
+  }
+  const float* g0 = din + (long long)(dir == 0 ? 0 : F) * DD;
+  for (long long e = tid; e < DD; e += kBT) dseed2[((long long)dir * BH + bh) * DD + e] = lam[e] + g0[e];
+}
+
+// ---------------------------------------------------------------- step 2 reversed (+ step 1 up to the conv)
+template <int D>
+struct StatsSmem {
+  float dAs[D * (D + 1)];   // dA + dA^T
+  float dB[D * (D + 1)];
+  float kf[kTok * (D + 1)];
+  float vf[kTok * (D + 1)];
+  float u[kTok * (D + 1)];  // (dA + dA^T) k'
+  float w[kTok * (D + 1)];  // dB^T v'
+  float z[kTok * (D + 1)];  // dB k'
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT) k_bwd_stats(const T* __restrict__ k, const T* __restrict__ v,
+                                                   const float* __restrict__ beta, const float* __restrict__ wk,
+                                                   const float* __restrict__ wv, int K,
+                                                   const float* __restrict__ dA2, const float* __restrict__ dB2,
+                                                   float* __restrict__ dkc, float* __restrict__ dvc,
+                                                   float* __restrict__ dbeta, int H, int F, int S) {
+  constexpr int PER = Lanes<D>::PER;
+  constexpr int TPW = kTok / (kBT / 32);      // tokens per warp and tile
+  extern __shared__ float smem_f[];
+  StatsSmem<D>& sm = *reinterpret_cast<StatsSmem<D>*>(smem_f);
+  const long long fi = blockIdx.x;
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long N = (long long)F * S;
+  const long long DD = (long long)D * D;
+  const long long BHF = (long long)gridDim.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (long long e = tid; e < DD; e += kBT) {
+    const int i = (int)(e / D), j = (int)(e % D);
+    const float a_ij = dA2[fi * DD + e] + dA2[(BHF + fi) * DD + e];
+    const float a_ji = dA2[fi * DD + j * D + i] + dA2[(BHF + fi) * DD + j * D + i];
+    sm.dAs[i * (D + 1) + j] = a_ij + a_ji;
+    sm.dB[i * (D + 1) + j] = dB2[fi * DD + e] + dB2[(BHF + fi) * DD + e];
+  }
+  const int pad = (K - 1) / 2;
+  for (int s0 = 0; s0 < S; s0 += kTok) {
+    // features of the tile's tokens; the pre-activations stay in registers
+    float kc[TPW][PER], vc[TPW][PER];
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int t = warp * TPW + tt, s = s0 + t;
+      float ks[PER];
+      float ss = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        kc[tt][r] = vc[tt][r] = ks[r] = 0.f;
+        const int c = lane + 32 * r;
+        if (s < S && Lanes<D>::has(lane, r)) {
+          float ak = 0.f, av = 0.f;
+          const long long base = ((b * N + (long long)f * S + s) * H + h) * D + c;
+          if (wk == nullptr) ak = to_f32(k[base]);
+          if (wv == nullptr) av = to_f32(v[base]);
+          for (int j = 0; j < K; ++j) {
+            const int sj = s + j - pad;
+            if (sj < 0 || sj >= S) continue;
+            const long long nb = ((b * N + (long long)f * S + sj) * H + h) * D + c;
+            if (wk) ak = fmaf(wk[((long long)h * D + c) * K + j], to_f32(k[nb]), ak);
+            if (wv) av = fmaf(wv[((long long)h * D + c) * K + j], to_f32(v[nb]), av);
+          }
+          kc[tt][r] = ak;
+          vc[tt][r] = av;
+          ks[r] = silu_precise(ak);
+        }
+        ss += ks[r] * ks[r];
+      }
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (Lanes<D>::has(lane, r)) {
+          sm.kf[t * (D + 1) + lane + 32 * r] = ks[r] * inv;
+          sm.vf[t * (D + 1) + lane + 32 * r] = s < S ? silu_precise(vc[tt][r]) : 0.f;
+        }
+    }
+    __syncthreads();
+    tile_matvec<D, false>(sm.u, sm.kf, sm.dAs);   // u_i = sum_j dAs[i][j] k'_j
+    tile_matvec<D, true>(sm.w, sm.vf, sm.dB);     // w_i = sum_j dB[j][i] v'_j
+    tile_matvec<D, false>(sm.z, sm.kf, sm.dB);    // z_i = sum_j dB[i][j] k'_j
+    __syncthreads();
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int t = warp * TPW + tt, s = s0 + t;
+      if (s >= S) continue;                        // warp-uniform
+      const long long tok = (b * N + (long long)f * S + s) * H + h;
+      const float bt = beta[tok];
+      float ks[PER], dkf[PER], dks[PER];
+      float kb = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        const int c = lane + 32 * r;
+        ks[r] = dkf[r] = 0.f;
+        if (!Lanes<D>::has(lane, r)) continue;
+        const float kfc = sm.kf[t * (D + 1) + c], vfc = sm.vf[t * (D + 1) + c];
+        const float u = sm.u[t * (D + 1) + c], w = sm.w[t * (D + 1) + c], z = sm.z[t * (D + 1) + c];
+        // d beta = k'^T dA k' + v'^T dB k' = 1/2 k'^T (dA + dA^T) k' + v' . (dB k')
+        kb += 0.5f * kfc * u + vfc * z;
+        dkf[r] = bt * (u + w);
+        ks[r] = silu_precise(kc[tt][r]);
+        dvc[tok * D + c] = silu_grad(vc[tt][r], bt * z);
+      }
+      kb = warp_sum(kb);
+      if (lane == 0) dbeta[tok] = kb;
+      l2n_grad<D>(ks, dkf, dks, lane);
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (Lanes<D>::has(lane, r)) dkc[tok * D + lane + 32 * r] = silu_grad(kc[tt][r], dks[r]);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- step 1 conv reversed
+// One warp per token (grid-stride within head h = blockIdx.y): dk[s] = sum_j w[j] dkc[s - j + p]
+// over in-frame indices; tap partials sum_s dkc[s] k[s + j - p] per block.
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT) k_bwd_conv(const T* __restrict__ k, const T* __restrict__ v,
+                                                  const float* __restrict__ wk, const float* __restrict__ wv,
+                                                  int K, const float* __restrict__ dkc,
+                                                  const float* __restrict__ dvc, T* __restrict__ dk,
+                                                  T* __restrict__ dv, float* __restrict__ tap_part, int B, int H,
+                                                  int F, int S) {
+  constexpr int PER = Lanes<D>::PER;
+  __shared__ float red[kBT / 32][2][D][3];
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long N = (long long)F * S;
+  const long long total = (long long)B * N;     // tokens of head h
+  const int pad = (K - 1) / 2;
+  float tk[PER][3], tv[PER][3];
+#pragma unroll
+  for (int r = 0; r < PER; ++r)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) tk[r][j] = tv[r][j] = 0.f;
+  for (long long tokn = (long long)blockIdx.x * (kBT / 32) + warp; tokn < total;
+       tokn += (long long)gridDim.x * (kBT / 32)) {
+    const long long b = tokn / N, n = tokn % N;
+    const int s = (int)(n % S);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      if (!Lanes<D>::has(lane, r)) continue;
+      const int c = lane + 32 * r;
+      const long long base = ((b * N + n) * H + h) * D + c;
+      float gk = 0.f, gv = 0.f;
+      if (wk == nullptr) gk = dkc[base];
+      if (wv == nullptr) gv = dvc[base];
+      for (int j = 0; j < K; ++j) {
+        // out[s'] uses x[s' + j - pad]: x[s] feeds out[s - j + pad]
+        const int so = s - j + pad;
+        if (so >= 0 && so < S) {
+          const long long ob = ((b * N + (n - s + so)) * H + h) * D + c;
+          if (wk) gk = fmaf(wk[((long long)h * D + c) * K + j], dkc[ob], gk);
+          if (wv) gv = fmaf(wv[((long long)h * D + c) * K + j], dvc[ob], gv);
+        }
+        const int sx = s + j - pad;               // tap j of out[s] reads x[s + j - pad]
+        if (sx >= 0 && sx < S) {
+          const long long xb = ((b * N + (n - s + sx)) * H + h) * D + c;
+          if (wk) tk[r][j] = fmaf(dkc[base], to_f32(k[xb]), tk[r][j]);
+          if (wv) tv[r][j] = fmaf(dvc[base], to_f32(v[xb]), tv[r][j]);
+        }
+      }
+      dk[base] = from_f32<T>(gk);
+      dv[base] = from_f32<T>(gv);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < PER; ++r)
+    if (Lanes<D>::has(lane, r))
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        red[warp][0][lane + 32 * r][j] = tk[r][j];
+        red[warp][1][lane + 32 * r][j] = tv[r][j];
+      }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 2 * D * 3; e += kBT) {
+    const int m = e / (D * 3), c = (e / 3) % D, j = e % 3;
+    float acc = 0.f;
+    for (int w = 0; w < kBT / 32; ++w) acc += red[w][m][c][j];
+    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * D * 3 + c * 3 + j] = acc;
+  }
+}
+
+// ---------------------------------------------------------------- reductions
+template <int D>
+__global__ void __launch_bounds__(kBT) k_bwd_finish(const float* __restrict__ rms_part, long long nfr,
+                                                    const float* __restrict__ tap_part, int conv_blocks, int K,
+                                                    const float* __restrict__ dseed2,
+                                                    const float* __restrict__ dalpha_g,
+                                                    const float* __restrict__ dalpha2, float* __restrict__ drms_w,
+                                                    float* __restrict__ dwk, float* __restrict__ dwv,
+                                                    float* __restrict__ dtext, float* __restrict__ dalpha, int B,
+                                                    int H, int F) {
+  const long long DD = (long long)D * D;
+  const long long BH = (long long)B * H;
+  const long long gtid = (long long)blockIdx.x * kBT + threadIdx.x;
+  const long long gsize = (long long)gridDim.x * kBT;
+  // d rms_w: sum over every (b, h, f) block of the read-out
+  for (long long c = gtid; c < D; c += gsize) {
+    float acc = 0.f;
+    for (long long i = 0; i < nfr; ++i) acc += rms_part[i * D + c];
+    drms_w[c] = acc;
+  }
+  // conv taps: sum over the conv blocks of each head
+  for (long long e = gtid; e < (long long)H * D * K; e += gsize) {
+    const int h = (int)(e / (D * K)), c = (int)((e / K) % D), j = (int)(e % K);
+    float ak = 0.f, av = 0.f;
+    for (int blk = 0; blk < conv_blocks; ++blk) {
+      const long long base = (((long long)h * conv_blocks + blk) * 2) * D * 3;
+      ak += tap_part[base + c * 3 + j];
+      av += tap_part[base + D * 3 + c * 3 + j];
+    }
+    if (dwk) dwk[e] = ak;
+    if (dwv) dwv[e] = av;
+  }
+  // text state: 0.5 (d seed of the prefix scan + d seed of the suffix scan), summed over the batch
+  if (dtext)
+    for (long long e = gtid; e < (long long)H * DD; e += gsize) {
+      const int h = (int)(e / DD);
+      const long long m = e % DD;
+      float acc = 0.f;
+      for (int b = 0; b < B; ++b) {
+        const long long bh = (long long)b * H + h;
+        acc += dseed2[bh * DD + m] + dseed2[(BH + bh) * DD + m];
+      }
+      dtext[e] = 0.5f * acc;
+    }
+  // d alpha [B, F, H, D] = bridge + prefix-scan + suffix-scan parts ([B, H, F, D] each)
+  for (long long e = gtid; e < BH * F * D; e += gsize) {
+    const int c = (int)(e % D);
+    const int f = (int)((e / D) % F);
+    const long long bh = e / ((long long)F * D);
+    const int h = (int)(bh % H);
+    const long long b = bh / H;
+    const float acc = dalpha_g[e] + dalpha2[e] + dalpha2[BH * F * D + e];
+    dalpha[((b * F + f) * H + h) * D + c] = acc;
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- host side
+BwdPlan plan_backward(const vdn_shape& sh, int rule) {
+  BwdPlan p;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const bool tc = use_tc(sh, VDN_IMPL_AUTO);
+  const size_t fwd = plan_workspace(sh, rule, tc).total;
+  const long long BH = (long long)sh.B * sh.H, NF = BH * sh.F, DD = (long long)sh.d * sh.d;
+  const long long tokens = (long long)sh.B * sh.F * sh.S * sh.H;
+  const size_t el = sh.dtype == VDN_DTYPE_BF16 ? 2 : 4;
+  p.fwd = take(fwd);
+  p.out = take(tokens * sh.d * el);
+  p.A = take(NF * DD * 4);
+  p.Bm = take(NF * DD * 4);
+  p.Nm = take(NF * DD * 4);
+  p.P = take(NF * DD * 4);
+  p.Q = take(NF * DD * 4);
+  p.W = take(NF * DD * 4);
+  p.dW = take(NF * DD * 4);
+  p.dPin = take(BH * (sh.F + 1) * DD * 4);
+  p.dQin = take(BH * (sh.F + 1) * DD * 4);
+  p.dA2 = take(2 * NF * DD * 4);
+  p.dB2 = take(2 * NF * DD * 4);
+  p.dalpha_g = take(NF * sh.d * 4);
+  p.dalpha2 = take(2 * NF * sh.d * 4);
+  p.dseed2 = take(2 * BH * DD * 4);
+  p.scan_scratch = take(BH * 2 * 4 * DD * 4);
+  p.rms_part = take(NF * sh.d * 4);
+  p.dkc = take(tokens * sh.d * 4);
+  p.dvc = take(tokens * sh.d * 4);
+  p.tap_part = take((size_t)sh.H * kBwdConvBlocks * 2 * sh.d * 3 * 4);
+  p.fwd_bytes = fwd;
+  p.total = off;
+  return p;
+}
+
+template <int D, typename T>
+static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p) {
+  auto at = [&](size_t o) { return reinterpret_cast<float*>(static_cast<char*>(ws) + o); };
+  const vdn_shape& sh = a.sh;
+  const long long BH = (long long)sh.B * sh.H, NF = BH * sh.F;
+  const int K = (a.conv_k_w || a.conv_v_w) ? sh.conv_width : 1;
+  // step 5 reversed
+  {
+    const size_t smem = sizeof(ReadoutSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_readout<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_bwd_readout<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.gate), static_cast<const T*>(g.dout), a.rms_w, at(p.W),
+        at(p.dW), at(p.rms_part), static_cast<T*>(g.dq), static_cast<T*>(g.dgate), sh.H, sh.F, sh.S);
+  }
+  // step 4 (gather + bridge) reversed
+  k_bwd_gather<D><<<(unsigned)BH, kBT, 0, a.stream>>>(at(p.P), at(p.Q), a.alpha, a.text_state, at(p.dW), at(p.dPin),
+                                                      at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk, a.radius);
+  // steps 3-4 (scans) reversed
+  k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(
+      at(p.Bm), at(p.Nm), at(p.P), at(p.Q), a.alpha, a.text_state, rule_coef(a.rule, a.c), at(p.dPin), at(p.dQin),
+      at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  // step 2 reversed
+  {
+    const size_t smem = sizeof(StatsSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_stats<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_bwd_stats<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
+        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.beta, a.conv_k_w, a.conv_v_w, K, at(p.dA2),
+        at(p.dB2), at(p.dkc), at(p.dvc), g.dbeta, sh.H, sh.F, sh.S);
+  }
+  // step 1 (conv) reversed
+  k_bwd_conv<D, T><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
+      static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, K, at(p.dkc), at(p.dvc),
+      static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  k_bwd_finish<D><<<148, kBT, 0, a.stream>>>(at(p.rms_part), NF, at(p.tap_part), kBwdConvBlocks, K, at(p.dseed2),
+                                             at(p.dalpha_g), at(p.dalpha2), g.drms_w, g.dconv_k_w, g.dconv_v_w,
+                                             g.dtext_state, g.dalpha, sh.B, sh.H, sh.F);
+  return cudaGetLastError();
+}
+
+cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p) {
+  const vdn_shape& sh = a.sh;
+  const long long BH = (long long)sh.B * sh.H, DD = (long long)sh.d * sh.d;
+  char* base = static_cast<char*>(ws);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(base + p.dPin, 0, BH * (sh.F + 1) * DD * 4, a.stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(base + p.dQin, 0, BH * (sh.F + 1) * DD * 4, a.stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(base + p.dalpha_g, 0, BH * sh.F * sh.d * 4, a.stream)) != cudaSuccess) return e;
+  const bool bf = sh.dtype == VDN_DTYPE_BF16;
+  if (sh.d == 16) return bf ? run_backward_t<16, __nv_bfloat16>(a, g, ws, p) : run_backward_t<16, float>(a, g, ws, p);
+  return bf ? run_backward_t<128, __nv_bfloat16>(a, g, ws, p) : run_backward_t<128, float>(a, g, ws, p);
+}
+
+}  // namespace vdn

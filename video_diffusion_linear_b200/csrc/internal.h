@@ -64,6 +64,37 @@ cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, 
 // dst = src * 2^expo[frame] (expo may be NULL)
 cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo = nullptr);
 
+// ---- backward pass of the branch (backward.cu)
+constexpr int kBwdConvBlocks = 148;   // blocks per head of the conv-reversal kernel
+// Byte offsets of the backward workspace (each 256-byte aligned): the forward's own workspace,
+// a scratch output, the forward's per-frame export and the adjoint buffers.
+struct BwdPlan {
+  size_t fwd = 0, out = 0;
+  size_t A = 0, Bm = 0, Nm = 0, P = 0, Q = 0, W = 0;   // fp32 [B, H, F, d, d]
+  size_t dW = 0;                                       // fp32 [B, H, F, d, d]
+  size_t dPin = 0, dQin = 0;                           // fp32 [B, H, F + 1, d, d]
+  size_t dA2 = 0, dB2 = 0;                             // fp32 [2][B, H, F, d, d] (prefix, suffix scan)
+  size_t dalpha_g = 0, dalpha2 = 0;                    // fp32 [B, H, F, d], [2][B, H, F, d]
+  size_t dseed2 = 0;                                   // fp32 [2][B, H, d, d]
+  size_t scan_scratch = 0;                             // fp32 [B, H, 2][4][d, d]
+  size_t rms_part = 0;                                 // fp32 [B, H, F][d]
+  size_t dkc = 0, dvc = 0;                             // fp32 [B, N, H, d]
+  size_t tap_part = 0;                                 // fp32 [H][kBwdConvBlocks][2][d][3]
+  size_t fwd_bytes = 0, total = 0;
+};
+struct BwdGrads {
+  const void* dout;
+  void* dq; void* dk; void* dv;
+  float* dbeta; float* dalpha;
+  void* dgate;
+  float* drms_w;
+  float* dconv_k_w; float* dconv_v_w;
+  float* dtext_state;
+};
+BwdPlan plan_backward(const vdn_shape& sh, int rule);
+// the backward kernels, after the forward has filled the plan's A .. W regions
+cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p);
+
 // standalone step 1 (dtype in, dtype out)
 cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,
                                 const float* wk, const float* wv, void* qo, void* ko, void* vo,

@@ -297,6 +297,97 @@ size_t vdn_branch_workspace_size(const vdn_shape* shape, int rule) {
   return vdn_branch_workspace_size_impl(shape, rule, VDN_IMPL_AUTO);
 }
 
+size_t vdn_branch_backward_workspace_size(const vdn_shape* shape, int rule) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  if (rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE) return 0;
+  return plan_backward(*shape, rule).total;
+}
+
+vdn_status vdn_branch_backward(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                               const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                               const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,
+                               float c, int chunk, int radius, const void* dout, void* workspace,
+                               size_t workspace_bytes, void* dq, void* dk, void* dv, float* dbeta, float* dalpha,
+                               void* dgate, float* drms_w, float* dconv_k_w, float* dconv_v_w,
+                               float* dtext_state, void* stream) {
+  // the forward's checks, with dq standing for the output (it must not overlap an input either)
+  if (check_shape(shape) != VDN_OK) return check_shape(shape);
+  const BwdPlan plan = plan_backward(*shape, rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE
+                                                 ? VDN_RULE_VDN_SOLVE : rule);
+  vdn_status s = validate(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                          radius, workspace, workspace_bytes, dq, VDN_IMPL_AUTO);
+  if (s != VDN_OK) return s;
+  if (workspace_bytes < plan.total) return VDN_ERR_WORKSPACE;
+  if (!dout || !dk || !dv || !dbeta || !dalpha || !dgate || !drms_w) return VDN_ERR_INVALID_ARG;
+  // a gradient exists exactly for the optional inputs that were given
+  if ((conv_k_w == nullptr) != (dconv_k_w == nullptr) || (conv_v_w == nullptr) != (dconv_v_w == nullptr) ||
+      (text_state == nullptr) != (dtext_state == nullptr))
+    return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {dout, dk, dv, dbeta, dalpha, dgate, drms_w, dconv_k_w, dconv_v_w, dtext_state};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  // gradients must not overlap each other, an input or the workspace
+  const size_t es = elem_size(shape->dtype);
+  const size_t tok = (size_t)shape->B * shape->F * shape->S * shape->H;
+  const size_t big = tok * shape->d * es;
+  const size_t d = (size_t)shape->d;
+  const size_t nal = (size_t)shape->B * shape->F * shape->H * d * 4;
+  const size_t ntap = (size_t)shape->H * d * shape->conv_width * 4;
+  const Range outs[] = {
+      {(uintptr_t)dq, (uintptr_t)dq + big}, {(uintptr_t)dk, (uintptr_t)dk + big},
+      {(uintptr_t)dv, (uintptr_t)dv + big}, {(uintptr_t)dgate, (uintptr_t)dgate + big},
+      {(uintptr_t)dbeta, (uintptr_t)dbeta + tok * 4}, {(uintptr_t)dalpha, (uintptr_t)dalpha + nal},
+      {(uintptr_t)drms_w, (uintptr_t)drms_w + d * 4},
+      {(uintptr_t)dconv_k_w, dconv_k_w ? (uintptr_t)dconv_k_w + ntap : 0},
+      {(uintptr_t)dconv_v_w, dconv_v_w ? (uintptr_t)dconv_v_w + ntap : 0},
+      {(uintptr_t)dtext_state, dtext_state ? (uintptr_t)dtext_state + (size_t)shape->H * d * d * 4 : 0},
+  };
+  const Range ins[] = {
+      {(uintptr_t)q, (uintptr_t)q + big}, {(uintptr_t)k, (uintptr_t)k + big}, {(uintptr_t)v, (uintptr_t)v + big},
+      {(uintptr_t)gate, (uintptr_t)gate + big}, {(uintptr_t)dout, (uintptr_t)dout + big},
+      {(uintptr_t)beta, (uintptr_t)beta + tok * 4}, {(uintptr_t)alpha, (uintptr_t)alpha + nal},
+      {(uintptr_t)rms_w, (uintptr_t)rms_w + d * 4},
+      {(uintptr_t)conv_k_w, conv_k_w ? (uintptr_t)conv_k_w + ntap : 0},
+      {(uintptr_t)conv_v_w, conv_v_w ? (uintptr_t)conv_v_w + ntap : 0},
+      {(uintptr_t)text_state, text_state ? (uintptr_t)text_state + (size_t)shape->H * d * d * 4 : 0},
+      {(uintptr_t)workspace, (uintptr_t)workspace + plan.total},
+  };
+  const int no = sizeof(outs) / sizeof(outs[0]), ni = sizeof(ins) / sizeof(ins[0]);
+  for (int i = 0; i < no; ++i) {
+    if (outs[i].hi <= outs[i].lo) continue;
+    for (int j = 0; j < ni; ++j)
+      if (ins[j].hi > ins[j].lo && overlap(outs[i], ins[j])) return VDN_ERR_INVALID_ARG;
+    for (int j = i + 1; j < no; ++j)
+      if (outs[j].hi > outs[j].lo && overlap(outs[i], outs[j])) return VDN_ERR_INVALID_ARG;
+  }
+  // forward with the per-frame export into the backward workspace
+  char* ws = static_cast<char*>(workspace);
+  vdn_debug_out dbg;
+  dbg.impl = VDN_IMPL_AUTO;
+  dbg.A = at<float>(ws, plan.A);
+  dbg.B = at<float>(ws, plan.Bm);
+  dbg.N = at<float>(ws, plan.Nm);
+  dbg.P = at<float>(ws, plan.P);
+  dbg.Q = at<float>(ws, plan.Q);
+  dbg.W = at<float>(ws, plan.W);
+  Args a;
+  a.sh = *shape;
+  a.q = q; a.k = k; a.v = v;
+  a.beta = beta; a.alpha = alpha; a.gate = gate; a.rms_w = rms_w;
+  a.conv_k_w = conv_k_w; a.conv_v_w = conv_v_w; a.text_state = text_state;
+  a.rule = rule; a.c = (rule == VDN_RULE_VDN_SOLVE || rule == VDN_RULE_ADDITIVE) ? 1.0f : c;
+  a.chunk = chunk; a.radius = radius;
+  a.out = ws + plan.out;
+  a.stream = (cudaStream_t)stream;
+  a.dbg = &dbg;
+  s = run_forward(a, ws + plan.fwd, VDN_IMPL_AUTO);
+  if (s != VDN_OK) return s;
+  a.dbg = nullptr;
+  BwdGrads g{dout, dq, dk, dv, dbeta, dalpha, dgate, drms_w, dconv_k_w, dconv_v_w, dtext_state};
+  if (run_backward(a, g, ws, plan) != cudaSuccess) return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
 vdn_status vdn_branch_forward(const vdn_shape* shape, const void* q, const void* k, const void* v,
                               const float* beta, const float* alpha, const void* gate, const float* rms_w,
                               const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,

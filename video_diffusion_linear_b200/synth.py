@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 # draw order / stream ids
-_Q, _K, _V, _BETA, _ALPHA, _GATE, _RMSW, _CONVK, _CONVV, _TEXT, _QR, _KR = range(12)
+_Q, _K, _V, _BETA, _ALPHA, _GATE, _RMSW, _CONVK, _CONVV, _TEXT, _QR, _KR, _DOUT = range(13)
 _CHUNK = 1 << 22
 
 RULE_IDS = {"sana_scaled": 0, "vdn_solve": 1, "vdn_scaled": 2, "additive": 3}
@@ -142,3 +142,11 @@ def make_inputs(w: Workload, *, threads: int | None = None, with_text: bool | No
             out["q_rope"] = _draw(w.seed, _QR, (B, N, H, d), "normal", 0.0, 2.0, dt, pool)
             out["k_rope"] = _draw(w.seed, _KR, (B, N, H, d), "normal", 0.0, 1.0, dt, pool)
     return out
+
+
+def make_cotangent(w: Workload, *, threads: int | None = None) -> torch.Tensor:
+    """Upstream gradient dL/d out for the backward pass: N(0, 1) of the output's shape
+    and dtype (the loss L = <dout, out>), from its own stream of the workload's seed."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    with ThreadPoolExecutor(threads) as pool:
+        return _draw(w.seed, _DOUT, (w.B, w.N, w.H, w.d), "normal", 0.0, 1.0, dt, pool)
