@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 768p] [--impl reference]
     python bench.py --path softmax|hybrid --steps 10 --warmup 3     # the windowed softmax branch / whole layer
+    python bench.py --path backward --steps 5 --warmup 3            # gradients of the linear branch
 
 One step is one vdn_branch_forward call over the whole workload (all heads,
 all frames) with the inputs resident in HBM.  Prints ONE JSON line (rank 0):
@@ -41,7 +42,9 @@ import torch  # noqa: E402
 from video_diffusion_linear_b200 import synth  # noqa: E402
 
 METRIC = "latent tokens/sec through VDN linear branch fwd (1 B200); % of roofline"
-METRIC_PATH = {"softmax": "latent tokens/sec through the windowed softmax branch fwd (1 B200)",
+METRIC_PATH = {"backward": "latent tokens/sec through the VDN linear branch backward (forward recompute + "
+                           "gradients of every input, 1 B200)",
+               "softmax": "latent tokens/sec through the windowed softmax branch fwd (1 B200)",
                "hybrid": "latent tokens/sec through the VDN-H3 hybrid attention layer fwd (softmax + linear branch, 1 B200)"}
 DEFAULT_WORKLOAD = "768p"
 KERNELS_TC = ["frame_stats", "frame_solve", "scan", "gather", "readout"]
@@ -102,6 +105,25 @@ def softmax_flops(w: synth.Workload) -> float:
         hi = min(w.F - 1, w.chunk * (c + w.radius + 1) - 1)
         pairs += w.S * (hi - lo + 1) * w.S
     return 4.0 * w.d * pairs * w.B * w.H
+
+
+BWD_KERNELS = ["forward_recompute", "readout_bwd", "gather_bwd", "scan_bwd", "stats_bwd", "conv_bwd", "finish_bwd"]
+
+
+def backward_flops(w: synth.Workload) -> dict:
+    """Algorithmic FLOPs of the backward kernels that are contractions: the read-out's
+    o = W q', dq' = W^T do and dW = sum do q'^T, and the statistics' (dA + dA^T) k',
+    dB^T v', dB k' (2 d^2 each per token-head); the adjoint scans' two d x d products
+    per frame and direction (2 d^3 each)."""
+    TH = w.B * w.F * w.S * w.H
+    NF = w.B * w.H * w.F
+    return {"readout_bwd": 6.0 * w.d * w.d * TH, "stats_bwd": 6.0 * w.d * w.d * TH,
+            "scan_bwd": 2 * 2 * 2.0 * w.d ** 3 * NF}
+
+
+def fp32_peak_tflops(sm_mhz: float) -> float:
+    """FP32 FMA rate of the SIMT pipes: 148 SMs x 128 lanes x 2 FLOP per cycle."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def load_peaks() -> tuple[dict, str]:
@@ -271,6 +293,8 @@ def run_reference(args, w: synth.Workload) -> None:
     rank, world, _ = dist_env()
     if rank != 0:
         return
+    if args.path == "backward":
+        return run_reference_backward(args, w)
     if args.path != "linear":
         return run_reference_softmax(args, w)
     inp = synth.make_inputs(w)
@@ -321,7 +345,161 @@ def run_reference_softmax(args, w: synth.Workload) -> None:
     }), flush=True)
 
 
+def backward_oracle_sample(inp: dict, dout, w: synth.Workload, h: int) -> tuple[float, int]:
+    """Runs the float64 backward oracle over one (batch 0, head h): all frames and tokens."""
+    from oracle import vdn_backward as BW
+    t0 = time.perf_counter()
+    BW.head_backward(inp, 0, h, w.F, w.S, w.rule, w.c, w.chunk, w.radius, dout[0, :, h, :])
+    return time.perf_counter() - t0, w.F * w.S
+
+
+def run_reference_backward(args, w: synth.Workload) -> None:
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, th = backward_oracle_sample(inp, dout, w, i % w.H)
+        if i >= args.warmup:
+            times.append(dt)
+    step = sum(times) / len(times)
+    value = (th / w.H) / step
+    sample = f"one head of {w.H} per step (all {w.F} frames x {w.S} tokens), batch 0; tokens counted x 1/H"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC_PATH["backward"], "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(w)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 # ----------------------------------------------------------------------------- GPU arm
+def run_gpu_backward(args, w: synth.Workload) -> None:
+    """The branch's backward pass (vdn_branch_backward: forward recompute, then the
+    gradients of every input) on one or more GPUs (independent clips per rank)."""
+    from video_diffusion_linear_b200 import _lib, api
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    _lib.load()
+    wr = rank_workload(w, rank)
+    host = synth.make_inputs(wr)
+    host["dout"] = synth.make_cotangent(wr)
+    dev = api.to_device(host, device)
+    args_t = api.forward_inputs(dev)
+    shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
+    ws = torch.empty(api.backward_workspace_size(shape, w.rule), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    # forward kernels + copies of its per-frame export (B, P, Q, W; SIMT also A, N) + backward kernels
+    nfwd = api.launch_count(shape)
+    launches = nfwd + (4 if nfwd == 5 else 6) + len(BWD_KERNELS) - 1
+    grads = api.branch_backward(*args_t, dout=dev["dout"], F=w.F, rule=w.rule, c=w.c, chunk=w.chunk,
+                                radius=w.radius, workspace=ws, stream=stream)
+
+    def step(events=None):
+        api.branch_backward(*args_t, dout=dev["dout"], F=w.F, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius,
+                            grads=grads, workspace=ws, stream=stream, events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if api.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+    nk = len(BWD_KERNELS)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    for evs in kev:
+        for e in evs:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(kev[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end)
+    ms_max = reduce_max(ms, device)
+    value = w.tokens * world * args.steps / (ms_max / 1e3)
+    per = {n: statistics.fmean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
+           for j, n in enumerate(BWD_KERNELS)}
+    flops = backward_flops(w)
+    bwd_only = {n: v for n, v in per.items() if n != "forward_recompute"}
+    dom = max(bwd_only, key=bwd_only.get)
+    csum = clk.summary()
+    clock = csum.get("sm_mhz") or csum.get("sm_max_mhz") or 1965.0
+    peak = fp32_peak_tflops(float(csum.get("sm_max_mhz") or 1965.0))
+    achieved = flops[dom] / (per[dom] / 1e3) / 1e12 if dom in flops else None
+    roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak if achieved else None,
+            "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock (fp32 FMA, SIMT kernels)",
+            "algorithmic_flops_per_launch": flops.get(dom), "traffic": None, "median_sm_mhz": clock}
+    kernels = {n: {"us": per[n] * 1e3, "share": per[n] / sum(per.values()),
+                   "tflops": (flops[n] / (per[n] / 1e3) / 1e12) if n in flops else None} for n in per}
+
+    e2e = None
+    if not args.no_e2e:
+        keys = ["q", "k", "v", "beta", "alpha", "gate", "dout"]
+        pinned = {k: host[k].pin_memory() for k in keys}
+        outs = ["dq", "dk", "dv", "dgate", "dbeta", "dalpha"]
+        host_out = {k: torch.empty(grads[k].shape, dtype=grads[k].dtype).pin_memory() for k in outs}
+        h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            for k in outs:
+                host_out[k].copy_(grads[k], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu and world == 1:
+        dt, th = backward_oracle_sample(host, host["dout"], w, 0)
+        cpu = {"value": (th / w.H) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"head 0 of {w.H}, batch 0, all {w.F} frames x {w.S} tokens ({dt:.1f} s); "
+                         "tokens counted x 1/H"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC_PATH["backward"], "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (bf16 inputs and gradients)", "data": "synthetic",
+        "config": {"workload": describe(w) + ", upstream gradient N(0, 1)", "global_batch": w.B * world,
+                   "tokens_per_step": w.tokens * world,
+                   "l2": "inputs larger than L2 (q, k, v, gate, dout: %.2f GB)" % (5 * w.tokens * w.H * w.d * 2 / 1e9),
+                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches * args.steps,
+        "clocks": csum,
+    }), flush=True)
+
+
 def run_gpu_softmax(args, w: synth.Workload) -> None:
     """The windowed softmax branch (--path softmax) or the whole hybrid layer
     (--path hybrid) on one or more GPUs (independent clips per rank)."""
@@ -606,8 +784,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=2)
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
-    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid"],
-                    help="linear branch (default), windowed softmax branch, or the whole hybrid layer")
+    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid", "backward"],
+                    help="linear branch (default), windowed softmax branch, the whole hybrid layer, or the "
+                         "linear branch's backward pass")
     ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -621,6 +800,8 @@ def main(argv=None):
         w = w.replace(H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.path == "backward":
+        run_gpu_backward(args, w)
     elif args.path != "linear":
         run_gpu_softmax(args, w)
     else:

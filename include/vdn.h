@@ -287,6 +287,24 @@ vdn_status vdn_branch_backward(const vdn_shape* shape,
                                float* dconv_k_w, float* dconv_v_w, float* dtext_state,
                                void* stream);
 
+/* vdn_branch_backward that also records caller-created CUDA events on `stream`:
+ * events[0] before the forward recompute, events[1] after it, then events[2..7]
+ * after each backward kernel (read-out, gather and bridge, adjoint scans, frame
+ * statistics, conv, reductions).  n_events must be at least 8. */
+vdn_status vdn_branch_backward_timed(const vdn_shape* shape,
+                                     const void* q, const void* k, const void* v,
+                                     const float* beta, const float* alpha,
+                                     const void* gate, const float* rms_w,
+                                     const float* conv_k_w, const float* conv_v_w,
+                                     const float* text_state,
+                                     int rule, float c, int chunk, int radius,
+                                     const void* dout,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* dq, void* dk, void* dv,
+                                     float* dbeta, float* dalpha, void* dgate, float* drms_w,
+                                     float* dconv_k_w, float* dconv_v_w, float* dtext_state,
+                                     void* stream, void* const* events, int n_events);
+
 /* Reads the device status word that bounded waits inside the kernels set (it
  * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
  * Synchronises `stream`. */

@@ -178,7 +178,7 @@ def head_backward(inp: dict, b: int, h: int, F: int, S: int, rule: str, c: float
     d = q.shape[-1]
     ts = inp.get("text_state")
     seed = O.seed_state(None if ts is None else O._f64(ts[h]), d)
-    dout = np.asarray(dout_bh, dtype=np.float64).reshape(F, S, d)
+    dout = O._f64(dout_bh).reshape(F, S, d)
 
     # forward, keeping what the reverse steps read
     q3, k3, v3 = q.reshape(F, S, d), k.reshape(F, S, d), v.reshape(F, S, d)

@@ -59,6 +59,10 @@ _SIGNATURES = {
     "vdn_branch_backward": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P, _P,
                                            ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vdn_branch_backward_timed": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                 _P, ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P,
+                                                 _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                 ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "vdn_workspace_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "vdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }

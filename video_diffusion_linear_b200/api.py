@@ -189,10 +189,13 @@ def backward_workspace_size(shape: VdnShape, rule="vdn_solve") -> int:
 
 
 def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *, dout,
-                    F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, grads=None, workspace=None, stream=None):
+                    F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, grads=None, workspace=None, stream=None,
+                    events=None):
     """vdn_branch_backward: gradients of <dout, branch_forward(...)> with respect to every
     input.  Returns a dict dq, dk, dv, dgate (q's dtype), dbeta, dalpha, drms_w, and
-    dconv_k_w, dconv_v_w, dtext_state (fp32; None where the input is None)."""
+    dconv_k_w, dconv_v_w, dtext_state (fp32; None where the input is None).  With
+    `events` (8 torch.cuda.Event), vdn_branch_backward_timed records them between the
+    forward recompute and each backward kernel."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
     dev = q.device
     if grads is None:
@@ -206,12 +209,16 @@ def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=N
     if workspace is None:
         workspace = torch.empty(backward_workspace_size(shape, rule), dtype=torch.uint8, device=dev)
     g = grads
-    st = _lib.load().vdn_branch_backward(
-        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
-        _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
-        _ptr(dout), _ptr(workspace), workspace.numel(), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
-        _ptr(g["dbeta"]), _ptr(g["dalpha"]), _ptr(g["dgate"]), _ptr(g["drms_w"]), _ptr(g["dconv_k_w"]),
-        _ptr(g["dconv_v_w"]), _ptr(g["dtext_state"]), _stream_ptr(stream))
+    args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
+            _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
+            _ptr(dout), _ptr(workspace), workspace.numel(), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+            _ptr(g["dbeta"]), _ptr(g["dalpha"]), _ptr(g["dgate"]), _ptr(g["drms_w"]), _ptr(g["dconv_k_w"]),
+            _ptr(g["dconv_v_w"]), _ptr(g["dtext_state"]), _stream_ptr(stream))
+    if events is None:
+        st = _lib.load().vdn_branch_backward(*args)
+    else:
+        arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        st = _lib.load().vdn_branch_backward_timed(*args, arr, len(events))
     check(st, "vdn_branch_backward")
     return grads
 

@@ -702,7 +702,13 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule) {
 }
 
 template <int D, typename T>
-static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p) {
+static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p,
+                                  void* const* events) {
+  int ev = 2;   // events[0], events[1]: before and after the forward recompute
+  auto mark = [&]() -> cudaError_t {
+    return events ? cudaEventRecord((cudaEvent_t)events[ev++], a.stream) : cudaSuccess;
+  };
+  cudaError_t e;
   auto at = [&](size_t o) { return reinterpret_cast<float*>(static_cast<char*>(ws) + o); };
   const vdn_shape& sh = a.sh;
   const long long BH = (long long)sh.B * sh.H, NF = BH * sh.F;
@@ -710,39 +716,45 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   // step 5 reversed
   {
     const size_t smem = sizeof(ReadoutSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_readout<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k_bwd_readout<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k_bwd_readout<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.gate), static_cast<const T*>(g.dout), a.rms_w, at(p.W),
         at(p.dW), at(p.rms_part), static_cast<T*>(g.dq), static_cast<T*>(g.dgate), sh.H, sh.F, sh.S);
   }
+  if ((e = mark()) != cudaSuccess) return e;
   // step 4 (gather + bridge) reversed
   k_bwd_gather<D><<<(unsigned)BH, kBT, 0, a.stream>>>(at(p.P), at(p.Q), a.alpha, a.text_state, at(p.dW), at(p.dPin),
                                                       at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk, a.radius);
+  if ((e = mark()) != cudaSuccess) return e;
   // steps 3-4 (scans) reversed
   k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(
       at(p.Bm), at(p.Nm), at(p.P), at(p.Q), a.alpha, a.text_state, rule_coef(a.rule, a.c), at(p.dPin), at(p.dQin),
       at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed
   {
     const size_t smem = sizeof(StatsSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_stats<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k_bwd_stats<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k_bwd_stats<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
         static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.beta, a.conv_k_w, a.conv_v_w, K, at(p.dA2),
         at(p.dB2), at(p.dkc), at(p.dvc), g.dbeta, sh.H, sh.F, sh.S);
   }
+  if ((e = mark()) != cudaSuccess) return e;
   // step 1 (conv) reversed
   k_bwd_conv<D, T><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
       static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, K, at(p.dkc), at(p.dvc),
       static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  if ((e = mark()) != cudaSuccess) return e;
   k_bwd_finish<D><<<148, kBT, 0, a.stream>>>(at(p.rms_part), NF, at(p.tap_part), kBwdConvBlocks, K, at(p.dseed2),
                                              at(p.dalpha_g), at(p.dalpha2), g.drms_w, g.dconv_k_w, g.dconv_v_w,
                                              g.dtext_state, g.dalpha, sh.B, sh.H, sh.F);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mark();
 }
 
-cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p) {
+cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events) {
   const vdn_shape& sh = a.sh;
   const long long BH = (long long)sh.B * sh.H, DD = (long long)sh.d * sh.d;
   char* base = static_cast<char*>(ws);
@@ -751,8 +763,8 @@ cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPl
   if ((e = cudaMemsetAsync(base + p.dQin, 0, BH * (sh.F + 1) * DD * 4, a.stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(base + p.dalpha_g, 0, BH * sh.F * sh.d * 4, a.stream)) != cudaSuccess) return e;
   const bool bf = sh.dtype == VDN_DTYPE_BF16;
-  if (sh.d == 16) return bf ? run_backward_t<16, __nv_bfloat16>(a, g, ws, p) : run_backward_t<16, float>(a, g, ws, p);
-  return bf ? run_backward_t<128, __nv_bfloat16>(a, g, ws, p) : run_backward_t<128, float>(a, g, ws, p);
+  if (sh.d == 16) return bf ? run_backward_t<16, __nv_bfloat16>(a, g, ws, p, events) : run_backward_t<16, float>(a, g, ws, p, events);
+  return bf ? run_backward_t<128, __nv_bfloat16>(a, g, ws, p, events) : run_backward_t<128, float>(a, g, ws, p, events);
 }
 
 }  // namespace vdn

@@ -92,8 +92,11 @@ struct BwdGrads {
   float* dtext_state;
 };
 BwdPlan plan_backward(const vdn_shape& sh, int rule);
-// the backward kernels, after the forward has filled the plan's A .. W regions
-cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p);
+// the backward kernels, after the forward has filled the plan's A .. W regions; when `events` is
+// not NULL, events[2 .. kBwdKernels + 1] are recorded after each of them (events[0] and events[1] bracket
+// the forward recompute)
+constexpr int kBwdKernels = 6;
+cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events);
 
 // standalone step 1 (dtype in, dtype out)
 cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,

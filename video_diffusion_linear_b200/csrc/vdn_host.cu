@@ -303,13 +303,15 @@ size_t vdn_branch_backward_workspace_size(const vdn_shape* shape, int rule) {
   return plan_backward(*shape, rule).total;
 }
 
-vdn_status vdn_branch_backward(const vdn_shape* shape, const void* q, const void* k, const void* v,
-                               const float* beta, const float* alpha, const void* gate, const float* rms_w,
-                               const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,
-                               float c, int chunk, int radius, const void* dout, void* workspace,
-                               size_t workspace_bytes, void* dq, void* dk, void* dv, float* dbeta, float* dalpha,
-                               void* dgate, float* drms_w, float* dconv_k_w, float* dconv_v_w,
-                               float* dtext_state, void* stream) {
+}  // extern "C"
+
+namespace {
+vdn_status backward_common(const vdn_shape* shape, const void* q, const void* k, const void* v, const float* beta,
+                           const float* alpha, const void* gate, const float* rms_w, const float* conv_k_w,
+                           const float* conv_v_w, const float* text_state, int rule, float c, int chunk, int radius,
+                           const void* dout, void* workspace, size_t workspace_bytes, void* dq, void* dk, void* dv,
+                           float* dbeta, float* dalpha, void* dgate, float* drms_w, float* dconv_k_w,
+                           float* dconv_v_w, float* dtext_state, void* stream, void* const* events, int n_events) {
   // the forward's checks, with dq standing for the output (it must not overlap an input either)
   if (check_shape(shape) != VDN_OK) return check_shape(shape);
   const BwdPlan plan = plan_backward(*shape, rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE
@@ -380,12 +382,48 @@ vdn_status vdn_branch_backward(const vdn_shape* shape, const void* q, const void
   a.out = ws + plan.out;
   a.stream = (cudaStream_t)stream;
   a.dbg = &dbg;
+  if (events) {
+    if (n_events < kBwdKernels + 2) return VDN_ERR_INVALID_ARG;
+    for (int i = 0; i < kBwdKernels + 2; ++i)
+      if (!events[i]) return VDN_ERR_INVALID_ARG;
+    if (cudaEventRecord((cudaEvent_t)events[0], a.stream) != cudaSuccess) return VDN_ERR_CUDA;
+  }
   s = run_forward(a, ws + plan.fwd, VDN_IMPL_AUTO);
   if (s != VDN_OK) return s;
+  if (events && cudaEventRecord((cudaEvent_t)events[1], a.stream) != cudaSuccess) return VDN_ERR_CUDA;
   a.dbg = nullptr;
   BwdGrads g{dout, dq, dk, dv, dbeta, dalpha, dgate, drms_w, dconv_k_w, dconv_v_w, dtext_state};
-  if (run_backward(a, g, ws, plan) != cudaSuccess) return VDN_ERR_CUDA;
+  if (run_backward(a, g, ws, plan, events) != cudaSuccess) return VDN_ERR_CUDA;
   return VDN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+vdn_status vdn_branch_backward(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                               const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                               const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,
+                               float c, int chunk, int radius, const void* dout, void* workspace,
+                               size_t workspace_bytes, void* dq, void* dk, void* dv, float* dbeta, float* dalpha,
+                               void* dgate, float* drms_w, float* dconv_k_w, float* dconv_v_w,
+                               float* dtext_state, void* stream) {
+  return backward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                         radius, dout, workspace, workspace_bytes, dq, dk, dv, dbeta, dalpha, dgate, drms_w,
+                         dconv_k_w, dconv_v_w, dtext_state, stream, nullptr, 0);
+}
+
+vdn_status vdn_branch_backward_timed(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                                     const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                                     const float* conv_k_w, const float* conv_v_w, const float* text_state,
+                                     int rule, float c, int chunk, int radius, const void* dout, void* workspace,
+                                     size_t workspace_bytes, void* dq, void* dk, void* dv, float* dbeta,
+                                     float* dalpha, void* dgate, float* drms_w, float* dconv_k_w,
+                                     float* dconv_v_w, float* dtext_state, void* stream, void* const* events,
+                                     int n_events) {
+  if (!events) return VDN_ERR_INVALID_ARG;
+  return backward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                         radius, dout, workspace, workspace_bytes, dq, dk, dv, dbeta, dalpha, dgate, drms_w,
+                         dconv_k_w, dconv_v_w, dtext_state, stream, events, n_events);
 }
 
 vdn_status vdn_branch_forward(const vdn_shape* shape, const void* q, const void* k, const void* v,
