@@ -17,6 +17,8 @@
 //   k_bwd_finish   reductions over CTAs, heads and batch; d alpha summed
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -713,8 +715,15 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   const vdn_shape& sh = a.sh;
   const long long BH = (long long)sh.B * sh.H, NF = BH * sh.F;
   const int K = (a.conv_k_w || a.conv_v_w) ? sh.conv_width : 1;
+  // bf16 at d = 128: the two per-token contractions on the tensor cores
+  constexpr bool kTc = D == 128 && std::is_same<T, __nv_bfloat16>::value;
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.fwd);   // the forward's status word
   // step 5 reversed
-  {
+  if (kTc) {
+    if ((e = launch_bwd_readout_tc(a, g.dout, at(p.W), at(p.dW), at(p.rms_part), g.dq, g.dgate, status)) !=
+        cudaSuccess)
+      return e;
+  } else {
     const size_t smem = sizeof(ReadoutSmem<D>);
     e = cudaFuncSetAttribute(k_bwd_readout<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -733,7 +742,10 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
       at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
   if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed
-  {
+  if (kTc) {
+    if ((e = launch_bwd_stats_tc(a, K, at(p.dA2), at(p.dB2), at(p.dkc), at(p.dvc), g.dbeta, status)) != cudaSuccess)
+      return e;
+  } else {
     const size_t smem = sizeof(StatsSmem<D>);
     e = cudaFuncSetAttribute(k_bwd_stats<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -96,6 +96,11 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule);
 // not NULL, events[2 .. kBwdKernels + 1] are recorded after each of them (events[0] and events[1] bracket
 // the forward recompute)
 constexpr int kBwdKernels = 6;
+// tensor-core versions of the read-out and statistics reversals (bf16, d = 128; tc_backward.cu)
+cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
+                                  void* dq, void* dgate, uint32_t* status);
+cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, float* dkc, float* dvc,
+                                float* dbeta, uint32_t* status);
 cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events);
 
 // standalone step 1 (dtype in, dtype out)

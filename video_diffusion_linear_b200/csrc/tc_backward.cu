@@ -1,0 +1,568 @@
+// Tensor-core kernels of the backward pass (bf16 inputs, d = 128): the two
+// per-token contractions of the branch's gradients, each over one (batch, head,
+// frame) in tiles of 128 tokens, one token per thread (= its TMEM lane).
+//
+//   k_bwd_readout_tc  (Step 5 reversed)  O = Q' W_t^T      (A = Q' K-major, B = W_t K-major)
+//                                        dQ' = DO W_t       (A = DO K-major, B = W_t read MN-major)
+//                                        dW_t += DO^T Q'    (A = DO MN-major, B = Q' MN-major)
+//   k_bwd_stats_tc    (Step 2 reversed)  U = K' (dA + dA^T), Z = K' dB^T   (B images K-major)
+//                                        V' dB                          (dB image read MN-major)
+//
+// Operands are bf16 images in the 128-byte-swizzled layout of image.cuh written by
+// the threads (q', do, k', v' per tile; W_t, dA + dA^T, dB once per frame);
+// accumulators fp32 in TMEM.  The elementwise parts (RMSNorm and gate reversed,
+// L2 norm and SiLU reversed, the conv recomputed from the raw tokens) run in the
+// epilogues in fp32, as in the SIMT kernels of backward.cu.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "image.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace vdn {
+namespace {
+
+constexpr int kBT = 128;                                                   // threads = tokens per tile
+constexpr uint32_t kIdKK = tc::idesc_bf16_f32(128, 128, false, false);    // A, B K-major
+constexpr uint32_t kIdKM = tc::idesc_bf16_f32(128, 128, false, true);     // A K-major, B MN-major
+constexpr uint32_t kIdMM = tc::idesc_bf16_f32(128, 128, true, true);      // A, B MN-major
+
+__device__ __forceinline__ void store_chunk_bf16(uint8_t* img, int n, int k, const float* v) {
+  *reinterpret_cast<uint4*>(img + img_offset(0, n, k)) =
+      make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// D (+)= A B over K = 128 for 128 x 128 bf16 operand tiles in the image layout.
+// K-major tile: rows are M (or N), 128-byte rows of K; its K step of 16 is +32 B within a
+// 64-element half, halves 16 KB apart.  MN-major: rows are K, 16 rows (2 KB) per K step.
+__device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    tc::umma_bf16(d, tc::smem_desc(a + off, 16, 1024), tc::smem_desc(b + off, 16, 1024), kIdKK,
+                  (acc || kk > 0) ? 1u : 0u);
+  }
+}
+__device__ __forceinline__ void mma_km(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    tc::umma_bf16(d, tc::smem_desc(a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                  tc::smem_desc(b + kk * 2048, 16384, 1024), kIdKM, (acc || kk > 0) ? 1u : 0u);
+}
+__device__ __forceinline__ void mma_mm(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    tc::umma_bf16(d, tc::smem_desc(a + kk * 2048, 16384, 1024), tc::smem_desc(b + kk * 2048, 16384, 1024), kIdMM,
+                  (acc || kk > 0) ? 1u : 0u);
+}
+
+// lane l receives the sum over the warp's lanes of v[l] (v[] is consumed)
+__device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = bf16lo(w[e]);
+    v[2 * e + 1] = bf16hi(w[e]);
+  }
+}
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ float silu_grad_f(float x, float g) {
+  const float s = 1.f / (1.f + expf(-x));
+  return g * s * (1.f + x * (1.f - s));
+}
+
+struct ReadoutTcSmem {
+  uint8_t w[32768];     // W_t image (rows i, K = j)
+  uint8_t qf[32768];    // Q' tile (rows tokens, K = j)
+  uint8_t dov[32768];   // DO tile (rows tokens, K = i)
+  float rms[4][128];
+  uint64_t bar;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// ---------------------------------------------------------------- Step 5 reversed
+__global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ gate,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        const float* __restrict__ rms_w,
+                                                        const float* __restrict__ Wall, float* __restrict__ dWall,
+                                                        float* __restrict__ rms_part, __nv_bfloat16* __restrict__ dq,
+                                                        __nv_bfloat16* __restrict__ dgate, int H, int F, int S,
+                                                        uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  ReadoutTcSmem& sm =
+      *reinterpret_cast<ReadoutTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const long long fi = blockIdx.x;
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long N = (long long)F * S;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort;
+  if (tid == 0) {
+    tc::mbar_init(&sm.bar, 1);
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&sm.tmem_base, 256);
+    tc::tmem_relinquish();
+  }
+  // W_t image: thread n writes row n
+  {
+    const float* wr = Wall + fi * 16384 + tid * 128;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      const float4 a = *reinterpret_cast<const float4*>(wr + 8 * c);
+      const float4 bq = *reinterpret_cast<const float4*>(wr + 8 * c + 4);
+      const float v[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+      store_chunk_bf16(sm.w, tid, 8 * c, v);
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;        // O / dQ' at columns 0..127, dW at 128..255
+  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t aw = tc::smem_u32(sm.w), aq = tc::smem_u32(sm.qf), ad = tc::smem_u32(sm.dov);
+  float racc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t ph = 0;
+  bool ok = true;
+  int tile = 0;
+  for (int s0 = 0; s0 < S && ok; s0 += kBT, ++tile) {
+    const int s = s0 + tid;
+    const bool valid = s < S;
+    const long long row = ((b * N + (long long)f * S + (valid ? s : 0)) * H + h) * 128;
+    // q' = l2n(silu(q)) into the Q' tile
+    float ss = 0.f;
+    if (valid)
+      for (int c = 0; c < 16; ++c) {
+        float v[8];
+        load8_bf16(q + row + 8 * c, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = silu_precise(v[e]);
+          ss = fmaf(x, x, ss);
+        }
+      }
+    const float inv = rsqrtf(ss + kL2Eps);
+    for (int c = 0; c < 16; ++c) {
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (valid) {
+        load8_bf16(q + row + 8 * c, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = silu_precise(v[e]) * inv;
+      }
+      store_chunk_bf16(sm.qf, tid, 8 * c, v);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (tid == 0) {
+      mma_kk(tmem, aq, aw, false);             // O = Q' W_t^T
+      tc::umma_commit(&sm.bar);
+    }
+    if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
+    ph ^= 1;
+    tc::tc_fence_after();
+    // this token's row of O, 32 columns at a time (re-read from TMEM for each pass)
+    auto ld_row = [&](int p, uint32_t (&r)[32]) {
+      tc::tmem_ld32(tmem + 32 * p + lane_off, r);
+      tc::tmem_ld_wait();
+    };
+    // RMSNorm and gate reversed
+    float so2 = 0.f;
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t o[32];
+      ld_row(p, o);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) so2 = fmaf(__uint_as_float(o[c]), __uint_as_float(o[c]), so2);
+    }
+    const float rr = rsqrtf(so2 * (1.f / 128.f) + kRmsEps);
+    float so = 0.f;
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t o[32];
+      ld_row(p, o);
+      float red[32];
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int c0 = 32 * p + 8 * c8;
+        float go[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, g[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (valid) {
+          load8_bf16(dout + row + c0, go);
+          load8_bf16(gate + row + c0, g);
+        }
+        float dg[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float rw = __ldg(rms_w + c0 + e);
+          const float ov = __uint_as_float(o[8 * c8 + e]);
+          const float oh = ov * rr;
+          const float dy = go[e] * g[e];
+          dg[e] = go[e] * oh * rw;
+          red[8 * c8 + e] = dy * oh;
+          so = fmaf(dy * rw, ov, so);
+        }
+        if (valid) store8_bf16(dgate + row + c0, dg);
+      }
+      racc[p] += transpose_sum32(red, lane);
+    }
+    const float k3 = rr * rr * rr * so * (1.f / 128.f);
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t o[32];
+      ld_row(p, o);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int c0 = 32 * p + 8 * c8;
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (valid) {
+          float go[8], g[8];
+          load8_bf16(dout + row + c0, go);
+          load8_bf16(gate + row + c0, g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float rw = __ldg(rms_w + c0 + e);
+            v[e] = rr * go[e] * g[e] * rw - k3 * __uint_as_float(o[8 * c8 + e]);
+          }
+        }
+        store_chunk_bf16(sm.dov, tid, c0, v);
+      }
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (tid == 0) {
+      mma_km(tmem, ad, aw, false);               // dQ' = DO W_t
+      mma_mm(tmem + 128, ad, aq, tile > 0);      // dW_t += DO^T Q'
+      tc::umma_commit(&sm.bar);
+    }
+    if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
+    ph ^= 1;
+    tc::tc_fence_after();
+    // q' = l2n(silu(q)) reversed: dx = (g - x (x.g) / n^2) / n with x = silu(q), g = dq'
+    float sx = 0.f, xg = 0.f;
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t o[32];
+      ld_row(p, o);
+      if (!valid) continue;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float v[8];
+        load8_bf16(q + row + 32 * p + 8 * c8, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = silu_precise(v[e]);
+          sx = fmaf(x, x, sx);
+          xg = fmaf(x, __uint_as_float(o[8 * c8 + e]), xg);
+        }
+      }
+    }
+    const float in = rsqrtf(sx + kL2Eps);
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t o[32];
+      ld_row(p, o);
+      if (!valid) continue;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float v[8], r8[8];
+        load8_bf16(q + row + 32 * p + 8 * c8, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = silu_precise(v[e]);
+          r8[e] = silu_grad_f(v[e], (__uint_as_float(o[8 * c8 + e]) - x * xg * in * in) * in);
+        }
+        store8_bf16(dq + row + 32 * p + 8 * c8, r8);
+      }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+  }
+  if (ok) {
+    float* dW = dWall + fi * 16384 + tid * 128;   // row i = tid
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      uint32_t r[32];
+      tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dW + 32 * p + e) =
+            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                        __uint_as_float(r[e + 3]));
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) sm.rms[warp][32 * p + lane] = racc[p];
+  tc::tc_fence_before();
+  __syncthreads();
+  rms_part[fi * 128 + tid] = sm.rms[0][tid] + sm.rms[1][tid] + sm.rms[2][tid] + sm.rms[3][tid];
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------- Step 2 reversed
+struct StatsTcSmem {
+  uint8_t da[32768];    // (dA + dA^T) image (rows i, K = j)
+  uint8_t db[32768];    // dB image (rows i, K = j)
+  uint8_t kf[32768];    // K' tile
+  uint8_t vf[32768];    // V' tile
+  uint64_t bar;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// the short conv of one channel chunk (8 channels c0..c0+7) of token s, in-frame taps
+__device__ __forceinline__ void conv8(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, int K,
+                                      long long frame_row0, int s, int S, int H, int c0, long long hoff, int h,
+                                      float* out) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out[e] = 0.f;
+  if (w == nullptr) {
+    load8_bf16(x + (frame_row0 + s) * H * 128 + hoff + c0, out);
+    return;
+  }
+  const int pad = (K - 1) / 2;
+  for (int j = 0; j < K; ++j) {
+    const int sj = s + j - pad;
+    if (sj < 0 || sj >= S) continue;
+    float v[8];
+    load8_bf16(x + (frame_row0 + sj) * H * 128 + hoff + c0, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = fmaf(__ldg(w + ((long long)h * 128 + c0 + e) * K + j), v[e], out[e]);
+  }
+}
+
+__global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __restrict__ k,
+                                                      const __nv_bfloat16* __restrict__ v,
+                                                      const float* __restrict__ beta, const float* __restrict__ wk,
+                                                      const float* __restrict__ wv, int K,
+                                                      const float* __restrict__ dA2, const float* __restrict__ dB2,
+                                                      float* __restrict__ dkc, float* __restrict__ dvc,
+                                                      float* __restrict__ dbeta, int H, int F, int S,
+                                                      uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  StatsTcSmem& sm = *reinterpret_cast<StatsTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const long long fi = blockIdx.x;
+  const long long NFt = gridDim.x;
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long N = (long long)F * S;
+  const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0 (times H * 128 below)
+  const long long hoff = (long long)h * 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort;
+  if (tid == 0) {
+    tc::mbar_init(&sm.bar, 1);
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&sm.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  // images of dA + dA^T and dB (both scans' parts summed); thread i writes row i
+  {
+    const float* a0 = dA2 + fi * 16384;
+    const float* a1 = dA2 + (NFt + fi) * 16384;
+    const float* b0 = dB2 + fi * 16384;
+    const float* b1 = dB2 + (NFt + fi) * 16384;
+    const int i = tid;
+    for (int c = 0; c < 16; ++c) {
+      float va[8], vb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = 8 * c + e;
+        va[e] = a0[i * 128 + j] + a1[i * 128 + j] + a0[j * 128 + i] + a1[j * 128 + i];
+        vb[e] = b0[i * 128 + j] + b1[i * 128 + j];
+      }
+      store_chunk_bf16(sm.da, i, 8 * c, va);
+      store_chunk_bf16(sm.db, i, 8 * c, vb);
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;        // U at 0, Z at 128, V' dB at 256
+  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t a_da = tc::smem_u32(sm.da), a_db = tc::smem_u32(sm.db), a_k = tc::smem_u32(sm.kf),
+                 a_v = tc::smem_u32(sm.vf);
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int s0 = 0; s0 < S && ok; s0 += kBT) {
+    const int s = s0 + tid;
+    const bool valid = s < S;
+    // k' = l2n(silu(conv k)), v' = silu(conv v) into the K', V' tiles
+    float ss = 0.f;
+    if (valid)
+      for (int c = 0; c < 16; ++c) {
+        float kc[8];
+        conv8(k, wk, K, frame_row0, s, S, H, 8 * c, hoff, h, kc);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = silu_precise(kc[e]);
+          ss = fmaf(x, x, ss);
+        }
+      }
+    const float inv = rsqrtf(ss + kL2Eps);
+    for (int c = 0; c < 16; ++c) {
+      float kv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (valid) {
+        conv8(k, wk, K, frame_row0, s, S, H, 8 * c, hoff, h, kv);
+        conv8(v, wv, K, frame_row0, s, S, H, 8 * c, hoff, h, vv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          kv[e] = silu_precise(kv[e]) * inv;
+          vv[e] = silu_precise(vv[e]);
+        }
+      }
+      store_chunk_bf16(sm.kf, tid, 8 * c, kv);
+      store_chunk_bf16(sm.vf, tid, 8 * c, vv);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (tid == 0) {
+      mma_kk(tmem, a_k, a_da, false);            // U = K' (dA + dA^T)^T = K' (dA + dA^T)
+      mma_kk(tmem + 128, a_k, a_db, false);      // Z: z_i = sum_j dB[i][j] k'_j
+      mma_km(tmem + 256, a_v, a_db, false);      // w_i = sum_j dB[j][i] v'_j
+      tc::umma_commit(&sm.bar);
+    }
+    if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
+    ph ^= 1;
+    tc::tc_fence_after();
+    // the TMEM loads are warp-collective: every thread loads, only valid tokens compute
+    const long long tok = frame_row0 * H + (long long)(valid ? s : 0) * H + h;
+    const float bt = valid ? beta[tok] : 0.f;
+    // pass 1: d beta and x . dk' (x = silu(conv k)), chunk by chunk of 32 channels
+    float dbt = 0.f, xg = 0.f;
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t u[32], z[32], w[32];
+      tc::tmem_ld32(tmem + 32 * p + lane_off, u);
+      tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, z);
+      tc::tmem_ld32(tmem + 256 + 32 * p + lane_off, w);
+      tc::tmem_ld_wait();
+      if (!valid) continue;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float kc[8], vc[8];
+        conv8(k, wk, K, frame_row0, s, S, H, 32 * p + 8 * c8, hoff, h, kc);
+        conv8(v, wv, K, frame_row0, s, S, H, 32 * p + 8 * c8, hoff, h, vc);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int m = 8 * c8 + e;
+          const float x = silu_precise(kc[e]);
+          const float uu = __uint_as_float(u[m]), zz = __uint_as_float(z[m]), ww = __uint_as_float(w[m]);
+          // d beta = 1/2 k'^T (dA + dA^T) k' + v'^T dB k'
+          dbt = fmaf(0.5f * x * inv, uu, dbt);
+          dbt = fmaf(silu_precise(vc[e]), zz, dbt);
+          xg = fmaf(x, bt * (uu + ww), xg);
+        }
+      }
+    }
+    if (valid) dbeta[tok] = dbt;
+    // pass 2: dkc = silu'(kc) (dk' - x (x . dk') / n^2) / n, dvc = silu'(vc) beta z
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+      uint32_t u[32], z[32], w[32];
+      tc::tmem_ld32(tmem + 32 * p + lane_off, u);
+      tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, z);
+      tc::tmem_ld32(tmem + 256 + 32 * p + lane_off, w);
+      tc::tmem_ld_wait();
+      if (!valid) continue;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int c0 = 32 * p + 8 * c8;
+        float kc[8], vc[8], gk[8], gv[8];
+        conv8(k, wk, K, frame_row0, s, S, H, c0, hoff, h, kc);
+        conv8(v, wv, K, frame_row0, s, S, H, c0, hoff, h, vc);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int m = 8 * c8 + e;
+          const float x = silu_precise(kc[e]);
+          const float dk = bt * (__uint_as_float(u[m]) + __uint_as_float(w[m]));
+          gk[e] = silu_grad_f(kc[e], (dk - x * xg * inv * inv) * inv);
+          gv[e] = silu_grad_f(vc[e], bt * __uint_as_float(z[m]));
+        }
+        float* pk = dkc + tok * 128 + c0;
+        float* pv = dvc + tok * 128 + c0;
+        *reinterpret_cast<float4*>(pk) = make_float4(gk[0], gk[1], gk[2], gk[3]);
+        *reinterpret_cast<float4*>(pk + 4) = make_float4(gk[4], gk[5], gk[6], gk[7]);
+        *reinterpret_cast<float4*>(pv) = make_float4(gv[0], gv[1], gv[2], gv[3]);
+        *reinterpret_cast<float4*>(pv + 4) = make_float4(gv[4], gv[5], gv[6], gv[7]);
+      }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
+                                  void* dq, void* dgate, uint32_t* status) {
+  const size_t smem = sizeof(ReadoutTcSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_bwd_readout_tc<<<(unsigned)a.NF(), kBT, smem, a.stream>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gate),
+      static_cast<const __nv_bfloat16*>(dout), a.rms_w, W, dW, rms_part, static_cast<__nv_bfloat16*>(dq),
+      static_cast<__nv_bfloat16*>(dgate), a.sh.H, a.sh.F, a.sh.S, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, float* dkc, float* dvc,
+                                float* dbeta, uint32_t* status) {
+  const size_t smem = sizeof(StatsTcSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_bwd_stats_tc<<<(unsigned)a.NF(), kBT, smem, a.stream>>>(
+      static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
+      a.conv_v_w, K, dA2, dB2, dkc, dvc, dbeta, a.sh.H, a.sh.F, a.sh.S, status);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn
