@@ -85,9 +85,14 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) =
       make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
+// sigma(x) = 1/2 + 1/2 tanh(x/2) by the hardware tanh (one MUFU op, relative error about 2^-11,
+// below the bf16 rounding of every gradient these kernels write), as the forward's tensor-core
+// kernels evaluate SiLU; silu(x) = x sigma(x), d silu = sigma (1 + x (1 - sigma)) dx
+__device__ __forceinline__ float sigm_fast(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+__device__ __forceinline__ float silu_f(float x) { return x * sigm_fast(x); }
 __device__ __forceinline__ float silu_grad_f(float x, float g) {
-  const float s = 1.f / (1.f + expf(-x));
-  return g * s * (1.f + x * (1.f - s));
+  const float s = sigm_fast(x);
+  return g * s * fmaf(x, 1.f - s, 1.f);
 }
 
 struct ReadoutTcSmem {
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         load8_bf16(q + row + 8 * c, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x = silu_precise(v[e]);
+          const float x = silu_f(v[e]);
           ss = fmaf(x, x, ss);
         }
       }
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
       if (valid) {
         load8_bf16(q + row + 8 * c, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = silu_precise(v[e]) * inv;
+        for (int e = 0; e < 8; ++e) v[e] = silu_f(v[e]) * inv;
       }
       store_chunk_bf16(sm.qf, tid, 8 * c, v);
     }
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         load8_bf16(q + row + 32 * p + 8 * c8, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x = silu_precise(v[e]);
+          const float x = silu_f(v[e]);
           sx = fmaf(x, x, sx);
           xg = fmaf(x, __uint_as_float(o[8 * c8 + e]), xg);
         }
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         load8_bf16(q + row + 32 * p + 8 * c8, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x = silu_precise(v[e]);
+          const float x = silu_f(v[e]);
           r8[e] = silu_grad_f(v[e], (__uint_as_float(o[8 * c8 + e]) - x * xg * in * in) * in);
         }
         store8_bf16(dq + row + 32 * p + 8 * c8, r8);
@@ -333,32 +338,36 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
 }
 
 // ---------------------------------------------------------------- Step 2 reversed
+constexpr int kRawStride = 272;     // bytes per staged token row (256 + 16: conflict-free 16-byte reads)
+constexpr int kRawRows = kBT + 2;    // the tile's tokens and one halo token on each side
 struct StatsTcSmem {
   uint8_t da[32768];    // (dA + dA^T) image (rows i, K = j)
   uint8_t db[32768];    // dB image (rows i, K = j)
   uint8_t kf[32768];    // K' tile
   uint8_t vf[32768];    // V' tile
+  uint8_t kraw[kRawRows * kRawStride];   // raw k rows s0 - 1 .. s0 + 128 (bf16; zero outside the frame)
+  uint8_t vraw[kRawRows * kRawStride];
   uint64_t bar;
   uint32_t tmem_base;
   int abort;
 };
 
-// the short conv of one channel chunk (8 channels c0..c0+7) of token s, in-frame taps
-__device__ __forceinline__ void conv8(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, int K,
-                                      long long frame_row0, int s, int S, int H, int c0, long long hoff, int h,
-                                      float* out) {
-#pragma unroll
-  for (int e = 0; e < 8; ++e) out[e] = 0.f;
+// the short conv of one channel chunk (8 channels c0..c0+7) of the tile's token t (frame index s),
+// in-frame taps, from the staged rows (row t + 1 holds token t)
+__device__ __forceinline__ void conv8(const uint8_t* raw, const float* __restrict__ w, int K, int t, int s, int S,
+                                      int c0, int h, float* out) {
   if (w == nullptr) {
-    load8_bf16(x + (frame_row0 + s) * H * 128 + hoff + c0, out);
+    load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1) * kRawStride + 2 * c0), out);
     return;
   }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out[e] = 0.f;
   const int pad = (K - 1) / 2;
   for (int j = 0; j < K; ++j) {
     const int sj = s + j - pad;
     if (sj < 0 || sj >= S) continue;
     float v[8];
-    load8_bf16(x + (frame_row0 + sj) * H * 128 + hoff + c0, v);
+    load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1 + j - pad) * kRawStride + 2 * c0), v);
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = fmaf(__ldg(w + ((long long)h * 128 + c0 + e) * K + j), v[e], out[e]);
   }
@@ -382,8 +391,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
   const long long b = bh / H;
   const long long N = (long long)F * S;
   const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0 (times H * 128 below)
-  const long long hoff = (long long)h * 128;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {
     tc::mbar_init(&sm.bar, 1);
@@ -426,40 +434,50 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
   for (int s0 = 0; s0 < S && ok; s0 += kBT) {
     const int s = s0 + tid;
     const bool valid = s < S;
-    // k' = l2n(silu(conv k)), v' = silu(conv v) into the K', V' tiles
-    float ss = 0.f;
-    if (valid)
-      for (int c = 0; c < 16; ++c) {
-        float kc[8];
-        conv8(k, wk, K, frame_row0, s, S, H, 8 * c, hoff, h, kc);
+    // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame)
+    for (int r = tid; r < kRawRows; r += kBT) {
+      const int sr = s0 - 1 + r;
+      const bool in = sr >= 0 && sr < S;
+      const long long base = ((frame_row0 + (in ? sr : 0)) * H + h) * 128;
+      uint4 kb[16], vb[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float x = silu_precise(kc[e]);
-          ss = fmaf(x, x, ss);
-        }
+      for (int c = 0; c < 16; ++c) {
+        kb[c] = in ? *reinterpret_cast<const uint4*>(k + base + 8 * c) : make_uint4(0, 0, 0, 0);
+        vb[c] = in ? *reinterpret_cast<const uint4*>(v + base + 8 * c) : make_uint4(0, 0, 0, 0);
       }
-    const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        *reinterpret_cast<uint4*>(sm.kraw + r * kRawStride + 16 * c) = kb[c];
+        *reinterpret_cast<uint4*>(sm.vraw + r * kRawStride + 16 * c) = vb[c];
+      }
+    }
+    __syncthreads();
+    // x = silu(conv k) (k' = x / |x|: the 1/|x| is applied to U and Z in the epilogue) and
+    // v' = silu(conv v) into the K', V' tiles
+    float ss = 0.f;
     for (int c = 0; c < 16; ++c) {
       float kv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
-        conv8(k, wk, K, frame_row0, s, S, H, 8 * c, hoff, h, kv);
-        conv8(v, wv, K, frame_row0, s, S, H, 8 * c, hoff, h, vv);
+        conv8(sm.kraw, wk, K, tid, s, S, 8 * c, h, kv);
+        conv8(sm.vraw, wv, K, tid, s, S, 8 * c, h, vv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          kv[e] = silu_precise(kv[e]) * inv;
-          vv[e] = silu_precise(vv[e]);
+          kv[e] = silu_f(kv[e]);
+          ss = fmaf(kv[e], kv[e], ss);
+          vv[e] = silu_f(vv[e]);
         }
       }
       store_chunk_bf16(sm.kf, tid, 8 * c, kv);
       store_chunk_bf16(sm.vf, tid, 8 * c, vv);
     }
+    const float inv = rsqrtf(ss + kL2Eps);
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     if (tid == 0) {
-      mma_kk(tmem, a_k, a_da, false);            // U = K' (dA + dA^T)^T = K' (dA + dA^T)
-      mma_kk(tmem + 128, a_k, a_db, false);      // Z: z_i = sum_j dB[i][j] k'_j
+      mma_kk(tmem, a_k, a_da, false);            // U |x|: X (dA + dA^T)
+      mma_kk(tmem + 128, a_k, a_db, false);      // Z |x|: z_i |x| = sum_j dB[i][j] x_j
       mma_km(tmem + 256, a_v, a_db, false);      // w_i = sum_j dB[j][i] v'_j
       tc::umma_commit(&sm.bar);
     }
@@ -469,7 +487,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
     // the TMEM loads are warp-collective: every thread loads, only valid tokens compute
     const long long tok = frame_row0 * H + (long long)(valid ? s : 0) * H + h;
     const float bt = valid ? beta[tok] : 0.f;
-    // pass 1: d beta and x . dk' (x = silu(conv k)), chunk by chunk of 32 channels
+    // pass 1: d beta and x . dk' from the tiles' x and v' (bf16) and U, Z, V'dB (u = inv U, z = inv Z)
     float dbt = 0.f, xg = 0.f;
 #pragma unroll 1
     for (int p = 0; p < 4; ++p) {
@@ -481,18 +499,18 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
       if (!valid) continue;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
-        float kc[8], vc[8];
-        conv8(k, wk, K, frame_row0, s, S, H, 32 * p + 8 * c8, hoff, h, kc);
-        conv8(v, wv, K, frame_row0, s, S, H, 32 * p + 8 * c8, hoff, h, vc);
+        float xk[8], xv[8];
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.kf + img_offset(0, tid, 32 * p + 8 * c8)), xk);
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.vf + img_offset(0, tid, 32 * p + 8 * c8)), xv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int m = 8 * c8 + e;
-          const float x = silu_precise(kc[e]);
-          const float uu = __uint_as_float(u[m]), zz = __uint_as_float(z[m]), ww = __uint_as_float(w[m]);
+          const float uu = inv * __uint_as_float(u[m]), zz = inv * __uint_as_float(z[m]);
+          const float ww = __uint_as_float(w[m]);
           // d beta = 1/2 k'^T (dA + dA^T) k' + v'^T dB k'
-          dbt = fmaf(0.5f * x * inv, uu, dbt);
-          dbt = fmaf(silu_precise(vc[e]), zz, dbt);
-          xg = fmaf(x, bt * (uu + ww), xg);
+          dbt = fmaf(0.5f * xk[e] * inv, uu, dbt);
+          dbt = fmaf(xv[e], zz, dbt);
+          xg = fmaf(xk[e], bt * (uu + ww), xg);
         }
       }
     }
@@ -510,15 +528,15 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
       for (int c8 = 0; c8 < 4; ++c8) {
         const int c0 = 32 * p + 8 * c8;
         float kc[8], vc[8], gk[8], gv[8];
-        conv8(k, wk, K, frame_row0, s, S, H, c0, hoff, h, kc);
-        conv8(v, wv, K, frame_row0, s, S, H, c0, hoff, h, vc);
+        conv8(sm.kraw, wk, K, tid, s, S, c0, h, kc);
+        conv8(sm.vraw, wv, K, tid, s, S, c0, h, vc);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int m = 8 * c8 + e;
-          const float x = silu_precise(kc[e]);
-          const float dk = bt * (__uint_as_float(u[m]) + __uint_as_float(w[m]));
+          const float x = silu_f(kc[e]);
+          const float dk = bt * (inv * __uint_as_float(u[m]) + __uint_as_float(w[m]));
           gk[e] = silu_grad_f(kc[e], (dk - x * xg * inv * inv) * inv);
-          gv[e] = silu_grad_f(vc[e], bt * __uint_as_float(z[m]));
+          gv[e] = silu_grad_f(vc[e], bt * inv * __uint_as_float(z[m]));
         }
         float* pk = dkc + tok * 128 + c0;
         float* pv = dvc + tok * 128 + c0;
