@@ -160,34 +160,28 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     const int s = s0 + tid;
     const bool valid = s < S;
     const long long row = ((b * N + (long long)f * S + (valid ? s : 0)) * H + h) * 128;
-    // q' = l2n(silu(q)) into the Q' tile
+    // x = silu(q) into the Q' tile (q' = x / |x|: the 1/|x| is folded into O, DO and dQ' below)
     float ss = 0.f;
-    if (valid)
-      for (int c = 0; c < 16; ++c) {
-        float v[8];
-        load8_bf16(q + row + 8 * c, v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float x = silu_f(v[e]);
-          ss = fmaf(x, x, ss);
-        }
-      }
-    const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll 4
     for (int c = 0; c < 16; ++c) {
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
         load8_bf16(q + row + 8 * c, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = silu_f(v[e]) * inv;
+        for (int e = 0; e < 8; ++e) {
+          v[e] = silu_f(v[e]);
+          ss = fmaf(v[e], v[e], ss);
+        }
       }
       store_chunk_bf16(sm.qf, tid, 8 * c, v);
     }
+    const float inv = rsqrtf(ss + kL2Eps), nrm = (ss + kL2Eps) * inv;   // 1/|x|, |x|
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     if (tid == 0) {
-      mma_kk(tmem, aq, aw, false);             // O = Q' W_t^T
+      mma_kk(tmem, aq, aw, false);             // O |x| = X W_t^T
       tc::umma_commit(&sm.bar);
     }
     if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
@@ -207,6 +201,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
 #pragma unroll
       for (int c = 0; c < 32; ++c) so2 = fmaf(__uint_as_float(o[c]), __uint_as_float(o[c]), so2);
     }
+    so2 *= inv * inv;
     const float rr = rsqrtf(so2 * (1.f / 128.f) + kRmsEps);
     float so = 0.f;
 #pragma unroll 1
@@ -222,11 +217,13 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
           load8_bf16(dout + row + c0, go);
           load8_bf16(gate + row + c0, g);
         }
-        float dg[8];
+        float dg[8], rw8[8];
+        *reinterpret_cast<float4*>(rw8) = __ldg(reinterpret_cast<const float4*>(rms_w + c0));
+        *reinterpret_cast<float4*>(rw8 + 4) = __ldg(reinterpret_cast<const float4*>(rms_w + c0 + 4));
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float rw = __ldg(rms_w + c0 + e);
-          const float ov = __uint_as_float(o[8 * c8 + e]);
+          const float rw = rw8[e];
+          const float ov = inv * __uint_as_float(o[8 * c8 + e]);
           const float oh = ov * rr;
           const float dy = go[e] * g[e];
           dg[e] = go[e] * oh * rw;
@@ -247,14 +244,15 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         const int c0 = 32 * p + 8 * c8;
         float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (valid) {
-          float go[8], g[8];
+          float go[8], g[8], rw8[8];
           load8_bf16(dout + row + c0, go);
           load8_bf16(gate + row + c0, g);
+          *reinterpret_cast<float4*>(rw8) = __ldg(reinterpret_cast<const float4*>(rms_w + c0));
+          *reinterpret_cast<float4*>(rw8 + 4) = __ldg(reinterpret_cast<const float4*>(rms_w + c0 + 4));
+          // the tile holds do / |x| (so that DO^T X sums do q'^T)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float rw = __ldg(rms_w + c0 + e);
-            v[e] = rr * go[e] * g[e] * rw - k3 * __uint_as_float(o[8 * c8 + e]);
-          }
+          for (int e = 0; e < 8; ++e)
+            v[e] = inv * (rr * go[e] * g[e] * rw8[e] - k3 * inv * __uint_as_float(o[8 * c8 + e]));
         }
         store_chunk_bf16(sm.dov, tid, c0, v);
       }
@@ -264,15 +262,16 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     __syncthreads();
     tc::tc_fence_after();
     if (tid == 0) {
-      mma_km(tmem, ad, aw, false);               // dQ' = DO W_t
-      mma_mm(tmem + 128, ad, aq, tile > 0);      // dW_t += DO^T Q'
+      mma_km(tmem, ad, aw, false);               // dQ' / |x| = (DO / |x|) W_t
+      mma_mm(tmem + 128, ad, aq, tile > 0);      // dW_t += (DO / |x|)^T X = DO^T Q'
       tc::umma_commit(&sm.bar);
     }
     if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
     ph ^= 1;
     tc::tc_fence_after();
-    // q' = l2n(silu(q)) reversed: dx = (g - x (x.g) / n^2) / n with x = silu(q), g = dq'
-    float sx = 0.f, xg = 0.f;
+    // q' = l2n(silu(q)) reversed: dx = (g - x (x.g) / |x|^2) / |x| with x = silu(q), g = dq';
+    // x.g from the tile's x (bf16), then dq = silu'(q) dx
+    float xg = 0.f;
 #pragma unroll 1
     for (int p = 0; p < 4; ++p) {
       uint32_t o[32];
@@ -280,17 +279,12 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
       if (!valid) continue;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
-        float v[8];
-        load8_bf16(q + row + 32 * p + 8 * c8, v);
+        float x[8];
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.qf + img_offset(0, tid, 32 * p + 8 * c8)), x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float x = silu_f(v[e]);
-          sx = fmaf(x, x, sx);
-          xg = fmaf(x, __uint_as_float(o[8 * c8 + e]), xg);
-        }
+        for (int e = 0; e < 8; ++e) xg = fmaf(x[e], nrm * __uint_as_float(o[8 * c8 + e]), xg);
       }
     }
-    const float in = rsqrtf(sx + kL2Eps);
 #pragma unroll 1
     for (int p = 0; p < 4; ++p) {
       uint32_t o[32];
@@ -302,8 +296,10 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         load8_bf16(q + row + 32 * p + 8 * c8, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x = silu_f(v[e]);
-          r8[e] = silu_grad_f(v[e], (__uint_as_float(o[8 * c8 + e]) - x * xg * in * in) * in);
+          const float sg = sigm_fast(v[e]);
+          const float x = v[e] * sg;
+          const float dx = (nrm * __uint_as_float(o[8 * c8 + e]) - x * xg * inv * inv) * inv;
+          r8[e] = dx * sg * fmaf(v[e], 1.f - sg, 1.f);
         }
         store8_bf16(dq + row + 32 * p + 8 * c8, r8);
       }
@@ -347,19 +343,16 @@ struct StatsTcSmem {
   uint8_t vf[32768];    // V' tile
   uint8_t kraw[kRawRows * kRawStride];   // raw k rows s0 - 1 .. s0 + 128 (bf16; zero outside the frame)
   uint8_t vraw[kRawRows * kRawStride];
+  float taps[2][3][128];                 // [k, v][tap][channel] of this head (identity: centre tap 1)
   uint64_t bar;
   uint32_t tmem_base;
   int abort;
 };
 
 // the short conv of one channel chunk (8 channels c0..c0+7) of the tile's token t (frame index s),
-// in-frame taps, from the staged rows (row t + 1 holds token t)
-__device__ __forceinline__ void conv8(const uint8_t* raw, const float* __restrict__ w, int K, int t, int s, int S,
-                                      int c0, int h, float* out) {
-  if (w == nullptr) {
-    load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1) * kRawStride + 2 * c0), out);
-    return;
-  }
+// in-frame taps, from the staged rows (row t + 1 holds token t) and the staged taps tp[tap][channel]
+__device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128], int K, int t, int s, int S,
+                                      int c0, float* out) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = 0.f;
   const int pad = (K - 1) / 2;
@@ -368,8 +361,11 @@ __device__ __forceinline__ void conv8(const uint8_t* raw, const float* __restric
     if (sj < 0 || sj >= S) continue;
     float v[8];
     load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1 + j - pad) * kRawStride + 2 * c0), v);
+    const float4 w0 = *reinterpret_cast<const float4*>(&tp[j][c0]);
+    const float4 w1 = *reinterpret_cast<const float4*>(&tp[j][c0 + 4]);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = fmaf(__ldg(w + ((long long)h * 128 + c0 + e) * K + j), v[e], out[e]);
+    for (int e = 0; e < 8; ++e) out[e] = fmaf(wv[e], v[e], out[e]);
   }
 }
 
@@ -392,6 +388,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
   const long long N = (long long)F * S;
   const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0 (times H * 128 below)
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int Kc = wk ? K : (wv ? K : 1);      // taps of the staged convs (a missing one: identity)
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {
     tc::mbar_init(&sm.bar, 1);
@@ -419,6 +416,12 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
       }
       store_chunk_bf16(sm.da, i, 8 * c, va);
       store_chunk_bf16(sm.db, i, 8 * c, vb);
+    }
+    // taps of this head, [tensor][tap][channel]; a missing conv is the identity (one centre tap)
+    for (int j = 0; j < 3; ++j) {
+      const bool centre = j == (Kc - 1) / 2;
+      sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+      sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
     }
   }
   tc::fence_proxy_async_smem();
@@ -458,8 +461,8 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
     for (int c = 0; c < 16; ++c) {
       float kv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
-        conv8(sm.kraw, wk, K, tid, s, S, 8 * c, h, kv);
-        conv8(sm.vraw, wv, K, tid, s, S, 8 * c, h, vv);
+        conv8(sm.kraw, sm.taps[0], Kc, tid, s, S, 8 * c, kv);
+        conv8(sm.vraw, sm.taps[1], Kc, tid, s, S, 8 * c, vv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           kv[e] = silu_f(kv[e]);
@@ -528,8 +531,8 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
       for (int c8 = 0; c8 < 4; ++c8) {
         const int c0 = 32 * p + 8 * c8;
         float kc[8], vc[8], gk[8], gv[8];
-        conv8(sm.kraw, wk, K, tid, s, S, c0, h, kc);
-        conv8(sm.vraw, wv, K, tid, s, S, c0, h, vc);
+        conv8(sm.kraw, sm.taps[0], Kc, tid, s, S, c0, kc);
+        conv8(sm.vraw, sm.taps[1], Kc, tid, s, S, c0, vc);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int m = 8 * c8 + e;
