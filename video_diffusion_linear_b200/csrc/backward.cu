@@ -291,6 +291,8 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout(const T* __restrict__ q, co
 // ---------------------------------------------------------------- step 4 (gather + bridge) reversed
 // dPin[b, h][0] receives the gradient of the seed as P_{-1}, dPin[b, h][f + 1] that of P_f;
 // dQin[b, h][f] that of Q_f, dQin[b, h][F] that of the seed as Q_F.  dalpha_g [B, H, F, D].
+// Block (b·h, column block): columns are independent here, so each block owns CB columns for
+// every query frame t (its updates of the boundary slots are ordered), rows split over RG groups.
 template <int D>
 __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P, const float* __restrict__ Q,
                                                     const float* __restrict__ alpha,
@@ -298,17 +300,20 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
                                                     const float* __restrict__ dWall, float* __restrict__ dPin,
                                                     float* __restrict__ dQin, float* __restrict__ dalpha_g, int H,
                                                     int F, int chunk, int radius) {
+  constexpr int CB = D < 32 ? D : 32;      // columns per block
+  constexpr int RG = kBT / CB;             // row groups
+  constexpr int RPT = D / RG;              // rows per thread
+  __shared__ float red[2][RG][CB];
   const long long bh = blockIdx.x;
   const int h = (int)(bh % H);
   const long long b = bh / H;
-  const int j = threadIdx.x;
-  if (j >= D) return;                          // thread j owns column j
+  const int jj = threadIdx.x % CB, rg = threadIdx.x / CB;
+  const int j = blockIdx.y * CB + jj;
   const long long DD = (long long)D * D;
   float* dP = dPin + bh * (F + 1) * DD;
   float* dQ = dQin + bh * (F + 1) * DD;
   float* dal = dalpha_g + bh * F * D;
   auto alpha_at = [&](int f) { return alpha[((b * F + f) * H + h) * D + j]; };
-  auto seed_at = [&](int i) { return text_state ? 0.5f * text_state[((long long)h * D + i) * D + j] : 0.f; };
   for (int t = 0; t < F; ++t) {
     int lo, hi;
     window_bounds(t, F, chunk, radius, lo, hi);
@@ -321,26 +326,41 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
     float* dpre = dP + (long long)lo * DD;          // slot lo: P_{lo-1} (slot 0: the seed)
     float* dsuf = dQ + (long long)(hi + 1) * DD;    // slot hi + 1: Q_{hi+1} (slot F: the seed)
     float da = 0.f, db = 0.f;
-    for (int i = 0; i < D; ++i) {
-      const float g = dW[i * D + j];
-      dpre[i * D + j] += g * a;
-      dsuf[i * D + j] += g * bb;
-      da = fmaf(pre ? pre[i * D + j] : seed_at(i), g, da);
-      db = fmaf(suf ? suf[i * D + j] : seed_at(i), g, db);
+#pragma unroll 4
+    for (int r = 0; r < RPT; ++r) {
+      const int i = rg + RG * r;
+      const long long e = (long long)i * D + j;
+      const float g = dW[e];
+      dpre[e] += g * a;
+      dsuf[e] += g * bb;
+      const float sd = text_state ? 0.5f * text_state[(long long)h * DD + e] : 0.f;
+      da = fmaf(pre ? pre[e] : sd, g, da);
+      db = fmaf(suf ? suf[e] : sd, g, db);
     }
-    // d prod / d alpha_f = product of the other factors
-    for (int f = lo; f <= t; ++f) {
-      float pr = 1.f;
-      for (int g2 = lo; g2 <= t; ++g2)
-        if (g2 != f) pr *= alpha_at(g2);
-      dal[f * D + j] += da * pr;
+    red[0][rg][jj] = da;
+    red[1][rg][jj] = db;
+    __syncthreads();
+    if (rg == 0) {
+      da = db = 0.f;
+      for (int r = 0; r < RG; ++r) {
+        da += red[0][r][jj];
+        db += red[1][r][jj];
+      }
+      // d prod / d alpha_f = product of the other factors
+      for (int f = lo; f <= t; ++f) {
+        float pr = 1.f;
+        for (int g2 = lo; g2 <= t; ++g2)
+          if (g2 != f) pr *= alpha_at(g2);
+        dal[f * D + j] += da * pr;
+      }
+      for (int f = t; f <= hi; ++f) {
+        float pr = 1.f;
+        for (int g2 = t; g2 <= hi; ++g2)
+          if (g2 != f) pr *= alpha_at(g2);
+        dal[f * D + j] += db * pr;
+      }
     }
-    for (int f = t; f <= hi; ++f) {
-      float pr = 1.f;
-      for (int g2 = t; g2 <= hi; ++g2)
-        if (g2 != f) pr *= alpha_at(g2);
-      dal[f * D + j] += db * pr;
-    }
+    __syncthreads();
   }
 }
 
@@ -536,72 +556,126 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats(const T* __restrict__ k, cons
 }
 
 // ---------------------------------------------------------------- step 1 conv reversed
-// One warp per token (grid-stride within head h = blockIdx.y): dk[s] = sum_j w[j] dkc[s - j + p]
-// over in-frame indices; tap partials sum_s dkc[s] k[s + j - p] per block.
-template <int D, typename T>
+template <typename T> __device__ __forceinline__ void load8t(const T* p, float* v);
+template <> __device__ __forceinline__ void load8t<float>(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <> __device__ __forceinline__ void load8t<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = bf16lo(w[e]);
+    v[2 * e + 1] = bf16hi(w[e]);
+  }
+}
+template <typename T> __device__ __forceinline__ void store8t(T* p, const float* v);
+template <> __device__ __forceinline__ void store8t<float>(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <> __device__ __forceinline__ void store8t<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// Thread = (token, group of 8 channels), grid-stride over the tokens of head h = blockIdx.y:
+// dk[s] = sum_j w[j] dkc[s - j + p] over in-frame indices (out[s'] reads x[s' + j - p]), and the
+// tap partials sum_s dkc[s] k[s + j - p], reduced per block.  A missing conv is the identity
+// (centre tap 1); KT is the tap count of the staged convs.
+template <int D, typename T, int KT>
 __global__ void __launch_bounds__(kBT) k_bwd_conv(const T* __restrict__ k, const T* __restrict__ v,
                                                   const float* __restrict__ wk, const float* __restrict__ wv,
-                                                  int K, const float* __restrict__ dkc,
-                                                  const float* __restrict__ dvc, T* __restrict__ dk,
-                                                  T* __restrict__ dv, float* __restrict__ tap_part, int B, int H,
-                                                  int F, int S) {
-  constexpr int PER = Lanes<D>::PER;
-  __shared__ float red[kBT / 32][2][D][3];
+                                                  const float* __restrict__ dkc, const float* __restrict__ dvc,
+                                                  T* __restrict__ dk, T* __restrict__ dv,
+                                                  float* __restrict__ tap_part, int B, int H, int F, int S) {
+  constexpr int G = D / 8;                 // channel groups
+  constexpr int TPI = kBT / G;             // tokens per block and iteration
+  constexpr int PAD = (KT - 1) / 2;
+  __shared__ float red[kBT / 32][G][2][KT][8];
   const int h = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long N = (long long)F * S;
-  const long long total = (long long)B * N;     // tokens of head h
-  const int pad = (K - 1) / 2;
-  float tk[PER][3], tv[PER][3];
+  const int tid = threadIdx.x, cg = tid % G, tl = tid / G, warp = tid >> 5, lane = tid & 31;
+  const int c0 = 8 * cg;
+  const long long N = (long long)F * S, total = (long long)B * N;
+  float wkr[KT][8], wvr[KT][8], tk[KT][8], tv[KT][8];
 #pragma unroll
-  for (int r = 0; r < PER; ++r)
+  for (int j = 0; j < KT; ++j)
 #pragma unroll
-    for (int j = 0; j < 3; ++j) tk[r][j] = tv[r][j] = 0.f;
-  for (long long tokn = (long long)blockIdx.x * (kBT / 32) + warp; tokn < total;
-       tokn += (long long)gridDim.x * (kBT / 32)) {
+    for (int e = 0; e < 8; ++e) {
+      wkr[j][e] = wk ? wk[((long long)h * D + c0 + e) * KT + j] : (j == PAD ? 1.f : 0.f);
+      wvr[j][e] = wv ? wv[((long long)h * D + c0 + e) * KT + j] : (j == PAD ? 1.f : 0.f);
+      tk[j][e] = tv[j][e] = 0.f;
+    }
+  for (long long tokn = (long long)blockIdx.x * TPI + tl; tokn < total; tokn += (long long)gridDim.x * TPI) {
     const long long b = tokn / N, n = tokn % N;
     const int s = (int)(n % S);
+    const long long row = (b * N + n) * H + h;     // token row (times D)
+    float ck[8], cv[8], gk[8], gv[8];
+    load8t(dkc + row * D + c0, ck);
+    load8t(dvc + row * D + c0, cv);
 #pragma unroll
-    for (int r = 0; r < PER; ++r) {
-      if (!Lanes<D>::has(lane, r)) continue;
-      const int c = lane + 32 * r;
-      const long long base = ((b * N + n) * H + h) * D + c;
-      float gk = 0.f, gv = 0.f;
-      if (wk == nullptr) gk = dkc[base];
-      if (wv == nullptr) gv = dvc[base];
-      for (int j = 0; j < K; ++j) {
-        // out[s'] uses x[s' + j - pad]: x[s] feeds out[s - j + pad]
-        const int so = s - j + pad;
-        if (so >= 0 && so < S) {
-          const long long ob = ((b * N + (n - s + so)) * H + h) * D + c;
-          if (wk) gk = fmaf(wk[((long long)h * D + c) * K + j], dkc[ob], gk);
-          if (wv) gv = fmaf(wv[((long long)h * D + c) * K + j], dvc[ob], gv);
+    for (int e = 0; e < 8; ++e) gk[e] = gv[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+      const int so = s - j + PAD;                  // out[so] reads x[s] through tap j
+      if (so >= 0 && so < S) {
+        float a[8], c[8];
+        if (so == s) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            a[e] = ck[e];
+            c[e] = cv[e];
+          }
+        } else {
+          load8t(dkc + (row + (long long)(so - s) * H) * D + c0, a);
+          load8t(dvc + (row + (long long)(so - s) * H) * D + c0, c);
         }
-        const int sx = s + j - pad;               // tap j of out[s] reads x[s + j - pad]
-        if (sx >= 0 && sx < S) {
-          const long long xb = ((b * N + (n - s + sx)) * H + h) * D + c;
-          if (wk) tk[r][j] = fmaf(dkc[base], to_f32(k[xb]), tk[r][j]);
-          if (wv) tv[r][j] = fmaf(dvc[base], to_f32(v[xb]), tv[r][j]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          gk[e] = fmaf(wkr[j][e], a[e], gk[e]);
+          gv[e] = fmaf(wvr[j][e], c[e], gv[e]);
         }
       }
-      dk[base] = from_f32<T>(gk);
-      dv[base] = from_f32<T>(gv);
+      const int sx = s + j - PAD;                  // tap j of out[s] reads x[sx]
+      if (sx >= 0 && sx < S) {
+        float x[8], y[8];
+        load8t(k + (row + (long long)(sx - s) * H) * D + c0, x);
+        load8t(v + (row + (long long)(sx - s) * H) * D + c0, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          tk[j][e] = fmaf(ck[e], x[e], tk[j][e]);
+          tv[j][e] = fmaf(cv[e], y[e], tv[j][e]);
+        }
+      }
     }
+    store8t(dk + row * D + c0, gk);
+    store8t(dv + row * D + c0, gv);
   }
+  // tap partials: lanes with the same channel group within the warp, then the block's warps
 #pragma unroll
-  for (int r = 0; r < PER; ++r)
-    if (Lanes<D>::has(lane, r))
+  for (int off = G; off < 32; off <<= 1)
 #pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        red[warp][0][lane + 32 * r][j] = tk[r][j];
-        red[warp][1][lane + 32 * r][j] = tv[r][j];
+    for (int j = 0; j < KT; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        tk[j][e] += __shfl_xor_sync(0xffffffffu, tk[j][e], off);
+        tv[j][e] += __shfl_xor_sync(0xffffffffu, tv[j][e], off);
+      }
+  if (lane < G)
+#pragma unroll
+    for (int j = 0; j < KT; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        red[warp][cg][0][j][e] = tk[j][e];
+        red[warp][cg][1][j][e] = tv[j][e];
       }
   __syncthreads();
-  for (int e = threadIdx.x; e < 2 * D * 3; e += kBT) {
-    const int m = e / (D * 3), c = (e / 3) % D, j = e % 3;
+  for (int idx = tid; idx < G * 2 * KT * 8; idx += kBT) {
+    const int e = idx % 8, j = (idx / 8) % KT, m = (idx / (8 * KT)) % 2, g2 = idx / (16 * KT);
     float acc = 0.f;
-    for (int w = 0; w < kBT / 32; ++w) acc += red[w][m][c][j];
-    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * D * 3 + c * 3 + j] = acc;
+    for (int w = 0; w < kBT / 32; ++w) acc += red[w][g2][m][j][e];
+    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * D * 3 + (8 * g2 + e) * 3 + j] = acc;
   }
 }
 
@@ -733,8 +807,9 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   }
   if ((e = mark()) != cudaSuccess) return e;
   // step 4 (gather + bridge) reversed
-  k_bwd_gather<D><<<(unsigned)BH, kBT, 0, a.stream>>>(at(p.P), at(p.Q), a.alpha, a.text_state, at(p.dW), at(p.dPin),
-                                                      at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk, a.radius);
+  k_bwd_gather<D><<<dim3((unsigned)BH, D < 32 ? 1 : D / 32), kBT, 0, a.stream>>>(
+      at(p.P), at(p.Q), a.alpha, a.text_state, at(p.dW), at(p.dPin), at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk,
+      a.radius);
   if ((e = mark()) != cudaSuccess) return e;
   // steps 3-4 (scans) reversed
   k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(
@@ -755,9 +830,14 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   }
   if ((e = mark()) != cudaSuccess) return e;
   // step 1 (conv) reversed
-  k_bwd_conv<D, T><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
-      static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, K, at(p.dkc), at(p.dvc),
-      static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  if (K == 3)
+    k_bwd_conv<D, T, 3><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
+        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, at(p.dkc), at(p.dvc),
+        static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  else
+    k_bwd_conv<D, T, 1><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
+        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, at(p.dkc), at(p.dvc),
+        static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
   if ((e = mark()) != cudaSuccess) return e;
   k_bwd_finish<D><<<148, kBT, 0, a.stream>>>(at(p.rms_part), NF, at(p.tap_part), kBwdConvBlocks, K, at(p.dseed2),
                                              at(p.dalpha_g), at(p.dalpha2), g.drms_w, g.dconv_k_w, g.dconv_v_w,
