@@ -344,6 +344,7 @@ struct StatsTcSmem {
   uint8_t kraw[kRawRows * kRawStride];   // raw k rows s0 - 1 .. s0 + 128 (bf16; zero outside the frame)
   uint8_t vraw[kRawRows * kRawStride];
   float taps[2][3][128];                 // [k, v][tap][channel] of this head (identity: centre tap 1)
+  float red[3][2][128];                  // per-token partial sums of the two column halves
   uint64_t bar;
   uint32_t tmem_base;
   int abort;
@@ -369,14 +370,20 @@ __device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128]
   }
 }
 
-__global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __restrict__ k,
-                                                      const __nv_bfloat16* __restrict__ v,
-                                                      const float* __restrict__ beta, const float* __restrict__ wk,
-                                                      const float* __restrict__ wv, int K,
-                                                      const float* __restrict__ dA2, const float* __restrict__ dB2,
-                                                      float* __restrict__ dkc, float* __restrict__ dvc,
-                                                      float* __restrict__ dbeta, int H, int F, int S,
-                                                      uint32_t* __restrict__ status) {
+// Two threads per token row: the warps w and w + 4 share TMEM lanes 32 (w % 4) .. and take the
+// column halves 64 hf .. 64 hf + 63 (hf = w / 4); per-token sums are combined in shared memory.
+constexpr int kStatsThreads = 256;
+
+__global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloat16* __restrict__ k,
+                                                                const __nv_bfloat16* __restrict__ v,
+                                                                const float* __restrict__ beta,
+                                                                const float* __restrict__ wk,
+                                                                const float* __restrict__ wv, int K,
+                                                                const float* __restrict__ dA2,
+                                                                const float* __restrict__ dB2,
+                                                                float* __restrict__ dkc, float* __restrict__ dvc,
+                                                                float* __restrict__ dbeta, int H, int F, int S,
+                                                                uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   StatsTcSmem& sm = *reinterpret_cast<StatsTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const long long fi = blockIdx.x;
@@ -386,8 +393,10 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
   const int h = (int)(bh % H);
   const long long b = bh / H;
   const long long N = (long long)F * S;
-  const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0 (times H * 128 below)
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, hf = warp >> 2;
+  const int m = 32 * quarter + lane;                       // token of the tile = TMEM lane
   const int Kc = wk ? K : (wv ? K : 1);      // taps of the staged convs (a missing one: identity)
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {
@@ -399,46 +408,45 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
     tc::tmem_alloc(&sm.tmem_base, 512);
     tc::tmem_relinquish();
   }
-  // images of dA + dA^T and dB (both scans' parts summed); thread i writes row i
+  // images of dA + dA^T (threads 0..127, row = tid) and dB (threads 128..255), both scans' parts summed
   {
-    const float* a0 = dA2 + fi * 16384;
-    const float* a1 = dA2 + (NFt + fi) * 16384;
-    const float* b0 = dB2 + fi * 16384;
-    const float* b1 = dB2 + (NFt + fi) * 16384;
-    const int i = tid;
+    const int i = tid & 127;
+    const float* x0 = (tid < 128 ? dA2 : dB2) + fi * 16384;
+    const float* x1 = (tid < 128 ? dA2 : dB2) + (NFt + fi) * 16384;
+    uint8_t* img = tid < 128 ? sm.da : sm.db;
     for (int c = 0; c < 16; ++c) {
-      float va[8], vb[8];
+      float va[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int j = 8 * c + e;
-        va[e] = a0[i * 128 + j] + a1[i * 128 + j] + a0[j * 128 + i] + a1[j * 128 + i];
-        vb[e] = b0[i * 128 + j] + b1[i * 128 + j];
+        va[e] = x0[i * 128 + j] + x1[i * 128 + j];
+        if (tid < 128) va[e] += x0[j * 128 + i] + x1[j * 128 + i];
       }
-      store_chunk_bf16(sm.da, i, 8 * c, va);
-      store_chunk_bf16(sm.db, i, 8 * c, vb);
+      store_chunk_bf16(img, i, 8 * c, va);
     }
     // taps of this head, [tensor][tap][channel]; a missing conv is the identity (one centre tap)
-    for (int j = 0; j < 3; ++j) {
-      const bool centre = j == (Kc - 1) / 2;
-      sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
-      sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
-    }
+    if (tid < 128)
+      for (int j = 0; j < 3; ++j) {
+        const bool centre = j == (Kc - 1) / 2;
+        sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+        sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+      }
   }
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;        // U at 0, Z at 128, V' dB at 256
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t tmem = sm.tmem_base;        // U |x| at 0, Z |x| at 128, V' dB at 256
+  const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
   const uint32_t a_da = tc::smem_u32(sm.da), a_db = tc::smem_u32(sm.db), a_k = tc::smem_u32(sm.kf),
                  a_v = tc::smem_u32(sm.vf);
   uint32_t ph = 0;
   bool ok = true;
   for (int s0 = 0; s0 < S && ok; s0 += kBT) {
-    const int s = s0 + tid;
+    const int s = s0 + m;
     const bool valid = s < S;
     // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame)
-    for (int r = tid; r < kRawRows; r += kBT) {
+    for (int r = tid; r < kRawRows; r += kStatsThreads) {
       const int sr = s0 - 1 + r;
       const bool in = sr >= 0 && sr < S;
       const long long base = ((frame_row0 + (in ? sr : 0)) * H + h) * 128;
@@ -456,13 +464,14 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
     }
     __syncthreads();
     // x = silu(conv k) (k' = x / |x|: the 1/|x| is applied to U and Z in the epilogue) and
-    // v' = silu(conv v) into the K', V' tiles
+    // v' = silu(conv v) into the K', V' tiles: this thread's 8 chunks of its token
     float ss = 0.f;
-    for (int c = 0; c < 16; ++c) {
+#pragma unroll 2
+    for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
       float kv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
-        conv8(sm.kraw, sm.taps[0], Kc, tid, s, S, 8 * c, kv);
-        conv8(sm.vraw, sm.taps[1], Kc, tid, s, S, 8 * c, vv);
+        conv8(sm.kraw, sm.taps[0], Kc, m, s, S, 8 * c, kv);
+        conv8(sm.vraw, sm.taps[1], Kc, m, s, S, 8 * c, vv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           kv[e] = silu_f(kv[e]);
@@ -470,10 +479,10 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
           vv[e] = silu_f(vv[e]);
         }
       }
-      store_chunk_bf16(sm.kf, tid, 8 * c, kv);
-      store_chunk_bf16(sm.vf, tid, 8 * c, vv);
+      store_chunk_bf16(sm.kf, m, 8 * c, kv);
+      store_chunk_bf16(sm.vf, m, 8 * c, vv);
     }
-    const float inv = rsqrtf(ss + kL2Eps);
+    sm.red[0][hf][m] = ss;
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
@@ -487,13 +496,14 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
     if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
     ph ^= 1;
     tc::tc_fence_after();
+    const float inv = rsqrtf(sm.red[0][0][m] + sm.red[0][1][m] + kL2Eps);
     // the TMEM loads are warp-collective: every thread loads, only valid tokens compute
     const long long tok = frame_row0 * H + (long long)(valid ? s : 0) * H + h;
     const float bt = valid ? beta[tok] : 0.f;
-    // pass 1: d beta and x . dk' from the tiles' x and v' (bf16) and U, Z, V'dB (u = inv U, z = inv Z)
+    // pass 1: d beta and x . dk' over this thread's half, from the tiles' x and v' (bf16)
     float dbt = 0.f, xg = 0.f;
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t u[32], z[32], w[32];
       tc::tmem_ld32(tmem + 32 * p + lane_off, u);
       tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, z);
@@ -503,13 +513,13 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float xk[8], xv[8];
-        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.kf + img_offset(0, tid, 32 * p + 8 * c8)), xk);
-        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.vf + img_offset(0, tid, 32 * p + 8 * c8)), xv);
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.kf + img_offset(0, m, 32 * p + 8 * c8)), xk);
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.vf + img_offset(0, m, 32 * p + 8 * c8)), xv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int m = 8 * c8 + e;
-          const float uu = inv * __uint_as_float(u[m]), zz = inv * __uint_as_float(z[m]);
-          const float ww = __uint_as_float(w[m]);
+          const int q8 = 8 * c8 + e;
+          const float uu = inv * __uint_as_float(u[q8]), zz = inv * __uint_as_float(z[q8]);
+          const float ww = __uint_as_float(w[q8]);
           // d beta = 1/2 k'^T (dA + dA^T) k' + v'^T dB k'
           dbt = fmaf(0.5f * xk[e] * inv, uu, dbt);
           dbt = fmaf(xv[e], zz, dbt);
@@ -517,10 +527,14 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
         }
       }
     }
-    if (valid) dbeta[tok] = dbt;
-    // pass 2: dkc = silu'(kc) (dk' - x (x . dk') / n^2) / n, dvc = silu'(vc) beta z
+    sm.red[1][hf][m] = dbt;
+    sm.red[2][hf][m] = xg;
+    __syncthreads();
+    xg = sm.red[2][0][m] + sm.red[2][1][m];
+    if (valid && hf == 0) dbeta[tok] = sm.red[1][0][m] + sm.red[1][1][m];
+    // pass 2: dkc = silu'(kc) (dk' - x (x . dk') / |x|^2) / |x|, dvc = silu'(vc) beta z
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t u[32], z[32], w[32];
       tc::tmem_ld32(tmem + 32 * p + lane_off, u);
       tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, z);
@@ -531,15 +545,16 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats_tc(const __nv_bfloat16* __res
       for (int c8 = 0; c8 < 4; ++c8) {
         const int c0 = 32 * p + 8 * c8;
         float kc[8], vc[8], gk[8], gv[8];
-        conv8(sm.kraw, sm.taps[0], Kc, tid, s, S, c0, kc);
-        conv8(sm.vraw, sm.taps[1], Kc, tid, s, S, c0, vc);
+        conv8(sm.kraw, sm.taps[0], Kc, m, s, S, c0, kc);
+        conv8(sm.vraw, sm.taps[1], Kc, m, s, S, c0, vc);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int m = 8 * c8 + e;
-          const float x = silu_f(kc[e]);
-          const float dk = bt * (inv * __uint_as_float(u[m]) + __uint_as_float(w[m]));
-          gk[e] = silu_grad_f(kc[e], (dk - x * xg * inv * inv) * inv);
-          gv[e] = silu_grad_f(vc[e], bt * inv * __uint_as_float(z[m]));
+          const int q8 = 8 * c8 + e;
+          const float sg = sigm_fast(kc[e]);
+          const float x = kc[e] * sg;
+          const float dk = bt * (inv * __uint_as_float(u[q8]) + __uint_as_float(w[q8]));
+          gk[e] = (dk - x * xg * inv * inv) * inv * sg * fmaf(kc[e], 1.f - sg, 1.f);
+          gv[e] = silu_grad_f(vc[e], bt * inv * __uint_as_float(z[q8]));
         }
         float* pk = dkc + tok * 128 + c0;
         float* pv = dvc + tok * 128 + c0;
@@ -580,7 +595,7 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
   const size_t smem = sizeof(StatsTcSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_bwd_stats_tc<<<(unsigned)a.NF(), kBT, smem, a.stream>>>(
+  k_bwd_stats_tc<<<(unsigned)a.NF(), kStatsThreads, smem, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
       a.conv_v_w, K, dA2, dB2, dkc, dvc, dbeta, a.sh.H, a.sh.F, a.sh.S, status);
   return cudaGetLastError();
