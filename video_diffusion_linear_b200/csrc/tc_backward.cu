@@ -95,25 +95,26 @@ __device__ __forceinline__ float silu_grad_f(float x, float g) {
   return g * s * fmaf(x, 1.f - s, 1.f);
 }
 
+constexpr int kReadoutThreads = 256;   // two threads per token row (column halves)
 struct ReadoutTcSmem {
   uint8_t w[32768];     // W_t image (rows i, K = j)
   uint8_t qf[32768];    // Q' tile (rows tokens, K = j)
   uint8_t dov[32768];   // DO tile (rows tokens, K = i)
-  float rms[4][128];
+  float rms[8][128];    // per-warp RMS-weight partials (zero outside the warp's column half)
+  float red[4][2][128]; // per-token partial sums of the two column halves
   uint64_t bar;
   uint32_t tmem_base;
   int abort;
 };
 
 // ---------------------------------------------------------------- Step 5 reversed
-__global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __restrict__ q,
-                                                        const __nv_bfloat16* __restrict__ gate,
-                                                        const __nv_bfloat16* __restrict__ dout,
-                                                        const float* __restrict__ rms_w,
-                                                        const float* __restrict__ Wall, float* __restrict__ dWall,
-                                                        float* __restrict__ rms_part, __nv_bfloat16* __restrict__ dq,
-                                                        __nv_bfloat16* __restrict__ dgate, int H, int F, int S,
-                                                        uint32_t* __restrict__ status) {
+// Two threads per token row: the warps w and w + 4 share TMEM lanes 32 (w % 4) .. and take the
+// column halves 64 hf .. 64 hf + 63 (hf = w / 4); per-token sums are combined in shared memory.
+__global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gate,
+    const __nv_bfloat16* __restrict__ dout, const float* __restrict__ rms_w, const float* __restrict__ Wall,
+    float* __restrict__ dWall, float* __restrict__ rms_part, __nv_bfloat16* __restrict__ dq,
+    __nv_bfloat16* __restrict__ dgate, int H, int F, int S, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ReadoutTcSmem& sm =
       *reinterpret_cast<ReadoutTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -124,6 +125,8 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
   const long long b = bh / H;
   const long long N = (long long)F * S;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, hf = warp >> 2;
+  const int m = 32 * quarter + lane;                // token of the tile = TMEM lane
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {
     tc::mbar_init(&sm.bar, 1);
@@ -134,15 +137,16 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     tc::tmem_alloc(&sm.tmem_base, 256);
     tc::tmem_relinquish();
   }
-  // W_t image: thread n writes row n
+  for (int e = tid; e < 8 * 128; e += kReadoutThreads) (&sm.rms[0][0])[e] = 0.f;
+  // W_t image: thread (m, hf) writes the 8 chunks of its half of row m
   {
-    const float* wr = Wall + fi * 16384 + tid * 128;
+    const float* wr = Wall + fi * 16384 + m * 128;
 #pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
       const float4 a = *reinterpret_cast<const float4*>(wr + 8 * c);
       const float4 bq = *reinterpret_cast<const float4*>(wr + 8 * c + 4);
       const float v[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-      store_chunk_bf16(sm.w, tid, 8 * c, v);
+      store_chunk_bf16(sm.w, m, 8 * c, v);
     }
   }
   tc::fence_proxy_async_smem();
@@ -150,20 +154,24 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;        // O / dQ' at columns 0..127, dW at 128..255
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
   const uint32_t aw = tc::smem_u32(sm.w), aq = tc::smem_u32(sm.qf), ad = tc::smem_u32(sm.dov);
-  float racc[4] = {0.f, 0.f, 0.f, 0.f};
+  auto ld_row = [&](int p, uint32_t (&r)[32]) {     // columns 32 p .. 32 p + 31 of this token's row
+    tc::tmem_ld32(tmem + 32 * p + lane_off, r);
+    tc::tmem_ld_wait();
+  };
+  float racc[2] = {0.f, 0.f};
   uint32_t ph = 0;
   bool ok = true;
   int tile = 0;
   for (int s0 = 0; s0 < S && ok; s0 += kBT, ++tile) {
-    const int s = s0 + tid;
+    const int s = s0 + m;
     const bool valid = s < S;
     const long long row = ((b * N + (long long)f * S + (valid ? s : 0)) * H + h) * 128;
     // x = silu(q) into the Q' tile (q' = x / |x|: the 1/|x| is folded into O, DO and dQ' below)
     float ss = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
         load8_bf16(q + row + 8 * c, v);
@@ -173,9 +181,9 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
           ss = fmaf(v[e], v[e], ss);
         }
       }
-      store_chunk_bf16(sm.qf, tid, 8 * c, v);
+      store_chunk_bf16(sm.qf, m, 8 * c, v);
     }
-    const float inv = rsqrtf(ss + kL2Eps), nrm = (ss + kL2Eps) * inv;   // 1/|x|, |x|
+    sm.red[0][hf][m] = ss;
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
@@ -187,25 +195,24 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     if (!(ok = tc::mbar_wait(&sm.bar, ph, abort_flag, status))) break;
     ph ^= 1;
     tc::tc_fence_after();
-    // this token's row of O, 32 columns at a time (re-read from TMEM for each pass)
-    auto ld_row = [&](int p, uint32_t (&r)[32]) {
-      tc::tmem_ld32(tmem + 32 * p + lane_off, r);
-      tc::tmem_ld_wait();
-    };
+    const float sst = sm.red[0][0][m] + sm.red[0][1][m] + kL2Eps;
+    const float inv = rsqrtf(sst), nrm = sst * inv;   // 1/|x|, |x|
     // RMSNorm and gate reversed
     float so2 = 0.f;
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t o[32];
       ld_row(p, o);
 #pragma unroll
       for (int c = 0; c < 32; ++c) so2 = fmaf(__uint_as_float(o[c]), __uint_as_float(o[c]), so2);
     }
-    so2 *= inv * inv;
-    const float rr = rsqrtf(so2 * (1.f / 128.f) + kRmsEps);
+    sm.red[1][hf][m] = so2;
+    __syncthreads();
+    const float rr = rsqrtf((sm.red[1][0][m] + sm.red[1][1][m]) * inv * inv * (1.f / 128.f) + kRmsEps);
     float so = 0.f;
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int pp = 0; pp < 2; ++pp) {
+      const int p = 2 * hf + pp;
       uint32_t o[32];
       ld_row(p, o);
       float red[32];
@@ -222,21 +229,22 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
         *reinterpret_cast<float4*>(rw8 + 4) = __ldg(reinterpret_cast<const float4*>(rms_w + c0 + 4));
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float rw = rw8[e];
           const float ov = inv * __uint_as_float(o[8 * c8 + e]);
           const float oh = ov * rr;
           const float dy = go[e] * g[e];
-          dg[e] = go[e] * oh * rw;
+          dg[e] = go[e] * oh * rw8[e];
           red[8 * c8 + e] = dy * oh;
-          so = fmaf(dy * rw, ov, so);
+          so = fmaf(dy * rw8[e], ov, so);
         }
         if (valid) store8_bf16(dgate + row + c0, dg);
       }
-      racc[p] += transpose_sum32(red, lane);
+      racc[pp] += transpose_sum32(red, lane);
     }
-    const float k3 = rr * rr * rr * so * (1.f / 128.f);
+    sm.red[2][hf][m] = so;
+    __syncthreads();
+    const float k3 = rr * rr * rr * (sm.red[2][0][m] + sm.red[2][1][m]) * (1.f / 128.f);
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t o[32];
       ld_row(p, o);
 #pragma unroll
@@ -254,7 +262,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
           for (int e = 0; e < 8; ++e)
             v[e] = inv * (rr * go[e] * g[e] * rw8[e] - k3 * inv * __uint_as_float(o[8 * c8 + e]));
         }
-        store_chunk_bf16(sm.dov, tid, c0, v);
+        store_chunk_bf16(sm.dov, m, c0, v);
       }
     }
     tc::fence_proxy_async_smem();
@@ -273,20 +281,23 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     // x.g from the tile's x (bf16), then dq = silu'(q) dx
     float xg = 0.f;
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t o[32];
       ld_row(p, o);
       if (!valid) continue;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float x[8];
-        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.qf + img_offset(0, tid, 32 * p + 8 * c8)), x);
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.qf + img_offset(0, m, 32 * p + 8 * c8)), x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) xg = fmaf(x[e], nrm * __uint_as_float(o[8 * c8 + e]), xg);
       }
     }
+    sm.red[3][hf][m] = xg;
+    __syncthreads();
+    xg = sm.red[3][0][m] + sm.red[3][1][m];
 #pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t o[32];
       ld_row(p, o);
       if (!valid) continue;
@@ -309,9 +320,9 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
     tc::tc_fence_after();
   }
   if (ok) {
-    float* dW = dWall + fi * 16384 + tid * 128;   // row i = tid
+    float* dW = dWall + fi * 16384 + m * 128;   // row i = m, this thread's column half
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
       uint32_t r[32];
       tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, r);
       tc::tmem_ld_wait();
@@ -322,11 +333,16 @@ __global__ void __launch_bounds__(kBT) k_bwd_readout_tc(const __nv_bfloat16* __r
                         __uint_as_float(r[e + 3]));
     }
   }
-#pragma unroll
-  for (int p = 0; p < 4; ++p) sm.rms[warp][32 * p + lane] = racc[p];
+  sm.rms[warp][32 * (2 * hf) + lane] = racc[0];
+  sm.rms[warp][32 * (2 * hf + 1) + lane] = racc[1];
   tc::tc_fence_before();
   __syncthreads();
-  rms_part[fi * 128 + tid] = sm.rms[0][tid] + sm.rms[1][tid] + sm.rms[2][tid] + sm.rms[3][tid];
+  if (tid < 128) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += sm.rms[w][tid];
+    rms_part[fi * 128 + tid] = acc;
+  }
   if (warp == 0) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 256);
@@ -583,7 +599,7 @@ cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* 
   const size_t smem = sizeof(ReadoutTcSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_bwd_readout_tc<<<(unsigned)a.NF(), kBT, smem, a.stream>>>(
+  k_bwd_readout_tc<<<(unsigned)a.NF(), kReadoutThreads, smem, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gate),
       static_cast<const __nv_bfloat16*>(dout), a.rms_w, W, dW, rms_part, static_cast<__nv_bfloat16*>(dq),
       static_cast<__nv_bfloat16*>(dgate), a.sh.H, a.sh.F, a.sh.S, status);
