@@ -172,10 +172,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
                                                            float scale, int accumulate,
                                                            __nv_bfloat16* __restrict__ out,
                                                            uint32_t* __restrict__ status) {
-  const long long bh = blockIdx.x;
+  // consecutive CTAs take consecutive query tiles of one (batch, head, chunk): the CTAs resident
+  // at a time share one K/V window in L2
+  const long long bh = blockIdx.y;
   const int h = (int)(bh % H);
   const long long b = bh / H;
-  const int c = blockIdx.y / tiles_per_chunk, tile = blockIdx.y % tiles_per_chunk;
+  const int c = blockIdx.x / tiles_per_chunk, tile = blockIdx.x % tiles_per_chunk;
   const int f0 = c * chunk;
   if (f0 >= F) return;
   const long long N = (long long)F * S;
@@ -456,11 +458,11 @@ cudaError_t launch_window_softmax_tc(const vdn_shape& sh, const void* qr, const 
     return cudaErrorInvalidValue;
   const int nchunks = (sh.F + chunk - 1) / chunk;
   const int tiles = (int)(((long long)chunk * sh.S + 127) / 128);
-  if ((long long)nchunks * tiles > 65535) return cudaErrorInvalidConfiguration;
+  if ((long long)sh.B * sh.H > 65535) return cudaErrorInvalidConfiguration;
   const size_t smem = sizeof(WsoftSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_wsoft_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((long long)sh.B * sh.H), (unsigned)(nchunks * tiles));
+  dim3 grid((unsigned)(nchunks * tiles), (unsigned)((long long)sh.B * sh.H));
   k_wsoft_tc<<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, sh.H, sh.F, sh.S, chunk, radius, tiles,
                                                  scale * kLog2e, accumulate, static_cast<__nv_bfloat16*>(out),
                                                  status);
