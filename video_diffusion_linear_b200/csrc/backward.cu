@@ -367,19 +367,17 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
 // ---------------------------------------------------------------- steps 3-4 (scans) reversed
 // Block (b, h, dir): dir 0 reverses the prefix scan P_f = step(P_{f-1}, f) from f = F-1 down,
 // dir 1 the suffix scan Q_f = step(Q_{f+1}, f) from f = 0 up.  For the generic step
-// S_out = (S_in D + cpre B) N + cpost B:
-//   dX = lam N^T (N symmetric), dS_in = dX D, dalpha_j = sum_i S_in[i][j] dX[i][j],
-//   dB = cpre dX + cpost lam, dA = -c2 S_out^T dX (N = (I + c2 A)^-1) or -c2 X^T lam (N = I - c2 A).
-// scratch: 4 D x D per block (lam, dX, X, seed).
+// S_out = (S_in D + cpre B) N + cpost B the recurrence needs only
+//   lam_f = (gradient reaching S_out) ,  dX_f = lam_f N^T (N symmetric) ,  next lam = dX_f D;
+// lam_f and dX_f of every frame are stored for k_bwd_scan_grads, which forms dA, dB, d alpha.
+// scratch: 2 D x D per block (the running lam, the seed).
 template <int D>
-__global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Bm, const float* __restrict__ Nm,
-                                                  const float* __restrict__ P, const float* __restrict__ Q,
-                                                  const float* __restrict__ alpha,
-                                                  const float* __restrict__ text_state, RuleCoef rc,
+__global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Nm, const float* __restrict__ alpha,
+                                                  const float* __restrict__ text_state,
                                                   const float* __restrict__ dPin, const float* __restrict__ dQin,
-                                                  float* __restrict__ dA2, float* __restrict__ dB2,
-                                                  float* __restrict__ dalpha2, float* __restrict__ dseed2,
-                                                  float* __restrict__ scratch, int H, int F) {
+                                                  float* __restrict__ lam_all, float* __restrict__ dX_all,
+                                                  float* __restrict__ dseed2, float* __restrict__ scratch, int H,
+                                                  int F) {
   __shared__ float slab[2 * 16 * (D + 1)];
   const long long bh = blockIdx.x;
   const int dir = blockIdx.y;
@@ -388,11 +386,8 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Bm, 
   const long long DD = (long long)D * D;
   const long long BH = gridDim.x;
   const int tid = threadIdx.x;
-  float* lam = scratch + (bh * 2 + dir) * 4 * DD;
-  float* dX = lam + DD;
-  float* X = dX + DD;
-  float* seed = X + DD;
-  const float* S = dir == 0 ? P : Q;
+  float* lam = scratch + (bh * 2 + dir) * 2 * DD;
+  float* seed = lam + DD;
   const float* din = (dir == 0 ? dPin : dQin) + bh * (F + 1) * DD;
   for (long long e = tid; e < DD; e += kBT) {
     seed[e] = text_state ? 0.5f * text_state[(long long)h * DD + e] : 0.f;
@@ -402,33 +397,13 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Bm, 
   for (int it = 0; it < F; ++it) {
     const int f = dir == 0 ? F - 1 - it : it;
     const long long fo = (bh * F + f) * DD;
-    const float* S_out = S + fo;
-    const float* S_in = dir == 0 ? (f == 0 ? seed : S + fo - DD) : (f == F - 1 ? seed : S + fo + DD);
+    const long long go = ((long long)dir * BH * F + bh * F + f) * DD;
     const float* gin = din + (long long)(dir == 0 ? f + 1 : f) * DD;
-    for (long long e = tid; e < DD; e += kBT) lam[e] += gin[e];
+    float* lf = lam_all + go;
+    for (long long e = tid; e < DD; e += kBT) lf[e] = lam[e] + gin[e];
     __syncthreads();
-    cta_mm<D>(dX, lam, false, Nm + fo, true, 1.f, slab);
-    float* dA = dA2 + ((long long)dir * BH * F + bh * F + f) * DD;
-    float* dB = dB2 + ((long long)dir * BH * F + bh * F + f) * DD;
-    if (rc.solve) {
-      cta_mm<D>(dA, S_out, true, dX, false, -rc.c2, slab);
-    } else if (rc.c2 != 0.f) {
-      for (long long e = tid; e < DD; e += kBT) {
-        const int jj = (int)(e % D);
-        X[e] = S_in[e] * alpha[((b * F + f) * H + h) * D + jj] + rc.cpre * Bm[fo + e];
-      }
-      __syncthreads();
-      cta_mm<D>(dA, X, true, lam, false, -rc.c2, slab);
-    } else {
-      for (long long e = tid; e < DD; e += kBT) dA[e] = 0.f;
-    }
-    for (long long e = tid; e < DD; e += kBT) dB[e] = rc.cpre * dX[e] + rc.cpost * lam[e];
-    if (tid < D) {
-      float acc = 0.f;
-      for (int i = 0; i < D; ++i) acc = fmaf(S_in[i * D + tid], dX[i * D + tid], acc);
-      dalpha2[((long long)dir * BH * F + bh * F + f) * D + tid] = acc;
-    }
-    __syncthreads();
+    cta_mm<D>(dX_all + go, lf, false, Nm + fo, true, 1.f, slab);
+    const float* dX = dX_all + go;
     for (long long e = tid; e < DD; e += kBT) {
       const int jj = (int)(e % D);
       lam[e] = dX[e] * alpha[((b * F + f) * H + h) * D + jj];
@@ -437,6 +412,61 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan(const float* __restrict__ Bm, 
   }
   const float* g0 = din + (long long)(dir == 0 ? 0 : F) * DD;
   for (long long e = tid; e < DD; e += kBT) dseed2[((long long)dir * BH + bh) * DD + e] = lam[e] + g0[e];
+}
+
+// Block (b h f, dir): the step's gradients from lam_f and dX_f,
+//   dB = cpre dX + cpost lam, d alpha_j = sum_i S_in[i][j] dX[i][j],
+//   dA = -c2 S_out^T dX (N = (I + c2 A)^-1) or -c2 X^T lam with X = S_in D + cpre B (N = I - c2 A).
+// Xbuf: one D x D per block.
+template <int D>
+__global__ void __launch_bounds__(kBT) k_bwd_scan_grads(const float* __restrict__ Bm, const float* __restrict__ P,
+                                                        const float* __restrict__ Q,
+                                                        const float* __restrict__ alpha, RuleCoef rc,
+                                                        const float* __restrict__ lam_all,
+                                                        const float* __restrict__ dX_all,
+                                                        const float* __restrict__ scan_scratch,
+                                                        float* __restrict__ dA2, float* __restrict__ dB2,
+                                                        float* __restrict__ dalpha2, float* __restrict__ Xbuf, int H,
+                                                        int F) {
+  __shared__ float slab[2 * 16 * (D + 1)];
+  const long long fi = blockIdx.x;            // (b, h, f)
+  const int dir = blockIdx.y;
+  const long long NFt = gridDim.x;
+  const int f = (int)(fi % F);
+  const long long bh = fi / F;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long DD = (long long)D * D;
+  const int tid = threadIdx.x;
+  const long long fo = fi * DD;
+  const long long go = ((long long)dir * NFt + fi) * DD;
+  const float* S = dir == 0 ? P : Q;
+  const float* seed = scan_scratch + (bh * 2 + dir) * 2 * DD + DD;
+  const float* S_out = S + fo;
+  const float* S_in = dir == 0 ? (f == 0 ? seed : S + fo - DD) : (f == F - 1 ? seed : S + fo + DD);
+  const float* lam = lam_all + go;
+  const float* dX = dX_all + go;
+  float* dA = dA2 + go;
+  float* dB = dB2 + go;
+  if (rc.solve) {
+    cta_mm<D>(dA, S_out, true, dX, false, -rc.c2, slab);
+  } else if (rc.c2 != 0.f) {
+    float* X = Xbuf + go;
+    for (long long e = tid; e < DD; e += kBT) {
+      const int jj = (int)(e % D);
+      X[e] = S_in[e] * alpha[((b * F + f) * H + h) * D + jj] + rc.cpre * Bm[fo + e];
+    }
+    __syncthreads();
+    cta_mm<D>(dA, X, true, lam, false, -rc.c2, slab);
+  } else {
+    for (long long e = tid; e < DD; e += kBT) dA[e] = 0.f;
+  }
+  for (long long e = tid; e < DD; e += kBT) dB[e] = rc.cpre * dX[e] + rc.cpost * lam[e];
+  if (tid < D) {
+    float acc = 0.f;
+    for (int i = 0; i < D; ++i) acc = fmaf(S_in[i * D + tid], dX[i * D + tid], acc);
+    dalpha2[((long long)dir * NFt + fi) * D + tid] = acc;
+  }
 }
 
 // ---------------------------------------------------------------- step 2 reversed (+ step 1 up to the conv)
@@ -767,7 +797,10 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule) {
   p.dalpha_g = take(NF * sh.d * 4);
   p.dalpha2 = take(2 * NF * sh.d * 4);
   p.dseed2 = take(2 * BH * DD * 4);
-  p.scan_scratch = take(BH * 2 * 4 * DD * 4);
+  p.scan_scratch = take(BH * 2 * 2 * DD * 4);
+  p.lam_all = take(2 * NF * DD * 4);
+  p.dX_all = take(2 * NF * DD * 4);
+  p.Xbuf = rule == VDN_RULE_SANA_SCALED ? take(2 * NF * DD * 4) : 0;
   p.rms_part = take(NF * sh.d * 4);
   p.dkc = take(tokens * sh.d * 4);
   p.dvc = take(tokens * sh.d * 4);
@@ -812,9 +845,12 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
       a.radius);
   if ((e = mark()) != cudaSuccess) return e;
   // steps 3-4 (scans) reversed
-  k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(
-      at(p.Bm), at(p.Nm), at(p.P), at(p.Q), a.alpha, a.text_state, rule_coef(a.rule, a.c), at(p.dPin), at(p.dQin),
-      at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(at(p.Nm), a.alpha, a.text_state, at(p.dPin),
+                                                               at(p.dQin), at(p.lam_all), at(p.dX_all),
+                                                               at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  k_bwd_scan_grads<D><<<dim3((unsigned)NF, 2), kBT, 0, a.stream>>>(
+      at(p.Bm), at(p.P), at(p.Q), a.alpha, rule_coef(a.rule, a.c), at(p.lam_all), at(p.dX_all), at(p.scan_scratch),
+      at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.Xbuf), sh.H, sh.F);
   if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed
   if (kTc) {

@@ -76,7 +76,9 @@ struct BwdPlan {
   size_t dA2 = 0, dB2 = 0;                             // fp32 [2][B, H, F, d, d] (prefix, suffix scan)
   size_t dalpha_g = 0, dalpha2 = 0;                    // fp32 [B, H, F, d], [2][B, H, F, d]
   size_t dseed2 = 0;                                   // fp32 [2][B, H, d, d]
-  size_t scan_scratch = 0;                             // fp32 [B, H, 2][4][d, d]
+  size_t scan_scratch = 0;                             // fp32 [B, H, 2][2][d, d] (running adjoint, seed)
+  size_t lam_all = 0, dX_all = 0;                      // fp32 [2][B, H, F, d, d]: adjoint and dX per step
+  size_t Xbuf = 0;                                     // fp32 [2][B, H, F, d, d] (sana_scaled only)
   size_t rms_part = 0;                                 // fp32 [B, H, F][d]
   size_t dkc = 0, dvc = 0;                             // fp32 [B, N, H, d]
   size_t tap_part = 0;                                 // fp32 [H][kBwdConvBlocks][2][d][3]
