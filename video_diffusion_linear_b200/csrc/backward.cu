@@ -610,29 +610,47 @@ template <> __device__ __forceinline__ void store8t<__nv_bfloat16>(__nv_bfloat16
       make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
-// Thread = (token, group of 8 channels), grid-stride over the tokens of head h = blockIdx.y:
+template <typename T> __device__ __forceinline__ void load4t(const T* p, float* v);
+template <> __device__ __forceinline__ void load4t<float>(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <> __device__ __forceinline__ void load4t<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+}
+template <typename T> __device__ __forceinline__ void store4t(T* p, const float* v);
+template <> __device__ __forceinline__ void store4t<float>(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <> __device__ __forceinline__ void store4t<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
+// Thread = (token, group of 4 channels), grid-stride over the tokens of head h = blockIdx.y:
 // dk[s] = sum_j w[j] dkc[s - j + p] over in-frame indices (out[s'] reads x[s' + j - p]), and the
 // tap partials sum_s dkc[s] k[s + j - p], reduced per block.  A missing conv is the identity
 // (centre tap 1); KT is the tap count of the staged convs.
 template <int D, typename T, int KT>
-__global__ void __launch_bounds__(kBT) k_bwd_conv(const T* __restrict__ k, const T* __restrict__ v,
+__global__ void __launch_bounds__(kBT, 2) k_bwd_conv(const T* __restrict__ k, const T* __restrict__ v,
                                                   const float* __restrict__ wk, const float* __restrict__ wv,
                                                   const float* __restrict__ dkc, const float* __restrict__ dvc,
                                                   T* __restrict__ dk, T* __restrict__ dv,
                                                   float* __restrict__ tap_part, int B, int H, int F, int S) {
-  constexpr int G = D / 8;                 // channel groups
+  constexpr int CW = 4;                    // channels per thread
+  constexpr int G = D / CW;                // channel groups
   constexpr int TPI = kBT / G;             // tokens per block and iteration
   constexpr int PAD = (KT - 1) / 2;
-  __shared__ float red[kBT / 32][G][2][KT][8];
+  __shared__ float red[kBT / 32][G][2][KT][CW];
   const int h = blockIdx.y;
   const int tid = threadIdx.x, cg = tid % G, tl = tid / G, warp = tid >> 5, lane = tid & 31;
-  const int c0 = 8 * cg;
+  const int c0 = CW * cg;
   const long long N = (long long)F * S, total = (long long)B * N;
-  float wkr[KT][8], wvr[KT][8], tk[KT][8], tv[KT][8];
+  float wkr[KT][CW], wvr[KT][CW], tk[KT][CW], tv[KT][CW];
 #pragma unroll
   for (int j = 0; j < KT; ++j)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < CW; ++e) {
       wkr[j][e] = wk ? wk[((long long)h * D + c0 + e) * KT + j] : (j == PAD ? 1.f : 0.f);
       wvr[j][e] = wv ? wv[((long long)h * D + c0 + e) * KT + j] : (j == PAD ? 1.f : 0.f);
       tk[j][e] = tv[j][e] = 0.f;
@@ -641,54 +659,54 @@ __global__ void __launch_bounds__(kBT) k_bwd_conv(const T* __restrict__ k, const
     const long long b = tokn / N, n = tokn % N;
     const int s = (int)(n % S);
     const long long row = (b * N + n) * H + h;     // token row (times D)
-    float ck[8], cv[8], gk[8], gv[8];
-    load8t(dkc + row * D + c0, ck);
-    load8t(dvc + row * D + c0, cv);
+    float ck[CW], cv[CW], gk[CW], gv[CW];
+    load4t(dkc + row * D + c0, ck);
+    load4t(dvc + row * D + c0, cv);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) gk[e] = gv[e] = 0.f;
+    for (int e = 0; e < CW; ++e) gk[e] = gv[e] = 0.f;
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
       const int so = s - j + PAD;                  // out[so] reads x[s] through tap j
       if (so >= 0 && so < S) {
-        float a[8], c[8];
+        float a[CW], c[CW];
         if (so == s) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < CW; ++e) {
             a[e] = ck[e];
             c[e] = cv[e];
           }
         } else {
-          load8t(dkc + (row + (long long)(so - s) * H) * D + c0, a);
-          load8t(dvc + (row + (long long)(so - s) * H) * D + c0, c);
+          load4t(dkc + (row + (long long)(so - s) * H) * D + c0, a);
+          load4t(dvc + (row + (long long)(so - s) * H) * D + c0, c);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < CW; ++e) {
           gk[e] = fmaf(wkr[j][e], a[e], gk[e]);
           gv[e] = fmaf(wvr[j][e], c[e], gv[e]);
         }
       }
       const int sx = s + j - PAD;                  // tap j of out[s] reads x[sx]
       if (sx >= 0 && sx < S) {
-        float x[8], y[8];
-        load8t(k + (row + (long long)(sx - s) * H) * D + c0, x);
-        load8t(v + (row + (long long)(sx - s) * H) * D + c0, y);
+        float x[CW], y[CW];
+        load4t(k + (row + (long long)(sx - s) * H) * D + c0, x);
+        load4t(v + (row + (long long)(sx - s) * H) * D + c0, y);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < CW; ++e) {
           tk[j][e] = fmaf(ck[e], x[e], tk[j][e]);
           tv[j][e] = fmaf(cv[e], y[e], tv[j][e]);
         }
       }
     }
-    store8t(dk + row * D + c0, gk);
-    store8t(dv + row * D + c0, gv);
+    store4t(dk + row * D + c0, gk);
+    store4t(dv + row * D + c0, gv);
   }
   // tap partials: lanes with the same channel group within the warp, then the block's warps
 #pragma unroll
-  for (int off = G; off < 32; off <<= 1)
+  for (int off = G; off < 32; off <<= 1)   // (no-op once a warp holds one token's groups)
 #pragma unroll
     for (int j = 0; j < KT; ++j)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < CW; ++e) {
         tk[j][e] += __shfl_xor_sync(0xffffffffu, tk[j][e], off);
         tv[j][e] += __shfl_xor_sync(0xffffffffu, tv[j][e], off);
       }
@@ -696,16 +714,16 @@ __global__ void __launch_bounds__(kBT) k_bwd_conv(const T* __restrict__ k, const
 #pragma unroll
     for (int j = 0; j < KT; ++j)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < CW; ++e) {
         red[warp][cg][0][j][e] = tk[j][e];
         red[warp][cg][1][j][e] = tv[j][e];
       }
   __syncthreads();
-  for (int idx = tid; idx < G * 2 * KT * 8; idx += kBT) {
-    const int e = idx % 8, j = (idx / 8) % KT, m = (idx / (8 * KT)) % 2, g2 = idx / (16 * KT);
+  for (int idx = tid; idx < G * 2 * KT * CW; idx += kBT) {
+    const int e = idx % CW, j = (idx / CW) % KT, m = (idx / (CW * KT)) % 2, g2 = idx / (2 * CW * KT);
     float acc = 0.f;
     for (int w = 0; w < kBT / 32; ++w) acc += red[w][g2][m][j][e];
-    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * D * 3 + (8 * g2 + e) * 3 + j] = acc;
+    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * D * 3 + (CW * g2 + e) * 3 + j] = acc;
   }
 }
 
