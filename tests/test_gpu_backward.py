@@ -90,3 +90,40 @@ def test_backward_is_deterministic():
     for n in NAMES:
         if a[n] is not None:
             assert torch.equal(a[n], b[n]), n
+
+
+BF16_RULES = [
+    synth.Workload("bw_bf16_sana", B=1, H=2, d=128, F=9, S=40, dtype="bf16", alpha_mu=2.0, text=True, seed=58,
+                   rule="sana_scaled", c=0.5, chunk=3, radius=1),
+    synth.Workload("bw_bf16_scaled", B=1, H=1, d=128, F=10, S=130, dtype="bf16", alpha_mu=2.0, text=True, seed=59,
+                   rule="vdn_scaled", c=0.7, chunk=2, radius=2),
+]
+
+
+@pytest.mark.parametrize("w", BF16_RULES, ids=[c.name for c in BF16_RULES])
+def test_bf16_gradients_other_rules(w):
+    got, ref = _run(w)
+    _compare(w, got, ref, TOL_BF16)
+
+
+def test_480p_full_size_per_head_gradients():
+    # the 480p workload at its full size, in the launch configuration the bench times; the
+    # per-head gradients of two heads against the oracle (the shared-parameter gradients sum over
+    # all heads and are covered by the smaller cases)
+    w = synth.WORKLOADS["480p"]
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w)
+    dev = api.to_device(inp)
+    shape = api.shape_from(dev["q"], w.F, dev.get("conv_k_w"))
+    ws = torch.empty(api.backward_workspace_size(shape, w.rule), dtype=torch.uint8, device="cuda")
+    got = api.branch_backward(*api.forward_inputs(dev), dout=dout.cuda(), F=w.F, rule=w.rule, c=w.c,
+                              chunk=w.chunk, radius=w.radius, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.workspace_status(ws) == 0
+    for h in (0, w.H - 1):
+        ref = BW.head_backward(inp, 0, h, w.F, w.S, w.rule, w.c, w.chunk, w.radius, dout[0, :, h, :])
+        pairs = {"dq": got["dq"][0, :, h], "dk": got["dk"][0, :, h], "dv": got["dv"][0, :, h],
+                 "dgate": got["dgate"][0, :, h], "dbeta": got["dbeta"][0, :, h], "dalpha": got["dalpha"][0, :, h]}
+        for n, g in pairs.items():
+            e = rel_err(to_np(g), ref[n])
+            assert e <= TOL_BF16, (h, n, e)

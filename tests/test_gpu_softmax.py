@@ -129,3 +129,22 @@ def test_repeated_full_size_calls_never_time_out():
             first = out
         else:
             assert torch.equal(out, first)
+
+
+EDGE = [
+    synth.Workload("sm_one_frame", B=1, H=2, d=128, F=1, S=100, dtype="bf16", alpha_mu=2.0, text=False, seed=48),
+    synth.Workload("sm_one_chunk", B=1, H=1, d=128, F=4, S=90, dtype="bf16", alpha_mu=2.0, text=False, seed=49,
+                   chunk=8, radius=1),
+    synth.Workload("sm_window_wider_than_clip", B=2, H=1, d=128, F=6, S=50, dtype="bf16", alpha_mu=2.0, text=False,
+                   seed=60, chunk=2, radius=5),
+    synth.Workload("sm_d16_one_frame", B=1, H=3, d=16, F=1, S=7, dtype="f32", alpha_mu=2.0, text=False, seed=61),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=[c.name for c in EDGE])
+def test_window_softmax_edge_cases(w):
+    inp = synth.make_inputs(w, with_rope_side=True)
+    got = _run(w, inp)
+    ref = O.window_softmax_forward(inp, w.F, w.S, w.chunk, w.radius)
+    tol = TOL_F32 if w.dtype == "f32" else TOL_BF16
+    assert rel_err(to_np(got), ref) <= tol, (w.name, rel_err(to_np(got), ref))
