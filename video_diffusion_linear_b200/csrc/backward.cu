@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan_grads(const float* __restrict_
                                                         const float* __restrict__ alpha, RuleCoef rc,
                                                         const float* __restrict__ lam_all,
                                                         const float* __restrict__ dX_all,
-                                                        const float* __restrict__ scan_scratch,
+                                                        const float* __restrict__ text_state,
                                                         float* __restrict__ dA2, float* __restrict__ dB2,
                                                         float* __restrict__ dalpha2, float* __restrict__ Xbuf, int H,
                                                         int F) {
@@ -441,9 +441,13 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan_grads(const float* __restrict_
   const long long fo = fi * DD;
   const long long go = ((long long)dir * NFt + fi) * DD;
   const float* S = dir == 0 ? P : Q;
-  const float* seed = scan_scratch + (bh * 2 + dir) * 2 * DD + DD;
   const float* S_out = S + fo;
-  const float* S_in = dir == 0 ? (f == 0 ? seed : S + fo - DD) : (f == F - 1 ? seed : S + fo + DD);
+  // S_in: the neighbouring state, or the seed 0.5 T at the clip edge (read elementwise only)
+  const bool edge = dir == 0 ? f == 0 : f == F - 1;
+  const float* S_nb = dir == 0 ? S + fo - DD : S + fo + DD;
+  auto s_in = [&](long long e) {
+    return edge ? (text_state ? 0.5f * text_state[(long long)h * DD + e] : 0.f) : S_nb[e];
+  };
   const float* lam = lam_all + go;
   const float* dX = dX_all + go;
   float* dA = dA2 + go;
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan_grads(const float* __restrict_
     float* X = Xbuf + go;
     for (long long e = tid; e < DD; e += kBT) {
       const int jj = (int)(e % D);
-      X[e] = S_in[e] * alpha[((b * F + f) * H + h) * D + jj] + rc.cpre * Bm[fo + e];
+      X[e] = s_in(e) * alpha[((b * F + f) * H + h) * D + jj] + rc.cpre * Bm[fo + e];
     }
     __syncthreads();
     cta_mm<D>(dA, X, true, lam, false, -rc.c2, slab);
@@ -464,7 +468,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_scan_grads(const float* __restrict_
   for (long long e = tid; e < DD; e += kBT) dB[e] = rc.cpre * dX[e] + rc.cpost * lam[e];
   if (tid < D) {
     float acc = 0.f;
-    for (int i = 0; i < D; ++i) acc = fmaf(S_in[i * D + tid], dX[i * D + tid], acc);
+    for (int i = 0; i < D; ++i) acc = fmaf(s_in((long long)i * D + tid), dX[i * D + tid], acc);
     dalpha2[((long long)dir * NFt + fi) * D + tid] = acc;
   }
 }
@@ -863,11 +867,20 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
       a.radius);
   if ((e = mark()) != cudaSuccess) return e;
   // steps 3-4 (scans) reversed
-  k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(at(p.Nm), a.alpha, a.text_state, at(p.dPin),
-                                                               at(p.dQin), at(p.lam_all), at(p.dX_all),
-                                                               at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  if (kTc) {
+    // the forward's hi/lo operand images of N_f (tensor-core path) serve the adjoint products
+    const WsPlan fp = plan_workspace(sh, a.rule, true);
+    const uint16_t* nimg = reinterpret_cast<const uint16_t*>(static_cast<char*>(ws) + p.fwd + fp.nimg);
+    if ((e = launch_bwd_scan_tc(a, nimg, at(p.dPin), at(p.dQin), at(p.lam_all), at(p.dX_all), at(p.dseed2),
+                                status)) != cudaSuccess)
+      return e;
+  } else {
+    k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(at(p.Nm), a.alpha, a.text_state, at(p.dPin),
+                                                                 at(p.dQin), at(p.lam_all), at(p.dX_all),
+                                                                 at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
+  }
   k_bwd_scan_grads<D><<<dim3((unsigned)NF, 2), kBT, 0, a.stream>>>(
-      at(p.Bm), at(p.P), at(p.Q), a.alpha, rule_coef(a.rule, a.c), at(p.lam_all), at(p.dX_all), at(p.scan_scratch),
+      at(p.Bm), at(p.P), at(p.Q), a.alpha, rule_coef(a.rule, a.c), at(p.lam_all), at(p.dX_all), a.text_state,
       at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.Xbuf), sh.H, sh.F);
   if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed

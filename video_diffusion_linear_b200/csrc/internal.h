@@ -103,6 +103,8 @@ cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* 
                                   void* dq, void* dgate, uint32_t* status);
 cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, float* dkc, float* dvc,
                                 float* dbeta, uint32_t* status);
+cudaError_t launch_bwd_scan_tc(const Args& a, const uint16_t* nimg, const float* dPin, const float* dQin,
+                               float* lam_all, float* dX_all, float* dseed2, uint32_t* status);
 cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events);
 
 // standalone step 1 (dtype in, dtype out)

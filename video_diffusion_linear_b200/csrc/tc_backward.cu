@@ -592,6 +592,175 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
   }
 }
 
+// ---------------------------------------------------------------- Steps 3-4 reversed: the adjoint scans
+// One CTA per (batch, head, direction) walks the frames in the reverse order of absorption:
+//     lam_f = lam + g_f                      (g_f: the bridge's gradient of the state after frame f)
+//     dX_f = lam_f N_f^T = lam_f N_f         (N_f symmetric for every rule; tcgen05, bf16 hi/lo)
+//     lam  = dX_f D_f
+// storing lam_f and dX_f for the batched kernel that forms dA, dB, d alpha.  The product splits
+// lam into bf16 hi + lo and uses the forward's hi/lo image of N_f (three MMAs per K step, about 16
+// significant bits per term, fp32 accumulation), as the forward scan does.
+struct __align__(1024) BwdScanSmem {
+  uint8_t aop[2][32768];     // lam hi, lam lo: K-major SW128 A operands
+  uint8_t nimg[65536];       // N_f hi | lo image
+  float alpha[128];
+  uint64_t bar_n, bar_mma, bar_nhi;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr int kBwdScanThreads = 256;   // two threads per state row (column halves)
+
+__device__ __forceinline__ void split_pair_bf16(float2 x, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(x.x, x.y);
+  lo = pack_bf16x2(x.x - bf16lo(hi), x.y - bf16hi(hi));
+}
+
+__global__ void __launch_bounds__(kBwdScanThreads, 1) k_bwd_scan_tc(const uint16_t* __restrict__ nimg_g,
+                                                                    const float* __restrict__ alpha,
+                                                                    const float* __restrict__ dPin,
+                                                                    const float* __restrict__ dQin,
+                                                                    float* __restrict__ lam_all,
+                                                                    float* __restrict__ dX_all,
+                                                                    float* __restrict__ dseed2, int H, int F,
+                                                                    uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdScanSmem& sm = *reinterpret_cast<BwdScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m = 32 * (warp & 3) + lane;     // state row = TMEM lane
+  const int k0 = 64 * (tid >> 7);           // column half
+  const int dir = blockIdx.y;
+  const long long bh = blockIdx.x;
+  const long long BH = gridDim.x;
+  const int h = (int)(bh % H);
+  const long long b = bh / H;
+  const long long DD = 128 * 128;
+  volatile int* abort_flag = &sm.abort;
+  if (tid == 0) {
+    tc::mbar_init(&sm.bar_n, 1);
+    tc::mbar_init(&sm.bar_mma, 1);
+    tc::mbar_init(&sm.bar_nhi, 1);
+    sm.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&sm.tmem_base, 128);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + k0;
+  const float* din = (dir == 0 ? dPin : dQin) + bh * (F + 1) * DD;
+  auto frame_of = [&](int step) { return dir == 0 ? F - 1 - step : step; };
+  auto load_n_part = [&](int step, int part) {
+    const long long fi = bh * F + frame_of(step);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2)) + part * 32768;
+    if (part == 0) tc::mbar_arrive_expect_tx(&sm.bar_n, kImgBytes);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) tc::bulk_load(sm.nimg + part * 32768 + j * 16384, src + j * 16384, 16384, &sm.bar_n);
+  };
+  if (tid == 0) {
+    load_n_part(0, 0);
+    load_n_part(0, 1);
+  }
+  float2 s[32];   // the running adjoint, row m, columns k0 .. k0 + 63
+#pragma unroll
+  for (int p = 0; p < 32; ++p) s[p] = make_float2(0.f, 0.f);
+  const uint32_t a_hi = tc::smem_u32(sm.aop[0]), a_lo = tc::smem_u32(sm.aop[1]);
+  const uint32_t n_hi = tc::smem_u32(sm.nimg), n_lo = n_hi + 32768;
+  uint32_t ph = 0;
+  for (int step = 0; step < F; ++step) {
+    const int f = frame_of(step);
+    const long long fi = bh * F + f;
+    const long long go = ((long long)dir * BH * F + fi) * DD + (long long)m * 128 + k0;
+    if (tid < 128) sm.alpha[tid] = alpha[((b * F + f) * H + h) * 128 + tid];
+    // lam_f = lam + g_f: stored, and split into the A operands
+    const float* g = din + (long long)(dir == 0 ? f + 1 : f) * DD + (long long)m * 128 + k0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 g0 = *reinterpret_cast<const float4*>(g + 8 * c);
+      const float4 g1 = *reinterpret_cast<const float4*>(g + 8 * c + 4);
+      s[4 * c + 0] = make_float2(s[4 * c + 0].x + g0.x, s[4 * c + 0].y + g0.y);
+      s[4 * c + 1] = make_float2(s[4 * c + 1].x + g0.z, s[4 * c + 1].y + g0.w);
+      s[4 * c + 2] = make_float2(s[4 * c + 2].x + g1.x, s[4 * c + 2].y + g1.y);
+      s[4 * c + 3] = make_float2(s[4 * c + 3].x + g1.z, s[4 * c + 3].y + g1.w);
+      *reinterpret_cast<float4*>(lam_all + go + 8 * c) = make_float4(s[4 * c].x, s[4 * c].y, s[4 * c + 1].x, s[4 * c + 1].y);
+      *reinterpret_cast<float4*>(lam_all + go + 8 * c + 4) =
+          make_float4(s[4 * c + 2].x, s[4 * c + 2].y, s[4 * c + 3].x, s[4 * c + 3].y);
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) split_pair_bf16(s[4 * c + q], hw[q], lw[q]);
+      const uint32_t off = img_offset(0, m, k0 + 8 * c);
+      *reinterpret_cast<uint4*>(sm.aop[0] + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm.aop[1] + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (tid == 0) {
+      if (tc::mbar_wait(&sm.bar_n, ph, abort_flag, status)) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024);
+          tc::umma_bf16(tmem, tc::smem_desc(a_hi + koff, 16, 1024), bhd, kIdKK, kk > 0 ? 1u : 0u);
+          tc::umma_bf16(tmem, tc::smem_desc(a_lo + koff, 16, 1024), bhd, kIdKK, 1u);
+        }
+        tc::umma_commit(&sm.bar_nhi);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::umma_bf16(tmem, tc::smem_desc(a_hi + koff, 16, 1024), tc::smem_desc(n_lo + koff, 16, 1024), kIdKK, 1u);
+        }
+        tc::umma_commit(&sm.bar_mma);
+        if (step + 1 < F && tc::mbar_wait(&sm.bar_nhi, ph, abort_flag, status)) load_n_part(step + 1, 0);
+      }
+    }
+    if (!tc::mbar_wait(&sm.bar_mma, ph, abort_flag, status)) break;
+    tc::tc_fence_after();
+    if (tid == 0 && step + 1 < F) load_n_part(step + 1, 1);   // the product that read N_lo is complete
+    // dX_f: stored; the next adjoint is dX_f D_f
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      uint32_t r[32];
+      tc::tmem_ld32(t_row + 32 * j, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const int p = 16 * j + e / 2;
+        const int kc = k0 + 32 * j + e;
+        const float4 dx = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                      __uint_as_float(r[e + 3]));
+        *reinterpret_cast<float4*>(dX_all + go + 32 * j + e) = dx;
+        const float4 al = *reinterpret_cast<const float4*>(&sm.alpha[kc]);
+        s[p] = make_float2(dx.x * al.x, dx.y * al.y);
+        s[p + 1] = make_float2(dx.z * al.z, dx.w * al.w);
+      }
+    }
+    tc::tc_fence_before();
+    __syncthreads();            // accumulator read, alpha slot and A operands free
+    ph ^= 1;
+  }
+  // the gradient of the seed: the final adjoint plus the bridge's direct use of the seed
+  {
+    const float* g0 = din + (long long)(dir == 0 ? 0 : F) * DD + (long long)m * 128 + k0;
+    float* ds = dseed2 + ((long long)dir * BH + bh) * DD + (long long)m * 128 + k0;
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      const float2 gg = *reinterpret_cast<const float2*>(g0 + 2 * p);
+      *reinterpret_cast<float2*>(ds + 2 * p) = make_float2(s[p].x + gg.x, s[p].y + gg.y);
+    }
+  }
+  // teardown: make sure no copy or product of ours is still in flight
+  __syncthreads();
+  if (sm.abort && tid == 0) tc::mbar_wait(&sm.bar_n, ph, abort_flag, nullptr);
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
@@ -614,6 +783,16 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
   k_bwd_stats_tc<<<(unsigned)a.NF(), kStatsThreads, smem, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
       a.conv_v_w, K, dA2, dB2, dkc, dvc, dbeta, a.sh.H, a.sh.F, a.sh.S, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_scan_tc(const Args& a, const uint16_t* nimg, const float* dPin, const float* dQin,
+                               float* lam_all, float* dX_all, float* dseed2, uint32_t* status) {
+  const size_t smem = sizeof(BwdScanSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_bwd_scan_tc<<<dim3((unsigned)((long long)a.sh.B * a.sh.H), 2), kBwdScanThreads, smem, a.stream>>>(
+      nimg, a.alpha, dPin, dQin, lam_all, dX_all, dseed2, a.sh.H, a.sh.F, status);
   return cudaGetLastError();
 }
 
