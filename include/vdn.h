@@ -266,7 +266,9 @@ size_t vdn_branch_backward_workspace_size(const vdn_shape* shape, int rule);
  *   dtext_state         [H, d, d]      fp32 (summed over the batch); NULL exactly
  *                       when text_state is NULL
  * The forward runs first, inside the call (its per-frame statistics, operators and
- * states are kept in the workspace); then fp32 kernels for d = 16 and 128.  No
+ * states are kept in the workspace); then the reversed steps: on the tensor cores
+ * for bf16 at d = 128 (read-out, frame statistics and the adjoint scans; fp32
+ * accumulation), in fp32 SIMT kernels otherwise (fp32 inputs, d = 16).  No
  * output may overlap another output, an input or the workspace.  Rules whose
  * states leave the fp32 range (divergent sana_scaled settings) give non-finite
  * gradients.  Errors: as vdn_branch_forward, plus VDN_ERR_INVALID_ARG for a
