@@ -289,6 +289,41 @@ vdn_status vdn_branch_backward(const vdn_shape* shape,
                                float* dconv_k_w, float* dconv_v_w, float* dtext_state,
                                void* stream);
 
+/* Save-for-backward (a training step: forward, then backward from the forward's state).
+ * vdn_branch_forward_train is vdn_branch_forward (same output) that also keeps, in the
+ * caller's `saved` buffer of vdn_branch_saved_size() bytes (256-byte aligned), the per-frame
+ * state the backward reads: A_f, B_f, N_f, P_f, Q_f, W_t in fp32 and, on the tensor-core
+ * path, the operand images of N_f.  vdn_branch_backward_saved is vdn_branch_backward without
+ * the forward recompute: same inputs (which must be those the saved state was made from),
+ * the saved buffer (read only), a workspace of vdn_branch_backward_saved_workspace_size()
+ * bytes whose first word is its device status word.  Errors as vdn_branch_forward and
+ * vdn_branch_backward, plus VDN_ERR_WORKSPACE for a short saved buffer and
+ * VDN_ERR_INVALID_ARG when it overlaps an input, an output or the workspace. */
+size_t vdn_branch_saved_size(const vdn_shape* shape);
+size_t vdn_branch_backward_saved_workspace_size(const vdn_shape* shape, int rule);
+vdn_status vdn_branch_forward_train(const vdn_shape* shape,
+                                    const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha,
+                                    const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w,
+                                    const float* text_state,
+                                    int rule, float c, int chunk, int radius,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* out, void* saved, size_t saved_bytes, void* stream);
+vdn_status vdn_branch_backward_saved(const vdn_shape* shape,
+                                     const void* q, const void* k, const void* v,
+                                     const float* beta, const float* alpha,
+                                     const void* gate, const float* rms_w,
+                                     const float* conv_k_w, const float* conv_v_w,
+                                     const float* text_state,
+                                     int rule, float c, int chunk, int radius,
+                                     const void* dout, const void* saved, size_t saved_bytes,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* dq, void* dk, void* dv,
+                                     float* dbeta, float* dalpha, void* dgate, float* drms_w,
+                                     float* dconv_k_w, float* dconv_v_w, float* dtext_state,
+                                     void* stream);
+
 /* vdn_branch_backward that also records caller-created CUDA events on `stream`:
  * events[0] before the forward recompute, events[1] after it, then events[2..7]
  * after each backward kernel (read-out, gather and bridge, adjoint scans, frame

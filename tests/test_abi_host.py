@@ -150,3 +150,46 @@ def test_backward_validation_rejects_before_launch(lib, case, expect):
     s = _shape(**case.get("shape", {}))
     args = _bwd_args(s, case.get("ws_bytes", 1 << 40), **case.get("ptr", {}))
     assert lib.vdn_branch_backward(*args) == expect
+
+
+def test_saved_state_sizes(lib):
+    s = _shape()
+    n = lib.vdn_branch_saved_size(ctypes.byref(s))
+    assert n > 0 and n % 256 == 0
+    w_saved = lib.vdn_branch_backward_saved_workspace_size(ctypes.byref(s), 1)
+    assert 0 < w_saved < lib.vdn_branch_backward_workspace_size(ctypes.byref(s), 1)
+    assert lib.vdn_branch_saved_size(ctypes.byref(_shape(d=64))) == 0
+
+
+def _saved_args(shape, saved=BASE + 30 * GAP, saved_bytes=1 << 40, ws=BASE + 11 * GAP):
+    args = list(_bwd_args(shape))
+    # vdn_branch_backward_saved: ..., dout, saved, saved_bytes, workspace, workspace_bytes, gradients..., stream
+    head, tail = args[:16], args[16:]
+    tail[0] = ctypes.c_void_p(ws)
+    return head + [None if saved is None else ctypes.c_void_p(saved), saved_bytes] + tail
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(saved=None), VDN_ERR_INVALID_ARG),
+    (dict(saved_bytes=1024), VDN_ERR_WORKSPACE),
+    (dict(saved=BASE + 30 * GAP + 16), VDN_ERR_ALIGNMENT),
+    (dict(saved=BASE + 11 * GAP + 4096), VDN_ERR_INVALID_ARG),        # saved state overlaps the workspace
+    (dict(saved=BASE + 12 * GAP), VDN_ERR_INVALID_ARG),               # saved state overlaps dq
+])
+def test_backward_saved_validation(lib, case, expect):
+    s = _shape()
+    assert lib.vdn_branch_backward_saved(*_saved_args(s, **case)) == expect
+
+
+def test_forward_train_validation(lib):
+    s = _shape()
+    base = list(_args(s, 1 << 40))
+    # vdn_branch_forward_train: forward arguments up to out, then saved, saved_bytes, stream
+    def call(saved, nbytes):
+        return lib.vdn_branch_forward_train(*base[:-1], None if saved is None else ctypes.c_void_p(saved), nbytes,
+                                            None)
+    assert call(None, 1 << 40) == VDN_ERR_INVALID_ARG
+    assert call(BASE + 30 * GAP, 1024) == VDN_ERR_WORKSPACE
+    assert call(BASE + 30 * GAP + 64, 1 << 40) == VDN_ERR_ALIGNMENT
+    assert call(BASE + 11 * GAP, 1 << 40) == VDN_ERR_INVALID_ARG       # overlaps the output
+    assert call(BASE + 10 * GAP, 1 << 40) == VDN_ERR_INVALID_ARG       # overlaps the workspace

@@ -127,3 +127,26 @@ def test_480p_full_size_per_head_gradients():
         for n, g in pairs.items():
             e = rel_err(to_np(g), ref[n])
             assert e <= TOL_BF16, (h, n, e)
+
+
+@pytest.mark.parametrize("w", [CASES[0], CASES[5], BF16[0]], ids=["d16_f32", "d128_f32", "d128_bf16"])
+def test_save_for_backward_matches_the_recomputing_pair(w):
+    # vdn_branch_forward_train gives the forward's output, and vdn_branch_backward_saved from its saved
+    # state gives the recomputing backward's gradients: bit for bit (same kernels, same state)
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w).cuda()
+    dev = api.to_device(inp)
+    args = api.forward_inputs(dev)
+    kw = dict(F=w.F, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius)
+    ref_out = api.branch_forward(*args, **kw)
+    out, saved = api.branch_forward_train(*args, **kw)
+    ref = api.branch_backward(*args, dout=dout, **kw)
+    shape = api.shape_from(dev["q"], w.F, dev.get("conv_k_w"))
+    ws = torch.empty(api.backward_workspace_size(shape, w.rule, saved=True), dtype=torch.uint8, device="cuda")
+    got = api.branch_backward(*args, dout=dout, saved=saved, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    assert api.workspace_status(ws) == 0
+    assert torch.equal(out, ref_out)
+    for n in NAMES:
+        if ref[n] is not None:
+            assert torch.equal(got[n], ref[n]), n

@@ -63,6 +63,13 @@ _SIGNATURES = {
                                                  _P, ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P,
                                                  _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                  ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+    "vdn_branch_saved_size": (ctypes.c_size_t, [ctypes.POINTER(VdnShape)]),
+    "vdn_branch_backward_saved_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(VdnShape), ctypes.c_int]),
+    "vdn_branch_forward_train": (ctypes.c_int, _FORWARD_ARGS[:-2] + [_P, _P, ctypes.c_size_t, _P]),
+    "vdn_branch_backward_saved": (ctypes.c_int, [ctypes.POINTER(VdnShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                 ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P, _P,
+                                                 ctypes.c_size_t, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P,
+                                                 _P, _P, _P, _P]),
     "vdn_workspace_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "vdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }

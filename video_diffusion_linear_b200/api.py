@@ -181,7 +181,38 @@ def to_device(inp: dict, device="cuda") -> dict:
     return {k: (None if t is None else t.to(device)) for k, t in inp.items()}
 
 
-def backward_workspace_size(shape: VdnShape, rule="vdn_solve") -> int:
+def saved_size(shape: VdnShape) -> int:
+    n = _lib.load().vdn_branch_saved_size(ctypes.byref(shape))
+    if n == 0:
+        raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_branch_saved_size")
+    return n
+
+
+def branch_forward_train(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *,
+                         F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, out=None, saved=None, workspace=None,
+                         stream=None):
+    """vdn_branch_forward_train: the branch's output and the per-frame state its backward
+    reads.  Returns (out, saved); pass `saved` to branch_backward(..., saved=saved)."""
+    shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    if out is None:
+        out = torch.empty_like(q)
+    if saved is None:
+        saved = torch.empty(saved_size(shape), dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, rule, "auto", q.device)
+    fa = _forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                       radius, workspace, out, stream)
+    st = _lib.load().vdn_branch_forward_train(*fa[:-1], _ptr(saved), saved.numel(), fa[-1])
+    check(st, "vdn_branch_forward_train")
+    return out, saved
+
+
+def backward_workspace_size(shape: VdnShape, rule="vdn_solve", saved=False) -> int:
+    if saved:
+        n = _lib.load().vdn_branch_backward_saved_workspace_size(ctypes.byref(shape), VDN_RULE[rule])
+        if n == 0:
+            raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_branch_backward_saved_workspace_size")
+        return n
     n = _lib.load().vdn_branch_backward_workspace_size(ctypes.byref(shape), VDN_RULE[rule])
     if n == 0:
         raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_branch_backward_workspace_size")
@@ -190,12 +221,13 @@ def backward_workspace_size(shape: VdnShape, rule="vdn_solve") -> int:
 
 def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=None, text_state=None, *, dout,
                     F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, grads=None, workspace=None, stream=None,
-                    events=None):
+                    events=None, saved=None):
     """vdn_branch_backward: gradients of <dout, branch_forward(...)> with respect to every
     input.  Returns a dict dq, dk, dv, dgate (q's dtype), dbeta, dalpha, drms_w, and
     dconv_k_w, dconv_v_w, dtext_state (fp32; None where the input is None).  With
     `events` (8 torch.cuda.Event), vdn_branch_backward_timed records them between the
-    forward recompute and each backward kernel."""
+    forward recompute and each backward kernel.  With `saved` (from branch_forward_train),
+    vdn_branch_backward_saved runs instead, without the forward recompute."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
     dev = q.device
     if grads is None:
@@ -207,14 +239,19 @@ def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=N
                  "dconv_v_w": None if conv_v_w is None else torch.empty(conv_v_w.shape, **f32),
                  "dtext_state": None if text_state is None else torch.empty(text_state.shape, **f32)}
     if workspace is None:
-        workspace = torch.empty(backward_workspace_size(shape, rule), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(backward_workspace_size(shape, rule, saved is not None), dtype=torch.uint8,
+                                device=dev)
     g = grads
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
             _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
             _ptr(dout), _ptr(workspace), workspace.numel(), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
             _ptr(g["dbeta"]), _ptr(g["dalpha"]), _ptr(g["dgate"]), _ptr(g["drms_w"]), _ptr(g["dconv_k_w"]),
             _ptr(g["dconv_v_w"]), _ptr(g["dtext_state"]), _stream_ptr(stream))
-    if events is None:
+    if saved is not None:
+        if events is not None:
+            raise ValueError("events are recorded by the recomputing backward only")
+        st = _lib.load().vdn_branch_backward_saved(*args[:16], _ptr(saved), saved.numel(), *args[16:])
+    elif events is None:
         st = _lib.load().vdn_branch_backward(*args)
     else:
         arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])

@@ -20,6 +20,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "image.cuh"
 #include "internal.h"
 
 namespace vdn {
@@ -790,7 +791,27 @@ __global__ void __launch_bounds__(kBT) k_bwd_finish(const float* __restrict__ rm
 }  // namespace
 
 // ---------------------------------------------------------------- host side
-BwdPlan plan_backward(const vdn_shape& sh, int rule) {
+SavedPlan plan_saved(const vdn_shape& sh) {
+  SavedPlan p;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const long long NF = (long long)sh.B * sh.H * sh.F, DD = (long long)sh.d * sh.d;
+  p.A = take(NF * DD * 4);
+  p.Bm = take(NF * DD * 4);
+  p.Nm = take(NF * DD * 4);
+  p.P = take(NF * DD * 4);
+  p.Q = take(NF * DD * 4);
+  p.W = take(NF * DD * 4);
+  p.nimg = use_tc(sh, VDN_IMPL_AUTO) ? take(NF * (size_t)kImgBytes) : 0;
+  p.total = off;
+  return p;
+}
+
+BwdPlan plan_backward(const vdn_shape& sh, int rule, bool recompute) {
   BwdPlan p;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -803,14 +824,18 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule) {
   const long long BH = (long long)sh.B * sh.H, NF = BH * sh.F, DD = (long long)sh.d * sh.d;
   const long long tokens = (long long)sh.B * sh.F * sh.S * sh.H;
   const size_t el = sh.dtype == VDN_DTYPE_BF16 ? 2 : 4;
-  p.fwd = take(fwd);
-  p.out = take(tokens * sh.d * el);
-  p.A = take(NF * DD * 4);
-  p.Bm = take(NF * DD * 4);
-  p.Nm = take(NF * DD * 4);
-  p.P = take(NF * DD * 4);
-  p.Q = take(NF * DD * 4);
-  p.W = take(NF * DD * 4);
+  if (recompute) {
+    p.fwd = take(fwd);                 // its first bytes hold the forward's status word
+    p.out = take(tokens * sh.d * el);
+    p.A = take(NF * DD * 4);
+    p.Bm = take(NF * DD * 4);
+    p.Nm = take(NF * DD * 4);
+    p.P = take(NF * DD * 4);
+    p.Q = take(NF * DD * 4);
+    p.W = take(NF * DD * 4);
+  } else {
+    p.status = take(256);
+  }
   p.dW = take(NF * DD * 4);
   p.dPin = take(BH * (sh.F + 1) * DD * 4);
   p.dQin = take(BH * (sh.F + 1) * DD * 4);
@@ -833,8 +858,8 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule) {
 }
 
 template <int D, typename T>
-static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p,
-                                  void* const* events) {
+static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, const BwdState& st, void* ws,
+                                  const BwdPlan& p, void* const* events) {
   int ev = 2;   // events[0], events[1]: before and after the forward recompute
   auto mark = [&]() -> cudaError_t {
     return events ? cudaEventRecord((cudaEvent_t)events[ev++], a.stream) : cudaSuccess;
@@ -846,10 +871,10 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   const int K = (a.conv_k_w || a.conv_v_w) ? sh.conv_width : 1;
   // bf16 at d = 128: the two per-token contractions on the tensor cores
   constexpr bool kTc = D == 128 && std::is_same<T, __nv_bfloat16>::value;
-  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.fwd);   // the forward's status word
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.status);   // first word of the workspace
   // step 5 reversed
   if (kTc) {
-    if ((e = launch_bwd_readout_tc(a, g.dout, at(p.W), at(p.dW), at(p.rms_part), g.dq, g.dgate, status)) !=
+    if ((e = launch_bwd_readout_tc(a, g.dout, st.W, at(p.dW), at(p.rms_part), g.dq, g.dgate, status)) !=
         cudaSuccess)
       return e;
   } else {
@@ -857,30 +882,29 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
     e = cudaFuncSetAttribute(k_bwd_readout<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k_bwd_readout<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.gate), static_cast<const T*>(g.dout), a.rms_w, at(p.W),
+        static_cast<const T*>(a.q), static_cast<const T*>(a.gate), static_cast<const T*>(g.dout), a.rms_w, st.W,
         at(p.dW), at(p.rms_part), static_cast<T*>(g.dq), static_cast<T*>(g.dgate), sh.H, sh.F, sh.S);
   }
   if ((e = mark()) != cudaSuccess) return e;
   // step 4 (gather + bridge) reversed
   k_bwd_gather<D><<<dim3((unsigned)BH, D < 32 ? 1 : D / 32), kBT, 0, a.stream>>>(
-      at(p.P), at(p.Q), a.alpha, a.text_state, at(p.dW), at(p.dPin), at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk,
+      st.P, st.Q, a.alpha, a.text_state, at(p.dW), at(p.dPin), at(p.dQin), at(p.dalpha_g), sh.H, sh.F, a.chunk,
       a.radius);
   if ((e = mark()) != cudaSuccess) return e;
   // steps 3-4 (scans) reversed
   if (kTc) {
     // the forward's hi/lo operand images of N_f (tensor-core path) serve the adjoint products
-    const WsPlan fp = plan_workspace(sh, a.rule, true);
-    const uint16_t* nimg = reinterpret_cast<const uint16_t*>(static_cast<char*>(ws) + p.fwd + fp.nimg);
+    const uint16_t* nimg = st.nimg;
     if ((e = launch_bwd_scan_tc(a, nimg, at(p.dPin), at(p.dQin), at(p.lam_all), at(p.dX_all), at(p.dseed2),
                                 status)) != cudaSuccess)
       return e;
   } else {
-    k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(at(p.Nm), a.alpha, a.text_state, at(p.dPin),
+    k_bwd_scan<D><<<dim3((unsigned)BH, 2), kBT, 0, a.stream>>>(st.Nm, a.alpha, a.text_state, at(p.dPin),
                                                                  at(p.dQin), at(p.lam_all), at(p.dX_all),
                                                                  at(p.dseed2), at(p.scan_scratch), sh.H, sh.F);
   }
   k_bwd_scan_grads<D><<<dim3((unsigned)NF, 2), kBT, 0, a.stream>>>(
-      at(p.Bm), at(p.P), at(p.Q), a.alpha, rule_coef(a.rule, a.c), at(p.lam_all), at(p.dX_all), a.text_state,
+      st.Bm, st.P, st.Q, a.alpha, rule_coef(a.rule, a.c), at(p.lam_all), at(p.dX_all), a.text_state,
       at(p.dA2), at(p.dB2), at(p.dalpha2), at(p.Xbuf), sh.H, sh.F);
   if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed
@@ -913,7 +937,8 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, void* ws, co
   return mark();
 }
 
-cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events) {
+cudaError_t run_backward(const Args& a, const BwdGrads& g, const BwdState& st, void* ws, const BwdPlan& p,
+                         void* const* events) {
   const vdn_shape& sh = a.sh;
   const long long BH = (long long)sh.B * sh.H, DD = (long long)sh.d * sh.d;
   char* base = static_cast<char*>(ws);
@@ -922,8 +947,8 @@ cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPl
   if ((e = cudaMemsetAsync(base + p.dQin, 0, BH * (sh.F + 1) * DD * 4, a.stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(base + p.dalpha_g, 0, BH * sh.F * sh.d * 4, a.stream)) != cudaSuccess) return e;
   const bool bf = sh.dtype == VDN_DTYPE_BF16;
-  if (sh.d == 16) return bf ? run_backward_t<16, __nv_bfloat16>(a, g, ws, p, events) : run_backward_t<16, float>(a, g, ws, p, events);
-  return bf ? run_backward_t<128, __nv_bfloat16>(a, g, ws, p, events) : run_backward_t<128, float>(a, g, ws, p, events);
+  if (sh.d == 16) return bf ? run_backward_t<16, __nv_bfloat16>(a, g, st, ws, p, events) : run_backward_t<16, float>(a, g, st, ws, p, events);
+  return bf ? run_backward_t<128, __nv_bfloat16>(a, g, st, ws, p, events) : run_backward_t<128, float>(a, g, st, ws, p, events);
 }
 
 }  // namespace vdn

@@ -69,7 +69,8 @@ constexpr int kBwdConvBlocks = 148;   // blocks per head of the conv-reversal ke
 // Byte offsets of the backward workspace (each 256-byte aligned): the forward's own workspace,
 // a scratch output, the forward's per-frame export and the adjoint buffers.
 struct BwdPlan {
-  size_t fwd = 0, out = 0;
+  size_t status = 0;                                   // device status word (first bytes of the workspace)
+  size_t fwd = 0, out = 0;                             // forward recompute only
   size_t A = 0, Bm = 0, Nm = 0, P = 0, Q = 0, W = 0;   // fp32 [B, H, F, d, d]
   size_t dW = 0;                                       // fp32 [B, H, F, d, d]
   size_t dPin = 0, dQin = 0;                           // fp32 [B, H, F + 1, d, d]
@@ -93,7 +94,18 @@ struct BwdGrads {
   float* dconv_k_w; float* dconv_v_w;
   float* dtext_state;
 };
-BwdPlan plan_backward(const vdn_shape& sh, int rule);
+// recompute = false: the forward's per-frame state comes from a saved buffer (no fwd, out, A .. W)
+BwdPlan plan_backward(const vdn_shape& sh, int rule, bool recompute = true);
+// The forward's per-frame state that the backward reads (fp32 [B, H, F, d, d] each, and on the
+// tensor-core path the hi/lo operand images of N_f): where vdn_branch_forward_train saves it.
+struct SavedPlan {
+  size_t A = 0, Bm = 0, Nm = 0, P = 0, Q = 0, W = 0, nimg = 0, total = 0;
+};
+SavedPlan plan_saved(const vdn_shape& sh);
+struct BwdState {
+  const float *A, *Bm, *Nm, *P, *Q, *W;
+  const uint16_t* nimg;   // tensor-core path only
+};
 // the backward kernels, after the forward has filled the plan's A .. W regions; when `events` is
 // not NULL, events[2 .. kBwdKernels + 1] are recorded after each of them (events[0] and events[1] bracket
 // the forward recompute)
@@ -105,7 +117,8 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
                                 float* dbeta, uint32_t* status);
 cudaError_t launch_bwd_scan_tc(const Args& a, const uint16_t* nimg, const float* dPin, const float* dQin,
                                float* lam_all, float* dX_all, float* dseed2, uint32_t* status);
-cudaError_t run_backward(const Args& a, const BwdGrads& g, void* ws, const BwdPlan& p, void* const* events);
+cudaError_t run_backward(const Args& a, const BwdGrads& g, const BwdState& st, void* ws, const BwdPlan& p,
+                         void* const* events);
 
 // standalone step 1 (dtype in, dtype out)
 cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,

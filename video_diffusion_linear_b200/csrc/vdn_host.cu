@@ -311,15 +311,22 @@ vdn_status backward_common(const vdn_shape* shape, const void* q, const void* k,
                            const float* conv_v_w, const float* text_state, int rule, float c, int chunk, int radius,
                            const void* dout, void* workspace, size_t workspace_bytes, void* dq, void* dk, void* dv,
                            float* dbeta, float* dalpha, void* dgate, float* drms_w, float* dconv_k_w,
-                           float* dconv_v_w, float* dtext_state, void* stream, void* const* events, int n_events) {
-  // the forward's checks, with dq standing for the output (it must not overlap an input either)
+                           float* dconv_v_w, float* dtext_state, void* stream, void* const* events, int n_events,
+                           const void* saved = nullptr, size_t saved_bytes = 0) {
+  // the forward's checks, with dq standing for the output (it must not overlap an input either);
+  // the backward's own workspace size is checked below
   if (check_shape(shape) != VDN_OK) return check_shape(shape);
+  const bool recompute = saved == nullptr;
   const BwdPlan plan = plan_backward(*shape, rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE
-                                                 ? VDN_RULE_VDN_SOLVE : rule);
+                                                 ? VDN_RULE_VDN_SOLVE : rule, recompute);
   vdn_status s = validate(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
-                          radius, workspace, workspace_bytes, dq, VDN_IMPL_AUTO);
+                          radius, workspace, SIZE_MAX, dq, VDN_IMPL_AUTO);
   if (s != VDN_OK) return s;
   if (workspace_bytes < plan.total) return VDN_ERR_WORKSPACE;
+  const SavedPlan sp = plan_saved(*shape);
+  if (!recompute && (saved_bytes < sp.total || !aligned(saved, 256))) return saved_bytes < sp.total
+                                                                              ? VDN_ERR_WORKSPACE
+                                                                              : VDN_ERR_ALIGNMENT;
   if (!dout || !dk || !dv || !dbeta || !dalpha || !dgate || !drms_w) return VDN_ERR_INVALID_ARG;
   // a gradient exists exactly for the optional inputs that were given
   if ((conv_k_w == nullptr) != (dconv_k_w == nullptr) || (conv_v_w == nullptr) != (dconv_v_w == nullptr) ||
@@ -353,6 +360,7 @@ vdn_status backward_common(const vdn_shape* shape, const void* q, const void* k,
       {(uintptr_t)conv_v_w, conv_v_w ? (uintptr_t)conv_v_w + ntap : 0},
       {(uintptr_t)text_state, text_state ? (uintptr_t)text_state + (size_t)shape->H * d * d * 4 : 0},
       {(uintptr_t)workspace, (uintptr_t)workspace + plan.total},
+      {(uintptr_t)saved, saved ? (uintptr_t)saved + sp.total : 0},
   };
   const int no = sizeof(outs) / sizeof(outs[0]), ni = sizeof(ins) / sizeof(ins[0]);
   for (int i = 0; i < no; ++i) {
@@ -362,16 +370,10 @@ vdn_status backward_common(const vdn_shape* shape, const void* q, const void* k,
     for (int j = i + 1; j < no; ++j)
       if (outs[j].hi > outs[j].lo && overlap(outs[i], outs[j])) return VDN_ERR_INVALID_ARG;
   }
-  // forward with the per-frame export into the backward workspace
   char* ws = static_cast<char*>(workspace);
-  vdn_debug_out dbg;
-  dbg.impl = VDN_IMPL_AUTO;
-  dbg.A = at<float>(ws, plan.A);
-  dbg.B = at<float>(ws, plan.Bm);
-  dbg.N = at<float>(ws, plan.Nm);
-  dbg.P = at<float>(ws, plan.P);
-  dbg.Q = at<float>(ws, plan.Q);
-  dbg.W = at<float>(ws, plan.W);
+  if (!recompute && ws + plan.total > static_cast<const char*>(saved) &&
+      static_cast<const char*>(saved) + sp.total > ws)
+    return VDN_ERR_INVALID_ARG;
   Args a;
   a.sh = *shape;
   a.q = q; a.k = k; a.v = v;
@@ -379,21 +381,43 @@ vdn_status backward_common(const vdn_shape* shape, const void* q, const void* k,
   a.conv_k_w = conv_k_w; a.conv_v_w = conv_v_w; a.text_state = text_state;
   a.rule = rule; a.c = (rule == VDN_RULE_VDN_SOLVE || rule == VDN_RULE_ADDITIVE) ? 1.0f : c;
   a.chunk = chunk; a.radius = radius;
-  a.out = ws + plan.out;
   a.stream = (cudaStream_t)stream;
-  a.dbg = &dbg;
+  a.dbg = nullptr;
   if (events) {
     if (n_events < kBwdKernels + 2) return VDN_ERR_INVALID_ARG;
     for (int i = 0; i < kBwdKernels + 2; ++i)
       if (!events[i]) return VDN_ERR_INVALID_ARG;
     if (cudaEventRecord((cudaEvent_t)events[0], a.stream) != cudaSuccess) return VDN_ERR_CUDA;
   }
-  s = run_forward(a, ws + plan.fwd, VDN_IMPL_AUTO);
-  if (s != VDN_OK) return s;
+  BwdState st;
+  if (recompute) {
+    // forward with the per-frame export into the backward workspace
+    vdn_debug_out dbg;
+    dbg.impl = VDN_IMPL_AUTO;
+    dbg.A = at<float>(ws, plan.A);
+    dbg.B = at<float>(ws, plan.Bm);
+    dbg.N = at<float>(ws, plan.Nm);
+    dbg.P = at<float>(ws, plan.P);
+    dbg.Q = at<float>(ws, plan.Q);
+    dbg.W = at<float>(ws, plan.W);
+    a.out = ws + plan.out;
+    a.dbg = &dbg;
+    s = run_forward(a, ws + plan.fwd, VDN_IMPL_AUTO);
+    if (s != VDN_OK) return s;
+    a.dbg = nullptr;
+    st = {dbg.A, dbg.B, dbg.N, dbg.P, dbg.Q, dbg.W,
+          use_tc(*shape, VDN_IMPL_AUTO)
+              ? at<uint16_t>(ws, plan.fwd + plan_workspace(*shape, rule, true).nimg) : nullptr};
+  } else {
+    if (cudaMemsetAsync(ws + plan.status, 0, sizeof(uint32_t), a.stream) != cudaSuccess) return VDN_ERR_CUDA;
+    char* sv = const_cast<char*>(static_cast<const char*>(saved));
+    st = {at<float>(sv, sp.A), at<float>(sv, sp.Bm), at<float>(sv, sp.Nm), at<float>(sv, sp.P),
+          at<float>(sv, sp.Q), at<float>(sv, sp.W), sp.nimg || use_tc(*shape, VDN_IMPL_AUTO)
+                                                         ? at<uint16_t>(sv, sp.nimg) : nullptr};
+  }
   if (events && cudaEventRecord((cudaEvent_t)events[1], a.stream) != cudaSuccess) return VDN_ERR_CUDA;
-  a.dbg = nullptr;
   BwdGrads g{dout, dq, dk, dv, dbeta, dalpha, dgate, drms_w, dconv_k_w, dconv_v_w, dtext_state};
-  if (run_backward(a, g, ws, plan, events) != cudaSuccess) return VDN_ERR_CUDA;
+  if (run_backward(a, g, st, ws, plan, events) != cudaSuccess) return VDN_ERR_CUDA;
   return VDN_OK;
 }
 }  // namespace
@@ -410,6 +434,73 @@ vdn_status vdn_branch_backward(const vdn_shape* shape, const void* q, const void
   return backward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
                          radius, dout, workspace, workspace_bytes, dq, dk, dv, dbeta, dalpha, dgate, drms_w,
                          dconv_k_w, dconv_v_w, dtext_state, stream, nullptr, 0);
+}
+
+size_t vdn_branch_saved_size(const vdn_shape* shape) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  return plan_saved(*shape).total;
+}
+
+size_t vdn_branch_backward_saved_workspace_size(const vdn_shape* shape, int rule) {
+  if (check_shape(shape) != VDN_OK) return 0;
+  if (rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE) return 0;
+  return plan_backward(*shape, rule, false).total;
+}
+
+vdn_status vdn_branch_forward_train(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                                    const float* conv_k_w, const float* conv_v_w, const float* text_state, int rule,
+                                    float c, int chunk, int radius, void* workspace, size_t workspace_bytes,
+                                    void* out, void* saved, size_t saved_bytes, void* stream) {
+  vdn_status s = check_shape(shape);
+  if (s != VDN_OK) return s;
+  if (!saved) return VDN_ERR_INVALID_ARG;
+  if (!aligned(saved, 256)) return VDN_ERR_ALIGNMENT;
+  const SavedPlan sp = plan_saved(*shape);
+  if (saved_bytes < sp.total) return VDN_ERR_WORKSPACE;
+  // the saved state must not overlap an input, the output or the workspace
+  const size_t big = (size_t)shape->B * shape->F * shape->S * shape->H * shape->d * elem_size(shape->dtype);
+  const Range rs{(uintptr_t)saved, (uintptr_t)saved + sp.total};
+  const Range others[] = {{(uintptr_t)q, (uintptr_t)q + big}, {(uintptr_t)k, (uintptr_t)k + big},
+                          {(uintptr_t)v, (uintptr_t)v + big}, {(uintptr_t)gate, (uintptr_t)gate + big},
+                          {(uintptr_t)out, (uintptr_t)out + big},
+                          {(uintptr_t)workspace, (uintptr_t)workspace + workspace_bytes}};
+  for (const Range& r : others)
+    if (r.hi > r.lo && overlap(rs, r)) return VDN_ERR_INVALID_ARG;
+  char* sv = static_cast<char*>(saved);
+  vdn_debug_out dbg;
+  dbg.impl = VDN_IMPL_AUTO;
+  dbg.A = at<float>(sv, sp.A);
+  dbg.B = at<float>(sv, sp.Bm);
+  dbg.N = at<float>(sv, sp.Nm);
+  dbg.P = at<float>(sv, sp.P);
+  dbg.Q = at<float>(sv, sp.Q);
+  dbg.W = at<float>(sv, sp.W);
+  s = forward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                     radius, workspace, workspace_bytes, out, stream, &dbg);
+  if (s != VDN_OK) return s;
+  if (sp.nimg) {
+    // the tensor-core path's operand images of N_f, which the backward's adjoint products read
+    const size_t nimg_off = plan_workspace(*shape, rule, true).nimg;
+    const size_t bytes = (size_t)shape->B * shape->H * shape->F * kImgBytes;
+    if (cudaMemcpyAsync(sv + sp.nimg, static_cast<char*>(workspace) + nimg_off, bytes, cudaMemcpyDeviceToDevice,
+                        (cudaStream_t)stream) != cudaSuccess)
+      return VDN_ERR_CUDA;
+  }
+  return VDN_OK;
+}
+
+vdn_status vdn_branch_backward_saved(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                                     const float* beta, const float* alpha, const void* gate, const float* rms_w,
+                                     const float* conv_k_w, const float* conv_v_w, const float* text_state,
+                                     int rule, float c, int chunk, int radius, const void* dout, const void* saved,
+                                     size_t saved_bytes, void* workspace, size_t workspace_bytes, void* dq,
+                                     void* dk, void* dv, float* dbeta, float* dalpha, void* dgate, float* drms_w,
+                                     float* dconv_k_w, float* dconv_v_w, float* dtext_state, void* stream) {
+  if (!saved) return VDN_ERR_INVALID_ARG;
+  return backward_common(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
+                         radius, dout, workspace, workspace_bytes, dq, dk, dv, dbeta, dalpha, dgate, drms_w,
+                         dconv_k_w, dconv_v_w, dtext_state, stream, nullptr, 0, saved, saved_bytes);
 }
 
 vdn_status vdn_branch_backward_timed(const vdn_shape* shape, const void* q, const void* k, const void* v,
