@@ -61,7 +61,8 @@ def describe(w: synth.Workload) -> str:
 
 
 def algorithmic_bytes(w: synth.Workload) -> dict:
-    """Bytes each kernel must move at least once ('roofline')."""
+    """Bytes each kernel must move at least once: the tokens it reads or writes once and the
+    per-frame matrices (fp32 statistics, operand images, states) it exchanges with its neighbours."""
     d = w.d
     TH = w.B * w.F * w.S * w.H                 # token-heads
     NF = w.B * w.H * w.F                       # (batch, head, frame) triples

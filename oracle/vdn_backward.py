@@ -1,6 +1,6 @@
 """Float64 oracle of the BACKWARD pass of the VDN-H3 bidirectional linear branch.
 
-Test infrastructure, like vdn_oracle.py: only tests/, __graft_entry__.smoke() and
+Test infrastructure, like vdn_oracle.py: only tests/, the package smoke check and
 bench.py's CPU legs use it; nothing on the product path imports it.
 
 The page ("VDN-Minimax-H3 bidirectional linear branch in five steps", section on
