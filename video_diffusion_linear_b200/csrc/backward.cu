@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats(const T* __restrict__ k, cons
                                                    const float* __restrict__ beta, const float* __restrict__ wk,
                                                    const float* __restrict__ wv, int K,
                                                    const float* __restrict__ dA2, const float* __restrict__ dB2,
-                                                   float* __restrict__ dkc, float* __restrict__ dvc,
+                                                   T* __restrict__ dkc, T* __restrict__ dvc,
                                                    float* __restrict__ dbeta, int H, int F, int S) {
   constexpr int PER = Lanes<D>::PER;
   constexpr int TPW = kTok / (kBT / 32);      // tokens per warp and tile
@@ -577,14 +577,14 @@ __global__ void __launch_bounds__(kBT) k_bwd_stats(const T* __restrict__ k, cons
         kb += 0.5f * kfc * u + vfc * z;
         dkf[r] = bt * (u + w);
         ks[r] = silu_precise(kc[tt][r]);
-        dvc[tok * D + c] = silu_grad(vc[tt][r], bt * z);
+        dvc[tok * D + c] = from_f32<T>(silu_grad(vc[tt][r], bt * z));
       }
       kb = warp_sum(kb);
       if (lane == 0) dbeta[tok] = kb;
       l2n_grad<D>(ks, dkf, dks, lane);
 #pragma unroll
       for (int r = 0; r < PER; ++r)
-        if (Lanes<D>::has(lane, r)) dkc[tok * D + lane + 32 * r] = silu_grad(kc[tt][r], dks[r]);
+        if (Lanes<D>::has(lane, r)) dkc[tok * D + lane + 32 * r] = from_f32<T>(silu_grad(kc[tt][r], dks[r]));
     }
     __syncthreads();
   }
@@ -639,7 +639,7 @@ template <> __device__ __forceinline__ void store4t<__nv_bfloat16>(__nv_bfloat16
 template <int D, typename T, int KT>
 __global__ void __launch_bounds__(kBT, 2) k_bwd_conv(const T* __restrict__ k, const T* __restrict__ v,
                                                   const float* __restrict__ wk, const float* __restrict__ wv,
-                                                  const float* __restrict__ dkc, const float* __restrict__ dvc,
+                                                  const T* __restrict__ dkc, const T* __restrict__ dvc,
                                                   T* __restrict__ dk, T* __restrict__ dv,
                                                   float* __restrict__ tap_part, int B, int H, int F, int S) {
   constexpr int CW = 4;                    // channels per thread
@@ -849,8 +849,8 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule, bool recompute) {
   p.dX_all = take(2 * NF * DD * 4);
   p.Xbuf = rule == VDN_RULE_SANA_SCALED ? take(2 * NF * DD * 4) : 0;
   p.rms_part = take(NF * sh.d * 4);
-  p.dkc = take(tokens * sh.d * 4);
-  p.dvc = take(tokens * sh.d * 4);
+  p.dkc = take(tokens * sh.d * el);          // the inputs' element type (bf16 on the tensor-core path)
+  p.dvc = take(tokens * sh.d * el);
   p.tap_part = take((size_t)sh.H * kBwdConvBlocks * 2 * sh.d * 3 * 4);
   p.fwd_bytes = fwd;
   p.total = off;
@@ -909,7 +909,8 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, const BwdSta
   if ((e = mark()) != cudaSuccess) return e;
   // step 2 reversed
   if (kTc) {
-    if ((e = launch_bwd_stats_tc(a, K, at(p.dA2), at(p.dB2), at(p.dkc), at(p.dvc), g.dbeta, status)) != cudaSuccess)
+    if ((e = launch_bwd_stats_tc(a, K, at(p.dA2), at(p.dB2), reinterpret_cast<void*>(at(p.dkc)),
+                                 reinterpret_cast<void*>(at(p.dvc)), g.dbeta, status)) != cudaSuccess)
       return e;
   } else {
     const size_t smem = sizeof(StatsSmem<D>);
@@ -917,17 +918,19 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, const BwdSta
     if (e != cudaSuccess) return e;
     k_bwd_stats<D, T><<<(unsigned)NF, kBT, smem, a.stream>>>(
         static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.beta, a.conv_k_w, a.conv_v_w, K, at(p.dA2),
-        at(p.dB2), at(p.dkc), at(p.dvc), g.dbeta, sh.H, sh.F, sh.S);
+        at(p.dB2), reinterpret_cast<T*>(at(p.dkc)), reinterpret_cast<T*>(at(p.dvc)), g.dbeta, sh.H, sh.F, sh.S);
   }
   if ((e = mark()) != cudaSuccess) return e;
   // step 1 (conv) reversed
   if (K == 3)
     k_bwd_conv<D, T, 3><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
-        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, at(p.dkc), at(p.dvc),
+        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w,
+        reinterpret_cast<const T*>(at(p.dkc)), reinterpret_cast<const T*>(at(p.dvc)),
         static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
   else
     k_bwd_conv<D, T, 1><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
-        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w, at(p.dkc), at(p.dvc),
+        static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w,
+        reinterpret_cast<const T*>(at(p.dkc)), reinterpret_cast<const T*>(at(p.dvc)),
         static_cast<T*>(g.dk), static_cast<T*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
   if ((e = mark()) != cudaSuccess) return e;
   k_bwd_finish<D><<<148, kBT, 0, a.stream>>>(at(p.rms_part), NF, at(p.tap_part), kBwdConvBlocks, K, at(p.dseed2),

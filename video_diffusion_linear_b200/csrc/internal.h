@@ -81,7 +81,7 @@ struct BwdPlan {
   size_t lam_all = 0, dX_all = 0;                      // fp32 [2][B, H, F, d, d]: adjoint and dX per step
   size_t Xbuf = 0;                                     // fp32 [2][B, H, F, d, d] (sana_scaled only)
   size_t rms_part = 0;                                 // fp32 [B, H, F][d]
-  size_t dkc = 0, dvc = 0;                             // fp32 [B, N, H, d]
+  size_t dkc = 0, dvc = 0;                             // [B, N, H, d] in the inputs' element type
   size_t tap_part = 0;                                 // fp32 [H][kBwdConvBlocks][2][d][3]
   size_t fwd_bytes = 0, total = 0;
 };
@@ -113,7 +113,7 @@ constexpr int kBwdKernels = 6;
 // tensor-core versions of the read-out and statistics reversals (bf16, d = 128; tc_backward.cu)
 cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
                                   void* dq, void* dgate, uint32_t* status);
-cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, float* dkc, float* dvc,
+cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, void* dkc, void* dvc,
                                 float* dbeta, uint32_t* status);
 cudaError_t launch_bwd_scan_tc(const Args& a, const uint16_t* nimg, const float* dPin, const float* dQin,
                                float* lam_all, float* dX_all, float* dseed2, uint32_t* status);

@@ -397,7 +397,8 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
                                                                 const float* __restrict__ wv, int K,
                                                                 const float* __restrict__ dA2,
                                                                 const float* __restrict__ dB2,
-                                                                float* __restrict__ dkc, float* __restrict__ dvc,
+                                                                __nv_bfloat16* __restrict__ dkc,
+                                                                __nv_bfloat16* __restrict__ dvc,
                                                                 float* __restrict__ dbeta, int H, int F, int S,
                                                                 uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -572,12 +573,9 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
           gk[e] = (dk - x * xg * inv * inv) * inv * sg * fmaf(kc[e], 1.f - sg, 1.f);
           gv[e] = silu_grad_f(vc[e], bt * inv * __uint_as_float(z[q8]));
         }
-        float* pk = dkc + tok * 128 + c0;
-        float* pv = dvc + tok * 128 + c0;
-        *reinterpret_cast<float4*>(pk) = make_float4(gk[0], gk[1], gk[2], gk[3]);
-        *reinterpret_cast<float4*>(pk + 4) = make_float4(gk[4], gk[5], gk[6], gk[7]);
-        *reinterpret_cast<float4*>(pv) = make_float4(gv[0], gv[1], gv[2], gv[3]);
-        *reinterpret_cast<float4*>(pv + 4) = make_float4(gv[4], gv[5], gv[6], gv[7]);
+        // bf16, as the gradients they feed (dk, dv) are written
+        store8_bf16(dkc + tok * 128 + c0, gk);
+        store8_bf16(dvc + tok * 128 + c0, gv);
       }
     }
     tc::tc_fence_before();
@@ -775,14 +773,15 @@ cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, float* dkc, float* dvc,
+cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, void* dkc, void* dvc,
                                 float* dbeta, uint32_t* status) {
   const size_t smem = sizeof(StatsTcSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_bwd_stats_tc<<<(unsigned)a.NF(), kStatsThreads, smem, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
-      a.conv_v_w, K, dA2, dB2, dkc, dvc, dbeta, a.sh.H, a.sh.F, a.sh.S, status);
+      a.conv_v_w, K, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
+      a.sh.F, a.sh.S, status);
   return cudaGetLastError();
 }
 
