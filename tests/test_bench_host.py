@@ -79,3 +79,35 @@ def test_two_gloo_ranks_take_the_max_time():
 
 def test_reduce_max_without_process_group():
     assert bench.reduce_max(3.5) == 3.5
+
+
+@pytest.mark.parametrize("name", ["480p", "768p", "14s"])
+def test_softmax_flops_count_chunk_pairs(name):
+    # chunk-aligned windows are symmetric: frame f is in the window of frame t exactly when their chunks
+    # differ by at most `radius`, so the (query, key) pairs are sums over chunk pairs
+    w = synth.WORKLOADS[name]
+    nch = -(-w.F // w.chunk)
+    size = [min(w.F, (c + 1) * w.chunk) - c * w.chunk for c in range(nch)]
+    pairs = sum(size[a] * size[b] for a in range(nch) for b in range(nch) if abs(a - b) <= w.radius) * w.S * w.S
+    assert bench.softmax_flops(w) == 4 * w.d * pairs * w.B * w.H
+
+
+def test_backward_accounting():
+    w = synth.WORKLOADS["768p"]
+    TH = w.B * w.F * w.S * w.H
+    nb = bench.backward_bytes(w)
+    tok = 2 * w.d * TH                                   # one bf16 token tensor
+    assert nb["readout_bwd"] >= 5 * tok                  # q, gate, dout in; dq, dgate out
+    assert nb["stats_bwd"] >= 2 * tok + 2 * tok          # k, v in; dk', dv' out
+    assert nb["conv_bwd"] >= 4 * tok                     # dk', dv' (or more), k, v in; dk, dv out
+    fl = bench.backward_flops(w)
+    assert fl["readout_bwd"] == fl["stats_bwd"] == 6 * w.d * w.d * TH
+    assert set(bench.BWD_KERNELS) >= set(nb) | set(fl)
+
+
+def test_recorded_traffic_of_the_softmax_kernel():
+    rec = bench.recorded_traffic("window_softmax")
+    if rec is not None:                                  # present while softmax.cu is unchanged
+        w = synth.WORKLOADS["768p"]
+        alg = 4 * 2 * w.d * w.B * w.F * w.S * w.H        # q_rope, k_rope, v in, out out
+        assert 0.9 * alg <= rec["bytes"] <= 1.2 * alg
