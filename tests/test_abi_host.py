@@ -193,3 +193,54 @@ def test_forward_train_validation(lib):
     assert call(BASE + 30 * GAP + 64, 1 << 40) == VDN_ERR_ALIGNMENT
     assert call(BASE + 11 * GAP, 1 << 40) == VDN_ERR_INVALID_ARG       # overlaps the output
     assert call(BASE + 10 * GAP, 1 << 40) == VDN_ERR_INVALID_ARG       # overlaps the workspace
+
+
+def _soft_args(shape, chunk=5, radius=1, scale=0.0, accumulate=0, ws_bytes=256, **over):
+    names = ["q_rope", "k_rope", "v", "ws", "out"]
+    ptr = {name: BASE + i * GAP for i, name in enumerate(names)}
+    ptr.update(over)
+    P = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n])
+    return (ctypes.byref(shape), P("q_rope"), P("k_rope"), P("v"), chunk, radius, scale, accumulate, P("ws"),
+            ws_bytes, P("out"), None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(chunk=0), VDN_ERR_INVALID_ARG),
+    (dict(radius=-1), VDN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), VDN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), VDN_ERR_INVALID_ARG),
+    (dict(accumulate=2), VDN_ERR_INVALID_ARG),
+    (dict(q_rope=None), VDN_ERR_INVALID_ARG),
+    (dict(out=None), VDN_ERR_INVALID_ARG),
+    (dict(ws=None), VDN_ERR_INVALID_ARG),
+    (dict(k_rope=BASE + GAP + 8), VDN_ERR_ALIGNMENT),
+    (dict(ws=BASE + 3 * GAP + 64), VDN_ERR_ALIGNMENT),
+    (dict(ws_bytes=128), VDN_ERR_WORKSPACE),
+    (dict(out=BASE + 2 * GAP + 4096), VDN_ERR_INVALID_ARG),            # out overlaps v
+    (dict(out=BASE + 3 * GAP), VDN_ERR_INVALID_ARG),                   # out overlaps the status word
+])
+def test_window_softmax_validation(lib, case, expect):
+    s = _shape()
+    assert lib.vdn_window_softmax_forward(*_soft_args(s, **case)) == expect
+
+
+def test_window_softmax_unsupported_shapes(lib):
+    assert lib.vdn_window_softmax_forward(*_soft_args(_shape(d=64))) == VDN_ERR_UNSUPPORTED
+    assert lib.vdn_window_softmax_forward(*_soft_args(_shape(d=16, dtype=1))) == VDN_ERR_UNSUPPORTED
+    assert lib.vdn_window_softmax_workspace_size(ctypes.byref(_shape())) == 256
+    assert lib.vdn_window_softmax_workspace_size(ctypes.byref(_shape(d=64))) == 0
+
+
+def test_hybrid_validation(lib):
+    s = _shape()
+    fwd = list(_args(s, 1 << 40))
+    # vdn_hybrid_forward: shape, q_rope, k_rope, then the forward's tensors, rule, c, chunk, radius, scale,
+    # workspace, workspace_bytes, out, stream
+    qr, kr = ctypes.c_void_p(BASE + 20 * GAP), ctypes.c_void_p(BASE + 21 * GAP)
+    def call(scale=0.0, qr_=qr, out=fwd[17]):
+        return lib.vdn_hybrid_forward(fwd[0], qr_, kr, *fwd[1:15], scale, fwd[15], fwd[16], out, None)
+    assert call(scale=float("nan")) == VDN_ERR_INVALID_ARG
+    assert call(qr_=None) == VDN_ERR_INVALID_ARG
+    assert call(qr_=ctypes.c_void_p(BASE + 20 * GAP + 4)) == VDN_ERR_ALIGNMENT
+    assert call(out=ctypes.c_void_p(BASE + 21 * GAP + 256)) == VDN_ERR_INVALID_ARG   # out overlaps k_rope
+    assert call(out=ctypes.c_void_p(BASE + 64)) == VDN_ERR_INVALID_ARG               # out overlaps q
