@@ -111,3 +111,17 @@ def test_recorded_traffic_of_the_softmax_kernel():
         w = synth.WORKLOADS["768p"]
         alg = 4 * 2 * w.d * w.B * w.F * w.S * w.H        # q_rope, k_rope, v in, out out
         assert 0.9 * alg <= rec["bytes"] <= 1.2 * alg
+
+
+@pytest.mark.parametrize("path", ["linear", "softmax", "backward"])
+def test_reference_arm_prints_one_contract_line(path, capsys):
+    # the oracle arm on the smallest workload: one JSON line with the contract's keys
+    import json
+    bench.main(["--impl", "reference", "--path", path, "--workload", "tiny", "--steps", "2", "--warmup", "3",
+                "--cpu-tokens", "8"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 2 and j["warmup"] == 3
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
