@@ -693,8 +693,18 @@ def run_gpu(args, w: synth.Workload) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     _lib.load()
-    wr = rank_workload(w, rank)
-    host = synth.make_inputs(wr)
+    if args.shard == "heads":
+        # strong scaling: one clip per job, its heads split across the ranks (no exchange)
+        from video_diffusion_linear_b200 import shard
+        if world > w.H:
+            raise SystemExit(f"--shard heads needs at most H = {w.H} ranks")
+        host = shard.shard_inputs(synth.make_inputs(w), world, rank)
+        wr = w.replace(H=int(host["q"].shape[2]))
+        job_tokens = w.tokens                       # the clip, counted once for the job
+    else:
+        wr = rank_workload(w, rank)
+        host = synth.make_inputs(wr)
+        job_tokens = w.tokens * world
     dev = api.to_device(host, device)
     args_t = api.forward_inputs(dev)
     shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
@@ -736,14 +746,14 @@ def run_gpu(args, w: synth.Workload) -> None:
     torch.cuda.synchronize(device)
     ms = start.elapsed_time(end)
     ms_max = reduce_max(ms, device)
-    tokens = w.tokens * world * args.steps
+    tokens = job_tokens * args.steps
     value = tokens / (ms_max / 1e3)
 
     names = KERNELS_TC if nl == 5 else [f"kernel{i}" for i in range(nl)]
     per = {n: statistics.fmean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
            for j, n in enumerate(names)}
     peaks, peak_src = load_peaks()
-    alg = algorithmic_bytes(w)
+    alg = algorithmic_bytes(wr)
     dom = max(per, key=per.get)
     dom_ms = per[dom]
     achieved = alg.get(dom, 0) / (dom_ms / 1e3) / 1e9 if dom in alg else None
@@ -753,7 +763,7 @@ def run_gpu(args, w: synth.Workload) -> None:
             "algorithmic_bytes_per_launch": alg.get(dom),
             "traffic": traffic["bytes"] if traffic else None,
             "traffic_workload": traffic["workload"] if traffic else None}
-    pr = path_roofline(w, peaks)
+    pr = path_roofline(wr, peaks)
     step_us = ms_max / args.steps * 1e3
     kernels = {n: {"us": per[n] * 1e3, "share": per[n] / sum(per.values()),
                    "gbs": (alg[n] / (per[n] / 1e3) / 1e9) if n in alg else None} for n in per}
@@ -784,7 +794,7 @@ def run_gpu(args, w: synth.Workload) -> None:
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = reduce_max(e0.elapsed_time(e1), device)
-        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_tokens * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
     cpu = None
@@ -802,11 +812,15 @@ def run_gpu(args, w: synth.Workload) -> None:
         return
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(w), "global_batch": w.B * world, "tokens_per_step": w.tokens * world,
+        "config": {"workload": describe(w), "global_batch": w.B * (1 if args.shard == "heads" else world),
+                   "tokens_per_step": job_tokens,
                    "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step)" % (4 * w.tokens * w.H * w.d * 2 / 1e9),
-                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+                   "parallelism": (f"heads{world}: one clip, heads {wr.H} per GPU, no collective"
+                                   if args.shard == "heads" else
+                                   f"dp{world}: independent clips per GPU, no collective")},
         "roofline": roof,
         "path_roofline": {"t_roof_us": pr["t_roof_us"], "t_step_us": step_us, "frac": pr["t_roof_us"] / step_us,
                           "bound": pr["bound"], "algorithmic_bytes": pr["bytes"], "flops": pr["flops"],
@@ -838,9 +852,14 @@ def main(argv=None):
                     help="linear branch (default), windowed softmax branch, the whole hybrid layer, or the "
                          "linear branch's backward pass")
     ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
+    ap.add_argument("--shard", default="clips", choices=["clips", "heads"],
+                    help="multi-GPU: independent clips per rank (weak scaling, default) or one clip with its "
+                         "heads split across the ranks (strong scaling); linear branch path")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.shard == "heads" and (args.path != "linear" or args.impl == "reference"):
+        ap.error("--shard heads applies to the linear branch path of the GPU arm")
     w = synth.WORKLOADS[args.workload]
     if args.rule:
         w = w.replace(rule=args.rule)

@@ -194,3 +194,20 @@ def test_divergent_sana_stays_finite_and_matches(w):
     # moves the float64 output by 1e-6; an fp32 emulation of the same arithmetic
     # lands 2.3e-4 from the oracle), so this stress case gets 1e-3
     assert rel_err(to_np(out), ref) <= (1e-3 if w.dtype == "f32" else TOL_BF16)
+
+
+@pytest.mark.parametrize("w,world", [(W["tiny_f20_text"].replace(H=3), 2), (W["tiny_f20_text"].replace(H=3), 3),
+                                     (BF16_SMALL, 2)], ids=["f32_d16_2", "f32_d16_3", "bf16_d128_2"])
+def test_head_sharded_calls_reassemble_the_clip(w, world):
+    """Each rank's call on its slice of the heads (run one after another here: the calls never wait
+    on one another) joins into the whole clip's output, which matches the oracle and the unsharded
+    call; the per-frame partial sums group differently when H changes, so the join is compared
+    within the parity tolerance, not bitwise."""
+    from video_diffusion_linear_b200 import shard
+    inp = synth.make_inputs(w)
+    parts = [gpu_forward(w, shard.shard_inputs(inp, world, r))[0] for r in range(world)]
+    joined = torch.cat(parts, dim=2)
+    full, _ = gpu_forward(w, inp)
+    tol = TOL_F32 if w.dtype == "f32" else TOL_BF16
+    assert rel_err(to_np(joined), oracle_forward(w, inp)) <= tol
+    assert rel_err(to_np(joined), to_np(full)) <= tol
