@@ -761,8 +761,9 @@ def run_gpu(args, w: synth.Workload) -> None:
     roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": (achieved / peaks["hbm_gbs"]) if achieved else None, "peak_source": peak_src,
             "algorithmic_bytes_per_launch": alg.get(dom),
-            "traffic": traffic["bytes"] if traffic else None,
-            "traffic_workload": traffic["workload"] if traffic else None}
+            "traffic": traffic["bytes"] * wr.H / w.H if traffic else None,   # units scale with the heads
+            "traffic_workload": (traffic["workload"] + ("" if wr.H == w.H else f", scaled by {wr.H}/{w.H} heads"))
+                                if traffic else None}
     pr = path_roofline(wr, peaks)
     step_us = ms_max / args.steps * 1e3
     kernels = {n: {"us": per[n] * 1e3, "share": per[n] / sum(per.values()),
@@ -817,7 +818,8 @@ def run_gpu(args, w: synth.Workload) -> None:
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(w), "global_batch": w.B * (1 if args.shard == "heads" else world),
                    "tokens_per_step": job_tokens,
-                   "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step)" % (4 * w.tokens * w.H * w.d * 2 / 1e9),
+                   "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step per GPU)"
+                         % (4 * wr.tokens * wr.H * wr.d * 2 / 1e9),
                    "parallelism": (f"heads{world}: one clip, heads {wr.H} per GPU, no collective"
                                    if args.shard == "heads" else
                                    f"dp{world}: independent clips per GPU, no collective")},
