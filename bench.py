@@ -39,7 +39,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from video_diffusion_linear_b200 import synth  # noqa: E402
+from video_diffusion_linear_b200 import shard, synth  # noqa: E402
 
 METRIC = "latent tokens/sec through VDN linear branch fwd (1 B200); % of roofline"
 METRIC_PATH = {"backward": "latent tokens/sec through the VDN linear branch backward (forward recompute + "
@@ -183,6 +183,31 @@ def dist_env() -> tuple[int, int, int]:
 def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
     """Each rank runs its own clip of the workload (weak scaling, no exchange)."""
     return w.replace(seed=w.seed + 1000 * rank)
+
+
+def rank_inputs(shard_mode: str, w: synth.Workload, world: int, rank: int, *, cotangent: bool = False, **make_kw):
+    """The rank's host inputs: its own clip ("clips": weak scaling) or its contiguous share of the
+    heads of the job's one clip ("heads": strong scaling; every rank draws the same clip).
+    Returns (inputs, the rank's workload, latent tokens the whole job processes per step,
+    the JSON line's scaling/global_batch/parallelism)."""
+    if shard_mode == "heads":
+        if world > w.H:
+            raise SystemExit(f"--shard heads needs at most H = {w.H} ranks")
+        full = synth.make_inputs(w, **make_kw)
+        if cotangent:
+            full["dout"] = synth.make_cotangent(w)
+        host = shard.shard_inputs(full, world, rank)
+        wr = w.replace(H=int(host["q"].shape[2]))
+        h0, h1 = shard.head_range(w.H, world, 0)
+        return host, wr, w.tokens, {"scaling": "strong", "global_batch": w.B,
+                                    "parallelism": f"heads{world}: one clip, its {w.H} heads split across the "
+                                                   f"GPUs ({h1 - h0} on the first), no exchange in the branch"}
+    wr = rank_workload(w, rank)
+    host = synth.make_inputs(wr, **make_kw)
+    if cotangent:
+        host["dout"] = synth.make_cotangent(wr)
+    return host, wr, w.tokens * world, {"scaling": "weak", "global_batch": w.B * world,
+                                        "parallelism": f"dp{world}: independent clips per GPU, no collective"}
 
 
 def reduce_max(value: float, device=None) -> float:
@@ -427,9 +452,9 @@ def run_gpu_backward(args, w: synth.Workload) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     _lib.load()
-    wr = rank_workload(w, rank)
-    host = synth.make_inputs(wr)
-    host["dout"] = synth.make_cotangent(wr)
+    host, wr, job_tokens, split = rank_inputs(args.shard, w, world, rank, cotangent=True)
+    if args.shard == "heads" and world > 1:
+        split["parallelism"] += "; NCCL all-reduce of the rms_w gradient (shared by every head) per step"
     dev = api.to_device(host, device)
     args_t = api.forward_inputs(dev)
     shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
@@ -444,6 +469,8 @@ def run_gpu_backward(args, w: synth.Workload) -> None:
     def step(events=None):
         api.branch_backward(*args_t, dout=dev["dout"], F=w.F, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius,
                             grads=grads, workspace=ws, stream=stream, events=events)
+        if args.shard == "heads" and world > 1:
+            shard.reduce_shared_grads(grads)
 
     for _ in range(args.warmup):
         step()
@@ -469,11 +496,11 @@ def run_gpu_backward(args, w: synth.Workload) -> None:
     torch.cuda.synchronize(device)
     ms = start.elapsed_time(end)
     ms_max = reduce_max(ms, device)
-    value = w.tokens * world * args.steps / (ms_max / 1e3)
+    value = job_tokens * args.steps / (ms_max / 1e3)
     per = {n: statistics.fmean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
            for j, n in enumerate(BWD_KERNELS)}
-    flops = backward_flops(w)
-    nbytes = backward_bytes(w)
+    flops = backward_flops(wr)
+    nbytes = backward_bytes(wr)
     bwd_only = {n: v for n, v in per.items() if n != "forward_recompute"}
     dom = max(bwd_only, key=bwd_only.get)
     csum = clk.summary()
@@ -518,7 +545,7 @@ def run_gpu_backward(args, w: synth.Workload) -> None:
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = reduce_max(e0.elapsed_time(e1), device)
-        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_tokens * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
     cpu = None
@@ -535,12 +562,14 @@ def run_gpu_backward(args, w: synth.Workload) -> None:
         return
     print(json.dumps({
         "metric": METRIC_PATH["backward"], "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 (bf16 inputs and gradients)", "data": "synthetic",
-        "config": {"workload": describe(w) + ", upstream gradient N(0, 1)", "global_batch": w.B * world,
-                   "tokens_per_step": w.tokens * world,
-                   "l2": "inputs larger than L2 (q, k, v, gate, dout: %.2f GB)" % (5 * w.tokens * w.H * w.d * 2 / 1e9),
-                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": split["scaling"], "vs_baseline": None, "dtype": "f32 (bf16 inputs and gradients)",
+        "data": "synthetic",
+        "config": {"workload": describe(w) + ", upstream gradient N(0, 1)", "global_batch": split["global_batch"],
+                   "tokens_per_step": job_tokens,
+                   "l2": "inputs larger than L2 (q, k, v, gate, dout: %.2f GB per GPU)"
+                         % (5 * wr.tokens * wr.H * wr.d * 2 / 1e9),
+                   "parallelism": split["parallelism"]},
         "roofline": roof,
         "kernels": kernels,
         "cpu_baseline": cpu,
@@ -561,8 +590,7 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     _lib.load()
-    wr = rank_workload(w, rank)
-    host = synth.make_inputs(wr, with_rope_side=True)
+    host, wr, job_tokens, split = rank_inputs(args.shard, w, world, rank, with_rope_side=True)
     dev = api.to_device(host, device)
     out = torch.empty_like(dev["q"])
     stream = torch.cuda.current_stream(device)
@@ -614,11 +642,11 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
         raise RuntimeError("device-side wait timed out during the timed steps")
     ms = start.elapsed_time(end)
     ms_max = reduce_max(ms, device)
-    value = w.tokens * world * args.steps / (ms_max / 1e3)
+    value = job_tokens * args.steps / (ms_max / 1e3)
     soft_ms = (statistics.fmean(kev[i].elapsed_time(kev[i + 1]) for i in range(args.steps)) if hybrid
                else ms / args.steps)
     peaks, peak_src = load_peaks()
-    flops = softmax_flops(w)
+    flops = softmax_flops(wr)
     achieved = flops / (soft_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roof = {"kernel": "window_softmax", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -626,8 +654,9 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
             "algorithmic_flops_per_launch": flops, "traffic": recorded_traffic("window_softmax"),
             "us_per_launch": soft_ms * 1e3}
     if roof["traffic"] is not None:
-        roof["traffic_workload"] = roof["traffic"]["workload"]
-        roof["traffic"] = roof["traffic"]["bytes"]
+        roof["traffic_workload"] = roof["traffic"]["workload"] + ("" if wr.H == w.H else
+                                                                  f", scaled by {wr.H}/{w.H} heads")
+        roof["traffic"] = roof["traffic"]["bytes"] * wr.H / w.H
 
     e2e = None
     if not args.no_e2e:
@@ -649,7 +678,7 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = reduce_max(e0.elapsed_time(e1), device)
-        e2e = {"value": w.tokens * world * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_tokens * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
     cpu = None
@@ -670,12 +699,13 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
         return
     print(json.dumps({
         "metric": METRIC_PATH[args.path], "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": split["scaling"], "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(w) + f", softmax window = chunk {w.chunk} +- {w.radius} chunks, "
-                   "scale 1/sqrt(d)", "global_batch": w.B * world, "tokens_per_step": w.tokens * world,
-                   "l2": "inputs larger than L2 (q_rope, k_rope, v: %.2f GB)" % (3 * w.tokens * w.H * w.d * 2 / 1e9),
-                   "parallelism": f"dp{world}: independent clips per GPU, no collective"},
+                   "scale 1/sqrt(d)", "global_batch": split["global_batch"], "tokens_per_step": job_tokens,
+                   "l2": "inputs larger than L2 (q_rope, k_rope, v: %.2f GB per GPU)"
+                         % (3 * wr.tokens * wr.H * wr.d * 2 / 1e9),
+                   "parallelism": split["parallelism"]},
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -693,18 +723,7 @@ def run_gpu(args, w: synth.Workload) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     _lib.load()
-    if args.shard == "heads":
-        # strong scaling: one clip per job, its heads split across the ranks (no exchange)
-        from video_diffusion_linear_b200 import shard
-        if world > w.H:
-            raise SystemExit(f"--shard heads needs at most H = {w.H} ranks")
-        host = shard.shard_inputs(synth.make_inputs(w), world, rank)
-        wr = w.replace(H=int(host["q"].shape[2]))
-        job_tokens = w.tokens                       # the clip, counted once for the job
-    else:
-        wr = rank_workload(w, rank)
-        host = synth.make_inputs(wr)
-        job_tokens = w.tokens * world
+    host, wr, job_tokens, split = rank_inputs(args.shard, w, world, rank)
     dev = api.to_device(host, device)
     args_t = api.forward_inputs(dev)
     shape = api.shape_from(dev["q"], w.F, dev["conv_k_w"])
@@ -814,15 +833,11 @@ def run_gpu(args, w: synth.Workload) -> None:
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "strong" if args.shard == "heads" else "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(w), "global_batch": w.B * (1 if args.shard == "heads" else world),
-                   "tokens_per_step": job_tokens,
+        "scaling": split["scaling"], "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w), "global_batch": split["global_batch"], "tokens_per_step": job_tokens,
                    "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step per GPU)"
                          % (4 * wr.tokens * wr.H * wr.d * 2 / 1e9),
-                   "parallelism": (f"heads{world}: one clip, heads {wr.H} per GPU, no collective"
-                                   if args.shard == "heads" else
-                                   f"dp{world}: independent clips per GPU, no collective")},
+                   "parallelism": split["parallelism"]},
         "roofline": roof,
         "path_roofline": {"t_roof_us": pr["t_roof_us"], "t_step_us": step_us, "frac": pr["t_roof_us"] / step_us,
                           "bound": pr["bound"], "algorithmic_bytes": pr["bytes"], "flops": pr["flops"],
@@ -856,12 +871,12 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
     ap.add_argument("--shard", default="clips", choices=["clips", "heads"],
                     help="multi-GPU: independent clips per rank (weak scaling, default) or one clip with its "
-                         "heads split across the ranks (strong scaling); linear branch path")
+                         "heads split across the ranks (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.shard == "heads" and (args.path != "linear" or args.impl == "reference"):
-        ap.error("--shard heads applies to the linear branch path of the GPU arm")
+    if args.shard == "heads" and args.impl == "reference":
+        ap.error("--shard heads applies to the GPU arm")
     w = synth.WORKLOADS[args.workload]
     if args.rule:
         w = w.replace(rule=args.rule)

@@ -1,11 +1,13 @@
 """Head sharding of the branch across ranks (one process per GPU).
 
 Every step of the branch is per (batch, head): statistics, solve, both scans, gather and read-out
-never mix heads.  A clip whose heads are split across ranks therefore needs no exchange inside the
-branch: each rank runs vdn_branch_forward on its contiguous range of heads, with the per-head
-parameters (text state, conv taps) of those heads and the shared ones (rms_w) whole.  Bringing a
-sequence-sharded layout to a head-sharded one (the Ulysses all-to-all of q, k, v, gate and back)
-belongs to the surrounding model, not to the branch.
+never mix heads, and neither does the windowed softmax branch.  A clip whose heads are split across
+ranks therefore needs no exchange in the forward: each rank runs the unchanged entry points on its
+contiguous range of heads, with the per-head parameters (text state, conv taps) of those heads and
+the shared ones (rms_w) whole.  The backward's one exchange is the gradient of rms_w, which every
+head shares: each rank's call sums it over its own heads, and reduce_shared_grads sums those
+partials across the ranks.  Bringing a sequence-sharded layout to a head-sharded one (the Ulysses
+all-to-all of q, k, v, gate and back) belongs to the surrounding model, not to the branch.
 """
 from __future__ import annotations
 
@@ -20,10 +22,14 @@ def head_range(H: int, world: int, rank: int) -> tuple[int, int]:
     return h0, h0 + base + (1 if rank < extra else 0)
 
 
-PER_HEAD = {  # tensor -> axis of the head index
-    "q": 2, "k": 2, "v": 2, "gate": 2, "beta": 2, "alpha": 2, "q_rope": 2, "k_rope": 2,
+PER_HEAD = {  # tensor -> axis of the head index (inputs, the upstream gradient and the gradients)
+    "q": 2, "k": 2, "v": 2, "gate": 2, "beta": 2, "alpha": 2, "q_rope": 2, "k_rope": 2, "dout": 2,
     "conv_k_w": 0, "conv_v_w": 0, "text_state": 0,
+    "dq": 2, "dk": 2, "dv": 2, "dgate": 2, "dbeta": 2, "dalpha": 2,
+    "dconv_k_w": 0, "dconv_v_w": 0, "dtext_state": 0,
 }
+
+SHARED_GRADS = ("drms_w",)  # gradients of parameters every head shares: summed across the ranks
 
 
 def shard_inputs(inputs: dict, world: int, rank: int) -> dict:
@@ -38,3 +44,16 @@ def shard_inputs(inputs: dict, world: int, rank: int) -> dict:
             continue
         out[name] = t.narrow(PER_HEAD[name], h0, h1 - h0).contiguous()
     return out
+
+
+def reduce_shared_grads(grads: dict, group=None) -> dict:
+    """Sum the gradients of the shared parameters (rms_w) over the ranks of `group`, in place, with
+    one all-reduce each (NCCL for CUDA tensors).  Per-head gradients stay on their rank.  A no-op
+    without an initialised process group of more than one rank."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return grads
+    for name in SHARED_GRADS:
+        if grads.get(name) is not None:
+            dist.all_reduce(grads[name], op=dist.ReduceOp.SUM, group=group)
+    return grads
