@@ -138,3 +138,149 @@ def test_two_gloo_ranks_reassemble_the_backward():
     # the shared gradient is a sum over heads: equal up to the order of the additions
     np.testing.assert_allclose(drms, ref["drms_w"], rtol=1e-12, atol=1e-12 * np.abs(ref["drms_w"]).max())
     assert not np.allclose(local_drms, ref["drms_w"])    # rank 0's own heads alone do not give it
+
+
+# ----------------------------------------------------------------------------- frame sharding
+@pytest.mark.parametrize("F,chunk", [(0, 5), (1, 5), (23, 3), (31, 5), (30, 2), (85, 5)])
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_frame_ranges_are_whole_chunks_covering_every_frame_once(F, chunk, world):
+    ranges = [shard.frame_range(F, world, r, chunk) for r in range(world)]
+    assert [f for f0, f1 in ranges for f in range(f0, f1)] == list(range(F))
+    assert all(f0 % chunk == 0 for f0, f1 in ranges if f1 > f0)
+    nchunks = [-(-(f1 - f0) // chunk) for f0, f1 in ranges]
+    assert max(nchunks) - min(nchunks) <= 1
+
+
+@pytest.mark.parametrize("F,chunk,radius,world", [(23, 3, 1, 3), (30, 2, 6, 3), (31, 5, 1, 4), (31, 5, 2, 2)])
+def test_exchange_plan_matches_the_window_geometry(F, chunk, radius, world):
+    # brute force from the oracle's window geometry: every state a window reads outside its rank is
+    # published by exactly the rank that owns it
+    owner = {f: r for r in range(world) for f in range(*shard.frame_range(F, world, r, chunk))}
+    need_pre, need_suf = set(), set()
+    for r in range(world):
+        f0, f1 = shard.frame_range(F, world, r, chunk)
+        pre, suf = shard.remote_states(F, chunk, radius, f0, f1)
+        want_pre = {lo - 1 for lo, hi in (O.window_bounds(t, F, chunk, radius) for t in range(f0, f1))
+                    if lo > 0 and owner[lo - 1] != r}
+        want_suf = {hi + 1 for lo, hi in (O.window_bounds(t, F, chunk, radius) for t in range(f0, f1))
+                    if hi < F - 1 and owner[hi + 1] != r}
+        assert set(pre) == want_pre and set(suf) == want_suf
+        need_pre |= want_pre
+        need_suf |= want_suf
+    pub = [shard.published_states(F, world, r, chunk, radius) for r in range(world)]
+    assert sorted(f for p, _ in pub for f in p) == sorted(need_pre)
+    assert sorted(f for _, s in pub for f in s) == sorted(need_suf)
+    assert all(owner[f] == r for r, (p, s) in enumerate(pub) for f in p + s)
+
+
+def _frame_worker(rank, world, port, w, q):
+    """One rank of the frame-sharded branch, its arithmetic taken from the oracle: local features,
+    statistics and per-frame affine maps; an all-gather of each rank's composed maps gives the seeds;
+    a local re-scan; an all-gather of the published boundary states; then gather and read-out.
+    States the plan does not deliver stay NaN, so a gap in it shows in the output."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = synth.make_inputs(w)
+        F, S, d, H = w.F, w.S, w.d, w.H
+        f0, f1 = shard.frame_range(F, world, rank, w.chunk)
+        n = f1 - f0
+        eye, zero = np.eye(d), np.zeros((d, d))
+
+        def step(s, f, st):
+            return O.rule_step(s, st["A"][f - f0], st["B"][f - f0], st["alpha"][f], w.rule, w.c)
+
+        local = {}
+        maps = {}
+        for h in range(H):
+            sl = slice(f0 * S, f1 * S)
+            qf, kf, vf = O.prepare_features(O._f64(inp["q"][0, sl, h]), O._f64(inp["k"][0, sl, h]),
+                                            O._f64(inp["v"][0, sl, h]), n, S, O._f64(inp["conv_k_w"][h]),
+                                            O._f64(inp["conv_v_w"][h]))
+            A, Bm = O.frame_statistics(kf, vf, O._f64(inp["beta"][0, sl, h]).reshape(n, S))
+            st = {"qf": qf, "A": A, "B": Bm, "alpha": O._f64(inp["alpha"][0, :, h]),
+                  "seed": O.seed_state(O._f64(inp["text_state"][h]), d)}
+            local[h] = st
+            Gf, Bf = eye, zero                        # frames f0..f1-1, in the prefix scan's order
+            for f in range(f0, f1):
+                Bp = step(zero, f, st)
+                Gf, Bf = Gf @ (step(eye, f, st) - Bp), Bf @ (step(eye, f, st) - Bp) + Bp
+            Gb, Bb = eye, zero                        # frames f1-1..f0, in the suffix scan's order
+            for f in reversed(range(f0, f1)):
+                Bp = step(zero, f, st)
+                Gb, Bb = Gb @ (step(eye, f, st) - Bp), Bb @ (step(eye, f, st) - Bp) + Bp
+            maps[h] = (Gf, Bf, Gb, Bb)
+        all_maps = [None] * world
+        dist.all_gather_object(all_maps, maps)
+
+        pub_pre, pub_suf = shard.published_states(F, world, rank, w.chunk, w.radius)
+        sent = {}
+        for h, st in local.items():
+            sp = st["seed"]
+            for r in range(rank):
+                sp = sp @ all_maps[r][h][0] + all_maps[r][h][1]
+            ss = st["seed"]
+            for r in reversed(range(rank + 1, world)):
+                ss = ss @ all_maps[r][h][2] + all_maps[r][h][3]
+            P = np.full((F, d, d), np.nan)
+            Q = np.full((F, d, d), np.nan)
+            for f in range(f0, f1):
+                sp = step(sp, f, st)
+                P[f] = sp
+            for f in reversed(range(f0, f1)):
+                ss = step(ss, f, st)
+                Q[f] = ss
+            st["P"], st["Q"] = P, Q
+            sent[h] = ({f: P[f] for f in pub_pre}, {f: Q[f] for f in pub_suf})
+        got = [None] * world
+        dist.all_gather_object(got, sent)
+
+        need_pre, need_suf = shard.remote_states(F, w.chunk, w.radius, f0, f1)
+        out = np.empty((n * S, H, d))
+        rms_w = O._f64(inp["rms_w"])
+        for h, st in local.items():
+            for r in range(world):
+                for f, x in got[r][h][0].items():
+                    if f in need_pre:
+                        st["P"][f] = x
+                for f, x in got[r][h][1].items():
+                    if f in need_suf:
+                        st["Q"][f] = x
+            g = O._f64(inp["gate"][0, f0 * S:f1 * S, h]).reshape(n, S, d)
+            for t in range(f0, f1):
+                W_t = O.gather_state(st["P"], st["Q"], st["seed"], st["alpha"], t, w.chunk, w.radius)
+                out[(t - f0) * S:(t - f0 + 1) * S, h] = O.readout(W_t, st["qf"][t - f0], g[t - f0], rms_w)
+        parts = [None] * world
+        dist.all_gather_object(parts, out)
+        if rank == 0:
+            q.put(np.concatenate(parts, axis=0))
+    finally:
+        dist.destroy_process_group()
+
+
+FRAME_CASES = [
+    # 8 chunks over 3 ranks (3, 3, 2): windows reach the neighbouring ranks
+    synth.Workload("fs_solve", B=1, H=2, d=8, F=23, S=7, dtype="f32", alpha_mu=2.0, text=True, seed=33,
+                   chunk=3, radius=1),
+    # 15 chunks of 2 frames over 3 ranks, windows 12 frames each side: states come from two ranks away
+    synth.Workload("fs_sana", B=1, H=1, d=8, F=30, S=5, dtype="f32", alpha_mu=2.0, text=True, seed=34,
+                   chunk=2, radius=6, rule="sana_scaled", c=0.7),
+]
+
+
+@pytest.mark.parametrize("w", FRAME_CASES, ids=[c.name for c in FRAME_CASES])
+def test_three_gloo_ranks_frame_sharded_branch_matches_the_whole_clip(w):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_frame_worker, args=(r, 3, port, w, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    joined = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ref = O.branch_forward(synth.make_inputs(w), w.F, w.S, w.rule, w.c, w.chunk, w.radius)[0]
+    assert np.isfinite(joined).all()
+    # composing the maps reorders the arithmetic of the scans: equal to rounding
+    np.testing.assert_allclose(joined, ref, rtol=1e-9, atol=1e-11 * np.abs(ref).max())

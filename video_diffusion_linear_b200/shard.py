@@ -57,3 +57,55 @@ def reduce_shared_grads(grads: dict, group=None) -> dict:
         if grads.get(name) is not None:
             dist.all_reduce(grads[name], op=dist.ReduceOp.SUM, group=group)
     return grads
+
+
+# ----------------------------------------------------------------------------- frame sharding
+# For clips too long for one GPU the frames split instead.  Every frame's statistics, solve and
+# read-out are local; the only coupling is the pair of scans.  Each rule's step is affine in the
+# state, S_out = S_in G_f + B'_f, so a rank's run of frames composes into one map per direction,
+# and the ranks before it (after it, for the suffix scan) fold into the seed it starts from.  A
+# window then reads the prefix state just before it and the suffix state just after it, which can
+# lie on another rank: those boundary states make the second, equally small exchange.  The
+# functions below fix who owns which frames and which states cross; the arithmetic runs on the
+# device.
+
+def _window(t: int, F: int, chunk: int, radius: int) -> tuple[int, int]:
+    # chunk-aligned window of query frame t: its chunk widened by `radius` chunks each side
+    c = t // chunk
+    return max(0, chunk * (c - radius)), min(F - 1, chunk * (c + radius + 1) - 1)
+
+
+def frame_range(F: int, world: int, rank: int, chunk: int) -> tuple[int, int]:
+    """Frames [f0, f1) of `rank` under frame sharding: a contiguous run of whole chunks of `chunk`
+    frames (the clip's last chunk may be short), the chunks split as head_range splits heads."""
+    if chunk < 1 or F < 0:
+        raise ValueError(f"bad frame shard: F={F} chunk={chunk}")
+    c0, c1 = head_range(-(-F // chunk), world, rank)
+    return min(F, c0 * chunk), min(F, c1 * chunk)
+
+
+def remote_states(F: int, chunk: int, radius: int, f0: int, f1: int) -> tuple[list[int], list[int]]:
+    """(pre, suf): the frames f whose prefix state P_f (read at lo - 1) and suffix state Q_f (read at
+    hi + 1) the windows of query frames [f0, f1) need and another rank computes.  A window at a
+    clip edge reads the seed and needs nothing."""
+    pre, suf = set(), set()
+    for t in range(f0, f1):
+        lo, hi = _window(t, F, chunk, radius)
+        if lo > 0 and not f0 <= lo - 1 < f1:
+            pre.add(lo - 1)
+        if hi < F - 1 and not f0 <= hi + 1 < f1:
+            suf.add(hi + 1)
+    return sorted(pre), sorted(suf)
+
+
+def published_states(F: int, world: int, rank: int, chunk: int, radius: int) -> tuple[list[int], list[int]]:
+    """(pre, suf): the frames of `rank` whose prefix / suffix states some other rank's windows read,
+    i.e. what `rank` contributes to the boundary exchange."""
+    f0, f1 = frame_range(F, world, rank, chunk)
+    pre, suf = set(), set()
+    for r in range(world):
+        if r != rank:
+            p, s = remote_states(F, chunk, radius, *frame_range(F, world, r, chunk))
+            pre.update(f for f in p if f0 <= f < f1)
+            suf.update(f for f in s if f0 <= f < f1)
+    return sorted(pre), sorted(suf)
