@@ -342,6 +342,58 @@ vdn_status vdn_branch_backward_timed(const vdn_shape* shape,
                                      float* dconv_k_w, float* dconv_v_w, float* dtext_state,
                                      void* stream, void* const* events, int n_events);
 
+/*
+ * Frame sharding -- the branch of one clip split by frames across `world` ranks
+ * (one process per GPU), page sections "Step 3" and "Step 4".
+ *
+ * Rank r owns a contiguous run of whole chunks of the F_total-frame clip
+ * (vdn_frame_range: the C = ceil(F_total / chunk) chunks split into `world`
+ * runs, the first C % world ranks taking one more; world <= C).  Its inputs are
+ * its own frames: q, k, v, gate [B, F*S, H, d] and beta [B, F*S, H] for those
+ * F = f1 - f0 frames, `shape` describing them (shape->F = F), alpha [B, F, H, d]
+ * of its frames for the first phase and of the whole clip for the second.
+ *
+ * Every rule's frame step is affine in the state, S_out = S_in G_f + B'_f.
+ * Phase 1, vdn_frames_maps: features, statistics and solves of the rank's frames,
+ * then for each of its chunks and both scan directions the chunk's composed map
+ * S -> S G_c + O_c, written to `maps`:
+ *     maps [B*H][2 directions][nch][G_c | O_c][d][d] fp32, nch = ceil(C / world)
+ *     (vdn_frames_map_bytes bytes; slots past the rank's own chunks are unused).
+ * The caller then concatenates every rank's buffer in rank order (an all-gather)
+ * into maps_all [world][vdn_frames_map_bytes / 4].
+ * Phase 2, vdn_frames_finish: folds the maps from 0.5 * text_state into the
+ * clip's chunk-edge states (P at chunk ends, Q at chunk starts), gathers the
+ * windows of the rank's query frames and writes their read-out to out
+ * [B, F*S, H, d].  The result equals vdn_branch_forward's rows of those frames
+ * up to rounding.
+ *
+ * Supported: bf16, d = 128 (the tensor-core path), chunk <= 16; otherwise
+ * VDN_ERR_UNSUPPORTED.  A partition that does not match shape->F, world > C or a
+ * rank outside [0, world) is VDN_ERR_INVALID_ARG.  Both phases take one
+ * workspace of vdn_frames_workspace_size bytes (256-byte aligned; it may be the
+ * same buffer).  Pointers as in vdn_branch_forward: 16-byte aligned device
+ * memory owned by the caller; out and maps must not overlap any other argument.
+ * Work is queued on `stream`; errors are returned before any launch.
+ */
+vdn_status vdn_frame_range(int F_total, int world, int rank, int chunk, int* f0, int* f1);
+/* the rank that owns frame `frame` (0 <= frame < F_total) under the same partition */
+vdn_status vdn_frame_owner(int F_total, int world, int chunk, int frame, int* rank);
+size_t vdn_frames_map_bytes(const vdn_shape* shape, int F_total, int world, int rank, int chunk);
+size_t vdn_frames_workspace_size(const vdn_shape* shape, int F_total, int world, int rank, int rule, int chunk);
+vdn_status vdn_frames_maps(const vdn_shape* shape, int F_total, int world, int rank,
+                           const void* k, const void* v, const float* beta, const float* alpha,
+                           const float* conv_k_w, const float* conv_v_w,
+                           int rule, float c, int chunk,
+                           void* workspace, size_t workspace_bytes,
+                           float* maps, size_t maps_bytes, void* stream);
+vdn_status vdn_frames_finish(const vdn_shape* shape, int F_total, int world, int rank,
+                             const void* q, const float* alpha_all, const void* gate, const float* rms_w,
+                             const float* text_state,
+                             int rule, float c, int chunk, int radius,
+                             const float* maps_all, size_t maps_all_bytes,
+                             void* workspace, size_t workspace_bytes,
+                             void* out, void* stream);
+
 /* Reads the device status word that bounded waits inside the kernels set (it
  * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
  * Synchronises `stream`. */

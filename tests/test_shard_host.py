@@ -284,3 +284,40 @@ def test_three_gloo_ranks_frame_sharded_branch_matches_the_whole_clip(w):
     assert np.isfinite(joined).all()
     # composing the maps reorders the arithmetic of the scans: equal to rounding
     np.testing.assert_allclose(joined, ref, rtol=1e-9, atol=1e-11 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("rule,c", [("vdn_solve", 1.0), ("vdn_scaled", 0.6), ("sana_scaled", 0.7), ("additive", 1.0)])
+@pytest.mark.parametrize("F,chunk", [(11, 3), (10, 5), (7, 2)])
+def test_chunk_maps_fold_into_the_scans_chunk_edge_states(rule, c, F, chunk):
+    """The device path's exchange, in the oracle's arithmetic: per chunk and direction, O_c is the
+    chunk's scan from zero and G_c the scan from the identity with B taken as zero (the linear part);
+    folding S <- S G_c + O_c from the seed in scan order gives P at every chunk end and Q at every
+    chunk start, as the whole-clip scans do."""
+    rng = np.random.default_rng(40 + F + chunk)
+    d = 6
+    R = rng.normal(size=(F, d, d))
+    A = np.einsum("fij,fkj->fik", R, R) / d
+    Bm = rng.normal(size=(F, d, d))
+    alpha = 1 / (1 + np.exp(-rng.normal(2, 1, size=(F, d))))
+    seed = rng.normal(size=(d, d))
+    P, Q = O.bidirectional_scan(A, Bm, alpha, seed, rule, c)
+    zero = np.zeros((d, d))
+    chunks = [list(range(j, min(F, j + chunk))) for j in range(0, F, chunk)]
+
+    def chunk_map(frames):
+        s0, s1 = zero, np.eye(d)
+        for f in frames:
+            s0 = O.rule_step(s0, A[f], Bm[f], alpha[f], rule, c)
+            s1 = O.rule_step(s1, A[f], zero, alpha[f], rule, c)
+        return s1, s0                                           # (G_c, O_c)
+
+    s = seed
+    for fr in chunks[:-1]:                                      # prefix: P at each chunk's last frame
+        G, Oc = chunk_map(fr)
+        s = s @ G + Oc
+        np.testing.assert_allclose(s, P[fr[-1]], rtol=1e-10, atol=1e-10 * np.abs(P).max())
+    s = seed
+    for fr in reversed(chunks[1:]):                             # suffix: Q at each chunk's first frame
+        G, Oc = chunk_map(fr[::-1])
+        s = s @ G + Oc
+        np.testing.assert_allclose(s, Q[fr[0]], rtol=1e-10, atol=1e-10 * np.abs(Q).max())

@@ -70,6 +70,20 @@ _SIGNATURES = {
                                                  ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, _P, _P,
                                                  ctypes.c_size_t, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P,
                                                  _P, _P, _P, _P]),
+    "vdn_frame_range": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "vdn_frame_owner": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int)]),
+    "vdn_frames_map_bytes": (ctypes.c_size_t, [ctypes.POINTER(VdnShape), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int]),
+    "vdn_frames_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(VdnShape), ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "vdn_frames_maps": (ctypes.c_int, [ctypes.POINTER(VdnShape), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                       _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "vdn_frames_finish": (ctypes.c_int, [ctypes.POINTER(VdnShape), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                         ctypes.c_int, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P, _P]),
     "vdn_workspace_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "vdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }

@@ -264,3 +264,73 @@ def forward_inputs(dev: dict):
     """Positional tensor arguments of branch_forward from a synth-style dict."""
     return (dev["q"], dev["k"], dev["v"], dev["beta"], dev["alpha"], dev["gate"], dev["rms_w"],
             dev.get("conv_k_w"), dev.get("conv_v_w"), dev.get("text_state"))
+
+
+# ----------------------------------------------------------------------------- frame sharding
+def frame_range(F: int, world: int, rank: int, chunk: int = 5) -> tuple[int, int]:
+    """vdn_frame_range: the frames [f0, f1) rank `rank` of `world` owns under frame sharding
+    (whole chunks, split as evenly as possible)."""
+    f0, f1 = ctypes.c_int(), ctypes.c_int()
+    check(_lib.load().vdn_frame_range(F, world, rank, chunk, ctypes.byref(f0), ctypes.byref(f1)), "vdn_frame_range")
+    return f0.value, f1.value
+
+
+def frame_owner(F: int, world: int, frame: int, chunk: int = 5) -> int:
+    r = ctypes.c_int()
+    check(_lib.load().vdn_frame_owner(F, world, chunk, frame, ctypes.byref(r)), "vdn_frame_owner")
+    return r.value
+
+
+def frames_map_bytes(shape: VdnShape, F_total: int, world: int, rank: int, chunk: int = 5) -> int:
+    n = _lib.load().vdn_frames_map_bytes(ctypes.byref(shape), F_total, world, rank, chunk)
+    if n == 0:
+        raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_frames_map_bytes")
+    return n
+
+
+def frames_workspace_size(shape: VdnShape, F_total: int, world: int, rank: int, rule="vdn_solve",
+                          chunk: int = 5) -> int:
+    n = _lib.load().vdn_frames_workspace_size(ctypes.byref(shape), F_total, world, rank, VDN_RULE[rule], chunk)
+    if n == 0:
+        raise _lib.VdnError(_lib.VDN_ERR_INVALID_ARG, "vdn_frames_workspace_size")
+    return n
+
+
+def frames_maps(k, v, beta, alpha, conv_k_w=None, conv_v_w=None, *, F_total: int, world: int, rank: int,
+                rule="vdn_solve", c=1.0, chunk=5, workspace=None, maps=None, stream=None) -> torch.Tensor:
+    """vdn_frames_maps, phase 1 of the frame-sharded branch: k, v, beta, alpha hold the rank's
+    frames only.  Returns the rank's per-chunk affine maps (flat fp32, frames_map_bytes / 4)."""
+    f0, f1 = frame_range(F_total, world, rank, chunk)
+    shape = shape_from(k, f1 - f0, conv_k_w if conv_k_w is not None else conv_v_w)
+    nb = frames_map_bytes(shape, F_total, world, rank, chunk)
+    if maps is None:
+        maps = torch.empty(nb // 4, dtype=torch.float32, device=k.device)
+    if workspace is None:
+        workspace = torch.empty(frames_workspace_size(shape, F_total, world, rank, rule, chunk), dtype=torch.uint8,
+                                device=k.device)
+    st = _lib.load().vdn_frames_maps(ctypes.byref(shape), F_total, world, rank, _ptr(k), _ptr(v), _ptr(beta),
+                                     _ptr(alpha), _ptr(conv_k_w), _ptr(conv_v_w), VDN_RULE[rule], float(c),
+                                     int(chunk), _ptr(workspace), workspace.numel(), _ptr(maps),
+                                     maps.numel() * maps.element_size(), _stream_ptr(stream))
+    check(st, "vdn_frames_maps")
+    return maps
+
+
+def frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_total: int, world: int, rank: int,
+                  rule="vdn_solve", c=1.0, chunk=5, radius=1, out=None, workspace=None, stream=None):
+    """vdn_frames_finish, phase 2: q and gate hold the rank's frames, alpha_all the whole clip's,
+    maps_all every rank's maps in rank order.  Returns the branch output of the rank's frames."""
+    f0, f1 = frame_range(F_total, world, rank, chunk)
+    shape = shape_from(q, f1 - f0)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(frames_workspace_size(shape, F_total, world, rank, rule, chunk), dtype=torch.uint8,
+                                device=q.device)
+    st = _lib.load().vdn_frames_finish(ctypes.byref(shape), F_total, world, rank, _ptr(q), _ptr(alpha_all),
+                                       _ptr(gate), _ptr(rms_w), _ptr(text_state), VDN_RULE[rule], float(c),
+                                       int(chunk), int(radius), _ptr(maps_all),
+                                       maps_all.numel() * maps_all.element_size(), _ptr(workspace),
+                                       workspace.numel(), _ptr(out), _stream_ptr(stream))
+    check(st, "vdn_frames_finish")
+    return out

@@ -100,6 +100,25 @@ __host__ __device__ __forceinline__ void window_bounds(int t, int F, int chunk, 
   hi = h > F - 1 ? F - 1 : (int)h;
 }
 
+// Frame sharding: C chunks split into `world` contiguous runs, the first C % world
+// ranks taking one chunk more.  chunk_range gives rank r's chunks [c0, c1);
+// chunk_owner the rank of chunk c and its index j there (requires world <= C).
+__host__ __device__ __forceinline__ void chunk_range(int C, int world, int r, int& c0, int& c1) {
+  const int base = C / world, extra = C % world;
+  c0 = r * base + (r < extra ? r : extra);
+  c1 = c0 + base + (r < extra ? 1 : 0);
+}
+__host__ __device__ __forceinline__ void chunk_owner(int c, int C, int world, int& r, int& j) {
+  const int base = C / world, extra = C % world;
+  if (c < extra * (base + 1)) {
+    r = c / (base + 1);
+    j = c - r * (base + 1);
+  } else {   // base >= 1 here: world <= C
+    r = extra + (c - extra * (base + 1)) / base;
+    j = c - (r * base + extra);
+  }
+}
+
 // Coefficients of the generic step  S_f = (S_{f-1} D_f + cpre B_f) N_f + cpost B_f,
 // which covers the three rules of the page plus the additive test rule.
 struct RuleCoef {

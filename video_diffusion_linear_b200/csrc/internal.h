@@ -61,6 +61,15 @@ cudaError_t launch_scan_simt(const Args& a, const float* Bm, const float* Nm, fl
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
                           uint16_t* wimg, int* wexp, int* wbexp);
 cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, const int* wexp);
+// longest chunk the per-chunk gather of the tensor-core path takes (frame sharding requires it)
+constexpr int kGatherMaxChunk = 16;
+// frame sharding (tensor-core path): the gather for query frames fq0 .. fq0 + Fq - 1 of the
+// a.sh.F-frame clip (P, Q, exponents and alpha cover the clip; W_t lands at index t - fq0)
+cudaError_t launch_gather_frames(const Args& a, int fq0, int Fq, const float* P, const float* Q, const int* pexp,
+                                 const int* qexp, float* W, uint16_t* wimg, int* wexp, int* wbexp);
+// the fold of every chunk's affine maps into the chunk-edge states P (chunk ends) and Q (chunk
+// starts) of the a.sh.F-frame clip, from 0.5 x the text state (frames.cu)
+cudaError_t launch_fold_maps(const Args& a, const float* maps_all, int world, int nch_stride, float* P, float* Q);
 // dst = src * 2^expo[frame] (expo may be NULL)
 cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo = nullptr);
 
@@ -127,8 +136,11 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 
 // tensor-core path (bf16, d = 128)
 cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
+// scan modes: the whole clip from the text seed, or per-chunk affine maps (frame sharding)
+constexpr int kScanWhole = 0, kScanSegZero = 1, kScanSegIdentity = 2;
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
-                           int* qexp, bool all_frames, uint32_t* status);
+                           int* qexp, bool all_frames, uint32_t* status, int seg_mode = kScanWhole,
+                           float* maps = nullptr, int nch_stride = 0);
 cudaError_t launch_window_softmax_simt(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
                                        int radius, float scale, int accumulate, void* out, cudaStream_t stream);
 cudaError_t launch_window_softmax_tc(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,

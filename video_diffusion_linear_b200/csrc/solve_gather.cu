@@ -602,7 +602,9 @@ __global__ void __launch_bounds__(512) k_gather128(const float* __restrict__ P, 
 // boundary states; their rows are read once and each frame's W_t differs only
 // in its two decay vectors.  The sides are aligned to the larger block exponent
 // (stored states are below 2^48, see the scans' block exponent), W_t is stored as 2^-e W_t.
-constexpr int kGatherMaxChunk = 16;
+// Frame sharding: the query frames are fq0 .. fq0 + Fq - 1 of an F-frame clip
+// (fq0 a multiple of chunk), P, Q, their exponents and alpha cover the whole
+// clip, and W_t is written at the query frame's local index t - fq0.
 constexpr int kGatherRows = 32;
 static_assert(kWBlockRows == kGatherRows, "one gather CTA per row block of the W image");
 
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict
                                                          const int* __restrict__ pexp, const int* __restrict__ qexp,
                                                          const float* __restrict__ alpha,
                                                          const float* __restrict__ text, int H, int F, int chunk,
-                                                         int radius, float* __restrict__ W,
+                                                         int radius, int fq0, int Fq, float* __restrict__ W,
                                                          uint16_t* __restrict__ wimg, int* __restrict__ wexp,
                                                          int* __restrict__ wbexp) {
   constexpr int D = 128;
@@ -620,7 +622,7 @@ __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict
   const long long bh = blockIdx.x;
   const int h = (int)(bh % H);
   const long long b = bh / H;
-  const int t0 = blockIdx.y * chunk, t1 = min(F, t0 + chunk);   // query frames of this chunk
+  const int t0 = fq0 + blockIdx.y * chunk, t1 = min(fq0 + Fq, t0 + chunk);   // query frames of this chunk
   int lo, hi;
   window_bounds(t0, F, chunk, radius, lo, hi);
   const float* pre = lo > 0 ? P + (bh * F + (lo - 1)) * D * D : nullptr;
@@ -664,7 +666,7 @@ __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict
   for (int t = t0; t < t1; ++t) {
     const float* dp = dpre[t - t0];
     const float* ds = dsuf[t - t0];
-    const long long fi = bh * F + t;
+    const long long fi = bh * Fq + (t - fq0);
     if (tid == 0 && blockIdx.z == 0) wexp[fi] = ew;
     float w[32];
 #pragma unroll
@@ -712,14 +714,20 @@ __global__ void __launch_bounds__(128) k_gather128_chunk(const float* __restrict
   }
 }
 
+cudaError_t launch_gather_frames(const Args& a, int fq0, int Fq, const float* P, const float* Q, const int* pexp,
+                                 const int* qexp, float* W, uint16_t* wimg, int* wexp, int* wbexp) {
+  if (a.sh.d != 128 || a.chunk > kGatherMaxChunk || fq0 % a.chunk != 0 || Fq < 1 || fq0 + Fq > a.sh.F)
+    return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((Fq + a.chunk - 1) / a.chunk), 128 / kGatherRows);
+  k_gather128_chunk<<<grid, 128, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
+                                                 a.radius, fq0, Fq, W, wimg, wexp, wbexp);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather(const Args& a, const float* P, const float* Q, const int* pexp, const int* qexp, float* W,
                           uint16_t* wimg, int* wexp, int* wbexp) {
-  if (a.sh.d == 128 && a.chunk <= kGatherMaxChunk) {
-    dim3 grid((unsigned)((long long)a.sh.B * a.sh.H), (unsigned)((a.sh.F + a.chunk - 1) / a.chunk), 128 / kGatherRows);
-    k_gather128_chunk<<<grid, 128, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F, a.chunk,
-                                                   a.radius, W, wimg, wexp, wbexp);
-    return cudaGetLastError();
-  }
+  if (a.sh.d == 128 && a.chunk <= kGatherMaxChunk) return launch_gather_frames(a, 0, a.sh.F, P, Q, pexp, qexp, W, wimg,
+                                                                               wexp, wbexp);
   if (a.sh.d == 128) {
     k_gather128<<<(unsigned)a.NF(), 512, 0, a.stream>>>(P, Q, pexp, qexp, a.alpha, a.text_state, a.sh.H, a.sh.F,
                                                         a.chunk, a.radius, W, wimg, wexp, wbexp);

@@ -13,6 +13,12 @@
 // through TMA with a 128-byte swizzle so that each thread reads its own row
 // without bank conflicts.  Only the states the window gather needs are stored:
 // P at chunk ends, Q at chunk starts (or every frame for the debug export).
+//
+// Segment mode (frame sharding): the state restarts at every chunk, from zero
+// with the rule's own coefficients (the chunk's offset O_c) or from the identity
+// with cpre = cpost = 0 (the chunk's linear part G_c = prod D_f N_f), and the
+// state at the chunk's last step in scan order is stored, at its true scale, as
+// the chunk's affine map S -> S G_c + O_c.
 #include "common.cuh"
 #include "image.cuh"
 #include "internal.h"
@@ -61,7 +67,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
                                                             const float* __restrict__ text, RuleCoef rc,
                                                             float* __restrict__ P, float* __restrict__ Q,
                                                             int* __restrict__ pexp, int* __restrict__ qexp, int H,
-                                                            int F, int chunk, int all_frames,
+                                                            int F, int chunk, int all_frames, int seg_mode,
+                                                            float* __restrict__ maps, int nch_stride,
                                                             uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -103,6 +110,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   }
 
   auto frame_of = [&](int step) { return dir == 0 ? step : F - 1 - step; };
+  // segment mode: first and last frame of a chunk in this direction's order
+  auto seg_first = [&](int f) { return dir == 0 ? f % chunk == 0 : ((f + 1) % chunk == 0 || f == F - 1); };
+  auto seg_last = [&](int f) { return dir == 0 ? ((f + 1) % chunk == 0 || f == F - 1) : f % chunk == 0; };
   // N_f image: the hi part (first 32 KB) and the lo part arrive on the same
   // barrier but are requested separately, each as soon as its buffer is free
   auto load_n_part = [&](int step, int part) {
@@ -141,6 +151,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   for (int step = 0; step < F; ++step) {
     const int f = frame_of(step);
     const long long fi = bh * F + f;
+    if (seg_mode != kScanWhole && seg_first(f)) {   // restart: zero, or the identity
+#pragma unroll
+      for (int p = 0; p < 32; ++p)
+        s[p] = seg_mode == kScanSegIdentity ? make_float2(k0 + 2 * p == m ? 1.f : 0.f, k0 + 2 * p + 1 == m ? 1.f : 0.f)
+                                            : make_float2(0.f, 0.f);
+      ex = 0;
+    }
     const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
     if (tid < 128) {
       sm.alpha[tid] = a_next;
@@ -205,8 +222,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     if (tid == 0 && step + 1 < F) load_n_part(step + 1, 1);   // the product that read N_lo is complete
 
     // S_f = D + cpost B_f
-    const bool store = all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0));
-    float* dst = (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0;
+    const bool seg_store = seg_mode != kScanWhole && seg_last(f);
+    const bool store = seg_mode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
+    float* dst = store ? (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0 : nullptr;
+    // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col]
+    float* mdst = seg_store ? maps + ((((bh * 2 + dir) * nch_stride + f / chunk) * 2 +
+                                       (seg_mode == kScanSegIdentity ? 0 : 1)) * 128 + m) * 128 + k0
+                            : nullptr;
+    const float mscale = ldexpf(1.f, ex);
     float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -226,6 +249,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
         amax = fmaxf(amax, fmaxf(fmaxf(fabsf(s[p].x), fabsf(s[p].y)), fmaxf(fabsf(s[p + 1].x), fabsf(s[p + 1].y))));
         if (store)
           *reinterpret_cast<float4*>(dst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
+        if (seg_store)
+          *reinterpret_cast<float4*>(mdst + 32 * j + e) =
+              make_float4(s[p].x * mscale, s[p].y * mscale, s[p + 1].x * mscale, s[p + 1].y * mscale);
       }
     }
     if (store && tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
@@ -251,15 +277,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
 }
 
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
-                           int* qexp, bool all_frames, uint32_t* status) {
+                           int* qexp, bool all_frames, uint32_t* status, int seg_mode, float* maps, int nch_stride) {
   CUtensorMap tmB;
   if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
   size_t smem = sizeof(ScanSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   RuleCoef rc = rule_coef(a.rule, a.c);
+  if (seg_mode == kScanSegIdentity) rc.cpre = rc.cpost = 0.f;   // the linear part alone
   k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
-      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, status);
+      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, seg_mode,
+      maps, nch_stride, status);
   return cudaGetLastError();
 }
 

@@ -636,3 +636,229 @@ const char* vdn_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------- frame sharding
+namespace {
+
+struct FramePart {
+  int f0 = 0, F_local = 0, nch_total = 0, nch_stride = 0;
+};
+
+// rank's frames: a contiguous run of whole chunks (the clip's last chunk may be short)
+vdn_status frame_part(int F_total, int world, int rank, int chunk, FramePart& fp) {
+  if (F_total < 1 || chunk < 1 || world < 1 || rank < 0 || rank >= world) return VDN_ERR_INVALID_ARG;
+  const long long C = ((long long)F_total + chunk - 1) / chunk;
+  if (world > C) return VDN_ERR_INVALID_ARG;   // every rank owns at least one chunk
+  int c0, c1;
+  chunk_range((int)C, world, rank, c0, c1);
+  const long long f1 = (long long)c1 * chunk < F_total ? (long long)c1 * chunk : F_total;
+  fp.f0 = (int)((long long)c0 * chunk);
+  fp.F_local = (int)(f1 - fp.f0);
+  fp.nch_total = (int)C;
+  fp.nch_stride = (int)((C + world - 1) / world);
+  return VDN_OK;
+}
+
+size_t frame_map_bytes(const vdn_shape& sh, const FramePart& fp) {
+  return (size_t)sh.B * sh.H * 2 * fp.nch_stride * 2 * sh.d * sh.d * sizeof(float);
+}
+
+// workspace of the second phase: the clip's chunk-edge states and the rank's read-out images
+struct FramesPlan {
+  size_t status = 0, P = 0, Q = 0, pexp = 0, qexp = 0, wimg = 0, wexp = 0, wbexp = 0, total = 0;
+};
+FramesPlan plan_frames(const vdn_shape& local, int F_total) {
+  FramesPlan p;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t BH = (size_t)local.B * local.H, d = (size_t)local.d;
+  const size_t NFg = BH * F_total, NFl = BH * local.F;
+  p.status = take(256);
+  p.P = take(NFg * d * d * sizeof(float));
+  p.Q = take(NFg * d * d * sizeof(float));
+  p.pexp = take(NFg * sizeof(int));
+  p.qexp = take(NFg * sizeof(int));
+  p.wimg = take(NFl * (size_t)kWImgBytes);
+  p.wexp = take(NFl * sizeof(int));
+  p.wbexp = take(NFl * kWRowBlocks * sizeof(int));
+  p.total = off;
+  return p;
+}
+
+// shape, partition and scalar checks shared by both phases
+vdn_status check_frames(const vdn_shape* local, int F_total, int world, int rank, int rule, float c, int chunk,
+                        FramePart& fp) {
+  vdn_status s = check_shape(local);
+  if (s != VDN_OK) return s;
+  if (local->dtype != VDN_DTYPE_BF16 || local->d != 128) return VDN_ERR_UNSUPPORTED;   // tensor-core path only
+  if (chunk > kGatherMaxChunk) return VDN_ERR_UNSUPPORTED;
+  if (rule < VDN_RULE_SANA_SCALED || rule > VDN_RULE_ADDITIVE || !std::isfinite(c)) return VDN_ERR_INVALID_ARG;
+  s = frame_part(F_total, world, rank, chunk, fp);
+  if (s != VDN_OK) return s;
+  if (local->F != fp.F_local) return VDN_ERR_INVALID_ARG;
+  vdn_shape g = *local;
+  g.F = F_total;
+  return check_shape(&g);   // the clip-wide banks obey the same index limits
+}
+
+size_t frames_workspace(const vdn_shape& local, int F_total, int rule) {
+  size_t a = plan_workspace(local, rule, true).total, b = plan_frames(local, F_total).total;
+  return a > b ? a : b;
+}
+
+Args frame_args(const vdn_shape& sh, int rule, float c, int chunk, int radius, void* stream) {
+  Args a{};
+  a.sh = sh;
+  a.rule = rule;
+  a.c = (rule == VDN_RULE_VDN_SOLVE || rule == VDN_RULE_ADDITIVE) ? 1.0f : c;
+  a.chunk = chunk;
+  a.radius = radius;
+  a.stream = (cudaStream_t)stream;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+vdn_status vdn_frame_range(int F_total, int world, int rank, int chunk, int* f0, int* f1) {
+  if (!f0 || !f1) return VDN_ERR_INVALID_ARG;
+  FramePart fp;
+  vdn_status s = frame_part(F_total, world, rank, chunk, fp);
+  if (s != VDN_OK) return s;
+  *f0 = fp.f0;
+  *f1 = fp.f0 + fp.F_local;
+  return VDN_OK;
+}
+
+vdn_status vdn_frame_owner(int F_total, int world, int chunk, int frame, int* rank) {
+  if (!rank || frame < 0 || frame >= F_total) return VDN_ERR_INVALID_ARG;
+  FramePart fp;
+  vdn_status s = frame_part(F_total, world, 0, chunk, fp);
+  if (s != VDN_OK) return s;
+  int j;
+  chunk_owner(frame / chunk, fp.nch_total, world, *rank, j);
+  return VDN_OK;
+}
+
+size_t vdn_frames_map_bytes(const vdn_shape* shape, int F_total, int world, int rank, int chunk) {
+  FramePart fp;
+  if (check_frames(shape, F_total, world, rank, VDN_RULE_VDN_SOLVE, 1.0f, chunk, fp) != VDN_OK) return 0;
+  return frame_map_bytes(*shape, fp);
+}
+
+size_t vdn_frames_workspace_size(const vdn_shape* shape, int F_total, int world, int rank, int rule, int chunk) {
+  FramePart fp;
+  if (check_frames(shape, F_total, world, rank, rule, 1.0f, chunk, fp) != VDN_OK) return 0;
+  return frames_workspace(*shape, F_total, rule);
+}
+
+vdn_status vdn_frames_maps(const vdn_shape* shape, int F_total, int world, int rank, const void* k, const void* v,
+                           const float* beta, const float* alpha, const float* conv_k_w, const float* conv_v_w,
+                           int rule, float c, int chunk, void* workspace, size_t workspace_bytes, float* maps,
+                           size_t maps_bytes, void* stream) {
+  FramePart fp;
+  vdn_status s = check_frames(shape, F_total, world, rank, rule, c, chunk, fp);
+  if (s != VDN_OK) return s;
+  if (!k || !v || !beta || !alpha || !maps || !workspace) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {k, v, beta, alpha, conv_k_w, conv_v_w, maps};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  if (!aligned(workspace, 256)) return VDN_ERR_ALIGNMENT;
+  const size_t need = frames_workspace(*shape, F_total, rule);
+  if (workspace_bytes < need) return VDN_ERR_WORKSPACE;
+  const size_t mb = frame_map_bytes(*shape, fp);
+  if (maps_bytes < mb) return VDN_ERR_INVALID_ARG;
+  const size_t tok = (size_t)shape->B * shape->F * shape->S * shape->H, d = (size_t)shape->d;
+  const size_t big = tok * d * 2;
+  Range rm{(uintptr_t)maps, (uintptr_t)maps + mb};
+  Range rin[] = {
+      {(uintptr_t)k, (uintptr_t)k + big},
+      {(uintptr_t)v, (uintptr_t)v + big},
+      {(uintptr_t)beta, (uintptr_t)beta + tok * 4},
+      {(uintptr_t)alpha, (uintptr_t)alpha + (size_t)shape->B * shape->F * shape->H * d * 4},
+      {(uintptr_t)conv_k_w, conv_k_w ? (uintptr_t)conv_k_w + (size_t)shape->H * d * shape->conv_width * 4 : 0},
+      {(uintptr_t)conv_v_w, conv_v_w ? (uintptr_t)conv_v_w + (size_t)shape->H * d * shape->conv_width * 4 : 0},
+      {(uintptr_t)workspace, (uintptr_t)workspace + need},
+  };
+  for (const Range& r : rin)
+    if (r.hi > r.lo && overlap(rm, r)) return VDN_ERR_INVALID_ARG;
+
+  Args a = frame_args(*shape, rule, c, chunk, 0, stream);
+  a.k = k; a.v = v; a.beta = beta; a.alpha = alpha;
+  a.conv_k_w = conv_k_w; a.conv_v_w = conv_v_w;
+  WsPlan p = plan_workspace(*shape, rule, true);
+  uint32_t* status = at<uint32_t>(workspace, p.status);
+  float* part = at<float>(workspace, p.part);
+  float* Bsum = at<float>(workspace, p.Bm);
+  uint16_t* nimg = at<uint16_t>(workspace, p.nimg);
+  VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), a.stream));
+  VDN_LAUNCH(launch_stats_tc(a, part, status));
+  VDN_LAUNCH(launch_solve(a, nullptr, nullptr, nimg, part, Bsum, nullptr));
+  VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, nullptr, nullptr, nullptr, nullptr, false, status, kScanSegZero, maps,
+                            fp.nch_stride));
+  VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, nullptr, nullptr, nullptr, nullptr, false, status, kScanSegIdentity, maps,
+                            fp.nch_stride));
+  return VDN_OK;
+}
+
+vdn_status vdn_frames_finish(const vdn_shape* shape, int F_total, int world, int rank, const void* q,
+                             const float* alpha_all, const void* gate, const float* rms_w, const float* text_state,
+                             int rule, float c, int chunk, int radius, const float* maps_all, size_t maps_all_bytes,
+                             void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  FramePart fp;
+  vdn_status s = check_frames(shape, F_total, world, rank, rule, c, chunk, fp);
+  if (s != VDN_OK) return s;
+  if (radius < 0) return VDN_ERR_INVALID_ARG;
+  if (!q || !alpha_all || !gate || !rms_w || !maps_all || !workspace || !out) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, alpha_all, gate, rms_w, text_state, maps_all, out};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return VDN_ERR_ALIGNMENT;
+  if (!aligned(workspace, 256)) return VDN_ERR_ALIGNMENT;
+  const size_t need = frames_workspace(*shape, F_total, rule);
+  if (workspace_bytes < need) return VDN_ERR_WORKSPACE;
+  const size_t mb = frame_map_bytes(*shape, fp) * (size_t)world;
+  if (maps_all_bytes < mb) return VDN_ERR_INVALID_ARG;
+  const size_t tok = (size_t)shape->B * shape->F * shape->S * shape->H, d = (size_t)shape->d;
+  const size_t big = tok * d * 2;
+  Range ro{(uintptr_t)out, (uintptr_t)out + big};
+  Range rin[] = {
+      {(uintptr_t)q, (uintptr_t)q + big},
+      {(uintptr_t)gate, (uintptr_t)gate + big},
+      {(uintptr_t)alpha_all, (uintptr_t)alpha_all + (size_t)shape->B * F_total * shape->H * d * 4},
+      {(uintptr_t)rms_w, (uintptr_t)rms_w + d * 4},
+      {(uintptr_t)text_state, text_state ? (uintptr_t)text_state + (size_t)shape->H * d * d * 4 : 0},
+      {(uintptr_t)maps_all, (uintptr_t)maps_all + mb},
+      {(uintptr_t)workspace, (uintptr_t)workspace + need},
+  };
+  for (const Range& r : rin)
+    if (r.hi > r.lo && overlap(ro, r)) return VDN_ERR_INVALID_ARG;
+
+  vdn_shape g = *shape;
+  g.F = F_total;
+  Args ag = frame_args(g, rule, c, chunk, radius, stream);   // the clip: fold and gather
+  ag.alpha = alpha_all;
+  ag.text_state = text_state;
+  Args al = frame_args(*shape, rule, c, chunk, radius, stream);   // the rank's frames: read-out
+  al.q = q; al.gate = gate; al.rms_w = rms_w; al.out = out;
+  FramesPlan p = plan_frames(*shape, F_total);
+  uint32_t* status = at<uint32_t>(workspace, p.status);
+  float *P = at<float>(workspace, p.P), *Q = at<float>(workspace, p.Q);
+  int *pexp = at<int>(workspace, p.pexp), *qexp = at<int>(workspace, p.qexp);
+  uint16_t* wimg = at<uint16_t>(workspace, p.wimg);
+  int *wexp = at<int>(workspace, p.wexp), *wbexp = at<int>(workspace, p.wbexp);
+  const size_t NFg = (size_t)g.B * g.H * F_total;
+  VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), ag.stream));
+  VDN_LAUNCH(cudaMemsetAsync(pexp, 0, NFg * sizeof(int), ag.stream));   // the folded states carry no exponent
+  VDN_LAUNCH(cudaMemsetAsync(qexp, 0, NFg * sizeof(int), ag.stream));
+  VDN_LAUNCH(launch_fold_maps(ag, maps_all, world, fp.nch_stride, P, Q));
+  VDN_LAUNCH(launch_gather_frames(ag, fp.f0, fp.F_local, P, Q, pexp, qexp, nullptr, wimg, wexp, wbexp));
+  VDN_LAUNCH(launch_readout_tc(al, wimg, wexp, wbexp, status));
+  return VDN_OK;
+}
+
+}  // extern "C"

@@ -68,6 +68,11 @@ def reduce_shared_grads(grads: dict, group=None) -> dict:
 # lie on another rank: those boundary states make the second, equally small exchange.  The
 # functions below fix who owns which frames and which states cross; the arithmetic runs on the
 # device.
+#
+# The device path (vdn_frames_maps / vdn_frames_finish) takes the exchange one step further: each
+# rank publishes the affine map of every one of its chunks (not one per rank), so after a single
+# all-gather every rank folds the maps into every chunk-edge state itself, and no state needs a
+# second exchange.  frame_sharded_forward runs that sequence.
 
 def _window(t: int, F: int, chunk: int, radius: int) -> tuple[int, int]:
     # chunk-aligned window of query frame t: its chunk widened by `radius` chunks each side
@@ -109,3 +114,45 @@ def published_states(F: int, world: int, rank: int, chunk: int, radius: int) -> 
             pre.update(f for f in p if f0 <= f < f1)
             suf.update(f for f in s if f0 <= f < f1)
     return sorted(pre), sorted(suf)
+
+
+TOKEN_AXIS = {"q": 1, "k": 1, "v": 1, "gate": 1, "beta": 1, "q_rope": 1, "k_rope": 1, "dout": 1}
+
+
+def frame_inputs(inputs: dict, F: int, world: int, rank: int, chunk: int) -> dict:
+    """The rank's share of a synth-style input dict under frame sharding: the tokens of its frames
+    (q, k, v, gate, beta, ...), alpha of its frames, and alpha of the whole clip as "alpha_all";
+    per-head and shared parameters as they are."""
+    f0, f1 = frame_range(F, world, rank, chunk)
+    S = inputs["q"].shape[1] // F
+    out = {}
+    for name, t in inputs.items():
+        if t is not None and name in TOKEN_AXIS:
+            out[name] = t.narrow(TOKEN_AXIS[name], f0 * S, (f1 - f0) * S).contiguous()
+        elif name == "alpha":
+            out[name] = t.narrow(1, f0, f1 - f0).contiguous()
+            out["alpha_all"] = t
+        else:
+            out[name] = t
+    return out
+
+
+def frame_sharded_forward(local: dict, F: int, world: int, rank: int, *, rule="vdn_solve", c=1.0, chunk=5,
+                          radius=1, group=None, stream=None):
+    """The branch output of this rank's frames (device tensors from frame_inputs): its chunk maps,
+    one all-gather of every rank's maps (NCCL for CUDA tensors; none with one rank), then the fold,
+    gather and read-out of its frames."""
+    from . import api
+    maps = api.frames_maps(local["k"], local["v"], local["beta"], local["alpha"], local.get("conv_k_w"),
+                           local.get("conv_v_w"), F_total=F, world=world, rank=rank, rule=rule, c=c, chunk=chunk,
+                           stream=stream)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        maps_all = torch.empty(world * maps.numel(), dtype=maps.dtype, device=maps.device)
+        dist.all_gather_into_tensor(maps_all, maps, group=group)
+    else:
+        maps_all = maps
+    return api.frames_finish(local["q"], local["alpha_all"], local["gate"], local["rms_w"], local.get("text_state"),
+                             maps_all, F_total=F, world=world, rank=rank, rule=rule, c=c, chunk=chunk, radius=radius,
+                             stream=stream)
