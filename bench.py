@@ -714,6 +714,117 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
     }), flush=True)
 
 
+def run_gpu_frames(args, w: synth.Workload) -> None:
+    """The linear branch of ONE clip split by frames across the ranks (strong scaling): each rank
+    writes the affine maps of its chunks, one all-gather gives every rank every map, and each rank
+    folds them, gathers and reads out its own frames (the step shard.frame_sharded_forward runs).
+    Per-kernel events are not recorded in this mode: the roofline is the rank's share of the path."""
+    from video_diffusion_linear_b200 import _lib, api
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    _lib.load()
+    if world > -(-w.F // w.chunk):
+        raise SystemExit(f"--shard frames needs at most {-(-w.F // w.chunk)} ranks (one chunk each)")
+    host = shard.frame_inputs(synth.make_inputs(w), w.F, world, rank, w.chunk)
+    f0, f1 = shard.frame_range(w.F, world, rank, w.chunk)
+    wr = w.replace(F=f1 - f0)
+    dev = api.to_device(host, device)
+    stream = torch.cuda.current_stream(device)
+    shape = api.shape_from(dev["q"], wr.F, dev["conv_k_w"])
+    ws = torch.empty(api.frames_workspace_size(shape, w.F, world, rank, w.rule, w.chunk), dtype=torch.uint8,
+                     device=device)
+    nmap = api.frames_map_bytes(shape, w.F, world, rank, w.chunk) // 4
+    maps = torch.empty(nmap, dtype=torch.float32, device=device)
+    maps_all = torch.empty(world * nmap, dtype=torch.float32, device=device) if world > 1 else maps
+    out = torch.empty_like(dev["q"])
+    kw = dict(F_total=w.F, world=world, rank=rank, rule=w.rule, c=w.c, chunk=w.chunk, workspace=ws, stream=stream)
+
+    def step():
+        api.frames_maps(dev["k"], dev["v"], dev["beta"], dev["alpha"], dev["conv_k_w"], dev["conv_v_w"], maps=maps,
+                        **kw)
+        if world > 1:
+            dist.all_gather_into_tensor(maps_all, maps)
+        api.frames_finish(dev["q"], dev["alpha_all"], dev["gate"], dev["rms_w"], dev["text_state"], maps_all,
+                          radius=w.radius, out=out, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if api.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ms_max = reduce_max(start.elapsed_time(end), device)
+    value = w.tokens * args.steps / (ms_max / 1e3)
+    peaks, peak_src = load_peaks()
+    pr = path_roofline(wr, peaks)
+    step_us = ms_max / args.steps * 1e3
+    achieved = pr["bytes"] / (step_us / 1e6) / 1e9
+    roof = {"kernel": "whole path, this rank's frames (per-kernel events not recorded with --shard frames)",
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": pr["bytes"], "traffic": None}
+
+    e2e = None
+    if not args.no_e2e:
+        keys = ["q", "k", "v", "beta", "alpha", "gate"]
+        pinned = {k: host[k].pin_memory() for k in keys}
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
+        d2h = out_host.numel() * out_host.element_size()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+        e2e = {"value": w.tokens * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w), "global_batch": w.B, "tokens_per_step": w.tokens,
+                   "l2": "inputs larger than L2 (q, k, v, gate: %.2f GB per step per GPU)"
+                         % (4 * wr.tokens * wr.H * wr.d * 2 / 1e9),
+                   "parallelism": f"frames{world}: one clip, frames {f0}..{f1 - 1} on rank 0 of {world}, one "
+                                  "all-gather of per-chunk maps per step"},
+        "roofline": roof,
+        "path_roofline": {"t_roof_us": pr["t_roof_us"], "t_step_us": step_us, "frac": pr["t_roof_us"] / step_us,
+                          "bound": pr["bound"], "peaks": peaks, "peak_source": peak_src},
+        "cpu_baseline": None,
+        "e2e": e2e,
+        "gpu_launches": 7 * args.steps,
+        "clocks": clk.summary(),
+    }), flush=True)
+
+
 def run_gpu(args, w: synth.Workload) -> None:
     from video_diffusion_linear_b200 import _lib, api
     rank, world, local = dist_env()
@@ -869,14 +980,16 @@ def main(argv=None):
                     help="linear branch (default), windowed softmax branch, the whole hybrid layer, or the "
                          "linear branch's backward pass")
     ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
-    ap.add_argument("--shard", default="clips", choices=["clips", "heads"],
-                    help="multi-GPU: independent clips per rank (weak scaling, default) or one clip with its "
-                         "heads split across the ranks (strong scaling)")
+    ap.add_argument("--shard", default="clips", choices=["clips", "heads", "frames"],
+                    help="multi-GPU: independent clips per rank (weak scaling, default), one clip with its "
+                         "heads split across the ranks, or (linear path) one clip split by frames (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.shard == "heads" and args.impl == "reference":
-        ap.error("--shard heads applies to the GPU arm")
+    if args.shard != "clips" and args.impl == "reference":
+        ap.error("--shard applies to the GPU arm")
+    if args.shard == "frames" and args.path != "linear":
+        ap.error("--shard frames applies to the linear branch path")
     w = synth.WORKLOADS[args.workload]
     if args.rule:
         w = w.replace(rule=args.rule)
@@ -890,6 +1003,8 @@ def main(argv=None):
         run_gpu_backward(args, w)
     elif args.path != "linear":
         run_gpu_softmax(args, w)
+    elif args.shard == "frames":
+        run_gpu_frames(args, w)
     else:
         run_gpu(args, w)
 
