@@ -321,3 +321,110 @@ def test_chunk_maps_fold_into_the_scans_chunk_edge_states(rule, c, F, chunk):
         G, Oc = chunk_map(fr[::-1])
         s = s @ G + Oc
         np.testing.assert_allclose(s, Q[fr[0]], rtol=1e-10, atol=1e-10 * np.abs(Q).max())
+
+
+# ----------------------------------------------------------------------------- frame-sharded orchestration
+def _fake_frames_maps(k, v, beta, alpha, conv_k_w, conv_v_w, *, F_total, world, rank, rule, c, chunk, **_):
+    """vdn_frames_maps in the oracle's arithmetic, in the header's layout:
+    [B*H][2 directions][nch][G_c | O_c][d][d], nch = ceil(C / world), float64 here."""
+    f0, f1 = shard.frame_range(F_total, world, rank, chunk)
+    n = f1 - f0
+    B, N, H, d = k.shape
+    S = N // n
+    nch = -(-(-(-F_total // chunk)) // world)
+    maps = np.full((B, H, 2, nch, 2, d, d), np.nan)
+    eye, zero = np.eye(d), np.zeros((d, d))
+    for b in range(B):
+        for h in range(H):
+            kh, vh = O._f64(k[b, :, h]), O._f64(v[b, :, h])
+            _, kf, vf = O.prepare_features(kh, kh, vh, n, S, O._f64(conv_k_w[h]), O._f64(conv_v_w[h]))
+            A, Bm = O.frame_statistics(kf, vf, O._f64(beta[b, :, h]).reshape(n, S))
+            al = O._f64(alpha[b, :, h])
+            for j, c0 in enumerate(range(0, n, chunk)):
+                frames = list(range(c0, min(n, c0 + chunk)))
+                for dr, order in ((0, frames), (1, frames[::-1])):
+                    g, o = eye, zero
+                    for f in order:
+                        g = O.rule_step(g, A[f], zero, al[f], rule, c)
+                        o = O.rule_step(o, A[f], Bm[f], al[f], rule, c)
+                    maps[b, h, dr, j] = g, o
+    return torch.from_numpy(maps.ravel())
+
+
+def _fake_frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_total, world, rank, rule, c, chunk,
+                        radius, **_):
+    """vdn_frames_finish in the oracle's arithmetic: fold every rank's maps (rank-major, as the
+    all-gather lays them out) into the chunk-edge states, gather and read out the rank's frames."""
+    f0, f1 = shard.frame_range(F_total, world, rank, chunk)
+    n = f1 - f0
+    B, N, H, d = q.shape
+    S = N // n
+    C = -(-F_total // chunk)
+    nch = -(-C // world)
+    maps = maps_all.numpy().reshape(world, B, H, 2, nch, 2, d, d)
+    first = [shard.frame_range(F_total, world, r, chunk)[0] // chunk for r in range(world)]
+    owner = lambda ch: max(r for r in range(world) if first[r] <= ch)
+    out = np.empty((B, N, H, d))
+    for b in range(B):
+        for h in range(H):
+            seed = O.seed_state(None if text_state is None else O._f64(text_state[h]), d)
+            P = np.full((F_total, d, d), np.nan)
+            Q = np.full((F_total, d, d), np.nan)
+            s = seed
+            for ch in range(C - 1):
+                r = owner(ch)
+                g, o = maps[r, b, h, 0, ch - first[r]]
+                s = s @ g + o
+                P[(ch + 1) * chunk - 1] = s
+            s = seed
+            for ch in range(C - 1, 0, -1):
+                r = owner(ch)
+                g, o = maps[r, b, h, 1, ch - first[r]]
+                s = s @ g + o
+                Q[ch * chunk] = s
+            qh = O._f64(q[b, :, h])
+            qf, _, _ = O.prepare_features(qh, qh, qh, n, S)
+            g = O._f64(gate[b, :, h]).reshape(n, S, d)
+            al = O._f64(alpha_all[b, :, h])
+            for t in range(f0, f1):
+                W_t = O.gather_state(P, Q, seed, al, t, chunk, radius)
+                out[b, (t - f0) * S:(t - f0 + 1) * S, h] = O.readout(W_t, qf[t - f0], g[t - f0], O._f64(rms_w))
+    return torch.from_numpy(out)
+
+
+def _orchestration_worker(rank, world, port, w, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from video_diffusion_linear_b200 import api
+        api.frames_maps, api.frames_finish = _fake_frames_maps, _fake_frames_finish
+        local = shard.frame_inputs(synth.make_inputs(w), w.F, world, rank, w.chunk)
+        out = shard.frame_sharded_forward(local, w.F, world, rank, rule=w.rule, c=w.c, chunk=w.chunk,
+                                          radius=w.radius)
+        got = [None] * world
+        dist.all_gather_object(got, out)
+        if rank == 0:
+            q.put(torch.cat(got, dim=1).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("w,world", [(FRAME_CASES[0], 3), (FRAME_CASES[1].replace(B=2), 2)],
+                         ids=["solve_3", "sana_2"])
+def test_frame_sharded_forward_orchestration_on_gloo_ranks(w, world):
+    """shard.frame_sharded_forward on gloo ranks, its two device phases stood in for by the oracle
+    following the header's map layout: the all-gather's rank order, the padding of the map buffers
+    to ceil(C / world) chunks and the frame slicing give the whole clip's output."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_orchestration_worker, args=(r, world, port, w, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    joined = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ref = O.branch_forward(synth.make_inputs(w), w.F, w.S, w.rule, w.c, w.chunk, w.radius)
+    assert np.isfinite(joined).all()
+    np.testing.assert_allclose(joined, ref, rtol=1e-9, atol=1e-11 * np.abs(ref).max())
