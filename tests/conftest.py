@@ -21,7 +21,7 @@ def lib():
 
 # Modules of paths that have not yet been through a hardware run: they go last, so that under -x
 # a failure there does not stop the established parity tests.
-RUN_LAST = ("test_gpu_frames.py",)
+RUN_LAST = ("test_gpu_sharding.py",)
 
 
 def pytest_collection_modifyitems(config, items):

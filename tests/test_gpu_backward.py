@@ -151,27 +151,3 @@ def test_save_for_backward_matches_the_recomputing_pair(w):
         if ref[n] is not None:
             assert torch.equal(got[n], ref[n]), n
 
-
-@pytest.mark.parametrize("world", [2, 3])
-def test_head_sharded_backward_reassembles_the_clip(world):
-    """Each rank's backward call on its slice of the heads (run one after another: the calls never
-    wait on one another); the per-head gradients join along the head axis and the rms_w gradient,
-    which every head shares, is the sum of the ranks' partials (what shard.reduce_shared_grads
-    all-reduces across GPUs)."""
-    from video_diffusion_linear_b200 import shard
-    w = BF16[0].replace(name="bw_bf16_shard", H=3)
-    inp = synth.make_inputs(w)
-    dout = synth.make_cotangent(w)
-    full = dict(inp, dout=dout)
-    parts = []
-    for r in range(world):
-        part = shard.shard_inputs(full, world, r)
-        dev = api.to_device(part)
-        parts.append(api.branch_backward(*api.forward_inputs(dev), dout=dev["dout"], F=w.F, rule=w.rule, c=w.c,
-                                         chunk=w.chunk, radius=w.radius))
-    torch.cuda.synchronize()
-    got = {n: None if parts[0][n] is None else
-           (sum(p[n] for p in parts) if n in shard.SHARED_GRADS else
-            torch.cat([p[n] for p in parts], dim=shard.PER_HEAD[n])) for n in NAMES}
-    ref = BW.branch_backward(inp, dout, w.F, w.S, w.rule, w.c, w.chunk, w.radius)
-    _compare(w, got, ref, TOL_BF16)

@@ -1,12 +1,16 @@
-"""GPU parity of the frame-sharded branch (vdn_frames_maps, then vdn_frames_finish) through the
-C ABI: the ranks run one after another on one GPU (their calls never wait on one another; the
-all-gather of the maps is a concatenation here), and the joined output must match the float64
-oracle of the whole clip within the bf16 bound, and the unsharded call."""
+"""GPU parity of the sharded paths that have not yet been through a hardware run, through the C ABI;
+the ranks run one after another on one GPU (their calls never wait on one another, and the
+collectives become concatenations and sums):
+  * the frame-sharded branch (vdn_frames_maps, then vdn_frames_finish): the joined output against
+    the float64 oracle of the whole clip within the bf16 bound, and against the unsharded call;
+  * the head-sharded backward: per-head gradients joined, the rms_w gradient summed."""
 import numpy as np
 import pytest
 import torch
 
 from harness import TOL_BF16, gpu_forward, oracle_forward, rel_err, to_np
+from oracle import vdn_backward as BW
+from test_gpu_backward import BF16, NAMES, _compare
 from video_diffusion_linear_b200 import api, shard, synth
 
 pytestmark = pytest.mark.gpu
@@ -53,3 +57,27 @@ def test_one_rank_equals_the_unsharded_call():
     joined = _sharded(w, inp, 1)
     full, _ = gpu_forward(w, inp)
     assert rel_err(to_np(joined), to_np(full)) <= 1e-2
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_sharded_backward_reassembles_the_clip(world):
+    """Each rank's backward call on its slice of the heads (run one after another: the calls never
+    wait on one another); the per-head gradients join along the head axis and the rms_w gradient,
+    which every head shares, is the sum of the ranks' partials (what shard.reduce_shared_grads
+    all-reduces across GPUs)."""
+    w = BF16[0].replace(name="bw_bf16_shard", H=3)
+    inp = synth.make_inputs(w)
+    dout = synth.make_cotangent(w)
+    full = dict(inp, dout=dout)
+    parts = []
+    for r in range(world):
+        part = shard.shard_inputs(full, world, r)
+        dev = api.to_device(part)
+        parts.append(api.branch_backward(*api.forward_inputs(dev), dout=dev["dout"], F=w.F, rule=w.rule, c=w.c,
+                                         chunk=w.chunk, radius=w.radius))
+    torch.cuda.synchronize()
+    got = {n: None if parts[0][n] is None else
+           (sum(p[n] for p in parts) if n in shard.SHARED_GRADS else
+            torch.cat([p[n] for p in parts], dim=shard.PER_HEAD[n])) for n in NAMES}
+    ref = BW.branch_backward(inp, dout, w.F, w.S, w.rule, w.c, w.chunk, w.radius)
+    _compare(w, got, ref, TOL_BF16)
