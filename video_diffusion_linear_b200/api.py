@@ -24,6 +24,47 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _validate(specs, device) -> None:
+    """Checks (name, tensor, shape, dtype, optional) specs before any pointer reaches the library:
+    the kernels read each buffer with the element type and extent vdn.h fixes, so a tensor of
+    another dtype, shape or device would be read out of its bounds."""
+    if device.type != "cuda":
+        raise ValueError(f"libvdn takes CUDA tensors, got a tensor on {device}")
+    for name, t, shape, dtype, optional in specs:
+        if t is None:
+            if optional:
+                continue
+            raise ValueError(f"{name} is required")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {device}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _bytes(name, t, device) -> None:
+    """A caller-owned byte buffer (workspace, saved state): a uint8 CUDA tensor on `device`, whose
+    numel is the byte count the library is told."""
+    if t is None:
+        return
+    if t.device != device or t.dtype != torch.uint8:
+        raise ValueError(f"{name} must be a uint8 tensor on {device}, got {t.dtype} on {t.device}")
+
+
+def _branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out=None):
+    """Specs of the branch's inputs (vdn.h, vdn_branch_forward) for q of shape [B, F*S, H, d]."""
+    B, N, H, d = q.shape
+    f32 = torch.float32
+    K = conv_k_w.shape[-1] if conv_k_w is not None else (conv_v_w.shape[-1] if conv_v_w is not None else 1)
+    return [("q", q, (B, N, H, d), q.dtype, False), ("k", k, (B, N, H, d), q.dtype, False),
+            ("v", v, (B, N, H, d), q.dtype, False), ("gate", gate, (B, N, H, d), q.dtype, False),
+            ("beta", beta, (B, N, H), f32, False), ("alpha", alpha, (B, F, H, d), f32, False),
+            ("rms_w", rms_w, (d,), f32, False), ("conv_k_w", conv_k_w, (H, d, K), f32, True),
+            ("conv_v_w", conv_v_w, (H, d, K), f32, True), ("text_state", text_state, (H, d, d), f32, True),
+            ("out", out, (B, N, H, d), q.dtype, True)]
+
+
 def _stream_ptr(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -66,10 +107,12 @@ def branch_forward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=No
                    F: int, rule="vdn_solve", c=1.0, chunk=5, radius=1, out=None, workspace=None, stream=None):
     """vdn_branch_forward: the whole branch.  Returns `out` ([B, F*S, H, d], q's dtype)."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate(_branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out), q.device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(shape, rule, "auto", q.device)
+    _bytes("workspace", workspace, q.device)
     st = _lib.load().vdn_branch_forward(*_forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w,
                                                        conv_v_w, text_state, rule, c, chunk, radius, workspace,
                                                        out, stream))
@@ -82,11 +125,14 @@ def window_softmax_forward(q_rope, k_rope, v, *, F: int, chunk=5, radius=1, scal
     """vdn_window_softmax_forward: the windowed softmax branch (out = or += its
     output).  Returns `out` ([B, F*S, H, d], q_rope's dtype)."""
     shape = shape_from(q_rope, F)
+    _validate([(n, t, q_rope.shape, q_rope.dtype, n == "out") for n, t in
+               (("q_rope", q_rope), ("k_rope", k_rope), ("v", v), ("out", out))], q_rope.device)
     if out is None:
         out = torch.zeros_like(q_rope) if accumulate else torch.empty_like(q_rope)
     if workspace is None:
         workspace = torch.empty(_lib.load().vdn_window_softmax_workspace_size(ctypes.byref(shape)),
                                 dtype=torch.uint8, device=q_rope.device)
+    _bytes("workspace", workspace, q_rope.device)
     st = _lib.load().vdn_window_softmax_forward(ctypes.byref(shape), _ptr(q_rope), _ptr(k_rope), _ptr(v), int(chunk),
                                                 int(radius), float(scale), int(bool(accumulate)), _ptr(workspace),
                                                 workspace.numel(), _ptr(out), _stream_ptr(stream))
@@ -99,10 +145,13 @@ def hybrid_forward(q_rope, k_rope, q, k, v, beta, alpha, gate, rms_w, conv_k_w=N
                    workspace=None, stream=None):
     """vdn_hybrid_forward: windowed softmax branch + linear branch.  Returns `out`."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate(_branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out) +
+              [("q_rope", q_rope, q.shape, q.dtype, False), ("k_rope", k_rope, q.shape, q.dtype, False)], q.device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(shape, rule, "auto", q.device)
+    _bytes("workspace", workspace, q.device)
     fa = _forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
                        radius, workspace, out, stream)
     st = _lib.load().vdn_hybrid_forward(fa[0], _ptr(q_rope), _ptr(k_rope), *fa[1:15], float(scale), *fa[15:])
@@ -121,10 +170,12 @@ def branch_forward_timed(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_
     objects with timing enabled, already recorded once so their handles exist) before the
     first kernel and after each kernel."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate(_branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out), q.device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(shape, rule, "auto", q.device)
+    _bytes("workspace", workspace, q.device)
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     st = _lib.load().vdn_branch_forward_timed(*_forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w,
                                                              conv_v_w, text_state, rule, c, chunk, radius,
@@ -141,10 +192,12 @@ def branch_forward_debug(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_
                          out=None, workspace=None, stream=None):
     """vdn_branch_forward_debug: returns (out, {name: fp32 [B, H, F, d, d]}) for the requested intermediates."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate(_branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out), q.device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(shape, rule, impl, q.device)
+    _bytes("workspace", workspace, q.device)
     B, N, H, d = q.shape
     mats = {name: torch.full((B, H, F, d, d), float("nan"), dtype=torch.float32, device=q.device) for name in want}
     dbg = VdnDebugOut(VDN_IMPL[impl], *[mats[n].data_ptr() if n in mats else None for n in DEBUG_FIELDS])
@@ -158,6 +211,8 @@ def branch_forward_debug(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_
 def feature_prep(q, k, v, conv_k_w=None, conv_v_w=None, *, F: int, stream=None):
     """vdn_feature_prep: Step 1 alone.  Returns (q', k', v') in q's dtype."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate([s for s in _branch_specs(q, k, v, None, None, None, None, conv_k_w, conv_v_w, None, F)
+               if s[0] in ("q", "k", "v", "conv_k_w", "conv_v_w")], q.device)
     qo, ko, vo = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     st = _lib.load().vdn_feature_prep(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_k_w),
                                       _ptr(conv_v_w), _ptr(qo), _ptr(ko), _ptr(vo), _stream_ptr(stream))
@@ -194,12 +249,15 @@ def branch_forward_train(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_
     """vdn_branch_forward_train: the branch's output and the per-frame state its backward
     reads.  Returns (out, saved); pass `saved` to branch_backward(..., saved=saved)."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate(_branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F, out), q.device)
     if out is None:
         out = torch.empty_like(q)
     if saved is None:
         saved = torch.empty(saved_size(shape), dtype=torch.uint8, device=q.device)
     if workspace is None:
         workspace = alloc_workspace(shape, rule, "auto", q.device)
+    _bytes("saved", saved, q.device)
+    _bytes("workspace", workspace, q.device)
     fa = _forward_args(shape, q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, rule, c, chunk,
                        radius, workspace, out, stream)
     st = _lib.load().vdn_branch_forward_train(*fa[:-1], _ptr(saved), saved.numel(), fa[-1])
@@ -230,6 +288,8 @@ def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=N
     vdn_branch_backward_saved runs instead, without the forward recompute."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
     dev = q.device
+    specs = _branch_specs(q, k, v, beta, alpha, gate, rms_w, conv_k_w, conv_v_w, text_state, F)
+    _validate(specs + [("dout", dout, q.shape, q.dtype, False)], dev)
     if grads is None:
         f32 = dict(dtype=torch.float32, device=dev)
         grads = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
@@ -241,6 +301,11 @@ def branch_backward(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_v_w=N
     if workspace is None:
         workspace = torch.empty(backward_workspace_size(shape, rule, saved is not None), dtype=torch.uint8,
                                 device=dev)
+    _bytes("workspace", workspace, dev)
+    _bytes("saved", saved, dev)
+    # each gradient has its input's shape: q's dtype for the token tensors, fp32 for the rest
+    _validate([("d" + n, grads.get("d" + n), shp, dt if n in ("q", "k", "v", "gate") else torch.float32, True)
+               for n, _, shp, dt, _ in specs if n != "out"], dev)
     g = grads
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate), _ptr(rms_w),
             _ptr(conv_k_w), _ptr(conv_v_w), _ptr(text_state), VDN_RULE[rule], float(c), int(chunk), int(radius),
@@ -302,12 +367,16 @@ def frames_maps(k, v, beta, alpha, conv_k_w=None, conv_v_w=None, *, F_total: int
     frames only.  Returns the rank's per-chunk affine maps (flat fp32, frames_map_bytes / 4)."""
     f0, f1 = frame_range(F_total, world, rank, chunk)
     shape = shape_from(k, f1 - f0, conv_k_w if conv_k_w is not None else conv_v_w)
+    _validate([s for s in _branch_specs(k, k, v, beta, alpha, k, None, conv_k_w, conv_v_w, None, f1 - f0)
+               if s[0] in ("k", "v", "beta", "alpha", "conv_k_w", "conv_v_w")], k.device)
     nb = frames_map_bytes(shape, F_total, world, rank, chunk)
     if maps is None:
         maps = torch.empty(nb // 4, dtype=torch.float32, device=k.device)
     if workspace is None:
         workspace = torch.empty(frames_workspace_size(shape, F_total, world, rank, rule, chunk), dtype=torch.uint8,
                                 device=k.device)
+    _validate([("maps", maps, (maps.numel(),), torch.float32, False)], k.device)
+    _bytes("workspace", workspace, k.device)
     st = _lib.load().vdn_frames_maps(ctypes.byref(shape), F_total, world, rank, _ptr(k), _ptr(v), _ptr(beta),
                                      _ptr(alpha), _ptr(conv_k_w), _ptr(conv_v_w), VDN_RULE[rule], float(c),
                                      int(chunk), _ptr(workspace), workspace.numel(), _ptr(maps),
@@ -322,11 +391,18 @@ def frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_total: i
     maps_all every rank's maps in rank order.  Returns the branch output of the rank's frames."""
     f0, f1 = frame_range(F_total, world, rank, chunk)
     shape = shape_from(q, f1 - f0)
+    B, N, H, d = q.shape
+    f32 = torch.float32
+    _validate([("q", q, q.shape, q.dtype, False), ("gate", gate, q.shape, q.dtype, False),
+               ("out", out, q.shape, q.dtype, True), ("alpha_all", alpha_all, (B, F_total, H, d), f32, False),
+               ("rms_w", rms_w, (d,), f32, False), ("text_state", text_state, (H, d, d), f32, True),
+               ("maps_all", maps_all, (maps_all.numel(),), f32, False)], q.device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = torch.empty(frames_workspace_size(shape, F_total, world, rank, rule, chunk), dtype=torch.uint8,
                                 device=q.device)
+    _bytes("workspace", workspace, q.device)
     st = _lib.load().vdn_frames_finish(ctypes.byref(shape), F_total, world, rank, _ptr(q), _ptr(alpha_all),
                                        _ptr(gate), _ptr(rms_w), _ptr(text_state), VDN_RULE[rule], float(c),
                                        int(chunk), int(radius), _ptr(maps_all),
