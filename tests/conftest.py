@@ -18,11 +18,3 @@ def lib():
     from video_diffusion_linear_b200 import _lib
     return _lib.load()
 
-
-# Modules of paths that have not yet been through a hardware run: they go last, so that under -x
-# a failure there does not stop the established parity tests.
-RUN_LAST = ("test_gpu_sharding.py",)
-
-
-def pytest_collection_modifyitems(config, items):
-    items.sort(key=lambda it: os.path.basename(str(it.fspath)) in RUN_LAST)

@@ -1,6 +1,5 @@
-"""GPU parity of the sharded paths that have not yet been through a hardware run, through the C ABI;
-the ranks run one after another on one GPU (their calls never wait on one another, and the
-collectives become concatenations and sums):
+"""GPU parity of the sharded paths through the C ABI; the ranks run one after another on one GPU
+(their calls never wait on one another, and the collectives become concatenations and sums):
   * the frame-sharded branch (vdn_frames_maps, then vdn_frames_finish): the joined output against
     the float64 oracle of the whole clip within the bf16 bound, and against the unsharded call;
   * the head-sharded backward: per-head gradients joined, the rms_w gradient summed."""
