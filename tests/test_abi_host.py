@@ -244,3 +244,17 @@ def test_hybrid_validation(lib):
     assert call(qr_=ctypes.c_void_p(BASE + 20 * GAP + 4)) == VDN_ERR_ALIGNMENT
     assert call(out=ctypes.c_void_p(BASE + 21 * GAP + 256)) == VDN_ERR_INVALID_ARG   # out overlaps k_rope
     assert call(out=ctypes.c_void_p(BASE + 64)) == VDN_ERR_INVALID_ARG               # out overlaps q
+
+
+def test_every_export_is_declared(lib):
+    # the boundary is the header: nothing the library exports is left undocumented
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    out = subprocess.run([nm, "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.split()[-2:-1] == ["T"]}
+    exported = {n for n in exported if n.startswith("vdn_")}
+    assert exported and exported <= set(_lib.header_symbols()), exported - set(_lib.header_symbols())
