@@ -125,3 +125,16 @@ def test_reference_arm_prints_one_contract_line(path, capsys):
     assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 2 and j["warmup"] == 3
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_rank_inputs_split_heads_or_clips():
+    w = synth.WORKLOADS["tiny_f20_text"].replace(H=3)
+    parts = [bench.rank_inputs("heads", w, 2, r) for r in range(2)]
+    assert [p[1].H for p in parts] == [2, 1]
+    assert all(p[2] == w.tokens and p[3]["scaling"] == "strong" and p[3]["global_batch"] == w.B for p in parts)
+    full = synth.make_inputs(w)
+    assert torch.equal(torch.cat([p[0]["q"] for p in parts], dim=2), full["q"])
+    host, wr, job, split = bench.rank_inputs("clips", w, 2, 1, cotangent=True)
+    assert wr.seed != w.seed and job == 2 * w.tokens and split["scaling"] == "weak" and "dout" in host
+    with pytest.raises(SystemExit):
+        bench.rank_inputs("heads", w, 4, 0)
