@@ -258,3 +258,26 @@ def test_every_export_is_declared(lib):
     exported = {ln.split()[-1] for ln in out.splitlines() if ln.split()[-2:-1] == ["T"]}
     exported = {n for n in exported if n.startswith("vdn_")}
     assert exported and exported <= set(_lib.header_symbols()), exported - set(_lib.header_symbols())
+
+
+@pytest.mark.parametrize("kw", [
+    dict(F=70000, S=40000),              # F*S tokens of one batch element past int32
+    dict(B=40000, H=60000, F=1, S=1),    # (batch, head, frame) triples past int32
+    dict(B=1 << 20, H=1 << 11, F=1, S=1),   # 2 B H past int32
+])
+def test_index_ranges_past_int32_are_refused(lib, kw):
+    # the kernels index tokens of one batch element and (batch, head, frame) triples in int32:
+    # shapes beyond that are refused before any allocation or launch, by every entry point
+    s = _shape(**kw)
+    assert lib.vdn_branch_workspace_size(ctypes.byref(s), 1) == 0
+    assert lib.vdn_branch_forward(*_args(s, ws_bytes=1 << 40)) == VDN_ERR_UNSUPPORTED
+    assert lib.vdn_window_softmax_workspace_size(ctypes.byref(s)) == 0
+    assert lib.vdn_branch_backward_workspace_size(ctypes.byref(s), 1) == 0
+
+
+def test_largest_single_gpu_sizes_are_accepted(lib):
+    # the 14 s and 1024^2 clips, and a 4x longer clip: sizes only (nothing runs)
+    for kw in (dict(F=85, S=1560, H=24), dict(B=2, F=31, S=4096, H=24), dict(F=340, S=1560, H=24)):
+        s = _shape(**kw)
+        n = lib.vdn_branch_workspace_size(ctypes.byref(s), 1)
+        assert 0 < n < 180e9
