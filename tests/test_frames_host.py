@@ -149,6 +149,7 @@ def _finish_args(shape, **over):
     (dict(maps_all_bytes=3 * 1024), VDN_ERR_INVALID_ARG),         # fewer than world map buffers
     (dict(ptr=dict(out=BASE + 0 * GAP + 256)), VDN_ERR_INVALID_ARG),   # out inside q
     (dict(ptr=dict(out=BASE + 6 * GAP + 4096)), VDN_ERR_INVALID_ARG),  # out inside the workspace
+    (dict(ptr=dict(maps_all=BASE + 6 * GAP + 1024)), VDN_ERR_INVALID_ARG),  # maps inside the workspace
 ])
 def test_finish_validation(lib, case, expect):
     case = dict(case)

@@ -837,6 +837,9 @@ vdn_status vdn_frames_finish(const vdn_shape* shape, int F_total, int world, int
   };
   for (const Range& r : rin)
     if (r.hi > r.lo && overlap(ro, r)) return VDN_ERR_INVALID_ARG;
+  // the fold reads the maps while it writes the workspace's state banks
+  if (overlap(Range{(uintptr_t)maps_all, (uintptr_t)maps_all + mb}, Range{(uintptr_t)workspace, (uintptr_t)workspace + need}))
+    return VDN_ERR_INVALID_ARG;
 
   vdn_shape g = *shape;
   g.F = F_total;
