@@ -729,6 +729,8 @@ def run_gpu_frames(args, w: synth.Workload) -> None:
     _lib.load()
     if world > -(-w.F // w.chunk):
         raise SystemExit(f"--shard frames needs at most {-(-w.F // w.chunk)} ranks (one chunk each)")
+    if w.dtype != "bf16" or w.d != 128 or w.chunk > 16:
+        raise SystemExit("--shard frames runs the tensor-core path: bf16, d = 128, chunk <= 16")
     host = shard.frame_inputs(synth.make_inputs(w), w.F, world, rank, w.chunk)
     f0, f1 = shard.frame_range(w.F, world, rank, w.chunk)
     wr = w.replace(F=f1 - f0)
