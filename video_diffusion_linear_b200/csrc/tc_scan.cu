@@ -61,13 +61,16 @@ __device__ __forceinline__ void split_pair(float2 x, uint32_t& hi, uint32_t& lo)
   lo = pack_bf16x2(r.x, r.y);
 }
 
+// kMode: kScanWhole (the clip, from the text seed) or a segment mode; a template parameter so that
+// the whole-clip instantiation carries none of the segment mode's work
+template <int kMode>
 __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmB,
                                                             const uint16_t* __restrict__ nimg_g,
                                                             const float* __restrict__ alpha,
                                                             const float* __restrict__ text, RuleCoef rc,
                                                             float* __restrict__ P, float* __restrict__ Q,
                                                             int* __restrict__ pexp, int* __restrict__ qexp, int H,
-                                                            int F, int chunk, int all_frames, int seg_mode,
+                                                            int F, int chunk, int all_frames,
                                                             float* __restrict__ maps, int nch_stride,
                                                             uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -151,11 +154,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   for (int step = 0; step < F; ++step) {
     const int f = frame_of(step);
     const long long fi = bh * F + f;
-    if (seg_mode != kScanWhole && seg_first(f)) {   // restart: zero, or the identity
+    if (kMode != kScanWhole && seg_first(f)) {   // restart: zero, or the identity
 #pragma unroll
       for (int p = 0; p < 32; ++p)
-        s[p] = seg_mode == kScanSegIdentity ? make_float2(k0 + 2 * p == m ? 1.f : 0.f, k0 + 2 * p + 1 == m ? 1.f : 0.f)
-                                            : make_float2(0.f, 0.f);
+        s[p] = kMode == kScanSegIdentity ? make_float2(k0 + 2 * p == m ? 1.f : 0.f, k0 + 2 * p + 1 == m ? 1.f : 0.f)
+                                         : make_float2(0.f, 0.f);
       ex = 0;
     }
     const float cpre = ldexpf(rc.cpre, -ex), cpost = ldexpf(rc.cpost, -ex);
@@ -222,14 +225,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     if (tid == 0 && step + 1 < F) load_n_part(step + 1, 1);   // the product that read N_lo is complete
 
     // S_f = D + cpost B_f
-    const bool seg_store = seg_mode != kScanWhole && seg_last(f);
-    const bool store = seg_mode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
-    float* dst = store ? (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0 : nullptr;
-    // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col]
-    float* mdst = seg_store ? maps + ((((bh * 2 + dir) * nch_stride + f / chunk) * 2 +
-                                       (seg_mode == kScanSegIdentity ? 0 : 1)) * 128 + m) * 128 + k0
-                            : nullptr;
-    const float mscale = ldexpf(1.f, ex);
+    const bool seg_store = kMode != kScanWhole && seg_last(f);
+    const bool store = kMode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
+    float* dst = kMode == kScanWhole ? (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0 : nullptr;
+    // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col], at the true scale 2^ex
+    float* mdst = kMode == kScanWhole ? nullptr
+                                      : maps + ((((bh * 2 + dir) * nch_stride + f / chunk) * 2 +
+                                                 (kMode == kScanSegIdentity ? 0 : 1)) * 128 + m) * 128 + k0;
+    const float mscale = kMode == kScanWhole ? 1.f : ldexpf(1.f, ex);
     float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -281,13 +284,16 @@ cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nim
   CUtensorMap tmB;
   if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
   size_t smem = sizeof(ScanSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   RuleCoef rc = rule_coef(a.rule, a.c);
   if (seg_mode == kScanSegIdentity) rc.cpre = rc.cpost = 0.f;   // the linear part alone
-  k_scan_tc<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
-      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, seg_mode,
-      maps, nch_stride, status);
+  auto kern = seg_mode == kScanSegZero ? k_scan_tc<kScanSegZero>
+              : seg_mode == kScanSegIdentity ? k_scan_tc<kScanSegIdentity> : k_scan_tc<kScanWhole>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
+      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, maps,
+      nch_stride, status);
   return cudaGetLastError();
 }
 
