@@ -32,5 +32,19 @@ int main(void) {
                            (const float*)(base + 4 * gap), base + 5 * gap, (const float*)(base + 6 * gap), NULL, NULL,
                            NULL, VDN_RULE_VDN_SOLVE, 1.0f, 5, 1, base + 7 * gap, fwd, base + 8 * gap, NULL);
     printf("null_q %d %s\n", (int)s, vdn_status_string(s));
+
+    /* frame sharding of the 31-frame clip over 3 ranks in chunks of 5: 7 chunks -> 3, 2, 2 */
+    int f0 = -1, f1 = -1, owner = -1;
+    printf("frames");
+    for (int r = 0; r < 3; ++r) {
+        s = vdn_frame_range(31, 3, r, 5, &f0, &f1);
+        printf(" %d:%d-%d", (int)s, f0, f1);
+    }
+    s = vdn_frame_owner(31, 3, 5, 30, &owner);
+    printf(" owner %d %d\n", (int)s, owner);
+    vdn_shape part = sh;
+    part.F = 15;
+    size_t maps = vdn_frames_map_bytes(&part, 31, 3, 0, 5);
+    printf("map_bytes %d\n", maps == (size_t)24 * 2 * 3 * 2 * 128 * 128 * 4);
     return 0;
 }

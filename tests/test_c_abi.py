@@ -27,3 +27,5 @@ def test_c_caller(tmp_path):
     assert out[2] == "sizes 1 1 1 256"
     assert out[3] == "unsupported 1"
     assert out[4].startswith("null_q 1 ")                 # validation error, before any launch
+    assert out[5] == "frames 0:0-15 0:15-25 0:25-31 owner 0 2"
+    assert out[6] == "map_bytes 1"
