@@ -783,7 +783,7 @@ def run_gpu_frames(args, w: synth.Workload) -> None:
 
     e2e = None
     if not args.no_e2e:
-        keys = ["q", "k", "v", "beta", "alpha", "gate"]
+        keys = ["q", "k", "v", "beta", "alpha", "alpha_all", "gate"]
         pinned = {k: host[k].pin_memory() for k in keys}
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
