@@ -1,4 +1,4 @@
-"""Head sharding of the branch across ranks (one process per GPU).
+"""Sharding of the branch across ranks (one process per GPU): by heads, and by frames (below).
 
 Every step of the branch is per (batch, head): statistics, solve, both scans, gather and read-out
 never mix heads, and neither does the windowed softmax branch.  A clip whose heads are split across
