@@ -8,7 +8,7 @@ import test_oracle_pins as pins
 
 _orig = {name: getattr(O, name) for name in
          ("window_bounds", "frame_statistics", "rule_step", "gather_state", "seed_state",
-          "prepare_features", "readout", "short_conv_frame")}
+          "prepare_features", "readout", "short_conv_frame", "sampled_outputs")}
 
 
 def _window_hi_plus_one(t, F, chunk, radius):
@@ -85,6 +85,27 @@ def _readout_W_transposed(W_t, qf_tokens, gate_tokens, rms_w, prenorm=False):
     return _orig["readout"](W_t.T, qf_tokens, gate_tokens, rms_w, prenorm)
 
 
+def _sampled_with(frame_of, gate_row):
+    """sampled_outputs with its token -> (frame, gate row) indexing replaced."""
+    def mutant(inp, F, S, rule, c, chunk, radius, b, h, tokens, prenorm=False):
+        st = O.head_state(inp, b, h, F, S, rule, c, chunk, radius)
+        rms_w = np.asarray(inp["rms_w"], dtype=np.float64)
+        g = np.asarray(inp["gate"][b, :, h, :], dtype=np.float64)
+        res = np.empty((len(tokens), st["qf"].shape[-1]))
+        for i, n in enumerate(np.asarray(tokens)):
+            t, s = frame_of(int(n), S, F), int(n) % S
+            res[i] = O.readout(st["W"][t], st["qf"][t, s][None, :], g[gate_row(int(n), S)][None, :], rms_w,
+                               prenorm)[0]
+        return res
+    return mutant
+
+
+# the last token of a frame read with the next frame's state
+_sampled_frame_off_by_one = _sampled_with(lambda n, S, F: min((n + 1) // S, F - 1), lambda n, S: n)
+# the gate row taken frame-local (token s of frame 0) instead of clip-wide
+_sampled_gate_frame_local = _sampled_with(lambda n, S, F: n // S, lambda n, S: n % S)
+
+
 MUTANTS = {
     "window_hi_plus_one": ("window_bounds", _window_hi_plus_one),
     "stats_B_transposed": ("frame_statistics", _stats_B_transposed),
@@ -100,6 +121,8 @@ MUTANTS = {
     "conv_flipped": ("short_conv_frame", _conv_flipped),
     "readout_no_gate": ("readout", _readout_no_gate),
     "readout_W_transposed": ("readout", _readout_W_transposed),
+    "sampled_frame_off_by_one": ("sampled_outputs", _sampled_frame_off_by_one),
+    "sampled_gate_frame_local": ("sampled_outputs", _sampled_gate_frame_local),
 }
 
 PINS = [
@@ -116,6 +139,8 @@ PINS = [
     lambda: pins.test_bridge_decays_across_exactly_the_frames_between(),
     lambda: pins.test_rmsnorm_gate_readout(),
     lambda: pins.test_prepare_features_from_library_routines(),
+    lambda: pins.test_sampled_outputs_are_rows_of_the_whole_branch("vdn_solve", True),
+    lambda: pins.test_sampled_outputs_prenorm_is_bruteforce_far_field_attention(),
 ]
 
 

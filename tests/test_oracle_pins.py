@@ -423,3 +423,54 @@ def test_prepare_features_from_library_routines():
         np.testing.assert_allclose(kf[f], ks / np.linalg.norm(ks, axis=1, keepdims=True), rtol=1e-10)
         np.testing.assert_allclose(qf[f], qs / np.linalg.norm(qs, axis=1, keepdims=True), rtol=1e-10)
         np.testing.assert_allclose(vf[f], vc * scipy.special.expit(vc), rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- sampled outputs
+def _frame_edge_tokens(F, S, rng, extra=2):
+    """First and last token of every frame plus a few random ones (indices into F*S)."""
+    toks = []
+    for t in range(F):
+        toks += [t * S, t * S + S - 1]
+        toks += list(t * S + rng.integers(0, S, size=extra))
+    return np.array(sorted(set(int(x) for x in toks)))
+
+
+@pytest.mark.parametrize("rule", RULES)
+@pytest.mark.parametrize("text", [False, True])
+def test_sampled_outputs_are_rows_of_the_whole_branch(rule, text):
+    """The full-size checker: sampled_outputs(b, h, tokens) must be exactly the
+    rows (b, tokens, h) of branch_forward, for every batch and head, the first
+    and last token of each frame, and a frame length (S = 7) that is not a
+    multiple of anything in the window geometry."""
+    rng = np.random.default_rng(40)
+    B, H, d, F, S = 2, 3, 6, 13, 7
+    inp = _inputs(rng, B=B, H=H, d=d, F=F, S=S, text=text)
+    c = 0.5 if rule in ("sana_scaled", "vdn_scaled") else 1.0
+    full = O.branch_forward(inp, F, S, rule, c, 5, 1)
+    for b in range(B):
+        for h in range(H):
+            toks = _frame_edge_tokens(F, S, rng)
+            got = O.sampled_outputs(inp, F, S, rule, c, 5, 1, b, h, toks)
+            np.testing.assert_allclose(got, full[b, toks, h, :], rtol=1e-13, atol=1e-13)
+
+
+def test_sampled_outputs_prenorm_is_bruteforce_far_field_attention():
+    """sampled_outputs against a definition that shares none of its indexing:
+    additive rule, alpha = 1, no text, batch 2 and 2 heads: the pre-norm output
+    of token n of (b, h) is the beta-weighted linear attention of its q' against
+    every token of the frames outside its window."""
+    rng = np.random.default_rng(41)
+    B, H, d, F, S, chunk, radius = 2, 2, 5, 11, 4, 2, 1
+    inp = _inputs(rng, B=B, H=H, d=d, F=F, S=S, alpha_one=True)
+    for b in range(B):
+        for h in range(H):
+            st = O.head_state(inp, b, h, F, S, "additive", 1.0, chunk, radius)
+            qf, kf, vf = (st[n].reshape(-1, d) for n in ("qf", "kf", "vf"))
+            beta = inp["beta"][b, :, h]
+            toks = _frame_edge_tokens(F, S, rng, extra=1)
+            got = O.sampled_outputs(inp, F, S, "additive", 1.0, chunk, radius, b, h, toks, prenorm=True)
+            for i, n in enumerate(toks):
+                t = n // S
+                far = [m for m in range(F * S) if abs((m // S) // chunk - t // chunk) > radius]
+                ref = sum(beta[m] * vf[m] * np.dot(kf[m], qf[n]) for m in far) if far else np.zeros(d)
+                np.testing.assert_allclose(got[i], ref, rtol=1e-11, atol=1e-13)
