@@ -15,8 +15,10 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
- *     never allocates device memory and keeps no global state, so calls on
- *     different streams with different workspaces may run concurrently.
+ *     never allocates device memory, so calls on different streams with
+ *     different workspaces may run concurrently.  Its one piece of global state
+ *     is the fixed device array behind vdn_branch_forward_static (the scratch
+ *     of that entry point alone); no other entry point touches it.
  *   - Every tensor is dense and contiguous in the layout given beside it, with
  *     a 16-byte aligned base address (VDN_ERR_ALIGNMENT otherwise).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
@@ -26,6 +28,13 @@
  *   - Element types: q, k, v, gate and out share `shape->dtype` (fp32 or
  *     bf16); beta, alpha, rms_w, the conv taps and the text state are fp32.
  *     State and accumulation are fp32 in every configuration.
+ *   - Input domains (not checked, the values live on the device): beta >= 0
+ *     and alpha in (0, 1], as the sigmoids of "Step 2" and "Step 3" produce
+ *     them.  The tensor-core path scales both statistics operands by
+ *     sqrt(beta) (a negative beta gives NaN there) and inverts I + c^2 A by
+ *     elimination without pivoting, which needs I + c^2 A symmetric positive
+ *     definite; beta >= 0 guarantees that.  alpha above 1 makes the states
+ *     grow and is kept in range only by the block exponents of the scans.
  */
 #ifndef VDN_H
 #define VDN_H
@@ -85,7 +94,7 @@ size_t vdn_branch_workspace_size_impl(const vdn_shape* shape, int rule, int impl
  * vdn_branch_forward -- the whole branch, page sections "Step 1" to "Step 5".
  *
  *   q, k, v    [B, F*S, H, d] dtype   pre-RoPE ("NoPE") features, token-major
- *   beta       [B, F*S, H]    fp32    per-token, per-head write strength (post-sigmoid)
+ *   beta       [B, F*S, H]    fp32    per-token, per-head write strength (post-sigmoid, >= 0)
  *   alpha      [B, F, H, d]   fp32    per-frame, per-channel forget gate in (0, 1]
  *   gate       [B, F*S, H, d] dtype   output gate values (post-sigmoid)
  *   rms_w      [d]            fp32    RMSNorm weight (shared by the heads)

@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     }
     if (store && tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
     tc::tc_fence_before();
-    // accumulator and B_f reads done, alpha slot free; rescale if any entry passed 2^64
+    // accumulator and B_f reads done, alpha slot free; rescale if any entry passed
+    // kRenormAbove (2^32)
     if (__syncthreads_or(amax > kRenormAbove)) {
 #pragma unroll
       for (int p = 0; p < 32; ++p) s[p] = __fmul2_rn(s[p], make_float2(kRenormScale, kRenormScale));
