@@ -365,9 +365,12 @@ vdn_status vdn_branch_backward_timed(const vdn_shape* shape,
  * Every rule's frame step is affine in the state, S_out = S_in G_f + B'_f.
  * Phase 1, vdn_frames_maps: features, statistics and solves of the rank's frames,
  * then for each of its chunks and both scan directions the chunk's composed map
- * S -> S G_c + O_c, written to `maps`:
- *     maps [B*H][2 directions][nch][G_c | O_c][d][d] fp32, nch = ceil(C / world)
- *     (vdn_frames_map_bytes bytes; slots past the rank's own chunks are unused).
+ * S -> S G_c + O_c, written to `maps` (vdn_frames_map_bytes bytes):
+ *     [B*H][2 directions][nch][G_c | O_c][d][d] fp32, nch = ceil(C / world),
+ *     then [B*H][2 directions][nch][G_c | O_c] int32 exponents e: the map is
+ *     2^e times the stored matrix (sana_scaled can grow the state past fp32
+ *     range over a clip; the maps and the fold carry power-of-two exponents);
+ *     slots past the rank's own chunks are unused, the size is padded to 16 bytes.
  * The caller then concatenates every rank's buffer in rank order (an all-gather)
  * into maps_all [world][vdn_frames_map_bytes / 4].
  * Phase 2, vdn_frames_finish: folds the maps from 0.5 * text_state into the
@@ -380,7 +383,11 @@ vdn_status vdn_branch_backward_timed(const vdn_shape* shape,
  * VDN_ERR_UNSUPPORTED.  A partition that does not match shape->F, world > C or a
  * rank outside [0, world) is VDN_ERR_INVALID_ARG.  Both phases take one
  * workspace of vdn_frames_workspace_size bytes (256-byte aligned; it may be the
- * same buffer).  Pointers as in vdn_branch_forward: 16-byte aligned device
+ * same buffer).  vdn_frames_maps clears the workspace's device status word and
+ * vdn_frames_finish does not: given the same workspace, vdn_workspace_status
+ * after phase 2 reports an expired wait of either phase; a separate phase-2
+ * workspace needs its first 4 bytes zeroed by the caller.  Pointers as in
+ * vdn_branch_forward: 16-byte aligned device
  * memory owned by the caller; out and maps must not overlap any other argument.
  * Work is queued on `stream`; errors are returned before any launch.
  */

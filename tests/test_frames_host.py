@@ -66,11 +66,20 @@ def _shape(**kw):
     return VdnShape(**base)
 
 
+def _map_bytes(B, H, nch, d=128):
+    """The header's rank buffer: fp32 maps [B*H][2][nch][G | O][d][d], then int32 exponents
+    [B*H][2][nch][G | O], padded to 16 bytes."""
+    n = B * H * 2 * nch * 2 * d * d * 4 + B * H * 2 * nch * 2 * 4
+    return (n + 15) // 16 * 16
+
+
 def test_map_bytes_and_workspace(lib):
     s = _shape()                                   # rank 0 of 3 over 23 frames in chunks of 3: 9 frames
-    assert lib.vdn_frames_map_bytes(ctypes.byref(s), 23, 3, 0, 3) == 1 * 2 * 2 * 3 * 2 * 128 * 128 * 4
+    assert lib.vdn_frames_map_bytes(ctypes.byref(s), 23, 3, 0, 3) == _map_bytes(1, 2, 3)
     s2 = _shape(F=5)                               # rank 2 owns the last two chunks (3 + 2 frames)
-    assert lib.vdn_frames_map_bytes(ctypes.byref(s2), 23, 3, 2, 3) == 1 * 2 * 2 * 3 * 2 * 128 * 128 * 4
+    assert lib.vdn_frames_map_bytes(ctypes.byref(s2), 23, 3, 2, 3) == _map_bytes(1, 2, 3)
+    s3 = _shape(B=3, H=1, F=5)                     # an exponent block that is not a multiple of 16 bytes
+    assert lib.vdn_frames_map_bytes(ctypes.byref(s3), 23, 3, 2, 3) == _map_bytes(3, 1, 3)
     n = lib.vdn_frames_workspace_size(ctypes.byref(s), 23, 3, 0, 1, 3)
     assert n > 0 and n % 256 == 0
     # the clip-wide chunk-edge banks: two [B, H, F_total, d, d] fp32 regions at least

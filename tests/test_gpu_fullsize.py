@@ -72,5 +72,8 @@ def test_rule_sweep_1024sq():
             inp_run["text_state"] = None
         api.branch_forward(*args, F=w.F, rule=rule, c=c, chunk=w.chunk, radius=w.radius, out=out, workspace=ws)
         torch.cuda.synchronize()
-        _check(w, inp_run, out, [(i % 2, (7 * i) % w.H)], rule, c, rng)
+        assert api.workspace_status(ws) == 0
+        # both batch elements (the second one's frames sit in other statistics slots), two heads each
+        heads = [(b, (7 * i + 11 * b + j * (w.H // 2)) % w.H) for b in range(w.B) for j in range(2)]
+        _check(w, inp_run, out, heads, rule, c, rng)
     _rms_property(w, dev, out)

@@ -128,6 +128,25 @@ def test_feature_prep(dtype, d, tol, K):
                 assert np.abs(g - r).max() <= tol * max(1.0, np.abs(r).max())
 
 
+@pytest.mark.parametrize("S", [1, 2, 63, 64, 65, 150])
+def test_feature_prep_token_runs(S):
+    """bf16, d = 128: the streaming kernel sweeps each frame in runs of 64 tokens, 2 tokens per
+    step; frames shorter than, equal to and longer than a run (the conv's neighbours across run
+    and step boundaries come from the sliding window) against the oracle."""
+    w = synth.Workload("fp_runs", B=1, H=2, d=128, F=3, S=S, dtype="bf16", alpha_mu=2.0, text=False, seed=28)
+    inp = synth.make_inputs(w)
+    dev = api.to_device(inp)
+    qo, ko, vo = api.feature_prep(dev["q"], dev["k"], dev["v"], dev["conv_k_w"], dev["conv_v_w"], F=w.F)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        ref = O.prepare_features(inp["q"][0, :, h].double().numpy(), inp["k"][0, :, h].double().numpy(),
+                                 inp["v"][0, :, h].double().numpy(), w.F, w.S,
+                                 inp["conv_k_w"][h].double().numpy(), inp["conv_v_w"][h].double().numpy())
+        for got, r in zip((qo, ko, vo), ref):
+            g = to_np(got[0, :, h]).reshape(w.F, w.S, w.d)
+            assert np.abs(g - r).max() <= 8e-3 * max(1.0, np.abs(r).max())
+
+
 EDGE = [
     dict(F=1, S=40, text=True),                  # one frame: only the seeds, decayed
     dict(F=1, S=40, text=False),                 # one frame, no text: exactly zero

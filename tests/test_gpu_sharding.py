@@ -9,6 +9,7 @@ import torch
 
 from harness import TOL_BF16, gpu_forward, oracle_forward, rel_err, to_np
 from oracle import vdn_backward as BW
+from oracle import vdn_oracle as O
 from test_gpu_backward import BF16, NAMES, _compare
 from video_diffusion_linear_b200 import api, shard, synth
 
@@ -16,14 +17,28 @@ pytestmark = pytest.mark.gpu
 
 
 def _sharded(w, inp, world):
+    """Each rank's two phases share one workspace; its device status word must stay clear after
+    phase 1 and after phase 2 (which keeps a phase-1 report)."""
     parts = [api.to_device(shard.frame_inputs(inp, w.F, world, r, w.chunk)) for r in range(world)]
+    wss = []
+    for r, p in enumerate(parts):
+        f0, f1 = shard.frame_range(w.F, world, r, w.chunk)
+        shape = api.shape_from(p["k"], f1 - f0, p["conv_k_w"])
+        wss.append(torch.empty(api.frames_workspace_size(shape, w.F, world, r, w.rule, w.chunk), dtype=torch.uint8,
+                               device=p["k"].device))
     maps = [api.frames_maps(p["k"], p["v"], p["beta"], p["alpha"], p["conv_k_w"], p["conv_v_w"], F_total=w.F,
-                            world=world, rank=r, rule=w.rule, c=w.c, chunk=w.chunk) for r, p in enumerate(parts)]
+                            world=world, rank=r, rule=w.rule, c=w.c, chunk=w.chunk, workspace=wss[r])
+            for r, p in enumerate(parts)]
+    for ws in wss:
+        assert api.workspace_status(ws) == 0
     maps_all = torch.cat(maps)
     outs = [api.frames_finish(p["q"], p["alpha_all"], p["gate"], p["rms_w"], p["text_state"], maps_all, F_total=w.F,
-                              world=world, rank=r, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius)
+                              world=world, rank=r, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius,
+                              workspace=wss[r])
             for r, p in enumerate(parts)]
     torch.cuda.synchronize()
+    for ws in wss:
+        assert api.workspace_status(ws) == 0
     return torch.cat(outs, dim=1)
 
 
@@ -48,6 +63,32 @@ def test_frame_sharded_branch_matches_the_whole_clip(w, world):
     assert rel_err(to_np(joined), ref) <= TOL_BF16
     full, _ = gpu_forward(w, inp)
     assert rel_err(to_np(joined), to_np(full)) <= TOL_BF16
+
+
+def test_frame_sharded_divergent_sana_stays_finite():
+    """sana_scaled at c = 1 on inputs whose per-frame operator I - A has an eigenvalue near
+    -0.2 beta S: the float64 scans pass 1e39, beyond fp32.  The chunk maps carry power-of-two
+    exponents through the all-gather and the fold, so the frame-sharded output stays finite and
+    matches the oracle (the same stress inputs as the whole-clip divergence test)."""
+    w = synth.Workload("fr_div", B=1, H=2, d=128, F=40, S=384, dtype="bf16", alpha_mu=3.0, text=True, seed=32,
+                       rule="sana_scaled", c=1.0)
+    inp = synth.make_inputs(w)
+    st = O.head_state(inp, 0, 0, w.F, w.S, "sana_scaled", 1.0, w.chunk, w.radius)
+    assert np.abs(st["P"]).max() > 1e39
+    joined = _sharded(w, inp, 3)
+    assert torch.isfinite(joined.float()).all()
+    assert rel_err(to_np(joined), oracle_forward(w, inp)) <= TOL_BF16
+
+
+def test_shard_frame_sharded_forward_checks_the_status_word():
+    """shard.frame_sharded_forward with one rank (no collective) shares a workspace between the
+    phases, reads its status word and returns the whole clip's output."""
+    w = CASES[2][0]
+    inp = synth.make_inputs(w)
+    local = api.to_device(shard.frame_inputs(inp, w.F, 1, 0, w.chunk))
+    out = shard.frame_sharded_forward(local, w.F, 1, 0, rule=w.rule, c=w.c, chunk=w.chunk, radius=w.radius)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(out), oracle_forward(w, inp)) <= TOL_BF16
 
 
 def test_one_rank_equals_the_unsharded_call():

@@ -325,8 +325,10 @@ def test_chunk_maps_fold_into_the_scans_chunk_edge_states(rule, c, F, chunk):
 
 # ----------------------------------------------------------------------------- frame-sharded orchestration
 def _fake_frames_maps(k, v, beta, alpha, conv_k_w, conv_v_w, *, F_total, world, rank, rule, c, chunk, **_):
-    """vdn_frames_maps in the oracle's arithmetic, in the header's layout:
-    [B*H][2 directions][nch][G_c | O_c][d][d], nch = ceil(C / world), float64 here."""
+    """vdn_frames_maps in the oracle's arithmetic, in the header's layout: the maps
+    [B*H][2 directions][nch][G_c | O_c][d][d], nch = ceil(C / world), then one exponent e per
+    map (the map is 2^e times the stored matrix; here e puts the largest entry in [0.5, 1)),
+    float64 throughout."""
     f0, f1 = shard.frame_range(F_total, world, rank, chunk)
     n = f1 - f0
     B, N, H, d = k.shape
@@ -348,7 +350,14 @@ def _fake_frames_maps(k, v, beta, alpha, conv_k_w, conv_v_w, *, F_total, world, 
                         g = O.rule_step(g, A[f], zero, al[f], rule, c)
                         o = O.rule_step(o, A[f], Bm[f], al[f], rule, c)
                     maps[b, h, dr, j] = g, o
-    return torch.from_numpy(maps.ravel())
+    exps = np.zeros(maps.shape[:-2])
+    for idx in np.ndindex(*exps.shape):
+        m = np.abs(maps[idx]).max()
+        if np.isfinite(m) and m > 0:
+            e = np.frexp(m)[1]
+            exps[idx] = e
+            maps[idx] = np.ldexp(maps[idx], -e)
+    return torch.from_numpy(np.concatenate([maps.ravel(), exps.ravel()]))
 
 
 def _fake_frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_total, world, rank, rule, c, chunk,
@@ -361,7 +370,10 @@ def _fake_frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_to
     S = N // n
     C = -(-F_total // chunk)
     nch = -(-C // world)
-    maps = maps_all.numpy().reshape(world, B, H, 2, nch, 2, d, d)
+    buf = maps_all.numpy().reshape(world, -1)
+    nm = B * H * 2 * nch * 2 * d * d
+    exps = buf[:, nm:].reshape(world, B, H, 2, nch, 2)
+    maps = np.ldexp(buf[:, :nm].reshape(world, B, H, 2, nch, 2, d, d), exps[..., None, None].astype(int))
     first = [shard.frame_range(F_total, world, r, chunk)[0] // chunk for r in range(world)]
     owner = lambda ch: max(r for r in range(world) if first[r] <= ch)
     out = np.empty((B, N, H, d))

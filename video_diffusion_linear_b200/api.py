@@ -402,6 +402,7 @@ def frames_finish(q, alpha_all, gate, rms_w, text_state, maps_all, *, F_total: i
     if workspace is None:
         workspace = torch.empty(frames_workspace_size(shape, F_total, world, rank, rule, chunk), dtype=torch.uint8,
                                 device=q.device)
+        workspace[:256].zero_()   # phase 2 keeps the device status word it is given
     _bytes("workspace", workspace, q.device)
     st = _lib.load().vdn_frames_finish(ctypes.byref(shape), F_total, world, rank, _ptr(q), _ptr(alpha_all),
                                        _ptr(gate), _ptr(rms_w), _ptr(text_state), VDN_RULE[rule], float(c),

@@ -69,7 +69,10 @@ cudaError_t launch_gather_frames(const Args& a, int fq0, int Fq, const float* P,
                                  const int* qexp, float* W, uint16_t* wimg, int* wexp, int* wbexp);
 // the fold of every chunk's affine maps into the chunk-edge states P (chunk ends) and Q (chunk
 // starts) of the a.sh.F-frame clip, from 0.5 x the text state (frames.cu)
-cudaError_t launch_fold_maps(const Args& a, const float* maps_all, int world, int nch_stride, float* P, float* Q);
+// maps_all holds `world` rank buffers of rank_bytes each, every one the maps followed (at
+// exp_off_bytes) by their int32 exponents; the folded states get exponents in pexp / qexp.
+cudaError_t launch_fold_maps(const Args& a, const float* maps_all, size_t rank_bytes, size_t exp_off_bytes, int world,
+                             int nch_stride, float* P, float* Q, int* pexp, int* qexp);
 // dst = src * 2^expo[frame] (expo may be NULL)
 cudaError_t launch_copy_frames(const Args& a, const float* src, float* dst, const int* expo = nullptr);
 
@@ -138,9 +141,12 @@ cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* 
 cudaError_t launch_stats_tc(const Args& a, float* partials, uint32_t* status);
 // scan modes: the whole clip from the text seed, or per-chunk affine maps (frame sharding)
 constexpr int kScanWhole = 0, kScanSegZero = 1, kScanSegIdentity = 2;
+// segment modes write map (b, h, direction, chunk j, G | O) of the rank's chunks to
+// maps[((((b H + h) 2 + dir) nch_stride + j) 2 + (0 G | 1 O))][128][128] and its exponent to
+// map_exp at the same index
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
                            int* qexp, bool all_frames, uint32_t* status, int seg_mode = kScanWhole,
-                           float* maps = nullptr, int nch_stride = 0);
+                           float* maps = nullptr, int* map_exp = nullptr, int nch_stride = 0);
 cudaError_t launch_window_softmax_simt(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,
                                        int radius, float scale, int accumulate, void* out, cudaStream_t stream);
 cudaError_t launch_window_softmax_tc(const vdn_shape& sh, const void* qr, const void* kr, const void* v, int chunk,

@@ -342,10 +342,135 @@ cudaError_t launch_readout_simt(const Args& a, const float* qf, const float* W, 
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- standalone Step 1
+// ---------------------------------------------------------------- standalone Step 1, bf16, d = 128
+// A streaming kernel: it reads q, k, v once and writes q', k', v' once, so it is
+// bound by HBM bandwidth.  A block of 256 threads serves one head: its 16
+// half-warps each own one (batch, frame) and a run of kFpRun consecutive tokens
+// of that frame, and lane c of a half-warp holds channels 8c .. 8c + 7, so every
+// load and store of a token row is one coalesced 16-byte access per lane (a
+// 256-byte row per half-warp).  The run is swept kFpStep tokens at a time with a
+// sliding window of rows, so the conv's neighbour rows are read once (plus one
+// row at each end of the run).  The head's conv taps sit in shared memory.  q and
+// k are normalised with a 16-lane shuffle reduction; SiLU uses the hardware tanh
+// (x sigmoid(x) = h + h tanh h, h = x/2), whose error is far below the bf16
+// rounding of the outputs.
+namespace {
+constexpr int kFpRun = 64;    // tokens per half-warp run
+constexpr int kFpStep = 2;    // tokens per step
+
+__device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
+  x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+  x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+}
+__device__ __forceinline__ uint4 pack8(const float (&x)[8], float s) {
+  return make_uint4(pack_bf16x2(x[0] * s, x[1] * s), pack_bf16x2(x[2] * s, x[3] * s), pack_bf16x2(x[4] * s, x[5] * s),
+                    pack_bf16x2(x[6] * s, x[7] * s));
+}
+__device__ __forceinline__ float silu_h(float hx) { return fmaf(hx, tanh_approx(hx), hx); }   // hx = x / 2
+}  // namespace
+
+__global__ void __launch_bounds__(256, 2) k_features128(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                        const uint4* __restrict__ v, const float* __restrict__ wk,
+                                                        const float* __restrict__ wv, int K, uint4* __restrict__ qo,
+                                                        uint4* __restrict__ ko, uint4* __restrict__ vo, int F, int S,
+                                                        int H, int nrun, long long runs) {
+  __shared__ __align__(16) float taps[2][3][128];   // [k|v][tap][channel] / 2
+  const int h = blockIdx.y;
+  for (int e = threadIdx.x; e < 2 * 3 * 128; e += blockDim.x) {
+    const int ten = e / 384, j = (e / 128) % 3, ch = e % 128;
+    const float* wg = ten == 0 ? wk : wv;
+    const long long i = (long long)h * 128 + ch;
+    const float val = wg ? (K == 3 ? wg[i * 3 + j] : (j == 1 ? wg[i] : 0.f)) : (j == 1 ? 1.f : 0.f);
+    taps[ten][j][ch] = 0.5f * val;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, c = lane & 15;
+  const long long g = (long long)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4);   // this half-warp's run
+  const bool live = g < runs;                   // a dead half-warp still joins the warp's shuffles
+  const long long gg = live ? g : 0;
+  const int run = (int)(gg % nrun);
+  const long long bf = gg / nrun;               // b * F + f
+  const int s0 = run * kFpRun, s1 = min(S, s0 + kFpRun);
+  const long long row0 = bf * (long long)S;     // token row of the frame's first token
+  auto at = [&](int s) { return ((row0 + s) * H + h) * 16 + c; };   // uint4 index of (token s, lane chunk)
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  auto ld = [&](const uint4* p, int s) { return (live && s >= 0 && s < S) ? __ldg(p + at(s)) : z; };
+  // window: rows s - 1 .. s + kFpStep of k and v for the step starting at token s
+  uint4 kw[kFpStep + 2], vw[kFpStep + 2];
+  kw[0] = ld(k, s0 - 1);
+  vw[0] = ld(v, s0 - 1);
+  kw[1] = ld(k, s0);
+  vw[1] = ld(v, s0);
+  for (int s = s0; s < s1; s += kFpStep) {
+    uint4 qw[kFpStep];
+#pragma unroll
+    for (int i = 0; i < kFpStep; ++i) {
+      kw[i + 2] = s + i + 1 < s1 + 1 ? ld(k, s + 1 + i) : z;
+      vw[i + 2] = s + i + 1 < s1 + 1 ? ld(v, s + 1 + i) : z;
+      qw[i] = s + i < s1 ? ld(q, s + i) : z;
+    }
+#pragma unroll
+    for (int i = 0; i < kFpStep; ++i) {
+      float k0[8], k1[8], k2[8], v0[8], v1[8], v2[8], qx[8];
+      unpack8(kw[i], k0); unpack8(kw[i + 1], k1); unpack8(kw[i + 2], k2);
+      unpack8(vw[i], v0); unpack8(vw[i + 1], v1); unpack8(vw[i + 2], v2);
+      unpack8(qw[i], qx);
+      float yk[8], yv[8], yq[8];
+      float ssk = 0.f, ssq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; e += 4) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&taps[0][0][8 * c + e]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&taps[0][1][8 * c + e]);
+        const float4 a2 = *reinterpret_cast<const float4*>(&taps[0][2][8 * c + e]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&taps[1][0][8 * c + e]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&taps[1][1][8 * c + e]);
+        const float4 b2 = *reinterpret_cast<const float4*>(&taps[1][2][8 * c + e]);
+        const float ta[3][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}, {a2.x, a2.y, a2.z, a2.w}};
+        const float tb[3][4] = {{b0.x, b0.y, b0.z, b0.w}, {b1.x, b1.y, b1.z, b1.w}, {b2.x, b2.y, b2.z, b2.w}};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float hk = fmaf(ta[0][u], k0[e + u], fmaf(ta[1][u], k1[e + u], ta[2][u] * k2[e + u]));
+          const float hv = fmaf(tb[0][u], v0[e + u], fmaf(tb[1][u], v1[e + u], tb[2][u] * v2[e + u]));
+          yk[e + u] = silu_h(hk);
+          yv[e + u] = silu_h(hv);
+          yq[e + u] = silu_h(0.5f * qx[e + u]);
+          ssk = fmaf(yk[e + u], yk[e + u], ssk);
+          ssq = fmaf(yq[e + u], yq[e + u], ssq);
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) {
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+      }
+      const int si = s + i;
+      if (live && si < s1) {
+        const long long o = at(si);
+        ko[o] = pack8(yk, rsqrtf(ssk + kL2Eps));
+        qo[o] = pack8(yq, rsqrtf(ssq + kL2Eps));
+        vo[o] = pack8(yv, 1.f);
+      }
+    }
+    // slide the window by kFpStep rows
+    kw[0] = kw[kFpStep];
+    vw[0] = vw[kFpStep];
+    kw[1] = kw[kFpStep + 1];
+    vw[1] = vw[kFpStep + 1];
+  }
+}
+
 cudaError_t launch_feature_prep(const vdn_shape& sh, const void* q, const void* k, const void* v,
                                 const float* wk, const float* wv, void* qo, void* ko, void* vo,
                                 cudaStream_t st) {
+  if (sh.dtype == VDN_DTYPE_BF16 && sh.d == 128) {
+    const int nrun = (sh.S + kFpRun - 1) / kFpRun;
+    const long long runs = (long long)sh.B * sh.F * nrun;   // per head
+    const dim3 grid((unsigned)((runs + 15) / 16), (unsigned)sh.H);
+    const int K = (wk || wv) ? sh.conv_width : 1;
+    k_features128<<<grid, 256, 0, st>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, wk, wv, K, (uint4*)qo,
+                                        (uint4*)ko, (uint4*)vo, sh.F, sh.S, sh.H, nrun, runs);
+    return cudaGetLastError();
+  }
   if (sh.dtype == VDN_DTYPE_BF16)
     return features_dispatch<__nv_bfloat16, __nv_bfloat16>(sh, q, k, v, wk, wv, qo, ko, vo, st);
   return features_dispatch<float, float>(sh, q, k, v, wk, wv, qo, ko, vo, st);

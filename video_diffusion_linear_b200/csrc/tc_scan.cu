@@ -17,8 +17,8 @@
 // Segment mode (frame sharding): the state restarts at every chunk, from zero
 // with the rule's own coefficients (the chunk's offset O_c) or from the identity
 // with cpre = cpost = 0 (the chunk's linear part G_c = prod D_f N_f), and the
-// state at the chunk's last step in scan order is stored, at its true scale, as
-// the chunk's affine map S -> S G_c + O_c.
+// state at the chunk's last step in scan order is stored with its block
+// exponent as the chunk's affine map S -> S G_c + O_c.
 #include "common.cuh"
 #include "image.cuh"
 #include "internal.h"
@@ -71,8 +71,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
                                                             float* __restrict__ P, float* __restrict__ Q,
                                                             int* __restrict__ pexp, int* __restrict__ qexp, int H,
                                                             int F, int chunk, int all_frames,
-                                                            float* __restrict__ maps, int nch_stride,
-                                                            uint32_t* __restrict__ status) {
+                                                            float* __restrict__ maps, int* __restrict__ map_exp,
+                                                            int nch_stride, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -228,11 +228,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     const bool seg_store = kMode != kScanWhole && seg_last(f);
     const bool store = kMode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
     float* dst = kMode == kScanWhole ? (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0 : nullptr;
-    // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col], at the true scale 2^ex
-    float* mdst = kMode == kScanWhole ? nullptr
-                                      : maps + ((((bh * 2 + dir) * nch_stride + f / chunk) * 2 +
-                                                 (kMode == kScanSegIdentity ? 0 : 1)) * 128 + m) * 128 + k0;
-    const float mscale = kMode == kScanWhole ? 1.f : ldexpf(1.f, ex);
+    // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col]; the map is 2^ex times the stored state
+    const long long mslot = ((bh * 2 + dir) * nch_stride + f / chunk) * 2 + (kMode == kScanSegIdentity ? 0 : 1);
+    float* mdst = kMode == kScanWhole ? nullptr : maps + (mslot * 128 + m) * 128 + k0;
     float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -253,11 +251,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
         if (store)
           *reinterpret_cast<float4*>(dst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
         if (seg_store)
-          *reinterpret_cast<float4*>(mdst + 32 * j + e) =
-              make_float4(s[p].x * mscale, s[p].y * mscale, s[p + 1].x * mscale, s[p + 1].y * mscale);
+          *reinterpret_cast<float4*>(mdst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
       }
     }
     if (store && tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
+    if (seg_store && tid == 0) map_exp[mslot] = ex;
     tc::tc_fence_before();
     // accumulator and B_f reads done, alpha slot free; rescale if any entry passed
     // kRenormAbove (2^32)
@@ -281,7 +279,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
 }
 
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
-                           int* qexp, bool all_frames, uint32_t* status, int seg_mode, float* maps, int nch_stride) {
+                           int* qexp, bool all_frames, uint32_t* status, int seg_mode, float* maps, int* map_exp,
+                           int nch_stride) {
   CUtensorMap tmB;
   if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
   size_t smem = sizeof(ScanSmem) + 1024;
@@ -294,7 +293,7 @@ cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nim
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
       tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, maps,
-      nch_stride, status);
+      map_exp, nch_stride, status);
   return cudaGetLastError();
 }
 

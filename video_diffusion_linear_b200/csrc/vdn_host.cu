@@ -659,8 +659,14 @@ vdn_status frame_part(int F_total, int world, int rank, int chunk, FramePart& fp
   return VDN_OK;
 }
 
+// a rank's map buffer: the maps [B*H][2][nch][G | O][d][d] fp32, then their exponents
+// [B*H][2][nch][G | O] int32, padded to 16 bytes
+size_t frame_map_floats(const vdn_shape& sh, const FramePart& fp) {
+  return (size_t)sh.B * sh.H * 2 * fp.nch_stride * 2 * sh.d * sh.d;
+}
 size_t frame_map_bytes(const vdn_shape& sh, const FramePart& fp) {
-  return (size_t)sh.B * sh.H * 2 * fp.nch_stride * 2 * sh.d * sh.d * sizeof(float);
+  const size_t exps = (size_t)sh.B * sh.H * 2 * fp.nch_stride * 2;
+  return (frame_map_floats(sh, fp) * sizeof(float) + exps * sizeof(int) + 15) & ~(size_t)15;
 }
 
 // workspace of the second phase: the clip's chunk-edge states and the rank's read-out images
@@ -799,10 +805,11 @@ vdn_status vdn_frames_maps(const vdn_shape* shape, int F_total, int world, int r
   VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), a.stream));
   VDN_LAUNCH(launch_stats_tc(a, part, status));
   VDN_LAUNCH(launch_solve(a, nullptr, nullptr, nimg, part, Bsum, nullptr));
+  int* map_exp = reinterpret_cast<int*>(maps + frame_map_floats(*shape, fp));
   VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, nullptr, nullptr, nullptr, nullptr, false, status, kScanSegZero, maps,
-                            fp.nch_stride));
+                            map_exp, fp.nch_stride));
   VDN_LAUNCH(launch_scan_tc(a, Bsum, nimg, nullptr, nullptr, nullptr, nullptr, false, status, kScanSegIdentity, maps,
-                            fp.nch_stride));
+                            map_exp, fp.nch_stride));
   return VDN_OK;
 }
 
@@ -854,11 +861,10 @@ vdn_status vdn_frames_finish(const vdn_shape* shape, int F_total, int world, int
   int *pexp = at<int>(workspace, p.pexp), *qexp = at<int>(workspace, p.qexp);
   uint16_t* wimg = at<uint16_t>(workspace, p.wimg);
   int *wexp = at<int>(workspace, p.wexp), *wbexp = at<int>(workspace, p.wbexp);
-  const size_t NFg = (size_t)g.B * g.H * F_total;
-  VDN_LAUNCH(cudaMemsetAsync(status, 0, sizeof(uint32_t), ag.stream));
-  VDN_LAUNCH(cudaMemsetAsync(pexp, 0, NFg * sizeof(int), ag.stream));   // the folded states carry no exponent
-  VDN_LAUNCH(cudaMemsetAsync(qexp, 0, NFg * sizeof(int), ag.stream));
-  VDN_LAUNCH(launch_fold_maps(ag, maps_all, world, fp.nch_stride, P, Q));
+  // the status word is not cleared here: with the workspace of vdn_frames_maps it keeps that
+  // phase's report, and an expired wait of either phase stays visible afterwards
+  VDN_LAUNCH(launch_fold_maps(ag, maps_all, frame_map_bytes(*shape, fp), frame_map_floats(*shape, fp) * sizeof(float),
+                              world, fp.nch_stride, P, Q, pexp, qexp));
   VDN_LAUNCH(launch_gather_frames(ag, fp.f0, fp.F_local, P, Q, pexp, qexp, nullptr, wimg, wexp, wbexp));
   VDN_LAUNCH(launch_readout_tc(al, wimg, wexp, wbexp, status));
   return VDN_OK;

@@ -138,14 +138,23 @@ def frame_inputs(inputs: dict, F: int, world: int, rank: int, chunk: int) -> dic
 
 
 def frame_sharded_forward(local: dict, F: int, world: int, rank: int, *, rule="vdn_solve", c=1.0, chunk=5,
-                          radius=1, group=None, stream=None):
+                          radius=1, group=None, stream=None, check_status=True):
     """The branch output of this rank's frames (device tensors from frame_inputs): its chunk maps,
     one all-gather of every rank's maps (NCCL for CUDA tensors; none with one rank), then the fold,
-    gather and read-out of its frames."""
+    gather and read-out of its frames.  Both phases share one workspace, so its device status word
+    reports an expired bounded wait of either phase; with check_status (CUDA tensors only) it is
+    read after phase 2 (a synchronisation) and a timeout raises."""
     from . import api
+    ws = None
+    if local["k"].is_cuda:
+        import torch
+        f0, f1 = frame_range(F, world, rank, chunk)
+        shape = api.shape_from(local["k"], f1 - f0, local.get("conv_k_w"))
+        ws = torch.empty(api.frames_workspace_size(shape, F, world, rank, rule, chunk), dtype=torch.uint8,
+                         device=local["k"].device)
     maps = api.frames_maps(local["k"], local["v"], local["beta"], local["alpha"], local.get("conv_k_w"),
                            local.get("conv_v_w"), F_total=F, world=world, rank=rank, rule=rule, c=c, chunk=chunk,
-                           stream=stream)
+                           workspace=ws, stream=stream)
     if world > 1:
         import torch
         import torch.distributed as dist
@@ -153,6 +162,9 @@ def frame_sharded_forward(local: dict, F: int, world: int, rank: int, *, rule="v
         dist.all_gather_into_tensor(maps_all, maps, group=group)
     else:
         maps_all = maps
-    return api.frames_finish(local["q"], local["alpha_all"], local["gate"], local["rms_w"], local.get("text_state"),
-                             maps_all, F_total=F, world=world, rank=rank, rule=rule, c=c, chunk=chunk, radius=radius,
-                             stream=stream)
+    out = api.frames_finish(local["q"], local["alpha_all"], local["gate"], local["rms_w"], local.get("text_state"),
+                            maps_all, F_total=F, world=world, rank=rank, rule=rule, c=c, chunk=chunk, radius=radius,
+                            workspace=ws, stream=stream)
+    if ws is not None and check_status:
+        api.check(api.workspace_status(ws, stream), "device status word after the frame-sharded branch")
+    return out
