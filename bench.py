@@ -45,7 +45,8 @@ METRIC = "latent tokens/sec through VDN linear branch fwd (1 B200); % of rooflin
 METRIC_PATH = {"backward": "latent tokens/sec through the VDN linear branch backward (forward recompute + "
                            "gradients of every input, 1 B200)",
                "softmax": "latent tokens/sec through the windowed softmax branch fwd (1 B200)",
-               "hybrid": "latent tokens/sec through the VDN-H3 hybrid attention layer fwd (softmax + linear branch, 1 B200)"}
+               "hybrid": "latent tokens/sec through the VDN-H3 hybrid attention layer fwd (softmax + linear branch, 1 B200)",
+               "features": "latent tokens/sec through the branch's Step 1 alone (conv, SiLU, L2 norm; 1 B200)"}
 DEFAULT_WORKLOAD = "768p"
 KERNELS_TC = ["frame_stats", "frame_solve", "scan", "gather", "readout"]
 KERNEL_SOURCES = {"frame_stats": "tc_stats.cu", "frame_solve": "solve_gather.cu", "scan": "tc_scan.cu",
@@ -714,6 +715,112 @@ def run_gpu_softmax(args, w: synth.Workload) -> None:
     }), flush=True)
 
 
+def run_gpu_features(args, w: synth.Workload) -> None:
+    """Step 1 alone (--path features): vdn_feature_prep over the workload's q, k, v, writing
+    q', k', v'.  A streaming kernel: its roofline is HBM, with algorithmic bytes = q, k, v read
+    once and q', k', v' written once (6 x d x 2 B per token-head in bf16)."""
+    from video_diffusion_linear_b200 import _lib, api
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    _lib.load()
+    host, wr, job_tokens, split = rank_inputs(args.shard, w, world, rank)
+    dev = api.to_device(host, device)
+    stream = torch.cuda.current_stream(device)
+    outs = tuple(torch.empty_like(dev[k]) for k in ("q", "k", "v"))
+
+    def step():
+        api.feature_prep(dev["q"], dev["k"], dev["v"], dev["conv_k_w"], dev["conv_v_w"], F=wr.F, stream=stream,
+                         out=outs)
+
+    for _ in range(args.warmup):
+        step()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end)
+    ms_max = reduce_max(ms, device)
+    value = job_tokens * args.steps / (ms_max / 1e3)
+    peaks, peak_src = load_peaks()
+    TH = wr.B * wr.F * wr.S * wr.H
+    nbytes = 6 * wr.d * (2 if wr.dtype == "bf16" else 4) * TH
+    us = ms / args.steps * 1e3
+    achieved = nbytes / (us / 1e6) / 1e9
+    roof = {"kernel": "feature_prep", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src, "algorithmic_bytes_per_launch": nbytes,
+            "traffic": None, "us_per_launch": us}
+
+    e2e = None
+    if not args.no_e2e:
+        keys = ["q", "k", "v"]
+        pinned = {k: host[k].pin_memory() for k in keys}
+        outs_host = tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs)
+        h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in keys)
+        d2h = sum(o.numel() * o.element_size() for o in outs_host)
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k in keys:
+                dev[k].copy_(pinned[k], non_blocking=True)
+            step()
+            for oh, o in zip(outs_host, outs):
+                oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+        e2e = {"value": job_tokens * n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu and world == 1:
+        from oracle import vdn_oracle as O
+        heads = list(range(min(args.cpu_heads, w.H)))
+        t0 = time.perf_counter()
+        for h in heads:
+            O.prepare_features(O._f64(host["q"][0, :, h]), O._f64(host["k"][0, :, h]), O._f64(host["v"][0, :, h]),
+                               w.F, w.S, None if host["conv_k_w"] is None else O._f64(host["conv_k_w"][h]),
+                               None if host["conv_v_w"] is None else O._f64(host["conv_v_w"][h]))
+        dt = time.perf_counter() - t0
+        cpu = {"value": len(heads) * w.F * w.S / w.H / dt, "unit": "tokens/s", "cores": blas_threads(),
+               "kind": "oracle", "sample": f"heads 0..{len(heads) - 1} of {w.H}, batch 0, all {w.F} frames x {w.S} "
+                                           f"tokens ({dt:.1f} s); tokens counted x heads/H"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC_PATH["features"], "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": split["scaling"], "vs_baseline": None, "dtype": wr.dtype, "data": "synthetic",
+        "config": {"workload": describe(w) + "; Step 1 only (conv, SiLU, L2 norm of q and k)",
+                   "global_batch": split["global_batch"], "tokens_per_step": job_tokens,
+                   "l2": "inputs larger than L2 (q, k, v: %.2f GB per GPU)" % (3 * wr.tokens * wr.H * wr.d * 2 / 1e9),
+                   "parallelism": split["parallelism"]},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }), flush=True)
+
+
 def run_gpu_frames(args, w: synth.Workload) -> None:
     """The linear branch of ONE clip split by frames across the ranks (strong scaling): each rank
     writes the affine maps of its chunks, one all-gather gives every rank every map, and each rank
@@ -978,9 +1085,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=2)
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
-    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid", "backward"],
-                    help="linear branch (default), windowed softmax branch, the whole hybrid layer, or the "
-                         "linear branch's backward pass")
+    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid", "backward", "features"],
+                    help="linear branch (default), windowed softmax branch, the whole hybrid layer, the "
+                         "linear branch's backward pass, or its Step 1 alone (vdn_feature_prep)")
     ap.add_argument("--cpu-tokens", type=int, default=256, help="query tokens in the softmax oracle sample")
     ap.add_argument("--shard", default="clips", choices=["clips", "heads", "frames"],
                     help="multi-GPU: independent clips per rank (weak scaling, default), one clip with its "
@@ -999,8 +1106,12 @@ def main(argv=None):
         w = w.replace(c=args.c)
     if args.heads:
         w = w.replace(H=args.heads)
+    if args.path == "features" and (args.impl == "reference" or args.shard == "frames"):
+        ap.error("--path features runs the GPU arm with --shard clips or heads")
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.path == "features":
+        run_gpu_features(args, w)
     elif args.path == "backward":
         run_gpu_backward(args, w)
     elif args.path != "linear":

@@ -81,6 +81,7 @@ def stubbed(monkeypatch):
     monkeypatch.setattr(api, "branch_backward", _grads)
     monkeypatch.setattr(api, "frames_maps", lambda *a, maps=None, **k: maps)
     monkeypatch.setattr(api, "frames_finish", lambda *a, out=None, **k: out)
+    monkeypatch.setattr(api, "feature_prep", lambda *a, out=None, **k: out)
     monkeypatch.setitem(synth.WORKLOADS, "tiny_bf16", synth.Workload("tiny_bf16", 1, 2, 128, 12, 8, "bf16", 2.0,
                                                                      True, 5))
 
@@ -96,6 +97,8 @@ def _line(argv):
     [], ["--shard", "heads"], ["--path", "softmax"], ["--path", "hybrid", "--shard", "heads"],
     ["--path", "backward"], ["--path", "backward", "--shard", "heads"],
     ["--workload", "tiny_bf16", "--shard", "frames"],
+    ["--workload", "tiny_bf16", "--path", "features"], ["--workload", "tiny_bf16", "--path", "features",
+                                                        "--shard", "heads"],
 ])
 def test_gpu_arms_assemble_the_contract_line(stubbed, extra):
     argv = ["--workload", "tiny_f20_text", "--steps", "2", "--warmup", "3", "--no-cpu"] + extra
@@ -110,3 +113,9 @@ def test_gpu_arms_assemble_the_contract_line(stubbed, extra):
 def test_default_arm_carries_the_oracle_baseline(stubbed):
     j = _line(["--workload", "tiny_f20_text", "--steps", "2", "--warmup", "3"])
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] > 0 and j["cpu_baseline"]["cores"] >= 1
+
+
+def test_features_arm_carries_the_oracle_baseline(stubbed):
+    j = _line(["--workload", "tiny_bf16", "--path", "features", "--steps", "2", "--warmup", "3"])
+    assert j["roofline"]["kernel"] == "feature_prep" and j["roofline"]["bound"] == "hbm"
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] > 0

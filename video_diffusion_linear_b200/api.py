@@ -208,12 +208,18 @@ def branch_forward_debug(q, k, v, beta, alpha, gate, rms_w, conv_k_w=None, conv_
     return out, mats
 
 
-def feature_prep(q, k, v, conv_k_w=None, conv_v_w=None, *, F: int, stream=None):
-    """vdn_feature_prep: Step 1 alone.  Returns (q', k', v') in q's dtype."""
+def feature_prep(q, k, v, conv_k_w=None, conv_v_w=None, *, F: int, stream=None, out=None):
+    """vdn_feature_prep: Step 1 alone.  Returns (q', k', v') in q's dtype (into `out`, a tuple
+    of three tensors shaped like q, when given)."""
     shape = shape_from(q, F, conv_k_w if conv_k_w is not None else conv_v_w)
     _validate([s for s in _branch_specs(q, k, v, None, None, None, None, conv_k_w, conv_v_w, None, F)
                if s[0] in ("q", "k", "v", "conv_k_w", "conv_v_w")], q.device)
-    qo, ko, vo = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if out is None:
+        qo, ko, vo = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        qo, ko, vo = out
+        _validate([("q_out", qo, q.shape, q.dtype, False), ("k_out", ko, q.shape, q.dtype, False),
+                   ("v_out", vo, q.shape, q.dtype, False)], q.device)
     st = _lib.load().vdn_feature_prep(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_k_w),
                                       _ptr(conv_v_w), _ptr(qo), _ptr(ko), _ptr(vo), _stream_ptr(stream))
     check(st, "vdn_feature_prep")
