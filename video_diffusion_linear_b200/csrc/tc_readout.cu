@@ -101,14 +101,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  auto coords = [&](long long x, int& h, int& s0, int& fb) {
-    long long fi = x / ntile;
-    int j = (int)(x % ntile);
-    int t = (int)(fi % F);
-    long long bh = fi / F;
-    h = (int)(bh % H);
-    fb = (int)((bh / H) * F + t);
-    s0 = j * 128;
+  // tile x = ((b H + h) F + t) ntile + j; each role decodes its first tile once
+  // and then steps the counters, so the loops carry no 64-bit division
+  struct Tile {
+    long long fi;   // (b H + h) F + t: the W_t slot
+    int j, t, h, b;
+  };
+  auto tile_at = [&](long long x) {
+    Tile u;
+    u.fi = x / ntile;
+    u.j = (int)(x - u.fi * ntile);
+    const long long bh = u.fi / F;
+    u.t = (int)(u.fi - bh * F);
+    u.b = (int)(bh / H);
+    u.h = (int)(bh - (long long)u.b * H);
+    return u;
+  };
+  auto tile_next = [&](Tile& u) {
+    if (++u.j == ntile) {
+      u.j = 0;
+      ++u.fi;
+      if (++u.t == F) {
+        u.t = 0;
+        if (++u.h == H) {
+          u.h = 0;
+          ++u.b;
+        }
+      }
+    }
   };
 
   if (warp == 0) {
@@ -117,8 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       long long cur = -1;
       uint32_t wph = 0;
       int it = 0;
-      for (long long x = x0; x < x1; ++x, ++it) {
-        long long fi = x / ntile;
+      Tile u = tile_at(x0);
+      for (long long x = x0; x < x1; ++x, ++it, tile_next(u)) {
+        const long long fi = u.fi;
         if (fi != cur) {
           if (cur >= 0) {
             if (!tc::mbar_wait(&sm.bar_w_empty, wph, abort_flag, status)) break;
@@ -129,8 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
           for (int q = 0; q < 2; ++q) tc::bulk_load(sm.wimg + q * 16384, src + q * 16384, 16384, &sm.bar_w_full);
           cur = fi;
         }
-        int h, s0, fb;
-        coords(x, h, s0, fb);
+        const int h = u.h, s0 = u.j * 128, fb = u.b * F + u.t;
         const int st = it % kQS;
         const uint32_t ph = (it / kQS) & 1;
         if (!tc::mbar_wait(&sm.bar_q_empty[st], ph ^ 1, abort_flag, status)) break;
@@ -146,8 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       uint32_t wph = 0;
       int it = 0;
       const uint32_t w = tc::smem_u32(sm.wimg);
-      for (long long x = x0; x < x1; ++x, ++it) {
-        long long fi = x / ntile;
+      Tile u = tile_at(x0);
+      for (long long x = x0; x < x1; ++x, ++it, tile_next(u)) {
+        const long long fi = u.fi;
         if (fi != cur) {
           if (!tc::mbar_wait(&sm.bar_w_full, wph, abort_flag, status)) break;
           wph ^= 1;
@@ -168,16 +189,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
         }
         tc::umma_commit(&sm.bar_q_empty[qs]);
         tc::umma_commit(&sm.bar_acc_full[ab]);
-        if (x + 1 == x1 || (x + 1) / ntile != fi) tc::umma_commit(&sm.bar_w_empty);
+        if (x + 1 == x1 || u.j + 1 == ntile) tc::umma_commit(&sm.bar_w_empty);
       }
     }
   } else if (warp == 18) {
     // ------------------------------------------------------------ gate producer
     if (lane == 0) {
       int it = 0;
-      for (long long x = x0; x < x1; ++x, ++it) {
-        int h, s0, fb;
-        coords(x, h, s0, fb);
+      Tile u = tile_at(x0);
+      for (long long x = x0; x < x1; ++x, ++it, tile_next(u)) {
+        const int h = u.h, s0 = u.j * 128, fb = u.b * F + u.t;
         const int st = it % kGS;
         const uint32_t ph = (it / kGS) & 1;
         if (!tc::mbar_wait(&sm.bar_g_empty[st], ph ^ 1, abort_flag, status)) break;
@@ -235,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
     const int hf = (warp - 10) >> 2;
     const bool leader = tid == 320;
     int it = 0;
-    for (long long x = x0; x < x1; ++x, ++it) {
+    Tile u = tile_at(x0);
+    for (long long x = x0; x < x1; ++x, ++it, tile_next(u)) {
       const int st = it & 1;
       const uint32_t ph = (it >> 1) & 1;
       if (leader && it > 1) {
@@ -244,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       }
       // exponents of W_t (issued before the wait, used after it): the whole
       // matrix (RMSNorm eps) and the two row blocks of this channel half
-      const long long fi = x / ntile;
+      const long long fi = u.fi;
       const int ew = wexp[fi];
       const int eb0 = wbexp[fi * kWRowBlocks + 2 * hf], eb1 = wbexp[fi * kWRowBlocks + 2 * hf + 1];
       if (!tc::mbar_wait(&sm.bar_acc_full[st], ph, abort_flag, status)) break;
@@ -304,8 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
       tc::fence_proxy_async_smem();
       tc::named_bar(1, 256);
       if (leader) {
-        int h, s0, fb;
-        coords(x, h, s0, fb);
+        const int h = u.h, s0 = u.j * 128, fb = u.b * F + u.t;
         tc::tma_store_4d(&tmO, base, 0, h, s0, fb);
         tc::tma_store_4d(&tmO, base + 16384, 64, h, s0, fb);
         tc::bulk_commit();

@@ -64,6 +64,37 @@ struct __align__(1024) StatsSmem {
 
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 256, true, true);
 
+// Work unit x = pf * nb + j: block j of frame segment pf = (b * F + f) * H + h.  The
+// loops advance it by increments: 64-bit division in every iteration would put a long
+// dependent instruction chain on each role's critical path.
+struct Unit {
+  long long pf;
+  int j, h, f, b;
+};
+__device__ __forceinline__ Unit unit_at(long long x, int nb, int H, int F) {
+  Unit u;
+  u.pf = x / nb;
+  u.j = (int)(x - u.pf * nb);
+  const long long fb = u.pf / H;
+  u.h = (int)(u.pf - fb * H);
+  u.b = (int)(fb / F);
+  u.f = (int)(fb - (long long)u.b * F);
+  return u;
+}
+__device__ __forceinline__ void unit_next(Unit& u, int nb, int H, int F) {
+  if (++u.j == nb) {
+    u.j = 0;
+    ++u.pf;
+    if (++u.h == H) {
+      u.h = 0;
+      if (++u.f == F) {
+        u.f = 0;
+        ++u.b;
+      }
+    }
+  }
+}
+
 
 // byte offset of the 16-byte chunk holding channels 8c..8c+7 of token t in an
 // MN-major SW128 operand of 128 channels x kBT tokens (atoms of 64 channels x
@@ -112,13 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  auto decode = [&](long long x, int& h, int& fb, int& s0) {
-    long long pf = x / nb;
-    s0 = (int)(x % nb) * kBT;
-    h = (int)(pf % H);
-    fb = (int)(pf / H);   // b * F + f
-  };
-  auto seg_last = [&](long long x) { return x + 1 == x1 || (x + 1) % nb == 0; };
+  // the last block of a frame segment: the frame's last block or the CTA's last unit
+  auto seg_last = [&](long long x, const Unit& u) { return x + 1 == x1 || u.j + 1 == nb; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
@@ -132,21 +158,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     for (int r = 0; r < kRS; ++r) slot_head[r] = -1;
     constexpr int BU = kBT / 32;
     float bnext[BU];
-    auto load_beta = [&](long long x) {
-      int h, fb, s0;
-      decode(x, h, fb, s0);
-      const long long nbase = (long long)(fb / F) * N + (long long)(fb % F) * S;
+    auto load_beta = [&](const Unit& un) {
+      const long long nbase = (long long)un.b * N + (long long)un.f * S;
 #pragma unroll
       for (int u = 0; u < BU; ++u) {
-        const int s = s0 + lane + 32 * u;
-        bnext[u] = s < S ? beta[(nbase + s) * H + h] : 0.f;
+        const int s = un.j * kBT + lane + 32 * u;
+        bnext[u] = s < S ? beta[(nbase + s) * H + un.h] : 0.f;
       }
     };
-    if (x0 < x1) load_beta(x0);
+    Unit un = unit_at(x0, nb, H, F);
+    if (x0 < x1) load_beta(un);
     int it = 0;
     for (long long x = x0; x < x1; ++x, ++it) {
-      int h, fb, s0;
-      decode(x, h, fb, s0);
+      const Unit u = un;
+      unit_next(un, nb, H, F);          // the next unit: its beta is loaded during this one
+      const int h = u.h, fb = u.b * F + u.f, s0 = u.j * kBT;
       const int rs = it % kRS;
       const uint32_t ph = (it / kRS) & 1;
       if (!tc::mbar_wait(&sm.raw_empty[rs], ph ^ 1, abort_flag, status)) break;
@@ -158,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       }
 #pragma unroll
       for (int u = 0; u < BU; ++u) sm.sqb[rs][lane + 32 * u] = sqrtf(bnext[u]);
-      if (x + 1 < x1) load_beta(x + 1);
+      if (x + 1 < x1) load_beta(un);
       int cached = slot_head[0];
 #pragma unroll
       for (int r = 0; r < kRS; ++r)
@@ -185,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     if (lane == 0) {
       int it = 0, seg = 0;
       bool first = true;
-      for (long long x = x0; x < x1; ++x, ++it) {
+      Unit u = unit_at(x0, nb, H, F);
+      for (long long x = x0; x < x1; ++x, ++it, unit_next(u, nb, H, F)) {
         const int os = it % kOS;
         const uint32_t oph = (it / kOS) & 1;
         const int ab = seg & 1;
@@ -203,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
         }
         tc::umma_commit(&sm.op_empty[os]);
         first = false;
-        if (seg_last(x)) {
+        if (seg_last(x, u)) {
           tc::umma_commit(&sm.acc_full[ab]);
           ++seg;
           first = true;
@@ -220,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
     const int quarter = warp & 3;
     int seg = 0;
     int it = 0;
-    for (long long x = x0; x < x1; ++x, ++it) {
+    Unit u = unit_at(x0, nb, H, F);
+    for (long long x = x0; x < x1; ++x, ++it, unit_next(u, nb, H, F)) {
       const int rs = it % kRS;
       const uint32_t rph = (it / kRS) & 1;
       const int os = it % kOS;
@@ -313,13 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       tc::fence_proxy_async_smem();   // each thread's stores, then one arrival per warp
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.op_full[os]);
-      if (flusher && seg_last(x)) {
+      const bool last = seg_last(x, u);
+      if (flusher && last) {
         // the segment of this frame is complete once its last block's MMA is:
         // copy the [A | B^T] accumulator rows to partial slot (blockIdx.x + frame)
         const int ab = seg & 1;
         if (!tc::mbar_wait(&sm.acc_full[ab], (seg >> 1) & 1, abort_flag, status)) break;
         tc::tc_fence_after();
-        const long long pf = x / nb;
+        const long long pf = u.pf;
         const int m = quarter * 32 + lane;
         float* dstp = part + ((long long)blockIdx.x + pf) * (128 * 256) + (long long)m * 256;
         const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quarter * 32) << 16);
@@ -335,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.acc_empty[ab]);
       }
-      if (seg_last(x)) ++seg;
+      if (last) ++seg;
     }
   }
 
