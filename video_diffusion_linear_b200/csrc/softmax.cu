@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_wsoft_tc(const __grid_constan
   const int nkt = (int)((k1 - k0 + 127) / 128);
 
   extern __shared__ uint8_t smem_raw[];
-  WsoftSmem& sm = *reinterpret_cast<WsoftSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  WsoftSmem& sm = tc::smem_align<WsoftSmem>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {

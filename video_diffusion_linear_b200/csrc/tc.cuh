@@ -14,6 +14,16 @@ namespace tc {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// The dynamic shared-memory array `raw` viewed as T at the next kAlign-byte boundary
+// (swizzled TMA / UMMA tiles want 1024).  The padding is added to the __shared__ array
+// itself: a round trip through an integer would hide the state space from the compiler,
+// which then addresses every access to T generically (64-bit addresses, generic loads).
+template <typename T, uint32_t kAlign = 1024>
+__device__ __forceinline__ T& smem_align(uint8_t* raw) {
+  const uint32_t pad = (kAlign - (smem_u32(raw) & (kAlign - 1))) & (kAlign - 1);
+  return *reinterpret_cast<T*>(raw + pad);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -116,8 +116,7 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     float* __restrict__ dWall, float* __restrict__ rms_part, __nv_bfloat16* __restrict__ dq,
     __nv_bfloat16* __restrict__ dgate, int H, int F, int S, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  ReadoutTcSmem& sm =
-      *reinterpret_cast<ReadoutTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  ReadoutTcSmem& sm = tc::smem_align<ReadoutTcSmem>(smem_raw);
   const long long fi = blockIdx.x;
   const int f = (int)(fi % F);
   const long long bh = fi / F;
@@ -402,7 +401,7 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
                                                                 float* __restrict__ dbeta, int H, int F, int S,
                                                                 uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  StatsTcSmem& sm = *reinterpret_cast<StatsTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  StatsTcSmem& sm = tc::smem_align<StatsTcSmem>(smem_raw);
   const long long fi = blockIdx.x;
   const long long NFt = gridDim.x;
   const int f = (int)(fi % F);
@@ -622,7 +621,7 @@ __global__ void __launch_bounds__(kBwdScanThreads, 1) k_bwd_scan_tc(const uint16
                                                                     float* __restrict__ dseed2, int H, int F,
                                                                     uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  BwdScanSmem& sm = *reinterpret_cast<BwdScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdScanSmem& sm = tc::smem_align<BwdScanSmem>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m = 32 * (warp & 3) + lane;     // state row = TMEM lane
   const int k0 = 64 * (tid >> 7);           // column half

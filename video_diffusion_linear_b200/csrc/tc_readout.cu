@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_readout_tc(const __grid_constan
                                                            const float* __restrict__ rms_w, int H, int F,
                                                            int ntile, long long T, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  ReadSmem& sm = *reinterpret_cast<ReadSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  ReadSmem& sm = tc::smem_align<ReadSmem>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = &sm.abort;
   const long long G = gridDim.x;

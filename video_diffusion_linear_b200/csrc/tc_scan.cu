@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
                                                             float* __restrict__ maps, int* __restrict__ map_exp,
                                                             int nch_stride, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  ScanSmem& sm = tc::smem_align<ScanSmem>(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int m = 32 * (warp & 3) + lane;     // state row (v channel) = TMEM lane

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
                                                          int K, int H, int F, int S, int nb, long long T,
                                                          float* __restrict__ part, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  StatsSmem& sm = *reinterpret_cast<StatsSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  StatsSmem& sm = tc::smem_align<StatsSmem>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = &sm.abort;
   const long long G = gridDim.x;
