@@ -34,7 +34,7 @@ struct __align__(1024) ScanSmem {
   uint8_t nimg[65536];       // N_f hi | lo image
   float bf[4][128 * 32];     // B_f, four swizzled [128 rows][32 cols] boxes
   float alpha[128];
-  uint64_t bar_n, bar_b, bar_mma, bar_nhi;
+  uint64_t bar_n[2], bar_b, bar_mma, bar_nlo;   // bar_n[part]: N_f hi / lo landed; bar_nlo: N_lo read
   uint32_t tmem_base;
   int abort;
 };
@@ -65,6 +65,8 @@ __device__ __forceinline__ void split_pair(float2 x, uint32_t& hi, uint32_t& lo)
 // the whole-clip instantiation carries none of the segment mode's work
 template <int kMode>
 __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmB,
+                                                            const __grid_constant__ CUtensorMap tmP,
+                                                            const __grid_constant__ CUtensorMap tmQ,
                                                             const uint16_t* __restrict__ nimg_g,
                                                             const float* __restrict__ alpha,
                                                             const float* __restrict__ text, RuleCoef rc,
@@ -87,10 +89,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   volatile int* abort_flag = &sm.abort;
 
   if (tid == 0) {
-    tc::mbar_init(&sm.bar_n, 1);
+    tc::mbar_init(&sm.bar_n[0], 1);
+    tc::mbar_init(&sm.bar_n[1], 1);
     tc::mbar_init(&sm.bar_b, 1);
     tc::mbar_init(&sm.bar_mma, 1);
-    tc::mbar_init(&sm.bar_nhi, 1);
+    tc::mbar_init(&sm.bar_nlo, 1);
     sm.abort = 0;
     tc::fence_barrier_init();
   }
@@ -108,23 +111,26 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
   {
     const float* T = text ? text + ((long long)h * 128 + m) * 128 + k0 : nullptr;
 #pragma unroll
-    for (int p = 0; p < 32; ++p)
-      s[p] = T ? make_float2(kTextStateScale * T[2 * p], kTextStateScale * T[2 * p + 1]) : make_float2(0.f, 0.f);
+    for (int p = 0; p < 32; p += 2) {   // the text state is 16-byte aligned (checked on entry)
+      const float4 t4 = T ? *reinterpret_cast<const float4*>(T + 2 * p) : make_float4(0.f, 0.f, 0.f, 0.f);
+      s[p] = make_float2(kTextStateScale * t4.x, kTextStateScale * t4.y);
+      s[p + 1] = make_float2(kTextStateScale * t4.z, kTextStateScale * t4.w);
+    }
   }
 
   auto frame_of = [&](int step) { return dir == 0 ? step : F - 1 - step; };
   // segment mode: first and last frame of a chunk in this direction's order
   auto seg_first = [&](int f) { return dir == 0 ? f % chunk == 0 : ((f + 1) % chunk == 0 || f == F - 1); };
   auto seg_last = [&](int f) { return dir == 0 ? ((f + 1) % chunk == 0 || f == F - 1) : f % chunk == 0; };
-  // N_f image: the hi part (first 32 KB) and the lo part arrive on the same
-  // barrier but are requested separately, each as soon as its buffer is free
+  // N_f image: the hi part (first 32 KB) and the lo part each land on their own
+  // barrier and are requested as soon as their buffer is free
   auto load_n_part = [&](int step, int part) {
     long long fi = bh * F + frame_of(step);
     const uint8_t* src = reinterpret_cast<const uint8_t*>(nimg_g + fi * (kImgBytes / 2)) + part * 32768;
-    if (part == 0) tc::mbar_arrive_expect_tx(&sm.bar_n, kImgBytes);
+    tc::mbar_arrive_expect_tx(&sm.bar_n[part], kImgBytes / 2);
 #pragma unroll
     for (int j = 0; j < 2; ++j)
-      tc::bulk_load(sm.nimg + part * 32768 + j * 16384, src + j * 16384, 16384, &sm.bar_n);
+      tc::bulk_load(sm.nimg + part * 32768 + j * 16384, src + j * 16384, 16384, &sm.bar_n[part]);
   };
   auto load_b = [&](int step) {
     long long fi = bh * F + frame_of(step);
@@ -167,6 +173,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
       if (step + 1 < F) a_next = alpha[((b * F + frame_of(step + 1)) * H + h) * 128 + tid];   // used next step
     }
     if (tid == 0 && step + 2 < F) prefetch(step + 2);
+    if (tid == 0) tc::bulk_wait_read_all();   // a state store still reading the X buffers
     __syncthreads();
     if (!tc::mbar_wait(&sm.bar_b, ph, abort_flag, status)) break;
 
@@ -198,36 +205,46 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
 
     if (tid == 0) {
       if (early_b && step + 1 < F) load_b(step + 1);
-      if (tc::mbar_wait(&sm.bar_n, ph, abort_flag, status)) {
+      // Xh Nl first: N_lo is free a third of the product in, and the next frame's
+      // N_lo loads meanwhile; the next frame's N_hi, requested once the whole
+      // product is done, has until after that frame's Xh Nl terms
+      if (tc::mbar_wait(&sm.bar_n[1], ph, abort_flag, status)) {
         tc::tc_fence_after();
-        // the terms with N_hi first (Xh Nh, Xl Nh), then Xh Nl: N_hi is free a
-        // third of the product earlier, and the next frame's N_hi can load
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          uint64_t ah = tc::smem_desc(a_hi + koff, 16, 1024), al = tc::smem_desc(a_lo + koff, 16, 1024);
-          uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024);
-          tc::umma_bf16(tmem, ah, bhd, kIdesc, kk > 0 ? 1u : 0u);
-          tc::umma_bf16(tmem, al, bhd, kIdesc, 1u);
+          tc::umma_bf16(tmem, tc::smem_desc(a_hi + koff, 16, 1024), tc::smem_desc(n_lo + koff, 16, 1024), kIdesc,
+                        kk > 0 ? 1u : 0u);
         }
-        tc::umma_commit(&sm.bar_nhi);
+        tc::umma_commit(&sm.bar_nlo);
+        if (tc::mbar_wait(&sm.bar_n[0], ph, abort_flag, status)) {
+          tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::umma_bf16(tmem, tc::smem_desc(a_hi + koff, 16, 1024), tc::smem_desc(n_lo + koff, 16, 1024), kIdesc, 1u);
+          for (int kk = 0; kk < 8; ++kk) {
+            uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+            uint64_t ah = tc::smem_desc(a_hi + koff, 16, 1024), al = tc::smem_desc(a_lo + koff, 16, 1024);
+            uint64_t bhd = tc::smem_desc(n_hi + koff, 16, 1024);
+            tc::umma_bf16(tmem, ah, bhd, kIdesc, 1u);
+            tc::umma_bf16(tmem, al, bhd, kIdesc, 1u);
+          }
+          tc::umma_commit(&sm.bar_mma);
         }
-        tc::umma_commit(&sm.bar_mma);
-        if (step + 1 < F && tc::mbar_wait(&sm.bar_nhi, ph, abort_flag, status)) load_n_part(step + 1, 0);
       }
+    } else if (tid == 32 && step + 1 < F) {
+      // the copies are requested by a thread of their own: the issuing thread stays
+      // blocked in the MMA queue until its last product is accepted
+      if (tc::mbar_wait(&sm.bar_nlo, ph, abort_flag, status)) load_n_part(step + 1, 1);
     }
     if (!tc::mbar_wait(&sm.bar_mma, ph, abort_flag, status)) break;
     tc::tc_fence_after();
-    if (tid == 0 && step + 1 < F) load_n_part(step + 1, 1);   // the product that read N_lo is complete
+    if (tid == 32 && step + 1 < F) load_n_part(step + 1, 0);   // the product that read N_hi is complete
 
     // S_f = D + cpost B_f
     const bool seg_store = kMode != kScanWhole && seg_last(f);
     const bool store = kMode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
-    float* dst = kMode == kScanWhole ? (dir == 0 ? P : Q) + fi * 128 * 128 + (long long)m * 128 + k0 : nullptr;
+    // whole clip: the stored state goes out through the (now free) X buffers and a TMA
+    // store, row-major and coalesced, in the swizzled [rows][32 cols] boxes of bf_offset
+    uint8_t* stage = sm.aop[0];
     // segment mode: map slot [b, h][dir][chunk][G_c | O_c][row][col]; the map is 2^ex times the stored state
     const long long mslot = ((bh * 2 + dir) * nch_stride + f / chunk) * 2 + (kMode == kScanSegIdentity ? 0 : 1);
     float* mdst = kMode == kScanWhole ? nullptr : maps + (mslot * 128 + m) * 128 + k0;
@@ -249,13 +266,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
                               make_float2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])));
         amax = fmaxf(amax, fmaxf(fmaxf(fabsf(s[p].x), fabsf(s[p].y)), fmaxf(fabsf(s[p + 1].x), fabsf(s[p + 1].y))));
         if (store)
-          *reinterpret_cast<float4*>(dst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
+          *reinterpret_cast<float4*>(stage + bf_offset(m, k0 + 32 * j + e)) =
+              make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
         if (seg_store)
           *reinterpret_cast<float4*>(mdst + 32 * j + e) = make_float4(s[p].x, s[p].y, s[p + 1].x, s[p + 1].y);
       }
     }
     if (store && tid == 0) (dir == 0 ? pexp : qexp)[fi] = ex;
     if (seg_store && tid == 0) map_exp[mslot] = ex;
+    if (store) tc::fence_proxy_async_smem();   // the staged rows, before the barrier and the TMA store
     tc::tc_fence_before();
     // accumulator and B_f reads done, alpha slot free; rescale if any entry passed
     // kRenormAbove (2^32)
@@ -264,14 +283,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
       for (int p = 0; p < 32; ++p) s[p] = __fmul2_rn(s[p], make_float2(kRenormScale, kRenormScale));
       ex += kRenormExp;
     }
+    if (store && tid == 0) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tc::tma_store_2d(dir == 0 ? &tmP : &tmQ, stage + j * 16384, 32 * j, (int)(fi * 128));
+      tc::bulk_commit();
+    }
     if (tid == 0 && !early_b && step + 1 < F) load_b(step + 1);
     ph ^= 1;
   }
 
   // teardown: make sure no copy or product of ours is still in flight
+  if (tid == 0) tc::bulk_wait_all();
   __syncthreads();
   if (sm.abort && tid == 0) {
-    tc::mbar_wait(&sm.bar_n, ph, abort_flag, nullptr);
+    tc::mbar_wait(&sm.bar_n[0], ph, abort_flag, nullptr);
+    tc::mbar_wait(&sm.bar_n[1], ph, abort_flag, nullptr);
     tc::mbar_wait(&sm.bar_b, ph, abort_flag, nullptr);
   }
   __syncthreads();
@@ -281,8 +307,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
 cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nimg, float* P, float* Q, int* pexp,
                            int* qexp, bool all_frames, uint32_t* status, int seg_mode, float* maps, int* map_exp,
                            int nch_stride) {
-  CUtensorMap tmB;
+  CUtensorMap tmB, tmP, tmQ;
   if (!tmap_rows_f32(&tmB, Bsum, a.NF() * 128)) return cudaErrorInvalidValue;
+  // P / Q: [B H F][128][128] fp32 state stores (segment modes store maps directly: placeholders)
+  if (!tmap_rows_f32(&tmP, P ? (const void*)P : (const void*)Bsum, a.NF() * 128) ||
+      !tmap_rows_f32(&tmQ, Q ? (const void*)Q : (const void*)Bsum, a.NF() * 128))
+    return cudaErrorInvalidValue;
   size_t smem = sizeof(ScanSmem) + 1024;
   cudaError_t e;
   RuleCoef rc = rule_coef(a.rule, a.c);
@@ -292,7 +322,7 @@ cudaError_t launch_scan_tc(const Args& a, const float* Bsum, const uint16_t* nim
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)(2LL * a.sh.B * a.sh.H), kScanThreads, smem, a.stream>>>(
-      tmB, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, maps,
+      tmB, tmP, tmQ, nimg, a.alpha, a.text_state, rc, P, Q, pexp, qexp, a.sh.H, a.sh.F, a.chunk, all_frames ? 1 : 0, maps,
       map_exp, nch_stride, status);
   return cudaGetLastError();
 }
