@@ -40,7 +40,7 @@ struct WsPlan {
   // block exponents: a stored state X means 2^e X (int32 [B, H, F] each)
   size_t pexp = 0, qexp = 0, wexp = 0;
   // tensor-core path
-  size_t part = 0;                      // fp32 [slots][d][2d]: rows of [A | B^T] partial sums
+  size_t part = 0;                      // fp32 [slots][2d][d]: partial sums laid out [A; B]
   size_t nimg = 0;                      // bf16 [B,H,F][2][d][d] operand images (hi, lo) of N_f
   size_t wimg = 0;                      // fp16 [B,H,F][d][d] read-out operand images of W_t
   size_t wbexp = 0;                     // int32 [B,H,F][4] row-block exponents of those images

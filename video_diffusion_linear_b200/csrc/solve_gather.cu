@@ -49,8 +49,8 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
 #pragma unroll
       for (int ib = 0; ib < R; ++ib) a[ia][ib] = Af[(ty + 16 * ia) * D + tx + 16 * ib];
   } else {
-    // Sum the partial [A | B^T] rows written by the statistics CTAs that
-    // covered this frame (frames are processed in (b, f, h) order there).
+    // Sum the partial slots ([A; B], 256 rows of 128) written by the statistics
+    // CTAs that covered this frame (frames are processed in (b, f, h) order there).
     long long pf = ((long long)b * F + f) * H + h;
     long long x0 = pf * nb, x1 = x0 + nb - 1;
     int i0 = sk_owner(x0, Tblocks, G), i1 = sk_owner(x1, Tblocks, G);
@@ -60,18 +60,18 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
       for (int ib = 0; ib < R; ++ib) a[ia][ib] = 0.f;
     for (int e = tid; e < D * D; e += 256) stage[(e / D) * LD + (e % D)] = 0.f;
     for (int ci = i0; ci <= i1; ++ci) {
-      const float* p = part + (long long)(ci + pf) * (D * 2 * D);
+      const float* p = part + (long long)(ci + pf) * (2 * D * D);
 #pragma unroll
       for (int ia = 0; ia < R; ++ia)
 #pragma unroll
-        for (int ib = 0; ib < R; ++ib) a[ia][ib] += p[(ty + 16 * ia) * (2 * D) + tx + 16 * ib];
-      // B^T half of the slot: float4 loads, all issued before use
+        for (int ib = 0; ib < R; ++ib) a[ia][ib] += p[(ty + 16 * ia) * D + tx + 16 * ib];
+      // B rows of the slot: float4 loads, all issued before use
       constexpr int NV4 = D * D / 4, NV = (NV4 + 255) / 256;
       float4 bv[NV];
 #pragma unroll
       for (int r = 0; r < NV; ++r) {
         const int e4 = tid + 256 * r, row = e4 / (D / 4), c4 = e4 % (D / 4);
-        if (e4 < NV4) bv[r] = *reinterpret_cast<const float4*>(p + row * (2 * D) + D + 4 * c4);
+        if (e4 < NV4) bv[r] = *reinterpret_cast<const float4*>(p + D * D + row * D + 4 * c4);
       }
 #pragma unroll
       for (int r = 0; r < NV; ++r) {
@@ -83,8 +83,8 @@ __global__ void __launch_bounds__(256) k_solve(const float* __restrict__ A, cons
       }
     }
     __syncthreads();
-    float* Bf = Bsum + fi * D * D;   // B[i][j] = (B^T)[j][i]
-    for (int e = tid; e < D * D; e += 256) Bf[e] = stage[(e % D) * LD + (e / D)];
+    float* Bf = Bsum + fi * D * D;
+    for (int e = tid; e < D * D; e += 256) Bf[e] = stage[(e / D) * LD + (e % D)];
     if (Aout) {
 #pragma unroll
       for (int ia = 0; ia < R; ++ia)
@@ -223,52 +223,51 @@ __global__ void __launch_bounds__(kSolveThreads, 3) k_solve128(const float* __re
   const long long x0 = pf * nb, x1 = x0 + nb - 1;
   const int i0 = sk_owner(x0, Tblocks, G), i1 = sk_owner(x1, Tblocks, G);
 
-  // ---- B = (B^T)^T: 4 x 8 pieces of B^T, summed and written transposed
+  // ---- B: rows 128 .. 255 of the frame's partial slots ([A; B], 256 rows of 128),
+  // summed with coalesced 16-byte accesses, eight in flight per thread and slot
   {
-    float* Bf = Bsum + fi * D * D;
-    for (int q = tid; q < 512; q += kSolveThreads) {
-      const int ib = q >> 5, jb = (q >> 1) & 15, hf = q & 1;   // B rows 8 ib.., B columns 8 jb + 4 hf ..
-      float acc[4][8];
+    constexpr int NV4 = D * D / 4;
+    float4* Bf = reinterpret_cast<float4*>(Bsum + fi * D * D);
+    for (int e0 = tid; e0 < NV4; e0 += 8 * kSolveThreads) {
+      float4 acc[8];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+      for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int ci = i0; ci <= i1; ++ci) {
-        const float* pp = part + (long long)(ci + pf) * (D * 2 * D) + (8 * jb + 4 * hf) * (2 * D) + D + 8 * ib;
-        float4 v[4][2];
+        const float4* src = reinterpret_cast<const float4*>(part + (long long)(ci + pf) * (2 * D * D) + D * D);
+        float4 v[8];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          v[r][0] = *reinterpret_cast<const float4*>(pp + r * (2 * D));
-          v[r][1] = *reinterpret_cast<const float4*>(pp + r * (2 * D) + 4);
+        for (int u = 0; u < 8; ++u) {
+          const int e4 = e0 + u * kSolveThreads;
+          v[u] = e4 < NV4 ? src[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          acc[r][0] += v[r][0].x; acc[r][1] += v[r][0].y; acc[r][2] += v[r][0].z; acc[r][3] += v[r][0].w;
-          acc[r][4] += v[r][1].x; acc[r][5] += v[r][1].y; acc[r][6] += v[r][1].z; acc[r][7] += v[r][1].w;
+        for (int u = 0; u < 8; ++u) {
+          acc[u].x += v[u].x; acc[u].y += v[u].y; acc[u].z += v[u].z; acc[u].w += v[u].w;
         }
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c)   // B[8 ib + c][8 jb + 4 hf + r] = B^T[8 jb + 4 hf + r][8 ib + c]
-        *reinterpret_cast<float4*>(Bf + (8 * ib + c) * D + 8 * jb + 4 * hf) =
-            make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
+      for (int u = 0; u < 8; ++u) {
+        const int e4 = e0 + u * kSolveThreads;
+        if (e4 < NV4) Bf[e4] = acc[u];
+      }
     }
   }
 
-  // ---- A: sum this block of the [A | B^T] partial slots of the frame
+  // ---- A: sum this block of the A rows (0 .. 127) of the frame's partial slots
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int p = 0; p < 4; ++p) a[i][p] = make_float2(0.f, 0.f);
   if (owner) {
     for (int ci = i0; ci <= i1; ++ci) {
-      const float* pp = part + (long long)(ci + pf) * (D * 2 * D) + r0 * (2 * D) + c0;
+      const float* pp = part + (long long)(ci + pf) * (2 * D * D) + r0 * D + c0;
 #pragma unroll
       for (int ih = 0; ih < 8; ih += 4) {   // four rows (8 float4) in flight
         float4 v[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          v[i][0] = *reinterpret_cast<const float4*>(pp + (ih + i) * (2 * D));
-          v[i][1] = *reinterpret_cast<const float4*>(pp + (ih + i) * (2 * D) + 4);
+          v[i][0] = *reinterpret_cast<const float4*>(pp + (ih + i) * D);
+          v[i][1] = *reinterpret_cast<const float4*>(pp + (ih + i) * D + 4);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -18,8 +18,9 @@
 // Work split: the (frame, 96-token block) pairs, frames ordered (batch, frame,
 // head), are cut into gridDim.x contiguous ranges (stream-K).  A CTA flushes its
 // accumulator whenever its range leaves a frame, into partial slot
-// (blockIdx.x + frame); the per-frame solve adds the slots of each frame in a
-// fixed order, so the result is deterministic.
+// (blockIdx.x + frame), laid out [A; B] (256 rows of 128 floats); the per-frame
+// solve adds the slots of each frame in a fixed order, so the result is
+// deterministic.
 //
 // Warp roles (448 threads): 0 TMA producer, 1 MMA issuer (TMEM owner),
 // 2-13 transform (4 tokens x 8 channels per thread); transform warps 2-5 (one
@@ -343,14 +344,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       if (lane == 0) tc::mbar_arrive(&sm.op_full[os]);
       const bool last = seg_last(x, u);
       if (flusher && last) {
-        // the segment of this frame is complete once its last block's MMA is:
-        // copy the [A | B^T] accumulator rows to partial slot (blockIdx.x + frame)
+        // the segment of this frame is complete once its last block's MMA is: copy
+        // the accumulator to partial slot (blockIdx.x + frame) as [A; B], 256 rows of
+        // 128: TMEM lane m holds row m of [A | B^T], i.e. column m of A (symmetric) and
+        // of B, which the warp's lanes write as consecutive floats of each slot row
         const int ab = seg & 1;
         if (!tc::mbar_wait(&sm.acc_full[ab], (seg >> 1) & 1, abort_flag, status)) break;
         tc::tc_fence_after();
         const long long pf = u.pf;
         const int m = quarter * 32 + lane;
-        float* dstp = part + ((long long)blockIdx.x + pf) * (128 * 256) + (long long)m * 256;
+        float* dstp = part + ((long long)blockIdx.x + pf) * (256 * 128) + m;
         const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
         for (int j = 0; j < 8; ++j) {
@@ -358,8 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           tc::tmem_ld32(taddr + 32 * j, r);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<uint4*>(dstp + 32 * j + e) = make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+          for (int e = 0; e < 32; ++e) dstp[(32 * j + e) * 128] = __uint_as_float(r[e]);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.acc_empty[ab]);
