@@ -19,6 +19,7 @@
 #include "image.cuh"
 #include "internal.h"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace vdn {
 namespace {
@@ -389,7 +390,9 @@ __device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128]
 // column halves 64 hf .. 64 hf + 63 (hf = w / 4); per-token sums are combined in shared memory.
 constexpr int kStatsThreads = 256;
 
-__global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_constant__ CUtensorMap tmDK,
+                                                                const __grid_constant__ CUtensorMap tmDV,
+                                                                const __nv_bfloat16* __restrict__ k,
                                                                 const __nv_bfloat16* __restrict__ v,
                                                                 const float* __restrict__ beta,
                                                                 const float* __restrict__ wk,
@@ -461,23 +464,30 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
   for (int s0 = 0; s0 < S && ok; s0 += kBT) {
     const int s = s0 + m;
     const bool valid = s < S;
-    // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame)
-    for (int r = tid; r < kRawRows; r += kStatsThreads) {
-      const int sr = s0 - 1 + r;
-      const bool in = sr >= 0 && sr < S;
-      const long long base = ((frame_row0 + (in ? sr : 0)) * H + h) * 128;
-      uint4 kb[16], vb[16];
+    // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame): sixteen
+    // threads per row, so each warp reads two whole 256-byte rows; all loads issued first
+    {
+      constexpr int kChunks = kRawRows * 16, kIt = (kChunks + kStatsThreads - 1) / kStatsThreads;
+      uint4 kb[kIt], vb[kIt];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        kb[c] = in ? *reinterpret_cast<const uint4*>(k + base + 8 * c) : make_uint4(0, 0, 0, 0);
-        vb[c] = in ? *reinterpret_cast<const uint4*>(v + base + 8 * c) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < kIt; ++u) {
+        const int idx = tid + u * kStatsThreads, r = idx >> 4, c = idx & 15;
+        const int sr = s0 - 1 + r;
+        const bool in = idx < kChunks && sr >= 0 && sr < S;
+        const long long off = ((frame_row0 + (in ? sr : 0)) * H + h) * 128 + 8 * c;
+        kb[u] = in ? *reinterpret_cast<const uint4*>(k + off) : make_uint4(0, 0, 0, 0);
+        vb[u] = in ? *reinterpret_cast<const uint4*>(v + off) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        *reinterpret_cast<uint4*>(sm.kraw + r * kRawStride + 16 * c) = kb[c];
-        *reinterpret_cast<uint4*>(sm.vraw + r * kRawStride + 16 * c) = vb[c];
+      for (int u = 0; u < kIt; ++u) {
+        const int idx = tid + u * kStatsThreads, r = idx >> 4, c = idx & 15;
+        if (idx < kChunks) {
+          *reinterpret_cast<uint4*>(sm.kraw + r * kRawStride + 16 * c) = kb[u];
+          *reinterpret_cast<uint4*>(sm.vraw + r * kRawStride + 16 * c) = vb[u];
+        }
       }
     }
+    if (tid == 0) tc::bulk_wait_read_all();   // the previous tile's gradient stores left kf / vf
     __syncthreads();
     // x = silu(conv k) (k' = x / |x|: the 1/|x| is applied to U and Z in the epilogue) and
     // v' = silu(conv v) into the K', V' tiles: this thread's 8 chunks of its token
@@ -572,15 +582,27 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __nv_bfloa
           gk[e] = (dk - x * xg * inv * inv) * inv * sg * fmaf(kc[e], 1.f - sg, 1.f);
           gv[e] = silu_grad_f(vc[e], bt * inv * __uint_as_float(z[q8]));
         }
-        // bf16, as the gradients they feed (dk, dv) are written
-        store8_bf16(dkc + tok * 128 + c0, gk);
-        store8_bf16(dvc + tok * 128 + c0, gv);
+        // bf16, as the gradients they feed (dk, dv) are written: into the (read) K', V'
+        // tiles, which leave through TMA stores in the same layout
+        store_chunk_bf16(sm.kf, m, c0, gk);
+        store_chunk_bf16(sm.vf, m, c0, gv);
       }
     }
+    tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    if (tid == 0) {   // rows past the frame end are clipped by the tensor maps
+      const int fb = (int)(b * F + f);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tc::tma_store_4d(&tmDK, sm.kf + hh * 16384, 64 * hh, h, s0, fb);
+        tc::tma_store_4d(&tmDV, sm.vf + hh * 16384, 64 * hh, h, s0, fb);
+      }
+      tc::bulk_commit();
+    }
   }
+  if (tid == 0) tc::bulk_wait_all();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -775,10 +797,15 @@ cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* 
 cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, void* dkc, void* dvc,
                                 float* dbeta, uint32_t* status) {
   const size_t smem = sizeof(StatsTcSmem) + 1024;
+  CUtensorMap tdk, tdv;
+  const long long BF = (long long)a.sh.B * a.sh.F;
+  if (!tmap_tokens_bf16(&tdk, dkc, a.sh.d, a.sh.H, a.sh.S, BF, kBT) ||
+      !tmap_tokens_bf16(&tdv, dvc, a.sh.d, a.sh.H, a.sh.S, BF, kBT))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_bwd_stats_tc<<<(unsigned)a.NF(), kStatsThreads, smem, a.stream>>>(
-      static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
+      tdk, tdv, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
       a.conv_v_w, K, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
       a.sh.F, a.sh.S, status);
   return cudaGetLastError();
