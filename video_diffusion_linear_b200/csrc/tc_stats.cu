@@ -198,7 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
           if (!wg) val = tap == 1 ? 1.f : 0.f;                       // identity
           else if (K == 3) val = wg[((long long)h * 128 + ch) * 3 + tap];
           else val = tap == 1 ? wg[(long long)h * 128 + ch] : 0.f;   // one tap: centre
-          sm.taps[rs][ten][tap][ch] = 0.5f * val;
+          // [tap][quad parity][chunk]: a quarter warp's 8 chunks are 128 contiguous bytes
+          sm.taps[rs][ten][tap][((ch >> 2) & 1) * 64 + (ch >> 3) * 4 + (ch & 3)] = 0.5f * val;
         }
 #pragma unroll
         for (int r = 0; r < kRS; ++r)
@@ -257,7 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
       if (!tc::mbar_wait(&sm.raw_full[rs], rph, abort_flag, status)) break;
       float sb[kTPT];
 #pragma unroll
-      for (int i = 0; i < kTPT; ++i) sb[i] = sm.sqb[rs][tok0 + i];
+      for (int i = 0; i < kTPT; i += 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&sm.sqb[rs][tok0 + i]);
+        sb[i] = q4.x; sb[i + 1] = q4.y; sb[i + 2] = q4.z; sb[i + 3] = q4.w;
+      }
 
       // y = SiLU(conv(x)) = h + h tanh(h), h = conv(x) / 2 (the taps carry the 1/2);
       // ss = sum of y^2 over this thread's channels
@@ -265,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_stats_tc(const __grid_constant_
         float2 w3[3][4];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-          const float4 a = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c]);
-          const float4 b = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][8 * c + 4]);
+          const float4 a = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][4 * c]);
+          const float4 b = *reinterpret_cast<const float4*>(&sm.taps[rs][ten][j][64 + 4 * c]);
           w3[j][0] = make_float2(a.x, a.y); w3[j][1] = make_float2(a.z, a.w);
           w3[j][2] = make_float2(b.x, b.y); w3[j][3] = make_float2(b.z, b.w);
         }
