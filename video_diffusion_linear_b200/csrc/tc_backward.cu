@@ -402,17 +402,10 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
                                                                 __nv_bfloat16* __restrict__ dkc,
                                                                 __nv_bfloat16* __restrict__ dvc,
                                                                 float* __restrict__ dbeta, int H, int F, int S,
-                                                                uint32_t* __restrict__ status) {
+                                                                long long NFt, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   StatsTcSmem& sm = tc::smem_align<StatsTcSmem>(smem_raw);
-  const long long fi = blockIdx.x;
-  const long long NFt = gridDim.x;
-  const int f = (int)(fi % F);
-  const long long bh = fi / F;
-  const int h = (int)(bh % H);
-  const long long b = bh / H;
   const long long N = (long long)F * S;
-  const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, hf = warp >> 2;
   const int m = 32 * quarter + lane;                       // token of the tile = TMEM lane
@@ -427,31 +420,6 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
     tc::tmem_alloc(&sm.tmem_base, 512);
     tc::tmem_relinquish();
   }
-  // images of dA + dA^T (threads 0..127, row = tid) and dB (threads 128..255), both scans' parts summed
-  {
-    const int i = tid & 127;
-    const float* x0 = (tid < 128 ? dA2 : dB2) + fi * 16384;
-    const float* x1 = (tid < 128 ? dA2 : dB2) + (NFt + fi) * 16384;
-    uint8_t* img = tid < 128 ? sm.da : sm.db;
-    for (int c = 0; c < 16; ++c) {
-      float va[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = 8 * c + e;
-        va[e] = x0[i * 128 + j] + x1[i * 128 + j];
-        if (tid < 128) va[e] += x0[j * 128 + i] + x1[j * 128 + i];
-      }
-      store_chunk_bf16(img, i, 8 * c, va);
-    }
-    // taps of this head, [tensor][tap][channel]; a missing conv is the identity (one centre tap)
-    if (tid < 128)
-      for (int j = 0; j < 3; ++j) {
-        const bool centre = j == (Kc - 1) / 2;
-        sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
-        sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
-      }
-  }
-  tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -459,9 +427,53 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
   const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
   const uint32_t a_da = tc::smem_u32(sm.da), a_db = tc::smem_u32(sm.db), a_k = tc::smem_u32(sm.kf),
                  a_v = tc::smem_u32(sm.vf);
+  // persistent: CTA i takes the contiguous range [i T / G, (i + 1) T / G) of the (frame, tile)
+  // units, T = B H F x tiles per frame, so no wave is left partly empty; the frame's operand
+  // images and taps are rebuilt whenever the range enters a new frame
+  const int ntile = (S + kBT - 1) / kBT;
+  const long long T = NFt * ntile, G = gridDim.x;
+  const long long u0 = (long long)blockIdx.x * T / G, u1 = ((long long)blockIdx.x + 1) * T / G;
+  long long cur = -1;
   uint32_t ph = 0;
   bool ok = true;
-  for (int s0 = 0; s0 < S && ok; s0 += kBT) {
+  for (long long u = u0; u < u1 && ok; ++u) {
+    const long long fi = u / ntile;
+    const int s0 = (int)(u - fi * ntile) * kBT;
+    const int f = (int)(fi % F);
+    const long long bh = fi / F;
+    const int h = (int)(bh % H);
+    const long long b = bh / H;
+    const long long frame_row0 = b * N + (long long)f * S;   // token row of s = 0
+    if (fi != cur) {
+      // images of dA + dA^T (threads 0..127, row = tid) and dB (threads 128..255), both scans'
+      // parts summed (the previous tile's products and reads of them are complete)
+      const int i = tid & 127;
+      const float* x0 = (tid < 128 ? dA2 : dB2) + fi * 16384;
+      const float* x1 = (tid < 128 ? dA2 : dB2) + (NFt + fi) * 16384;
+      uint8_t* img = tid < 128 ? sm.da : sm.db;
+      for (int c = 0; c < 16; ++c) {
+        float va[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = 8 * c + e;
+          va[e] = x0[i * 128 + j] + x1[i * 128 + j];
+          if (tid < 128) va[e] += x0[j * 128 + i] + x1[j * 128 + i];
+        }
+        store_chunk_bf16(img, i, 8 * c, va);
+      }
+      // taps of this head, [tensor][tap][channel]; a missing conv is the identity (one centre tap)
+      if (tid < 128)
+        for (int j = 0; j < 3; ++j) {
+          const bool centre = j == (Kc - 1) / 2;
+          sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+          sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+        }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      tc::tc_fence_after();
+      cur = fi;
+    }
     const int s = s0 + m;
     const bool valid = s < S;
     // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame): sixteen
@@ -804,10 +816,12 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_bwd_stats_tc<<<(unsigned)a.NF(), kStatsThreads, smem, a.stream>>>(
+  const long long units = a.NF() * ((a.sh.S + kBT - 1) / kBT);
+  const unsigned grid = (unsigned)(units < kStatsGrid ? units : kStatsGrid);   // one CTA per SM
+  k_bwd_stats_tc<<<grid, kStatsThreads, smem, a.stream>>>(
       tdk, tdv, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
       a.conv_v_w, K, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
-      a.sh.F, a.sh.S, status);
+      a.sh.F, a.sh.S, a.NF(), status);
   return cudaGetLastError();
 }
 
