@@ -849,6 +849,10 @@ BwdPlan plan_backward(const vdn_shape& sh, int rule, bool recompute) {
   p.dX_all = take(2 * NF * DD * 4);
   p.Xbuf = rule == VDN_RULE_SANA_SCALED ? take(2 * NF * DD * 4) : 0;
   p.rms_part = take(NF * sh.d * 4);
+  if (sh.d == 128 && sh.dtype == VDN_DTYPE_BF16) {   // the tensor-core read-out reversal's slots
+    p.dW_slots = take((NF + kBwdReadoutGrid) * DD * 4);
+    p.rms_slots = take((NF + kBwdReadoutGrid) * sh.d * 4);
+  }
   p.dkc = take(tokens * sh.d * el);          // the inputs' element type (bf16 on the tensor-core path)
   p.dvc = take(tokens * sh.d * el);
   p.tap_part = take((size_t)sh.H * kBwdConvBlocks * 2 * sh.d * 3 * 4);
@@ -874,8 +878,8 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, const BwdSta
   uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p.status);   // first word of the workspace
   // step 5 reversed
   if (kTc) {
-    if ((e = launch_bwd_readout_tc(a, g.dout, st.W, at(p.dW), at(p.rms_part), g.dq, g.dgate, status)) !=
-        cudaSuccess)
+    if ((e = launch_bwd_readout_tc(a, g.dout, st.W, at(p.dW), at(p.rms_part), at(p.dW_slots), at(p.rms_slots),
+                                   g.dq, g.dgate, status)) != cudaSuccess)
       return e;
   } else {
     const size_t smem = sizeof(ReadoutSmem<D>);

@@ -93,6 +93,8 @@ struct BwdPlan {
   size_t lam_all = 0, dX_all = 0;                      // fp32 [2][B, H, F, d, d]: adjoint and dX per step
   size_t Xbuf = 0;                                     // fp32 [2][B, H, F, d, d] (sana_scaled only)
   size_t rms_part = 0;                                 // fp32 [B, H, F][d]
+  size_t dW_slots = 0, rms_slots = 0;                  // tensor-core read-out reversal's partial slots:
+                                                       // fp32 [B H F + kBwdReadoutGrid][d, d] and [..][d]
   size_t dkc = 0, dvc = 0;                             // [B, N, H, d] in the inputs' element type
   size_t tap_part = 0;                                 // fp32 [H][kBwdConvBlocks][2][d][3]
   size_t fwd_bytes = 0, total = 0;
@@ -123,8 +125,12 @@ struct BwdState {
 // the forward recompute)
 constexpr int kBwdKernels = 6;
 // tensor-core versions of the read-out and statistics reversals (bf16, d = 128; tc_backward.cu)
+// the read-out reversal runs two CTAs per SM over the (frame, tile) units; each (CTA, frame)
+// pair it touches leaves partial dW_t and RMS-weight sums in slot (CTA + frame), which the launch
+// then adds per frame into dW and rms_part (slots: B H F + kBwdReadoutGrid, of d^2 and d floats)
+constexpr int kBwdReadoutGrid = 296;
 cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
-                                  void* dq, void* dgate, uint32_t* status);
+                                  float* dW_slots, float* rms_slots, void* dq, void* dgate, uint32_t* status);
 cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const float* dB2, void* dkc, void* dvc,
                                 float* dbeta, uint32_t* status);
 cudaError_t launch_bwd_scan_tc(const Args& a, const uint16_t* nimg, const float* dPin, const float* dQin,

@@ -111,18 +111,23 @@ struct ReadoutTcSmem {
 // ---------------------------------------------------------------- Step 5 reversed
 // Two threads per token row: the warps w and w + 4 share TMEM lanes 32 (w % 4) .. and take the
 // column halves 64 hf .. 64 hf + 63 (hf = w / 4); per-token sums are combined in shared memory.
+// Persistent: CTA i takes the contiguous range [i T / G, (i + 1) T / G) of the (frame, tile)
+// units, T = B H F x tiles per frame, so no wave is left partly empty.  Where its range enters a
+// frame it builds that frame's W_t image; where it leaves one (or ends) it writes the partial
+// dW_t accumulated in TMEM and its RMS-weight partial sums to slot (i + frame) -- distinct for
+// every (CTA, frame) pair, as in the forward statistics -- and k_bwd_sum_slots adds each frame's
+// slots in a fixed order.
+__device__ __forceinline__ long long bwd_unit_owner(long long x, long long T, long long G) {
+  return ((x + 1) * G + T - 1) / T - 1;   // the largest i with i T / G <= x
+}
+
 __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gate,
     const __nv_bfloat16* __restrict__ dout, const float* __restrict__ rms_w, const float* __restrict__ Wall,
-    float* __restrict__ dWall, float* __restrict__ rms_part, __nv_bfloat16* __restrict__ dq,
-    __nv_bfloat16* __restrict__ dgate, int H, int F, int S, uint32_t* __restrict__ status) {
+    float* __restrict__ dWslot, float* __restrict__ rms_slot, __nv_bfloat16* __restrict__ dq,
+    __nv_bfloat16* __restrict__ dgate, int H, int F, int S, long long NFt, uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   ReadoutTcSmem& sm = tc::smem_align<ReadoutTcSmem>(smem_raw);
-  const long long fi = blockIdx.x;
-  const int f = (int)(fi % F);
-  const long long bh = fi / F;
-  const int h = (int)(bh % H);
-  const long long b = bh / H;
   const long long N = (long long)F * S;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, hf = warp >> 2;
@@ -138,18 +143,6 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     tc::tmem_relinquish();
   }
   for (int e = tid; e < 8 * 128; e += kReadoutThreads) (&sm.rms[0][0])[e] = 0.f;
-  // W_t image: thread (m, hf) writes the 8 chunks of its half of row m
-  {
-    const float* wr = Wall + fi * 16384 + m * 128;
-#pragma unroll 4
-    for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
-      const float4 a = *reinterpret_cast<const float4*>(wr + 8 * c);
-      const float4 bq = *reinterpret_cast<const float4*>(wr + 8 * c + 4);
-      const float v[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-      store_chunk_bf16(sm.w, m, 8 * c, v);
-    }
-  }
-  tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -160,11 +153,40 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     tc::tmem_ld32(tmem + 32 * p + lane_off, r);
     tc::tmem_ld_wait();
   };
+  const int ntile = (S + kBT - 1) / kBT;
+  const long long T = NFt * ntile, G = gridDim.x;
+  const long long u0 = (long long)blockIdx.x * T / G, u1 = ((long long)blockIdx.x + 1) * T / G;
   float racc[2] = {0.f, 0.f};
   uint32_t ph = 0;
   bool ok = true;
   int tile = 0;
-  for (int s0 = 0; s0 < S && ok; s0 += kBT, ++tile) {
+  long long cur = -1;
+  for (long long u = u0; u < u1 && ok; ++u, ++tile) {
+    const long long fi = u / ntile;
+    const int s0 = (int)(u - fi * ntile) * kBT;
+    const int f = (int)(fi % F);
+    const long long bh = fi / F;
+    const int h = (int)(bh % H);
+    const long long b = bh / H;
+    if (fi != cur) {
+      // W_t image of the frame: thread (m, hf) writes the 8 chunks of its half of row m
+      const float* wr = Wall + fi * 16384 + m * 128;
+#pragma unroll 4
+      for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
+        const float4 a = *reinterpret_cast<const float4*>(wr + 8 * c);
+        const float4 bq = *reinterpret_cast<const float4*>(wr + 8 * c + 4);
+        const float v[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+        store_chunk_bf16(sm.w, m, 8 * c, v);
+      }
+      racc[0] = racc[1] = 0.f;
+      tile = 0;
+      cur = fi;
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      tc::tc_fence_after();
+    }
+    {
     const int s = s0 + m;
     const bool valid = s < S;
     const long long row = ((b * N + (long long)f * S + (valid ? s : 0)) * H + h) * 128;
@@ -318,34 +340,65 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-  }
-  if (ok) {
-    float* dW = dWall + fi * 16384 + m * 128;   // row i = m, this thread's column half
+    }
+    if (u + 1 == u1 || (u + 1) % ntile == 0) {
+      // the range leaves the frame: its partial dW_t (row i = m, this thread's column half) and
+      // RMS-weight sums to slot (blockIdx.x + frame)
+      const long long slot = (long long)blockIdx.x + fi;
+      float* dW = dWslot + slot * 16384 + m * 128;
 #pragma unroll
-    for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
-      uint32_t r[32];
-      tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, r);
-      tc::tmem_ld_wait();
+      for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
+        uint32_t r[32];
+        tc::tmem_ld32(tmem + 128 + 32 * p + lane_off, r);
+        tc::tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dW + 32 * p + e) =
-            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                        __uint_as_float(r[e + 3]));
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dW + 32 * p + e) =
+              make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                          __uint_as_float(r[e + 3]));
+      }
+      sm.rms[warp][32 * (2 * hf) + lane] = racc[0];
+      sm.rms[warp][32 * (2 * hf + 1) + lane] = racc[1];
+      tc::tc_fence_before();
+      __syncthreads();
+      if (tid < 128) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc += sm.rms[w][tid];
+        rms_slot[slot * 128 + tid] = acc;
+      }
+      __syncthreads();
+      tc::tc_fence_after();
     }
   }
-  sm.rms[warp][32 * (2 * hf) + lane] = racc[0];
-  sm.rms[warp][32 * (2 * hf + 1) + lane] = racc[1];
   tc::tc_fence_before();
   __syncthreads();
-  if (tid < 128) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) acc += sm.rms[w][tid];
-    rms_part[fi * 128 + tid] = acc;
-  }
   if (warp == 0) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// Each frame's dW_t and RMS-weight partial sums: the slots (i + frame) of the read-out reversal's
+// CTAs i whose ranges covered the frame, added in CTA order.  Block (frame, part): 256 threads,
+// one float4 of dW_t each per part of 1024 floats; part 0 also sums the 128 RMS-weight entries.
+__global__ void __launch_bounds__(256) k_bwd_sum_slots(const float* __restrict__ dWslot,
+                                                       const float* __restrict__ rms_slot, int ntile, long long T,
+                                                       long long G, float* __restrict__ dW,
+                                                       float* __restrict__ rms_part) {
+  const long long fi = blockIdx.x;
+  const long long c0 = bwd_unit_owner(fi * ntile, T, G), c1 = bwd_unit_owner(fi * ntile + ntile - 1, T, G);
+  const int e4 = blockIdx.y * 256 + threadIdx.x;   // float4 index within the frame's 4096
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long c = c0; c <= c1; ++c) {
+    const float4 v = reinterpret_cast<const float4*>(dWslot + (c + fi) * 16384)[e4];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  reinterpret_cast<float4*>(dW + fi * 16384)[e4] = acc;
+  if (blockIdx.y == 0 && threadIdx.x < 128) {
+    float r = 0.f;
+    for (long long c = c0; c <= c1; ++c) r += rms_slot[(c + fi) * 128 + threadIdx.x];
+    rms_part[fi * 128 + threadIdx.x] = r;
   }
 }
 
@@ -795,14 +848,19 @@ __global__ void __launch_bounds__(kBwdScanThreads, 1) k_bwd_scan_tc(const uint16
 }  // namespace
 
 cudaError_t launch_bwd_readout_tc(const Args& a, const void* dout, const float* W, float* dW, float* rms_part,
-                                  void* dq, void* dgate, uint32_t* status) {
+                                  float* dW_slots, float* rms_slots, void* dq, void* dgate, uint32_t* status) {
   const size_t smem = sizeof(ReadoutTcSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_bwd_readout_tc<<<(unsigned)a.NF(), kReadoutThreads, smem, a.stream>>>(
+  const int ntile = (a.sh.S + kBT - 1) / kBT;
+  const long long T = a.NF() * ntile;
+  const long long G = T < kBwdReadoutGrid ? T : kBwdReadoutGrid;
+  k_bwd_readout_tc<<<(unsigned)G, kReadoutThreads, smem, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gate),
-      static_cast<const __nv_bfloat16*>(dout), a.rms_w, W, dW, rms_part, static_cast<__nv_bfloat16*>(dq),
-      static_cast<__nv_bfloat16*>(dgate), a.sh.H, a.sh.F, a.sh.S, status);
+      static_cast<const __nv_bfloat16*>(dout), a.rms_w, W, dW_slots, rms_slots, static_cast<__nv_bfloat16*>(dq),
+      static_cast<__nv_bfloat16*>(dgate), a.sh.H, a.sh.F, a.sh.S, a.NF(), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_bwd_sum_slots<<<dim3((unsigned)a.NF(), 16), 256, 0, a.stream>>>(dW_slots, rms_slots, ntile, T, G, dW, rms_part);
   return cudaGetLastError();
 }
 
