@@ -732,6 +732,110 @@ __global__ void __launch_bounds__(kBT, 2) k_bwd_conv(const T* __restrict__ k, co
   }
 }
 
+// bf16, d = 128: thread = (tensor, 8 channels, run of 32 tokens of one frame).  The 16 threads
+// of a channel row read it as one 256-byte line, and each thread slides a window of rows along its
+// run (rows loaded four tokens ahead, each row of x and of the conv-output gradient read once), so
+// the kernel streams k, v, dkc, dvc once and writes dk, dv once.  Same sums as k_bwd_conv:
+// dx[s] = sum_j w[j] g[s - j + p], taps sum_s g[s] x[s + j - p], rows outside the frame zero.
+constexpr int kConvRun = 32;
+__device__ __forceinline__ void unpack_row8(uint4 u, float (&x)[8]) {
+  x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+  x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+}
+template <int KT>
+__global__ void __launch_bounds__(512, 1) k_bwd_conv128(const __nv_bfloat16* __restrict__ k,
+                                                        const __nv_bfloat16* __restrict__ v,
+                                                        const float* __restrict__ wk, const float* __restrict__ wv,
+                                                        const __nv_bfloat16* __restrict__ dkc,
+                                                        const __nv_bfloat16* __restrict__ dvc,
+                                                        __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                                                        float* __restrict__ tap_part, int B, int H, int F, int S) {
+  constexpr int PAD = (KT - 1) / 2;
+  __shared__ float red[8][2][16][KT][8];     // [warp of the tensor][tensor][channel group][tap][channel]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int ten = tid >> 8;                  // 0: k, 1: v
+  const int g = tid & 15;                    // channels 8 g .. 8 g + 7
+  const int sl = (tid >> 4) & 15;            // run slot of the block
+  const int h = blockIdx.y;
+  const __nv_bfloat16* x = ten ? v : k;
+  const __nv_bfloat16* gx = ten ? dvc : dkc;
+  __nv_bfloat16* out = ten ? dv : dk;
+  const float* wg = ten ? wv : wk;
+  float w[KT][8], tp[KT][8];
+#pragma unroll
+  for (int j = 0; j < KT; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      w[j][e] = wg ? wg[((long long)h * 128 + 8 * g + e) * KT + j] : (j == PAD ? 1.f : 0.f);
+      tp[j][e] = 0.f;
+    }
+  const int nrun = (S + kConvRun - 1) / kConvRun;
+  const long long runs = (long long)B * F * nrun;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (long long r = (long long)blockIdx.x * 16 + sl; r < runs; r += (long long)gridDim.x * 16) {
+    const long long fb = r / nrun;                         // b F + f
+    const int s0 = (int)(r - fb * nrun) * kConvRun, s1 = min(S, s0 + kConvRun);
+    auto at = [&](int s) { return ((fb * S + s) * H + h) * 128 + 8 * g; };
+    auto ld = [&](const __nv_bfloat16* p, int s) {
+      return (s >= 0 && s < S) ? __ldg(reinterpret_cast<const uint4*>(p + at(s))) : z;
+    };
+    uint4 gw[6], xw[6];                                    // rows s - 1 .. s + 4 of the batch at s
+    gw[0] = ld(gx, s0 - 1); xw[0] = ld(x, s0 - 1);
+    gw[1] = ld(gx, s0);     xw[1] = ld(x, s0);
+    for (int s = s0; s < s1; s += 4) {
+#pragma unroll
+      for (int i = 2; i < 6; ++i) {
+        gw[i] = ld(gx, s - 1 + i);
+        xw[i] = KT > 1 ? ld(x, s - 1 + i) : z;
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (s + t >= s1) break;
+        float gm[8], gc[8], gp[8], xm[8], xc[8], xp[8];
+        unpack_row8(gw[t], gm); unpack_row8(gw[t + 1], gc); unpack_row8(gw[t + 2], gp);
+        unpack_row8(xw[t], xm); unpack_row8(xw[t + 1], xc); unpack_row8(xw[t + 2], xp);
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (KT == 3) {
+            o[e] = fmaf(w[0][e], gp[e], fmaf(w[1][e], gc[e], w[2][e] * gm[e]));
+            tp[0][e] = fmaf(gc[e], xm[e], tp[0][e]);
+            tp[1][e] = fmaf(gc[e], xc[e], tp[1][e]);
+            tp[2][e] = fmaf(gc[e], xp[e], tp[2][e]);
+          } else {
+            o[e] = w[0][e] * gc[e];
+            tp[0][e] = fmaf(gc[e], xc[e], tp[0][e]);
+          }
+        }
+        *reinterpret_cast<uint4*>(out + at(s + t)) =
+            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                       pack_bf16x2(o[6], o[7]));
+      }
+      gw[0] = gw[4]; xw[0] = xw[4];
+      gw[1] = gw[5]; xw[1] = xw[5];
+    }
+  }
+  // tap partials: the two run slots of a warp (lanes l and l + 16), then the tensor's 8 warps
+#pragma unroll
+  for (int j = 0; j < KT; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tp[j][e] += __shfl_xor_sync(0xffffffffu, tp[j][e], 16);
+  const int wt = (tid >> 5) & 7;
+  if (lane < 16)
+#pragma unroll
+    for (int j = 0; j < KT; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[wt][ten][g][j][e] = tp[j][e];
+  __syncthreads();
+  for (int idx = tid; idx < 2 * 16 * KT * 8; idx += 512) {
+    const int e = idx % 8, j = (idx / 8) % KT, g2 = (idx / (8 * KT)) % 16, m = idx / (8 * KT * 16);
+    float acc = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) acc += red[w2][m][g2][j][e];
+    tap_part[(((long long)h * gridDim.x + blockIdx.x) * 2 + m) * 128 * 3 + (8 * g2 + e) * 3 + j] = acc;
+  }
+}
+
 // ---------------------------------------------------------------- reductions
 template <int D>
 __global__ void __launch_bounds__(kBT) k_bwd_finish(const float* __restrict__ rms_part, long long nfr,
@@ -926,7 +1030,17 @@ static cudaError_t run_backward_t(const Args& a, const BwdGrads& g, const BwdSta
   }
   if ((e = mark()) != cudaSuccess) return e;
   // step 1 (conv) reversed
-  if (K == 3)
+  if (kTc && K == 3)
+    k_bwd_conv128<3><<<dim3(kBwdConvBlocks, sh.H), 512, 0, a.stream>>>(
+        static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.conv_k_w, a.conv_v_w,
+        reinterpret_cast<const __nv_bfloat16*>(at(p.dkc)), reinterpret_cast<const __nv_bfloat16*>(at(p.dvc)),
+        static_cast<__nv_bfloat16*>(g.dk), static_cast<__nv_bfloat16*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  else if (kTc)
+    k_bwd_conv128<1><<<dim3(kBwdConvBlocks, sh.H), 512, 0, a.stream>>>(
+        static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.conv_k_w, a.conv_v_w,
+        reinterpret_cast<const __nv_bfloat16*>(at(p.dkc)), reinterpret_cast<const __nv_bfloat16*>(at(p.dvc)),
+        static_cast<__nv_bfloat16*>(g.dk), static_cast<__nv_bfloat16*>(g.dv), at(p.tap_part), sh.B, sh.H, sh.F, sh.S);
+  else if (K == 3)
     k_bwd_conv<D, T, 3><<<dim3(kBwdConvBlocks, sh.H), kBT, 0, a.stream>>>(
         static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.conv_k_w, a.conv_v_w,
         reinterpret_cast<const T*>(at(p.dkc)), reinterpret_cast<const T*>(at(p.dvc)),
