@@ -27,6 +27,7 @@ namespace vdn {
 namespace {
 
 constexpr int kBT = 256;   // threads of every backward block
+constexpr int kBwdMaxWindow = 64;   // frames of a window whose alpha the gather reversal stages
 constexpr int kTok = 32;   // tokens per tile of the per-token kernels
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
@@ -305,6 +306,9 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
   constexpr int RG = kBT / CB;             // row groups
   constexpr int RPT = D / RG;              // rows per thread
   __shared__ float red[2][RG][CB];
+  // alpha of the current window's frames (a chunk's frames share the window), and the suffix
+  // products used for "the product of the other factors"
+  __shared__ float aw[kBwdMaxWindow][CB], rt[kBwdMaxWindow][CB];
   const long long bh = blockIdx.x;
   const int h = (int)(bh % H);
   const long long b = bh / H;
@@ -315,12 +319,25 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
   float* dQ = dQin + bh * (F + 1) * DD;
   float* dal = dalpha_g + bh * F * D;
   auto alpha_at = [&](int f) { return alpha[((b * F + f) * H + h) * D + j]; };
+  int wlo = -1, whi = -1;
   for (int t = 0; t < F; ++t) {
     int lo, hi;
     window_bounds(t, F, chunk, radius, lo, hi);
+    const bool staged = hi - lo + 1 <= kBwdMaxWindow;   // uniform over the block
+    if (staged && (lo != wlo || hi != whi)) {   // stage the window's alpha (all loads issued together)
+      __syncthreads();
+      for (int e = threadIdx.x; e < (hi - lo + 1) * CB; e += kBT) {
+        const int f = lo + e / CB, c = e % CB;
+        aw[f - lo][c] = alpha[((b * F + f) * H + h) * D + blockIdx.y * CB + c];
+      }
+      wlo = lo;
+      whi = hi;
+      __syncthreads();
+    }
+    auto al = [&](int f) { return staged ? aw[f - lo][jj] : alpha_at(f); };
     float a = 1.f, bb = 1.f;
-    for (int f = lo; f <= t; ++f) a *= alpha_at(f);
-    for (int f = t; f <= hi; ++f) bb *= alpha_at(f);
+    for (int f = lo; f <= t; ++f) a *= al(f);
+    for (int f = t; f <= hi; ++f) bb *= al(f);
     const float* dW = dWall + (bh * F + t) * DD;
     const float* pre = lo == 0 ? nullptr : P + (bh * F + lo - 1) * DD;
     const float* suf = hi == F - 1 ? nullptr : Q + (bh * F + hi + 1) * DD;
@@ -347,18 +364,43 @@ __global__ void __launch_bounds__(kBT) k_bwd_gather(const float* __restrict__ P,
         da += red[0][r][jj];
         db += red[1][r][jj];
       }
-      // d prod / d alpha_f = product of the other factors
-      for (int f = lo; f <= t; ++f) {
-        float pr = 1.f;
-        for (int g2 = lo; g2 <= t; ++g2)
-          if (g2 != f) pr *= alpha_at(g2);
-        dal[f * D + j] += da * pr;
+      // d prod / d alpha_f = product of the other factors = (left of f) x (right of f); a window
+      // wider than the staging buffer takes the products factor by factor
+      if (!staged) {
+        for (int f = lo; f <= t; ++f) {
+          float pr = 1.f;
+          for (int g2 = lo; g2 <= t; ++g2)
+            if (g2 != f) pr *= alpha_at(g2);
+          dal[f * D + j] += da * pr;
+        }
+        for (int f = t; f <= hi; ++f) {
+          float pr = 1.f;
+          for (int g2 = t; g2 <= hi; ++g2)
+            if (g2 != f) pr *= alpha_at(g2);
+          dal[f * D + j] += db * pr;
+        }
       }
-      for (int f = t; f <= hi; ++f) {
-        float pr = 1.f;
-        for (int g2 = t; g2 <= hi; ++g2)
-          if (g2 != f) pr *= alpha_at(g2);
-        dal[f * D + j] += db * pr;
+      if (staged) {
+        float right = 1.f;
+        for (int f = t; f >= lo; --f) {
+          rt[f - lo][jj] = right;
+          right *= aw[f - lo][jj];
+        }
+        float left = 1.f;
+        for (int f = lo; f <= t; ++f) {
+          dal[f * D + j] += da * (left * rt[f - lo][jj]);
+          left *= aw[f - lo][jj];
+        }
+        right = 1.f;
+        for (int f = hi; f >= t; --f) {
+          rt[f - lo][jj] = right;
+          right *= aw[f - lo][jj];
+        }
+        left = 1.f;
+        for (int f = t; f <= hi; ++f) {
+          dal[f * D + j] += db * (left * rt[f - lo][jj]);
+          left *= aw[f - lo][jj];
+        }
       }
     }
     __syncthreads();
