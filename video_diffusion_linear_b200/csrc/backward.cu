@@ -102,13 +102,27 @@ __device__ void cta_mm(float* __restrict__ C, const float* __restrict__ A, bool 
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int s = 0; s < R; ++s) acc[r][s] = 0.f;
+  // the next 16-wide slab is read into registers while this one is multiplied
+  constexpr int NL = 16 * D / kBT;   // elements of each operand per thread and slab
+  float na[NL], nb[NL];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < NL; ++u) {
+      const int e = tid + u * kBT, kk = e / D, i = e % D, k = k0 + kk;
+      na[u] = tA ? A[k * D + i] : A[i * D + k];
+      nb[u] = tB ? Bm[i * D + k] : Bm[k * D + i];
+    }
+  };
+  fetch(0);
   for (int k0 = 0; k0 < D; k0 += 16) {
-    for (int e = tid; e < 16 * D; e += kBT) {
-      const int kk = e / D, i = e % D, k = k0 + kk;
-      As[kk * (D + 1) + i] = tA ? A[k * D + i] : A[i * D + k];
-      Bs[kk * (D + 1) + i] = tB ? Bm[i * D + k] : Bm[k * D + i];
+#pragma unroll
+    for (int u = 0; u < NL; ++u) {
+      const int e = tid + u * kBT, kk = e / D, i = e % D;
+      As[kk * (D + 1) + i] = na[u];
+      Bs[kk * (D + 1) + i] = nb[u];
     }
     __syncthreads();
+    if (k0 + 16 < D) fetch(k0 + 16);
 #pragma unroll 4
     for (int kk = 0; kk < 16; ++kk) {
       float a[R], b[R];
