@@ -125,18 +125,19 @@ def backward_flops(w: synth.Workload) -> dict:
 
 
 def backward_bytes(w: synth.Workload) -> dict:
-    """Bytes each token-parallel backward kernel must move at least once (bf16 tokens, fp32
-    per-frame matrices and conv-output gradients):
-      readout_bwd: q, gate, dout in, dq, dgate out (5 x 2d B per token-head) + W_t in, dW_t out;
-      stats_bwd:   k, v, beta in, dk', dv' (fp32) and d beta out + dA, dB of both scans in;
-      conv_bwd:    dk', dv' (fp32), k, v in, dk, dv out."""
+    """Bytes each token-parallel backward kernel must move at least once (tokens and the
+    conv-output gradients dk', dv' in the workload's element type, fp32 per-frame matrices):
+      readout_bwd: q, gate, dout in, dq, dgate out (5 x d elements per token-head) + W_t in, dW_t out;
+      stats_bwd:   k, v, beta in, dk', dv' and d beta out + dA, dB of both scans in;
+      conv_bwd:    dk', dv', k, v in, dk, dv out."""
     d = w.d
+    el = 2 if w.dtype == "bf16" else 4
     TH = w.B * w.F * w.S * w.H
     NF = w.B * w.H * w.F
     mat = d * d * 4
-    return {"readout_bwd": 5 * 2 * d * TH + 2 * mat * NF,
-            "stats_bwd": (2 * 2 * d + 4 + 2 * 4 * d + 4) * TH + 4 * mat * NF,
-            "conv_bwd": (2 * 4 * d + 2 * 2 * d + 2 * 2 * d) * TH}
+    return {"readout_bwd": 5 * el * d * TH + 2 * mat * NF,
+            "stats_bwd": (2 * el * d + 4 + 2 * el * d + 4) * TH + 4 * mat * NF,
+            "conv_bwd": 6 * el * d * TH}
 
 
 def fp32_peak_tflops(sm_mhz: float) -> float:
