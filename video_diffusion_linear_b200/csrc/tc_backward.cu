@@ -82,6 +82,10 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* v) {
     v[2 * e + 1] = bf16hi(w[e]);
   }
 }
+__device__ __forceinline__ void unpack_bf16x8(uint4 u, float* v) {
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
 __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) =
       make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
@@ -121,7 +125,7 @@ __device__ __forceinline__ long long bwd_unit_owner(long long x, long long T, lo
   return ((x + 1) * G + T - 1) / T - 1;   // the largest i with i T / G <= x
 }
 
-__global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
+__global__ void __launch_bounds__(kReadoutThreads, 2) k_bwd_readout_tc(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gate,
     const __nv_bfloat16* __restrict__ dout, const float* __restrict__ rms_w, const float* __restrict__ Wall,
     float* __restrict__ dWslot, float* __restrict__ rms_slot, __nv_bfloat16* __restrict__ dq,
@@ -192,18 +196,22 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     const long long row = ((b * N + (long long)f * S + (valid ? s : 0)) * H + h) * 128;
     // x = silu(q) into the Q' tile (q' = x / |x|: the 1/|x| is folded into O, DO and dQ' below)
     float ss = 0.f;
-#pragma unroll 4
-    for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (valid) {
-        load8_bf16(q + row + 8 * c, v);
+    {
+      uint4 qu[8];   // this thread's 64 channels, all loads issued before any use
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        qu[c] = valid ? __ldg(reinterpret_cast<const uint4*>(q + row + 8 * (8 * hf + c))) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float v[8];
+        unpack_bf16x8(qu[c], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          v[e] = silu_f(v[e]);
+          v[e] = valid ? silu_f(v[e]) : 0.f;
           ss = fmaf(v[e], v[e], ss);
         }
+        store_chunk_bf16(sm.qf, m, 8 * (8 * hf + c), v);
       }
-      store_chunk_bf16(sm.qf, m, 8 * c, v);
     }
     sm.red[0][hf][m] = ss;
     tc::fence_proxy_async_smem();
@@ -235,17 +243,22 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
 #pragma unroll 1
     for (int pp = 0; pp < 2; ++pp) {
       const int p = 2 * hf + pp;
+      uint4 gou[4], gau[4];   // dout, gate of this half of the row, issued before the TMEM load
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int c0 = 32 * p + 8 * c8;
+        gou[c8] = valid ? __ldg(reinterpret_cast<const uint4*>(dout + row + c0)) : make_uint4(0, 0, 0, 0);
+        gau[c8] = valid ? __ldg(reinterpret_cast<const uint4*>(gate + row + c0)) : make_uint4(0, 0, 0, 0);
+      }
       uint32_t o[32];
       ld_row(p, o);
       float red[32];
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         const int c0 = 32 * p + 8 * c8;
-        float go[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, g[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (valid) {
-          load8_bf16(dout + row + c0, go);
-          load8_bf16(gate + row + c0, g);
-        }
+        float go[8], g[8], dyv[8];
+        unpack_bf16x8(gou[c8], go);
+        unpack_bf16x8(gau[c8], g);
         float dg[8], rw8[8];
         *reinterpret_cast<float4*>(rw8) = __ldg(reinterpret_cast<const float4*>(rms_w + c0));
         *reinterpret_cast<float4*>(rw8 + 4) = __ldg(reinterpret_cast<const float4*>(rms_w + c0 + 4));
@@ -254,11 +267,13 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
           const float ov = inv * __uint_as_float(o[8 * c8 + e]);
           const float oh = ov * rr;
           const float dy = go[e] * g[e];
+          dyv[e] = dy;
           dg[e] = go[e] * oh * rw8[e];
           red[8 * c8 + e] = dy * oh;
           so = fmaf(dy * rw8[e], ov, so);
         }
         if (valid) store8_bf16(dgate + row + c0, dg);
+        store_chunk_bf16(sm.dov, m, c0, dyv);   // dy for the next pass, where DO then overwrites it
       }
       racc[pp] += transpose_sum32(red, lane);
     }
@@ -274,15 +289,14 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
         const int c0 = 32 * p + 8 * c8;
         float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (valid) {
-          float go[8], g[8], rw8[8];
-          load8_bf16(dout + row + c0, go);
-          load8_bf16(gate + row + c0, g);
+          float dy[8], rw8[8];
+          load8_bf16(reinterpret_cast<const __nv_bfloat16*>(sm.dov + img_offset(0, m, c0)), dy);
           *reinterpret_cast<float4*>(rw8) = __ldg(reinterpret_cast<const float4*>(rms_w + c0));
           *reinterpret_cast<float4*>(rw8 + 4) = __ldg(reinterpret_cast<const float4*>(rms_w + c0 + 4));
           // the tile holds do / |x| (so that DO^T X sums do q'^T)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            v[e] = inv * (rr * go[e] * g[e] * rw8[e] - k3 * inv * __uint_as_float(o[8 * c8 + e]));
+            v[e] = inv * (rr * dy[e] * rw8[e] - k3 * inv * __uint_as_float(o[8 * c8 + e]));
         }
         store_chunk_bf16(sm.dov, m, c0, v);
       }
@@ -320,13 +334,17 @@ __global__ void __launch_bounds__(kReadoutThreads) k_bwd_readout_tc(
     xg = sm.red[3][0][m] + sm.red[3][1][m];
 #pragma unroll 1
     for (int p = 2 * hf; p < 2 * hf + 2; ++p) {
+      uint4 qu[4];   // issued before the TMEM load
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        qu[c8] = valid ? __ldg(reinterpret_cast<const uint4*>(q + row + 32 * p + 8 * c8)) : make_uint4(0, 0, 0, 0);
       uint32_t o[32];
       ld_row(p, o);
       if (!valid) continue;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float v[8], r8[8];
-        load8_bf16(q + row + 32 * p + 8 * c8, v);
+        unpack_bf16x8(qu[c8], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float sg = sigm_fast(v[e]);
