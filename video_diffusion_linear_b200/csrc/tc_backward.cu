@@ -439,16 +439,16 @@ struct StatsTcSmem {
 
 // the short conv of one channel chunk (8 channels c0..c0+7) of the tile's token t (frame index s),
 // in-frame taps, from the staged rows (row t + 1 holds token t) and the staged taps tp[tap][channel]
-__device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128], int K, int t, int s, int S,
-                                      int c0, float* out) {
+// (the staged rows are zero outside the frame, so every tap is applied: an outside row adds 0)
+template <int KT>
+__device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128], int t, int c0, float* out) {
+  constexpr int PAD = (KT - 1) / 2;
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = 0.f;
-  const int pad = (K - 1) / 2;
-  for (int j = 0; j < K; ++j) {
-    const int sj = s + j - pad;
-    if (sj < 0 || sj >= S) continue;
+#pragma unroll
+  for (int j = 0; j < KT; ++j) {
     float v[8];
-    load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1 + j - pad) * kRawStride + 2 * c0), v);
+    load8_bf16(reinterpret_cast<const __nv_bfloat16*>(raw + (t + 1 + j - PAD) * kRawStride + 2 * c0), v);
     const float4 w0 = *reinterpret_cast<const float4*>(&tp[j][c0]);
     const float4 w1 = *reinterpret_cast<const float4*>(&tp[j][c0 + 4]);
     const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -461,6 +461,7 @@ __device__ __forceinline__ void conv8(const uint8_t* raw, const float (*tp)[128]
 // column halves 64 hf .. 64 hf + 63 (hf = w / 4); per-token sums are combined in shared memory.
 constexpr int kStatsThreads = 256;
 
+template <int KT>   // taps of the staged convs (a missing conv: the identity, one centre tap)
 __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_constant__ CUtensorMap tmDK,
                                                                 const __grid_constant__ CUtensorMap tmDV,
                                                                 const __nv_bfloat16* __restrict__ k,
@@ -480,7 +481,6 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, hf = warp >> 2;
   const int m = 32 * quarter + lane;                       // token of the tile = TMEM lane
-  const int Kc = wk ? K : (wv ? K : 1);      // taps of the staged convs (a missing one: identity)
   volatile int* abort_flag = &sm.abort;
   if (tid == 0) {
     tc::mbar_init(&sm.bar, 1);
@@ -535,9 +535,9 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
       // taps of this head, [tensor][tap][channel]; a missing conv is the identity (one centre tap)
       if (tid < 128)
         for (int j = 0; j < 3; ++j) {
-          const bool centre = j == (Kc - 1) / 2;
-          sm.taps[0][j][i] = j < Kc ? (wk ? wk[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
-          sm.taps[1][j][i] = j < Kc ? (wv ? wv[((long long)h * 128 + i) * K + j] : (centre ? 1.f : 0.f)) : 0.f;
+          const bool centre = j == (KT - 1) / 2;
+          sm.taps[0][j][i] = j < KT ? (wk ? wk[((long long)h * 128 + i) * KT + j] : (centre ? 1.f : 0.f)) : 0.f;
+          sm.taps[1][j][i] = j < KT ? (wv ? wv[((long long)h * 128 + i) * KT + j] : (centre ? 1.f : 0.f)) : 0.f;
         }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
@@ -547,6 +547,8 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
     }
     const int s = s0 + m;
     const bool valid = s < S;
+    const long long tok = frame_row0 * H + (long long)(valid ? s : 0) * H + h;
+    const float bt = valid ? __ldg(beta + tok) : 0.f;   // issued here, used after the product
     // stage the raw k, v rows of tokens s0 - 1 .. s0 + 128 (zero outside the frame): sixteen
     // threads per row, so each warp reads two whole 256-byte rows; all loads issued first
     {
@@ -579,8 +581,8 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
     for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
       float kv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (valid) {
-        conv8(sm.kraw, sm.taps[0], Kc, m, s, S, 8 * c, kv);
-        conv8(sm.vraw, sm.taps[1], Kc, m, s, S, 8 * c, vv);
+        conv8<KT>(sm.kraw, sm.taps[0], m, 8 * c, kv);
+        conv8<KT>(sm.vraw, sm.taps[1], m, 8 * c, vv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           kv[e] = silu_f(kv[e]);
@@ -607,8 +609,6 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
     tc::tc_fence_after();
     const float inv = rsqrtf(sm.red[0][0][m] + sm.red[0][1][m] + kL2Eps);
     // the TMEM loads are warp-collective: every thread loads, only valid tokens compute
-    const long long tok = frame_row0 * H + (long long)(valid ? s : 0) * H + h;
-    const float bt = valid ? beta[tok] : 0.f;
     // pass 1: d beta and x . dk' over this thread's half, from the tiles' x and v' (bf16)
     float dbt = 0.f, xg = 0.f;
 #pragma unroll 1
@@ -654,8 +654,8 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
       for (int c8 = 0; c8 < 4; ++c8) {
         const int c0 = 32 * p + 8 * c8;
         float kc[8], vc[8], gk[8], gv[8];
-        conv8(sm.kraw, sm.taps[0], Kc, m, s, S, c0, kc);
-        conv8(sm.vraw, sm.taps[1], Kc, m, s, S, c0, vc);
+        conv8<KT>(sm.kraw, sm.taps[0], m, c0, kc);
+        conv8<KT>(sm.vraw, sm.taps[1], m, c0, vc);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int q8 = 8 * c8 + e;
@@ -890,11 +890,13 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
   if (!tmap_tokens_bf16(&tdk, dkc, a.sh.d, a.sh.H, a.sh.S, BF, kBT) ||
       !tmap_tokens_bf16(&tdv, dvc, a.sh.d, a.sh.H, a.sh.S, BF, kBT))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (K != 1 && K != 3) return cudaErrorInvalidValue;
+  auto kern = K == 3 ? k_bwd_stats_tc<3> : k_bwd_stats_tc<1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long units = a.NF() * ((a.sh.S + kBT - 1) / kBT);
   const unsigned grid = (unsigned)(units < kStatsGrid ? units : kStatsGrid);   // one CTA per SM
-  k_bwd_stats_tc<<<grid, kStatsThreads, smem, a.stream>>>(
+  kern<<<grid, kStatsThreads, smem, a.stream>>>(
       tdk, tdv, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
       a.conv_v_w, K, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
       a.sh.F, a.sh.S, a.NF(), status);
