@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kStatsThreads) k_bwd_stats_tc(const __grid_con
                                                                 const __nv_bfloat16* __restrict__ v,
                                                                 const float* __restrict__ beta,
                                                                 const float* __restrict__ wk,
-                                                                const float* __restrict__ wv, int K,
+                                                                const float* __restrict__ wv,
                                                                 const float* __restrict__ dA2,
                                                                 const float* __restrict__ dB2,
                                                                 __nv_bfloat16* __restrict__ dkc,
@@ -898,7 +898,7 @@ cudaError_t launch_bwd_stats_tc(const Args& a, int K, const float* dA2, const fl
   const unsigned grid = (unsigned)(units < kStatsGrid ? units : kStatsGrid);   // one CTA per SM
   kern<<<grid, kStatsThreads, smem, a.stream>>>(
       tdk, tdv, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v), a.beta, a.conv_k_w,
-      a.conv_v_w, K, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
+      a.conv_v_w, dA2, dB2, static_cast<__nv_bfloat16*>(dkc), static_cast<__nv_bfloat16*>(dvc), dbeta, a.sh.H,
       a.sh.F, a.sh.S, a.NF(), status);
   return cudaGetLastError();
 }

@@ -6,13 +6,17 @@
 //     X_f = S_{f-1} D_f + cpre B_f            (fp32, two threads per state row)
 //     S_f = X_f N_f + cpost B_f               (tcgen05, 128x128x128)
 // The product runs in bf16 with hi/lo splitting of both operands
-// (X = Xh + Xl, N = Nh + Nl; D = Xh Nh + Xh Nl + Xl Nh), which keeps about 16
+// (X = Xh + Xl, N = Nh + Nl; D = Xh Nl + Xh Nh + Xl Nh), which keeps about 16
 // significant bits in every term and accumulates in fp32 in TMEM, so the state
 // stays an fp32 quantity at tensor-core speed.  N_f arrives as a pre-swizzled
-// operand image (written by the per-frame solve) through one bulk copy, B_f
-// through TMA with a 128-byte swizzle so that each thread reads its own row
-// without bank conflicts.  Only the states the window gather needs are stored:
-// P at chunk ends, Q at chunk starts (or every frame for the debug export).
+// operand image (written by the per-frame solve) through bulk copies, its hi and
+// lo halves on barriers of their own: the Xh Nl terms run first, so the next
+// frame's N_lo can be requested a third of the way into the product (by a thread
+// other than the one issuing the MMAs, which stays blocked in the MMA queue).
+// B_f comes through TMA with a 128-byte swizzle so that each thread reads its own
+// row without bank conflicts.  Only the states the window gather needs are
+// stored: P at chunk ends, Q at chunk starts (or every frame for the debug
+// export), staged in the free X buffers and written by TMA store.
 //
 // Segment mode (frame sharding): the state restarts at every chunk, from zero
 // with the rule's own coefficients (the chunk's offset O_c) or from the identity
