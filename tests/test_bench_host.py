@@ -138,3 +138,13 @@ def test_rank_inputs_split_heads_or_clips():
     assert wr.seed != w.seed and job == 2 * w.tokens and split["scaling"] == "weak" and "dout" in host
     with pytest.raises(SystemExit):
         bench.rank_inputs("heads", w, 4, 0)
+
+
+@pytest.mark.parametrize("path", ["linear", "softmax", "backward"])
+def test_reference_arm_runs_on_rank_zero_only(path, capsys, monkeypatch):
+    # under torchrun every rank but 0 returns at once, printing nothing and running no oracle
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: pytest.fail("oracle ran on rank 1"))
+    bench.main(["--impl", "reference", "--path", path, "--workload", "tiny", "--steps", "2", "--warmup", "3"])
+    assert capsys.readouterr().out == ""

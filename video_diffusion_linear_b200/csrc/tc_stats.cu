@@ -54,7 +54,7 @@ constexpr int kMnAtomStride = kKAtoms * 1024;         // descriptor leading offs
 struct __align__(1024) StatsSmem {
   uint8_t raw[kRS][2][2][kRawHalf];    // [stage][k|v][channel half]
   uint8_t op[kOS][2 * kOpHalf];        // X | Y, MN-major SW128
-  float taps[kRS][2][3][128];          // [stage][k|v][tap][channel] conv taps / 2 of the stage's head
+  float taps[kRS][2][3][128];          // [stage][k|v][tap][channel, permuted as staged] conv taps / 2 of the stage's head
   float sqb[kRS][kBT];                 // [stage][token] sqrt(beta), 0 past the frame end
   uint64_t raw_full[kRS], raw_empty[kRS];
   uint64_t op_full[kOS], op_empty[kOS];
