@@ -282,7 +282,8 @@ size_t vdn_branch_backward_workspace_size(const vdn_shape* shape, int rule);
  * states leave the fp32 range (divergent sana_scaled settings) give non-finite
  * gradients.  Errors: as vdn_branch_forward, plus VDN_ERR_INVALID_ARG for a
  * missing or overlapping gradient buffer.  The device status word (first word
- * of the workspace) is that of the forward pass.
+ * of the workspace) records an expired bounded wait of the forward recompute or
+ * of a tensor-core backward kernel (vdn_workspace_status reads it).
  */
 vdn_status vdn_branch_backward(const vdn_shape* shape,
                                const void* q, const void* k, const void* v,
@@ -335,8 +336,9 @@ vdn_status vdn_branch_backward_saved(const vdn_shape* shape,
 
 /* vdn_branch_backward that also records caller-created CUDA events on `stream`:
  * events[0] before the forward recompute, events[1] after it, then events[2..7]
- * after each backward kernel (read-out, gather and bridge, adjoint scans, frame
- * statistics, conv, reductions).  n_events must be at least 8. */
+ * after each backward stage (read-out with its per-frame slot sums, gather and
+ * bridge, adjoint scans with their per-frame gradients, frame statistics, conv,
+ * reductions).  n_events must be at least 8. */
 vdn_status vdn_branch_backward_timed(const vdn_shape* shape,
                                      const void* q, const void* k, const void* v,
                                      const float* beta, const float* alpha,
