@@ -67,28 +67,4 @@ __device__ __forceinline__ void write_image128(const float* src, int ld, bool tr
   }
 }
 
-// Same, for src[n*ld + k] with ld a multiple of 4: each thread reads its eight
-// consecutive elements as two 16-byte loads (conflict-free).
-__device__ __forceinline__ void write_image128_rows(const float* src, int ld, uint16_t* img) {
-  uint4* dst = reinterpret_cast<uint4*>(img);
-  for (int idx = threadIdx.x; idx < 128 * 16; idx += blockDim.x) {
-    const int n = idx >> 4, c = idx & 15;
-    const float4 u = *reinterpret_cast<const float4*>(src + n * ld + 8 * c);
-    const float4 v = *reinterpret_cast<const float4*>(src + n * ld + 8 * c + 4);
-    const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-    uint32_t hw[4], lw[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      __nv_bfloat16 h0, l0, h1, l1;
-      split_bf16(x[e], h0, l0);
-      split_bf16(x[e + 1], h1, l1);
-      hw[e / 2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-      lw[e / 2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-    }
-    const uint32_t off = img_offset(0, n, 8 * c) >> 4;
-    dst[off] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    dst[off + 2048] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-  }
-}
-
 }  // namespace vdn
