@@ -1,0 +1,152 @@
+"""The arithmetic the tensor-core path uses in place of the plain definition, checked against it.
+
+The kernels do not evaluate the oracle's formulas literally in four places:
+  * scans: each state is kept as 2^e x an fp32 matrix.  After a step whose result has an entry
+    above 2^32 the matrix is multiplied by 2^-32 and e grows by 32; B_f enters the next steps
+    scaled by 2^-e (through the rule's coefficients); a stored state is the matrix before that
+    rescale, with its e;
+  * gather: the two bridged sides are added after aligning them to the larger exponent;
+  * read-out: the scaled row is normalised with the RMSNorm eps scaled by 2^-2e;
+  * scan products: X N runs as Xh Nl + Xh Nh + Xl Nh on bf16 hi/lo splits, accumulated in fp32.
+Each scheme is restated here in float64 and compared with the oracle ("Step 4" and "Step 5" of
+"VDN-Minimax-H3 bidirectional linear branch in five steps"): exactly where the scheme only moves
+powers of two, within the derived bound for the hi/lo products.  These check the schemes, not the
+kernels; the GPU parity tests check the kernels."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vdn_oracle as O
+
+RENORM_ABOVE = 2.0 ** 32
+RENORM_EXP = 32
+
+
+def _divergent_frames(F=31, S=1024, d=16, seed=7):
+    """Per-frame A, B from SiLU / L2 features with a large common component (as the workloads'
+    k' have), so sana_scaled at c = 1 grows the state by a factor of tens per frame."""
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((F * S, d))
+    v = rng.standard_normal((F * S, d))
+    _, kf, vf = O.prepare_features(k, k, v, F, S)
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((F, S))))
+    A, Bm = O.frame_statistics(kf, vf, beta)
+    alpha = 1.0 / (1.0 + np.exp(-(2.0 + rng.standard_normal((F, d)))))
+    seed_T = O.seed_state(0.5 * rng.normal(0.0, 0.1, (d, d)), d)
+    return A, Bm, alpha, seed_T
+
+
+def _aligned_frames(F=12, S=4096, d=16, seed=3):
+    """The worst case of the growth bound: every token of a frame carries the same unit key
+    with beta = 1, so A = S u u^T and |1 - c^2 lambda_max| = S - 1 at c = 1."""
+    rng = np.random.default_rng(seed)
+    A = np.empty((F, d, d))
+    Bm = np.empty((F, d, d))
+    for f in range(F):
+        u = rng.standard_normal(d)
+        u /= np.linalg.norm(u)
+        A[f] = S * np.outer(u, u)
+        w = rng.standard_normal(d)
+        Bm[f] = S * np.outer(w / np.linalg.norm(w), u)
+    alpha = np.ones((F, d))
+    return A, Bm, alpha, np.eye(d)
+
+
+def _scan_block_exponent(A, Bm, alpha, seed, rule, c, order):
+    """One scan direction with the kernels' block exponent: returns the stored matrices and
+    their exponents in frame order (state = 2^e x matrix)."""
+    s, e = seed.copy(), 0
+    mats, exps = np.empty_like(A), np.zeros(A.shape[0], dtype=np.int64)
+    for f in order:
+        s = O.rule_step(s, A[f], np.ldexp(Bm[f], -e), alpha[f], rule, c)
+        mats[f], exps[f] = s, e
+        if np.abs(s).max() > RENORM_ABOVE:
+            s = np.ldexp(s, -RENORM_EXP)
+            e += RENORM_EXP
+    return mats, exps
+
+
+@pytest.mark.parametrize("rule,c", [("sana_scaled", 1.0), ("sana_scaled", 0.5), ("vdn_scaled", 1.0),
+                                    ("vdn_solve", 1.0)])
+def test_block_exponent_scan_reproduces_the_states(rule, c):
+    A, Bm, alpha, seed = _divergent_frames()
+    F = A.shape[0]
+    P, Q = O.bidirectional_scan(A, Bm, alpha, seed, rule, c)
+    Pm, Pe = _scan_block_exponent(A, Bm, alpha, seed, rule, c, range(F))
+    Qm, Qe = _scan_block_exponent(A, Bm, alpha, seed, rule, c, reversed(range(F)))
+    for f in range(F):
+        assert np.array_equal(np.ldexp(Pm[f], Pe[f]), P[f])
+        assert np.array_equal(np.ldexp(Qm[f], Qe[f]), Q[f])
+    if rule == "sana_scaled" and c == 1.0:
+        assert np.abs(P[-1]).max() > 2.0 ** 128        # beyond fp32: the exponent is needed
+        assert Pe[-1] >= 128
+    if rule != "sana_scaled":
+        assert Pe.max() == 0 and Qe.max() == 0         # the exact-solve rules contract
+
+
+@pytest.mark.parametrize("make", [_divergent_frames, _aligned_frames])
+@pytest.mark.parametrize("c", [1.0, 0.5])
+def test_stored_states_stay_below_two_to_48(make, c):
+    # one step grows a row norm by at most 1 + c^2 S (|k'| = 1, beta <= 1, alpha <= 1), and a
+    # matrix whose entries are at most 2^32 has row norms at most 2^32 sqrt(d): the fp32 gather
+    # can add two aligned sides without overflow
+    A, Bm, alpha, seed = make()
+    F = A.shape[0]
+    for order in (range(F), reversed(range(F))):
+        mats, _ = _scan_block_exponent(A, Bm, alpha, seed, "sana_scaled", c, order)
+        assert np.abs(mats).max() < 2.0 ** 48
+    # the same bound at the kernels' sizes: d = 128, S up to 4096 tokens per frame
+    assert 2.0 ** 32 * np.sqrt(128) * (1 + c * c * 4096) < 2.0 ** 48
+
+
+@pytest.mark.parametrize("chunk,radius", [(5, 1), (3, 0), (4, 2)])
+def test_aligned_gather_and_scaled_eps_readout_reproduce_the_output(chunk, radius):
+    A, Bm, alpha, seed = _divergent_frames()
+    F, d = A.shape[0], A.shape[1]
+    rule, c = "sana_scaled", 1.0
+    P, Q = O.bidirectional_scan(A, Bm, alpha, seed, rule, c)
+    Pm, Pe = _scan_block_exponent(A, Bm, alpha, seed, rule, c, range(F))
+    Qm, Qe = _scan_block_exponent(A, Bm, alpha, seed, rule, c, reversed(range(F)))
+    rng = np.random.default_rng(11)
+    q = O.l2_normalize(O.silu(rng.standard_normal((8, d))))
+    gate = 1.0 / (1.0 + np.exp(-rng.standard_normal((8, d))))
+    rms_w = 1.0 + 0.1 * rng.standard_normal(d)
+    for t in range(F):
+        lo, hi = O.window_bounds(t, F, chunk, radius)
+        pre, ep = (seed, 0) if lo == 0 else (Pm[lo - 1], Pe[lo - 1])
+        suf, eq = (seed, 0) if hi == F - 1 else (Qm[hi + 1], Qe[hi + 1])
+        dpre = np.prod(alpha[lo:t + 1], axis=0)
+        dsuf = np.prod(alpha[t:hi + 1], axis=0)
+        em = max(ep, eq)
+        W_e = np.ldexp(pre * dpre[None, :], ep - em) + np.ldexp(suf * dsuf[None, :], eq - em)
+        W = O.gather_state(P, Q, seed, alpha, t, chunk, radius)
+        assert np.array_equal(np.ldexp(W_e, em), W)
+        o = q @ W_e.T
+        y = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + np.ldexp(O.RMS_EPS, -2 * em)) * rms_w
+        assert np.array_equal(y * gate, O.readout(W, q, gate, rms_w))
+
+
+def _bf16(x: np.ndarray) -> np.ndarray:
+    """Round to bf16 (nearest even) and back, exactly."""
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_hi_lo_product_keeps_sixteen_bits():
+    # X = Xh + Xl + dX, |Xl| <= 2^-8 |X|, |dX| <= 2^-16 |X| (same for N): the dropped terms
+    # Xl Nl, Xh dN, dX N are each at most about 2^-16 |X| |N|
+    rng = np.random.default_rng(5)
+    d = 128
+    X = (rng.standard_normal((d, d)) * np.exp2(rng.integers(-6, 7, (d, d)))).astype(np.float32).astype(np.float64)
+    K = O.l2_normalize(O.silu(rng.standard_normal((512, d))))
+    N = np.linalg.inv(np.eye(d) + (K.T * rng.uniform(0, 1, 512)) @ K).astype(np.float32).astype(np.float64)
+    Xh = _bf16(X)
+    Xl = _bf16((X.astype(np.float32) - Xh.astype(np.float32)).astype(np.float64))
+    Nh = _bf16(N)
+    Nl = _bf16((N.astype(np.float32) - Nh.astype(np.float32)).astype(np.float64))
+    got = Xh @ Nl + Xh @ Nh + Xl @ Nh
+    exact = X @ N
+    scale = np.abs(X) @ np.abs(N)
+    assert np.all(np.abs(got - exact) <= 3.1 * 2.0 ** -16 * scale)
+    # a single bf16 product misses that bound by far: the split is what buys the bits
+    plain = Xh @ Nh
+    assert np.max(np.abs(plain - exact) / scale) > 2.0 ** -12

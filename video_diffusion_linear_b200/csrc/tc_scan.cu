@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tc(const __grid_consta
     tc::tc_fence_after();
     if (tid == 32 && step + 1 < F) load_n_part(step + 1, 0);   // the product that read N_hi is complete
 
-    // S_f = D + cpost B_f
+    // S_f = X_f N_f (the TMEM accumulator) + cpost B_f
     const bool seg_store = kMode != kScanWhole && seg_last(f);
     const bool store = kMode == kScanWhole && (all_frames || (dir == 0 ? ((f + 1) % chunk == 0) : (f % chunk == 0)));
     // whole clip: the stored state goes out through the (now free) X buffers and a TMA
