@@ -150,3 +150,63 @@ def test_hi_lo_product_keeps_sixteen_bits():
     # a single bf16 product misses that bound by far: the split is what buys the bits
     plain = Xh @ Nh
     assert np.max(np.abs(plain - exact) / scale) > 2.0 ** -12
+
+
+def _sweep_every_pivot(M: np.ndarray, dtype=np.float64):
+    """The per-frame solve's elimination, without pivoting: for pivot k with d = M[k, k],
+    M[i, j] -= (M[i, k] / d) M[k, j] for every (i, j), then row and column k divided by d and
+    M[k, k] = -1 / d.  Sweeping every pivot of a symmetric positive definite M leaves -M^-1.
+    Returns that matrix and the pivots in elimination order."""
+    M = M.astype(dtype).copy()
+    piv = np.empty(M.shape[0])
+    for k in range(M.shape[0]):
+        d = M[k, k]
+        piv[k] = d
+        r = dtype(1) / d
+        col, row = M[:, k].copy(), M[k, :].copy()
+        M -= np.outer(col * r, row)
+        M[k, :] = row * r
+        M[:, k] = col * r
+        M[k, k] = -r
+    return M, piv
+
+
+def _frame_matrix(d, S, c, seed):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((S, d))
+    _, kf, _ = O.prepare_features(k, k, k, 1, S)
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((1, S))))
+    A, _ = O.frame_statistics(kf, kf, beta)
+    return np.eye(d) + c * c * A[0]
+
+
+@pytest.mark.parametrize("d,S,c", [(16, 1024, 1.0), (128, 1024, 1.0), (128, 4096, 0.5)])
+def test_sweep_without_pivoting_inverts_and_every_pivot_is_at_least_one(d, S, c):
+    # every pivot is a Schur complement of M = I + c^2 A; its inverse is a diagonal block of
+    # M^-1, which is at most I because M is at least I, so each pivot is at least 1: the
+    # elimination never divides by a small number and needs no row exchanges
+    M = _frame_matrix(d, S, c, seed=d + S)
+    neg_inv, piv = _sweep_every_pivot(M)
+    assert piv.min() >= 1.0 - 1e-12
+    np.testing.assert_allclose(-neg_inv, np.linalg.inv(M), rtol=0, atol=1e-13)
+    # the rule step with the swept inverse equals the oracle's solve
+    rng = np.random.default_rng(1)
+    S_in, Bf = rng.standard_normal((d, d)), rng.standard_normal((d, d))
+    alpha = rng.uniform(0.5, 1.0, d)
+    A = (M - np.eye(d)) / (c * c)
+    X = S_in @ np.diag(alpha) + c * Bf
+    np.testing.assert_allclose(X @ -neg_inv, O.rule_step(S_in, A, Bf, alpha, "vdn_scaled", c), rtol=0, atol=1e-12)
+
+
+def test_fp32_sweep_error_within_the_conditioning_bound():
+    # in fp32 the sweep's forward error stays within n u cond(M) of the inverse's largest
+    # entry (u = 2^-24): the solve's fp32 arithmetic is as accurate as the problem allows
+    d = 128
+    M = _frame_matrix(d, 4096, 1.0, seed=2)
+    neg_inv32, piv32 = _sweep_every_pivot(M.astype(np.float32), np.float32)
+    inv = np.linalg.inv(M)
+    cond = np.linalg.cond(M)
+    assert cond > 10                                   # lambda_max(A) ~ 250: one dominant key direction
+    err = np.abs(-neg_inv32.astype(np.float64) - inv).max()
+    assert err <= d * 2.0 ** -24 * cond * np.abs(inv).max()
+    assert piv32.min() >= 1.0 - 1e-4
