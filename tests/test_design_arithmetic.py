@@ -210,3 +210,35 @@ def test_fp32_sweep_error_within_the_conditioning_bound():
     err = np.abs(-neg_inv32.astype(np.float64) - inv).max()
     assert err <= d * 2.0 ** -24 * cond * np.abs(inv).max()
     assert piv32.min() >= 1.0 - 1e-4
+
+
+def test_fp16_row_block_image_of_w_keeps_eleven_bits():
+    # the gather scales W_t by the power of two that puts its largest entry in [0.5, 1), then
+    # writes each block of 32 rows in fp16 scaled again so that the block's largest entry is in
+    # [0.5, 1); the read-out undoes both exponents in its RMSNorm.  Each entry then carries fp16's
+    # 11 significant bits (2^-25 absolute below the block's normal range).
+    A, Bm, alpha, seed = _divergent_frames(d=128)
+    F, d = A.shape[0], A.shape[1]
+    P, Q = O.bidirectional_scan(A, Bm, alpha, seed, "sana_scaled", 1.0)
+    rng = np.random.default_rng(4)
+    q = O.l2_normalize(O.silu(rng.standard_normal((64, d))))
+    gate = 1.0 / (1.0 + np.exp(-rng.standard_normal((64, d))))
+    rms_w = 1.0 + 0.1 * rng.standard_normal(d)
+    worst = {"fp16": 0.0, "bf16": 0.0}
+    for t in range(F):
+        W = O.gather_state(P, Q, seed, alpha, t, 5, 1)
+        _, ew = np.frexp(np.abs(W).max())
+        Wn = np.ldexp(W, -int(ew))                                    # largest entry in [0.5, 1)
+        _, eb = np.frexp(np.abs(Wn).reshape(d // 32, -1).max(axis=1))
+        eb = np.repeat(np.clip(eb, -125, 126), 32)[:, None]
+        img = np.ldexp(Wn, -eb).astype(np.float16).astype(np.float64)
+        back = np.ldexp(img, eb)
+        bound = np.ldexp(np.maximum(2.0 ** -11 * np.abs(np.ldexp(Wn, -eb)), 2.0 ** -25), eb)
+        assert np.all(np.abs(back - Wn) <= bound)
+        ref = O.readout(W, q, gate, rms_w)
+        for name, img_w in (("fp16", back), ("bf16", np.ldexp(_bf16(np.ldexp(Wn, -eb)), eb))):
+            o = q @ img_w.T
+            y = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + np.ldexp(O.RMS_EPS, -2 * int(ew))) * rms_w
+            worst[name] = max(worst[name], np.abs(y * gate - ref).max() / np.abs(ref).max())
+    assert np.abs(P[-1]).max() > 2.0 ** 128
+    assert worst["fp16"] < 2e-3 and worst["bf16"] > 4 * worst["fp16"]   # the three extra bits show
