@@ -242,3 +242,48 @@ def test_fp16_row_block_image_of_w_keeps_eleven_bits():
             worst[name] = max(worst[name], np.abs(y * gate - ref).max() / np.abs(ref).max())
     assert np.abs(P[-1]).max() > 2.0 ** 128
     assert worst["fp16"] < 2e-3 and worst["bf16"] > 4 * worst["fp16"]   # the three extra bits show
+
+
+def _lazy_two_group_softmax(qr, kr, v, scale, tile=128, move_above=8.0):
+    """The windowed softmax kernel's schedule for one block of query rows: key tiles alternate
+    between two groups; each group keeps, per row, a reference maximum m (log2 units), a running
+    normaliser l and an accumulator O, and moves m to a tile's maximum only when that maximum
+    exceeds m by more than `move_above` (O and l then scaled by 2^(m_old - m_new)); exponents
+    are taken against m, so every weight is at most 2^move_above.  The groups are combined at
+    the end against their larger reference.  Returns the output and the largest weight used."""
+    n, L = qr.shape[0], kr.shape[0]
+    s2 = (qr @ kr.T) * scale * np.log2(np.e)                     # scores in log2 units
+    m = np.full((2, n), -np.inf)
+    l = np.zeros((2, n))
+    acc = np.zeros((2, n, v.shape[1]))
+    pmax = 0.0
+    for j, t0 in enumerate(range(0, L, tile)):
+        g, t1 = j % 2, min(L, t0 + tile)
+        tmax = s2[:, t0:t1].max(axis=1)
+        move = tmax > m[g] + move_above
+        corr = np.where(move, np.exp2(np.where(np.isinf(m[g]), -np.inf, m[g] - tmax)), 1.0)
+        l[g] *= corr
+        acc[g] *= corr[:, None]
+        m[g] = np.where(move, tmax, m[g])
+        p = np.exp2(s2[:, t0:t1] - m[g][:, None])
+        pmax = max(pmax, p.max())
+        l[g] += p.sum(axis=1)
+        acc[g] += p @ v[t0:t1]
+    top = m.max(axis=0)
+    w = np.where(np.isinf(m), 0.0, np.exp2(m - top))
+    return (acc[0] * w[0][:, None] + acc[1] * w[1][:, None]) / (l[0] * w[0] + l[1] * w[1])[:, None], pmax
+
+
+@pytest.mark.parametrize("L,rising", [(128, False), (200, False), (1000, True), (4 * 1560 + 37, True)])
+def test_lazy_reference_two_group_softmax_equals_softmax(L, rising):
+    rng = np.random.default_rng(L)
+    d = 32
+    qr = 2.0 * rng.standard_normal((16, d))
+    kr = rng.standard_normal((L, d))
+    if rising:                                       # key norms rising along the window: the
+        kr *= np.linspace(0.5, 6.0, L)[:, None]      # reference maximum moves again and again
+    v = rng.standard_normal((L, d))
+    scale = 1.0 / np.sqrt(d)
+    got, pmax = _lazy_two_group_softmax(qr, kr, v, scale)
+    np.testing.assert_allclose(got, O.window_softmax_frame(qr, kr, v, scale), rtol=0, atol=1e-12)
+    assert pmax <= 2.0 ** 8 * (1 + 1e-12)            # stored as bf16 without overflow, l < L 2^8
