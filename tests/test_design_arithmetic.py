@@ -287,3 +287,44 @@ def test_lazy_reference_two_group_softmax_equals_softmax(L, rising):
     got, pmax = _lazy_two_group_softmax(qr, kr, v, scale)
     np.testing.assert_allclose(got, O.window_softmax_frame(qr, kr, v, scale), rtol=0, atol=1e-12)
     assert pmax <= 2.0 ** 8 * (1 + 1e-12)            # stored as bf16 without overflow, l < L 2^8
+
+
+# The kernels run every rule as one generic step with coefficients (cpre, cpost, c2, solve,
+# identity):  S_out = (S_in D + cpre B) N + cpost B,  N = (I + c2 A)^-1 (solve), I - c2 A, or I.
+_RULE_COEF = {
+    "vdn_solve": lambda c: (1.0, 0.0, 1.0, True, False),
+    "vdn_scaled": lambda c: (c, 0.0, c * c, True, False),
+    "sana_scaled": lambda c: (0.0, c, c * c, False, False),
+    "additive": lambda c: (1.0, 0.0, 0.0, False, True),
+}
+
+
+def _generic_step_and_adjoint(S_in, A, B, alpha, rule, c, lam):
+    """The generic step and its adjoint as the backward kernels form them from the forward's
+    explicit N: dX = lam N^T, dS_in = dX D, dB = cpre dX + cpost lam, dalpha_j = sum_i S_in[i, j]
+    dX[i, j], and dA = -c2 S_out^T dX when N is an inverse (dN^-1 = -N^T dN N^T), -c2 X^T lam
+    when N = I - c2 A, 0 for the identity."""
+    cpre, cpost, c2, solve, identity = _RULE_COEF[rule](c)
+    d = A.shape[0]
+    N = np.eye(d) if identity else (np.linalg.inv(np.eye(d) + c2 * A) if solve else np.eye(d) - c2 * A)
+    X = S_in * alpha[None, :] + cpre * B
+    S_out = X @ N + cpost * B
+    dX = lam @ N.T
+    dA = np.zeros_like(A) if identity else (-c2 * S_out.T @ dX if solve else -c2 * X.T @ lam)
+    return S_out, (dX * alpha[None, :], dA, cpre * dX + cpost * lam, np.sum(S_in * dX, axis=0))
+
+
+@pytest.mark.parametrize("rule,c", [("vdn_solve", 1.0), ("vdn_scaled", 0.6), ("sana_scaled", 0.3),
+                                    ("additive", 1.0)])
+def test_generic_step_and_its_adjoint_match_the_oracles_rules(rule, c):
+    from oracle import vdn_backward as OB
+    A, Bm, alpha, _ = _divergent_frames(F=3, S=64, d=16)
+    rng = np.random.default_rng(9)
+    for f in range(A.shape[0]):
+        S_in = rng.standard_normal((16, 16))
+        lam = rng.standard_normal((16, 16))
+        S_out, grads = _generic_step_and_adjoint(S_in, A[f], Bm[f], alpha[f], rule, c, lam)
+        ref_out = O.rule_step(S_in, A[f], Bm[f], alpha[f], rule, c)
+        np.testing.assert_allclose(S_out, ref_out, rtol=0, atol=1e-12 * np.abs(ref_out).max())
+        for got, ref in zip(grads, OB.rule_step_grad(S_in, A[f], Bm[f], alpha[f], rule, c, lam)):
+            np.testing.assert_allclose(got, ref, rtol=0, atol=1e-11 * max(1.0, np.abs(ref).max()))
