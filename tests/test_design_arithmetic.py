@@ -328,3 +328,30 @@ def test_generic_step_and_its_adjoint_match_the_oracles_rules(rule, c):
         np.testing.assert_allclose(S_out, ref_out, rtol=0, atol=1e-12 * np.abs(ref_out).max())
         for got, ref in zip(grads, OB.rule_step_grad(S_in, A[f], Bm[f], alpha[f], rule, c, lam)):
             np.testing.assert_allclose(got, ref, rtol=0, atol=1e-11 * max(1.0, np.abs(ref).max()))
+
+
+def test_stream_k_owner_and_partial_slots():
+    # CTA i of G owns units [floor(i T / G), floor((i + 1) T / G)) of the T (frame, block) units,
+    # frames in unit order; the solve finds the CTAs covering a frame from the closed form
+    # owner(x) = ceil((x + 1) G / T) - 1 and reads slot (CTA + frame).  The closed form must be the
+    # CTA whose range holds x, and no two (CTA, frame) pairs may share a slot.
+    rng = np.random.default_rng(0)
+    cases = [(744, 42, 148), (31, 42, 148), (1, 1, 148), (3, 5, 148), (2976, 43, 148), (5, 1, 7)]
+    cases += [(int(rng.integers(1, 400)), int(rng.integers(1, 50)), int(rng.integers(1, 300))) for _ in range(40)]
+    for NF, nb, G0 in cases:
+        T = NF * nb
+        G = min(G0, T)
+        begin = [(i * T) // G for i in range(G + 1)]
+        owner_def = np.repeat(np.arange(G), np.diff(begin))           # the CTA holding each unit
+        x = np.arange(T)
+        owner = -((-(x + 1) * G) // T) - 1                           # ceil((x + 1) G / T) - 1
+        assert np.array_equal(owner, owner_def)
+        slots = {}
+        for i in range(G):
+            for pf in range(begin[i] // nb, (begin[i + 1] - 1) // nb + 1) if begin[i + 1] > begin[i] else ():
+                assert (i + pf) not in slots
+                slots[i + pf] = (i, pf)
+        assert max(slots) < NF + G
+        for pf in range(NF):                                          # the solve's CTA range per frame
+            i0, i1 = owner[pf * nb], owner[pf * nb + nb - 1]
+            assert {i for i, f in slots.values() if f == pf} == set(range(i0, i1 + 1))
