@@ -4,16 +4,20 @@
 // A1/A2, but prints no backward; this is the exact gradient of the forward).
 //
 // The forward runs first with its per-frame export (A_f, B_f, N_f, P_f, Q_f, W_t
-// in fp32); then, all in fp32 SIMT for d = 16 and 128:
+// in fp32); then, in fp32 SIMT kernels (fp32 inputs, d = 16 and 128; for bf16 at
+// d = 128 the read-out, statistics and scan reversals run on the tensor cores in
+// tc_backward.cu and the conv reversal in k_bwd_conv128):
 //   k_bwd_readout  (batch, head, frame): recompute q', o = W_t q', RMSNorm; write
 //                  dgate and dq; dW_t = sum_s do_s q'_s^T; RMS-weight partials
-//   k_bwd_gather   (batch, head): dW_t onto the boundary states P_{lo-1} and
+//   k_bwd_gather   (batch, column block): dW_t onto the boundary states P_{lo-1} and
 //                  Q_{hi+1} (or the seed at a clip edge), d alpha of the bridge
-//   k_bwd_scan     (batch, head, direction): the adjoint of each scan, frame by
-//                  frame in reverse order of absorption
+//   k_bwd_scan     (batch, head, direction): the adjoint recurrence of each scan,
+//                  frame by frame in reverse order of absorption, storing lam_f, dX_f
+//   k_bwd_scan_grads (batch, head, frame, direction): dA, dB, d alpha of each step
 //   k_bwd_stats    (batch, head, frame): dk', dv', d beta from dA_f, dB_f; L2-norm
 //                  and SiLU reversed into the gradients of the conv outputs
-//   k_bwd_conv     the short conv reversed (dk, dv, tap partials)
+//   k_bwd_conv     the short conv reversed (dk, dv, tap partials); k_bwd_conv128
+//                  the bf16, d = 128 form (8 channels x a run of 32 tokens per thread)
 //   k_bwd_finish   reductions over CTAs, heads and batch; d alpha summed
 #include <cuda_bf16.h>
 

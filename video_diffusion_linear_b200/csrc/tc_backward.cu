@@ -1,18 +1,28 @@
 // Tensor-core kernels of the backward pass (bf16 inputs, d = 128): the two
-// per-token contractions of the branch's gradients, each over one (batch, head,
-// frame) in tiles of 128 tokens, one token per thread (= its TMEM lane).
+// per-token contractions of the branch's gradients and the adjoint recurrence of
+// the scans.  The per-token kernels work in tiles of 128 tokens of one (batch,
+// head, frame), two threads per token (TMEM lane = token, one column half each),
+// and are persistent: each CTA walks a contiguous range of the (frame, tile) units.
 //
 //   k_bwd_readout_tc  (Step 5 reversed)  O = Q' W_t^T      (A = Q' K-major, B = W_t K-major)
 //                                        dQ' = DO W_t       (A = DO K-major, B = W_t read MN-major)
 //                                        dW_t += DO^T Q'    (A = DO MN-major, B = Q' MN-major)
+//                     296 CTAs (two per SM); the partial dW_t and RMS-weight sums of each
+//                     (CTA, frame) pair go to slot CTA + frame, added per frame in CTA order by
+//                     k_bwd_sum_slots
 //   k_bwd_stats_tc    (Step 2 reversed)  U = K' (dA + dA^T), Z = K' dB^T   (B images K-major)
 //                                        V' dB                          (dB image read MN-major)
+//                     148 CTAs; raw k, v rows (+ halo) staged in shared memory, the conv
+//                     unrolled over its taps; dk', dv' written in bf16 by TMA store
+//   k_bwd_scan_tc     (Step 4 scans reversed)  dX_f = lam_f N_f, one CTA per (batch, head,
+//                     direction), lam split into bf16 hi + lo against the forward's hi/lo N_f
 //
 // Operands are bf16 images in the 128-byte-swizzled layout of image.cuh written by
-// the threads (q', do, k', v' per tile; W_t, dA + dA^T, dB once per frame);
-// accumulators fp32 in TMEM.  The elementwise parts (RMSNorm and gate reversed,
-// L2 norm and SiLU reversed, the conv recomputed from the raw tokens) run in the
-// epilogues in fp32, as in the SIMT kernels of backward.cu.
+// the threads (q', do, k', v' per tile; W_t, dA + dA^T, dB where a CTA's range
+// enters a frame); accumulators fp32 in TMEM.  The elementwise parts (RMSNorm and
+// gate reversed, L2 norm and SiLU reversed, the conv recomputed from the raw
+// tokens) run in the epilogues in fp32, as in the SIMT kernels of backward.cu.
+// Every wait is bounded and reports through the device status word.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -24,7 +34,7 @@
 namespace vdn {
 namespace {
 
-constexpr int kBT = 128;                                                   // threads = tokens per tile
+constexpr int kBT = 128;                                                   // tokens per tile
 constexpr uint32_t kIdKK = tc::idesc_bf16_f32(128, 128, false, false);    // A, B K-major
 constexpr uint32_t kIdKM = tc::idesc_bf16_f32(128, 128, false, true);     // A K-major, B MN-major
 constexpr uint32_t kIdMM = tc::idesc_bf16_f32(128, 128, true, true);      // A, B MN-major
