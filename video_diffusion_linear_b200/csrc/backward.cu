@@ -9,7 +9,7 @@
 // tc_backward.cu and the conv reversal in k_bwd_conv128):
 //   k_bwd_readout  (batch, head, frame): recompute q', o = W_t q', RMSNorm; write
 //                  dgate and dq; dW_t = sum_s do_s q'_s^T; RMS-weight partials
-//   k_bwd_gather   (batch, column block): dW_t onto the boundary states P_{lo-1} and
+//   k_bwd_gather   (batch, head, column block): dW_t onto the boundary states P_{lo-1} and
 //                  Q_{hi+1} (or the seed at a clip edge), d alpha of the bridge
 //   k_bwd_scan     (batch, head, direction): the adjoint recurrence of each scan,
 //                  frame by frame in reverse order of absorption, storing lam_f, dX_f
