@@ -281,3 +281,18 @@ def test_largest_single_gpu_sizes_are_accepted(lib):
         s = _shape(**kw)
         n = lib.vdn_branch_workspace_size(ctypes.byref(s), 1)
         assert 0 < n < 180e9
+
+
+def test_static_forward_refuses_before_any_cuda_call(lib):
+    # without a GPU any CUDA call would fail: a too-large problem must be refused by its size
+    # alone (VDN_ERR_WORKSPACE), an invalid shape by the regular validation
+    fn = lib.vdn_branch_forward_static
+    fn.restype = ctypes.c_int
+    fn.argtypes = ([ctypes.POINTER(VdnShape)] + [ctypes.c_void_p] * 10
+                   + [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p])
+    big = _shape(H=24, F=31, S=4032)                       # the 768p clip
+    assert lib.vdn_branch_workspace_size(ctypes.byref(big), 1) > 64 << 20
+    a = _args(big)
+    assert fn(*(a[:15] + a[17:])) == VDN_ERR_WORKSPACE
+    bad = _shape(H=24, F=31, S=4032, d=64)
+    assert fn(*((ctypes.byref(bad),) + a[1:15] + a[17:])) == VDN_ERR_UNSUPPORTED
