@@ -414,7 +414,9 @@ vdn_status vdn_frames_finish(const vdn_shape* shape, int F_total, int world, int
 
 /* Reads the device status word that bounded waits inside the kernels set (it
  * lives in the workspace of the last call): VDN_OK or VDN_ERR_TIMEOUT.
- * Synchronises `stream`. */
+ * Synchronises `stream`.  VDN_ERR_INVALID_ARG for a NULL workspace or one of
+ * fewer than 256 bytes (checked before any CUDA call); VDN_ERR_CUDA if the
+ * copy or the synchronisation fails. */
 vdn_status vdn_workspace_status(const void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static description of a status code. */

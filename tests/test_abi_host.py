@@ -296,3 +296,11 @@ def test_static_forward_refuses_before_any_cuda_call(lib):
     assert fn(*(a[:15] + a[17:])) == VDN_ERR_WORKSPACE
     bad = _shape(H=24, F=31, S=4032, d=64)
     assert fn(*((ctypes.byref(bad),) + a[1:15] + a[17:])) == VDN_ERR_UNSUPPORTED
+
+
+def test_workspace_status_argument_checks(lib):
+    fn = lib.vdn_workspace_status
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert fn(None, 1 << 20, None) == VDN_ERR_INVALID_ARG
+    assert fn(ctypes.c_void_p(BASE), 16, None) == VDN_ERR_INVALID_ARG
